@@ -1,0 +1,398 @@
+"""LLSA oracle: a plain, slow, obviously correct CPU reference (numpy, fp64).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  The CUDA library and its
+Python binding never import it, and it imports nothing from them: the only code
+both sides share is the seeded input generator in ``synthetic/``.
+
+What it computes (Log-linear Sparse Attention, non-causal, per batch b and head h):
+
+1. ``build_pyramid`` -- block-wise compression of tokens, 16 tokens per block,
+   applied recursively for L levels ("Trainable Log-linear Sparse Attention for
+   Efficient Diffusion Transformers", abstract: compressing tokens into block-wise
+   representations; skill page "Log Linear Sparse Attention", Core Technique 1;
+   ``block_size=16`` from the LLSA GitHub README usage section).
+2. ``select`` -- hierarchical Top-K: full block scoring at the coarsest level, and at
+   every finer level a sparse Top-K over only the children of the blocks the level
+   above selected (skill page, Core Technique 1, "progressively adopting sparse
+   Top-K selection with the indices found at the previous level", paraphrased).
+3. ``kv_index`` -- hierarchical KV enrichment: each query block attends to its
+   selected fine blocks plus coarse tokens taken from the coarser levels (skill
+   page, Core Technique 2; abstract: coarse representations from several levels).
+4. ``forward`` / ``backward`` -- softmax attention restricted to that KV list, with
+   the ``scaled_dot_product_attention`` conventions the README's usage section
+   replaces (non-causal, scale 1/sqrt(D), no dropout), and its exact gradient.
+5. ``index_transpose`` -- the sparse index transpose: query -> key lists turned into
+   key -> query lists without a dense mask (skill page, Core Technique 3).
+
+Readings where the pages are silent (each one is also listed in the design notes):
+
+* Levels: level l in 1..L has n_l = N / 16^l tokens; level l token j is the mean
+  of the 16 level-(l-1) tokens 16j..16j+15 (so a mean over 16^l input tokens).
+* Pyramid arithmetic: fp32, the 16 terms added one after another in index order
+  starting from 0.0, then multiplied by 1/16 (exact).  Level l is pooled from the
+  stored fp32 level l-1.
+* Scores for selection: raw dot products q.k / sqrt(D) in fp64 from the fp32
+  pyramid.  Top-K of the logits equals Top-K of their softmax, so no softmax.
+* Tie-break: among equal scores the lower key index wins; each list is stored in
+  ascending key order.  The same K is used at every level.  A query block's own
+  block is not forced into its list.
+* Enrichment: for l = 2..L the K level-l tokens selected by the block's level-l
+  ancestor are appended after the 16K fine tokens, each as one ordinary KV entry
+  (unit weight, no score bias).  Level-1 pooled tokens are not attended.
+* Gradients: the selection and the pooled queries carry no gradient; coarse K/V
+  tokens pass their gradient back to the input tokens through the mean-pool
+  adjoint (each of the 16^l tokens under a level-l token receives 1/16^l of it).
+* LSE is the natural-log log-sum-exp of the scaled scores.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+BLOCK = 16
+
+
+# ----------------------------------------------------------------------------- shapes
+
+def level_sizes(N: int, levels: int) -> list[int]:
+    """n_l = N / 16^l for l = 0..L (level 0 is the input sequence)."""
+    return [N // BLOCK ** l for l in range(levels + 1)]
+
+
+def kv_len(topk: int, levels: int) -> int:
+    """Length of a query block's KV list: 16K fine tokens and K coarse tokens per level 2..L."""
+    return BLOCK * topk + (levels - 1) * topk
+
+
+# ----------------------------------------------------------------------------- step 1: pyramid
+
+def build_pyramid(x: np.ndarray, levels: int, acc_dtype=np.float32) -> list[np.ndarray]:
+    """Mean-pooled pyramid of x [B, H, N, D]; returns [level 1, ..., level L], level l of
+    shape [B, H, N / 16^l, D] in ``acc_dtype``.
+
+    Each output value is (((0 + x_0) + x_1) + ... + x_15) * (1/16), every addition
+    rounded in ``acc_dtype`` (fp32 by default; fp64 is used by the finite-difference
+    test so that small perturbations survive).
+    """
+    out = []
+    prev = np.asarray(x).astype(acc_dtype)
+    inv = acc_dtype(1.0 / BLOCK)
+    for _ in range(levels):
+        B, H, n, D = prev.shape
+        assert n % BLOCK == 0
+        groups = prev.reshape(B, H, n // BLOCK, BLOCK, D)
+        acc = np.zeros((B, H, n // BLOCK, D), dtype=acc_dtype)
+        for r in range(BLOCK):
+            acc = acc + groups[:, :, :, r, :]
+        prev = acc * inv
+        out.append(prev)
+    return out
+
+
+# ----------------------------------------------------------------------------- step 2: selection
+
+def selection_scores(q_rows: np.ndarray, k_rows: np.ndarray) -> np.ndarray:
+    """fp64 logits q.k / sqrt(D) for every (query row, key row) pair: [Rq, Rk]."""
+    D = q_rows.shape[-1]
+    return (q_rows.astype(np.float64) @ k_rows.astype(np.float64).T) / math.sqrt(D)
+
+
+def topk_positions(scores: np.ndarray, topk: int) -> np.ndarray:
+    """For each row of ``scores`` (candidates listed in ascending key order), the
+    positions of the K largest scores, lower position first among equal scores,
+    returned in ascending position order.  A stable sort on the negated scores keeps
+    equal scores in ascending position, which is the lower-index tie-break."""
+    order = np.argsort(-scores, axis=-1, kind="stable")[..., :topk]
+    return np.sort(order, axis=-1)
+
+
+def children(parent_keys: np.ndarray) -> np.ndarray:
+    """Level-l keys under the given level-(l+1) keys: 16c + r for r = 0..15, ascending
+    when ``parent_keys`` is ascending."""
+    parent_keys = np.asarray(parent_keys, dtype=np.int64)
+    return (BLOCK * parent_keys[..., :, None] + np.arange(BLOCK)).reshape(*parent_keys.shape[:-1], -1)
+
+
+def select(q_pyr: list[np.ndarray], k_pyr: list[np.ndarray], topk: int) -> list[np.ndarray]:
+    """Hierarchical Top-K.  Returns idx[l-1] of shape [B, H, n_l, K] (int32, ascending)
+    for l = 1..L.
+
+    Coarsest level L: every query token scores every key token.  Level l < L: query a
+    scores only the 16K children of the K level-(l+1) keys its parent a // 16 selected.
+    """
+    L = len(q_pyr)
+    B, H, nL, _ = q_pyr[L - 1].shape
+    if not 1 <= topk <= nL:
+        raise ValueError(f"topk={topk} must be in [1, n_L={nL}]: the coarsest level must hold K keys")
+    idx: list[np.ndarray | None] = [None] * L
+    out = np.empty((B, H, nL, topk), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            s = selection_scores(q_pyr[L - 1][b, h], k_pyr[L - 1][b, h])
+            out[b, h] = topk_positions(s, topk)
+    idx[L - 1] = out
+    for lev in range(L - 1, 0, -1):
+        n = q_pyr[lev - 1].shape[2]
+        out = np.empty((B, H, n, topk), dtype=np.int32)
+        for b in range(B):
+            for h in range(H):
+                qs, ks = q_pyr[lev - 1][b, h], k_pyr[lev - 1][b, h]
+                for g in range(n // BLOCK):                    # sibling group = one parent
+                    cand = children(idx[lev][b, h, g])          # [16K] ascending
+                    s = selection_scores(qs[BLOCK * g:BLOCK * (g + 1)], ks[cand])
+                    out[b, h, BLOCK * g:BLOCK * (g + 1)] = cand[topk_positions(s, topk)]
+        idx[lev - 1] = out
+    return idx  # type: ignore[return-value]
+
+
+# ----------------------------------------------------------------------------- step 3: KV list
+
+def kv_sources(x: np.ndarray, x_pyr: list[np.ndarray]) -> tuple[np.ndarray, list[int]]:
+    """Stack, per (b, h), the attended token sources: the input tokens (level 0) followed
+    by the pooled levels 2..L.  Returns the stacked [B, H, rows, D] array and the row
+    offset of each level (offset[0] = 0, offset[1] unused, offset[l] for l >= 2)."""
+    L = len(x_pyr)
+    parts = [np.asarray(x)]
+    offsets = [0, -1]
+    rows = x.shape[2]
+    for lev in range(2, L + 1):
+        offsets.append(rows)
+        parts.append(x_pyr[lev - 1])
+        rows += x_pyr[lev - 1].shape[2]
+    return np.concatenate([p.astype(np.float64) for p in parts], axis=2), offsets
+
+
+def kv_index(p: int, bh: tuple[int, int], idx: list[np.ndarray], offsets: list[int]) -> np.ndarray:
+    """Rows (into ``kv_sources``) of query block p's KV list: the 16 tokens of each
+    selected level-1 block, then for l = 2..L the K level-l tokens selected by p's
+    level-l ancestor p // 16^(l-1)."""
+    b, h = bh
+    L = len(idx)
+    rows = [children(idx[0][b, h, p])]
+    for lev in range(2, L + 1):
+        anc = p // BLOCK ** (lev - 1)
+        rows.append(offsets[lev] + idx[lev - 1][b, h, anc].astype(np.int64))
+    return np.concatenate(rows)
+
+
+def kv_index_table(b: int, h: int, idx: list[np.ndarray], offsets: list[int]) -> np.ndarray:
+    """[n_1, T] table of ``kv_index`` for every query block of (b, h)."""
+    n1 = idx[0].shape[2]
+    return np.stack([kv_index(p, (b, h), idx, offsets) for p in range(n1)])
+
+
+# ----------------------------------------------------------------------------- step 4: attention
+
+def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256):
+    """Softmax attention of every query over its block's KV list.
+
+    Returns (O [B, H, N, D], LSE [B, H, N]) in fp64.  For query i of block p with
+    list E(p): z_e = q_i . k_e / sqrt(D), O_i = sum_e softmax(z)_e v_e,
+    LSE_i = max z + ln sum_e exp(z_e - max z).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, H, N, D = q.shape
+    ksrc, offsets = kv_sources(k, k_pyr)
+    vsrc, _ = kv_sources(v, v_pyr)
+    n1 = N // BLOCK
+    o = np.empty((B, H, N, D))
+    lse = np.empty((B, H, N))
+    scale = 1.0 / math.sqrt(D)
+    for b in range(B):
+        for h in range(H):
+            table = kv_index_table(b, h, idx, offsets)
+            qb = q[b, h].reshape(n1, BLOCK, D)
+            for s0 in range(0, n1, chunk):
+                sl = slice(s0, min(n1, s0 + chunk))
+                ke = ksrc[b, h][table[sl]]                   # [nb, T, D]
+                ve = vsrc[b, h][table[sl]]
+                z = np.einsum("nqd,ntd->nqt", qb[sl], ke) * scale
+                m = z.max(axis=-1, keepdims=True)
+                e = np.exp(z - m)
+                zsum = e.sum(axis=-1, keepdims=True)
+                o[b, h].reshape(n1, BLOCK, D)[sl] = np.einsum("nqt,ntd->nqd", e / zsum, ve)
+                lse[b, h].reshape(n1, BLOCK)[sl] = (m + np.log(zsum))[..., 0]
+    return o, lse
+
+
+def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256):
+    """Exact gradient of the attention above with the selection held fixed.
+
+    With P = softmax(z) on each query's list, Delta_i = sum_d dO_id O_id and
+    dS = P * (dO v^T - Delta):  dQ_i = sum_e dS_ie k_e / sqrt(D),
+    dK_e += dS_ie q_i / sqrt(D), dV_e += P_ie dO_i.  Gradients that land on coarse
+    level-l tokens are then spread over their 16^l input tokens with weight 1/16^l
+    (the adjoint of the mean pool).  Returns (dQ, dK, dV) [B, H, N, D] in fp64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    B, H, N, D = q.shape
+    L = len(idx)
+    ksrc, offsets = kv_sources(k, k_pyr)
+    vsrc, _ = kv_sources(v, v_pyr)
+    n1 = N // BLOCK
+    scale = 1.0 / math.sqrt(D)
+    dq = np.empty((B, H, N, D))
+    dk = np.empty((B, H, N, D))
+    dv = np.empty((B, H, N, D))
+    for b in range(B):
+        for h in range(H):
+            table = kv_index_table(b, h, idx, offsets)
+            qb = q[b, h].reshape(n1, BLOCK, D)
+            dob = do[b, h].reshape(n1, BLOCK, D)
+            delta = (do[b, h] * o[b, h]).sum(axis=-1).reshape(n1, BLOCK)
+            lseb = lse[b, h].reshape(n1, BLOCK)
+            dksrc = np.zeros_like(ksrc[b, h])
+            dvsrc = np.zeros_like(vsrc[b, h])
+            for s0 in range(0, n1, chunk):
+                sl = slice(s0, min(n1, s0 + chunk))
+                rows = table[sl]
+                ke = ksrc[b, h][rows]
+                ve = vsrc[b, h][rows]
+                z = np.einsum("nqd,ntd->nqt", qb[sl], ke) * scale
+                p = np.exp(z - lseb[sl][..., None])
+                dp = np.einsum("nqd,ntd->nqt", dob[sl], ve)
+                ds = p * (dp - delta[sl][..., None])
+                dq[b, h].reshape(n1, BLOCK, D)[sl] = np.einsum("nqt,ntd->nqd", ds, ke) * scale
+                dke = np.einsum("nqt,nqd->ntd", ds, qb[sl]) * scale
+                dve = np.einsum("nqt,nqd->ntd", p, dob[sl])
+                for i in range(rows.shape[0]):               # rows within one list are distinct
+                    dksrc[rows[i]] += dke[i]
+                    dvsrc[rows[i]] += dve[i]
+            gk = dksrc[:N].copy()
+            gv = dvsrc[:N].copy()
+            for lev in range(2, L + 1):
+                n_l = N // BLOCK ** lev
+                span = BLOCK ** lev
+                ck = dksrc[offsets[lev]:offsets[lev] + n_l]
+                cv = dvsrc[offsets[lev]:offsets[lev] + n_l]
+                gk += np.repeat(ck, span, axis=0) / span
+                gv += np.repeat(cv, span, axis=0) / span
+            dk[b, h] = gk
+            dv[b, h] = gv
+    return dq, dk, dv
+
+
+# ----------------------------------------------------------------------------- step 5: transpose
+
+def index_transpose(idx_level: np.ndarray, n_keys: int) -> tuple[np.ndarray, np.ndarray]:
+    """Key -> query lists of one (b, h, level) selection ``idx_level`` [n_q, K].
+
+    Returns (row_ptr [n_keys + 1], col [n_q * K]) int32: row j holds, in ascending
+    order, every query a whose list contains key j.  A stable sort of the flattened
+    entries by key keeps equal keys in ascending entry order, i.e. ascending query.
+    """
+    n_q, K = idx_level.shape
+    flat = idx_level.reshape(-1).astype(np.int64)
+    counts = np.bincount(flat, minlength=n_keys)
+    row_ptr = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    col = (np.argsort(flat, kind="stable") // K).astype(np.int32)
+    return row_ptr, col
+
+
+def index_transpose_all(idx: list[np.ndarray]) -> tuple[list[np.ndarray], list[np.ndarray]]:
+    """Per level, row_ptr [B, H, n_l + 1] and col [B, H, n_l * K]."""
+    rps, cols = [], []
+    for lv in idx:
+        B, H, n, K = lv.shape
+        rp = np.empty((B, H, n + 1), dtype=np.int32)
+        cl = np.empty((B, H, n * K), dtype=np.int32)
+        for b in range(B):
+            for h in range(H):
+                rp[b, h], cl[b, h] = index_transpose(lv[b, h], n)
+        rps.append(rp)
+        cols.append(cl)
+    return rps, cols
+
+
+# ----------------------------------------------------------------------------- whole path
+
+def llsa_step(q, k, v, do, levels: int, topk: int):
+    """Pyramid, selection, forward, backward and transposes with the oracle's own
+    selection.  Inputs are exact widenings of the device inputs."""
+    q_pyr = build_pyramid(q, levels)
+    k_pyr = build_pyramid(k, levels)
+    v_pyr = build_pyramid(v, levels)
+    idx = select(q_pyr, k_pyr, topk)
+    o, lse = forward(q, k, v, k_pyr, v_pyr, idx)
+    out = dict(q_pyr=q_pyr, k_pyr=k_pyr, v_pyr=v_pyr, idx=idx, o=o, lse=lse)
+    if do is not None:
+        out["dq"], out["dk"], out["dv"] = backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx)
+    out["row_ptr"], out["col"] = index_transpose_all(idx)
+    return out
+
+
+# ----------------------------------------------------------------------------- selection check
+
+def dot_error_floor(q_rows: np.ndarray, k_rows: np.ndarray) -> np.ndarray:
+    """Forward error bound of an fp32 length-D dot product, gamma_D * sum_d |q_d k_d| / sqrt(D)
+    with gamma_D = D u / (1 - D u), u = 2^-24 (Higham, Accuracy and Stability of
+    Numerical Algorithms, section 3.1).  Used only as the absolute floor of the tie window."""
+    D = q_rows.shape[-1]
+    u = 2.0 ** -24
+    gamma = D * u / (1.0 - D * u)
+    return gamma * (np.abs(q_rows.astype(np.float64)) @ np.abs(k_rows.astype(np.float64)).T) / math.sqrt(D)
+
+
+def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5) -> dict:
+    """Check a selection produced elsewhere, level by level from the coarsest down.
+
+    At level l the candidates of query a are taken from ``idx_test`` at level l+1 (so a
+    near-tie swap above does not cascade into failures below).  A row passes if it is
+    the oracle's Top-K exactly, or if it is a valid Top-K under the tie window: the
+    lowest selected score is at least the highest rejected score minus
+    max(rel_tol * max(|s_sel|, |s_rej|), fp32 dot-product error floor).
+    Returns counts: exact rows, tie-window rows, rows that used the absolute floor,
+    bad rows, and the first few bad rows for diagnosis.
+    """
+    L = len(q_pyr)
+    res = {"rows": 0, "exact": 0, "tie_window": 0, "floor_used": 0, "bad": 0, "bad_examples": []}
+    for lev in range(L, 0, -1):
+        test = np.asarray(idx_test[lev - 1])
+        B, H, n, K = test.shape
+        assert K == topk
+        for b in range(B):
+            for h in range(H):
+                qs = q_pyr[lev - 1][b, h]
+                ks = k_pyr[lev - 1][b, h]
+                if lev == L:
+                    groups = [(np.arange(n), np.arange(n))]
+                else:
+                    groups = [(np.arange(BLOCK * g, BLOCK * (g + 1)), children(idx_test[lev][b, h, g]))
+                              for g in range(n // BLOCK)]
+                for qrows, cand in groups:
+                    s = selection_scores(qs[qrows], ks[cand])
+                    floor = dot_error_floor(qs[qrows], ks[cand])
+                    want = cand[topk_positions(s, topk)]
+                    for r, a in enumerate(qrows):
+                        res["rows"] += 1
+                        got = test[b, h, a].astype(np.int64)
+                        if np.array_equal(got, want[r]):
+                            res["exact"] += 1
+                            continue
+                        pos = np.searchsorted(cand, got)
+                        valid = (np.all(np.diff(got) > 0) and np.all(pos < cand.size)
+                                 and np.array_equal(cand[np.minimum(pos, cand.size - 1)], got))
+                        ok = False
+                        used_floor = False
+                        if valid:
+                            selm = np.zeros(cand.size, dtype=bool)
+                            selm[pos] = True
+                            lo = s[r, selm].min()
+                            hi = s[r, ~selm].max() if (~selm).any() else -np.inf
+                            rel = rel_tol * max(abs(lo), abs(hi))
+                            fl = max(floor[r, selm].max(), floor[r, ~selm].max() if (~selm).any() else 0.0)
+                            ok = lo >= hi - max(rel, fl)
+                            used_floor = ok and not (lo >= hi - rel)
+                        if ok:
+                            res["tie_window"] += 1
+                            res["floor_used"] += int(used_floor)
+                        else:
+                            res["bad"] += 1
+                            if len(res["bad_examples"]) < 5:
+                                res["bad_examples"].append((lev, b, h, int(a), got.tolist(), want[r].tolist()))
+    return res
