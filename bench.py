@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the LLSA training step (forward + backward of the attention op).
+
+One step = the whole hot path on one batch of device-resident synthetic input:
+pyramid -> hierarchical selection -> attention forward -> index transpose -> attention
+backward (five C-ABI calls, 12 kernel launches at the default workload).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 4]
+
+Multi-GPU runs (torchrun, one process per GPU) are weak-scaled independent replicas: every
+rank runs the whole workload on its own GPU, with no data-path collective; the step time is
+the maximum over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LLSA fwd+bwd tokens/sec at N=65536 bf16, 1 B200; % of roofline"
+UNIT = "tokens/s"
+KERNELS_PER_STEP_HINT = 16
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world, local):
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_done(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons while running."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_uuid: str):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self, load_threshold_w: float = 250.0) -> dict:
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r[2] >= load_threshold_w] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ----------------------------------------------------------------------------- algorithmic counts
+
+def workload_counts(cfg, pairs_l1: int):
+    """Algorithmic bytes and FLOPs per launch of each kernel for one step of ``cfg``.
+
+    Per query block the forward gathers the KV list (T tokens x 64 channels x 2 bytes for K
+    and for V) and streams Q, O and LSE; the query-major backward gathers the same list and
+    streams Q, dO, O, dQ, LSE and Delta; the key-major backward streams K_j, V_j, dK_j, dV_j
+    per fine key block and Q, dO, LSE, Delta per (key block, query block) pair.  FLOPs are
+    4*16*T*64 per block (forward), 6*16*T*64 (query-major backward: S, dP, dQ) and
+    8*16*16*64 per pair (key-major backward: S, dP, dV, dK).
+    """
+    D, e = cfg.D, 2
+    bh = cfg.B * cfg.H
+    n = cfg.level_sizes()
+    n1 = n[1]
+    T = cfg.kv_len
+    blocks = bh * n1
+    tile = 16 * D * e
+    row_stream = 16 * 4
+    counts = {
+        "attn_fwd_bf16": dict(bytes=blocks * (T * D * e * 2 + 2 * tile + row_stream),
+                              flops=4 * blocks * 16 * T * D),
+        "attn_bwd_dq_bf16": dict(bytes=blocks * (T * D * e * 2 + 4 * tile + 2 * row_stream),
+                                 flops=6 * blocks * 16 * T * D),
+        "attn_bwd_dkdv_bf16": dict(bytes=blocks * 4 * tile + pairs_l1 * (2 * tile + 2 * row_stream),
+                                   flops=8 * pairs_l1 * 16 * 16 * D),
+        "pyramid_l12": dict(bytes=3 * (bh * cfg.N * D * e + bh * (n1 + (n[2] if cfg.levels >= 2 else 0)) * D * 4),
+                            flops=0),
+    }
+    return counts
+
+
+# ----------------------------------------------------------------------------- oracle sample
+
+def oracle_sample(cfg, inputs, heads: int, nblocks: int | None):
+    """Time the CPU oracle on ``heads`` (b=0) heads of the workload: pyramid, selection and
+    transpose for each whole head, forward and backward for ``nblocks`` query blocks per
+    head (all blocks if None).  Returns (tokens/s extrapolated to the full workload, dict)."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from oracle import llsa_oracle as orc
+    from synthetic import to_f32_numpy, to_f64_numpy
+
+    n1 = cfg.N // 16
+    blocks = None if nblocks is None or nblocks >= n1 else np.linspace(0, n1 - 1, nblocks).astype(np.int64)
+    nb = n1 if blocks is None else len(blocks)
+    t_fixed = t_attn = 0.0
+    with threadpool_limits(1):
+        for h in range(heads):
+            sl = (slice(0, 1), slice(h, h + 1))
+            q32, k32, v32 = (to_f32_numpy(inputs[x][sl]) for x in ("q", "k", "v"))
+            q, k, v, do = (to_f64_numpy(inputs[x][sl]) for x in ("q", "k", "v", "do"))
+            t0 = time.perf_counter()
+            qp, kp, vp = (orc.build_pyramid(a, cfg.levels) for a in (q32, k32, v32))
+            idx = orc.select(qp, kp, cfg.topk)
+            orc.index_transpose_all(idx)
+            t1 = time.perf_counter()
+            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks)
+            if cfg.backward:
+                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks)
+            t2 = time.perf_counter()
+            t_fixed += t1 - t0
+            t_attn += t2 - t1
+    # per head: fixed part + attention scaled from nb sampled blocks to all n1 blocks
+    per_head = (t_fixed + t_attn * (n1 / nb)) / heads
+    full_step = per_head * cfg.B * cfg.H
+    info = {"heads": heads, "blocks_per_head": nb, "seconds": t_fixed + t_attn, "t_full_step_est_s": full_step,
+            "t_fixed_per_head": t_fixed / heads, "t_attn_per_block": t_attn / (heads * nb)}
+    return cfg.B * cfg.N / full_step, info
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.nn.functional as F
+
+    from log_linear_hierarchical_b200 import api
+    from synthetic import CONFIGS, make_config_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dist_init(world, local)
+    cfg = CONFIGS[args.config]
+    dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    host = make_config_inputs(cfg, with_do=True)
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    dev = {k: v.cuda(non_blocking=True) for k, v in pinned.items()}
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype)
+    buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = api.llsa_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    # one traced step to size the trace of the timed region
+    probe = api.LaunchTrace(64)
+    with probe:
+        step()
+    per_step = probe.used
+    torch.cuda.synchronize()
+
+    trace = api.LaunchTrace(per_step * args.steps)
+    props = torch.cuda.get_device_properties(local)
+    sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 or world == 1 else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.start()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    with trace:
+        for _ in range(args.steps):
+            step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    if sampler:
+        sampler.stop()
+    ms_local = start.elapsed_time(end)
+    ms_total = dist_max(ms_local, world)
+    status = api.llsa_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    # per-kernel averages over the timed region
+    launches = trace.launches()
+    per_kernel: dict[str, list[float]] = {}
+    for name, ms in launches:
+        per_kernel.setdefault(name, []).append(ms)
+    kern = {k: {"launches": len(v), "avg_us": 1000 * sum(v) / len(v), "total_ms": sum(v)} for k, v in per_kernel.items()}
+    total_kernel_ms = sum(x["total_ms"] for x in kern.values())
+    for x in kern.values():
+        x["share"] = x["total_ms"] / total_kernel_ms
+
+    tokens_per_step = cfg.B * cfg.N
+    value = world * args.steps * tokens_per_step / (ms_total / 1000.0)
+    ms_per_step = ms_total / args.steps
+
+    # algorithmic roofline of the dominant kernel
+    rps, _ = buf.csr_levels()
+    pairs_l1 = int(rps[0][..., -1].sum().item())
+    counts = workload_counts(cfg, pairs_l1)
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
+    hbm_peak = peaks["hbm_gbs"] if peaks else 6650.0
+    tensor_peak = peaks["bf16_tflops_sustained"] if peaks else 1400.0
+    dominant = max(kern, key=lambda k: kern[k]["total_ms"])
+    roofline = None
+    if dominant in counts:
+        c = counts[dominant]
+        sec = kern[dominant]["avg_us"] * 1e-6
+        achieved = c["bytes"] / sec / 1e9
+        roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                    "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                    "traffic": traffic_per_launch(dominant, cfg),
+                    "peak_source": "measured" if peaks else "fallback",
+                    "algorithmic_bytes_per_launch": c["bytes"],
+                    "tensor_achieved_tflops": round(c["flops"] / sec / 1e12, 2),
+                    "tensor_frac_of_sustained_bf16": round(c["flops"] / sec / 1e12 / tensor_peak, 4)}
+    kernels_roof = {}
+    for k, c in counts.items():
+        if k in kern:
+            sec = kern[k]["avg_us"] * 1e-6
+            kernels_roof[k] = {"avg_us": round(kern[k]["avg_us"], 2), "share": round(kern[k]["share"], 4),
+                               "hbm_frac": round(c["bytes"] / sec / 1e9 / hbm_peak, 4),
+                               "tensor_frac": round(c["flops"] / sec / 1e12 / tensor_peak, 4) if c["flops"] else 0.0}
+    # whole-step roofline as the workload defines it: the slower of the step's FLOPs at the
+    # bf16 tensor peak and its modelled bytes at the HBM peak
+    step_bytes = sum(c["bytes"] for k, c in counts.items() if k in kern)
+    step_flops = sum(c["flops"] for k, c in counts.items() if k in kern)
+    step_roof_ms = 1000 * max(step_bytes / (hbm_peak * 1e9), step_flops / (tensor_peak * 1e12))
+
+    # end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.steps, 10))
+    host_out = {k: torch.empty(cfg.B, cfg.H, cfg.N, cfg.D, dtype=dtype).pin_memory() for k in ("o", "dq", "dk", "dv")}
+    in_bytes = sum(t.numel() * t.element_size() for t in pinned.values())
+    out_bytes = sum(t.numel() * t.element_size() for t in host_out.values())
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for k in ("q", "k", "v", "do"):
+            dev[k].copy_(pinned[k], non_blocking=True)
+        step()
+        host_out["o"].copy_(buf.o, non_blocking=True)
+        host_out["dq"].copy_(buf.dq, non_blocking=True)
+        host_out["dk"].copy_(buf.dk, non_blocking=True)
+        host_out["dv"].copy_(buf.dv, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(e0.elapsed_time(e1), world)
+    e2e_value = world * e2e_steps * tokens_per_step / (e2e_ms / 1000.0)
+
+    # dense attention at the same shape (torch SDPA, flash backend), forward + backward
+    dense = None
+    if world == 1:
+        q = dev["q"].detach().clone().requires_grad_(True)
+        k = dev["k"].detach().clone().requires_grad_(True)
+        v = dev["v"].detach().clone().requires_grad_(True)
+        for _ in range(2):
+            F.scaled_dot_product_attention(q, k, v).backward(dev["do"])
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        d0.record(stream)
+        for _ in range(reps):
+            F.scaled_dot_product_attention(q, k, v).backward(dev["do"])
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = d0.elapsed_time(d1) / reps
+        dense = {"impl": "torch scaled_dot_product_attention (bf16, non-causal), forward + backward",
+                 "ms_per_step": round(dms, 3), "tokens_per_s": round(tokens_per_step / (dms / 1000.0), 1),
+                 "llsa_speedup": round(dms / ms_per_step, 2)}
+        del q, k, v
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, info = oracle_sample(cfg, host, heads=2, nblocks=None)
+        cpu = {"value": round(val, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": (f"numpy fp64 oracle, 1 thread: pyramid, selection, transpose, forward and backward of "
+                          f"heads (b=0, h=0..1), {info['seconds']:.1f} s, extrapolated to {cfg.B * cfg.H} heads")}
+
+    clocks = sampler.summary() if sampler else None
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded smooth-field Q/K in Z order, N(0,1) V and dO)",
+        "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
+                   "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk, "kv_len": cfg.kv_len,
+                   "step": "pyramid + select + forward + index transpose + backward",
+                   "parallelism": f"dp{world}: independent replicas, no collective",
+                   "l2": "inputs larger than L2: q, k, v, dO are 201 MB per replica vs 126 MB L2; no flush"},
+        "roofline": roofline,
+        "step_roofline": {"modelled_bytes": step_bytes, "flops": step_flops, "roofline_ms": round(step_roof_ms, 4),
+                          "frac": round(step_roof_ms / ms_per_step, 4)},
+        "kernels": kernels_roof,
+        "kernel_times": {k: {"launches": v["launches"], "avg_us": round(v["avg_us"], 2), "share": round(v["share"], 4)}
+                         for k, v in sorted(kern.items(), key=lambda kv: -kv[1]["total_ms"])},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": out_bytes, "steps": e2e_steps,
+                "api": "log_linear_hierarchical_b200.llsa_train_step with pinned host copies in and out"},
+        "dense_attention": dense,
+        "gpu_launches": trace.used,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    del trace
+    dist_done(world)
+
+
+def traffic_per_launch(kernel: str, cfg):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel sources (profiles/ncu_traffic.txt lines: kernel workload bytes source-hash)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    h = source_hash()
+    for ln in open(path):
+        parts = ln.split()
+        if len(parts) == 4 and parts[0] == kernel and parts[1] == cfg.name and parts[3] == h:
+            return float(parts[2])
+    return None
+
+
+def source_hash() -> str:
+    import hashlib
+    d = os.path.join(ROOT, "log_linear_hierarchical_b200", "csrc")
+    m = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        m.update(open(os.path.join(d, f), "rb").read())
+    return m.hexdigest()[:12]
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: rank 0 only, each step a bounded sample."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from synthetic import CONFIGS, make_config_inputs
+
+    cfg = CONFIGS[args.config]
+    host = make_config_inputs(cfg, with_do=True)
+    n1 = cfg.N // 16
+    # size each step's sample so that warm-up + steps stay near two minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    _, probe = oracle_sample(cfg, host, heads=1, nblocks=16)
+    per_block = max(1e-6, probe["t_attn_per_block"])
+    nblocks = int(max(16, min(n1, (budget - probe["t_fixed_per_head"]) / per_block)))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, host, heads=1, nblocks=nblocks)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        v, info = oracle_sample(cfg, host, heads=1, nblocks=nblocks)
+        vals.append(v)
+        secs += info["seconds"]
+    value = statistics.median(vals)
+    tokens_per_step = cfg.B * cfg.N
+    ms_per_step = 1000.0 * tokens_per_step / value
+    sample = (f"numpy fp64 oracle, 1 thread, per step: pyramid, selection and transpose of head (b=0, h=0) and "
+              f"forward+backward of {nblocks} of its {n1} query blocks, extrapolated to all blocks and "
+              f"{cfg.B * cfg.H} heads; median over {args.steps} steps")
+    result = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the CUDA arm)",
+        "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
+                   "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=4, help="workload number (4 = the headline N=65536 step)")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

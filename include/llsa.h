@@ -1,0 +1,190 @@
+/*
+ * llsa.h -- C ABI of the B200 (sm_100a) Log-linear Sparse Attention hot path.
+ *
+ * Log-linear Sparse Attention (LLSA) is non-causal multi-head attention in which each
+ * block of 16 queries attends to K selected blocks of 16 keys plus K coarse (mean-pooled)
+ * key tokens from each coarser level of a 16x pyramid ("Trainable Log-linear Sparse
+ * Attention for Efficient Diffusion Transformers", abstract; skill page "Log Linear
+ * Sparse Attention", Core Technique 1-3).  The LLSA GitHub README's usage section makes
+ * it a drop-in for scaled_dot_product_attention(q, k, v, dropout_p=0, is_causal=False)
+ * with block_size=16, and states that only non-causal attention is supported and that
+ * the token length and topk must be powers of two.
+ *
+ * The path is split into five calls, in this order for one training step:
+ *   llsa_build_pyramid -> llsa_select -> llsa_forward            (forward)
+ *   llsa_index_transpose -> llsa_backward                        (backward)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Shapes: B batches, H heads, N tokens, D channels per head, block = 16, topk = K,
+ *    levels = L.  Level l (1..L) has n_l = N / 16^l tokens; level 0 is the input.
+ *  - q, k, v, o, dO, dq, dk, dv: [B, H, N, D] contiguous row-major, element type
+ *    `dtype` (bf16 or fp32): the scaled_dot_product_attention layout.
+ *  - Pyramids q_pyr/k_pyr/v_pyr: fp32, levels 1..L concatenated level-major:
+ *    [L][B, H, n_l, D]; llsa_pyramid_elems() gives the element count per tensor.
+ *  - idx: int32 level-major [L][B, H, n_l, K]; row (l, b, h, a) holds the K level-l key
+ *    indices selected for level-l query token a, strictly ascending.  Level-1 rows are
+ *    the selected fine blocks of query block a (tokens 16a..16a+15).
+ *  - row_ptr: int32 level-major [L][B, H, n_l + 1]; col: int32 level-major
+ *    [L][B, H, n_l * K].  Row j of (l, b, h) lists, ascending, every level-l query a whose
+ *    idx row contains key j (a CSR matrix; row_ptr offsets are local to (l, b, h)).
+ *  - lse: fp32 [B, H, N], natural-log log-sum-exp of each query's scaled scores.
+ *  - Every pointer is device memory owned by the caller, 16-byte aligned (256-byte
+ *    alignment recommended).  The library allocates no memory, keeps no state between
+ *    calls and is reentrant; calls on different streams must not share output buffers.
+ *  - Every call is asynchronous on `stream` (NULL = legacy default stream) and never
+ *    synchronises the host, except llsa_device_status.
+ *  - Arguments are checked on the host before any launch.  A rejected call launches
+ *    nothing and returns LLSA_ERR_INVALID_ARG (bad value, null pointer, misalignment,
+ *    shape rules below) or LLSA_ERR_UNSUPPORTED (a legal value this build does not
+ *    implement).  A launch failure returns LLSA_ERR_CUDA.  No exception crosses the ABI.
+ *  - Shape rules: B, H >= 1; N a power of two with N >= 16^L (so N / 16^L >= 1);
+ *    topk a power of two with 1 <= topk <= n_L; block == 16; 1 <= levels <= 4;
+ *    D == 64; N <= 2^20; n_L <= 16384; topk <= 64; (levels - 1) * topk <= 32;
+ *    B * H * N < 2^31.
+ *  - Device-side checks: every gathered index (idx entries, CSR entries) is range
+ *    checked on the device; an out-of-range value is not dereferenced, and the call
+ *    records LLSA_ERR_INTERNAL in a device status word that llsa_device_status reads.
+ *    Bounded waits inside kernels that time out record LLSA_ERR_TIMEOUT the same way.
+ */
+#ifndef LLSA_H_
+#define LLSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (a pointer to the opaque CUstream_st). */
+struct CUstream_st;
+typedef struct CUstream_st* llsa_stream_t;
+
+typedef enum {
+  LLSA_OK = 0,
+  LLSA_ERR_INVALID_ARG = 1,
+  LLSA_ERR_UNSUPPORTED = 2,
+  LLSA_ERR_WORKSPACE = 3,
+  LLSA_ERR_CUDA = 4,
+  LLSA_ERR_INTERNAL = 5,
+  LLSA_ERR_TIMEOUT = 6
+} llsa_status;
+
+typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
+
+typedef struct {
+  int32_t B, H, N, D;
+  int32_t block;   /* must be 16 (README usage section: block_size=16) */
+  int32_t topk;    /* K, a power of two */
+  int32_t levels;  /* L, number of pooled levels; llsa_l1 <-> 1, llsa_l2 <-> 2 */
+  int32_t dtype;   /* llsa_dtype of q, k, v, o, dO, dq, dk, dv */
+} llsa_shape;
+
+/* Static text for a status code. */
+const char* llsa_status_string(llsa_status status);
+
+/* Host-only check of a shape against the rules above. */
+llsa_status llsa_validate_shape(const llsa_shape* shape);
+
+/* Element counts of the caller-allocated buffers (0 for an invalid shape). */
+size_t llsa_pyramid_elems(const llsa_shape* shape);   /* fp32 elements per pyramid tensor */
+size_t llsa_index_elems(const llsa_shape* shape);     /* int32 elements of idx and of col */
+size_t llsa_row_ptr_elems(const llsa_shape* shape);   /* int32 elements of row_ptr */
+
+/* Scratch bytes llsa_index_transpose / llsa_backward need in `workspace`. */
+size_t llsa_transpose_workspace_bytes(const llsa_shape* shape);
+size_t llsa_backward_workspace_bytes(const llsa_shape* shape);
+
+/*
+ * Step 1 -- the mean-pooled Q/K/V pyramid (abstract: block-wise compression; skill page,
+ * Core Technique 1: hierarchical compression).  For l = 1..L and every token j < n_l,
+ * X_l[j] = (((0 + X_{l-1}[16j]) + X_{l-1}[16j+1]) + ... + X_{l-1}[16j+15]) * (1/16),
+ * every addition rounded to fp32 in this order (X_0 = the input, widened exactly).
+ * q, k, v: [B,H,N,D] `dtype`; q_pyr, k_pyr, v_pyr: [L][B,H,n_l,D] fp32 outputs.
+ */
+llsa_status llsa_build_pyramid(const llsa_shape* shape, const void* q, const void* k, const void* v,
+                               float* q_pyr, float* k_pyr, float* v_pyr, llsa_stream_t stream);
+
+/*
+ * Step 2 -- hierarchical Top-K (skill page, Core Technique 1: sparse Top-K at each level
+ * over the indices found at the previous level).  At level L every query token scores all
+ * n_L key tokens; at level l < L query a scores only the 16K children 16c+r (r < 16) of
+ * the K level-(l+1) keys c selected for its parent a/16.  Score = fp32 dot product of the
+ * pooled q and k rows; the K largest are kept, the lower key index winning equal scores,
+ * and written ascending.  q_pyr, k_pyr: pyramids from step 1; idx: output [L][B,H,n_l,K].
+ */
+llsa_status llsa_select(const llsa_shape* shape, const float* q_pyr, const float* k_pyr, int32_t* idx,
+                        llsa_stream_t stream);
+
+/*
+ * Step 5 -- the sparse index transpose (skill page, Core Technique 3: a transpose that
+ * works on the sparse indices and builds no dense mask).  For every level, batch and head
+ * it turns the query -> key lists `idx` into key -> query CSR lists (row_ptr, col),
+ * queries ascending within each row.  It is a stable counting sort by key bucket then by
+ * key (histogram + scan + scatter), with no atomics, so the output is deterministic.
+ * workspace: device scratch of at least llsa_transpose_workspace_bytes(shape) bytes,
+ * 256-byte aligned; its contents are not read before being written.
+ */
+llsa_status llsa_index_transpose(const llsa_shape* shape, const int32_t* idx, int32_t* row_ptr,
+                                 int32_t* col, void* workspace, size_t workspace_bytes,
+                                 llsa_stream_t stream);
+
+/*
+ * Step 4a -- block-sparse attention forward with hierarchical KV enrichment (skill page,
+ * Core Technique 2).  Query block p (tokens 16p..16p+15) attends to the KV list: the 16
+ * tokens of each selected level-1 block j in idx[1][p], then for l = 2..L the K pooled
+ * level-l tokens idx[l][p / 16^(l-1)] (k_pyr/v_pyr rows, each one ordinary KV entry).
+ * O_i = softmax(q_i . k_e / sqrt(D)) over that list applied to v_e; lse_i = natural-log
+ * log-sum-exp of the scaled scores.  Arithmetic: bf16 inputs use bf16 tensor-core
+ * products (coarse fp32 rows rounded to bf16) with fp32 accumulation and fp32 softmax;
+ * fp32 inputs use fp32 throughout.  o: [B,H,N,D] `dtype`; lse: [B,H,N] fp32.
+ */
+llsa_status llsa_forward(const llsa_shape* shape, const void* q, const void* k, const void* v,
+                         const float* k_pyr, const float* v_pyr, const int32_t* idx, void* o, float* lse,
+                         llsa_stream_t stream);
+
+/*
+ * Step 4b -- gradient of step 4a with the selection held fixed (the pages train LLSA
+ * end to end: "trainable" in the title; skill page, Practical Results: training speedup).
+ * With P the softmax over each query's list, Delta_i = sum_d dO_id * O_id and
+ * dS = P * (dO v^T - Delta): dq_i = sum_e dS_ie k_e / sqrt(D); dk_e += dS_ie q_i / sqrt(D);
+ * dv_e += P_ie dO_i.  Gradients of pooled level-l tokens are spread over their 16^l input
+ * tokens with weight 1/16^l (the mean-pool adjoint); pooled queries get no gradient.
+ * Fine-token dk/dv are gathered through the level-1 CSR (row_ptr, col from step 5) and
+ * coarse-token gradients through the level-l CSRs, so no atomics are used.
+ * o, lse: outputs of llsa_forward; dO: [B,H,N,D] `dtype`; dq, dk, dv: [B,H,N,D] `dtype`.
+ * workspace: at least llsa_backward_workspace_bytes(shape) bytes, 256-byte aligned.
+ */
+llsa_status llsa_backward(const llsa_shape* shape, const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dO, const float* k_pyr,
+                          const float* v_pyr, const int32_t* idx, const int32_t* row_ptr,
+                          const int32_t* col, void* dq, void* dk, void* dv, void* workspace,
+                          size_t workspace_bytes, llsa_stream_t stream);
+
+/*
+ * Reads and clears the device status word that kernels set on an out-of-range index
+ * (LLSA_ERR_INTERNAL) or a bounded wait that timed out (LLSA_ERR_TIMEOUT).  Synchronises
+ * `stream` first.  *code_out receives LLSA_OK or the first error recorded since the last
+ * call.  Returns LLSA_ERR_CUDA if the device cannot be queried.
+ */
+llsa_status llsa_device_status(int32_t* code_out, llsa_stream_t stream);
+
+/*
+ * Per-launch trace (instrumentation; no counterpart on the pages).  Between
+ * llsa_trace_begin and llsa_trace_end, every kernel launch made by the calling host thread
+ * through the calls above is bracketed by two cudaEventRecord calls on that call's stream:
+ * launch i records events[2i] just before and events[2i+1] just after, and stores its kernel
+ * id (llsa_kernel_name gives the name) in kernel_ids[i].  `events` holds 2 * capacity
+ * cudaEvent_t handles created by the caller (timing enabled); launches beyond `capacity`
+ * are not traced.  llsa_trace_end stops tracing and reports the number of launches traced.
+ */
+llsa_status llsa_trace_begin(void** events, int32_t* kernel_ids, int32_t capacity);
+llsa_status llsa_trace_end(int32_t* launches_out);
+const char* llsa_kernel_name(int32_t kernel_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLSA_H_ */

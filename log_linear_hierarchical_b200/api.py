@@ -1,0 +1,301 @@
+"""Python binding of the LLSA C ABI (same names as include/llsa.h).
+
+Torch provides device memory and streams; each call passes ``data_ptr()`` values and the
+current CUDA stream to libllsa.so and raises ``LLSAError`` on a non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import LLSA_BF16, LLSA_F32, LLSAShape
+
+_DTYPES = {torch.bfloat16: LLSA_BF16, torch.float32: LLSA_F32}
+
+
+class LLSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        name = _lib.STATUS_NAMES.get(status, str(status))
+        try:
+            text = _lib.load().llsa_status_string(status).decode()
+        except Exception:  # pragma: no cover - message only
+            text = ""
+        super().__init__(f"{fn} returned {name}: {text}")
+        self.status = status
+
+
+def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16) -> LLSAShape:
+    code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return LLSAShape(B, H, N, D, block, topk, levels, code)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise LLSAError(fn, status)
+
+
+def _p(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("LLSA buffers must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ref(shape: LLSAShape):
+    return ctypes.byref(shape)
+
+
+# ----------------------------------------------------------------------------- sizes
+
+def llsa_validate_shape(shape: LLSAShape) -> int:
+    return _lib.load().llsa_validate_shape(_ref(shape))
+
+
+def llsa_pyramid_elems(shape: LLSAShape) -> int:
+    return _lib.load().llsa_pyramid_elems(_ref(shape))
+
+
+def llsa_index_elems(shape: LLSAShape) -> int:
+    return _lib.load().llsa_index_elems(_ref(shape))
+
+
+def llsa_row_ptr_elems(shape: LLSAShape) -> int:
+    return _lib.load().llsa_row_ptr_elems(_ref(shape))
+
+
+def llsa_transpose_workspace_bytes(shape: LLSAShape) -> int:
+    return _lib.load().llsa_transpose_workspace_bytes(_ref(shape))
+
+
+def llsa_backward_workspace_bytes(shape: LLSAShape) -> int:
+    return _lib.load().llsa_backward_workspace_bytes(_ref(shape))
+
+
+# ----------------------------------------------------------------------------- the five calls
+
+def llsa_build_pyramid(shape, q, k, v, q_pyr, k_pyr, v_pyr, stream=None) -> None:
+    _check("llsa_build_pyramid", _lib.load().llsa_build_pyramid(
+        _ref(shape), _p(q), _p(k), _p(v), _p(q_pyr), _p(k_pyr), _p(v_pyr), _stream(stream)))
+
+
+def llsa_select(shape, q_pyr, k_pyr, idx, stream=None) -> None:
+    _check("llsa_select", _lib.load().llsa_select(_ref(shape), _p(q_pyr), _p(k_pyr), _p(idx), _stream(stream)))
+
+
+def llsa_index_transpose(shape, idx, row_ptr, col, workspace, stream=None) -> None:
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("llsa_index_transpose", _lib.load().llsa_index_transpose(
+        _ref(shape), _p(idx), _p(row_ptr), _p(col), _p(workspace), nbytes, _stream(stream)))
+
+
+def llsa_forward(shape, q, k, v, k_pyr, v_pyr, idx, o, lse, stream=None) -> None:
+    _check("llsa_forward", _lib.load().llsa_forward(
+        _ref(shape), _p(q), _p(k), _p(v), _p(k_pyr), _p(v_pyr), _p(idx), _p(o), _p(lse), _stream(stream)))
+
+
+def llsa_backward(shape, q, k, v, o, lse, do, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace,
+                  stream=None) -> None:
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("llsa_backward", _lib.load().llsa_backward(
+        _ref(shape), _p(q), _p(k), _p(v), _p(o), _p(lse), _p(do), _p(k_pyr), _p(v_pyr), _p(idx), _p(row_ptr),
+        _p(col), _p(dq), _p(dk), _p(dv), _p(workspace), nbytes, _stream(stream)))
+
+
+def llsa_device_status(stream=None) -> int:
+    code = ctypes.c_int32(0)
+    _check("llsa_device_status", _lib.load().llsa_device_status(ctypes.byref(code), _stream(stream)))
+    return int(code.value)
+
+
+def llsa_kernel_name(kernel_id: int) -> str:
+    return _lib.load().llsa_kernel_name(kernel_id).decode()
+
+
+class LaunchTrace:
+    """Context manager over llsa_trace_begin / llsa_trace_end: every kernel the library
+    launches from this thread inside the block is bracketed by two CUDA events on its stream."""
+
+    def __init__(self, capacity: int):
+        self.capacity = capacity
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.events:       # creates the underlying cudaEvent_t
+            e.record()
+        self._handles = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.events])
+        self._ids = (ctypes.c_int32 * max(1, capacity))()
+        self.used = 0
+
+    def __enter__(self):
+        _check("llsa_trace_begin", _lib.load().llsa_trace_begin(self._handles, self._ids, self.capacity))
+        return self
+
+    def __exit__(self, *exc):
+        used = ctypes.c_int32(0)
+        _lib.load().llsa_trace_end(ctypes.byref(used))
+        self.used = int(used.value)
+        return False
+
+    def launches(self):
+        """[(kernel name, milliseconds)] of every traced launch; synchronises."""
+        torch.cuda.synchronize()
+        return [(llsa_kernel_name(self._ids[i]), self.events[2 * i].elapsed_time(self.events[2 * i + 1]))
+                for i in range(self.used)]
+
+
+# ----------------------------------------------------------------------------- buffers
+
+@dataclass
+class LLSABuffers:
+    """Every intermediate and output of one LLSA step for one shape, on one device."""
+
+    shape: LLSAShape
+    q_pyr: torch.Tensor
+    k_pyr: torch.Tensor
+    v_pyr: torch.Tensor
+    idx: torch.Tensor
+    row_ptr: torch.Tensor
+    col: torch.Tensor
+    o: torch.Tensor
+    lse: torch.Tensor
+    dq: torch.Tensor
+    dk: torch.Tensor
+    dv: torch.Tensor
+    ws_transpose: torch.Tensor
+    ws_backward: torch.Tensor
+
+    @staticmethod
+    def allocate(shape: LLSAShape, device, dtype: torch.dtype) -> "LLSABuffers":
+        st = llsa_validate_shape(shape)
+        if st != 0:
+            raise LLSAError("llsa_validate_shape", st)
+        B, H, N, D = shape.B, shape.H, shape.N, shape.D
+        f32 = dict(device=device, dtype=torch.float32)
+        i32 = dict(device=device, dtype=torch.int32)
+        npyr = llsa_pyramid_elems(shape)
+
+        def bytes_buf(n):
+            return torch.empty((n + 3) // 4, **f32)
+
+        return LLSABuffers(
+            shape=shape,
+            q_pyr=torch.empty(npyr, **f32), k_pyr=torch.empty(npyr, **f32), v_pyr=torch.empty(npyr, **f32),
+            idx=torch.empty(llsa_index_elems(shape), **i32),
+            row_ptr=torch.empty(llsa_row_ptr_elems(shape), **i32),
+            col=torch.empty(llsa_index_elems(shape), **i32),
+            o=torch.empty(B, H, N, D, device=device, dtype=dtype),
+            lse=torch.empty(B, H, N, **f32),
+            dq=torch.empty(B, H, N, D, device=device, dtype=dtype),
+            dk=torch.empty(B, H, N, D, device=device, dtype=dtype),
+            dv=torch.empty(B, H, N, D, device=device, dtype=dtype),
+            ws_transpose=bytes_buf(llsa_transpose_workspace_bytes(shape)),
+            ws_backward=bytes_buf(llsa_backward_workspace_bytes(shape)),
+        )
+
+    # Level views of the packed, level-major buffers.
+    def level_sizes(self):
+        s = self.shape
+        return [s.N // 16 ** l for l in range(1, s.levels + 1)]
+
+    def pyramid_levels(self, buf: torch.Tensor):
+        s = self.shape
+        out, off = [], 0
+        for n in self.level_sizes():
+            cnt = s.B * s.H * n * s.D
+            out.append(buf[off:off + cnt].view(s.B, s.H, n, s.D))
+            off += cnt
+        return out
+
+    def idx_levels(self):
+        s = self.shape
+        out, off = [], 0
+        for n in self.level_sizes():
+            cnt = s.B * s.H * n * s.topk
+            out.append(self.idx[off:off + cnt].view(s.B, s.H, n, s.topk))
+            off += cnt
+        return out
+
+    def csr_levels(self):
+        s = self.shape
+        rps, cols, ro, co = [], [], 0, 0
+        for n in self.level_sizes():
+            rc = s.B * s.H * (n + 1)
+            cc = s.B * s.H * n * s.topk
+            rps.append(self.row_ptr[ro:ro + rc].view(s.B, s.H, n + 1))
+            cols.append(self.col[co:co + cc].view(s.B, s.H, n * s.topk))
+            ro += rc
+            co += cc
+        return rps, cols
+
+
+def llsa_forward_path(shape, q, k, v, buf: LLSABuffers, stream=None) -> None:
+    """Pyramid, selection and attention forward (steps 1, 2, 4a)."""
+    llsa_build_pyramid(shape, q, k, v, buf.q_pyr, buf.k_pyr, buf.v_pyr, stream)
+    llsa_select(shape, buf.q_pyr, buf.k_pyr, buf.idx, stream)
+    llsa_forward(shape, q, k, v, buf.k_pyr, buf.v_pyr, buf.idx, buf.o, buf.lse, stream)
+
+
+def llsa_backward_path(shape, q, k, v, do, buf: LLSABuffers, stream=None) -> None:
+    """Index transpose and attention backward (steps 5, 4b), after ``llsa_forward_path``."""
+    llsa_index_transpose(shape, buf.idx, buf.row_ptr, buf.col, buf.ws_transpose, stream)
+    llsa_backward(shape, q, k, v, buf.o, buf.lse, do, buf.k_pyr, buf.v_pyr, buf.idx, buf.row_ptr, buf.col,
+                  buf.dq, buf.dk, buf.dv, buf.ws_backward, stream)
+
+
+def llsa_train_step(shape, q, k, v, do, buf: LLSABuffers, stream=None) -> None:
+    """One full LLSA training step of the attention op: forward and backward."""
+    llsa_forward_path(shape, q, k, v, buf, stream)
+    llsa_backward_path(shape, q, k, v, do, buf, stream)
+
+
+# ----------------------------------------------------------------------------- autograd op
+
+class _LLSAFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, topk: int, levels: int):
+        B, H, N, D = q.shape
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        shape = make_shape(B, H, N, D, topk, levels, q.dtype)
+        buf = LLSABuffers.allocate(shape, q.device, q.dtype)
+        llsa_forward_path(shape, q, k, v, buf)
+        ctx.save_for_backward(q, k, v)
+        ctx.buf = buf
+        ctx.shape = shape
+        return buf.o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v = ctx.saved_tensors
+        buf = ctx.buf
+        llsa_backward_path(ctx.shape, q, k, v, do.contiguous(), buf)
+        return buf.dq, buf.dk, buf.dv, None, None
+
+
+def llsa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk: int = 8, levels: int = 1) -> torch.Tensor:
+    """Drop-in for ``F.scaled_dot_product_attention(q, k, v)`` (non-causal, no dropout) on
+    [B, H, N, 64] CUDA tensors, bf16 or fp32, with LLSA's hierarchical block-sparse KV lists."""
+    return _LLSAFunction.apply(q, k, v, topk, levels)
+
+
+def llsa_l1(q, k, v, block_size: int = 16, topk: int = 8):
+    """One pooled level (the README recommends it for sequences shorter than 16384 tokens)."""
+    if block_size != 16:
+        raise ValueError("block_size must be 16")
+    return llsa_attention(q, k, v, topk=topk, levels=1)
+
+
+def llsa_l2(q, k, v, block_size: int = 16, topk: int = 8):
+    """Two pooled levels (the README recommends it from 16384 tokens on)."""
+    if block_size != 16:
+        raise ValueError("block_size must be 16")
+    return llsa_attention(q, k, v, topk=topk, levels=2)

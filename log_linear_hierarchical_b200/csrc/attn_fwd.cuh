@@ -1,0 +1,325 @@
+// Step 4a: block-sparse attention forward with hierarchical KV enrichment (skill page
+// "Log Linear Sparse Attention", Core Technique 2; README usage section: drop-in for
+// non-causal scaled_dot_product_attention with block_size=16).
+//
+// Work unit: one warp owns 4 consecutive query blocks (64 queries).  Those blocks share
+// their level-2.. ancestors, so the coarse KV entries are gathered once per unit.  For each
+// block the warp streams its KV list -- K selected 16-token blocks of K and V, gathered by
+// index with 2-D TMA copies (one 16 x 64 bf16 box per tile, 128-byte swizzle, no multicast)
+// through a ring of mbarrier-tracked stages, then the (L-1)K coarse tokens -- and keeps the
+// online softmax state (row max, row sum, 16 x 64 fp32 output) in registers:
+//   S = Q K^T (mma.sync m16n8k16 bf16, fp32 accumulate), P = exp2(S*scale*log2e - m),
+//   O = O*exp2(m_old - m) + P V.
+// Coarse rows are fp32 in the pyramid; they are rounded to bf16 as they are staged.
+//
+// Bound: the gathered K/V bytes (T * 64 * 2 * 2 per query block; one head's K and V are
+// 16.8 MB at N = 65536, so most re-gathers hit L2) against HBM bandwidth, and the
+// 4 * 16 * T * 64 tensor FLOPs per block.
+#pragma once
+
+#include "llsa_common.cuh"
+
+namespace llsa {
+
+constexpr int kUnitBlocks = 4;   // query blocks per warp unit
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnParams {
+  Geometry g;
+  float scale_log2;   // log2(e) / sqrt(D)
+  float scale;        // 1 / sqrt(D)
+  int warp_bytes;     // shared memory per warp
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// A-operand fragments of a 16 x 64 bf16 tile (rows = M, channels = K) for the 4 k-steps.
+__device__ __forceinline__ void load_a_frags(uint32_t tile, uint32_t (&f)[4][4]) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    ldsm_x4(tile + swz(lane & 15, 2 * kk + (lane >> 4)), f[kk][0], f[kk][1], f[kk][2], f[kk][3]);
+}
+
+// acc[2][4] (16 x 16) += A (16 x 64, fragments) * B^T where B is a 16-row x 64 tile (rows = N).
+__device__ __forceinline__ void mma_a_bt(float (&acc)[2][4], const uint32_t (&a)[4][4], uint32_t btile) {
+  const int lane = lane_id();
+  const int row = (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4(btile + swz(row, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
+    mma_bf16(acc[0], a[kk][0], a[kk][1], a[kk][2], a[kk][3], b0, b1);
+    mma_bf16(acc[1], a[kk][0], a[kk][1], a[kk][2], a[kk][3], b2, b3);
+  }
+}
+
+// acc[8][4] (16 x 64) += A (16 x 16: a0..a3) * B where B is a 16-row x 64 tile (rows = K).
+__device__ __forceinline__ void mma_a_b(float (&acc)[8][4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t btile) {
+  const int lane = lane_id();
+  const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+  for (int dc = 0; dc < 4; ++dc) {
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_t(btile + swz(row, 2 * dc + (lane >> 4)), b0, b1, b2, b3);
+    mma_bf16(acc[2 * dc], a0, a1, a2, a3, b0, b1);
+    mma_bf16(acc[2 * dc + 1], a0, a1, a2, a3, b2, b3);
+  }
+}
+
+// Stage (L-1)K coarse rows of a pyramid (fp32) as bf16 16-row swizzled tiles; padding rows
+// (index >= C) are zero.  Row c is level 2 + c / K, slot c % K of the ancestor's list.
+__device__ __forceinline__ void stage_coarse_rows(const Geometry& g, const float* __restrict__ pyr,
+                                                  const int* __restrict__ idx, int bh, int p, uint32_t dst) {
+  const int lane = lane_id();
+  const int K = g.K;
+  for (int t = lane; t < g.coarse_pad * 8; t += 32) {
+    const int row = t >> 3;
+    const int ch = t & 7;
+    uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+    if (row < g.coarse) {
+      const int lev = 2 + row / K;
+      const int slot = row - (lev - 2) * K;
+      int span = 1;
+      for (int i = 1; i < lev; ++i) span *= kBlock;      // 16^(lev-1)
+      const int anc = p / span;
+      const int nl = g.n[lev];
+      const int j = checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + anc) * K + slot), nl);
+      const float4* src = reinterpret_cast<const float4*>(pyr + g.pyr_off[lev] + ((long long)bh * nl + j) * kD + ch * 8);
+      const float4 x = __ldg(src);
+      const float4 y = __ldg(src + 1);
+      packed = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+    }
+    const uint32_t addr = dst + (row >> 4) * kTileBytes + swz(row & 15, ch);
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(packed.x), "r"(packed.y), "r"(packed.z),
+                 "r"(packed.w)
+                 : "memory");
+  }
+}
+
+// Write a 16 x 64 fp32 accumulator (fragment layout, already scaled) as bf16 rows
+// [row0, row0 + 16) of a [rows, 64] global array, through a swizzled shared staging tile.
+__device__ __forceinline__ void store_tile_bf16(const float (&acc)[8][4], float s0, float s1, uint32_t stage,
+                                                __nv_bfloat16* __restrict__ dst_rows) {
+  const int lane = lane_id();
+  const int r0 = lane >> 2;
+  const uint32_t cb = (lane & 3) * 4;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const uint32_t v0 = pack_bf16(acc[n][0] * s0, acc[n][1] * s0);
+    const uint32_t v1 = pack_bf16(acc[n][2] * s1, acc[n][3] * s1);
+    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(stage + swz(r0, n) + cb), "r"(v0) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(stage + swz(r0 + 8, n) + cb), "r"(v1) : "memory");
+  }
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int ci = lane + 32 * it;
+    const int row = ci >> 3;
+    const int c = ci & 7;
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(stage + swz(row, c)));
+    *reinterpret_cast<uint4*>(dst_rows + row * kD + c * 8) = v;
+  }
+  // the staging tile is refilled by TMA later: order these generic accesses before it
+  fence_proxy_async();
+  __syncwarp();
+}
+
+// One 16-token chunk of the online softmax.  `valid` < 16 masks the padding of the last
+// coarse tile.
+__device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t ktile, uint32_t vtile, int valid,
+                                          float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[8][4]) {
+  const int lane = lane_id();
+  float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  mma_a_bt(s, qf, ktile);
+#pragma unroll
+  for (int n = 0; n < 2; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int col = n * 8 + 2 * (lane & 3) + (e & 1);
+      s[n][e] = (col < valid) ? s[n][e] * scale_log2 : -INFINITY;
+    }
+  float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+  float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float mn0 = fmaxf(m[0], mx0);
+  const float mn1 = fmaxf(m[1], mx1);
+  const float c0 = exp2f(m[0] - mn0);
+  const float c1 = exp2f(m[1] - mn1);
+  float p[2][4];
+#pragma unroll
+  for (int n = 0; n < 2; ++n) {
+    p[n][0] = exp2f(s[n][0] - mn0);
+    p[n][1] = exp2f(s[n][1] - mn0);
+    p[n][2] = exp2f(s[n][2] - mn1);
+    p[n][3] = exp2f(s[n][3] - mn1);
+  }
+  l[0] = l[0] * c0 + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+  l[1] = l[1] * c1 + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
+  m[0] = mn0;
+  m[1] = mn1;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    acc[n][0] *= c0;
+    acc[n][1] *= c0;
+    acc[n][2] *= c1;
+    acc[n][3] *= c1;
+  }
+  mma_a_b(acc, pack_bf16(p[0][0], p[0][1]), pack_bf16(p[0][2], p[0][3]), pack_bf16(p[1][0], p[1][1]),
+          pack_bf16(p[1][2], p[1][3]), vtile);
+}
+
+// Shared-memory map of one forward warp (byte offsets from its 1024-aligned base).
+struct FwdWarpMap {
+  uint32_t q, ring, ck, cv;
+  int* idx;
+  uint32_t bar_q, bar_kv;  // bar_q[2] then bar_kv[STAGES], 8 bytes each
+};
+
+template <int STAGES>
+__device__ __forceinline__ FwdWarpMap fwd_warp_map(uint8_t* base, const Geometry& g) {
+  FwdWarpMap m;
+  const uint32_t b = smem_u32(base);
+  m.q = b;
+  m.ring = b + 2 * kTileBytes;
+  m.ck = m.ring + STAGES * 2 * kTileBytes;
+  m.cv = m.ck + g.coarse_pad * 128;
+  uint8_t* after = base + 2 * kTileBytes + STAGES * 2 * kTileBytes + 2 * g.coarse_pad * 128;
+  m.idx = reinterpret_cast<int*>(after);
+  uint8_t* bars = after + ((kUnitBlocks * g.K * 4 + 15) & ~15);
+  m.bar_q = smem_u32(bars);
+  m.bar_kv = m.bar_q + 16;
+  return m;
+}
+
+template <int STAGES>
+inline int fwd_warp_bytes(const Geometry& g) {
+  int bytes = 2 * kTileBytes + STAGES * 2 * kTileBytes + 2 * g.coarse_pad * 128 + ((kUnitBlocks * g.K * 4 + 15) & ~15) +
+              8 * (2 + STAGES);
+  return (bytes + 1023) & ~1023;
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                            const __grid_constant__ CUtensorMap tm_k,
+                                                            const __grid_constant__ CUtensorMap tm_v, AttnParams P,
+                                                            const float* __restrict__ k_pyr,
+                                                            const float* __restrict__ v_pyr,
+                                                            const int* __restrict__ idx, __nv_bfloat16* __restrict__ o,
+                                                            float* __restrict__ lse) {
+  extern __shared__ uint8_t fwd_smem_raw[];
+  const Geometry& g = P.g;
+  const int lane = lane_id();
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int n1 = g.n[1];
+  const int K = g.K;
+  const int total_blocks = g.BH * n1;
+  const int first = (blockIdx.x * nwarps + warp) * kUnitBlocks;
+  if (first >= total_blocks) return;  // warp-uniform; this kernel has no CTA-wide barrier
+  const int nblk = min(kUnitBlocks, total_blocks - first);
+  const FwdWarpMap sm = fwd_warp_map<STAGES>(align1024(fwd_smem_raw) + warp * P.warp_bytes, g);
+
+  for (int i = lane; i < nblk * K; i += 32)
+    sm.idx[i] = checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1);
+  if (lane == 0) {
+    for (int b = 0; b < 2 + STAGES; ++b) mbar_init(sm.bar_q + 8 * b, 1);
+    mbar_fence_init();
+  }
+  __syncwarp();
+
+  const int total_loads = nblk * K;
+  auto issue_kv = [&](int seq) {
+    const int gb = first + seq / K;
+    const int bh = gb / n1;
+    const int row = bh * g.N + sm.idx[seq] * kBlock;
+    const int stage = seq % STAGES;
+    const uint32_t bar = sm.bar_kv + 8 * stage;
+    const uint32_t dst = sm.ring + stage * 2 * kTileBytes;
+    mbar_expect_tx(bar, 2 * kTileBytes);
+    tma_load_2d(dst, &tm_k, 0, row, bar);
+    tma_load_2d(dst + kTileBytes, &tm_v, 0, row, bar);
+  };
+  auto issue_q = [&](int i) {
+    const uint32_t bar = sm.bar_q + 8 * (i & 1);
+    mbar_expect_tx(bar, kTileBytes);
+    tma_load_2d(sm.q + (i & 1) * kTileBytes, &tm_q, 0, (first + i) * kBlock, bar);
+  };
+  if (lane == 0) {
+    issue_q(0);
+    for (int s = 0; s < min(STAGES, total_loads); ++s) issue_kv(s);
+  }
+  if (g.L >= 2) {
+    const int bh0 = first / n1;
+    const int p0 = first - bh0 * n1;
+    stage_coarse_rows(g, k_pyr, idx, bh0, p0, sm.ck);
+    stage_coarse_rows(g, v_pyr, idx, bh0, p0, sm.cv);
+    __syncwarp();
+  }
+
+  bool ok = true;
+  int next_seq = 0;  // first KV load not yet consumed
+  int next_q = 0;    // first Q load not yet consumed
+  for (int i = 0; i < nblk && ok; ++i) {
+    const int gb = first + i;
+    ok = __all_sync(0xffffffffu, mbar_wait(sm.bar_q + 8 * (i & 1), (i >> 1) & 1));
+    if (!ok) break;
+    next_q = i + 1;
+    uint32_t qf[4][4];
+    load_a_frags(sm.q + (i & 1) * kTileBytes, qf);
+    __syncwarp();
+    if (lane == 0 && i + 1 < nblk) issue_q(i + 1);
+
+    float m[2] = {-INFINITY, -INFINITY};
+    float l[2] = {0.f, 0.f};
+    float acc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+
+    for (int s = 0; s < K; ++s) {
+      const int seq = i * K + s;
+      const int stage = seq % STAGES;
+      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar_kv + 8 * stage, (seq / STAGES) & 1));
+      if (!ok) break;
+      next_seq = seq + 1;
+      const uint32_t kt = sm.ring + stage * 2 * kTileBytes;
+      fwd_chunk(qf, kt, kt + kTileBytes, kBlock, P.scale_log2, m, l, acc);
+      __syncwarp();
+      if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
+    }
+    if (!ok) break;
+    for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
+      fwd_chunk(qf, sm.ck + cc * kTileBytes, sm.cv + cc * kTileBytes, min(kBlock, g.coarse - cc * kBlock),
+                P.scale_log2, m, l, acc);
+
+    l[0] += __shfl_xor_sync(0xffffffffu, l[0], 1);
+    l[0] += __shfl_xor_sync(0xffffffffu, l[0], 2);
+    l[1] += __shfl_xor_sync(0xffffffffu, l[1], 1);
+    l[1] += __shfl_xor_sync(0xffffffffu, l[1], 2);
+    store_tile_bf16(acc, 1.0f / l[0], 1.0f / l[1], sm.q + (i & 1) * kTileBytes, o + (long long)gb * kBlock * kD);
+    if ((lane & 3) == 0) {
+      const int r0 = lane >> 2;
+      lse[(long long)gb * kBlock + r0] = (m[0] + log2f(l[0])) * kLn2;
+      lse[(long long)gb * kBlock + r0 + 8] = (m[1] + log2f(l[1])) * kLn2;
+    }
+  }
+  if (!ok) {
+    // A copy did not land in time (recorded as LLSA_ERR_TIMEOUT).  Give each copy still in
+    // flight one more bounded wait so none lands after this warp has gone.
+    for (int seq = next_seq; seq < min(total_loads, next_seq + STAGES); ++seq)
+      mbar_wait(sm.bar_kv + 8 * (seq % STAGES), (seq / STAGES) & 1);
+    for (int i = next_q; i < min(nblk, next_q + 2); ++i) mbar_wait(sm.bar_q + 8 * (i & 1), (i >> 1) & 1);
+  }
+}
+
+}  // namespace llsa

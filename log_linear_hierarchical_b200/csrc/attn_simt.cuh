@@ -1,0 +1,295 @@
+// Steps 4a/4b for fp32 inputs: plain fp32 CUDA-core kernels with the same KV lists,
+// workspace layout and coarse-gradient reduction as the bf16 tensor-core kernels.  fp32
+// tensor-core modes round operands to 10 mantissa bits, which would not meet a 1e-4
+// tolerance, so this path uses FMA units.  It is the small-problem / full-precision path;
+// the bf16 kernels are the throughput path.
+#pragma once
+
+#include "attn_bwd.cuh"
+
+namespace llsa {
+
+constexpr int kSimtThreads = 128;
+
+// Row pointers of block p's KV list: 16K fine tokens then (L-1)K coarse pyramid rows.
+__device__ __forceinline__ void simt_kv_rows(const Geometry& g, int bh, int p, const float* __restrict__ k,
+                                             const float* __restrict__ v, const float* __restrict__ k_pyr,
+                                             const float* __restrict__ v_pyr, const int* __restrict__ idx,
+                                             const float** krow, const float** vrow) {
+  const int K = g.K;
+  const int n1 = g.n[1];
+  const int T = kBlock * K + g.coarse;
+  for (int e = threadIdx.x; e < T; e += blockDim.x) {
+    long long r;
+    const float* kb;
+    const float* vb;
+    if (e < kBlock * K) {
+      const int j = checked_index(__ldg(idx + g.idx_off[1] + ((long long)bh * n1 + p) * K + e / kBlock), n1);
+      r = (long long)bh * g.N + (long long)j * kBlock + (e % kBlock);
+      kb = k;
+      vb = v;
+    } else {
+      const int c = e - kBlock * K;
+      const int lev = 2 + c / K;
+      const int slot = c - (lev - 2) * K;
+      int span = 1;
+      for (int i = 1; i < lev; ++i) span *= kBlock;
+      const int nl = g.n[lev];
+      const int jj = checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + p / span) * K + slot), nl);
+      r = (long long)bh * nl + jj;
+      kb = k_pyr + g.pyr_off[lev];
+      vb = v_pyr + g.pyr_off[lev];
+    }
+    krow[e] = kb + r * kD;
+    vrow[e] = vb + r * kD;
+  }
+}
+
+__device__ __forceinline__ float dot64(const float* a, const float* b) {
+  float s = 0.f;
+#pragma unroll 16
+  for (int d = 0; d < kD; ++d) s = fmaf(a[d], b[d], s);
+  return s;
+}
+
+// One CTA per query block.  smem: q[16][64], krow[T], vrow[T], S[16][T].
+__global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, float scale,
+                                                                    const float* __restrict__ q,
+                                                                    const float* __restrict__ k,
+                                                                    const float* __restrict__ v,
+                                                                    const float* __restrict__ k_pyr,
+                                                                    const float* __restrict__ v_pyr,
+                                                                    const int* __restrict__ idx, float* __restrict__ o,
+                                                                    float* __restrict__ lse) {
+  extern __shared__ __align__(16) uint8_t simt_smem[];
+  const int T = kBlock * g.K + g.coarse;
+  const int gb = blockIdx.x;
+  const int bh = gb / g.n[1];
+  const int p = gb - bh * g.n[1];
+  float* qs = reinterpret_cast<float*>(simt_smem);
+  const float** krow = reinterpret_cast<const float**>(qs + kBlock * kD);
+  const float** vrow = krow + T;
+  float* S = reinterpret_cast<float*>(vrow + T);
+  const float* qb = q + (long long)gb * kBlock * kD;
+  for (int i = threadIdx.x; i < kBlock * kD; i += blockDim.x) qs[i] = qb[i];
+  simt_kv_rows(g, bh, p, k, v, k_pyr, v_pyr, idx, krow, vrow);
+  __syncthreads();
+  for (int pr = threadIdx.x; pr < kBlock * T; pr += blockDim.x) {
+    const int qi = pr / T;
+    const int e = pr - qi * T;
+    S[pr] = dot64(qs + qi * kD, krow[e]) * scale;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int qi = warp; qi < kBlock; qi += blockDim.x >> 5) {
+    float* row = S + qi * T;
+    float m = -INFINITY;
+    for (int e = lane; e < T; e += 32) m = fmaxf(m, row[e]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float l = 0.f;
+    for (int e = lane; e < T; e += 32) {
+      const float pe = expf(row[e] - m);
+      row[e] = pe;
+      l += pe;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    const float inv = 1.0f / l;
+    for (int e = lane; e < T; e += 32) row[e] *= inv;
+    if (lane == 0) lse[(long long)gb * kBlock + qi] = m + logf(l);
+  }
+  __syncthreads();
+  for (int od = threadIdx.x; od < kBlock * kD; od += blockDim.x) {
+    const int qi = od / kD;
+    const int d = od - qi * kD;
+    const float* prow = S + qi * T;
+    float acc = 0.f;
+    for (int e = 0; e < T; ++e) acc = fmaf(prow[e], vrow[e][d], acc);
+    o[(long long)gb * kBlock * kD + od] = acc;
+  }
+}
+
+inline size_t simt_fwd_smem(const Geometry& g) {
+  const int T = kBlock * g.K + g.coarse;
+  return sizeof(float) * kBlock * kD + 2 * sizeof(void*) * T + sizeof(float) * kBlock * T;
+}
+
+// Query-major fp32 backward.  One CTA per level-2 group (16 query blocks) when L >= 2, so
+// the coarse partials match the bf16 path's layout; one CTA per query block when L = 1.
+// smem: q, dO [16][64]; krow, vrow [T]; P, dS [16][T]; cacc_k, cacc_v [C][64]; delta[16].
+__global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
+    Geometry g, float scale, const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    const float* __restrict__ o, const float* __restrict__ lse, const float* __restrict__ dO,
+    const float* __restrict__ k_pyr, const float* __restrict__ v_pyr, const int* __restrict__ idx,
+    float* __restrict__ dq_out, float* __restrict__ ws) {
+  extern __shared__ __align__(16) uint8_t simt_smem[];
+  const BwdWorkspace W = bwd_workspace_layout(g);
+  const int T = kBlock * g.K + g.coarse;
+  const int C = g.coarse;
+  const int per_cta = g.L >= 2 ? kBlock : 1;
+  float* qs = reinterpret_cast<float*>(simt_smem);
+  float* ds_ = qs + kBlock * kD;  // dO rows
+  const float** krow = reinterpret_cast<const float**>(ds_ + kBlock * kD);
+  const float** vrow = krow + T;
+  float* Pm = reinterpret_cast<float*>(vrow + T);
+  float* dS = Pm + kBlock * T;
+  float* cacc_k = dS + kBlock * T;
+  float* cacc_v = cacc_k + C * kD;
+  float* delta = cacc_v + C * kD;
+  for (int i = threadIdx.x; i < 2 * C * kD; i += blockDim.x) cacc_k[i] = 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int bi = 0; bi < per_cta; ++bi) {
+    const int gb = blockIdx.x * per_cta + bi;
+    const int bh = gb / g.n[1];
+    const int p = gb - bh * g.n[1];
+    const long long rbase = (long long)gb * kBlock;
+    __syncthreads();
+    for (int i = threadIdx.x; i < kBlock * kD; i += blockDim.x) {
+      qs[i] = q[rbase * kD + i];
+      ds_[i] = dO[rbase * kD + i];
+    }
+    simt_kv_rows(g, bh, p, k, v, k_pyr, v_pyr, idx, krow, vrow);
+    for (int qi = warp; qi < kBlock; qi += blockDim.x >> 5) {
+      float s = 0.f;
+      for (int d = lane; d < kD; d += 32) s = fmaf(dO[(rbase + qi) * kD + d], o[(rbase + qi) * kD + d], s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      if (lane == 0) {
+        delta[qi] = s;
+        ws[W.delta + rbase + qi] = s;
+      }
+    }
+    __syncthreads();
+    for (int pr = threadIdx.x; pr < kBlock * T; pr += blockDim.x) {
+      const int qi = pr / T;
+      const int e = pr - qi * T;
+      const float pe = expf(dot64(qs + qi * kD, krow[e]) * scale - lse[rbase + qi]);
+      const float dp = dot64(ds_ + qi * kD, vrow[e]);
+      Pm[pr] = pe;
+      dS[pr] = pe * (dp - delta[qi]);
+    }
+    __syncthreads();
+    for (int od = threadIdx.x; od < kBlock * kD; od += blockDim.x) {
+      const int qi = od / kD;
+      const int d = od - qi * kD;
+      float acc = 0.f;
+      for (int e = 0; e < T; ++e) acc = fmaf(dS[qi * T + e], krow[e][d], acc);
+      dq_out[rbase * kD + od] = acc * scale;
+    }
+    for (int cd = threadIdx.x; cd < C * kD; cd += blockDim.x) {
+      const int c = cd / kD;
+      const int d = cd - c * kD;
+      const int e = kBlock * g.K + c;
+      float ak = 0.f, av = 0.f;
+      for (int qi = 0; qi < kBlock; ++qi) {
+        ak = fmaf(dS[qi * T + e], qs[qi * kD + d], ak);
+        av = fmaf(Pm[qi * T + e], ds_[qi * kD + d], av);
+      }
+      cacc_k[cd] += ak;
+      cacc_v[cd] += av;
+    }
+  }
+  if (g.L < 2) return;
+  __syncthreads();
+  const int group = blockIdx.x;
+  for (int cd = threadIdx.x; cd < C * kD; cd += blockDim.x) {
+    ws[W.part_k + (long long)group * C * kD + cd] = cacc_k[cd];
+    ws[W.part_v + (long long)group * C * kD + cd] = cacc_v[cd];
+  }
+}
+
+inline size_t simt_dq_smem(const Geometry& g) {
+  const int T = kBlock * g.K + g.coarse;
+  return sizeof(float) * 2 * kBlock * kD + 2 * sizeof(void*) * T + sizeof(float) * 2 * kBlock * T +
+         sizeof(float) * 2 * g.coarse * kD + sizeof(float) * kBlock;
+}
+
+// Key-major fp32 backward: one CTA per fine key block; thread t owns 8 of the 16 x 64 dK and
+// dV outputs.  smem: K_j, V_j, Q_p, dO_p [16][64]; Pt, dSt [16][16]; lse, delta [16].
+__global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
+    Geometry g, float scale, const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    const float* __restrict__ lse, const float* __restrict__ dO, const int* __restrict__ row_ptr,
+    const int* __restrict__ col, const float* __restrict__ ws, float* __restrict__ dk_out,
+    float* __restrict__ dv_out) {
+  __shared__ float ks[kBlock * kD], vs[kBlock * kD], qs[kBlock * kD], dos[kBlock * kD];
+  __shared__ float Pt[kBlock][kBlock + 1], dSt[kBlock][kBlock + 1];
+  __shared__ float ls[kBlock], dl[kBlock];
+  const BwdWorkspace W = bwd_workspace_layout(g);
+  const int n1 = g.n[1];
+  const int kb = blockIdx.x;
+  const int bh = kb / n1;
+  const int j = kb - bh * n1;
+  const long long krow0 = (long long)bh * g.N + (long long)j * kBlock;
+  for (int i = threadIdx.x; i < kBlock * kD; i += blockDim.x) {
+    ks[i] = k[krow0 * kD + i];
+    vs[i] = v[krow0 * kD + i];
+  }
+  const int E = n1 * g.K;
+  const int* rp = row_ptr + g.rp_off[1] + (long long)bh * (n1 + 1);
+  int rs = rp[j], re = rp[j + 1];
+  if (rs < 0 || re > E || rs > re) {
+    if (threadIdx.x == 0) record_error(LLSA_ERR_INTERNAL);
+    rs = re = 0;
+  }
+  const int* cl = col + g.idx_off[1] + (long long)bh * E;
+  float ak[8], av[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ak[i] = av[i] = 0.f;
+  for (int e = rs; e < re; ++e) {
+    const int p = checked_index(cl[e], n1);
+    const long long qrow0 = (long long)bh * g.N + (long long)p * kBlock;
+    __syncthreads();
+    for (int i = threadIdx.x; i < kBlock * kD; i += blockDim.x) {
+      qs[i] = q[qrow0 * kD + i];
+      dos[i] = dO[qrow0 * kD + i];
+    }
+    if (threadIdx.x < kBlock) {
+      ls[threadIdx.x] = lse[qrow0 + threadIdx.x];
+      dl[threadIdx.x] = ws[W.delta + qrow0 + threadIdx.x];
+    }
+    __syncthreads();
+    for (int pr = threadIdx.x; pr < kBlock * kBlock; pr += blockDim.x) {
+      const int kk = pr / kBlock;
+      const int qi = pr - kk * kBlock;
+      const float pe = expf(dot64(ks + kk * kD, qs + qi * kD) * scale - ls[qi]);
+      const float dp = dot64(vs + kk * kD, dos + qi * kD);
+      Pt[kk][qi] = pe;
+      dSt[kk][qi] = pe * (dp - dl[qi]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int od = threadIdx.x + i * kSimtThreads;
+      const int kk = od / kD;
+      const int d = od - kk * kD;
+      float a = 0.f, b = 0.f;
+      for (int qi = 0; qi < kBlock; ++qi) {
+        a = fmaf(dSt[kk][qi], qs[qi * kD + d], a);
+        b = fmaf(Pt[kk][qi], dos[qi * kD + d], b);
+      }
+      ak[i] += a;
+      av[i] += b;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int od = threadIdx.x + i * kSimtThreads;
+    const int kk = od / kD;
+    const int d = od - kk * kD;
+    float rk = ak[i] * scale, rv = av[i];
+    int span = 1;
+    float wgt = 1.0f / kBlock;
+    for (int lev = 2; lev <= g.L; ++lev) {
+      span *= kBlock;
+      wgt *= 1.0f / kBlock;
+      const long long crow = W.cg_off[lev] + ((long long)bh * g.n[lev] + j / span) * kD + d;
+      rk += wgt * ws[W.cg_k + crow];
+      rv += wgt * ws[W.cg_v + crow];
+    }
+    dk_out[(krow0 + kk) * kD + d] = rk;
+    dv_out[(krow0 + kk) * kD + d] = rv;
+  }
+}
+
+}  // namespace llsa

@@ -1,0 +1,478 @@
+// C ABI of the LLSA hot path (declarations and contracts in include/llsa.h).
+// Single translation unit: every kernel header is included here, so the device status word
+// is one module global per device.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "attn_simt.cuh"
+#include "pyramid.cuh"
+#include "select.cuh"
+#include "transpose.cuh"
+
+using namespace llsa;
+
+namespace {
+
+bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int ilog2(long long x) {
+  int r = 0;
+  while ((1LL << r) < x) ++r;
+  return r;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+llsa_status validate(const llsa_shape* s) {
+  if (!s) return LLSA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->N < 1 || s->D < 1 || s->block < 1 || s->topk < 1 || s->levels < 1)
+    return LLSA_ERR_INVALID_ARG;
+  if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
+  if (!is_pow2(s->N) || !is_pow2(s->topk)) return LLSA_ERR_INVALID_ARG;  // README usage notes
+  if (s->block != kBlock) return LLSA_ERR_UNSUPPORTED;
+  if (s->D != kD) return LLSA_ERR_UNSUPPORTED;
+  if (s->levels > kMaxLevels) return LLSA_ERR_UNSUPPORTED;
+  if (ilog2(s->N) < 4 * s->levels) return LLSA_ERR_INVALID_ARG;  // need N / 16^L >= 1
+  const long long nL = (long long)s->N >> (4 * s->levels);
+  if (s->topk > nL) return LLSA_ERR_INVALID_ARG;  // the coarsest level must hold K keys
+  if (s->N > (1 << 20)) return LLSA_ERR_UNSUPPORTED;
+  if (nL > 16384) return LLSA_ERR_UNSUPPORTED;
+  if (s->topk > 64) return LLSA_ERR_UNSUPPORTED;
+  if ((long long)(s->levels - 1) * s->topk > 32) return LLSA_ERR_UNSUPPORTED;
+  if ((long long)s->B * s->H * s->N >= (1LL << 31)) return LLSA_ERR_UNSUPPORTED;
+  return LLSA_OK;
+}
+
+Geometry make_geometry(const llsa_shape* s) {
+  Geometry g{};
+  g.B = s->B;
+  g.H = s->H;
+  g.N = s->N;
+  g.D = s->D;
+  g.K = s->topk;
+  g.L = s->levels;
+  g.BH = s->B * s->H;
+  for (int l = 0; l <= g.L; ++l) g.n[l] = s->N >> (4 * l);
+  long long po = 0, io = 0, ro = 0;
+  for (int l = 1; l <= g.L; ++l) {
+    g.pyr_off[l] = po;
+    g.idx_off[l] = io;
+    g.rp_off[l] = ro;
+    po += (long long)g.BH * g.n[l] * kD;
+    io += (long long)g.BH * g.n[l] * g.K;
+    ro += (long long)g.BH * (g.n[l] + 1);
+  }
+  g.coarse = (g.L - 1) * g.K;
+  g.coarse_pad = (g.coarse + kBlock - 1) / kBlock * kBlock;
+  return g;
+}
+
+TransposeGeo make_transpose_geo(const Geometry& g, long long* ent_total, long long* hist_total) {
+  TransposeGeo t{};
+  t.L = g.L;
+  t.BH = g.BH;
+  t.K = g.K;
+  int cta_t = 0, cta_b = 0;
+  long long hist = 0;
+  for (int l = 1; l <= g.L; ++l) {
+    TransposeLevel& L = t.lv[l - 1];
+    L.n = g.n[l];
+    L.E = g.n[l] * g.K;
+    L.tiles = (L.E + kTrTile - 1) / kTrTile;
+    L.nb = L.n < kTrMaxBuckets ? L.n : kTrMaxBuckets;
+    L.wshift = ilog2(L.n / L.nb);
+    L.cta_tiles = cta_t;
+    L.cta_buckets = cta_b;
+    L.hist_off = hist;
+    L.ent_off = g.idx_off[l];
+    L.rp_off = g.rp_off[l];
+    cta_t += g.BH * L.tiles;
+    cta_b += g.BH * L.nb;
+    hist += (long long)g.BH * L.nb * L.tiles;
+  }
+  *ent_total = (long long)g.BH * g.K * [&] {
+    long long s = 0;
+    for (int l = 1; l <= g.L; ++l) s += g.n[l];
+    return s;
+  }();
+  *hist_total = hist;
+  return t;
+}
+
+size_t transpose_ws_bytes(const Geometry& g) {
+  long long ent, hist;
+  make_transpose_geo(g, &ent, &hist);
+  return (size_t)(((ent + 63) & ~63LL) + hist) * 4;
+}
+
+// ---------------------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [rows, 64] bf16 row-major viewed as 2-D; box = 16 rows x 64 channels, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* m, const void* base, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)kBlock};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+llsa_status launch_status() { return cudaGetLastError() == cudaSuccess ? LLSA_OK : LLSA_ERR_CUDA; }
+
+template <typename Kern>
+bool allow_smem(Kern k, size_t bytes) {
+  if (bytes <= 48 * 1024) return true;
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------- launch trace
+enum KernelId {
+  kKPyramidL12 = 1,
+  kKPyramidUp,
+  kKSelect,
+  kKTransposeHist,
+  kKTransposeScatter,
+  kKTransposeBucket,
+  kKFwdBf16,
+  kKBwdDqBf16,
+  kKBwdCoarseReduce,
+  kKBwdDkdvBf16,
+  kKFwdF32,
+  kKBwdDqF32,
+  kKBwdDkdvF32,
+  kKNumKernels
+};
+
+const char* const kKernelNames[kKNumKernels] = {
+    "unknown",          "pyramid_l12",          "pyramid_up",   "select",           "transpose_hist",
+    "transpose_scatter", "transpose_bucket",    "attn_fwd_bf16", "attn_bwd_dq_bf16", "coarse_grad_reduce",
+    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32"};
+
+struct TraceState {
+  cudaEvent_t* ev = nullptr;
+  int32_t* ids = nullptr;
+  int cap = 0;
+  int used = 0;
+};
+thread_local TraceState g_trace;
+
+// Launches through `f`, checks the launch, and records the trace events if tracing is on.
+template <class F>
+llsa_status launch(int id, cudaStream_t cs, F&& f) {
+  const bool tr = g_trace.ev != nullptr && g_trace.used < g_trace.cap;
+  if (tr) cudaEventRecord(g_trace.ev[2 * g_trace.used], cs);
+  f();
+  const llsa_status st = launch_status();
+  if (tr) {
+    cudaEventRecord(g_trace.ev[2 * g_trace.used + 1], cs);
+    g_trace.ids[g_trace.used] = id;
+    ++g_trace.used;
+  }
+  return st;
+}
+
+constexpr int kFwdStages = 4;
+constexpr int kDqStages = 2;
+constexpr int kDkvStages = 3;
+constexpr int kAttnWarps = 4;
+
+llsa_status launch_coarse_reduce(const Geometry& g, float scale, const int32_t* idx, const int32_t* row_ptr,
+                                 const int32_t* col, float* ws, cudaStream_t cs) {
+  if (g.L < 2) return LLSA_OK;
+  long long warps = 0;
+  for (int l = 2; l <= g.L; ++l) warps += (long long)g.BH * g.n[l];
+  return launch(kKBwdCoarseReduce, cs, [&] {
+    coarse_grad_reduce_kernel<<<(unsigned)((warps * 32 + 127) / 128), 128, 0, cs>>>(g, scale, idx, row_ptr, col, ws);
+  });
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* llsa_status_string(llsa_status s) {
+  switch (s) {
+    case LLSA_OK: return "ok";
+    case LLSA_ERR_INVALID_ARG: return "invalid argument";
+    case LLSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case LLSA_ERR_WORKSPACE: return "workspace too small";
+    case LLSA_ERR_CUDA: return "CUDA launch or runtime error";
+    case LLSA_ERR_INTERNAL: return "out-of-range index seen on the device";
+    case LLSA_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+llsa_status llsa_validate_shape(const llsa_shape* shape) { return validate(shape); }
+
+size_t llsa_pyramid_elems(const llsa_shape* s) {
+  if (validate(s) != LLSA_OK) return 0;
+  const Geometry g = make_geometry(s);
+  return (size_t)(g.pyr_off[g.L] + (long long)g.BH * g.n[g.L] * kD);
+}
+
+size_t llsa_index_elems(const llsa_shape* s) {
+  if (validate(s) != LLSA_OK) return 0;
+  const Geometry g = make_geometry(s);
+  return (size_t)(g.idx_off[g.L] + (long long)g.BH * g.n[g.L] * g.K);
+}
+
+size_t llsa_row_ptr_elems(const llsa_shape* s) {
+  if (validate(s) != LLSA_OK) return 0;
+  const Geometry g = make_geometry(s);
+  return (size_t)(g.rp_off[g.L] + (long long)g.BH * (g.n[g.L] + 1));
+}
+
+size_t llsa_transpose_workspace_bytes(const llsa_shape* s) {
+  if (validate(s) != LLSA_OK) return 0;
+  return transpose_ws_bytes(make_geometry(s));
+}
+
+size_t llsa_backward_workspace_bytes(const llsa_shape* s) {
+  if (validate(s) != LLSA_OK) return 0;
+  return (size_t)bwd_workspace_layout(make_geometry(s)).total * sizeof(float);
+}
+
+llsa_status llsa_build_pyramid(const llsa_shape* s, const void* q, const void* k, const void* v, float* q_pyr,
+                               float* k_pyr, float* v_pyr, llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  const void* ptrs[6] = {q, k, v, q_pyr, k_pyr, v_pyr};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (s->dtype == LLSA_BF16) {
+    constexpr int rows = kPyrThreads / (kD / 8);
+    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
+    st = launch(kKPyramidL12, cs, [&] {
+      pyramid_l12_kernel<__nv_bfloat16><<<grid, kPyrThreads, 0, cs>>>(
+          g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+          static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr);
+    });
+  } else {
+    constexpr int rows = kPyrThreads / (kD / 4);
+    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
+    st = launch(kKPyramidL12, cs, [&] {
+      pyramid_l12_kernel<float><<<grid, kPyrThreads, 0, cs>>>(g, static_cast<const float*>(q),
+                                                               static_cast<const float*>(k),
+                                                               static_cast<const float*>(v), q_pyr, k_pyr, v_pyr);
+    });
+  }
+  if (st != LLSA_OK) return st;
+  for (int l = 3; l <= g.L; ++l) {
+    const long long total = (long long)g.BH * g.n[l] * kD;
+    dim3 grid((unsigned)((total + kPyrThreads - 1) / kPyrThreads), 3);
+    st = launch(kKPyramidUp, cs, [&] { pyramid_up_kernel<<<grid, kPyrThreads, 0, cs>>>(g, l, q_pyr, k_pyr, v_pyr); });
+    if (st != LLSA_OK) return st;
+  }
+  return LLSA_OK;
+}
+
+llsa_status llsa_select(const llsa_shape* s, const float* q_pyr, const float* k_pyr, int32_t* idx,
+                        llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  if (!q_pyr || !k_pyr || !idx || !aligned16(q_pyr) || !aligned16(k_pyr) || !aligned16(idx))
+    return LLSA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  for (int l = g.L; l >= 1; --l) {
+    const bool sparse = l < g.L;
+    const int n = g.n[l];
+    int gq, nc;
+    if (sparse) {
+      gq = kBlock;
+      nc = kBlock * g.K;
+    } else {
+      nc = n;
+      gq = kBlock;
+      while (gq > 1 && (gq > n || (long long)gq * n > 16384)) gq >>= 1;
+    }
+    const size_t smem = select_smem_bytes(gq, nc, g.K, sparse);
+    if (!allow_smem(select_kernel, smem)) return LLSA_ERR_CUDA;
+    const int groups = (n + gq - 1) / gq;
+    st = launch(kKSelect, cs, [&] {
+      select_kernel<<<g.BH * groups, kSelThreads, smem, cs>>>(g, l, gq, q_pyr + g.pyr_off[l], k_pyr + g.pyr_off[l],
+                                                             sparse ? idx + g.idx_off[l + 1] : nullptr,
+                                                             idx + g.idx_off[l]);
+    });
+    if (st != LLSA_OK) return st;
+  }
+  return LLSA_OK;
+}
+
+llsa_status llsa_index_transpose(const llsa_shape* s, const int32_t* idx, int32_t* row_ptr, int32_t* col,
+                                 void* workspace, size_t workspace_bytes, llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  if (!idx || !row_ptr || !col || !workspace || !aligned16(idx) || !aligned16(row_ptr) || !aligned16(col) ||
+      !aligned16(workspace))
+    return LLSA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s);
+  if (workspace_bytes < transpose_ws_bytes(g)) return LLSA_ERR_WORKSPACE;
+  long long ent_total, hist_total;
+  const TransposeGeo tg = make_transpose_geo(g, &ent_total, &hist_total);
+  uint32_t* ws_ent = static_cast<uint32_t*>(workspace);
+  int* ws_hist = reinterpret_cast<int*>(ws_ent + ((ent_total + 63) & ~63LL));
+  const TransposeLevel& last = tg.lv[g.L - 1];
+  const int tile_ctas = last.cta_tiles + g.BH * last.tiles;
+  const int bucket_ctas = last.cta_buckets + g.BH * last.nb;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  st = launch(kKTransposeHist, cs,
+              [&] { transpose_hist_kernel<<<tile_ctas, kTrThreads, 0, cs>>>(tg, idx, ws_hist); });
+  if (st != LLSA_OK) return st;
+  st = launch(kKTransposeScatter, cs,
+              [&] { transpose_scatter_kernel<<<tile_ctas, kTrThreads, 0, cs>>>(tg, idx, ws_hist, ws_ent); });
+  if (st != LLSA_OK) return st;
+  return launch(kKTransposeBucket, cs, [&] {
+    transpose_bucket_kernel<<<bucket_ctas, kTrThreads, 0, cs>>>(tg, ws_ent, ws_hist, row_ptr, col);
+  });
+}
+
+llsa_status llsa_forward(const llsa_shape* s, const void* q, const void* k, const void* v, const float* k_pyr,
+                         const float* v_pyr, const int32_t* idx, void* o, float* lse, llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  const void* ptrs[8] = {q, k, v, k_pyr, v_pyr, idx, o, lse};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const float scale = 1.0f / sqrtf((float)kD);
+  const int total_blocks = g.BH * g.n[1];
+  if (s->dtype == LLSA_BF16) {
+    CUtensorMap tq, tk, tv;
+    const long long rows = (long long)g.BH * g.N;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
+      return LLSA_ERR_CUDA;
+    AttnParams P{g, scale * kLog2e, scale, fwd_warp_bytes<kFwdStages>(g)};
+    const size_t smem = (size_t)kAttnWarps * P.warp_bytes + 1024;
+    auto kern = attn_fwd_bf16_kernel<kFwdStages>;
+    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+    const int per_cta = kAttnWarps * kUnitBlocks;
+    return launch(kKFwdBf16, cs, [&] {
+      kern<<<(total_blocks + per_cta - 1) / per_cta, 32 * kAttnWarps, smem, cs>>>(
+          tq, tk, tv, P, k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse);
+    });
+  }
+  const size_t smem = simt_fwd_smem(g);
+  if (!allow_smem(attn_fwd_f32_kernel, smem)) return LLSA_ERR_CUDA;
+  return launch(kKFwdF32, cs, [&] {
+    attn_fwd_f32_kernel<<<total_blocks, kSimtThreads, smem, cs>>>(
+        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
+        v_pyr, idx, static_cast<float*>(o), lse);
+  });
+}
+
+llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
+                          const int32_t* idx, const int32_t* row_ptr, const int32_t* col, void* dq, void* dk,
+                          void* dv, void* workspace, size_t workspace_bytes, llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  const void* ptrs[16] = {q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s);
+  const BwdWorkspace W = bwd_workspace_layout(g);
+  if (workspace_bytes < (size_t)W.total * sizeof(float)) return LLSA_ERR_WORKSPACE;
+  float* ws = static_cast<float*>(workspace);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const float scale = 1.0f / sqrtf((float)kD);
+  const int total_blocks = g.BH * g.n[1];
+  if (s->dtype == LLSA_BF16) {
+    CUtensorMap tq, tk, tv, tdo;
+    const long long rows = (long long)g.BH * g.N;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
+        !make_tile_map(&tdo, dO, rows))
+      return LLSA_ERR_CUDA;
+    {
+      AttnParams P{g, scale * kLog2e, scale, dq_warp_bytes<kDqStages>(g)};
+      const size_t smem = (size_t)kAttnWarps * P.warp_bytes + 1024;
+      auto kern = attn_bwd_dq_bf16_kernel<kDqStages>;
+      if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+      const int per_cta = kAttnWarps * kUnitBlocks;
+      st = launch(kKBwdDqBf16, cs, [&] {
+        kern<<<(total_blocks + per_cta - 1) / per_cta, 32 * kAttnWarps, smem, cs>>>(
+            tq, tk, tv, tdo, P, k_pyr, v_pyr, idx, static_cast<const __nv_bfloat16*>(o), lse,
+            static_cast<__nv_bfloat16*>(dq), ws);
+      });
+      if (st != LLSA_OK) return st;
+    }
+    if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
+    AttnParams P{g, scale * kLog2e, scale, dkv_warp_bytes<kDkvStages>()};
+    const size_t smem = (size_t)kAttnWarps * P.warp_bytes + 1024;
+    auto kern = attn_bwd_dkdv_bf16_kernel<kDkvStages>;
+    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+    return launch(kKBwdDkdvBf16, cs, [&] {
+      kern<<<(total_blocks + kAttnWarps - 1) / kAttnWarps, 32 * kAttnWarps, smem, cs>>>(
+          tq, tk, tv, tdo, P, lse, row_ptr, col, ws, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+    });
+  }
+  const size_t smem = simt_dq_smem(g);
+  if (!allow_smem(attn_bwd_dq_f32_kernel, smem)) return LLSA_ERR_CUDA;
+  const int per_cta = g.L >= 2 ? kBlock : 1;
+  st = launch(kKBwdDqF32, cs, [&] {
+    attn_bwd_dq_f32_kernel<<<total_blocks / per_cta, kSimtThreads, smem, cs>>>(
+        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<const float*>(o), lse, static_cast<const float*>(dO), k_pyr, v_pyr, idx,
+        static_cast<float*>(dq), ws);
+  });
+  if (st != LLSA_OK) return st;
+  if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
+  return launch(kKBwdDkdvF32, cs, [&] {
+    attn_bwd_dkdv_f32_kernel<<<total_blocks, kSimtThreads, 0, cs>>>(
+        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), lse,
+        static_cast<const float*>(dO), row_ptr, col, ws, static_cast<float*>(dk), static_cast<float*>(dv));
+  });
+}
+
+llsa_status llsa_device_status(int32_t* code_out, llsa_stream_t stream) {
+  if (!code_out) return LLSA_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return LLSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_llsa_status, sizeof(int)) != cudaSuccess) return LLSA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_llsa_status, &zero, sizeof(int)) != cudaSuccess) return LLSA_ERR_CUDA;
+  *code_out = v;
+  return LLSA_OK;
+}
+
+llsa_status llsa_trace_begin(void** events, int32_t* kernel_ids, int32_t capacity) {
+  if (!events || !kernel_ids || capacity < 0) return LLSA_ERR_INVALID_ARG;
+  g_trace.ev = reinterpret_cast<cudaEvent_t*>(events);
+  g_trace.ids = kernel_ids;
+  g_trace.cap = capacity;
+  g_trace.used = 0;
+  return LLSA_OK;
+}
+
+llsa_status llsa_trace_end(int32_t* launches_out) {
+  if (launches_out) *launches_out = g_trace.used;
+  g_trace = TraceState{};
+  return LLSA_OK;
+}
+
+const char* llsa_kernel_name(int32_t kernel_id) {
+  return (kernel_id > 0 && kernel_id < kKNumKernels) ? kKernelNames[kernel_id] : kKernelNames[0];
+}
+
+}  // extern "C"

@@ -185,27 +185,30 @@ def kv_index_table(b: int, h: int, idx: list[np.ndarray], offsets: list[int]) ->
 
 # ----------------------------------------------------------------------------- step 4: attention
 
-def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256):
+def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None):
     """Softmax attention of every query over its block's KV list.
 
     Returns (O [B, H, N, D], LSE [B, H, N]) in fp64.  For query i of block p with
     list E(p): z_e = q_i . k_e / sqrt(D), O_i = sum_e softmax(z)_e v_e,
     LSE_i = max z + ln sum_e exp(z_e - max z).
+    ``blocks`` (ascending level-1 block indices) restricts the work to those query
+    blocks of every (b, h); the other rows of O and LSE are left as NaN.
     """
     q = np.asarray(q, dtype=np.float64)
     B, H, N, D = q.shape
     ksrc, offsets = kv_sources(k, k_pyr)
     vsrc, _ = kv_sources(v, v_pyr)
     n1 = N // BLOCK
-    o = np.empty((B, H, N, D))
-    lse = np.empty((B, H, N))
+    o = np.full((B, H, N, D), np.nan)
+    lse = np.full((B, H, N), np.nan)
     scale = 1.0 / math.sqrt(D)
+    sel_blocks = np.arange(n1) if blocks is None else np.asarray(blocks, dtype=np.int64)
     for b in range(B):
         for h in range(H):
             table = kv_index_table(b, h, idx, offsets)
             qb = q[b, h].reshape(n1, BLOCK, D)
-            for s0 in range(0, n1, chunk):
-                sl = slice(s0, min(n1, s0 + chunk))
+            for s0 in range(0, len(sel_blocks), chunk):
+                sl = sel_blocks[s0:s0 + chunk]
                 ke = ksrc[b, h][table[sl]]                   # [nb, T, D]
                 ve = vsrc[b, h][table[sl]]
                 z = np.einsum("nqd,ntd->nqt", qb[sl], ke) * scale
@@ -217,7 +220,7 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256):
     return o, lse
 
 
-def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256):
+def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None):
     """Exact gradient of the attention above with the selection held fixed.
 
     With P = softmax(z) on each query's list, Delta_i = sum_d dO_id O_id and
@@ -225,6 +228,7 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256):
     dK_e += dS_ie q_i / sqrt(D), dV_e += P_ie dO_i.  Gradients that land on coarse
     level-l tokens are then spread over their 16^l input tokens with weight 1/16^l
     (the adjoint of the mean pool).  Returns (dQ, dK, dV) [B, H, N, D] in fp64.
+    ``blocks`` restricts the sum to those query blocks (dQ rows of the others are NaN).
     """
     q = np.asarray(q, dtype=np.float64)
     do = np.asarray(do, dtype=np.float64)
@@ -236,9 +240,10 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256):
     vsrc, _ = kv_sources(v, v_pyr)
     n1 = N // BLOCK
     scale = 1.0 / math.sqrt(D)
-    dq = np.empty((B, H, N, D))
+    dq = np.full((B, H, N, D), np.nan)
     dk = np.empty((B, H, N, D))
     dv = np.empty((B, H, N, D))
+    sel_blocks = np.arange(n1) if blocks is None else np.asarray(blocks, dtype=np.int64)
     for b in range(B):
         for h in range(H):
             table = kv_index_table(b, h, idx, offsets)
@@ -248,8 +253,8 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256):
             lseb = lse[b, h].reshape(n1, BLOCK)
             dksrc = np.zeros_like(ksrc[b, h])
             dvsrc = np.zeros_like(vsrc[b, h])
-            for s0 in range(0, n1, chunk):
-                sl = slice(s0, min(n1, s0 + chunk))
+            for s0 in range(0, len(sel_blocks), chunk):
+                sl = sel_blocks[s0:s0 + chunk]
                 rows = table[sl]
                 ke = ksrc[b, h][rows]
                 ve = vsrc[b, h][rows]

@@ -1,0 +1,95 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every symbol the header
+declares, and its host-side checks and size queries behave as documented.  No call here
+reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from log_linear_hierarchical_b200 import _lib
+from log_linear_hierarchical_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "llsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(llsa_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from log_linear_hierarchical_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert "llsa_forward" in names and "llsa_backward" in names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(_lib.SIGNATURES), "binding and header declare different functions"
+
+
+def shape(**kw):
+    base = dict(B=1, H=6, N=65536, D=64, topk=8, levels=3, dtype=0)
+    base.update(kw)
+    return api.make_shape(base["B"], base["H"], base["N"], base["D"], base["topk"], base["levels"],
+                          base["dtype"], block=base.get("block", 16))
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({}, 0),
+    (dict(levels=1, N=1024, topk=8, dtype=1, H=2), 0),
+    (dict(N=3000), 1),                 # not a power of two
+    (dict(topk=6), 1),                 # not a power of two
+    (dict(topk=32), 1),                # topk > n_L = 16
+    (dict(N=2048), 1),                 # N < 16^L
+    (dict(B=0), 1),
+    (dict(dtype=7), 1),
+    (dict(D=128), 2),                  # legal, not built
+    (dict(block=32), 2),
+    (dict(levels=5, N=1 << 20, topk=1), 2),
+    (dict(N=1 << 21), 2),
+    (dict(levels=3, N=262144, topk=16), 0),
+    (dict(levels=3, N=1 << 20, topk=32), 2),   # (L-1) K = 64 coarse entries: above the 32 built
+])
+def test_validation(lib, kw, status):
+    assert api.llsa_validate_shape(shape(**kw)) == status
+
+
+def test_sizes_match_layout(lib):
+    s = shape()
+    n = [4096, 256, 16]
+    assert api.llsa_pyramid_elems(s) == 6 * 64 * sum(n)
+    assert api.llsa_index_elems(s) == 6 * 8 * sum(n)
+    assert api.llsa_row_ptr_elems(s) == 6 * sum(x + 1 for x in n)
+    assert api.llsa_transpose_workspace_bytes(s) >= 4 * 6 * 8 * sum(n)
+    # delta + partials + coarse grads
+    assert api.llsa_backward_workspace_bytes(s) >= 4 * (6 * 65536 + 2 * 6 * 256 * 16 * 64 + 2 * 6 * (256 + 16) * 64)
+    bad = shape(N=3000)
+    assert api.llsa_pyramid_elems(bad) == 0 and api.llsa_backward_workspace_bytes(bad) == 0
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(lib):
+    s = shape()
+    null = None
+    assert lib.llsa_build_pyramid(ctypes.byref(s), null, null, null, null, null, null, null) == 1
+    assert lib.llsa_select(ctypes.byref(s), 16, 32, 49, null) == 1    # idx misaligned
+    assert lib.llsa_forward(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 17, 16, null) == 1   # o misaligned
+    ws = api.llsa_transpose_workspace_bytes(s)
+    assert lib.llsa_index_transpose(ctypes.byref(s), 16, 16, 16, 16, ws - 1, null) == 3  # workspace too small
+    assert lib.llsa_status_string(3).decode() == "workspace too small"
+
+
+def test_status_error_message(lib):
+    err = api.LLSAError("llsa_select", 2)
+    assert "LLSA_ERR_UNSUPPORTED" in str(err)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(_lib.LLSAExtensionMissing):
+        _lib.load(str(tmp_path / "nope.so"))

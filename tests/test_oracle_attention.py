@@ -175,3 +175,20 @@ def test_list_order_does_not_matter(seed):
     rev = [idx[0][..., ::-1].copy(), idx[1]]
     o2, l2 = forward(q, k, v, kp, vp, rev)
     assert np.abs(o1 - o2).max() < 1e-13 and np.abs(l1 - l2).max() < 1e-13
+
+
+def test_block_subset_matches_full_run():
+    rng = np.random.default_rng(8)
+    B, H, N, D = 1, 2, 4096, 8
+    q, k, v, do = (rand(rng, B, H, N, D) for _ in range(4))
+    qp, kp, vp = (build_pyramid(x, 2) for x in (q, k, v))
+    idx = select(qp, kp, 4)
+    o, lse = forward(q, k, v, kp, vp, idx)
+    blocks = np.array([0, 17, 18, 255])
+    o2, l2 = forward(q, k, v, kp, vp, idx, blocks=blocks)
+    rows = (16 * blocks[:, None] + np.arange(16)).ravel()
+    assert np.abs(o2[:, :, rows] - o[:, :, rows]).max() < 1e-13
+    assert np.isnan(o2[:, :, 16]).all()
+    dq, dk, dv = backward(q, k, v, o, lse, do, kp, vp, idx)
+    dq2, dk2, dv2 = backward(q, k, v, o, lse, do, kp, vp, idx, blocks=np.arange(N // 16))
+    assert np.abs(dq2 - dq).max() < 1e-13 and np.abs(dk2 - dk).max() < 1e-13 and np.abs(dv2 - dv).max() < 1e-13
