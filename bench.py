@@ -464,6 +464,27 @@ def run_reference(args):
     print(json.dumps(result), flush=True)
 
 
+def run_profile(args):
+    """Only the timed step, for profilers: W warm-up steps then K steps, one line of output."""
+    import torch
+
+    from log_linear_hierarchical_b200 import api
+    from synthetic import CONFIGS, make_config_inputs
+
+    cfg = CONFIGS[args.config]
+    dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    dev = {k: v.cuda() for k, v in make_config_inputs(cfg, with_do=True).items()}
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype)
+    buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
+    for _ in range(args.warmup + args.steps):
+        api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+    torch.cuda.synchronize()
+    status = api.llsa_device_status()
+    print(json.dumps({"profile_run": cfg.name, "steps": args.steps, "warmup": args.warmup, "status": status}))
+    if status != 0:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,10 +493,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=4, help="workload number (4 = the headline N=65536 step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    ap.add_argument("--profile", action="store_true", help="run only the steps (for ncu), print no metric")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -29,7 +29,6 @@ struct AttnParams {
   Geometry g;
   float scale_log2;   // log2(e) / sqrt(D)
   float scale;        // 1 / sqrt(D)
-  int warp_bytes;     // shared memory per warp
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -73,11 +72,12 @@ __device__ __forceinline__ void mma_a_b(float (&acc)[8][4], uint32_t a0, uint32_
 
 // Stage (L-1)K coarse rows of a pyramid (fp32) as bf16 16-row swizzled tiles; padding rows
 // (index >= C) are zero.  Row c is level 2 + c / K, slot c % K of the ancestor's list.
+// Threads `tid` = 0..nthreads-1 share the work (a warp or a whole CTA).
 __device__ __forceinline__ void stage_coarse_rows(const Geometry& g, const float* __restrict__ pyr,
-                                                  const int* __restrict__ idx, int bh, int p, uint32_t dst) {
-  const int lane = lane_id();
+                                                  const int* __restrict__ idx, int bh, int p, uint32_t dst, int tid,
+                                                  int nthreads) {
   const int K = g.K;
-  for (int t = lane; t < g.coarse_pad * 8; t += 32) {
+  for (int t = tid; t < g.coarse_pad * 8; t += nthreads) {
     const int row = t >> 3;
     const int ch = t & 7;
     uint4 packed = make_uint4(0u, 0u, 0u, 0u);
@@ -132,8 +132,9 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[8][4], float 
   __syncwarp();
 }
 
-// One 16-token chunk of the online softmax.  `valid` < 16 masks the padding of the last
-// coarse tile.
+// One 16-token chunk of the online softmax.  With MASK, columns >= `valid` (the padding of
+// the last coarse tile) are excluded.
+template <bool MASK>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t ktile, uint32_t vtile, int valid,
                                           float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[8][4]) {
   const int lane = lane_id();
@@ -144,7 +145,7 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int col = n * 8 + 2 * (lane & 3) + (e & 1);
-      s[n][e] = (col < valid) ? s[n][e] * scale_log2 : -INFINITY;
+      s[n][e] = (!MASK || col < valid) ? s[n][e] * scale_log2 : -INFINITY;
     }
   float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
   float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
@@ -179,36 +180,34 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
           pack_bf16(p[1][2], p[1][3]), vtile);
 }
 
-// Shared-memory map of one forward warp (byte offsets from its 1024-aligned base).
-struct FwdWarpMap {
-  uint32_t q, ring, ck, cv;
-  int* idx;
-  uint32_t bar_q, bar_kv;  // bar_q[2] then bar_kv[STAGES], 8 bytes each
+// Shared memory of the attention kernels: a CTA region (the group's coarse K and V tiles),
+// then per warp a block of 1024-aligned tiles, then per warp a small tail (indices,
+// mbarriers).  Offsets are in bytes from the 1024-aligned base.
+struct CtaSmem {
+  int coarse_bytes;  // 2 * coarse_pad * 128
+  int warp_tiles;    // bytes of tiles per warp (multiple of 1024)
+  int warp_tail;     // bytes of tail per warp (multiple of 16)
+  int nwarps;
+  __host__ __device__ int total() const { return 1024 + coarse_bytes + nwarps * (warp_tiles + warp_tail); }
+  __device__ uint8_t* tiles(uint8_t* base, int w) const { return base + coarse_bytes + w * warp_tiles; }
+  __device__ uint8_t* tail(uint8_t* base, int w) const {
+    return base + coarse_bytes + nwarps * warp_tiles + w * warp_tail;
+  }
 };
 
 template <int STAGES>
-__device__ __forceinline__ FwdWarpMap fwd_warp_map(uint8_t* base, const Geometry& g) {
-  FwdWarpMap m;
-  const uint32_t b = smem_u32(base);
-  m.q = b;
-  m.ring = b + 2 * kTileBytes;
-  m.ck = m.ring + STAGES * 2 * kTileBytes;
-  m.cv = m.ck + g.coarse_pad * 128;
-  uint8_t* after = base + 2 * kTileBytes + STAGES * 2 * kTileBytes + 2 * g.coarse_pad * 128;
-  m.idx = reinterpret_cast<int*>(after);
-  uint8_t* bars = after + ((kUnitBlocks * g.K * 4 + 15) & ~15);
-  m.bar_q = smem_u32(bars);
-  m.bar_kv = m.bar_q + 16;
-  return m;
+__host__ __device__ inline CtaSmem fwd_smem(const Geometry& g, int nwarps) {
+  CtaSmem c;
+  c.coarse_bytes = 2 * g.coarse_pad * 128;
+  c.warp_tiles = 2 * kTileBytes + STAGES * 2 * kTileBytes;
+  c.warp_tail = ((kUnitBlocks * g.K * 4 + 15) & ~15) + ((8 * (2 + STAGES) + 15) & ~15);
+  c.nwarps = nwarps;
+  return c;
 }
 
-template <int STAGES>
-inline int fwd_warp_bytes(const Geometry& g) {
-  int bytes = 2 * kTileBytes + STAGES * 2 * kTileBytes + 2 * g.coarse_pad * 128 + ((kUnitBlocks * g.K * 4 + 15) & ~15) +
-              8 * (2 + STAGES);
-  return (bytes + 1023) & ~1023;
-}
-
+// One CTA = 4 warps = 16 consecutive query blocks (one level-2 group when L >= 2, so the
+// coarse KV entries are staged once per CTA).  Each warp owns 4 blocks and streams their
+// fine KV tiles through its own ring of STAGES mbarrier-tracked TMA stages.
 template <int STAGES>
 __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                             const __grid_constant__ CUtensorMap tm_k,
@@ -225,15 +224,31 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   const int n1 = g.n[1];
   const int K = g.K;
   const int total_blocks = g.BH * n1;
-  const int first = (blockIdx.x * nwarps + warp) * kUnitBlocks;
-  if (first >= total_blocks) return;  // warp-uniform; this kernel has no CTA-wide barrier
+  const CtaSmem cs = fwd_smem<STAGES>(g, nwarps);
+  uint8_t* base = align1024(fwd_smem_raw);
+  const uint32_t ck = smem_u32(base);
+  const uint32_t cv = ck + g.coarse_pad * 128;
+  const int cta_first = blockIdx.x * nwarps * kUnitBlocks;
+  if (g.L >= 2) {  // the CTA's 16 blocks share one ancestor per level (n_1 % 16 == 0 here)
+    const int bh0 = cta_first / n1;
+    const int p0 = cta_first - bh0 * n1;
+    stage_coarse_rows(g, k_pyr, idx, bh0, p0, ck, threadIdx.x, blockDim.x);
+    stage_coarse_rows(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
+    __syncthreads();
+  }
+  const int first = cta_first + warp * kUnitBlocks;
+  if (first >= total_blocks) return;  // warp-uniform; no CTA-wide barrier after this point
   const int nblk = min(kUnitBlocks, total_blocks - first);
-  const FwdWarpMap sm = fwd_warp_map<STAGES>(align1024(fwd_smem_raw) + warp * P.warp_bytes, g);
+  const uint32_t sq = smem_u32(cs.tiles(base, warp));
+  const uint32_t ring = sq + 2 * kTileBytes;
+  int* sidx = reinterpret_cast<int*>(cs.tail(base, warp));
+  const uint32_t bar_q = smem_u32(sidx) + ((kUnitBlocks * K * 4 + 15) & ~15);
+  const uint32_t bar_kv = bar_q + 16;
 
   for (int i = lane; i < nblk * K; i += 32)
-    sm.idx[i] = checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1);
+    sidx[i] = checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1);
   if (lane == 0) {
-    for (int b = 0; b < 2 + STAGES; ++b) mbar_init(sm.bar_q + 8 * b, 1);
+    for (int b = 0; b < 2 + STAGES; ++b) mbar_init(bar_q + 8 * b, 1);
     mbar_fence_init();
   }
   __syncwarp();
@@ -242,29 +257,22 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   auto issue_kv = [&](int seq) {
     const int gb = first + seq / K;
     const int bh = gb / n1;
-    const int row = bh * g.N + sm.idx[seq] * kBlock;
+    const int row = bh * g.N + sidx[seq] * kBlock;
     const int stage = seq % STAGES;
-    const uint32_t bar = sm.bar_kv + 8 * stage;
-    const uint32_t dst = sm.ring + stage * 2 * kTileBytes;
+    const uint32_t bar = bar_kv + 8 * stage;
+    const uint32_t dst = ring + stage * 2 * kTileBytes;
     mbar_expect_tx(bar, 2 * kTileBytes);
     tma_load_2d(dst, &tm_k, 0, row, bar);
     tma_load_2d(dst + kTileBytes, &tm_v, 0, row, bar);
   };
   auto issue_q = [&](int i) {
-    const uint32_t bar = sm.bar_q + 8 * (i & 1);
+    const uint32_t bar = bar_q + 8 * (i & 1);
     mbar_expect_tx(bar, kTileBytes);
-    tma_load_2d(sm.q + (i & 1) * kTileBytes, &tm_q, 0, (first + i) * kBlock, bar);
+    tma_load_2d(sq + (i & 1) * kTileBytes, &tm_q, 0, (first + i) * kBlock, bar);
   };
   if (lane == 0) {
     issue_q(0);
     for (int s = 0; s < min(STAGES, total_loads); ++s) issue_kv(s);
-  }
-  if (g.L >= 2) {
-    const int bh0 = first / n1;
-    const int p0 = first - bh0 * n1;
-    stage_coarse_rows(g, k_pyr, idx, bh0, p0, sm.ck);
-    stage_coarse_rows(g, v_pyr, idx, bh0, p0, sm.cv);
-    __syncwarp();
   }
 
   bool ok = true;
@@ -272,11 +280,11 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   int next_q = 0;    // first Q load not yet consumed
   for (int i = 0; i < nblk && ok; ++i) {
     const int gb = first + i;
-    ok = __all_sync(0xffffffffu, mbar_wait(sm.bar_q + 8 * (i & 1), (i >> 1) & 1));
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_q + 8 * (i & 1), (i >> 1) & 1));
     if (!ok) break;
     next_q = i + 1;
     uint32_t qf[4][4];
-    load_a_frags(sm.q + (i & 1) * kTileBytes, qf);
+    load_a_frags(sq + (i & 1) * kTileBytes, qf);
     __syncwarp();
     if (lane == 0 && i + 1 < nblk) issue_q(i + 1);
 
@@ -289,24 +297,24 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     for (int s = 0; s < K; ++s) {
       const int seq = i * K + s;
       const int stage = seq % STAGES;
-      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar_kv + 8 * stage, (seq / STAGES) & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_kv + 8 * stage, (seq / STAGES) & 1));
       if (!ok) break;
       next_seq = seq + 1;
-      const uint32_t kt = sm.ring + stage * 2 * kTileBytes;
-      fwd_chunk(qf, kt, kt + kTileBytes, kBlock, P.scale_log2, m, l, acc);
+      const uint32_t kt = ring + stage * 2 * kTileBytes;
+      fwd_chunk<false>(qf, kt, kt + kTileBytes, kBlock, P.scale_log2, m, l, acc);
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
-      fwd_chunk(qf, sm.ck + cc * kTileBytes, sm.cv + cc * kTileBytes, min(kBlock, g.coarse - cc * kBlock),
-                P.scale_log2, m, l, acc);
+      fwd_chunk<true>(qf, ck + cc * kTileBytes, cv + cc * kTileBytes, min(kBlock, g.coarse - cc * kBlock),
+                      P.scale_log2, m, l, acc);
 
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 1);
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 2);
     l[1] += __shfl_xor_sync(0xffffffffu, l[1], 1);
     l[1] += __shfl_xor_sync(0xffffffffu, l[1], 2);
-    store_tile_bf16(acc, 1.0f / l[0], 1.0f / l[1], sm.q + (i & 1) * kTileBytes, o + (long long)gb * kBlock * kD);
+    store_tile_bf16(acc, 1.0f / l[0], 1.0f / l[1], sq + (i & 1) * kTileBytes, o + (long long)gb * kBlock * kD);
     if ((lane & 3) == 0) {
       const int r0 = lane >> 2;
       lse[(long long)gb * kBlock + r0] = (m[0] + log2f(l[0])) * kLn2;
@@ -317,8 +325,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     // A copy did not land in time (recorded as LLSA_ERR_TIMEOUT).  Give each copy still in
     // flight one more bounded wait so none lands after this warp has gone.
     for (int seq = next_seq; seq < min(total_loads, next_seq + STAGES); ++seq)
-      mbar_wait(sm.bar_kv + 8 * (seq % STAGES), (seq / STAGES) & 1);
-    for (int i = next_q; i < min(nblk, next_q + 2); ++i) mbar_wait(sm.bar_q + 8 * (i & 1), (i >> 1) & 1);
+      mbar_wait(bar_kv + 8 * (seq % STAGES), (seq / STAGES) & 1);
+    for (int i = next_q; i < min(nblk, next_q + 2); ++i) mbar_wait(bar_q + 8 * (i & 1), (i >> 1) & 1);
   }
 }
 

@@ -156,13 +156,14 @@ enum KernelId {
   kKFwdF32,
   kKBwdDqF32,
   kKBwdDkdvF32,
+  kKBwdCoarseBf16,
   kKNumKernels
 };
 
 const char* const kKernelNames[kKNumKernels] = {
     "unknown",          "pyramid_l12",          "pyramid_up",   "select",           "transpose_hist",
     "transpose_scatter", "transpose_bucket",    "attn_fwd_bf16", "attn_bwd_dq_bf16", "coarse_grad_reduce",
-    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32"};
+    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32", "attn_bwd_coarse_bf16"};
 
 struct TraceState {
   cudaEvent_t* ev = nullptr;
@@ -187,18 +188,27 @@ llsa_status launch(int id, cudaStream_t cs, F&& f) {
   return st;
 }
 
-constexpr int kFwdStages = 4;
-constexpr int kDqStages = 2;
-constexpr int kDkvStages = 3;
+#ifndef LLSA_FWD_STAGES
+#define LLSA_FWD_STAGES 2
+#endif
+#ifndef LLSA_DQ_STAGES
+#define LLSA_DQ_STAGES 2
+#endif
+#ifndef LLSA_KV_STAGES
+#define LLSA_KV_STAGES 2
+#endif
+constexpr int kFwdStages = LLSA_FWD_STAGES;
+constexpr int kDqStages = LLSA_DQ_STAGES;
+constexpr int kDkvStages = LLSA_KV_STAGES;
 constexpr int kAttnWarps = 4;
 
 llsa_status launch_coarse_reduce(const Geometry& g, float scale, const int32_t* idx, const int32_t* row_ptr,
                                  const int32_t* col, float* ws, cudaStream_t cs) {
   if (g.L < 2) return LLSA_OK;
-  long long warps = 0;
-  for (int l = 2; l <= g.L; ++l) warps += (long long)g.BH * g.n[l];
+  long long tokens = 0;
+  for (int l = 2; l <= g.L; ++l) tokens += (long long)g.BH * g.n[l];
   return launch(kKBwdCoarseReduce, cs, [&] {
-    coarse_grad_reduce_kernel<<<(unsigned)((warps * 32 + 127) / 128), 128, 0, cs>>>(g, scale, idx, row_ptr, col, ws);
+    coarse_grad_reduce_kernel<<<(unsigned)tokens, kReduceWarps * 32, 0, cs>>>(g, scale, idx, row_ptr, col, ws);
   });
 }
 
@@ -362,8 +372,8 @@ llsa_status llsa_forward(const llsa_shape* s, const void* q, const void* k, cons
     const long long rows = (long long)g.BH * g.N;
     if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
       return LLSA_ERR_CUDA;
-    AttnParams P{g, scale * kLog2e, scale, fwd_warp_bytes<kFwdStages>(g)};
-    const size_t smem = (size_t)kAttnWarps * P.warp_bytes + 1024;
+    AttnParams P{g, scale * kLog2e, scale};
+    const size_t smem = (size_t)fwd_smem<kFwdStages>(g, kAttnWarps).total();
     auto kern = attn_fwd_bf16_kernel<kFwdStages>;
     if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
     const int per_cta = kAttnWarps * kUnitBlocks;
@@ -404,8 +414,8 @@ llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, con
         !make_tile_map(&tdo, dO, rows))
       return LLSA_ERR_CUDA;
     {
-      AttnParams P{g, scale * kLog2e, scale, dq_warp_bytes<kDqStages>(g)};
-      const size_t smem = (size_t)kAttnWarps * P.warp_bytes + 1024;
+      AttnParams P{g, scale * kLog2e, scale};
+      const size_t smem = (size_t)dq_smem<kDqStages>(g, kAttnWarps).total();
       auto kern = attn_bwd_dq_bf16_kernel<kDqStages>;
       if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
       const int per_cta = kAttnWarps * kUnitBlocks;
@@ -416,14 +426,23 @@ llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, con
       });
       if (st != LLSA_OK) return st;
     }
+    AttnParams P{g, scale * kLog2e, scale};
+    const size_t kv_bytes = (size_t)kv_smem<kDkvStages>(1).total();
+    if (g.L >= 2) {
+      auto kern = attn_bwd_coarse_bf16_kernel<kDkvStages>;
+      if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
+      const int ctas = g.BH * g.n[2] * (g.coarse_pad / kBlock);
+      st = launch(kKBwdCoarseBf16, cs, [&] {
+        kern<<<ctas, 32, kv_bytes, cs>>>(tq, tdo, P, k_pyr, v_pyr, idx, lse, ws);
+      });
+      if (st != LLSA_OK) return st;
+    }
     if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
-    AttnParams P{g, scale * kLog2e, scale, dkv_warp_bytes<kDkvStages>()};
-    const size_t smem = (size_t)kAttnWarps * P.warp_bytes + 1024;
     auto kern = attn_bwd_dkdv_bf16_kernel<kDkvStages>;
-    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+    if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
     return launch(kKBwdDkdvBf16, cs, [&] {
-      kern<<<(total_blocks + kAttnWarps - 1) / kAttnWarps, 32 * kAttnWarps, smem, cs>>>(
-          tq, tk, tv, tdo, P, lse, row_ptr, col, ws, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+      kern<<<total_blocks, 32, kv_bytes, cs>>>(tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
+                                                static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
     });
   }
   const size_t smem = simt_dq_smem(g);

@@ -7,9 +7,9 @@
 //   * finer levels:   the 16 sibling queries of one parent, candidates = the 16K children
 //                     16c + r of the parent's K selected keys c (ascending).
 // Scores are fp32 dot products of the fp32 pyramid rows (the 1/sqrt(D) scale does not
-// change the order and is not applied).  The K winners come from K warp-wide argmax
-// rounds over the scores held in shared memory; the order is (score desc, key asc), so
-// the lower key index wins equal scores.  Output rows are written in ascending key order.
+// change the order and is not applied).  The K winners come from K warp-wide rounds of
+// redux.sync max (score) then min (candidate position); the order is (score desc, key asc),
+// so the lower key index wins equal scores.  Output rows are written in ascending key order.
 //
 // Bound: L2 reads of the candidate key rows (each group's 16K rows are read once and
 // reused by its 16 queries); the arithmetic is 16 * 16K * 64 FMA per group.
@@ -21,12 +21,15 @@ namespace llsa {
 
 constexpr int kSelThreads = 256;
 
-// True if (s1, c1) ranks before (s2, c2): higher score first, then lower candidate position.
-__device__ __forceinline__ bool sel_better(float s1, int c1, float s2, int c2) {
-  return s1 > s2 || (s1 == s2 && c1 < c2);
+// Order-preserving map of an fp32 score to an unsigned key: a larger score gives a larger
+// key; -0 and +0 both map to the key of +0 (they compare equal as floats).  Every real
+// score maps above 0, so 0 marks a removed candidate.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  const uint32_t u = __float_as_uint(s + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// grid.x = B*H * groups; dynamic smem = gq*64 + nc + gq*nc + gq*K ints/floats.
+// grid.x = B*H * groups; dynamic smem = gq*64 + nc + gq*nc + gq*K words.
 // parent_idx == nullptr selects the coarsest-level mode.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int level, int gq,
                                                              const float* __restrict__ qp,
@@ -44,10 +47,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
   const int a0 = grp * gq;
   const int rows = min(gq, n - a0);
 
-  float* qs = sel_smem;                          // [gq][64]
-  int* cand = reinterpret_cast<int*>(qs + gq * kD);  // [nc] (sparse only)
-  float* sc = reinterpret_cast<float*>(cand + (sparse ? nc : 0));  // [gq][nc]
-  int* win = reinterpret_cast<int*>(sc + gq * nc);                 // [gq][K]
+  float* qs = sel_smem;                                           // [gq][64]
+  int* cand = reinterpret_cast<int*>(qs + gq * kD);                // [nc] (sparse only)
+  uint32_t* sk = reinterpret_cast<uint32_t*>(cand + (sparse ? nc : 0));  // [gq][nc] score keys
+  int* win = reinterpret_cast<int*>(sk + gq * nc);                 // [gq][K]
 
   const int tid = threadIdx.x;
   const float* qbase = qp + ((long long)bh * n + a0) * kD;
@@ -62,7 +65,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
   }
   __syncthreads();
 
-  // ---- scores: thread owns one candidate row (in registers) and a subset of the queries
+  // ---- scores: a thread owns one candidate row (in registers) and every nsplit-th query;
+  // four queries at a time keep four independent FMA chains in flight.
   const int nsplit = nc >= kSelThreads ? 1 : kSelThreads / nc;
   const int cstep = nc >= kSelThreads ? kSelThreads : nc;
   const int qsub = tid / cstep;
@@ -72,61 +76,71 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
     float4 kr[kD / 4];
 #pragma unroll
     for (int i = 0; i < kD / 4; ++i) kr[i] = __ldg(krow + i);
-    for (int qi = qsub; qi < gq; qi += nsplit) {
-      const float4* qrow = reinterpret_cast<const float4*>(qs + qi * kD);
-      float s = 0.0f;
+    for (int q0 = qsub; q0 < gq; q0 += 4 * nsplit) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float4* qr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) qr[u] = reinterpret_cast<const float4*>(qs + min(q0 + u * nsplit, gq - 1) * kD);
 #pragma unroll
       for (int i = 0; i < kD / 4; ++i) {
-        const float4 qv = qrow[i];
-        s = fmaf(qv.x, kr[i].x, s);
-        s = fmaf(qv.y, kr[i].y, s);
-        s = fmaf(qv.z, kr[i].z, s);
-        s = fmaf(qv.w, kr[i].w, s);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 qv = qr[u][i];
+          acc[u] = fmaf(qv.x, kr[i].x, acc[u]);
+          acc[u] = fmaf(qv.y, kr[i].y, acc[u]);
+          acc[u] = fmaf(qv.z, kr[i].z, acc[u]);
+          acc[u] = fmaf(qv.w, kr[i].w, acc[u]);
+        }
       }
-      sc[qi * nc + c] = s;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int qi = q0 + u * nsplit;
+        if (qi < gq) sk[qi * nc + c] = score_key(acc[u]);
+      }
     }
   }
   __syncthreads();
 
-  // ---- K argmax rounds per query, one warp per query
+  // ---- K rounds per query, one warp per query: each lane keeps the best of its candidates
+  // c = lane + 32 i; redux.sync finds the largest key, then the lowest candidate holding it.
   const int warp = tid >> 5;
   const int lane = tid & 31;
   for (int qi = warp; qi < rows; qi += kSelThreads / 32) {
-    float* srow = sc + qi * nc;
+    uint32_t* krow = sk + qi * nc;
     int* wrow = win + qi * K;
-    for (int r = 0; r < K; ++r) {
-      float bs = -INFINITY;
-      int bc = 0x7fffffff;
-      for (int c = lane; c < nc; c += 32) {
-        const float s = srow[c];
-        if (sel_better(s, c, bs, bc)) {
-          bs = s;
-          bc = c;
-        }
+    uint32_t bk = 0u;
+    int bc = 0x7fffffff;
+    for (int c = lane; c < nc; c += 32) {
+      const uint32_t k = krow[c];
+      if (k > bk) {
+        bk = k;
+        bc = c;
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-        const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
-        if (sel_better(os, oc, bs, bc)) {
-          bs = os;
-          bc = oc;
-        }
-      }
-      if (bc < 0 || bc >= nc) {  // only reachable with NaN scores
-        record_error(LLSA_ERR_INTERNAL);
-        bc = 0;
-      }
-      if (lane == (bc & 31)) srow[bc] = -INFINITY;
-      if (lane == 0) wrow[r] = bc;
-      __syncwarp();
     }
+    for (int r = 0; r < K; ++r) {
+      const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t w = __reduce_min_sync(0xffffffffu, bk == m ? (uint32_t)bc : 0x7fffffffu);
+      if (lane == 0) wrow[r] = (int)w;
+      if (bc == (int)w && bk == m) {  // the owner drops its winner and finds its next best
+        krow[w] = 0u;
+        bk = 0u;
+        bc = 0x7fffffff;
+        for (int c = lane; c < nc; c += 32) {
+          const uint32_t k = krow[c];
+          if (k > bk) {
+            bk = k;
+            bc = c;
+          }
+        }
+      }
+    }
+    __syncwarp();
     // ascending order: each winner's rank is the number of smaller winners
     int* orow = out_idx + ((long long)bh * n + a0 + qi) * K;
     for (int r = lane; r < K; r += 32) {
-      const int mine = wrow[r];
+      const int mine = min(max(wrow[r], 0), nc - 1);
       int rank = 0;
-      for (int r2 = 0; r2 < K; ++r2) rank += wrow[r2] < mine;
+      for (int r2 = 0; r2 < K; ++r2) rank += wrow[r2] < wrow[r];
       orow[rank] = sparse ? cand[mine] : mine;
     }
     __syncwarp();
