@@ -88,7 +88,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[4][4], const uint3
     for (int e = 0; e < 4; ++e) {
       const int col = n * 8 + 2 * (lane & 3) + (e & 1);
       const int r = e >> 1;
-      const float p = (!MASK || col < valid) ? exp2f(s[n][e] * scale_log2 - lse2[r]) : 0.0f;
+      const float p = (!MASK || col < valid) ? ex2(fmaf(s[n][e], scale_log2, -lse2[r])) : 0.0f;
       ds[n][e] = p * (dp[n][e] - delta[r]);
     }
   mma_a_b(dq, pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]), pack_bf16(ds[1][0], ds[1][1]),
@@ -144,9 +144,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int gb = first + seq / K;
-    const int bh = gb / n1;
-    const int row = bh * g.N + sidx[seq] * kBlock;
+    const int gb = first + (seq >> g.log_k);
+    const int row = ((gb >> g.log_n1) << (g.log_n1 + 4)) + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * kTileBytes;
@@ -253,14 +252,20 @@ __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32
   float dpt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt(st, kf, qt);   // S^T: rows = keys, cols = queries
   mma_a_bt(dpt, vf, dt);  // dP^T
+  // this lane's four query columns: c2, c2 + 1 (n = 0) and c2 + 8, c2 + 9 (n = 1)
+  const float2 l0 = *reinterpret_cast<const float2*>(ls + c2);
+  const float2 l1 = *reinterpret_cast<const float2*>(ls + 8 + c2);
+  const float2 d0 = *reinterpret_cast<const float2*>(dl + c2);
+  const float2 d1 = *reinterpret_cast<const float2*>(dl + 8 + c2);
+  const float lq[2][2] = {{l0.x * kLog2e, l0.y * kLog2e}, {l1.x * kLog2e, l1.y * kLog2e}};
+  const float dq[2][2] = {{d0.x, d0.y}, {d1.x, d1.y}};
   float pt[2][4], dst[2][4];
 #pragma unroll
   for (int n = 0; n < 2; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int qcol = n * 8 + c2 + (e & 1);
-      pt[n][e] = exp2f(st[n][e] * scale_log2 - ls[qcol] * kLog2e);
-      dst[n][e] = pt[n][e] * (dpt[n][e] - dl[qcol]);
+      pt[n][e] = ex2(fmaf(st[n][e], scale_log2, -lq[n][e & 1]));
+      dst[n][e] = pt[n][e] * (dpt[n][e] - dq[n][e & 1]);
     }
   mma_a_b(dv, pack_bf16(pt[0][0], pt[0][1]), pack_bf16(pt[0][2], pt[0][3]), pack_bf16(pt[1][0], pt[1][1]),
           pack_bf16(pt[1][2], pt[1][3]), dt);
@@ -292,19 +297,21 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
                                           uint32_t bar_ring, int npairs, PairBlock pair_block, float scale_log2,
                                           float (&dk)[8][4], float (&dv)[8][4]) {
   const int lane = lane_id();
+  // called by the whole warp (pair_block may shuffle); lane 0 issues the copies
   auto issue_pair = [&](int i) {
     const int row = pair_block(i) * kBlock;
-    const int stage = i % STAGES;
-    const uint32_t bar = bar_ring + 8 * stage;
-    const uint32_t dst = ring + stage * 2 * kTileBytes;
-    mbar_expect_tx(bar, 2 * kTileBytes + 2 * kBlock * 4);
-    tma_load_2d(dst, tm_q, 0, row, bar);
-    tma_load_2d(dst + kTileBytes, tm_do, 0, row, bar);
-    bulk_load(smem_u32(sls + stage * kBlock), lse + row, kBlock * 4, bar);
-    bulk_load(smem_u32(sdl + stage * kBlock), delta + row, kBlock * 4, bar);
+    if (lane == 0) {
+      const int stage = i % STAGES;
+      const uint32_t bar = bar_ring + 8 * stage;
+      const uint32_t dst = ring + stage * 2 * kTileBytes;
+      mbar_expect_tx(bar, 2 * kTileBytes + 2 * kBlock * 4);
+      tma_load_2d(dst, tm_q, 0, row, bar);
+      tma_load_2d(dst + kTileBytes, tm_do, 0, row, bar);
+      bulk_load(smem_u32(sls + stage * kBlock), lse + row, kBlock * 4, bar);
+      bulk_load(smem_u32(sdl + stage * kBlock), delta + row, kBlock * 4, bar);
+    }
   };
-  if (lane == 0)
-    for (int i = 0; i < min(STAGES, npairs); ++i) issue_pair(i);
+  for (int i = 0; i < min(STAGES, npairs); ++i) issue_pair(i);
   if (bar_tile != 0u && !__all_sync(0xffffffffu, mbar_wait(bar_tile, 0))) {
     for (int j = 0; j < min(npairs, STAGES); ++j) mbar_wait(bar_ring + 8 * (j % STAGES), (j / STAGES) & 1);
     return false;
@@ -321,7 +328,7 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
     const uint32_t qt = ring + stage * 2 * kTileBytes;
     kv_pair(kf, vf, qt, qt + kTileBytes, sls + stage * kBlock, sdl + stage * kBlock, scale_log2, dk, dv);
     __syncwarp();
-    if (lane == 0 && i + STAGES < npairs) issue_pair(i + STAGES);
+    if (i + STAGES < npairs) issue_pair(i + STAGES);
   }
   return true;
 }
@@ -570,8 +577,19 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
   const int bh_block0 = bh * n1;
+  // the row's query blocks are read 32 at a time by the whole warp and handed to the
+  // issuing lane by shuffle, so no load sits on the TMA issue path
+  int cached_base = -64, cached = 0;
   const bool ok = kv_stream<STAGES>(&tm_q, &tm_do, lse, ws + W.delta, kvt, bar_kv, ring, sls, sdl, bar_ring, re - rs,
-                                    [&](int i) { return bh_block0 + checked_index(__ldg(cl + i), n1); },
+                                    [&](int i) {
+                                      const int base32 = i & ~31;
+                                      if (base32 != cached_base) {
+                                        cached_base = base32;
+                                        const int e = base32 + lane;
+                                        cached = e < re - rs ? checked_index(__ldg(cl + e), n1) : 0;
+                                      }
+                                      return bh_block0 + __shfl_sync(0xffffffffu, cached, i & 31);
+                                    },
                                     P.scale_log2, dk, dv);
   if (!ok) return;
   // epilogue: scale dK, add the mean-pool adjoint of the ancestors' coarse gradients

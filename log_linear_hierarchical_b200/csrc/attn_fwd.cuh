@@ -133,49 +133,56 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[8][4], float 
 }
 
 // One 16-token chunk of the online softmax.  With MASK, columns >= `valid` (the padding of
-// the last coarse tile) are excluded.
+// the last coarse tile) are excluded.  m holds the running row maxima of the scaled scores
+// (log2 domain), l the per-lane partial row sums.
 template <bool MASK>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t ktile, uint32_t vtile, int valid,
                                           float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[8][4]) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt(s, qf, ktile);
+  if (MASK) {
 #pragma unroll
-  for (int n = 0; n < 2; ++n)
+    for (int n = 0; n < 2; ++n)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int col = n * 8 + 2 * (lane & 3) + (e & 1);
-      s[n][e] = (!MASK || col < valid) ? s[n][e] * scale_log2 : -INFINITY;
-    }
+      for (int e = 0; e < 4; ++e)
+        if (n * 8 + 2 * (lane & 3) + (e & 1) >= valid) s[n][e] = -INFINITY;
+  }
   float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
   float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
   mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
   mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
   mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
   mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-  const float mn0 = fmaxf(m[0], mx0);
-  const float mn1 = fmaxf(m[1], mx1);
-  const float c0 = exp2f(m[0] - mn0);
-  const float c1 = exp2f(m[1] - mn1);
+  // the scale is positive, so the maximum of the scaled scores is the scaled maximum
+  const float mn0 = fmaxf(m[0], mx0 * scale_log2);
+  const float mn1 = fmaxf(m[1], mx1 * scale_log2);
   float p[2][4];
 #pragma unroll
   for (int n = 0; n < 2; ++n) {
-    p[n][0] = exp2f(s[n][0] - mn0);
-    p[n][1] = exp2f(s[n][1] - mn0);
-    p[n][2] = exp2f(s[n][2] - mn1);
-    p[n][3] = exp2f(s[n][3] - mn1);
+    p[n][0] = ex2(fmaf(s[n][0], scale_log2, -mn0));
+    p[n][1] = ex2(fmaf(s[n][1], scale_log2, -mn0));
+    p[n][2] = ex2(fmaf(s[n][2], scale_log2, -mn1));
+    p[n][3] = ex2(fmaf(s[n][3], scale_log2, -mn1));
   }
-  l[0] = l[0] * c0 + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-  l[1] = l[1] * c1 + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-  m[0] = mn0;
-  m[1] = mn1;
+  // rescale the running sums only when a row maximum moved (decided for the whole warp)
+  if (__any_sync(0xffffffffu, mn0 != m[0] || mn1 != m[1])) {
+    const float c0 = ex2(m[0] - mn0);
+    const float c1 = ex2(m[1] - mn1);
+    l[0] *= c0;
+    l[1] *= c1;
 #pragma unroll
-  for (int n = 0; n < 8; ++n) {
-    acc[n][0] *= c0;
-    acc[n][1] *= c0;
-    acc[n][2] *= c1;
-    acc[n][3] *= c1;
+    for (int n = 0; n < 8; ++n) {
+      acc[n][0] *= c0;
+      acc[n][1] *= c0;
+      acc[n][2] *= c1;
+      acc[n][3] *= c1;
+    }
+    m[0] = mn0;
+    m[1] = mn1;
   }
+  l[0] += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+  l[1] += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
   mma_a_b(acc, pack_bf16(p[0][0], p[0][1]), pack_bf16(p[0][2], p[0][3]), pack_bf16(p[1][0], p[1][1]),
           pack_bf16(p[1][2], p[1][3]), vtile);
 }
@@ -255,9 +262,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int gb = first + seq / K;
-    const int bh = gb / n1;
-    const int row = bh * g.N + sidx[seq] * kBlock;
+    const int gb = first + (seq >> g.log_k);
+    const int row = ((gb >> g.log_n1) << (g.log_n1 + 4)) + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * kTileBytes;

@@ -63,6 +63,8 @@ Geometry make_geometry(const llsa_shape* s) {
     io += (long long)g.BH * g.n[l] * g.K;
     ro += (long long)g.BH * (g.n[l] + 1);
   }
+  g.log_k = ilog2(g.K);
+  g.log_n1 = ilog2(g.n[1]);
   g.coarse = (g.L - 1) * g.K;
   g.coarse_pad = (g.coarse + kBlock - 1) / kBlock * kBlock;
   return g;

@@ -18,6 +18,7 @@ constexpr int kTileBytes = 2048;  // one 16-token x 64-channel bf16 tile
 // Per-call geometry: level sizes and the level-major offsets of every packed buffer.
 struct Geometry {
   int B, H, N, D, K, L, BH;
+  int log_k, log_n1;                     // log2 K and log2 n_1 (both powers of two)
   int n[kMaxLevels + 1];                 // n[l] = N / 16^l, l = 0..L
   long long pyr_off[kMaxLevels + 1];     // element offset of level l (1..L) in a pyramid
   long long idx_off[kMaxLevels + 1];     // element offset of level l in idx / col
@@ -82,6 +83,14 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// 2^x by the PTX ex2.approx.ftz.f32 instruction (relative error about 2^-22; subnormal
+// results flush to zero, which only affects probabilities below 2^-126).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
 

@@ -29,7 +29,48 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// grid.x = B*H * groups; dynamic smem = gq*64 + nc + gq*nc + gq*K words.
+// Candidate rows are staged in shared memory with a padded stride (68 floats: a quarter
+// warp's 16-byte reads of 8 consecutive rows hit 8 distinct bank groups).
+constexpr int kSelRowStride = kD + 4;
+// Candidates scored per pass; larger candidate sets (coarsest level with n_L > 256) are
+// scored in passes of this many rows.
+constexpr int kSelChunk = 256;
+
+// Top-K of one query's score keys krow[0..nc) by one warp: each lane keeps the best of its
+// candidates c = lane + 32 i; redux.sync finds the largest key, then the lowest candidate
+// holding it; the owner removes it (key 0) and rescans.  Winners go to wrow[0..K).
+__device__ __forceinline__ void warp_topk(uint32_t* krow, int nc, int K, int* wrow) {
+  const int lane = lane_id();
+  uint32_t bk = 0u;
+  int bc = 0x7fffffff;
+  for (int c = lane; c < nc; c += 32) {
+    const uint32_t k = krow[c];
+    if (k > bk) {
+      bk = k;
+      bc = c;
+    }
+  }
+  for (int r = 0; r < K; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t w = __reduce_min_sync(0xffffffffu, bk == m ? (uint32_t)bc : 0x7fffffffu);
+    if (lane == 0) wrow[r] = (int)w;
+    if (bc == (int)w && bk == m) {  // the owner drops its winner and finds its next best
+      krow[w] = 0u;
+      bk = 0u;
+      bc = 0x7fffffff;
+      for (int c = lane; c < nc; c += 32) {
+        const uint32_t k = krow[c];
+        if (k > bk) {
+          bk = k;
+          bc = c;
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// grid.x = B*H * groups; dynamic smem: see select_smem_bytes.
 // parent_idx == nullptr selects the coarsest-level mode.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int level, int gq,
                                                              const float* __restrict__ qp,
@@ -46,11 +87,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
   const int grp = blockIdx.x - bh * groups;
   const int a0 = grp * gq;
   const int rows = min(gq, n - a0);
+  const int chunk = min(nc, kSelChunk);
 
-  float* qs = sel_smem;                                           // [gq][64]
-  int* cand = reinterpret_cast<int*>(qs + gq * kD);                // [nc] (sparse only)
+  float* qs = sel_smem;                                             // [gq][64]
+  float* ks = qs + gq * kD;                                         // [chunk][68]
+  int* cand = reinterpret_cast<int*>(ks + chunk * kSelRowStride);   // [nc] (sparse only)
   uint32_t* sk = reinterpret_cast<uint32_t*>(cand + (sparse ? nc : 0));  // [gq][nc] score keys
-  int* win = reinterpret_cast<int*>(sk + gq * nc);                 // [gq][K]
+  int* win = reinterpret_cast<int*>(sk + gq * nc);                  // [gq][K]
 
   const int tid = threadIdx.x;
   const float* qbase = qp + ((long long)bh * n + a0) * kD;
@@ -65,76 +108,72 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
   }
   __syncthreads();
 
-  // ---- scores: a thread owns one candidate row (in registers) and every nsplit-th query;
-  // four queries at a time keep four independent FMA chains in flight.
-  const int nsplit = nc >= kSelThreads ? 1 : kSelThreads / nc;
-  const int cstep = nc >= kSelThreads ? kSelThreads : nc;
-  const int qsub = tid / cstep;
-  for (int c = tid % cstep; c < nc; c += cstep) {
-    const int key = sparse ? cand[c] : c;
-    const float4* krow = reinterpret_cast<const float4*>(kp + ((long long)bh * n + key) * kD);
-    float4 kr[kD / 4];
+  // ---- scores, one chunk of candidate rows at a time.  Thread t computes a tile of 2
+  // queries (t / tpq selects the pair) x 4 candidates strided by tpq (t % tpq selects the
+  // first) from shared memory.
+  const int qgroups = (gq + 1) / 2;
+  const int tpq = kSelThreads / qgroups;      // threads per query pair (32 for 16 queries)
+  const int qg = tid / tpq;
+  const int ct0 = tid - qg * tpq;
+  for (int c0 = 0; c0 < nc; c0 += chunk) {
+    const int cn = min(chunk, nc - c0);
+    // stage rows c0 .. c0+cn-1 (coalesced: 16 threads copy one 256-byte row)
+    for (int i = tid; i < cn * (kD / 4); i += kSelThreads) {
+      const int r = i / (kD / 4);
+      const int piece = i - r * (kD / 4);
+      const int key = sparse ? cand[c0 + r] : c0 + r;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + key) * kD) + piece);
+      *reinterpret_cast<float4*>(ks + r * kSelRowStride + piece * 4) = v;
+    }
+    __syncthreads();
+    for (int c = ct0; c < cn; c += 4 * tpq) {
+      float acc[2][4];
 #pragma unroll
-    for (int i = 0; i < kD / 4; ++i) kr[i] = __ldg(krow + i);
-    for (int q0 = qsub; q0 < gq; q0 += 4 * nsplit) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const float4* qr[4];
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) qr[u] = reinterpret_cast<const float4*>(qs + min(q0 + u * nsplit, gq - 1) * kD);
+        for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+      const float4* kr[4];
 #pragma unroll
+      for (int v = 0; v < 4; ++v) kr[v] = reinterpret_cast<const float4*>(ks + min(c + v * tpq, cn - 1) * kSelRowStride);
+      const float4* qr[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) qr[u] = reinterpret_cast<const float4*>(qs + min(2 * qg + u, gq - 1) * kD);
+#pragma unroll 4
       for (int i = 0; i < kD / 4; ++i) {
+        float4 kv[4], qv[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 qv = qr[u][i];
-          acc[u] = fmaf(qv.x, kr[i].x, acc[u]);
-          acc[u] = fmaf(qv.y, kr[i].y, acc[u]);
-          acc[u] = fmaf(qv.z, kr[i].z, acc[u]);
-          acc[u] = fmaf(qv.w, kr[i].w, acc[u]);
+        for (int v = 0; v < 4; ++v) kv[v] = kr[v][i];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) qv[u] = qr[u][i];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            acc[u][v] = fmaf(qv[u].x, kv[v].x, acc[u][v]);
+            acc[u][v] = fmaf(qv[u].y, kv[v].y, acc[u][v]);
+            acc[u][v] = fmaf(qv[u].z, kv[v].z, acc[u][v]);
+            acc[u][v] = fmaf(qv[u].w, kv[v].w, acc[u][v]);
+          }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int qi = 2 * qg + u;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int cc = c + v * tpq;
+          if (qi < gq && cc < cn) sk[qi * nc + c0 + cc] = score_key(acc[u][v]);
         }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int qi = q0 + u * nsplit;
-        if (qi < gq) sk[qi * nc + c] = score_key(acc[u]);
-      }
     }
+    __syncthreads();
   }
-  __syncthreads();
 
-  // ---- K rounds per query, one warp per query: each lane keeps the best of its candidates
-  // c = lane + 32 i; redux.sync finds the largest key, then the lowest candidate holding it.
+  // ---- K rounds per query, one warp per query
   const int warp = tid >> 5;
   const int lane = tid & 31;
   for (int qi = warp; qi < rows; qi += kSelThreads / 32) {
-    uint32_t* krow = sk + qi * nc;
     int* wrow = win + qi * K;
-    uint32_t bk = 0u;
-    int bc = 0x7fffffff;
-    for (int c = lane; c < nc; c += 32) {
-      const uint32_t k = krow[c];
-      if (k > bk) {
-        bk = k;
-        bc = c;
-      }
-    }
-    for (int r = 0; r < K; ++r) {
-      const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-      const uint32_t w = __reduce_min_sync(0xffffffffu, bk == m ? (uint32_t)bc : 0x7fffffffu);
-      if (lane == 0) wrow[r] = (int)w;
-      if (bc == (int)w && bk == m) {  // the owner drops its winner and finds its next best
-        krow[w] = 0u;
-        bk = 0u;
-        bc = 0x7fffffff;
-        for (int c = lane; c < nc; c += 32) {
-          const uint32_t k = krow[c];
-          if (k > bk) {
-            bk = k;
-            bc = c;
-          }
-        }
-      }
-    }
-    __syncwarp();
+    warp_topk(sk + qi * nc, nc, K, wrow);
     // ascending order: each winner's rank is the number of smaller winners
     int* orow = out_idx + ((long long)bh * n + a0 + qi) * K;
     for (int r = lane; r < K; r += 32) {
@@ -148,7 +187,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
 }
 
 inline size_t select_smem_bytes(int gq, int nc, int K, bool sparse) {
-  return sizeof(float) * ((size_t)gq * kD + (sparse ? nc : 0) + (size_t)gq * nc + (size_t)gq * K);
+  const int chunk = nc < kSelChunk ? nc : kSelChunk;
+  return sizeof(float) * ((size_t)gq * kD + (size_t)chunk * kSelRowStride + (sparse ? nc : 0) + (size_t)gq * nc +
+                          (size_t)gq * K);
 }
 
 }  // namespace llsa

@@ -43,6 +43,7 @@ def full_check(B, H, N, D, topk, levels, dtype, qk_kind, seed, backward=True):
     (1, 1, 8192, 2, 3),      # three levels, n_3 = 2
     (2, 1, 16384, 8, 2),
     (1, 1, 65536, 1, 4),     # four levels, n_4 = 1, K = 1
+    (1, 2, 8192, 4, 1),      # coarsest level of 512 keys: scored in two passes of 256
 ])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_small_shapes(B, H, N, topk, levels, dtype):
@@ -153,3 +154,10 @@ def test_autograd_op_matches_buffers_path():
     assert np.array_equal(o.detach().float().cpu().numpy(), gpu["o"])
     assert np.array_equal(q.grad.float().cpu().numpy(), gpu["dq"])
     assert np.array_equal(k.grad.float().cpu().numpy(), gpu["dk"])
+
+
+def test_single_level_long_sequence():
+    """L = 1 at N = 65536: the coarsest level is 4096 keys (16 scoring passes, 4 queries per
+    CTA), and the CSR rows are long."""
+    sel, rep = full_check(1, 1, 65536, 64, 8, 1, "bf16", "smooth", seed=41)
+    print(sel, rep)
