@@ -41,12 +41,12 @@ def dist_env():
     return rank, world, local
 
 
-def dist_init(world, local):
+def dist_init(world, local, backend: str = "nccl"):
     import torch
     import torch.distributed as dist
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
 
 
 def dist_barrier(world):
@@ -55,14 +55,20 @@ def dist_barrier(world):
         dist.barrier()
 
 
-def dist_max(x: float, world: int) -> float:
+def dist_max(x: float, world: int, device: str = "cuda") -> float:
+    """Maximum of x over all ranks (the step time of a multi-GPU run is the slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(tokens_per_step: int, steps: int, world: int, ms_total: float) -> float:
+    """Whole-job tokens/s: every rank runs `steps` steps of its own replica."""
+    return world * steps * tokens_per_step / (ms_total / 1000.0)
 
 
 def dist_done(world):
@@ -271,7 +277,7 @@ def run_ours(args):
         x["share"] = x["total_ms"] / total_kernel_ms
 
     tokens_per_step = cfg.B * cfg.N
-    value = world * args.steps * tokens_per_step / (ms_total / 1000.0)
+    value = weak_scaling_value(tokens_per_step, args.steps, world, ms_total)
     ms_per_step = ms_total / args.steps
 
     # algorithmic roofline of the dominant kernel

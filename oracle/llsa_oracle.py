@@ -44,6 +44,12 @@ Readings where the pages are silent (each one is also listed in the design notes
   tokens pass their gradient back to the input tokens through the mean-pool
   adjoint (each of the 16^l tokens under a level-l token receives 1/16^l of it).
 * LSE is the natural-log log-sum-exp of the scaled scores.
+
+Parity unpinned against the paper: no page fixes the enrichment content or weighting or
+the pyramid's rounding order, so those follow the readings above.  The oracle is pinned to
+those readings by closed forms (dense attention over the concatenated levels, a dense-mask
+restatement, finite differences) and to the method's fixed parts by brute force, but not
+to the authors' own code, which the pages do not include.
 """
 from __future__ import annotations
 
