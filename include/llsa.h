@@ -171,6 +171,33 @@ llsa_status llsa_backward(const llsa_shape* shape, const void* q, const void* k,
 llsa_status llsa_device_status(int32_t* code_out, llsa_stream_t stream);
 
 /*
+ * Index transpose for callers that cannot hand the library any device memory
+ * (no counterpart on the pages: an interface addition of this library).
+ *
+ * llsa_index_transpose needs scratch that its caller allocates.  Some callers cannot do
+ * that: a plugin host that passes kernels only their inputs and outputs, or a runtime whose
+ * device memory is planned once at start-up and may not grow or be requested per call.
+ * This entry point takes no workspace and allocates nothing (no cudaMalloc, no allocating
+ * library routine).  Its scratch is a fixed array inside libllsa.so of
+ * LLSA_NOALLOC_SCRATCH_BYTES (8 MiB), which every GPU that loads the library holds until the
+ * process exits.
+ *
+ *  - Shapes whose llsa_transpose_workspace_bytes() exceeds LLSA_NOALLOC_SCRATCH_BYTES are
+ *    rejected with LLSA_ERR_WORKSPACE before anything is launched (the headline shape
+ *    B=1, H=6, N=65536, L=3, K=8 needs about 0.9 MB; N=262144, K=16 about 6.8 MB).
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current; make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents.  The transpose
+ *    writes every scratch word before it reads it, so nothing needs clearing, but calls
+ *    whose kernels can overlap on the GPU (different streams, or different host threads
+ *    without ordering) race on the array: order them, e.g. on one stream.
+ *  - Arguments, outputs, validation and results are those of llsa_index_transpose.
+ */
+#define LLSA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+llsa_status llsa_index_transpose_noalloc(const llsa_shape* shape, const int32_t* idx, int32_t* row_ptr,
+                                         int32_t* col, llsa_stream_t stream);
+
+/*
  * Per-launch trace (instrumentation; no counterpart on the pages).  Between
  * llsa_trace_begin and llsa_trace_end, every kernel launch made by the calling host thread
  * through the calls above is bracketed by two cudaEventRecord calls on that call's stream:

@@ -51,6 +51,7 @@ SIGNATURES = {
     "llsa_build_pyramid": (_I, [_SP, _P, _P, _P, _P, _P, _P, _P]),
     "llsa_select": (_I, [_SP, _P, _P, _P, _P]),
     "llsa_index_transpose": (_I, [_SP, _P, _P, _P, _P, _S, _P]),
+    "llsa_index_transpose_noalloc": (_I, [_SP, _P, _P, _P, _P]),
     "llsa_forward": (_I, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "llsa_backward": (_I, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "llsa_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _P]),
@@ -63,6 +64,9 @@ SIGNATURES = {
 class LLSAExtensionMissing(RuntimeError):
     pass
 
+
+# Size of the fixed scratch array behind llsa_index_transpose_noalloc (LLSA_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _lib = None
 

@@ -100,6 +100,14 @@ def llsa_index_transpose(shape, idx, row_ptr, col, workspace, stream=None) -> No
         _ref(shape), _p(idx), _p(row_ptr), _p(col), _p(workspace), nbytes, _stream(stream)))
 
 
+def llsa_index_transpose_noalloc(shape, idx, row_ptr, col, stream=None) -> None:
+    """llsa_index_transpose without a workspace, for callers that cannot allocate device
+    memory: the library's own fixed 8 MiB scratch array is used (calls on overlapping
+    streams race on it; the first call on a device must precede any stream capture)."""
+    _check("llsa_index_transpose_noalloc", _lib.load().llsa_index_transpose_noalloc(
+        _ref(shape), _p(idx), _p(row_ptr), _p(col), _stream(stream)))
+
+
 def llsa_forward(shape, q, k, v, k_pyr, v_pyr, idx, o, lse, stream=None) -> None:
     _check("llsa_forward", _lib.load().llsa_forward(
         _ref(shape), _p(q), _p(k), _p(v), _p(k_pyr), _p(v_pyr), _p(idx), _p(o), _p(lse), _stream(stream)))

@@ -12,6 +12,11 @@
 
 using namespace llsa;
 
+// Scratch of llsa_index_transpose_noalloc: one fixed array per device that loads the
+// library.  Host code must not use this name as an address; it asks the runtime for the
+// device address (cudaGetSymbolAddress) once per device.
+static __device__ __align__(256) unsigned char g_llsa_noalloc_scratch[LLSA_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -214,6 +219,26 @@ llsa_status launch_coarse_reduce(const Geometry& g, float scale, const int32_t* 
   });
 }
 
+// Device address of g_llsa_noalloc_scratch on the current device, looked up on the first
+// call per device (with that device current) and remembered.
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+llsa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LLSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LLSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_llsa_noalloc_scratch) != cudaSuccess || p == nullptr) return LLSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LLSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -356,6 +381,18 @@ llsa_status llsa_index_transpose(const llsa_shape* s, const int32_t* idx, int32_
   return launch(kKTransposeBucket, cs, [&] {
     transpose_bucket_kernel<<<bucket_ctas, kTrThreads, 0, cs>>>(tg, ws_ent, ws_hist, row_ptr, col);
   });
+}
+
+llsa_status llsa_index_transpose_noalloc(const llsa_shape* s, const int32_t* idx, int32_t* row_ptr, int32_t* col,
+                                         llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  if (!idx || !row_ptr || !col || !aligned16(idx) || !aligned16(row_ptr) || !aligned16(col))
+    return LLSA_ERR_INVALID_ARG;
+  if (transpose_ws_bytes(make_geometry(s)) > LLSA_NOALLOC_SCRATCH_BYTES) return LLSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != LLSA_OK) return st;
+  return llsa_index_transpose(s, idx, row_ptr, col, scratch, LLSA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 llsa_status llsa_forward(const llsa_shape* s, const void* q, const void* k, const void* v, const float* k_pyr,
