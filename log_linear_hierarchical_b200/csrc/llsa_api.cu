@@ -195,15 +195,6 @@ llsa_status launch(int id, cudaStream_t cs, F&& f) {
   return st;
 }
 
-#ifndef LLSA_FWD_STAGES
-#define LLSA_FWD_STAGES 2
-#endif
-#ifndef LLSA_DQ_STAGES
-#define LLSA_DQ_STAGES 2
-#endif
-#ifndef LLSA_KV_STAGES
-#define LLSA_KV_STAGES 2
-#endif
 constexpr int kFwdStages = LLSA_FWD_STAGES;
 constexpr int kDqStages = LLSA_DQ_STAGES;
 constexpr int kDkvStages = LLSA_KV_STAGES;

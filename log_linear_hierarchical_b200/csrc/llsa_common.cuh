@@ -15,6 +15,19 @@ constexpr int kD = 64;          // channels per head handled by this build
 constexpr int kMaxLevels = 4;
 constexpr int kTileBytes = 2048;  // one 16-token x 64-channel bf16 tile
 
+// TMA ring depths of the attention kernels (forward, query-major dQ, key-major dK/dV).  A
+// sweep on B200 at the headline workload preferred 2 stages everywhere: deeper rings cost
+// more shared memory per warp than they hide, since occupancy hides the L2 latency better.
+#ifndef LLSA_FWD_STAGES
+#define LLSA_FWD_STAGES 2
+#endif
+#ifndef LLSA_DQ_STAGES
+#define LLSA_DQ_STAGES 2
+#endif
+#ifndef LLSA_KV_STAGES
+#define LLSA_KV_STAGES 2
+#endif
+
 // Per-call geometry: level sizes and the level-major offsets of every packed buffer.
 struct Geometry {
   int B, H, N, D, K, L, BH;
