@@ -1,6 +1,9 @@
 """Builds libllsa.so (the CUDA C-ABI library) in-tree for sm_100a with nvcc.
 
-Usage: python -m log_linear_hierarchical_b200.build [--verbose-ptxas]
+Usage: python -m log_linear_hierarchical_b200.build [--verbose-ptxas] [--define NAME=VALUE ...]
+
+--define passes a compile-time switch to nvcc, e.g. LLSA_KEY_MAJOR_TC=1 selects the tcgen05
+key-major dK/dV kernel instead of the mma.sync one.
 """
 from __future__ import annotations
 
@@ -32,13 +35,14 @@ def sources_newer_than_lib() -> bool:
     return any(os.path.getmtime(f) > t for f in files if os.path.isfile(f))
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+def build(force: bool = False, ptxas_verbose: bool = False, defines: tuple[str, ...] = ()) -> str:
     if not force and not sources_newer_than_lib():
         return LIB
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp"]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
+    cmd += ["-D" + d for d in defines]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
@@ -50,5 +54,7 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv)
+    args = sys.argv[1:]
+    defs = tuple(args[i + 1] for i, a in enumerate(args) if a == "--define" and i + 1 < len(args))
+    build(force=True, ptxas_verbose="--verbose-ptxas" in args, defines=defs)
     print(LIB)

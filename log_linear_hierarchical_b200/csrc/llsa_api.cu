@@ -6,6 +6,9 @@
 #include <mutex>
 
 #include "attn_simt.cuh"
+#if LLSA_KEY_MAJOR_TC
+#include "attn_bwd_tc.cuh"
+#endif
 #include "pyramid.cuh"
 #include "select.cuh"
 #include "transpose.cuh"
@@ -164,13 +167,15 @@ enum KernelId {
   kKBwdDqF32,
   kKBwdDkdvF32,
   kKBwdCoarseBf16,
+  kKBwdDkdvTc,
+  kKBwdDkdvEmpty,
   kKNumKernels
 };
 
 const char* const kKernelNames[kKNumKernels] = {
     "unknown",          "pyramid_l12",          "pyramid_up",   "select",           "transpose_hist",
     "transpose_scatter", "transpose_bucket",    "attn_fwd_bf16", "attn_bwd_dq_bf16", "coarse_grad_reduce",
-    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32", "attn_bwd_coarse_bf16"};
+    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32", "attn_bwd_coarse_bf16", "attn_bwd_dkdv_tc", "dkdv_empty_rows"};
 
 struct TraceState {
   cudaEvent_t* ev = nullptr;
@@ -468,6 +473,25 @@ llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, con
       if (st != LLSA_OK) return st;
     }
     if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
+#if LLSA_KEY_MAJOR_TC
+    {
+      int dev = 0, sms = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LLSA_ERR_CUDA;
+      if (!allow_smem(attn_bwd_dkdv_tc_kernel, kTcSmemBytes)) return LLSA_ERR_CUDA;
+      const int grid = total_blocks < 2 * sms ? total_blocks : 2 * sms;
+      st = launch(kKBwdDkdvEmpty, cs, [&] {
+        dkdv_empty_rows_kernel<<<(total_blocks + 3) / 4, 128, 0, cs>>>(P, row_ptr, ws, static_cast<__nv_bfloat16*>(dk),
+                                                                      static_cast<__nv_bfloat16*>(dv));
+      });
+      if (st != LLSA_OK) return st;
+      return launch(kKBwdDkdvTc, cs, [&] {
+        attn_bwd_dkdv_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, cs>>>(
+            tq, tk, tv, tdo, P, lse, row_ptr, col, ws, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+      });
+    }
+#endif
     auto kern = attn_bwd_dkdv_bf16_kernel<kDkvStages>;
     if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
     return launch(kKBwdDkdvBf16, cs, [&] {

@@ -27,6 +27,14 @@ constexpr int kTileBytes = 2048;  // one 16-token x 64-channel bf16 tile
 #ifndef LLSA_KV_STAGES
 #define LLSA_KV_STAGES 2
 #endif
+// Key-major dK/dV on tcgen05 (1) or on mma.sync warps (0, the default).  At 16-key blocks
+// the tcgen05 kernel is the slower one on B200 (301 us against 195 us at B1 H6 N65536 L3
+// K8): every MMA reads its 4 KB query-side operand from shared memory, Q and dO are read
+// twice per batch, and 4 batches in flight per SM do not cover the ~2 us latency of the
+// gathered tiles; the mma.sync warps keep K/V fragments and accumulators in registers.
+#ifndef LLSA_KEY_MAJOR_TC
+#define LLSA_KEY_MAJOR_TC 0
+#endif
 
 // Per-call geometry: level sizes and the level-major offsets of every packed buffer.
 struct Geometry {
@@ -129,6 +137,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of the phase with the given parity (no suspend hint), for a thread that
+// polls several barriers.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
