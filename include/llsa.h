@@ -13,6 +13,8 @@
  * The path is split into five calls, in this order for one training step:
  *   llsa_build_pyramid -> llsa_select -> llsa_forward            (forward)
  *   llsa_index_transpose -> llsa_backward                        (backward)
+ * llsa_train_step makes all five (the transpose on a second stream), and a plan replays
+ * a captured sequence of steps as one CUDA graph.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -30,8 +32,9 @@
  *    idx row contains key j (a CSR matrix; row_ptr offsets are local to (l, b, h)).
  *  - lse: fp32 [B, H, N], natural-log log-sum-exp of each query's scaled scores.
  *  - Every pointer is device memory owned by the caller, 16-byte aligned (256-byte
- *    alignment recommended).  The library allocates no memory, keeps no state between
- *    calls and is reentrant; calls on different streams must not share output buffers.
+ *    alignment recommended).  The library allocates no device memory, keeps no state
+ *    between calls (a plan, below, is state its handle owns) and is reentrant; calls on
+ *    different streams must not share output buffers.
  *  - Every call is asynchronous on `stream` (NULL = legacy default stream) and never
  *    synchronises the host, except llsa_device_status.
  *  - Arguments are checked on the host before any launch.  A rejected call launches
@@ -161,6 +164,54 @@ llsa_status llsa_backward(const llsa_shape* shape, const void* q, const void* k,
                           const float* v_pyr, const int32_t* idx, const int32_t* row_ptr,
                           const int32_t* col, void* dq, void* dk, void* dv, void* workspace,
                           size_t workspace_bytes, llsa_stream_t stream);
+
+/*
+ * One training step (steps 1, 2, 4a, 5, 4b of this header) over caller-owned buffers
+ * (no counterpart on the pages: an interface addition of this library).
+ *
+ * Device buffers of one step, each as described for the single calls above; the two
+ * workspaces are those of llsa_index_transpose and llsa_backward and must not be shared
+ * with concurrent work.
+ */
+typedef struct {
+  const void* q; const void* k; const void* v; const void* dO;  /* inputs [B,H,N,D] `dtype` */
+  float* q_pyr; float* k_pyr; float* v_pyr;                      /* [L][B,H,n_l,D] fp32 */
+  int32_t* idx; int32_t* row_ptr; int32_t* col;                  /* selection and its CSR */
+  void* o; float* lse;                                           /* forward outputs */
+  void* dq; void* dk; void* dv;                                  /* gradients [B,H,N,D] `dtype` */
+  void* transpose_workspace; size_t transpose_workspace_bytes;
+  void* backward_workspace; size_t backward_workspace_bytes;
+} llsa_step_buffers;
+
+/*
+ * llsa_build_pyramid -> llsa_select -> llsa_forward -> llsa_backward on `stream`, with
+ * llsa_index_transpose on `side_stream`: the transpose is forked after the selection and
+ * joined before the part of the backward that reads the CSR (the coarse-token reduction and
+ * dK/dV), so it runs concurrently with the forward and dQ.  side_stream NULL or equal to
+ * `stream` runs the transpose on `stream`.  Results are those of the five calls in order.
+ * All checks are made before the first launch; a rejected step launches nothing.  Two
+ * CUDA events are created and released per call (no device memory is allocated).
+ */
+llsa_status llsa_train_step(const llsa_shape* shape, const llsa_step_buffers* buffers, llsa_stream_t stream,
+                            llsa_stream_t side_stream);
+
+/*
+ * A plan is `repeat` consecutive llsa_train_step calls on a fixed set of buffers, captured
+ * once into a CUDA graph (two internal streams; the transpose on the second) and
+ * instantiated; llsa_plan_launch replays it on `stream` with no per-kernel launch cost.
+ * The graph holds the buffer addresses and the shape: the buffers must stay allocated and
+ * unchanged in size while the plan exists, and their contents are read at launch time.
+ * Kernel launches made while the calling thread traces (llsa_trace_begin) are captured
+ * with their trace events, which the graph then records at every launch.
+ * llsa_plan_create: repeat in [1, 4096]; *plan_out is NULL on failure.  The plan owns the
+ * graph; llsa_plan_destroy releases it (NULL is ignored) and must not race a launch that
+ * has not been ordered before it on the host.
+ */
+typedef struct llsa_plan llsa_plan;
+llsa_status llsa_plan_create(const llsa_shape* shape, const llsa_step_buffers* buffers, int32_t repeat,
+                             llsa_plan** plan_out);
+llsa_status llsa_plan_launch(const llsa_plan* plan, llsa_stream_t stream);
+void llsa_plan_destroy(llsa_plan* plan);
 
 /*
  * Reads and clears the device status word that kernels set on an out-of-range index

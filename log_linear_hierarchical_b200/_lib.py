@@ -40,6 +40,18 @@ class LLSAShape(ctypes.Structure):
 
 _SP = ctypes.POINTER(LLSAShape)
 
+
+class LLSAStepBuffers(ctypes.Structure):
+    """Mirror of ``llsa_step_buffers``."""
+
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q", "k", "v", "dO", "q_pyr", "k_pyr", "v_pyr", "idx", "row_ptr",
+                                                 "col", "o", "lse", "dq", "dk", "dv")] + \
+               [("transpose_workspace", ctypes.c_void_p), ("transpose_workspace_bytes", ctypes.c_size_t),
+                ("backward_workspace", ctypes.c_void_p), ("backward_workspace_bytes", ctypes.c_size_t)]
+
+
+_BP = ctypes.POINTER(LLSAStepBuffers)
+
 SIGNATURES = {
     "llsa_status_string": (ctypes.c_char_p, [_I]),
     "llsa_validate_shape": (_I, [_SP]),
@@ -54,6 +66,10 @@ SIGNATURES = {
     "llsa_index_transpose_noalloc": (_I, [_SP, _P, _P, _P, _P]),
     "llsa_forward": (_I, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "llsa_backward": (_I, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "llsa_train_step": (_I, [_SP, _BP, _P, _P]),
+    "llsa_plan_create": (_I, [_SP, _BP, ctypes.c_int32, ctypes.POINTER(_P)]),
+    "llsa_plan_launch": (_I, [_P, _P]),
+    "llsa_plan_destroy": (None, [_P]),
     "llsa_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _P]),
     "llsa_trace_begin": (_I, [ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]),
     "llsa_trace_end": (_I, [ctypes.POINTER(ctypes.c_int32)]),

@@ -260,10 +260,68 @@ def llsa_backward_path(shape, q, k, v, do, buf: LLSABuffers, stream=None) -> Non
                   buf.dq, buf.dk, buf.dv, buf.ws_backward, stream)
 
 
-def llsa_train_step(shape, q, k, v, do, buf: LLSABuffers, stream=None) -> None:
-    """One full LLSA training step of the attention op: forward and backward."""
-    llsa_forward_path(shape, q, k, v, buf, stream)
-    llsa_backward_path(shape, q, k, v, do, buf, stream)
+def step_buffers(shape, q, k, v, do, buf: LLSABuffers) -> _lib.LLSAStepBuffers:
+    """The ``llsa_step_buffers`` of one step over ``buf`` (raw device addresses)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    return _lib.LLSAStepBuffers(
+        _p(q), _p(k), _p(v), _p(do), _p(buf.q_pyr), _p(buf.k_pyr), _p(buf.v_pyr), _p(buf.idx), _p(buf.row_ptr),
+        _p(buf.col), _p(buf.o), _p(buf.lse), _p(buf.dq), _p(buf.dk), _p(buf.dv),
+        _p(buf.ws_transpose), buf.ws_transpose.numel() * 4, _p(buf.ws_backward), buf.ws_backward.numel() * 4)
+
+
+_side_streams: dict[int, torch.cuda.Stream] = {}
+
+
+def side_stream(device=None) -> torch.cuda.Stream:
+    """The second stream a step forks its index transpose onto (one per device)."""
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index
+    if dev not in _side_streams:
+        _side_streams[dev] = torch.cuda.Stream(device=dev)
+    return _side_streams[dev]
+
+
+def llsa_train_step(shape, q, k, v, do, buf: LLSABuffers, stream=None, side=None) -> None:
+    """One full LLSA training step of the attention op (forward and backward) through
+    ``llsa_train_step``: the index transpose runs on ``side`` (default: this module's side
+    stream for the device) concurrently with the forward and dQ."""
+    sb = step_buffers(shape, q, k, v, do, buf)
+    side = side_stream(q.device) if side is None else side
+    _check("llsa_train_step", _lib.load().llsa_train_step(_ref(shape), ctypes.byref(sb), _stream(stream),
+                                                          _stream(side)))
+
+
+class LLSAPlan:
+    """``repeat`` training steps on fixed buffers, captured once into a CUDA graph
+    (``llsa_plan_create``) and replayed by ``launch`` (``llsa_plan_launch``).  Keeps the
+    tensors it was built on alive; ``close`` releases the graph."""
+
+    def __init__(self, shape, q, k, v, do, buf: LLSABuffers, repeat: int = 1):
+        self._keep = (q, k, v, do, buf)
+        sb = step_buffers(shape, q, k, v, do, buf)
+        handle = ctypes.c_void_p()
+        _check("llsa_plan_create", _lib.load().llsa_plan_create(_ref(shape), ctypes.byref(sb), repeat,
+                                                                ctypes.byref(handle)))
+        self._handle = handle
+        self.repeat = repeat
+
+    def launch(self, stream=None) -> None:
+        if not self._handle:
+            raise LLSAError("llsa_plan_launch", 1)
+        _check("llsa_plan_launch", _lib.load().llsa_plan_launch(self._handle, _stream(stream)))
+
+    def close(self) -> None:
+        if self._handle:
+            torch.cuda.synchronize()
+            _lib.load().llsa_plan_destroy(self._handle)
+            self._handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ----------------------------------------------------------------------------- autograd op

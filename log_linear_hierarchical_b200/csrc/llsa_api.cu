@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <new>
 
 #include "attn_simt.cuh"
 #if LLSA_KEY_MAJOR_TC
@@ -186,14 +187,24 @@ struct TraceState {
 thread_local TraceState g_trace;
 
 // Launches through `f`, checks the launch, and records the trace events if tracing is on.
+// Under stream capture the events become event-record nodes of the graph (external
+// records), so a captured plan is traced each time it is launched.
+void trace_record(cudaEvent_t e, cudaStream_t cs) {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(cs, &cap) == cudaSuccess && cap == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, cs, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, cs);
+}
+
 template <class F>
 llsa_status launch(int id, cudaStream_t cs, F&& f) {
   const bool tr = g_trace.ev != nullptr && g_trace.used < g_trace.cap;
-  if (tr) cudaEventRecord(g_trace.ev[2 * g_trace.used], cs);
+  if (tr) trace_record(g_trace.ev[2 * g_trace.used], cs);
   f();
   const llsa_status st = launch_status();
   if (tr) {
-    cudaEventRecord(g_trace.ev[2 * g_trace.used + 1], cs);
+    trace_record(g_trace.ev[2 * g_trace.used + 1], cs);
     g_trace.ids[g_trace.used] = id;
     ++g_trace.used;
   }
@@ -236,6 +247,166 @@ llsa_status noalloc_scratch(void** out) {
 }
 
 }  // namespace
+
+namespace {
+
+// The backward in two phases.  The query side (dQ, Delta and the coarse-token partials)
+// reads only the query-major selection; the key side (coarse-token gradients reduced
+// through the level-l CSRs, then dK/dV through the level-1 CSR) needs the transpose, so a
+// step can run the transpose concurrently with the forward and the query side.
+constexpr unsigned kQuerySide = 1, kKeySide = 2;
+
+llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
+                            const int32_t* idx, const int32_t* row_ptr, const int32_t* col, void* dq, void* dk,
+                            void* dv, void* workspace, unsigned phases, cudaStream_t cs) {
+  llsa_status st = LLSA_OK;
+  const Geometry g = make_geometry(s);
+  float* ws = static_cast<float*>(workspace);
+  const float scale = 1.0f / sqrtf((float)kD);
+  const int total_blocks = g.BH * g.n[1];
+  if (s->dtype == LLSA_BF16) {
+    CUtensorMap tq, tk, tv, tdo;
+    const long long rows = (long long)g.BH * g.N;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
+        !make_tile_map(&tdo, dO, rows))
+      return LLSA_ERR_CUDA;
+    AttnParams P{g, scale * kLog2e, scale};
+    const size_t kv_bytes = (size_t)kv_smem<kDkvStages>(1).total();
+    if (phases & kQuerySide) {
+      const size_t smem = (size_t)dq_smem<kDqStages>(g, kAttnWarps).total();
+      auto kern = attn_bwd_dq_bf16_kernel<kDqStages>;
+      if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+      const int per_cta = kAttnWarps * kUnitBlocks;
+      st = launch(kKBwdDqBf16, cs, [&] {
+        kern<<<(total_blocks + per_cta - 1) / per_cta, 32 * kAttnWarps, smem, cs>>>(
+            tq, tk, tv, tdo, P, k_pyr, v_pyr, idx, static_cast<const __nv_bfloat16*>(o), lse,
+            static_cast<__nv_bfloat16*>(dq), ws);
+      });
+      if (st != LLSA_OK) return st;
+      if (g.L >= 2) {
+        auto ckern = attn_bwd_coarse_bf16_kernel<kDkvStages>;
+        if (!allow_smem(ckern, kv_bytes)) return LLSA_ERR_CUDA;
+        const int ctas = g.BH * g.n[2] * (g.coarse_pad / kBlock);
+        st = launch(kKBwdCoarseBf16, cs, [&] {
+          ckern<<<ctas, 32, kv_bytes, cs>>>(tq, tdo, P, k_pyr, v_pyr, idx, lse, ws);
+        });
+        if (st != LLSA_OK) return st;
+      }
+    }
+    if (!(phases & kKeySide)) return LLSA_OK;
+    if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
+#if LLSA_KEY_MAJOR_TC
+    {
+      int dev = 0, sms = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LLSA_ERR_CUDA;
+      if (!allow_smem(attn_bwd_dkdv_tc_kernel, kTcSmemBytes)) return LLSA_ERR_CUDA;
+      const int grid = total_blocks < 2 * sms ? total_blocks : 2 * sms;
+      st = launch(kKBwdDkdvEmpty, cs, [&] {
+        dkdv_empty_rows_kernel<<<(total_blocks + 3) / 4, 128, 0, cs>>>(P, row_ptr, ws, static_cast<__nv_bfloat16*>(dk),
+                                                                      static_cast<__nv_bfloat16*>(dv));
+      });
+      if (st != LLSA_OK) return st;
+      return launch(kKBwdDkdvTc, cs, [&] {
+        attn_bwd_dkdv_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, cs>>>(
+            tq, tk, tv, tdo, P, lse, row_ptr, col, ws, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+      });
+    }
+#endif
+    auto kern = attn_bwd_dkdv_bf16_kernel<kDkvStages>;
+    if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
+    return launch(kKBwdDkdvBf16, cs, [&] {
+      kern<<<total_blocks, 32, kv_bytes, cs>>>(tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
+                                                static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+    });
+  }
+  if (phases & kQuerySide) {
+    const size_t smem = simt_dq_smem(g);
+    if (!allow_smem(attn_bwd_dq_f32_kernel, smem)) return LLSA_ERR_CUDA;
+    const int per_cta = g.L >= 2 ? kBlock : 1;
+    st = launch(kKBwdDqF32, cs, [&] {
+      attn_bwd_dq_f32_kernel<<<total_blocks / per_cta, kSimtThreads, smem, cs>>>(
+          g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+          static_cast<const float*>(o), lse, static_cast<const float*>(dO), k_pyr, v_pyr, idx,
+          static_cast<float*>(dq), ws);
+    });
+    if (st != LLSA_OK) return st;
+  }
+  if (!(phases & kKeySide)) return LLSA_OK;
+  if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
+  return launch(kKBwdDkdvF32, cs, [&] {
+    attn_bwd_dkdv_f32_kernel<<<total_blocks, kSimtThreads, 0, cs>>>(
+        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), lse,
+        static_cast<const float*>(dO), row_ptr, col, ws, static_cast<float*>(dk), static_cast<float*>(dv));
+  });
+}
+
+
+// ---------------------------------------------------------------------------- one step
+// Host-side checks of a step's buffers (the per-call checks, done up front so that a
+// rejected step launches nothing).
+llsa_status validate_step(const llsa_shape* s, const llsa_step_buffers* b) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  if (!b) return LLSA_ERR_INVALID_ARG;
+  const void* ptrs[17] = {b->q,   b->k,   b->v,  b->dO, b->q_pyr, b->k_pyr,
+                          b->v_pyr, b->idx, b->row_ptr, b->col, b->o, b->lse,
+                          b->dq,  b->dk,  b->dv, b->transpose_workspace, b->backward_workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s);
+  if (b->transpose_workspace_bytes < transpose_ws_bytes(g)) return LLSA_ERR_WORKSPACE;
+  if (b->backward_workspace_bytes < (size_t)bwd_workspace_layout(g).total * sizeof(float)) return LLSA_ERR_WORKSPACE;
+  return LLSA_OK;
+}
+
+// pyramid -> selection -> forward -> backward query side on `cs`; the transpose on `side`
+// (forked after the selection, joined before the backward key side), or on `cs` if side
+// is null.  The join is made on every path once the fork was made, so a capture that
+// fails part-way still ends with both streams joined.
+llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStream_t cs, cudaStream_t side) {
+  llsa_status st = llsa_build_pyramid(s, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, cs);
+  if (st == LLSA_OK) st = llsa_select(s, b->q_pyr, b->k_pyr, b->idx, cs);
+  if (st != LLSA_OK) return st;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (side) {
+    if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess) return LLSA_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventDestroy(fork);
+      return LLSA_ERR_CUDA;
+    }
+    if (cudaEventRecord(fork, cs) != cudaSuccess || cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)
+      st = LLSA_ERR_CUDA;
+    if (st == LLSA_OK)
+      st = llsa_index_transpose(s, b->idx, b->row_ptr, b->col, b->transpose_workspace, b->transpose_workspace_bytes,
+                                side);
+    if (cudaEventRecord(join, side) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
+  }
+  if (st == LLSA_OK) st = llsa_forward(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs);
+  if (st == LLSA_OK)
+    st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
+                         b->dq, b->dk, b->dv, b->backward_workspace, kQuerySide, cs);
+  if (side) {
+    if (cudaStreamWaitEvent(cs, join, 0) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
+    cudaEventDestroy(fork);
+    cudaEventDestroy(join);
+  } else if (st == LLSA_OK) {
+    st = llsa_index_transpose(s, b->idx, b->row_ptr, b->col, b->transpose_workspace, b->transpose_workspace_bytes, cs);
+  }
+  if (st == LLSA_OK)
+    st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
+                         b->dq, b->dk, b->dv, b->backward_workspace, kKeySide, cs);
+  return st;
+}
+
+}  // namespace
+
+struct llsa_plan {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
 
 extern "C" {
 
@@ -435,86 +606,63 @@ llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, con
   const void* ptrs[16] = {q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
-  const Geometry g = make_geometry(s);
-  const BwdWorkspace W = bwd_workspace_layout(g);
-  if (workspace_bytes < (size_t)W.total * sizeof(float)) return LLSA_ERR_WORKSPACE;
-  float* ws = static_cast<float*>(workspace);
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const float scale = 1.0f / sqrtf((float)kD);
-  const int total_blocks = g.BH * g.n[1];
-  if (s->dtype == LLSA_BF16) {
-    CUtensorMap tq, tk, tv, tdo;
-    const long long rows = (long long)g.BH * g.N;
-    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
-        !make_tile_map(&tdo, dO, rows))
-      return LLSA_ERR_CUDA;
-    {
-      AttnParams P{g, scale * kLog2e, scale};
-      const size_t smem = (size_t)dq_smem<kDqStages>(g, kAttnWarps).total();
-      auto kern = attn_bwd_dq_bf16_kernel<kDqStages>;
-      if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
-      const int per_cta = kAttnWarps * kUnitBlocks;
-      st = launch(kKBwdDqBf16, cs, [&] {
-        kern<<<(total_blocks + per_cta - 1) / per_cta, 32 * kAttnWarps, smem, cs>>>(
-            tq, tk, tv, tdo, P, k_pyr, v_pyr, idx, static_cast<const __nv_bfloat16*>(o), lse,
-            static_cast<__nv_bfloat16*>(dq), ws);
-      });
-      if (st != LLSA_OK) return st;
-    }
-    AttnParams P{g, scale * kLog2e, scale};
-    const size_t kv_bytes = (size_t)kv_smem<kDkvStages>(1).total();
-    if (g.L >= 2) {
-      auto kern = attn_bwd_coarse_bf16_kernel<kDkvStages>;
-      if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
-      const int ctas = g.BH * g.n[2] * (g.coarse_pad / kBlock);
-      st = launch(kKBwdCoarseBf16, cs, [&] {
-        kern<<<ctas, 32, kv_bytes, cs>>>(tq, tdo, P, k_pyr, v_pyr, idx, lse, ws);
-      });
-      if (st != LLSA_OK) return st;
-    }
-    if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
-#if LLSA_KEY_MAJOR_TC
-    {
-      int dev = 0, sms = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return LLSA_ERR_CUDA;
-      if (!allow_smem(attn_bwd_dkdv_tc_kernel, kTcSmemBytes)) return LLSA_ERR_CUDA;
-      const int grid = total_blocks < 2 * sms ? total_blocks : 2 * sms;
-      st = launch(kKBwdDkdvEmpty, cs, [&] {
-        dkdv_empty_rows_kernel<<<(total_blocks + 3) / 4, 128, 0, cs>>>(P, row_ptr, ws, static_cast<__nv_bfloat16*>(dk),
-                                                                      static_cast<__nv_bfloat16*>(dv));
-      });
-      if (st != LLSA_OK) return st;
-      return launch(kKBwdDkdvTc, cs, [&] {
-        attn_bwd_dkdv_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, cs>>>(
-            tq, tk, tv, tdo, P, lse, row_ptr, col, ws, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
-      });
-    }
-#endif
-    auto kern = attn_bwd_dkdv_bf16_kernel<kDkvStages>;
-    if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
-    return launch(kKBwdDkdvBf16, cs, [&] {
-      kern<<<total_blocks, 32, kv_bytes, cs>>>(tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
-                                                static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
-    });
-  }
-  const size_t smem = simt_dq_smem(g);
-  if (!allow_smem(attn_bwd_dq_f32_kernel, smem)) return LLSA_ERR_CUDA;
-  const int per_cta = g.L >= 2 ? kBlock : 1;
-  st = launch(kKBwdDqF32, cs, [&] {
-    attn_bwd_dq_f32_kernel<<<total_blocks / per_cta, kSimtThreads, smem, cs>>>(
-        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        static_cast<const float*>(o), lse, static_cast<const float*>(dO), k_pyr, v_pyr, idx,
-        static_cast<float*>(dq), ws);
-  });
+  if (workspace_bytes < (size_t)bwd_workspace_layout(make_geometry(s)).total * sizeof(float)) return LLSA_ERR_WORKSPACE;
+  return backward_phases(s, q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace,
+                         kQuerySide | kKeySide, reinterpret_cast<cudaStream_t>(stream));
+}
+
+llsa_status llsa_train_step(const llsa_shape* s, const llsa_step_buffers* b, llsa_stream_t stream,
+                            llsa_stream_t side_stream) {
+  const llsa_status st = validate_step(s, b);
   if (st != LLSA_OK) return st;
-  if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
-  return launch(kKBwdDkdvF32, cs, [&] {
-    attn_bwd_dkdv_f32_kernel<<<total_blocks, kSimtThreads, 0, cs>>>(
-        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), lse,
-        static_cast<const float*>(dO), row_ptr, col, ws, static_cast<float*>(dk), static_cast<float*>(dv));
-  });
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t side = reinterpret_cast<cudaStream_t>(side_stream);
+  return step_impl(s, b, cs, side == cs ? nullptr : side);
+}
+
+llsa_status llsa_plan_create(const llsa_shape* s, const llsa_step_buffers* b, int32_t repeat, llsa_plan** plan_out) {
+  if (!plan_out) return LLSA_ERR_INVALID_ARG;
+  *plan_out = nullptr;
+  if (repeat < 1 || repeat > 4096) return LLSA_ERR_INVALID_ARG;
+  llsa_status st = validate_step(s, b);
+  if (st != LLSA_OK) return st;
+  cudaStream_t cs = nullptr, side = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return LLSA_ERR_CUDA;
+  if (cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return LLSA_ERR_CUDA;
+  }
+  llsa_plan* plan = new (std::nothrow) llsa_plan();
+  if (!plan) st = LLSA_ERR_CUDA;
+  if (st == LLSA_OK && cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) != cudaSuccess) st = LLSA_ERR_CUDA;
+  if (st == LLSA_OK) {
+    for (int r = 0; r < repeat && st == LLSA_OK; ++r) st = step_impl(s, b, cs, side);
+    cudaGraph_t graph = nullptr;
+    if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
+    plan->graph = graph;
+    if (st == LLSA_OK && cudaGraphInstantiate(&plan->exec, graph, 0) != cudaSuccess) st = LLSA_ERR_CUDA;
+  }
+  cudaStreamDestroy(side);
+  cudaStreamDestroy(cs);
+  cudaGetLastError();  // clears the error a failed capture leaves behind; `st` reports it
+  if (st != LLSA_OK) {
+    llsa_plan_destroy(plan);
+    return st;
+  }
+  *plan_out = plan;
+  return LLSA_OK;
+}
+
+llsa_status llsa_plan_launch(const llsa_plan* plan, llsa_stream_t stream) {
+  if (!plan || !plan->exec) return LLSA_ERR_INVALID_ARG;
+  return cudaGraphLaunch(plan->exec, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? LLSA_OK : LLSA_ERR_CUDA;
+}
+
+void llsa_plan_destroy(llsa_plan* plan) {
+  if (!plan) return;
+  if (plan->exec) cudaGraphExecDestroy(plan->exec);
+  if (plan->graph) cudaGraphDestroy(plan->graph);
+  delete plan;
 }
 
 llsa_status llsa_device_status(int32_t* code_out, llsa_stream_t stream) {

@@ -93,3 +93,25 @@ def test_status_error_message(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(_lib.LLSAExtensionMissing):
         _lib.load(str(tmp_path / "nope.so"))
+
+
+def test_step_and_plan_rejected_before_launch(lib):
+    """llsa_train_step and llsa_plan_create check every buffer before any CUDA call."""
+    s = shape()
+    empty = _lib.LLSAStepBuffers()
+    assert lib.llsa_train_step(ctypes.byref(s), ctypes.byref(empty), None, None) == 1
+    assert lib.llsa_train_step(ctypes.byref(s), None, None, None) == 1
+    ptrs = {n: 256 for n, _ in _lib.LLSAStepBuffers._fields_ if not n.endswith("_bytes")}
+    small_ws = _lib.LLSAStepBuffers(**ptrs, transpose_workspace_bytes=api.llsa_transpose_workspace_bytes(s) - 1,
+                                    backward_workspace_bytes=api.llsa_backward_workspace_bytes(s))
+    assert lib.llsa_train_step(ctypes.byref(s), ctypes.byref(small_ws), None, None) == 3
+    misaligned = _lib.LLSAStepBuffers(**dict(ptrs, lse=260), transpose_workspace_bytes=1 << 30,
+                                      backward_workspace_bytes=1 << 30)
+    assert lib.llsa_train_step(ctypes.byref(s), ctypes.byref(misaligned), None, None) == 1
+    handle = ctypes.c_void_p(1234)
+    assert lib.llsa_plan_create(ctypes.byref(s), ctypes.byref(small_ws), 1, ctypes.byref(handle)) == 3
+    assert not handle.value
+    assert lib.llsa_plan_create(ctypes.byref(s), ctypes.byref(small_ws), 0, ctypes.byref(handle)) == 1
+    assert lib.llsa_plan_create(ctypes.byref(s), ctypes.byref(small_ws), 1, None) == 1
+    assert lib.llsa_plan_launch(None, None) == 1
+    lib.llsa_plan_destroy(None)

@@ -1,0 +1,117 @@
+"""The one-call step (llsa_train_step, transpose on a second stream) and its CUDA-graph
+plan give the same bits as the five calls made one after another on one stream."""
+import numpy as np
+import pytest
+import torch
+
+from log_linear_hierarchical_b200 import api
+from llsa_testlib import TORCH_DTYPE, run_gpu
+from synthetic import CONFIGS, make_config_inputs, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+KEYS = ("o", "lse", "dq", "dk", "dv")
+
+
+def outputs(buf):
+    out = {k: getattr(buf, k).float().cpu().numpy() for k in KEYS}
+    out["idx"] = buf.idx.cpu().numpy()
+    out["row_ptr"] = buf.row_ptr.cpu().numpy()
+    out["col"] = buf.col.cpu().numpy()
+    return out
+
+
+def assert_same(a, b):
+    for x, y in zip(a["idx"], b["idx"]):
+        assert np.array_equal(x, y)
+    for x, y in zip(a["col"], b["col"]):
+        assert np.array_equal(x, y)
+    for x, y in zip(a["row_ptr"], b["row_ptr"]):
+        assert np.array_equal(x, y)
+    for k in KEYS:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def separate_calls(cfg, inputs):
+    ref = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs)
+    ref["idx"] = np.concatenate([x.ravel() for x in ref["idx"]])
+    ref["row_ptr"] = np.concatenate([x.ravel() for x in ref["row_ptr"]])
+    ref["col"] = np.concatenate([x.ravel() for x in ref["col"]])
+    return ref
+
+
+def setup(cfg, inputs):
+    tdt = TORCH_DTYPE[cfg.dtype]
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, tdt)
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    return shape, dev, api.LLSABuffers.allocate(shape, "cuda", tdt)
+
+
+def flat(out):
+    return {k: (v.ravel() if k in ("idx", "row_ptr", "col") else v) for k, v in out.items()}
+
+
+@pytest.mark.parametrize("cfg_id", [1, 3])
+def test_train_step_matches_separate_calls(cfg_id):
+    cfg = CONFIGS[cfg_id]
+    inputs = make_config_inputs(cfg)
+    ref = separate_calls(cfg, inputs)
+    shape, dev, buf = setup(cfg, inputs)
+    api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+    torch.cuda.synchronize()
+    assert api.llsa_device_status() == 0
+    assert_same(flat(outputs(buf)), ref)
+
+
+def test_train_step_without_side_stream():
+    cfg = CONFIGS[3]
+    inputs = make_config_inputs(cfg)
+    ref = separate_calls(cfg, inputs)
+    shape, dev, buf = setup(cfg, inputs)
+    s = torch.cuda.current_stream()
+    api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, side=s)
+    torch.cuda.synchronize()
+    assert_same(flat(outputs(buf)), ref)
+
+
+def test_plan_replays_match_separate_calls():
+    cfg = CONFIGS[3]
+    inputs = make_config_inputs(cfg)
+    ref = separate_calls(cfg, inputs)
+    shape, dev, buf = setup(cfg, inputs)
+    plan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=2)
+    for _ in range(2):
+        for t in (buf.o, buf.dq, buf.dk, buf.dv):
+            t.zero_()
+        plan.launch()
+        torch.cuda.synchronize()
+        assert api.llsa_device_status() == 0
+        assert_same(flat(outputs(buf)), ref)
+    # the plan reads its inputs at launch time: new inputs in the same buffers, new results
+    other = make_inputs(cfg.B, cfg.H, cfg.N, cfg.D, cfg.dtype, cfg.qk_kind, cfg.cfg_id + 100)
+    ref2 = separate_calls(cfg, other)
+    for k in ("q", "k", "v", "do"):
+        dev[k].copy_(other[k].cuda())
+    plan.launch()
+    torch.cuda.synchronize()
+    assert_same(flat(outputs(buf)), ref2)
+    plan.close()
+
+
+def test_plan_is_traced_at_every_launch():
+    cfg = CONFIGS[3]
+    inputs = make_config_inputs(cfg)
+    shape, dev, buf = setup(cfg, inputs)
+    with api.LaunchTrace(64) as eager:
+        api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+    per_step = eager.used
+    assert per_step >= 10
+    tr = api.LaunchTrace(64)
+    with tr:
+        plan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=3)
+    assert tr.used == 3 * per_step
+    plan.launch()
+    times = tr.launches()
+    assert [n for n, _ in times] == [n for n, _ in eager.launches()] * 3
+    assert all(ms > 0 for _, ms in times)
+    plan.close()
