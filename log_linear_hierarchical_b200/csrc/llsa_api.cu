@@ -509,6 +509,27 @@ llsa_status llsa_select(const llsa_shape* s, const float* q_pyr, const float* k_
       gq = kBlock;
       while (gq > 1 && (gq > n || (long long)gq * n > 16384)) gq >>= 1;
     }
+    if (sparse && g.K >= 2 && g.K <= 16) {
+      // children of the parent's K keys scored in registers (select_children_kernel)
+      const size_t smem = select_children_smem_bytes(nc);
+      const float* qpl = q_pyr + g.pyr_off[l];
+      const float* kpl = k_pyr + g.pyr_off[l];
+      const int* par = idx + g.idx_off[l + 1];
+      int* out = idx + g.idx_off[l];
+      const unsigned grid = (unsigned)(g.BH * (n / kBlock));
+      auto run = [&](auto kern) -> llsa_status {
+        if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+        return launch(kKSelect, cs, [&] { kern<<<grid, kSelThreads, smem, cs>>>(g, l, qpl, kpl, par, out); });
+      };
+      switch (g.K) {
+        case 2: st = run(select_children_kernel<1>); break;
+        case 4: st = run(select_children_kernel<2>); break;
+        case 8: st = run(select_children_kernel<4>); break;
+        default: st = run(select_children_kernel<8>); break;
+      }
+      if (st != LLSA_OK) return st;
+      continue;
+    }
     const size_t smem = select_smem_bytes(gq, nc, g.K, sparse);
     if (!allow_smem(select_kernel, smem)) return LLSA_ERR_CUDA;
     const int groups = (n + gq - 1) / gq;

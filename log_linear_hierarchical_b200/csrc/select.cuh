@@ -192,4 +192,123 @@ inline size_t select_smem_bytes(int gq, int nc, int K, bool sparse) {
                           (size_t)gq * K);
 }
 
+// Finer levels with 16K = 32 * CPT candidates (K = 2, 4, 8, 16): the 16 sibling queries of
+// one parent, 8 warps, warp w scoring queries 2w and 2w + 1 against all candidates.  Lane l
+// holds candidates l + 32 j (j < CPT) of both queries in registers, which is the layout the
+// warp Top-K walks, so scores never leave registers: K rounds of redux.sync max (score key)
+// then min (candidate position), the two queries' rounds interleaved.  The dot products
+// accumulate channels 0..63 in order, as in select_kernel, so both give the same scores.
+template <int CPT>
+__global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g, int level,
+                                                                      const float* __restrict__ qp,
+                                                                      const float* __restrict__ kp,
+                                                                      const int* __restrict__ parent_idx,
+                                                                      int* __restrict__ out_idx) {
+  constexpr int NC = 32 * CPT;
+  constexpr int K = 2 * CPT;  // NC = 16 K
+  extern __shared__ __align__(16) float sel_smem[];
+  const int n = g.n[level];
+  const int groups = n / kBlock;
+  const int bh = blockIdx.x / groups;
+  const int grp = blockIdx.x - bh * groups;
+  const int a0 = grp * kBlock;
+
+  float* qs = sel_smem;                                          // [16][64]
+  float* ks = qs + kBlock * kD;                                  // [NC][68]
+  int* cand = reinterpret_cast<int*>(ks + NC * kSelRowStride);   // [NC]
+
+  const int tid = threadIdx.x;
+  const float4* qbase = reinterpret_cast<const float4*>(qp + ((long long)bh * n + a0) * kD);
+  for (int i = tid; i < kBlock * kD / 4; i += kSelThreads) reinterpret_cast<float4*>(qs)[i] = __ldg(qbase + i);
+  const int np = g.n[level + 1];
+  const int* prow = parent_idx + ((long long)bh * np + a0 / kBlock) * K;
+  for (int i = tid; i < NC; i += kSelThreads) cand[i] = checked_index(__ldg(prow + i / kBlock), np) * kBlock + (i % kBlock);
+  // candidate rows: 16 threads copy one 256-byte row; the key of a row is computed from the
+  // parent list directly so the copies need not wait for `cand`
+  for (int i = tid; i < NC * (kD / 4); i += kSelThreads) {
+    const int r = i >> 4, piece = i & 15;
+    const int key = checked_index(__ldg(prow + r / kBlock), np) * kBlock + (r % kBlock);
+    const float4 v = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + key) * kD) + piece);
+    *reinterpret_cast<float4*>(ks + r * kSelRowStride + piece * 4) = v;
+  }
+  __syncthreads();
+
+  const int warp = tid >> 5, lane = tid & 31;
+  const float4* q0 = reinterpret_cast<const float4*>(qs + (2 * warp) * kD);
+  const float4* q1 = reinterpret_cast<const float4*>(qs + (2 * warp + 1) * kD);
+  float acc[2][CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) acc[0][j] = acc[1][j] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < kD / 4; ++i) {
+    const float4 a = q0[i], b = q1[i];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const float4 kv = reinterpret_cast<const float4*>(ks + (lane + 32 * j) * kSelRowStride)[i];
+      acc[0][j] = fmaf(a.x, kv.x, acc[0][j]);
+      acc[0][j] = fmaf(a.y, kv.y, acc[0][j]);
+      acc[0][j] = fmaf(a.z, kv.z, acc[0][j]);
+      acc[0][j] = fmaf(a.w, kv.w, acc[0][j]);
+      acc[1][j] = fmaf(b.x, kv.x, acc[1][j]);
+      acc[1][j] = fmaf(b.y, kv.y, acc[1][j]);
+      acc[1][j] = fmaf(b.z, kv.z, acc[1][j]);
+      acc[1][j] = fmaf(b.w, kv.w, acc[1][j]);
+    }
+  }
+  uint32_t key[2][CPT];
+  uint32_t bk[2] = {0u, 0u};
+  int bc[2] = {0x7fffffff, 0x7fffffff};
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      key[u][j] = score_key(acc[u][j]);
+      if (key[u][j] > bk[u]) {
+        bk[u] = key[u][j];
+        bc[u] = lane + 32 * j;
+      }
+    }
+  int win[2] = {0, 0};  // lane r < K keeps the r-th winner of each query
+#pragma unroll 1
+  for (int r = 0; r < K; ++r) {
+    uint32_t m[2];
+    int w[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) m[u] = __reduce_max_sync(0xffffffffu, bk[u]);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) w[u] = (int)__reduce_min_sync(0xffffffffu, bk[u] == m[u] ? (uint32_t)bc[u] : 0x7fffffffu);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (lane == r) win[u] = w[u];
+      if (bc[u] == w[u]) {  // the owner drops its winner and finds its next best
+        bk[u] = 0u;
+        bc[u] = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+          if (lane + 32 * j == w[u]) key[u][j] = 0u;
+          if (key[u][j] > bk[u]) {
+            bk[u] = key[u][j];
+            bc[u] = lane + 32 * j;
+          }
+        }
+      }
+    }
+  }
+  // ascending order: each winner's rank is the number of smaller winners
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    int rank = 0;
+#pragma unroll
+    for (int r2 = 0; r2 < K; ++r2) rank += __shfl_sync(0xffffffffu, win[u], r2) < win[u];
+    if (lane < K) {
+      int* orow = out_idx + ((long long)bh * n + a0 + 2 * warp + u) * K;
+      orow[rank] = cand[min(max(win[u], 0), NC - 1)];
+    }
+  }
+}
+
+inline size_t select_children_smem_bytes(int nc) {
+  return sizeof(float) * ((size_t)kBlock * kD + (size_t)nc * kSelRowStride + (size_t)nc);
+}
+
 }  // namespace llsa
