@@ -244,11 +244,12 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     # The timed region is one launch of a plan: the K steps captured into one CUDA graph
-    # (transpose on a second stream), each launch bracketed by trace events that the graph
-    # records.  The plan is built and launched once before timing (graph upload).
-    trace = api.LaunchTrace(per_step * args.steps)
-    with trace:
-        plan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=args.steps)
+    # (transpose on a second stream, kernels chained by programmatic dependent launch).
+    # The plan is built and launched once before timing (graph upload).  Per-kernel times
+    # come from a second plan of the same K steps captured with trace events around every
+    # kernel, launched after the timed region (event nodes between kernels turn the
+    # programmatic edges into full ones, so it runs slightly slower than the timed plan).
+    plan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=args.steps)
     plan.launch(stream)
     torch.cuda.synchronize()
     props = torch.cuda.get_device_properties(local)
@@ -270,6 +271,21 @@ def run_ours(args):
     status = api.llsa_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
+    plan.close()
+
+    # the traced plan: same steps, trace events recorded by the graph at every kernel
+    trace = api.LaunchTrace(per_step * args.steps)
+    with trace:
+        tplan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=args.steps)
+    tplan.launch(stream)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    t0.record(stream)
+    tplan.launch(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    traced_ms_per_step = dist_max(t0.elapsed_time(t1), world) / args.steps
 
     # per-kernel averages over the timed region
     launches = trace.launches()
@@ -320,7 +336,7 @@ def run_ours(args):
     step_roof_ms = 1000 * max(step_bytes / (hbm_peak * 1e9), step_flops / (tensor_peak * 1e12))
 
     # end to end through the public API with host buffers: a one-step plan per step
-    plan.close()
+    tplan.close()
     plan1 = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=1)
     plan1.launch(stream)
     e2e_steps = max(1, min(args.steps, 10))
@@ -391,7 +407,10 @@ def run_ours(args):
         "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
                    "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk, "kv_len": cfg.kv_len,
                    "step": "pyramid + select + forward + index transpose + backward",
-                   "launch": "K steps as one CUDA graph (llsa_plan_create repeat=K); transpose on a second stream",
+                   "launch": ("K steps as one CUDA graph (llsa_plan_create repeat=K), kernels chained by "
+                              "programmatic dependent launch; transpose on a second stream"),
+                   "kernel_times_from": ("a second plan of the same K steps with trace events around every "
+                                         f"kernel, launched after the timed one: {traced_ms_per_step:.4f} ms per step"),
                    "parallelism": f"dp{world}: independent replicas, no collective",
                    "l2": "inputs larger than L2: q, k, v, dO are 201 MB per replica vs 126 MB L2; no flush"},
         "roofline": roofline,

@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const float* __restrict__ k_pyr, const float* __restrict__ v_pyr, const int* __restrict__ idx,
     const __nv_bfloat16* __restrict__ o, const float* __restrict__ lse, __nv_bfloat16* __restrict__ dq_out,
     float* __restrict__ ws) {
+  pdl_enter();
   extern __shared__ uint8_t dq_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -344,6 +345,7 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
                                                                   const int* __restrict__ idx,
                                                                   const float* __restrict__ lse,
                                                                   float* __restrict__ ws) {
+  pdl_enter();
   extern __shared__ uint8_t co_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -435,6 +437,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
                                                                               const int* __restrict__ row_ptr,
                                                                               const int* __restrict__ col,
                                                                               float* __restrict__ ws) {
+  pdl_enter();
   __shared__ float2 red_k[kReduceWarps][32], red_v[kReduceWarps][32];
   __shared__ int slot_of[64];
   __shared__ int anc_of[64];
@@ -528,12 +531,19 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
 
 // Fine-token dK, dV.  One warp per CTA and per fine key block (flat (b*H + h) * n_1 + j), so
 // a long CSR row never holds other warps' slots.
+// coarse_late != 0: the kernel ahead of this one on the stream is coarse_grad_reduce_kernel,
+// whose output (the coarse-token gradients) only the epilogue reads; everything the main
+// loop reads was complete before that kernel could start, so the wait for it is deferred
+// to the epilogue and the main loop overlaps the reduction.
 template <int STAGES>
 __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
     const float* __restrict__ lse, const int* __restrict__ row_ptr, const int* __restrict__ col,
-    const float* __restrict__ ws, __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out) {
+    const float* __restrict__ ws, __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out,
+    int coarse_late) {
+  if (!coarse_late) pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ uint8_t dkv_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -592,6 +602,7 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
                                     },
                                     P.scale_log2, dk, dv);
   if (!ok) return;
+  if (coarse_late) pdl_wait();
   // epilogue: scale dK, add the mean-pool adjoint of the ancestors' coarse gradients
   const int c2 = 2 * (lane & 3);
 #pragma unroll

@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_bwd_dkdv_tc_kernel(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
     const float* __restrict__ lse, const int* __restrict__ row_ptr, const int* __restrict__ col,
     const float* __restrict__ ws, __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out) {
+  pdl_enter();
   extern __shared__ uint8_t tc_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -487,6 +488,7 @@ __global__ void __launch_bounds__(128) dkdv_empty_rows_kernel(AttnParams P, cons
                                                                const float* __restrict__ ws,
                                                                __nv_bfloat16* __restrict__ dk_out,
                                                                __nv_bfloat16* __restrict__ dv_out) {
+  pdl_enter();
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
   const int lane = lane_id();

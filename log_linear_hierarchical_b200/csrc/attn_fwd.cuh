@@ -223,6 +223,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
                                                             const float* __restrict__ v_pyr,
                                                             const int* __restrict__ idx, __nv_bfloat16* __restrict__ o,
                                                             float* __restrict__ lse) {
+  pdl_enter();
   extern __shared__ uint8_t fwd_smem_raw[];
   const Geometry& g = P.g;
   const int lane = lane_id();

@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
                                                                     const float* __restrict__ v_pyr,
                                                                     const int* __restrict__ idx, float* __restrict__ o,
                                                                     float* __restrict__ lse) {
+  pdl_enter();
   extern __shared__ __align__(16) uint8_t simt_smem[];
   const int T = kBlock * g.K + g.coarse;
   const int gb = blockIdx.x;
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
     const float* __restrict__ o, const float* __restrict__ lse, const float* __restrict__ dO,
     const float* __restrict__ k_pyr, const float* __restrict__ v_pyr, const int* __restrict__ idx,
     float* __restrict__ dq_out, float* __restrict__ ws) {
+  pdl_enter();
   extern __shared__ __align__(16) uint8_t simt_smem[];
   const BwdWorkspace W = bwd_workspace_layout(g);
   const int T = kBlock * g.K + g.coarse;
@@ -212,6 +214,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
     const float* __restrict__ lse, const float* __restrict__ dO, const int* __restrict__ row_ptr,
     const int* __restrict__ col, const float* __restrict__ ws, float* __restrict__ dk_out,
     float* __restrict__ dv_out) {
+  pdl_enter();
   __shared__ float ks[kBlock * kD], vs[kBlock * kD], qs[kBlock * kD], dos[kBlock * kD];
   __shared__ float Pt[kBlock][kBlock + 1], dSt[kBlock][kBlock + 1];
   __shared__ float ls[kBlock], dl[kBlock];

@@ -152,6 +152,24 @@ bool allow_smem(Kern k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
 }
 
+// Launch with programmatic stream serialization (see pdl_wait): the kernel may be scheduled
+// while the one ahead of it on the stream drains; it waits for it on the device.  A failed
+// launch is reported by cudaGetLastError, as for a triple-chevron launch.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t cs, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = cs;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------- launch trace
 enum KernelId {
   kKPyramidL12 = 1,
@@ -222,7 +240,7 @@ llsa_status launch_coarse_reduce(const Geometry& g, float scale, const int32_t* 
   long long tokens = 0;
   for (int l = 2; l <= g.L; ++l) tokens += (long long)g.BH * g.n[l];
   return launch(kKBwdCoarseReduce, cs, [&] {
-    coarse_grad_reduce_kernel<<<(unsigned)tokens, kReduceWarps * 32, 0, cs>>>(g, scale, idx, row_ptr, col, ws);
+    launch_pdl(coarse_grad_reduce_kernel, dim3((unsigned)tokens), dim3(kReduceWarps * 32), 0, cs, g, scale, idx, row_ptr, col, ws);
   });
 }
 
@@ -279,7 +297,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
       if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
       const int per_cta = kAttnWarps * kUnitBlocks;
       st = launch(kKBwdDqBf16, cs, [&] {
-        kern<<<(total_blocks + per_cta - 1) / per_cta, 32 * kAttnWarps, smem, cs>>>(
+        launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, 
             tq, tk, tv, tdo, P, k_pyr, v_pyr, idx, static_cast<const __nv_bfloat16*>(o), lse,
             static_cast<__nv_bfloat16*>(dq), ws);
       });
@@ -289,7 +307,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
         if (!allow_smem(ckern, kv_bytes)) return LLSA_ERR_CUDA;
         const int ctas = g.BH * g.n[2] * (g.coarse_pad / kBlock);
         st = launch(kKBwdCoarseBf16, cs, [&] {
-          ckern<<<ctas, 32, kv_bytes, cs>>>(tq, tdo, P, k_pyr, v_pyr, idx, lse, ws);
+          launch_pdl(ckern, dim3(ctas), dim3(32), kv_bytes, cs, tq, tdo, P, k_pyr, v_pyr, idx, lse, ws);
         });
         if (st != LLSA_OK) return st;
       }
@@ -305,12 +323,12 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
       if (!allow_smem(attn_bwd_dkdv_tc_kernel, kTcSmemBytes)) return LLSA_ERR_CUDA;
       const int grid = total_blocks < 2 * sms ? total_blocks : 2 * sms;
       st = launch(kKBwdDkdvEmpty, cs, [&] {
-        dkdv_empty_rows_kernel<<<(total_blocks + 3) / 4, 128, 0, cs>>>(P, row_ptr, ws, static_cast<__nv_bfloat16*>(dk),
+        launch_pdl(dkdv_empty_rows_kernel, dim3((total_blocks + 3) / 4), dim3(128), 0, cs, P, row_ptr, ws, static_cast<__nv_bfloat16*>(dk),
                                                                       static_cast<__nv_bfloat16*>(dv));
       });
       if (st != LLSA_OK) return st;
       return launch(kKBwdDkdvTc, cs, [&] {
-        attn_bwd_dkdv_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, cs>>>(
+        launch_pdl(attn_bwd_dkdv_tc_kernel, dim3(grid), dim3(kTcThreads), kTcSmemBytes, cs, 
             tq, tk, tv, tdo, P, lse, row_ptr, col, ws, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
       });
     }
@@ -318,8 +336,8 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
     auto kern = attn_bwd_dkdv_bf16_kernel<kDkvStages>;
     if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
     return launch(kKBwdDkdvBf16, cs, [&] {
-      kern<<<total_blocks, 32, kv_bytes, cs>>>(tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
-                                                static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+      launch_pdl(kern, dim3(total_blocks), dim3(32), kv_bytes, cs, tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
+                 static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), g.L >= 2 ? 1 : 0);
     });
   }
   if (phases & kQuerySide) {
@@ -327,7 +345,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
     if (!allow_smem(attn_bwd_dq_f32_kernel, smem)) return LLSA_ERR_CUDA;
     const int per_cta = g.L >= 2 ? kBlock : 1;
     st = launch(kKBwdDqF32, cs, [&] {
-      attn_bwd_dq_f32_kernel<<<total_blocks / per_cta, kSimtThreads, smem, cs>>>(
+      launch_pdl(attn_bwd_dq_f32_kernel, dim3(total_blocks / per_cta), dim3(kSimtThreads), smem, cs, 
           g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
           static_cast<const float*>(o), lse, static_cast<const float*>(dO), k_pyr, v_pyr, idx,
           static_cast<float*>(dq), ws);
@@ -337,7 +355,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
   if (!(phases & kKeySide)) return LLSA_OK;
   if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
   return launch(kKBwdDkdvF32, cs, [&] {
-    attn_bwd_dkdv_f32_kernel<<<total_blocks, kSimtThreads, 0, cs>>>(
+    launch_pdl(attn_bwd_dkdv_f32_kernel, dim3(total_blocks), dim3(kSimtThreads), 0, cs, 
         g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), lse,
         static_cast<const float*>(dO), row_ptr, col, ws, static_cast<float*>(dk), static_cast<float*>(dv));
   });
@@ -466,7 +484,7 @@ llsa_status llsa_build_pyramid(const llsa_shape* s, const void* q, const void* k
     constexpr int rows = kPyrThreads / (kD / 8);
     dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
     st = launch(kKPyramidL12, cs, [&] {
-      pyramid_l12_kernel<__nv_bfloat16><<<grid, kPyrThreads, 0, cs>>>(
+      launch_pdl(pyramid_l12_kernel<__nv_bfloat16>, dim3(grid), dim3(kPyrThreads), 0, cs, 
           g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
           static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr);
     });
@@ -474,7 +492,7 @@ llsa_status llsa_build_pyramid(const llsa_shape* s, const void* q, const void* k
     constexpr int rows = kPyrThreads / (kD / 4);
     dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
     st = launch(kKPyramidL12, cs, [&] {
-      pyramid_l12_kernel<float><<<grid, kPyrThreads, 0, cs>>>(g, static_cast<const float*>(q),
+      launch_pdl(pyramid_l12_kernel<float>, dim3(grid), dim3(kPyrThreads), 0, cs, g, static_cast<const float*>(q),
                                                                static_cast<const float*>(k),
                                                                static_cast<const float*>(v), q_pyr, k_pyr, v_pyr);
     });
@@ -483,7 +501,7 @@ llsa_status llsa_build_pyramid(const llsa_shape* s, const void* q, const void* k
   for (int l = 3; l <= g.L; ++l) {
     const long long total = (long long)g.BH * g.n[l] * kD;
     dim3 grid((unsigned)((total + kPyrThreads - 1) / kPyrThreads), 3);
-    st = launch(kKPyramidUp, cs, [&] { pyramid_up_kernel<<<grid, kPyrThreads, 0, cs>>>(g, l, q_pyr, k_pyr, v_pyr); });
+    st = launch(kKPyramidUp, cs, [&] { launch_pdl(pyramid_up_kernel, dim3(grid), dim3(kPyrThreads), 0, cs, g, l, q_pyr, k_pyr, v_pyr); });
     if (st != LLSA_OK) return st;
   }
   return LLSA_OK;
@@ -519,7 +537,7 @@ llsa_status llsa_select(const llsa_shape* s, const float* q_pyr, const float* k_
       const unsigned grid = (unsigned)(g.BH * (n / kBlock));
       auto run = [&](auto kern) -> llsa_status {
         if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
-        return launch(kKSelect, cs, [&] { kern<<<grid, kSelThreads, smem, cs>>>(g, l, qpl, kpl, par, out); });
+        return launch(kKSelect, cs, [&] { launch_pdl(kern, dim3(grid), dim3(kSelThreads), smem, cs, g, l, qpl, kpl, par, out); });
       };
       switch (g.K) {
         case 2: st = run(select_children_kernel<1>); break;
@@ -534,7 +552,7 @@ llsa_status llsa_select(const llsa_shape* s, const float* q_pyr, const float* k_
     if (!allow_smem(select_kernel, smem)) return LLSA_ERR_CUDA;
     const int groups = (n + gq - 1) / gq;
     st = launch(kKSelect, cs, [&] {
-      select_kernel<<<g.BH * groups, kSelThreads, smem, cs>>>(g, l, gq, q_pyr + g.pyr_off[l], k_pyr + g.pyr_off[l],
+      launch_pdl(select_kernel, dim3(g.BH * groups), dim3(kSelThreads), smem, cs, g, l, gq, q_pyr + g.pyr_off[l], k_pyr + g.pyr_off[l],
                                                              sparse ? idx + g.idx_off[l + 1] : nullptr,
                                                              idx + g.idx_off[l]);
     });
@@ -561,13 +579,13 @@ llsa_status llsa_index_transpose(const llsa_shape* s, const int32_t* idx, int32_
   const int bucket_ctas = last.cta_buckets + g.BH * last.nb;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   st = launch(kKTransposeHist, cs,
-              [&] { transpose_hist_kernel<<<tile_ctas, kTrThreads, 0, cs>>>(tg, idx, ws_hist); });
+              [&] { launch_pdl(transpose_hist_kernel, dim3(tile_ctas), dim3(kTrThreads), 0, cs, tg, idx, ws_hist); });
   if (st != LLSA_OK) return st;
   st = launch(kKTransposeScatter, cs,
-              [&] { transpose_scatter_kernel<<<tile_ctas, kTrThreads, 0, cs>>>(tg, idx, ws_hist, ws_ent); });
+              [&] { launch_pdl(transpose_scatter_kernel, dim3(tile_ctas), dim3(kTrThreads), 0, cs, tg, idx, ws_hist, ws_ent); });
   if (st != LLSA_OK) return st;
   return launch(kKTransposeBucket, cs, [&] {
-    transpose_bucket_kernel<<<bucket_ctas, kTrThreads, 0, cs>>>(tg, ws_ent, ws_hist, row_ptr, col);
+    launch_pdl(transpose_bucket_kernel, dim3(bucket_ctas), dim3(kTrThreads), 0, cs, tg, ws_ent, ws_hist, row_ptr, col);
   });
 }
 
@@ -605,14 +623,14 @@ llsa_status llsa_forward(const llsa_shape* s, const void* q, const void* k, cons
     if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
     const int per_cta = kAttnWarps * kUnitBlocks;
     return launch(kKFwdBf16, cs, [&] {
-      kern<<<(total_blocks + per_cta - 1) / per_cta, 32 * kAttnWarps, smem, cs>>>(
+      launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, 
           tq, tk, tv, P, k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse);
     });
   }
   const size_t smem = simt_fwd_smem(g);
   if (!allow_smem(attn_fwd_f32_kernel, smem)) return LLSA_ERR_CUDA;
   return launch(kKFwdF32, cs, [&] {
-    attn_fwd_f32_kernel<<<total_blocks, kSimtThreads, smem, cs>>>(
+    launch_pdl(attn_fwd_f32_kernel, dim3(total_blocks), dim3(kSimtThreads), smem, cs, 
         g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
         v_pyr, idx, static_cast<float*>(o), lse);
   });

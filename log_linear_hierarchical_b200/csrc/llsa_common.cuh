@@ -143,6 +143,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Programmatic dependent launch.  Every kernel is launched with programmatic stream
+// serialization, so it may be scheduled before the kernel ahead of it on the stream has
+// finished.  pdl_wait blocks until that kernel has completed and its writes are visible
+// (it returns at once for a kernel launched without the attribute); no kernel touches
+// global memory before it, unless the kernel documents what it reads early.
+// pdl_launch_dependents lets the next kernel's CTAs be scheduled once every CTA of this
+// grid has issued it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_launch_dependents();
+}
+
 // Non-blocking test of the phase with the given parity (no suspend hint), for a thread that
 // polls several barriers.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {

@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(kPyrThreads) pyramid_l12_kernel(Geometry g, co
                                                                   const T* __restrict__ x1,
                                                                   const T* __restrict__ x2, float* __restrict__ p0,
                                                                   float* __restrict__ p1, float* __restrict__ p2) {
+  pdl_enter();
   constexpr int VE = Vec16<T>::kElems;
   constexpr int TPR = kD / VE;                   // threads per row
   constexpr int ROWS = kPyrThreads / TPR;         // level-1 rows per CTA (32 for bf16, 16 for fp32)
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kPyrThreads) pyramid_l12_kernel(Geometry g, co
 // Level l >= 3 from level l-1 (fp32).  One thread per output value; grid.y = tensor.
 __global__ void __launch_bounds__(kPyrThreads) pyramid_up_kernel(Geometry g, int level, float* __restrict__ p0,
                                                                  float* __restrict__ p1, float* __restrict__ p2) {
+  pdl_enter();
   float* pyr = blockIdx.y == 0 ? p0 : (blockIdx.y == 1 ? p1 : p2);
   const long long total = (long long)g.BH * g.n[level] * kD;
   const long long i = (long long)blockIdx.x * kPyrThreads + threadIdx.x;

@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
                                                              const float* __restrict__ kp,
                                                              const int* __restrict__ parent_idx,
                                                              int* __restrict__ out_idx) {
+  pdl_enter();
   extern __shared__ __align__(16) float sel_smem[];
   const int n = g.n[level];
   const int K = g.K;
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g
                                                                       const float* __restrict__ kp,
                                                                       const int* __restrict__ parent_idx,
                                                                       int* __restrict__ out_idx) {
+  pdl_enter();
   constexpr int NC = 32 * CPT;
   constexpr int K = 2 * CPT;  // NC = 16 K
   extern __shared__ __align__(16) float sel_smem[];

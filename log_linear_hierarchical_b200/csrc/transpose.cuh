@@ -86,6 +86,7 @@ __device__ __forceinline__ void tr_warp_bucket_counts(const int* __restrict__ ke
 
 __global__ void __launch_bounds__(kTrThreads) transpose_hist_kernel(TransposeGeo tg, const int* __restrict__ idx,
                                                                     int* __restrict__ ws_hist) {
+  pdl_enter();
   __shared__ int cnt[kTrWarps][kTrMaxBuckets];
   const int l = tr_level_of(tg, blockIdx.x, false);
   const TransposeLevel& L = tg.lv[l];
@@ -131,6 +132,7 @@ __device__ __forceinline__ void tr_scan64(int* vals, int count, int* total_out) 
 __global__ void __launch_bounds__(kTrThreads) transpose_scatter_kernel(TransposeGeo tg, const int* __restrict__ idx,
                                                                        const int* __restrict__ ws_hist,
                                                                        uint32_t* __restrict__ ws_ent) {
+  pdl_enter();
   __shared__ int cnt[kTrWarps][kTrMaxBuckets];
   __shared__ int tot[kTrMaxBuckets];
   __shared__ int pre[kTrMaxBuckets];
@@ -194,6 +196,7 @@ __global__ void __launch_bounds__(kTrThreads) transpose_scatter_kernel(Transpose
 __global__ void __launch_bounds__(kTrThreads) transpose_bucket_kernel(TransposeGeo tg, const uint32_t* __restrict__ ws_ent,
                                                                       const int* __restrict__ ws_hist,
                                                                       int* __restrict__ row_ptr, int* __restrict__ col) {
+  pdl_enter();
   __shared__ int kc[kTrWarps][kTrMaxBucketKeys];
   __shared__ int kpre[kTrMaxBucketKeys];
   __shared__ int part[kTrThreads];

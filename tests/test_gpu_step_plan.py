@@ -115,3 +115,27 @@ def test_plan_is_traced_at_every_launch():
     assert [n for n, _ in times] == [n for n, _ in eager.launches()] * 3
     assert all(ms > 0 for _, ms in times)
     plan.close()
+
+
+def test_plan_headline_matches_serialized_calls():
+    """Full headline size: the plan (kernels chained by programmatic dependent launch, dK/dV
+    overlapping the coarse reduction) against the five calls run with trace events between
+    every kernel, which serialises them; bit for bit over three replays."""
+    cfg = CONFIGS[4]
+    inputs = make_config_inputs(cfg)
+    shape, dev, buf = setup(cfg, inputs)
+    with api.LaunchTrace(64):
+        api.llsa_forward_path(shape, dev["q"], dev["k"], dev["v"], buf)
+        api.llsa_backward_path(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+    torch.cuda.synchronize()
+    assert api.llsa_device_status() == 0
+    ref = outputs(buf)
+    plan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=3)
+    for _ in range(3):
+        for t in (buf.o, buf.lse, buf.dq, buf.dk, buf.dv, buf.ws_backward, buf.row_ptr, buf.col):
+            t.fill_(7)
+        plan.launch()
+        torch.cuda.synchronize()
+        assert api.llsa_device_status() == 0
+        assert_same(outputs(buf), ref)
+    plan.close()
