@@ -31,8 +31,21 @@ struct BwdWorkspace {
   long long part_k, part_v; // [B*H*n_2][C][64]
   long long cg_k, cg_v;     // coarse gradients, level-major [l=2..L][B*H*n_l][64]
   long long cg_off[kMaxLevels + 1];
+  long long order;          // int32 [B*H*n_1]: fine key blocks, longest CSR row first
+  long long order_counts;   // int32 [kOrdClasses][order tiles]
   long long total;
 };
+
+// Longest-first order of the fine key blocks for the key-major dK/dV kernel: its CTAs are
+// scheduled roughly in launch order, and a row of up to ~150 query blocks started last would
+// run alone long after the rest.  Rows are grouped into classes by floor(log2(length))
+// (class 0: >= 128 query blocks, ..., class 7: one, class 8: empty), stable within a class.
+constexpr int kOrdClasses = 9;
+constexpr int kOrdThreads = 256;
+constexpr int kOrdRowsPerThread = 8;
+constexpr int kOrdTile = kOrdThreads * kOrdRowsPerThread;
+
+__host__ __device__ inline int order_tiles(const Geometry& g) { return (g.BH * g.n[1] + kOrdTile - 1) / kOrdTile; }
 
 __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) {
   auto up = [](long long x) { return (x + 63) & ~63LL; };
@@ -55,6 +68,10 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   off = up(off + cg);
   w.cg_v = off;
   off = up(off + cg);
+  w.order = off;
+  off = up(off + (long long)g.BH * g.n[1]);
+  w.order_counts = off;
+  off = up(off + (long long)kOrdClasses * order_tiles(g));
   w.total = off;
   return w;
 }
@@ -529,6 +546,128 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
   }
 }
 
+// ---------------------------------------------------------------------------- dK/dV order
+
+__device__ __forceinline__ int order_class(int len) {
+  return len <= 0 ? kOrdClasses - 1 : 7 - min(31 - __clz(len), 7);
+}
+
+// Length of flat level-1 row kb = bh * n_1 + j (0 for kb past the end).
+__device__ __forceinline__ int order_row_len(const Geometry& g, const int* __restrict__ rp1, int kb) {
+  if (kb >= g.BH * g.n[1]) return 0;
+  const int* r = rp1 + (long long)(kb >> g.log_n1) * (g.n[1] + 1) + (kb & (g.n[1] - 1));
+  return __ldg(r + 1) - __ldg(r);
+}
+
+// Per tile of kOrdTile rows: the number of rows of each class (counts[c * tiles + tile]).
+__global__ void __launch_bounds__(kOrdThreads) dkdv_order_count_kernel(Geometry g, const int* __restrict__ row_ptr,
+                                                                       float* __restrict__ ws) {
+  pdl_enter();
+  __shared__ int part[kOrdThreads / 32][kOrdClasses];
+  const BwdWorkspace W = bwd_workspace_layout(g);
+  const int* rp1 = row_ptr + g.rp_off[1];
+  const int row0 = blockIdx.x * kOrdTile + threadIdx.x * kOrdRowsPerThread;
+  int cnt[kOrdClasses];
+#pragma unroll
+  for (int c = 0; c < kOrdClasses; ++c) cnt[c] = 0;
+  for (int i = 0; i < kOrdRowsPerThread; ++i) {
+    if (row0 + i >= g.BH * g.n[1]) break;
+    const int c = order_class(order_row_len(g, rp1, row0 + i));
+#pragma unroll
+    for (int cc = 0; cc < kOrdClasses; ++cc) cnt[cc] += (cc == c);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < kOrdClasses; ++c) {
+    int v = cnt[c];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) part[warp][c] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < kOrdClasses) {
+    int v = 0;
+    for (int w = 0; w < kOrdThreads / 32; ++w) v += part[w][threadIdx.x];
+    reinterpret_cast<int*>(ws + W.order_counts)[threadIdx.x * order_tiles(g) + blockIdx.x] = v;
+  }
+}
+
+// Writes order[pos] = kb: class by class, tiles in order, rows in order within a tile.
+__global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometry g, const int* __restrict__ row_ptr,
+                                                                         float* __restrict__ ws) {
+  pdl_enter();
+  __shared__ int start[kOrdClasses];
+  __shared__ int wsum[kOrdThreads / 32][kOrdClasses];
+  const BwdWorkspace W = bwd_workspace_layout(g);
+  const int tiles = order_tiles(g);
+  const int* counts = reinterpret_cast<const int*>(ws + W.order_counts);
+  if (threadIdx.x < 32) {
+    // start of (class c, this tile) = rows of lower classes + rows of class c in earlier tiles
+    const int lane = threadIdx.x;
+    int before = 0, mine = 0;
+    for (int c = 0; c < kOrdClasses; ++c) {
+      int tot = 0, pre = 0;
+      for (int t = lane; t < tiles; t += 32) {
+        const int v = counts[c * tiles + t];
+        tot += v;
+        if (t < (int)blockIdx.x) pre += v;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        tot += __shfl_xor_sync(0xffffffffu, tot, off);
+        pre += __shfl_xor_sync(0xffffffffu, pre, off);
+      }
+      if (lane == c) mine = before + pre;
+      before += tot;
+    }
+    if (lane < kOrdClasses) start[lane] = mine;
+  }
+  const int* rp1 = row_ptr + g.rp_off[1];
+  const int row0 = blockIdx.x * kOrdTile + threadIdx.x * kOrdRowsPerThread;
+  int cls[kOrdRowsPerThread];
+  int cnt[kOrdClasses];
+#pragma unroll
+  for (int c = 0; c < kOrdClasses; ++c) cnt[c] = 0;
+#pragma unroll
+  for (int i = 0; i < kOrdRowsPerThread; ++i) {
+    cls[i] = row0 + i < g.BH * g.n[1] ? order_class(order_row_len(g, rp1, row0 + i)) : -1;
+#pragma unroll
+    for (int cc = 0; cc < kOrdClasses; ++cc) cnt[cc] += (cc == cls[i]);
+  }
+  // exclusive scan of the per-thread counts over the CTA, class by class
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int pre[kOrdClasses];
+#pragma unroll
+  for (int c = 0; c < kOrdClasses; ++c) {
+    int v = cnt[c];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += o;
+    }
+    pre[c] = v - cnt[c];
+    if (lane == 31) wsum[warp][c] = v;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < kOrdClasses; ++c) {
+    int base = start[c];
+    for (int w = 0; w < warp; ++w) base += wsum[w][c];
+    pre[c] += base;
+  }
+  int* order = reinterpret_cast<int*>(ws + W.order);
+#pragma unroll
+  for (int i = 0; i < kOrdRowsPerThread; ++i) {
+    const int c = cls[i];
+    if (c < 0) continue;
+    int pos = 0;
+#pragma unroll
+    for (int cc = 0; cc < kOrdClasses; ++cc)
+      if (cc == c) pos = pre[cc]++;
+    order[pos] = row0 + i;
+  }
+}
+
 // Fine-token dK, dV.  One warp per CTA and per fine key block (flat (b*H + h) * n_1 + j), so
 // a long CSR row never holds other warps' slots.
 // coarse_late != 0: the kernel ahead of this one on the stream is coarse_grad_reduce_kernel,
@@ -550,7 +689,9 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   const int lane = lane_id();
   const int n1 = g.n[1];
   const int K = g.K;
-  const int kb = blockIdx.x;
+  // key blocks are taken longest row first (dkdv_order_*_kernel, complete before this
+  // kernel's predecessor started)
+  const int kb = checked_index(__ldg(reinterpret_cast<const int*>(ws + W.order) + blockIdx.x), g.BH * n1);
   const int bh = kb / n1;
   const int j = kb - bh * n1;
   const CtaSmem cs = kv_smem<STAGES>(1);

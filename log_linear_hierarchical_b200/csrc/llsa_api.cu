@@ -188,13 +188,16 @@ enum KernelId {
   kKBwdCoarseBf16,
   kKBwdDkdvTc,
   kKBwdDkdvEmpty,
+  kKDkdvOrderCount,
+  kKDkdvOrderScatter,
   kKNumKernels
 };
 
 const char* const kKernelNames[kKNumKernels] = {
     "unknown",          "pyramid_l12",          "pyramid_up",   "select",           "transpose_hist",
     "transpose_scatter", "transpose_bucket",    "attn_fwd_bf16", "attn_bwd_dq_bf16", "coarse_grad_reduce",
-    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32", "attn_bwd_coarse_bf16", "attn_bwd_dkdv_tc", "dkdv_empty_rows"};
+    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32", "attn_bwd_coarse_bf16", "attn_bwd_dkdv_tc", "dkdv_empty_rows",
+    "dkdv_order_count", "dkdv_order_scatter"};
 
 struct TraceState {
   cudaEvent_t* ev = nullptr;
@@ -272,7 +275,9 @@ namespace {
 // reads only the query-major selection; the key side (coarse-token gradients reduced
 // through the level-l CSRs, then dK/dV through the level-1 CSR) needs the transpose, so a
 // step can run the transpose concurrently with the forward and the query side.
-constexpr unsigned kQuerySide = 1, kKeySide = 2;
+// A third phase, the longest-first order of the fine key blocks for dK/dV, reads only the
+// level-1 CSR and can run beside the query side too.
+constexpr unsigned kQuerySide = 1, kKeySide = 2, kOrder = 4;
 
 llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
                             const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
@@ -283,6 +288,15 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
   float* ws = static_cast<float*>(workspace);
   const float scale = 1.0f / sqrtf((float)kD);
   const int total_blocks = g.BH * g.n[1];
+  if ((phases & kOrder) && s->dtype == LLSA_BF16 && !LLSA_KEY_MAJOR_TC) {
+    const int tiles = order_tiles(g);
+    st = launch(kKDkdvOrderCount, cs,
+                [&] { launch_pdl(dkdv_order_count_kernel, dim3(tiles), dim3(kOrdThreads), 0, cs, g, row_ptr, ws); });
+    if (st != LLSA_OK) return st;
+    st = launch(kKDkdvOrderScatter, cs,
+                [&] { launch_pdl(dkdv_order_scatter_kernel, dim3(tiles), dim3(kOrdThreads), 0, cs, g, row_ptr, ws); });
+    if (st != LLSA_OK) return st;
+  }
   if (s->dtype == LLSA_BF16) {
     CUtensorMap tq, tk, tv, tdo;
     const long long rows = (long long)g.BH * g.N;
@@ -400,6 +414,9 @@ llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStrea
     if (st == LLSA_OK)
       st = llsa_index_transpose(s, b->idx, b->row_ptr, b->col, b->transpose_workspace, b->transpose_workspace_bytes,
                                 side);
+    if (st == LLSA_OK)
+      st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
+                           b->dq, b->dk, b->dv, b->backward_workspace, kOrder, side);
     if (cudaEventRecord(join, side) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
   }
   if (st == LLSA_OK) st = llsa_forward(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs);
@@ -412,6 +429,9 @@ llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStrea
     cudaEventDestroy(join);
   } else if (st == LLSA_OK) {
     st = llsa_index_transpose(s, b->idx, b->row_ptr, b->col, b->transpose_workspace, b->transpose_workspace_bytes, cs);
+    if (st == LLSA_OK)
+      st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
+                           b->dq, b->dk, b->dv, b->backward_workspace, kOrder, cs);
   }
   if (st == LLSA_OK)
     st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
@@ -647,7 +667,7 @@ llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, con
     if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
   if (workspace_bytes < (size_t)bwd_workspace_layout(make_geometry(s)).total * sizeof(float)) return LLSA_ERR_WORKSPACE;
   return backward_phases(s, q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace,
-                         kQuerySide | kKeySide, reinterpret_cast<cudaStream_t>(stream));
+                         kOrder | kQuerySide | kKeySide, reinterpret_cast<cudaStream_t>(stream));
 }
 
 llsa_status llsa_train_step(const llsa_shape* s, const llsa_step_buffers* b, llsa_stream_t stream,
