@@ -376,6 +376,102 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
 }
 
 
+// ---------------------------------------------------------------------------- pyramid, select
+// Levels 1-2 of the pyramid, and levels 3..L too when `upper`.
+llsa_status pyramid_launch(const Geometry& g, int dtype, const void* q, const void* k, const void* v, float* q_pyr,
+                           float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs) {
+  llsa_status st;
+  if (dtype == LLSA_BF16) {
+    constexpr int rows = kPyrThreads / (kD / 8);
+    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
+    st = launch(kKPyramidL12, cs, [&] {
+      launch_pdl(pyramid_l12_kernel<__nv_bfloat16>, dim3(grid), dim3(kPyrThreads), 0, cs, g,
+                 static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                 static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr);
+    });
+  } else {
+    constexpr int rows = kPyrThreads / (kD / 4);
+    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
+    st = launch(kKPyramidL12, cs, [&] {
+      launch_pdl(pyramid_l12_kernel<float>, dim3(grid), dim3(kPyrThreads), 0, cs, g, static_cast<const float*>(q),
+                 static_cast<const float*>(k), static_cast<const float*>(v), q_pyr, k_pyr, v_pyr);
+    });
+  }
+  if (st != LLSA_OK || !upper) return st;
+  for (int l = 3; l <= g.L; ++l) {
+    const long long total = (long long)g.BH * g.n[l] * kD;
+    dim3 grid((unsigned)((total + kPyrThreads - 1) / kPyrThreads), 3);
+    st = launch(kKPyramidUp, cs,
+                [&] { launch_pdl(pyramid_up_kernel, dim3(grid), dim3(kPyrThreads), 0, cs, g, l, q_pyr, k_pyr, v_pyr); });
+    if (st != LLSA_OK) return st;
+  }
+  return LLSA_OK;
+}
+
+// The pooled levels 3..L and the coarsest selection fit one small kernel per (b, h).
+bool small_top(const Geometry& g) { return g.n[g.L] <= kTopMaxN && g.K <= 32 && (g.L < 3 || g.n[3] <= kTopMaxN); }
+
+// Selection of every level, coarsest first.  With `pool_top` (only when small_top), the
+// coarsest launch also pools levels 3..L (pyramid_launch was made with upper = false);
+// v_pyr is needed only then.
+llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* v_pyr, int32_t* idx, bool pool_top,
+                          cudaStream_t cs) {
+  llsa_status st;
+  for (int l = g.L; l >= 1; --l) {
+    const bool sparse = l < g.L;
+    const int n = g.n[l];
+    if (!sparse && small_top(g)) {
+      st = launch(kKSelect, cs, [&] {
+        if (pool_top)
+          launch_pdl(coarsest_small_kernel<true>, dim3(g.BH), dim3(kTopThreads), 0, cs, g, q_pyr, k_pyr, v_pyr, idx);
+        else
+          launch_pdl(coarsest_small_kernel<false>, dim3(g.BH), dim3(kTopThreads), 0, cs, g, q_pyr, k_pyr, v_pyr, idx);
+      });
+      if (st != LLSA_OK) return st;
+      continue;
+    }
+    int gq, nc;
+    if (sparse) {
+      gq = kBlock;
+      nc = kBlock * g.K;
+    } else {
+      nc = n;
+      gq = kBlock;
+      while (gq > 1 && (gq > n || (long long)gq * n > 16384)) gq >>= 1;
+    }
+    if (sparse && g.K >= 2 && g.K <= 16) {
+      // children of the parent's K keys scored in registers (select_children_kernel)
+      const size_t smem = select_children_smem_bytes(nc);
+      const float* qpl = q_pyr + g.pyr_off[l];
+      const float* kpl = k_pyr + g.pyr_off[l];
+      const int* par = idx + g.idx_off[l + 1];
+      int* out = idx + g.idx_off[l];
+      const unsigned grid = (unsigned)(g.BH * (n / kBlock));
+      auto run = [&](auto kern) -> llsa_status {
+        if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+        return launch(kKSelect, cs, [&] { launch_pdl(kern, dim3(grid), dim3(kSelThreads), smem, cs, g, l, qpl, kpl, par, out); });
+      };
+      switch (g.K) {
+        case 2: st = run(select_children_kernel<1>); break;
+        case 4: st = run(select_children_kernel<2>); break;
+        case 8: st = run(select_children_kernel<4>); break;
+        default: st = run(select_children_kernel<8>); break;
+      }
+      if (st != LLSA_OK) return st;
+      continue;
+    }
+    const size_t smem = select_smem_bytes(gq, nc, g.K, sparse);
+    if (!allow_smem(select_kernel, smem)) return LLSA_ERR_CUDA;
+    const int groups = (n + gq - 1) / gq;
+    st = launch(kKSelect, cs, [&] {
+      launch_pdl(select_kernel, dim3(g.BH * groups), dim3(kSelThreads), smem, cs, g, l, gq, q_pyr + g.pyr_off[l],
+                 k_pyr + g.pyr_off[l], sparse ? idx + g.idx_off[l + 1] : nullptr, idx + g.idx_off[l]);
+    });
+    if (st != LLSA_OK) return st;
+  }
+  return LLSA_OK;
+}
+
 // ---------------------------------------------------------------------------- one step
 // Host-side checks of a step's buffers (the per-call checks, done up front so that a
 // rejected step launches nothing).
@@ -399,8 +495,11 @@ llsa_status validate_step(const llsa_shape* s, const llsa_step_buffers* b) {
 // is null.  The join is made on every path once the fork was made, so a capture that
 // fails part-way still ends with both streams joined.
 llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStream_t cs, cudaStream_t side) {
-  llsa_status st = llsa_build_pyramid(s, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, cs);
-  if (st == LLSA_OK) st = llsa_select(s, b->q_pyr, b->k_pyr, b->idx, cs);
+  // pooled levels >= 3 are made by the coarsest-selection launch when they are small
+  const Geometry g = make_geometry(s);
+  const bool fuse_top = g.L >= 3 && small_top(g);
+  llsa_status st = pyramid_launch(g, s->dtype, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, !fuse_top, cs);
+  if (st == LLSA_OK) st = select_launch(g, b->q_pyr, b->k_pyr, b->v_pyr, b->idx, fuse_top, cs);
   if (st != LLSA_OK) return st;
   cudaEvent_t fork = nullptr, join = nullptr;
   if (side) {
@@ -498,33 +597,8 @@ llsa_status llsa_build_pyramid(const llsa_shape* s, const void* q, const void* k
   const void* ptrs[6] = {q, k, v, q_pyr, k_pyr, v_pyr};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
-  const Geometry g = make_geometry(s);
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (s->dtype == LLSA_BF16) {
-    constexpr int rows = kPyrThreads / (kD / 8);
-    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
-    st = launch(kKPyramidL12, cs, [&] {
-      launch_pdl(pyramid_l12_kernel<__nv_bfloat16>, dim3(grid), dim3(kPyrThreads), 0, cs, 
-          g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-          static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr);
-    });
-  } else {
-    constexpr int rows = kPyrThreads / (kD / 4);
-    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
-    st = launch(kKPyramidL12, cs, [&] {
-      launch_pdl(pyramid_l12_kernel<float>, dim3(grid), dim3(kPyrThreads), 0, cs, g, static_cast<const float*>(q),
-                                                               static_cast<const float*>(k),
-                                                               static_cast<const float*>(v), q_pyr, k_pyr, v_pyr);
-    });
-  }
-  if (st != LLSA_OK) return st;
-  for (int l = 3; l <= g.L; ++l) {
-    const long long total = (long long)g.BH * g.n[l] * kD;
-    dim3 grid((unsigned)((total + kPyrThreads - 1) / kPyrThreads), 3);
-    st = launch(kKPyramidUp, cs, [&] { launch_pdl(pyramid_up_kernel, dim3(grid), dim3(kPyrThreads), 0, cs, g, l, q_pyr, k_pyr, v_pyr); });
-    if (st != LLSA_OK) return st;
-  }
-  return LLSA_OK;
+  return pyramid_launch(make_geometry(s), s->dtype, q, k, v, q_pyr, k_pyr, v_pyr, true,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 llsa_status llsa_select(const llsa_shape* s, const float* q_pyr, const float* k_pyr, int32_t* idx,
@@ -533,52 +607,8 @@ llsa_status llsa_select(const llsa_shape* s, const float* q_pyr, const float* k_
   if (st != LLSA_OK) return st;
   if (!q_pyr || !k_pyr || !idx || !aligned16(q_pyr) || !aligned16(k_pyr) || !aligned16(idx))
     return LLSA_ERR_INVALID_ARG;
-  const Geometry g = make_geometry(s);
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  for (int l = g.L; l >= 1; --l) {
-    const bool sparse = l < g.L;
-    const int n = g.n[l];
-    int gq, nc;
-    if (sparse) {
-      gq = kBlock;
-      nc = kBlock * g.K;
-    } else {
-      nc = n;
-      gq = kBlock;
-      while (gq > 1 && (gq > n || (long long)gq * n > 16384)) gq >>= 1;
-    }
-    if (sparse && g.K >= 2 && g.K <= 16) {
-      // children of the parent's K keys scored in registers (select_children_kernel)
-      const size_t smem = select_children_smem_bytes(nc);
-      const float* qpl = q_pyr + g.pyr_off[l];
-      const float* kpl = k_pyr + g.pyr_off[l];
-      const int* par = idx + g.idx_off[l + 1];
-      int* out = idx + g.idx_off[l];
-      const unsigned grid = (unsigned)(g.BH * (n / kBlock));
-      auto run = [&](auto kern) -> llsa_status {
-        if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
-        return launch(kKSelect, cs, [&] { launch_pdl(kern, dim3(grid), dim3(kSelThreads), smem, cs, g, l, qpl, kpl, par, out); });
-      };
-      switch (g.K) {
-        case 2: st = run(select_children_kernel<1>); break;
-        case 4: st = run(select_children_kernel<2>); break;
-        case 8: st = run(select_children_kernel<4>); break;
-        default: st = run(select_children_kernel<8>); break;
-      }
-      if (st != LLSA_OK) return st;
-      continue;
-    }
-    const size_t smem = select_smem_bytes(gq, nc, g.K, sparse);
-    if (!allow_smem(select_kernel, smem)) return LLSA_ERR_CUDA;
-    const int groups = (n + gq - 1) / gq;
-    st = launch(kKSelect, cs, [&] {
-      launch_pdl(select_kernel, dim3(g.BH * groups), dim3(kSelThreads), smem, cs, g, l, gq, q_pyr + g.pyr_off[l], k_pyr + g.pyr_off[l],
-                                                             sparse ? idx + g.idx_off[l + 1] : nullptr,
-                                                             idx + g.idx_off[l]);
-    });
-    if (st != LLSA_OK) return st;
-  }
-  return LLSA_OK;
+  return select_launch(make_geometry(s), const_cast<float*>(q_pyr), const_cast<float*>(k_pyr), nullptr, idx, false,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 llsa_status llsa_index_transpose(const llsa_shape* s, const int32_t* idx, int32_t* row_ptr, int32_t* col,

@@ -313,4 +313,118 @@ inline size_t select_children_smem_bytes(int nc) {
   return sizeof(float) * ((size_t)kBlock * kD + (size_t)nc * kSelRowStride + (size_t)nc);
 }
 
+// Coarsest level with few tokens (n_L <= 64), one CTA per (b, h): optionally first the
+// pooled levels 3..L of q, k and v from level 2 (POOL; the same sequential fp32 sums as
+// pyramid_up_kernel), then the full Top-K of each of the n_L queries over the n_L keys,
+// one warp per query, lane l scoring keys l and l + 32 (channels in order, as in
+// select_kernel), K rounds of redux.sync max then min.  This replaces launches of 6..72
+// CTAs whose time is all latency.
+constexpr int kTopMaxN = 64;
+
+constexpr int kTopThreads = 512;
+
+template <bool POOL>
+__global__ void __launch_bounds__(kTopThreads) coarsest_small_kernel(Geometry g, float* __restrict__ q_pyr,
+                                                                     float* __restrict__ k_pyr,
+                                                                     float* __restrict__ v_pyr,
+                                                                     int* __restrict__ idx) {
+  pdl_enter();
+  __shared__ __align__(16) float qs[kTopMaxN * kSelRowStride];
+  __shared__ __align__(16) float ks[kTopMaxN * kSelRowStride];
+  const int bh = blockIdx.x;
+  const int L = g.L, K = g.K, n = g.n[L];
+  if (POOL) {
+    for (int l = 3; l <= L; ++l) {
+      const int nl = g.n[l], np = g.n[l - 1];
+      const int items = 3 * nl * kD;
+      // two values per pass: their 32 loads are issued before the in-order sums
+      for (int i0 = threadIdx.x; i0 < items; i0 += 2 * kTopThreads) {
+        float x[2][kBlock];
+        float* dst[2] = {nullptr, nullptr};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int i = i0 + u * kTopThreads;
+          if (i < items) {
+            const int t = i / (nl * kD);
+            const int rem = i - t * nl * kD;
+            const int j = rem >> 6, d = rem & (kD - 1);
+            float* pyr = t == 0 ? q_pyr : (t == 1 ? k_pyr : v_pyr);
+            const float* src = pyr + g.pyr_off[l - 1] + ((long long)bh * np + (long long)j * kBlock) * kD + d;
+#pragma unroll
+            for (int r = 0; r < kBlock; ++r) x[u][r] = src[r * kD];
+            dst[u] = pyr + g.pyr_off[l] + ((long long)bh * nl + j) * kD + d;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (!dst[u]) continue;
+          float acc = 0.0f;
+#pragma unroll
+          for (int r = 0; r < kBlock; ++r) acc = __fadd_rn(acc, x[u][r]);
+          *dst[u] = __fmul_rn(acc, 0.0625f);
+        }
+      }
+      __syncthreads();  // level l is read back by this CTA
+    }
+  }
+  const float* qrow = q_pyr + g.pyr_off[L] + (long long)bh * n * kD;
+  const float* krow = k_pyr + g.pyr_off[L] + (long long)bh * n * kD;
+  for (int i = threadIdx.x; i < n * (kD / 4); i += blockDim.x) {
+    const int r = i >> 4, piece = i & 15;
+    *reinterpret_cast<float4*>(qs + r * kSelRowStride + piece * 4) = reinterpret_cast<const float4*>(qrow + r * kD)[piece];
+    *reinterpret_cast<float4*>(ks + r * kSelRowStride + piece * 4) = reinterpret_cast<const float4*>(krow + r * kD)[piece];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int a = warp; a < n; a += blockDim.x >> 5) {
+    const float4* qa = reinterpret_cast<const float4*>(qs + a * kSelRowStride);
+    float acc[2] = {0.f, 0.f};
+#pragma unroll 4
+    for (int i = 0; i < kD / 4; ++i) {
+      const float4 qv = qa[i];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int c = min(lane + 32 * j, n - 1);
+        const float4 kv = reinterpret_cast<const float4*>(ks + c * kSelRowStride)[i];
+        acc[j] = fmaf(qv.x, kv.x, acc[j]);
+        acc[j] = fmaf(qv.y, kv.y, acc[j]);
+        acc[j] = fmaf(qv.z, kv.z, acc[j]);
+        acc[j] = fmaf(qv.w, kv.w, acc[j]);
+      }
+    }
+    uint32_t key[2];
+    uint32_t bk = 0u;
+    int bc = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      key[j] = lane + 32 * j < n ? score_key(acc[j]) : 0u;
+      if (key[j] > bk) {
+        bk = key[j];
+        bc = lane + 32 * j;
+      }
+    }
+    int win = 0;  // lane r < K keeps the r-th winner
+    for (int r = 0; r < K; ++r) {
+      const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+      const int w = (int)__reduce_min_sync(0xffffffffu, bk == m ? (uint32_t)bc : 0x7fffffffu);
+      if (lane == r) win = w;
+      if (bc == w) {
+        bk = 0u;
+        bc = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (lane + 32 * j == w) key[j] = 0u;
+          if (key[j] > bk) {
+            bk = key[j];
+            bc = lane + 32 * j;
+          }
+        }
+      }
+    }
+    int rank = 0;
+    for (int r2 = 0; r2 < K; ++r2) rank += __shfl_sync(0xffffffffu, win, r2) < win;
+    if (lane < K) idx[g.idx_off[L] + ((long long)bh * n + a) * K + rank] = min(max(win, 0), n - 1);
+  }
+}
+
 }  // namespace llsa
