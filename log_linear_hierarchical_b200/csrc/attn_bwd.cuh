@@ -187,8 +187,21 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 
   bool ok = true;
   int next_seq = 0, next_q = 0;
+  // O rows of the block being started, loaded one block ahead (lane: row lane/2, half lane%2)
+  auto load_o = [&](int i, uint4 (&dst)[4]) {
+    const uint4* orow =
+        reinterpret_cast<const uint4*>(o + ((long long)(first + i) * kBlock + (lane >> 1)) * kD + (lane & 1) * 32);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) dst[c] = __ldg(orow + c);
+  };
+  uint4 onext[4];
+  load_o(0, onext);
   for (int i = 0; i < nblk && ok; ++i) {
     const int gb = first + i;
+    uint4 ocur[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) ocur[c] = onext[c];
+    if (i + 1 < nblk) load_o(i + 1, onext);
     ok = __all_sync(0xffffffffu, mbar_wait(bar_qd + 8 * (i & 1), (i >> 1) & 1));
     if (!ok) break;
     next_q = i + 1;
@@ -199,16 +212,15 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     uint32_t qf[4][4], df[4][4];
     load_a_frags(qt, qf);
     load_a_frags(dt, df);
-    // Delta_r = sum_d dO[r][d] * O[r][d] (O from global, dO from the staged tile)
+    // Delta_r = sum_d dO[r][d] * O[r][d] (O loaded a block ahead, dO from the staged tile)
     float dlt;
     {
       const int r = lane >> 1;
       const int h = lane & 1;
-      const uint4* orow = reinterpret_cast<const uint4*>(o + ((long long)gb * kBlock + r) * kD + h * 32);
       float acc = 0.0f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint4 ov = __ldg(orow + c);
+        const uint4 ov = ocur[c];
         uint4 dv;
         asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                      : "=r"(dv.x), "=r"(dv.y), "=r"(dv.z), "=r"(dv.w)
