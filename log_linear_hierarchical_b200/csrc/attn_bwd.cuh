@@ -33,6 +33,7 @@ struct BwdWorkspace {
   long long cg_off[kMaxLevels + 1];
   long long order;          // int32 [B*H*n_1]: fine key blocks, longest CSR row first
   long long order_counts;   // int32 [kOrdClasses][order tiles]
+  long long order_nonempty; // int32: rows with at least one query block (they come first)
   long long total;
 };
 
@@ -72,6 +73,8 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   off = up(off + (long long)g.BH * g.n[1]);
   w.order_counts = off;
   off = up(off + (long long)kOrdClasses * order_tiles(g));
+  w.order_nonempty = off;
+  off = up(off + 1);
   w.total = off;
   return w;
 }
@@ -630,6 +633,8 @@ __global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometr
         pre += __shfl_xor_sync(0xffffffffu, pre, off);
       }
       if (lane == c) mine = before + pre;
+      if (c == kOrdClasses - 1 && blockIdx.x == 0 && lane == 0)
+        reinterpret_cast<int*>(ws + W.order_nonempty)[0] = before;  // the empty class comes last
       before += tot;
     }
     if (lane < kOrdClasses) start[lane] = mine;
@@ -701,6 +706,47 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   const int lane = lane_id();
   const int n1 = g.n[1];
   const int K = g.K;
+  // CTAs past the non-empty rows write the empty rows, 16 per CTA: no query block selected
+  // them, so dK and dV are only the mean-pool adjoint of their ancestors' coarse gradients
+  // (the same for the 16 keys).  The CTAs beyond those return at once.
+  {
+    const int ne = min(max(__ldg(reinterpret_cast<const int*>(ws + W.order_nonempty)), 0), g.BH * n1);
+    if ((int)blockIdx.x >= ne) {
+      const int e0 = ne + ((int)blockIdx.x - ne) * kBlock;
+      if (e0 >= g.BH * n1) return;
+      if (coarse_late) pdl_wait();
+      const int* order = reinterpret_cast<const int*>(ws + W.order);
+      for (int r = e0; r < min(e0 + kBlock, g.BH * n1); ++r) {
+        const int kb = checked_index(__ldg(order + r), g.BH * n1);
+        const int bh = kb / n1, j = kb - bh * n1;
+        float2 ak = make_float2(0.f, 0.f), av = make_float2(0.f, 0.f);  // channels 2 lane, 2 lane + 1
+        int span = 1, nl = n1;
+        float wgt = 1.0f / kBlock;
+        long long cg_level = 0;
+        for (int lev = 2; lev <= g.L; ++lev) {
+          span *= kBlock;
+          wgt *= 1.0f / kBlock;
+          nl /= kBlock;
+          const long long off = cg_level + ((long long)bh * nl + j / span) * kD + 2 * lane;
+          const float2 xk = *reinterpret_cast<const float2*>(ws + W.cg_k + off);
+          const float2 xv = *reinterpret_cast<const float2*>(ws + W.cg_v + off);
+          ak.x += wgt * xk.x;
+          ak.y += wgt * xk.y;
+          av.x += wgt * xv.x;
+          av.y += wgt * xv.y;
+          cg_level += (long long)g.BH * nl * kD;
+        }
+        const uint32_t pk = pack_bf16(ak.x, ak.y), pv = pack_bf16(av.x, av.y);
+        const long long row0 = (long long)bh * g.N + (long long)j * kBlock;
+#pragma unroll
+        for (int t = 0; t < kBlock; ++t) {
+          reinterpret_cast<uint32_t*>(dk_out + (row0 + t) * kD)[lane] = pk;
+          reinterpret_cast<uint32_t*>(dv_out + (row0 + t) * kD)[lane] = pv;
+        }
+      }
+      return;
+    }
+  }
   // key blocks are taken longest row first (dkdv_order_*_kernel, complete before this
   // kernel's predecessor started)
   const int kb = checked_index(__ldg(reinterpret_cast<const int*>(ws + W.order) + blockIdx.x), g.BH * n1);
