@@ -31,7 +31,7 @@ struct BwdWorkspace {
   long long part_k, part_v; // [B*H*n_2][C][64]
   long long cg_k, cg_v;     // coarse gradients, level-major [l=2..L][B*H*n_l][64]
   long long cg_off[kMaxLevels + 1];
-  long long order;          // int32 [B*H*n_1]: fine key blocks, longest CSR row first
+  long long order;          // int4 [B*H*n_1] {key block, CSR row start, row end, 0}, longest row first
   long long order_counts;   // int32 [kOrdClasses][order tiles]
   long long order_nonempty; // int32: rows with at least one query block (they come first)
   long long total;
@@ -70,7 +70,7 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   w.cg_v = off;
   off = up(off + cg);
   w.order = off;
-  off = up(off + (long long)g.BH * g.n[1]);
+  off = up(off + 4LL * g.BH * g.n[1]);
   w.order_counts = off;
   off = up(off + (long long)kOrdClasses * order_tiles(g));
   w.order_nonempty = off;
@@ -567,11 +567,16 @@ __device__ __forceinline__ int order_class(int len) {
   return len <= 0 ? kOrdClasses - 1 : 7 - min(31 - __clz(len), 7);
 }
 
-// Length of flat level-1 row kb = bh * n_1 + j (0 for kb past the end).
-__device__ __forceinline__ int order_row_len(const Geometry& g, const int* __restrict__ rp1, int kb) {
-  if (kb >= g.BH * g.n[1]) return 0;
+// CSR extent [rs, re) of flat level-1 row kb = bh * n_1 + j (empty for kb past the end).
+__device__ __forceinline__ int2 order_row(const Geometry& g, const int* __restrict__ rp1, int kb) {
+  if (kb >= g.BH * g.n[1]) return make_int2(0, 0);
   const int* r = rp1 + (long long)(kb >> g.log_n1) * (g.n[1] + 1) + (kb & (g.n[1] - 1));
-  return __ldg(r + 1) - __ldg(r);
+  return make_int2(__ldg(r), __ldg(r + 1));
+}
+
+__device__ __forceinline__ int order_row_len(const Geometry& g, const int* __restrict__ rp1, int kb) {
+  const int2 e = order_row(g, rp1, kb);
+  return e.y - e.x;
 }
 
 // Per tile of kOrdTile rows: the number of rows of each class (counts[c * tiles + tile]).
@@ -642,12 +647,14 @@ __global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometr
   const int* rp1 = row_ptr + g.rp_off[1];
   const int row0 = blockIdx.x * kOrdTile + threadIdx.x * kOrdRowsPerThread;
   int cls[kOrdRowsPerThread];
+  int2 ext[kOrdRowsPerThread];
   int cnt[kOrdClasses];
 #pragma unroll
   for (int c = 0; c < kOrdClasses; ++c) cnt[c] = 0;
 #pragma unroll
   for (int i = 0; i < kOrdRowsPerThread; ++i) {
-    cls[i] = row0 + i < g.BH * g.n[1] ? order_class(order_row_len(g, rp1, row0 + i)) : -1;
+    ext[i] = order_row(g, rp1, row0 + i);
+    cls[i] = row0 + i < g.BH * g.n[1] ? order_class(ext[i].y - ext[i].x) : -1;
 #pragma unroll
     for (int cc = 0; cc < kOrdClasses; ++cc) cnt[cc] += (cc == cls[i]);
   }
@@ -672,7 +679,7 @@ __global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometr
     for (int w = 0; w < warp; ++w) base += wsum[w][c];
     pre[c] += base;
   }
-  int* order = reinterpret_cast<int*>(ws + W.order);
+  int4* order = reinterpret_cast<int4*>(ws + W.order);
 #pragma unroll
   for (int i = 0; i < kOrdRowsPerThread; ++i) {
     const int c = cls[i];
@@ -681,7 +688,7 @@ __global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometr
 #pragma unroll
     for (int cc = 0; cc < kOrdClasses; ++cc)
       if (cc == c) pos = pre[cc]++;
-    order[pos] = row0 + i;
+    order[pos] = make_int4(row0 + i, ext[i].x, ext[i].y, 0);
   }
 }
 
@@ -715,9 +722,9 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
       const int e0 = ne + ((int)blockIdx.x - ne) * kBlock;
       if (e0 >= g.BH * n1) return;
       if (coarse_late) pdl_wait();
-      const int* order = reinterpret_cast<const int*>(ws + W.order);
+      const int4* order = reinterpret_cast<const int4*>(ws + W.order);
       for (int r = e0; r < min(e0 + kBlock, g.BH * n1); ++r) {
-        const int kb = checked_index(__ldg(order + r), g.BH * n1);
+        const int kb = checked_index(__ldg(&order[r].x), g.BH * n1);
         const int bh = kb / n1, j = kb - bh * n1;
         float2 ak = make_float2(0.f, 0.f), av = make_float2(0.f, 0.f);  // channels 2 lane, 2 lane + 1
         int span = 1, nl = n1;
@@ -748,8 +755,9 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
     }
   }
   // key blocks are taken longest row first (dkdv_order_*_kernel, complete before this
-  // kernel's predecessor started)
-  const int kb = checked_index(__ldg(reinterpret_cast<const int*>(ws + W.order) + blockIdx.x), g.BH * n1);
+  // kernel's predecessor started); the entry carries the row's CSR extent
+  const int4 ent = __ldg(reinterpret_cast<const int4*>(ws + W.order) + blockIdx.x);
+  const int kb = checked_index(ent.x, g.BH * n1);
   const int bh = kb / n1;
   const int j = kb - bh * n1;
   const CtaSmem cs = kv_smem<STAGES>(1);
@@ -762,8 +770,7 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   const uint32_t bar_ring = bar_kv + 8;
 
   const int E = n1 * K;
-  const int* rp = row_ptr + g.rp_off[1] + (long long)bh * (n1 + 1);
-  int rs = __ldg(rp + j), re = __ldg(rp + j + 1);
+  int rs = ent.y, re = ent.z;
   if (rs < 0 || re > E || rs > re) {
     if (lane == 0) record_error(LLSA_ERR_INTERNAL);
     rs = re = 0;
