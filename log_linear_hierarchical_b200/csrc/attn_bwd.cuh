@@ -246,6 +246,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     float dq[8][4];
 #pragma unroll
     for (int n = 0; n < 8; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
+#pragma unroll kQmUnroll
     for (int s = 0; s < K; ++s) {
       const int seq = i * K + s;
       const int stage = seq % STAGES;
@@ -352,6 +353,7 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
   uint32_t kf[4][4], vf[4][4];
   load_a_frags(kvtile, kf);
   load_a_frags(kvtile + kTileBytes, vf);
+#pragma unroll kKvUnroll
   for (int i = 0; i < npairs; ++i) {
     const int stage = i % STAGES;
     if (!__all_sync(0xffffffffu, mbar_wait(bar_ring + 8 * stage, (i / STAGES) & 1))) {

@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
 #pragma unroll
     for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 
+#pragma unroll kQmUnroll
     for (int s = 0; s < K; ++s) {
       const int seq = i * K + s;
       const int stage = seq % STAGES;

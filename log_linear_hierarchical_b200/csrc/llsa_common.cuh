@@ -27,6 +27,17 @@ constexpr int kTileBytes = 2048;  // one 16-token x 64-channel bf16 tile
 #ifndef LLSA_KV_STAGES
 #define LLSA_KV_STAGES 2
 #endif
+// Unroll of the key-major pair loop and of the query-major fine-tile loops (a sweep on B200
+// at the headline workload, 1 -> 4: dK/dV 136.6 -> 131.9 us, forward 100.4 -> 91.6 us,
+// dQ 116.6 -> 114.3 us; 8 was slower for the pair loop).
+#ifndef LLSA_KV_UNROLL
+#define LLSA_KV_UNROLL 4
+#endif
+#ifndef LLSA_QM_UNROLL
+#define LLSA_QM_UNROLL 4
+#endif
+constexpr int kKvUnroll = LLSA_KV_UNROLL;
+constexpr int kQmUnroll = LLSA_QM_UNROLL;
 // Key-major dK/dV on tcgen05 (1) or on mma.sync warps (0, the default).  At 16-key blocks
 // the tcgen05 kernel is the slower one on B200 (301 us against 195 us at B1 H6 N65536 L3
 // K8): every MMA reads its 4 KB query-side operand from shared memory, Q and dO are read
