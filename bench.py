@@ -163,6 +163,40 @@ def workload_counts(cfg, pairs_l1: int):
         "pyramid_l12": dict(bytes=3 * (bh * cfg.N * D * e + bh * (n1 + (n[2] if cfg.levels >= 2 else 0)) * D * 4),
                             flops=0),
     }
+    L, K = cfg.levels, cfg.topk
+    f4 = 4
+    # selection, all levels of a step (its launches share the name "select"): the coarsest
+    # level reads its q and k rows (plus, pooled in the same launch, levels >= 3 read from the
+    # level below); a finer level l reads, per parent group, the 16K candidate rows once and
+    # the 16 query rows, and writes the indices.
+    sel_bytes = 2 * bh * n[L] * D * f4 + bh * n[L] * K * 4
+    sel_flops = 2 * bh * n[L] * n[L] * D
+    for lev in range(3, L + 1):
+        sel_bytes += 3 * (bh * n[lev - 1] * D * f4 + bh * n[lev] * D * f4)
+    for lev in range(L - 1, 0, -1):
+        groups = bh * n[lev + 1]
+        sel_bytes += groups * (16 * K * D * f4 + 16 * D * f4 + K * 4) + bh * n[lev] * K * 4
+        sel_flops += 2 * bh * n[lev] * 16 * K * D
+    counts["select"] = dict(bytes=sel_bytes // L, flops=sel_flops // L)  # per launch (L per step)
+    # transpose: E entries over all levels; hist reads idx, scatter reads idx and writes the
+    # bucketed entries, bucket reads them and writes col and row_ptr
+    entries = sum(bh * n[lev] * K for lev in range(1, L + 1))
+    rows = sum(bh * (n[lev] + 1) for lev in range(1, L + 1))
+    counts["transpose_hist"] = dict(bytes=entries * 4, flops=0)
+    counts["transpose_scatter"] = dict(bytes=2 * entries * 4, flops=0)
+    counts["transpose_bucket"] = dict(bytes=2 * entries * 4 + rows * 4, flops=0)
+    counts["dkdv_order_count"] = dict(bytes=bh * (n1 + 1) * 4, flops=0)
+    counts["dkdv_order_scatter"] = dict(bytes=bh * (n1 + 1) * 4 + bh * n1 * 16, flops=0)
+    if L >= 2:
+        coarse = (L - 1) * K
+        ctas = bh * n[2] * ((coarse + 15) // 16)
+        # per (level-2 group, coarse tile): 16 query blocks' Q, dO, LSE, Delta, the coarse K/V
+        # rows (fp32), the fp32 partials written
+        counts["attn_bwd_coarse_bf16"] = dict(
+            bytes=ctas * (16 * (2 * tile + 2 * row_stream) + 2 * 16 * D * f4) + 2 * bh * n[2] * coarse * D * f4,
+            flops=8 * ctas * 16 * 16 * 16 * D)
+        cg_rows = sum(bh * n[lev] for lev in range(2, L + 1))
+        counts["coarse_grad_reduce"] = dict(bytes=2 * bh * n[2] * coarse * D * f4 + 2 * cg_rows * D * f4, flops=0)
     return counts
 
 
@@ -329,10 +363,12 @@ def run_ours(args):
             kernels_roof[k] = {"avg_us": round(kern[k]["avg_us"], 2), "share": round(kern[k]["share"], 4),
                                "hbm_frac": round(c["bytes"] / sec / 1e9 / hbm_peak, 4),
                                "tensor_frac": round(c["flops"] / sec / 1e12 / tensor_peak, 4) if c["flops"] else 0.0}
-    # whole-step roofline as the workload defines it: the slower of the step's FLOPs at the
-    # bf16 tensor peak and its modelled bytes at the HBM peak
-    step_bytes = sum(c["bytes"] for k, c in counts.items() if k in kern)
-    step_flops = sum(c["flops"] for k, c in counts.items() if k in kern)
+    # whole-step roofline as the workload defines it: the slower of the selected attention's
+    # FLOPs at the bf16 tensor peak and its modelled bytes (gathers and pyramid) at the HBM
+    # peak; the other kernels have their own fractions in `kernels`
+    step_kernels = ("attn_fwd_bf16", "attn_bwd_dq_bf16", "attn_bwd_dkdv_bf16", "pyramid_l12")
+    step_bytes = sum(c["bytes"] for k, c in counts.items() if k in kern and k in step_kernels)
+    step_flops = sum(c["flops"] for k, c in counts.items() if k in kern and k in step_kernels)
     step_roof_ms = 1000 * max(step_bytes / (hbm_peak * 1e9), step_flops / (tensor_peak * 1e12))
 
     # end to end through the public API with host buffers: a one-step plan per step
