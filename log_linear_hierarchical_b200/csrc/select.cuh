@@ -196,8 +196,9 @@ inline size_t select_smem_bytes(int gq, int nc, int K, bool sparse) {
 // Finer levels with 16K = 32 * CPT candidates (K = 2, 4, 8, 16): the 16 sibling queries of
 // one parent, 8 warps, warp w scoring queries 2w and 2w + 1 against all candidates.  Lane l
 // holds candidates l + 32 j (j < CPT) of both queries in registers, which is the layout the
-// warp Top-K walks, so scores never leave registers: K rounds of redux.sync max (score key)
-// then min (candidate position), the two queries' rounds interleaved.  The dot products
+// warp Top-K walks, so scores never leave registers.  Each lane orders its candidates once
+// (score desc, position asc); then K rounds of redux.sync max (score key) then min
+// (candidate position) over the lanes' heads, the two queries' rounds interleaved.  The dot products
 // accumulate channels 0..63 in order, as in select_kernel, so both give the same scores.
 template <int CPT>
 __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g, int level,
@@ -260,17 +261,32 @@ __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g
   uint32_t key[2][CPT];
   uint32_t bk[2] = {0u, 0u};
   int bc[2] = {0x7fffffff, 0x7fffffff};
+  // each lane orders its CPT candidates once (score desc, index asc); a winner's owner then
+  // only shifts its list
+  int ci[2][CPT];
 #pragma unroll
-  for (int u = 0; u < 2; ++u)
+  for (int u = 0; u < 2; ++u) {
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       key[u][j] = score_key(acc[u][j]);
-      if (key[u][j] > bk[u]) {
-        bk[u] = key[u][j];
-        bc[u] = lane + 32 * j;
-      }
+      ci[u][j] = lane + 32 * j;
     }
-  int win[2] = {0, 0};  // lane r < K keeps the r-th winner of each query
+#pragma unroll
+    for (int pass = 0; pass < CPT; ++pass)
+#pragma unroll
+      for (int j = pass & 1; j + 1 < CPT; j += 2)
+        if (key[u][j + 1] > key[u][j]) {  // indices ascend with j, so equal keys stay in order
+          const uint32_t tk = key[u][j];
+          key[u][j] = key[u][j + 1];
+          key[u][j + 1] = tk;
+          const int tc = ci[u][j];
+          ci[u][j] = ci[u][j + 1];
+          ci[u][j + 1] = tc;
+        }
+    bk[u] = key[u][0];
+    bc[u] = ci[u][0];
+  }
+  int win[2] = {0, 0};
 #pragma unroll 1
   for (int r = 0; r < K; ++r) {
     uint32_t m[2];
@@ -282,17 +298,16 @@ __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       if (lane == r) win[u] = w[u];
-      if (bc[u] == w[u]) {  // the owner drops its winner and finds its next best
-        bk[u] = 0u;
-        bc[u] = 0x7fffffff;
+      if (bc[u] == w[u]) {
 #pragma unroll
-        for (int j = 0; j < CPT; ++j) {
-          if (lane + 32 * j == w[u]) key[u][j] = 0u;
-          if (key[u][j] > bk[u]) {
-            bk[u] = key[u][j];
-            bc[u] = lane + 32 * j;
-          }
+        for (int j = 0; j + 1 < CPT; ++j) {
+          key[u][j] = key[u][j + 1];
+          ci[u][j] = ci[u][j + 1];
         }
+        key[u][CPT - 1] = 0u;
+        ci[u][CPT - 1] = 0x7fffffff;
+        bk[u] = key[u][0];
+        bc[u] = key[u][0] ? ci[u][0] : 0x7fffffff;
       }
     }
   }
