@@ -222,17 +222,29 @@ __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g
 
   const int tid = threadIdx.x;
   const float4* qbase = reinterpret_cast<const float4*>(qp + ((long long)bh * n + a0) * kD);
-  for (int i = tid; i < kBlock * kD / 4; i += kSelThreads) reinterpret_cast<float4*>(qs)[i] = __ldg(qbase + i);
+  const float4 qv = __ldg(qbase + tid);  // 16 rows x 16 pieces = one per thread
   const int np = g.n[level + 1];
   const int* prow = parent_idx + ((long long)bh * np + a0 / kBlock) * K;
   for (int i = tid; i < NC; i += kSelThreads) cand[i] = checked_index(__ldg(prow + i / kBlock), np) * kBlock + (i % kBlock);
-  // candidate rows: 16 threads copy one 256-byte row; the key of a row is computed from the
-  // parent list directly so the copies need not wait for `cand`
-  for (int i = tid; i < NC * (kD / 4); i += kSelThreads) {
-    const int r = i >> 4, piece = i & 15;
-    const int key = checked_index(__ldg(prow + r / kBlock), np) * kBlock + (r % kBlock);
-    const float4 v = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + key) * kD) + piece);
-    *reinterpret_cast<float4*>(ks + r * kSelRowStride + piece * 4) = v;
+  reinterpret_cast<float4*>(qs)[tid] = qv;
+  __syncthreads();
+  // candidate rows: 16 threads copy one 256-byte row; each thread issues all its loads
+  // (up to 8 at a time) before storing any, so they share one memory latency
+  constexpr int kPer = NC * (kD / 4) / kSelThreads;  // float4 pieces per thread
+  constexpr int kBatch = kPer < 8 ? kPer : 8;
+#pragma unroll
+  for (int b0 = 0; b0 < kPer; b0 += kBatch) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = tid + (b0 + u) * kSelThreads;
+      v[u] = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + cand[i >> 4]) * kD) + (i & 15));
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = tid + (b0 + u) * kSelThreads;
+      *reinterpret_cast<float4*>(ks + (i >> 4) * kSelRowStride + (i & 15) * 4) = v[u];
+    }
   }
   __syncthreads();
 
