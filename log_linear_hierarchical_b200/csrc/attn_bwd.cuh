@@ -725,32 +725,53 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
       if (e0 >= g.BH * n1) return;
       if (coarse_late) pdl_wait();
       const int4* order = reinterpret_cast<const int4*>(ws + W.order);
-      for (int r = e0; r < min(e0 + kBlock, g.BH * n1); ++r) {
-        const int kb = checked_index(__ldg(&order[r].x), g.BH * n1);
-        const int bh = kb / n1, j = kb - bh * n1;
-        float2 ak = make_float2(0.f, 0.f), av = make_float2(0.f, 0.f);  // channels 2 lane, 2 lane + 1
-        int span = 1, nl = n1;
-        float wgt = 1.0f / kBlock;
-        long long cg_level = 0;
-        for (int lev = 2; lev <= g.L; ++lev) {
-          span *= kBlock;
-          wgt *= 1.0f / kBlock;
-          nl /= kBlock;
-          const long long off = cg_level + ((long long)bh * nl + j / span) * kD + 2 * lane;
-          const float2 xk = *reinterpret_cast<const float2*>(ws + W.cg_k + off);
-          const float2 xv = *reinterpret_cast<const float2*>(ws + W.cg_v + off);
-          ak.x += wgt * xk.x;
-          ak.y += wgt * xk.y;
-          av.x += wgt * xv.x;
-          av.y += wgt * xv.y;
-          cg_level += (long long)g.BH * nl * kD;
-        }
-        const uint32_t pk = pack_bf16(ak.x, ak.y), pv = pack_bf16(av.x, av.y);
-        const long long row0 = (long long)bh * g.N + (long long)j * kBlock;
+      const int cnt = min(kBlock, g.BH * n1 - e0);
+      const int my_kb = lane < cnt ? checked_index(__ldg(&order[e0 + lane].x), g.BH * n1) : 0;
+      // four rows at a time: all their coarse-gradient loads are issued before any sum
+      for (int r0 = 0; r0 < cnt; r0 += 4) {
+        float2 xk[4][kMaxLevels], xv[4][kMaxLevels];
+        int kbs[4];
 #pragma unroll
-        for (int t = 0; t < kBlock; ++t) {
-          reinterpret_cast<uint32_t*>(dk_out + (row0 + t) * kD)[lane] = pk;
-          reinterpret_cast<uint32_t*>(dv_out + (row0 + t) * kD)[lane] = pv;
+        for (int u = 0; u < 4; ++u) {
+          kbs[u] = __shfl_sync(0xffffffffu, my_kb, min(r0 + u, cnt - 1));
+          const int bh = kbs[u] / n1, j = kbs[u] - bh * n1;
+          int span = 1, nl = n1;
+          long long cg_level = 0;
+#pragma unroll
+          for (int lev = 2; lev <= kMaxLevels; ++lev) {
+            xk[u][lev - 1] = xv[u][lev - 1] = make_float2(0.f, 0.f);
+            if (lev <= g.L) {
+              span *= kBlock;
+              nl /= kBlock;
+              const long long off = cg_level + ((long long)bh * nl + j / span) * kD + 2 * lane;
+              xk[u][lev - 1] = *reinterpret_cast<const float2*>(ws + W.cg_k + off);
+              xv[u][lev - 1] = *reinterpret_cast<const float2*>(ws + W.cg_v + off);
+              cg_level += (long long)g.BH * nl * kD;
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (r0 + u >= cnt) break;
+          const int bh = kbs[u] / n1, j = kbs[u] - bh * n1;
+          float2 ak = make_float2(0.f, 0.f), av = make_float2(0.f, 0.f);  // channels 2 lane, 2 lane + 1
+          float wgt = 1.0f / kBlock;
+#pragma unroll
+          for (int lev = 2; lev <= kMaxLevels; ++lev) {
+            if (lev > g.L) break;
+            wgt *= 1.0f / kBlock;
+            ak.x += wgt * xk[u][lev - 1].x;
+            ak.y += wgt * xk[u][lev - 1].y;
+            av.x += wgt * xv[u][lev - 1].x;
+            av.y += wgt * xv[u][lev - 1].y;
+          }
+          const uint32_t pk = pack_bf16(ak.x, ak.y), pv = pack_bf16(av.x, av.y);
+          const long long row0 = (long long)bh * g.N + (long long)j * kBlock;
+#pragma unroll
+          for (int t = 0; t < kBlock; ++t) {
+            reinterpret_cast<uint32_t*>(dk_out + (row0 + t) * kD)[lane] = pk;
+            reinterpret_cast<uint32_t*>(dv_out + (row0 + t) * kD)[lane] = pv;
+          }
         }
       }
       return;
