@@ -40,6 +40,9 @@ Readings where the pages are silent (each one is also listed in the design notes
 * Enrichment: for l = 2..L the K level-l tokens selected by the block's level-l
   ancestor are appended after the 16K fine tokens, each as one ordinary KV entry
   (unit weight, no score bias).  Level-1 pooled tokens are not attended.
+* Enrichment variant, off by default (``log_bias=True``): a level-l coarse token's
+  scaled score gets + ln(16^l), the log of the number of input tokens it averages, so
+  that it carries the softmax mass of those tokens when they are all equal.
 * Gradients: the selection and the pooled queries carry no gradient; coarse K/V
   tokens pass their gradient back to the input tokens through the mean-pool
   adjoint (each of the 16^l tokens under a level-l token receives 1/16^l of it).
@@ -189,14 +192,24 @@ def kv_index_table(b: int, h: int, idx: list[np.ndarray], offsets: list[int]) ->
     return np.stack([kv_index(p, (b, h), idx, offsets) for p in range(n1)])
 
 
+def kv_bias(topk: int, levels: int) -> np.ndarray:
+    """Additive score bias of each KV-list entry under the log-count enrichment variant:
+    0 for the 16K fine tokens, ln(16^l) for each of the K level-l coarse tokens."""
+    parts = [np.zeros(BLOCK * topk)]
+    for lev in range(2, levels + 1):
+        parts.append(np.full(topk, lev * math.log(BLOCK)))
+    return np.concatenate(parts)
+
+
 # ----------------------------------------------------------------------------- step 4: attention
 
-def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None):
+def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False):
     """Softmax attention of every query over its block's KV list.
 
     Returns (O [B, H, N, D], LSE [B, H, N]) in fp64.  For query i of block p with
     list E(p): z_e = q_i . k_e / sqrt(D), O_i = sum_e softmax(z)_e v_e,
-    LSE_i = max z + ln sum_e exp(z_e - max z).
+    LSE_i = max z + ln sum_e exp(z_e - max z).  With ``log_bias`` z_e also gets
+    ``kv_bias`` (ln(16^l) for a level-l coarse token).
     ``blocks`` (ascending level-1 block indices) restricts the work to those query
     blocks of every (b, h); the other rows of O and LSE are left as NaN.
     """
@@ -208,6 +221,7 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None):
     o = np.full((B, H, N, D), np.nan)
     lse = np.full((B, H, N), np.nan)
     scale = 1.0 / math.sqrt(D)
+    bias = kv_bias(idx[0].shape[-1], len(idx)) if log_bias else 0.0
     sel_blocks = np.arange(n1) if blocks is None else np.asarray(blocks, dtype=np.int64)
     for b in range(B):
         for h in range(H):
@@ -217,7 +231,7 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None):
                 sl = sel_blocks[s0:s0 + chunk]
                 ke = ksrc[b, h][table[sl]]                   # [nb, T, D]
                 ve = vsrc[b, h][table[sl]]
-                z = np.einsum("nqd,ntd->nqt", qb[sl], ke) * scale
+                z = np.einsum("nqd,ntd->nqt", qb[sl], ke) * scale + bias
                 m = z.max(axis=-1, keepdims=True)
                 e = np.exp(z - m)
                 zsum = e.sum(axis=-1, keepdims=True)
@@ -226,7 +240,7 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None):
     return o, lse
 
 
-def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None):
+def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False):
     """Exact gradient of the attention above with the selection held fixed.
 
     With P = softmax(z) on each query's list, Delta_i = sum_d dO_id O_id and
@@ -235,6 +249,7 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
     level-l tokens are then spread over their 16^l input tokens with weight 1/16^l
     (the adjoint of the mean pool).  Returns (dQ, dK, dV) [B, H, N, D] in fp64.
     ``blocks`` restricts the sum to those query blocks (dQ rows of the others are NaN).
+    ``log_bias`` as in ``forward`` (a constant bias leaves the gradient formulas as they are).
     """
     q = np.asarray(q, dtype=np.float64)
     do = np.asarray(do, dtype=np.float64)
@@ -246,6 +261,7 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
     vsrc, _ = kv_sources(v, v_pyr)
     n1 = N // BLOCK
     scale = 1.0 / math.sqrt(D)
+    bias = kv_bias(idx[0].shape[-1], L) if log_bias else 0.0
     dq = np.full((B, H, N, D), np.nan)
     dk = np.empty((B, H, N, D))
     dv = np.empty((B, H, N, D))
@@ -264,7 +280,7 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
                 rows = table[sl]
                 ke = ksrc[b, h][rows]
                 ve = vsrc[b, h][rows]
-                z = np.einsum("nqd,ntd->nqt", qb[sl], ke) * scale
+                z = np.einsum("nqd,ntd->nqt", qb[sl], ke) * scale + bias
                 p = np.exp(z - lseb[sl][..., None])
                 dp = np.einsum("nqd,ntd->nqt", dob[sl], ve)
                 ds = p * (dp - delta[sl][..., None])
@@ -322,17 +338,17 @@ def index_transpose_all(idx: list[np.ndarray]) -> tuple[list[np.ndarray], list[n
 
 # ----------------------------------------------------------------------------- whole path
 
-def llsa_step(q, k, v, do, levels: int, topk: int):
+def llsa_step(q, k, v, do, levels: int, topk: int, log_bias: bool = False):
     """Pyramid, selection, forward, backward and transposes with the oracle's own
     selection.  Inputs are exact widenings of the device inputs."""
     q_pyr = build_pyramid(q, levels)
     k_pyr = build_pyramid(k, levels)
     v_pyr = build_pyramid(v, levels)
     idx = select(q_pyr, k_pyr, topk)
-    o, lse = forward(q, k, v, k_pyr, v_pyr, idx)
+    o, lse = forward(q, k, v, k_pyr, v_pyr, idx, log_bias=log_bias)
     out = dict(q_pyr=q_pyr, k_pyr=k_pyr, v_pyr=v_pyr, idx=idx, o=o, lse=lse)
     if do is not None:
-        out["dq"], out["dk"], out["dv"] = backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx)
+        out["dq"], out["dk"], out["dv"] = backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, log_bias=log_bias)
     out["row_ptr"], out["col"] = index_transpose_all(idx)
     return out
 

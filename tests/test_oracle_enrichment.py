@@ -1,0 +1,91 @@
+"""Pins for the oracle's log-count enrichment variant (``log_bias``), on CPU.
+
+The variant adds ln(16^l) to the scaled score of every level-l coarse token.  The pin does
+not restate that formula: when every key and value inside each coarsest-level group is the
+same vector, a level-l pooled token equals each of the 16^l input tokens it averages, so
+attention over the biased list must equal plain softmax attention (torch, fp64) over the
+explicit multiset in which each coarse token is repeated 16^l times.  Finite differences
+check the backward with the bias on.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle.llsa_oracle import (BLOCK, backward, build_pyramid, forward, kv_index, kv_sources, select)
+
+
+def grouped(rng, B, H, N, D, group):
+    """[B, H, N, D] with all tokens inside each run of `group` tokens equal."""
+    g = rng.standard_normal((B, H, N // group, D))
+    return np.repeat(g, group, axis=2)
+
+
+@pytest.mark.parametrize("N,L,K", [(4096, 2, 2), (8192, 3, 2)])
+def test_log_bias_equals_attention_over_repeated_coarse_tokens(N, L, K):
+    rng = np.random.default_rng(11)
+    B, H, D = 1, 1, 8
+    group = BLOCK ** L  # constant over every coarsest-level group, hence over all levels below
+    q = rng.standard_normal((B, H, N, D))
+    k = grouped(rng, B, H, N, D, group)
+    v = grouped(rng, B, H, N, D, group)
+    qp, kp, vp = (build_pyramid(x, L, np.float64) for x in (q, k, v))
+    idx = select(qp, kp, K)
+    o, lse = forward(q, k, v, kp, vp, idx, log_bias=True)
+    ksrc, offsets = kv_sources(k, kp)
+    vsrc, _ = kv_sources(v, vp)
+    n1 = N // BLOCK
+    for p in range(0, n1, max(1, n1 // 16)):
+        rows = kv_index(p, (0, 0), idx, offsets)
+        reps = np.ones(len(rows), dtype=np.int64)
+        for lev in range(2, L + 1):  # the K level-l entries follow the 16K fine ones, levels in order
+            start = BLOCK * K + (lev - 2) * K
+            reps[start:start + K] = BLOCK ** lev
+        km = torch.tensor(np.repeat(ksrc[0, 0][rows], reps, axis=0))[None, None]
+        vm = torch.tensor(np.repeat(vsrc[0, 0][rows], reps, axis=0))[None, None]
+        qb = torch.tensor(q[0, 0, p * BLOCK:(p + 1) * BLOCK])[None, None]
+        ref = F.scaled_dot_product_attention(qb, km, vm)[0, 0].numpy()
+        ref_lse = torch.logsumexp(qb @ km.transpose(-1, -2) / math.sqrt(D), dim=-1)[0, 0].numpy()
+        assert np.abs(o[0, 0, p * BLOCK:(p + 1) * BLOCK] - ref).max() < 1e-12
+        assert np.abs(lse[0, 0, p * BLOCK:(p + 1) * BLOCK] - ref_lse).max() < 1e-11
+
+
+def test_log_bias_changes_only_coarse_weights():
+    # L = 1 has no coarse entries: the variant must be the identity there
+    rng = np.random.default_rng(12)
+    B, H, N, D = 1, 1, 1024, 8
+    q, k, v = (rng.standard_normal((B, H, N, D)) for _ in range(3))
+    qp, kp, vp = (build_pyramid(x, 1, np.float64) for x in (q, k, v))
+    idx = select(qp, kp, 4)
+    a = forward(q, k, v, kp, vp, idx)
+    b = forward(q, k, v, kp, vp, idx, log_bias=True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_log_bias_finite_differences_with_frozen_selection():
+    rng = np.random.default_rng(13)
+    B, H, N, D, K, L = 1, 1, 8192, 4, 2, 3
+    q, k, v, do = (rng.standard_normal((B, H, N, D)) for _ in range(4))
+    idx = select(build_pyramid(q, L, np.float64), build_pyramid(k, L, np.float64), K)
+
+    def loss(q_, k_, v_):
+        kp, vp = build_pyramid(k_, L, np.float64), build_pyramid(v_, L, np.float64)
+        o, _ = forward(q_, k_, v_, kp, vp, idx, log_bias=True)
+        return float((o * do).sum())
+
+    kp, vp = build_pyramid(k, L, np.float64), build_pyramid(v, L, np.float64)
+    o, lse = forward(q, k, v, kp, vp, idx, log_bias=True)
+    dq, dk, dv = backward(q, k, v, o, lse, do, kp, vp, idx, log_bias=True)
+    eps = 1e-6
+    picks = [(0, 0, 7, 1), (0, 0, 2049, 3), (0, 0, 8190, 0), (0, 0, 5000, 2)]
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for pos in picks:
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[name][pos] += eps
+            up = loss(args["q"], args["k"], args["v"])
+            args[name][pos] -= 2 * eps
+            dn = loss(args["q"], args["k"], args["v"])
+            fd = (up - dn) / (2 * eps)
+            assert abs(fd - grad[pos]) < 1e-7 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
