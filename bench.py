@@ -202,7 +202,7 @@ def workload_counts(cfg, pairs_l1: int):
 
 # ----------------------------------------------------------------------------- oracle sample
 
-def oracle_sample(cfg, inputs, heads: int, nblocks: int | None):
+def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool = False):
     """Time the CPU oracle on ``heads`` (b=0) heads of the workload: pyramid, selection and
     transpose for each whole head, forward and backward for ``nblocks`` query blocks per
     head (all blocks if None).  Returns (tokens/s extrapolated to the full workload, dict)."""
@@ -226,9 +226,9 @@ def oracle_sample(cfg, inputs, heads: int, nblocks: int | None):
             idx = orc.select(qp, kp, cfg.topk)
             orc.index_transpose_all(idx)
             t1 = time.perf_counter()
-            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks)
+            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks, log_bias=log_bias)
             if cfg.backward:
-                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks)
+                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks, log_bias=log_bias)
             t2 = time.perf_counter()
             t_fixed += t1 - t0
             t_attn += t2 - t1
@@ -257,7 +257,7 @@ def run_ours(args):
     host = make_config_inputs(cfg, with_do=True)
     pinned = {k: v.pin_memory() for k, v in host.items()}
     dev = {k: v.cuda(non_blocking=True) for k, v in pinned.items()}
-    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype)
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, log_bias=args.log_bias)
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     stream = torch.cuda.current_stream()
 
@@ -421,7 +421,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, info = oracle_sample(cfg, host, heads=2, nblocks=None)
+        val, info = oracle_sample(cfg, host, heads=2, nblocks=None, log_bias=args.log_bias)
         cpu = {"value": round(val, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": (f"numpy fp64 oracle, 1 thread: pyramid, selection, transpose, forward and backward of "
                           f"heads (b=0, h=0..1), {info['seconds']:.1f} s, extrapolated to {cfg.B * cfg.H} heads")}
@@ -443,6 +443,7 @@ def run_ours(args):
         "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
                    "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk, "kv_len": cfg.kv_len,
                    "step": "pyramid + select + forward + index transpose + backward",
+                   "enrichment": "log-count bias ln(16^l) on coarse scores" if args.log_bias else "unit weight",
                    "launch": ("K steps as one CUDA graph (llsa_plan_create repeat=K), kernels chained by "
                               "programmatic dependent launch; transpose on a second stream"),
                    "kernel_times_from": ("a second plan of the same K steps with trace events around every "
@@ -508,14 +509,14 @@ def run_reference(args):
     n1 = cfg.N // 16
     # size each step's sample so that warm-up + steps stay near two minutes
     budget = 120.0 / max(1, args.steps + args.warmup)
-    _, probe = oracle_sample(cfg, host, heads=1, nblocks=16)
+    _, probe = oracle_sample(cfg, host, heads=1, nblocks=16, log_bias=args.log_bias)
     per_block = max(1e-6, probe["t_attn_per_block"])
     nblocks = int(max(16, min(n1, (budget - probe["t_fixed_per_head"]) / per_block)))
     for _ in range(args.warmup):
-        oracle_sample(cfg, host, heads=1, nblocks=nblocks)
+        oracle_sample(cfg, host, heads=1, nblocks=nblocks, log_bias=args.log_bias)
     vals, secs = [], 0.0
     for _ in range(args.steps):
-        v, info = oracle_sample(cfg, host, heads=1, nblocks=nblocks)
+        v, info = oracle_sample(cfg, host, heads=1, nblocks=nblocks, log_bias=args.log_bias)
         vals.append(v)
         secs += info["seconds"]
     value = statistics.median(vals)
@@ -547,7 +548,7 @@ def run_profile(args):
     cfg = CONFIGS[args.config]
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     dev = {k: v.cuda() for k, v in make_config_inputs(cfg, with_do=True).items()}
-    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype)
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, log_bias=args.log_bias)
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     for _ in range(args.warmup + args.steps):
         api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
@@ -567,6 +568,8 @@ def main():
     ap.add_argument("--config", type=int, default=4, help="workload number (4 = the headline N=65536 step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--profile", action="store_true", help="run only the steps (for ncu), print no metric")
+    ap.add_argument("--log-bias", action="store_true",
+                    help="the log-count enrichment variant (ln 16^l on level-l coarse scores)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -76,12 +76,21 @@ typedef enum {
 
 typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
 
+/*
+ * Enrichment variant (no counterpart on the pages, which give no weighting for the coarse
+ * tokens): with LLSA_FLAG_LOG_BIAS the scaled score of every level-l coarse KV entry gets
+ * + ln(16^l), the log of the number of input tokens the pooled token averages, so that it
+ * carries their softmax mass when they are all equal.  Default 0: unit-weight entries.
+ */
+#define LLSA_FLAG_LOG_BIAS 1
+
 typedef struct {
   int32_t B, H, N, D;
   int32_t block;   /* must be 16 (README usage section: block_size=16) */
   int32_t topk;    /* K, a power of two */
   int32_t levels;  /* L, number of pooled levels; llsa_l1 <-> 1, llsa_l2 <-> 2 */
   int32_t dtype;   /* llsa_dtype of q, k, v, o, dO, dq, dk, dv */
+  int32_t flags;   /* 0 or LLSA_FLAG_LOG_BIAS; other bits -> LLSA_ERR_INVALID_ARG */
 } llsa_shape;
 
 /* Static text for a status code. */

@@ -35,7 +35,11 @@ class LLSAShape(ctypes.Structure):
 
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("block", ctypes.c_int32), ("topk", ctypes.c_int32), ("levels", ctypes.c_int32),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+
+# llsa_shape.flags: log-count score bias on the coarse KV entries (ln 16^l at level l)
+LLSA_FLAG_LOG_BIAS = 1
 
 
 _SP = ctypes.POINTER(LLSAShape)

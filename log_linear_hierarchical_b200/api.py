@@ -27,9 +27,11 @@ class LLSAError(RuntimeError):
         self.status = status
 
 
-def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16) -> LLSAShape:
+def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16,
+               log_bias: bool = False) -> LLSAShape:
+    """``log_bias``: the log-count enrichment variant (LLSA_FLAG_LOG_BIAS)."""
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
-    return LLSAShape(B, H, N, D, block, topk, levels, code)
+    return LLSAShape(B, H, N, D, block, topk, levels, code, _lib.LLSA_FLAG_LOG_BIAS if log_bias else 0)
 
 
 def _check(fn: str, status: int) -> None:

@@ -95,7 +95,8 @@ __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
 template <bool MASK>
 __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[4][4], const uint32_t (&df)[4][4], uint32_t ktile,
                                          uint32_t vtile, int valid, float scale_log2, const float (&lse2)[2],
-                                         const float (&delta)[2], float (&dq)[8][4]) {
+                                         const float (&delta)[2], float (&dq)[8][4], const Geometry* bias_g = nullptr,
+                                         int c0 = 0) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -108,7 +109,9 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[4][4], const uint3
     for (int e = 0; e < 4; ++e) {
       const int col = n * 8 + 2 * (lane & 3) + (e & 1);
       const int r = e >> 1;
-      const float p = (!MASK || col < valid) ? ex2(fmaf(s[n][e], scale_log2, -lse2[r])) : 0.0f;
+      float sb = s[n][e];
+      if (MASK && bias_g && bias_g->log_bias && col < valid) sb += coarse_log_bias(*bias_g, c0 + col) * kSqrtD;
+      const float p = (!MASK || col < valid) ? ex2(fmaf(sb, scale_log2, -lse2[r])) : 0.0f;
       ds[n][e] = p * (dp[n][e] - delta[r]);
     }
   mma_a_b(dq, pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]), pack_bf16(ds[1][0], ds[1][1]),
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
       dq_chunk<true>(qf, df, ck + cc * kTileBytes, cv + cc * kTileBytes, min(kBlock, g.coarse - cc * kBlock),
-                     P.scale_log2, lse2, delta, dq);
+                     P.scale_log2, lse2, delta, dq, &g, cc * kBlock);
     __syncwarp();
     store_tile_bf16(dq, P.scale, P.scale, qt, dq_out + (long long)gb * kBlock * kD);
   }
@@ -278,9 +281,12 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 // and the query block's Q and dO tiles, LSE and Delta staged:
 //   S^T = K Q^T, P^T = exp2(S^T*scale*log2e - LSE*log2e), dP^T = V dO^T,
 //   dS^T = P^T (dP^T - Delta), dV += P^T dO, dK += dS^T Q  (dK unscaled).
+// BIAS: the key rows are coarse tokens under the log-count variant; kb[0], kb[1] are the
+// biases (unscaled-dot units) of this lane's key rows r0 and r0 + 8.
+template <bool BIAS = false>
 __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32_t (&vf)[4][4], uint32_t qt,
                                         uint32_t dt, const float* ls, const float* dl, float scale_log2,
-                                        float (&dk)[8][4], float (&dv)[8][4]) {
+                                        float (&dk)[8][4], float (&dv)[8][4], const float (&kb)[2] = {0.f, 0.f}) {
   const int c2 = 2 * (lane_id() & 3);
   float st[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dpt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -298,7 +304,7 @@ __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32
   for (int n = 0; n < 2; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      pt[n][e] = ex2(fmaf(st[n][e], scale_log2, -lq[n][e & 1]));
+      pt[n][e] = ex2(fmaf(BIAS ? st[n][e] + kb[e >> 1] : st[n][e], scale_log2, -lq[n][e & 1]));
       dst[n][e] = pt[n][e] * (dpt[n][e] - dq[n][e & 1]);
     }
   mma_a_b(dv, pack_bf16(pt[0][0], pt[0][1]), pack_bf16(pt[0][2], pt[0][3]), pack_bf16(pt[1][0], pt[1][1]),
@@ -324,12 +330,13 @@ __host__ __device__ inline CtaSmem kv_smem(int nwarps) {
 // `bar_tile` is non-zero the key tile is still arriving on that mbarrier (phase 0) and is
 // waited for after the first pair loads are issued.  Returns false (after draining the
 // copies in flight) if a wait timed out.
-template <int STAGES, class PairBlock>
+template <int STAGES, bool BIAS = false, class PairBlock>
 __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtensorMap* tm_do,
                                           const float* __restrict__ lse, const float* __restrict__ delta,
                                           uint32_t kvtile, uint32_t bar_tile, uint32_t ring, float* sls, float* sdl,
                                           uint32_t bar_ring, int npairs, PairBlock pair_block, float scale_log2,
-                                          float (&dk)[8][4], float (&dv)[8][4]) {
+                                          float (&dk)[8][4], float (&dv)[8][4],
+                                          const float (&kbias)[2] = {0.f, 0.f}) {
   const int lane = lane_id();
   // called by the whole warp (pair_block may shuffle); lane 0 issues the copies
   auto issue_pair = [&](int i) {
@@ -361,7 +368,7 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
       return false;
     }
     const uint32_t qt = ring + stage * 2 * kTileBytes;
-    kv_pair(kf, vf, qt, qt + kTileBytes, sls + stage * kBlock, sdl + stage * kBlock, scale_log2, dk, dv);
+    kv_pair<BIAS>(kf, vf, qt, qt + kTileBytes, sls + stage * kBlock, sdl + stage * kBlock, scale_log2, dk, dv, kbias);
     __syncwarp();
     if (i + STAGES < npairs) issue_pair(i + STAGES);
   }
@@ -440,8 +447,17 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
   for (int n = 0; n < 8; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
-  const bool ok = kv_stream<STAGES>(&tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
-                                    [&](int i) { return first_block + i; }, P.scale_log2, dk, dv);
+  bool ok;
+  if (g.log_bias) {  // this lane's key rows are coarse entries tile * 16 + r0 and + 8
+    const int r0 = tile * kBlock + (lane >> 2);
+    const float kb[2] = {r0 < g.coarse ? coarse_log_bias(g, r0) * kSqrtD : 0.f,
+                         r0 + 8 < g.coarse ? coarse_log_bias(g, r0 + 8) * kSqrtD : 0.f};
+    ok = kv_stream<STAGES, true>(&tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
+                                 [&](int i) { return first_block + i; }, P.scale_log2, dk, dv, kb);
+  } else {
+    ok = kv_stream<STAGES>(&tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
+                           [&](int i) { return first_block + i; }, P.scale_log2, dk, dv);
+  }
   if (!ok) return;
   const int r0 = lane >> 2;
   const int c2 = 2 * (lane & 3);

@@ -132,12 +132,16 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[8][4], float 
   __syncwarp();
 }
 
-// One 16-token chunk of the online softmax.  With MASK, columns >= `valid` (the padding of
-// the last coarse tile) are excluded.  m holds the running row maxima of the scaled scores
-// (log2 domain), l the per-lane partial row sums.
+constexpr float kSqrtD = 8.0f;  // sqrt(kD): score bias in units of the unscaled dot product
+
+// One 16-token chunk of the online softmax.  With MASK (the coarse chunks), columns >=
+// `valid` (the padding of the last coarse tile) are excluded and, under the log-count
+// variant, column c gets the bias of coarse entry c0 + c.  m holds the running row maxima
+// of the scaled scores (log2 domain), l the per-lane partial row sums.
 template <bool MASK>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t ktile, uint32_t vtile, int valid,
-                                          float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[8][4]) {
+                                          float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[8][4],
+                                          const Geometry* bias_g = nullptr, int c0 = 0) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt(s, qf, ktile);
@@ -145,8 +149,11 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
 #pragma unroll
     for (int n = 0; n < 2; ++n)
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (n * 8 + 2 * (lane & 3) + (e & 1) >= valid) s[n][e] = -INFINITY;
+      for (int e = 0; e < 4; ++e) {
+        const int col = n * 8 + 2 * (lane & 3) + (e & 1);
+        if (col >= valid) s[n][e] = -INFINITY;
+        else if (bias_g && bias_g->log_bias) s[n][e] += coarse_log_bias(*bias_g, c0 + col) * kSqrtD;
+      }
   }
   float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
   float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
       fwd_chunk<true>(qf, ck + cc * kTileBytes, cv + cc * kTileBytes, min(kBlock, g.coarse - cc * kBlock),
-                      P.scale_log2, m, l, acc);
+                      P.scale_log2, m, l, acc, &g, cc * kBlock);
 
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 1);
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 2);

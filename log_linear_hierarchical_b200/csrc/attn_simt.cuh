@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
   for (int pr = threadIdx.x; pr < kBlock * T; pr += blockDim.x) {
     const int qi = pr / T;
     const int e = pr - qi * T;
-    S[pr] = dot64(qs + qi * kD, krow[e]) * scale;
+    S[pr] = dot64(qs + qi * kD, krow[e]) * scale + (e >= kBlock * g.K ? coarse_log_bias(g, e - kBlock * g.K) : 0.0f);
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -166,7 +166,8 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
     for (int pr = threadIdx.x; pr < kBlock * T; pr += blockDim.x) {
       const int qi = pr / T;
       const int e = pr - qi * T;
-      const float pe = expf(dot64(qs + qi * kD, krow[e]) * scale - lse[rbase + qi]);
+      const float bias = e >= kBlock * g.K ? coarse_log_bias(g, e - kBlock * g.K) : 0.0f;
+      const float pe = expf(dot64(qs + qi * kD, krow[e]) * scale + bias - lse[rbase + qi]);
       const float dp = dot64(ds_ + qi * kD, vrow[e]);
       Pm[pr] = pe;
       dS[pr] = pe * (dp - delta[qi]);

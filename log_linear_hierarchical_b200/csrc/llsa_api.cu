@@ -38,6 +38,7 @@ llsa_status validate(const llsa_shape* s) {
   if (s->B < 1 || s->H < 1 || s->N < 1 || s->D < 1 || s->block < 1 || s->topk < 1 || s->levels < 1)
     return LLSA_ERR_INVALID_ARG;
   if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
+  if (s->flags & ~LLSA_FLAG_LOG_BIAS) return LLSA_ERR_INVALID_ARG;  // unknown flag bits
   if (!is_pow2(s->N) || !is_pow2(s->topk)) return LLSA_ERR_INVALID_ARG;  // README usage notes
   if (s->block != kBlock) return LLSA_ERR_UNSUPPORTED;
   if (s->D != kD) return LLSA_ERR_UNSUPPORTED;
@@ -76,6 +77,7 @@ Geometry make_geometry(const llsa_shape* s) {
   g.log_n1 = ilog2(g.n[1]);
   g.coarse = (g.L - 1) * g.K;
   g.coarse_pad = (g.coarse + kBlock - 1) / kBlock * kBlock;
+  g.log_bias = (s->flags & LLSA_FLAG_LOG_BIAS) ? 1 : 0;
   return g;
 }
 

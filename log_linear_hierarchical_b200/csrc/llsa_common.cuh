@@ -57,7 +57,15 @@ struct Geometry {
   long long rp_off[kMaxLevels + 1];      // element offset of level l in row_ptr
   int coarse;                            // C = (L-1) K coarse KV entries per query block
   int coarse_pad;                        // C rounded up to a multiple of 16
+  int log_bias;                          // LLSA_FLAG_LOG_BIAS: coarse scores + ln(16^l)
 };
+
+// Additive score bias of coarse entry c (0 <= c < C, level 2 + c / K) under the log-count
+// enrichment variant, in units of the scaled score: ln(16^l) = l ln 16; 0 when it is off.
+constexpr float kLn16 = 2.7725887222397811f;
+__host__ __device__ inline float coarse_log_bias(const Geometry& g, int c) {
+  return g.log_bias ? (float)(2 + (c >> g.log_k)) * kLn16 : 0.0f;  // K = 2^log_k
+}
 
 // ---------------------------------------------------------------------------- status word
 // One per device (a module global); kernels record the first error, llsa_device_status

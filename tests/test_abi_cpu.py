@@ -115,3 +115,13 @@ def test_step_and_plan_rejected_before_launch(lib):
     assert lib.llsa_plan_create(ctypes.byref(s), ctypes.byref(small_ws), 1, None) == 1
     assert lib.llsa_plan_launch(None, None) == 1
     lib.llsa_plan_destroy(None)
+
+
+def test_flags_validated(lib):
+    s = shape()
+    s.flags = 1  # LLSA_FLAG_LOG_BIAS
+    assert lib.llsa_validate_shape(ctypes.byref(s)) == 0
+    for bad in (2, 4, 1 << 30, -1):
+        s.flags = bad
+        assert lib.llsa_validate_shape(ctypes.byref(s)) == 1, bad
+    assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True).flags == _lib.LLSA_FLAG_LOG_BIAS
