@@ -24,6 +24,8 @@ What it computes (Log-linear Sparse Attention, non-causal, per batch b and head 
    replaces (non-causal, scale 1/sqrt(D), no dropout), and its exact gradient.
 5. ``index_transpose`` -- the sparse index transpose: query -> key lists turned into
    key -> query lists without a dense mask (skill page, Core Technique 3).
+6. ``to_z_order`` / ``from_z_order`` -- the quadtree token order of a square 2-D token
+   grid that the README recommends for images (its token reordering example).
 
 Readings where the pages are silent (each one is also listed in the design notes):
 
@@ -334,6 +336,41 @@ def index_transpose_all(idx: list[np.ndarray]) -> tuple[list[np.ndarray], list[n
         rps.append(rp)
         cols.append(cl)
     return rps, cols
+
+
+# ----------------------------------------------------------------------------- token order
+
+def zorder_index(side: int) -> np.ndarray:
+    """Quadtree (Z) index of every position of a side x side grid, row-major: position
+    (r, c) gets z = sum_b (2 r_b + c_b) 4^b over the bits b of r and c, i.e. at every scale
+    the quadrants in the order top-left, top-right, bottom-left, bottom-right (the LLSA
+    GitHub README, token reordering example: similar, nearby tokens get adjacent indices)."""
+    if side < 1 or side & (side - 1):
+        raise ValueError("side must be a power of two")
+    r, c = np.divmod(np.arange(side * side, dtype=np.int64), side)
+    z = np.zeros_like(r)
+    for b in range(int(side).bit_length()):
+        z |= ((r >> b) & 1) << (2 * b + 1)
+        z |= ((c >> b) & 1) << (2 * b)
+    return z
+
+
+def to_z_order(x: np.ndarray) -> np.ndarray:
+    """[..., N, D] in row-major grid order -> Z order (N a power of four)."""
+    n = x.shape[-2]
+    side = int(round(math.sqrt(n)))
+    if side * side != n:
+        raise ValueError("N must be a square grid")
+    out = np.empty_like(x)
+    out[..., zorder_index(side), :] = x
+    return out
+
+
+def from_z_order(x: np.ndarray) -> np.ndarray:
+    """Inverse of ``to_z_order``."""
+    n = x.shape[-2]
+    side = int(round(math.sqrt(n)))
+    return x[..., zorder_index(side), :]
 
 
 # ----------------------------------------------------------------------------- whole path
