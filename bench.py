@@ -397,6 +397,27 @@ def run_ours(args):
     plan1.close()
     e2e_value = world * e2e_steps * tokens_per_step / (e2e_ms / 1000.0)
 
+    # quadtree token order (llsa_token_permute) of one input tensor: HBM streaming
+    zperm = None
+    side_ok = (cfg.N & (cfg.N - 1)) == 0 and int(round(cfg.N ** 0.5)) ** 2 == cfg.N
+    if side_ok:
+        zdst = torch.empty_like(dev["q"])
+        for _ in range(3):
+            api.llsa_token_permute(shape, dev["q"], zdst, to_z_order=True, stream=stream)
+        torch.cuda.synchronize()
+        z0, z1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        zreps = 20
+        z0.record(stream)
+        for _ in range(zreps):
+            api.llsa_token_permute(shape, dev["q"], zdst, to_z_order=True, stream=stream)
+        z1.record(stream)
+        torch.cuda.synchronize()
+        zus = 1000 * z0.elapsed_time(z1) / zreps
+        zbytes = 2 * dev["q"].numel() * dev["q"].element_size()
+        zperm = {"tensor": "q to Z order", "avg_us": round(zus, 2), "bytes": zbytes,
+                 "gbs": round(zbytes / (zus * 1e-6) / 1e9, 1), "hbm_frac": round(zbytes / (zus * 1e-6) / 1e9 / hbm_peak, 4)}
+        del zdst
+
     # dense attention at the same shape (torch SDPA, flash backend), forward + backward
     dense = None
     if world == 1:
@@ -462,6 +483,7 @@ def run_ours(args):
                 "api": ("log_linear_hierarchical_b200.LLSAPlan (one captured step, llsa_plan_launch) with pinned "
                         "host copies in and out")},
         "dense_attention": dense,
+        "token_permute": zperm,
         "gpu_launches": trace.used,
         "clocks": clocks,
     }

@@ -223,6 +223,19 @@ llsa_status llsa_plan_launch(const llsa_plan* plan, llsa_stream_t stream);
 void llsa_plan_destroy(llsa_plan* plan);
 
 /*
+ * Quadtree (Z) token order of a square token grid (LLSA GitHub README, token reordering
+ * example: for images, reorder tokens so that nearby, similar tokens get adjacent indices;
+ * each 16-token block is then a 4 x 4 square and each level-l pooled token a
+ * 4^l x 4^l square).  N must be a power of four (side = sqrt(N)); grid position (r, c),
+ * row-major index r * side + c, has Z index z = sum_b (2 r_b + c_b) 4^b.
+ * to_z_order != 0: dst[b, h, z(p)] = src[b, h, p]; 0: the inverse, dst[b, h, p] =
+ * src[b, h, z(p)].  src, dst: [B, H, N, D] `dtype`, distinct (not in place), 16-byte
+ * aligned.  Non-square N or src == dst -> LLSA_ERR_INVALID_ARG.
+ */
+llsa_status llsa_token_permute(const llsa_shape* shape, const void* src, void* dst, int32_t to_z_order,
+                               llsa_stream_t stream);
+
+/*
  * Reads and clears the device status word that kernels set on an out-of-range index
  * (LLSA_ERR_INTERNAL) or a bounded wait that timed out (LLSA_ERR_TIMEOUT).  Synchronises
  * `stream` first.  *code_out receives LLSA_OK or the first error recorded since the last

@@ -74,6 +74,7 @@ SIGNATURES = {
     "llsa_plan_create": (_I, [_SP, _BP, ctypes.c_int32, ctypes.POINTER(_P)]),
     "llsa_plan_launch": (_I, [_P, _P]),
     "llsa_plan_destroy": (None, [_P]),
+    "llsa_token_permute": (_I, [_SP, _P, _P, ctypes.c_int32, _P]),
     "llsa_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _P]),
     "llsa_trace_begin": (_I, [ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]),
     "llsa_trace_end": (_I, [ctypes.POINTER(ctypes.c_int32)]),

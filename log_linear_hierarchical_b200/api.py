@@ -123,6 +123,13 @@ def llsa_backward(shape, q, k, v, o, lse, do, k_pyr, v_pyr, idx, row_ptr, col, d
         _p(col), _p(dq), _p(dk), _p(dv), _p(workspace), nbytes, _stream(stream)))
 
 
+def llsa_token_permute(shape, src, dst, to_z_order: bool = True, stream=None) -> None:
+    """Quadtree (Z) token order of a square token grid: row-major -> Z (``to_z_order``) or
+    back; src and dst are distinct [B, H, N, D] tensors."""
+    _check("llsa_token_permute", _lib.load().llsa_token_permute(_ref(shape), _p(src), _p(dst), int(bool(to_z_order)),
+                                                                _stream(stream)))
+
+
 def llsa_device_status(stream=None) -> int:
     code = ctypes.c_int32(0)
     _check("llsa_device_status", _lib.load().llsa_device_status(ctypes.byref(code), _stream(stream)))

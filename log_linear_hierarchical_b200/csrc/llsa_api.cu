@@ -13,6 +13,7 @@
 #include "pyramid.cuh"
 #include "select.cuh"
 #include "transpose.cuh"
+#include "zorder.cuh"
 
 using namespace llsa;
 
@@ -192,6 +193,7 @@ enum KernelId {
   kKBwdDkdvEmpty,
   kKDkdvOrderCount,
   kKDkdvOrderScatter,
+  kKZOrder,
   kKNumKernels
 };
 
@@ -199,7 +201,7 @@ const char* const kKernelNames[kKNumKernels] = {
     "unknown",          "pyramid_l12",          "pyramid_up",   "select",           "transpose_hist",
     "transpose_scatter", "transpose_bucket",    "attn_fwd_bf16", "attn_bwd_dq_bf16", "coarse_grad_reduce",
     "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32", "attn_bwd_coarse_bf16", "attn_bwd_dkdv_tc", "dkdv_empty_rows",
-    "dkdv_order_count", "dkdv_order_scatter"};
+    "dkdv_order_count", "dkdv_order_scatter", "zorder_permute"};
 
 struct TraceState {
   cudaEvent_t* ev = nullptr;
@@ -754,6 +756,25 @@ void llsa_plan_destroy(llsa_plan* plan) {
   if (plan->exec) cudaGraphExecDestroy(plan->exec);
   if (plan->graph) cudaGraphDestroy(plan->graph);
   delete plan;
+}
+
+llsa_status llsa_token_permute(const llsa_shape* s, const void* src, void* dst, int32_t to_z_order,
+                               llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  if (!src || !dst || !aligned16(src) || !aligned16(dst) || src == dst) return LLSA_ERR_INVALID_ARG;
+  const int lg = ilog2(s->N);
+  if (lg & 1) return LLSA_ERR_INVALID_ARG;  // N must be a square grid: side = 2^(lg/2)
+  const long long rows = (long long)s->B * s->H * s->N;
+  const int row_bytes = kD * (s->dtype == LLSA_BF16 ? 2 : 4);
+  const int pieces = row_bytes / 16;
+  const long long threads = rows * pieces;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  return launch(kKZOrder, cs, [&] {
+    launch_pdl(zorder_permute_kernel, dim3((unsigned)((threads + kZThreads - 1) / kZThreads)), dim3(kZThreads), 0,
+               cs, static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows, s->N, lg / 2, pieces,
+               to_z_order ? 1 : 0);
+  });
 }
 
 llsa_status llsa_device_status(int32_t* code_out, llsa_stream_t stream) {

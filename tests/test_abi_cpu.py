@@ -125,3 +125,12 @@ def test_flags_validated(lib):
         s.flags = bad
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 1, bad
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True).flags == _lib.LLSA_FLAG_LOG_BIAS
+
+
+def test_token_permute_rejected_before_launch(lib):
+    s = shape(levels=1, N=2048, topk=8)   # 2048 is not a square grid
+    assert lib.llsa_token_permute(ctypes.byref(s), 256, 512, 1, None) == 1
+    s = shape(levels=1, N=4096, topk=8)
+    assert lib.llsa_token_permute(ctypes.byref(s), 256, 256, 1, None) == 1   # in place
+    assert lib.llsa_token_permute(ctypes.byref(s), None, 256, 0, None) == 1
+    assert lib.llsa_token_permute(ctypes.byref(s), 264, 512, 0, None) == 1   # misaligned
