@@ -126,7 +126,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const float* __restrict__ k_pyr, const float* __restrict__ v_pyr, const int* __restrict__ idx,
     const __nv_bfloat16* __restrict__ o, const float* __restrict__ lse, __nv_bfloat16* __restrict__ dq_out,
     float* __restrict__ ws) {
-  pdl_enter();
+  pdl_launch_dependents();  // the coarse tiles come from the pyramid and the
+  // coarser selection levels, complete before the kernel ahead of this one started; they are
+  // staged before waiting for it
   extern __shared__ uint8_t dq_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     stage_coarse_rows(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
     __syncthreads();
   }
+  pdl_wait();
   const int first = cta_first + warp * kUnitBlocks;
   if (first >= total_blocks) return;  // warp-uniform; no CTA-wide barrier after this point
   const int nblk = min(kUnitBlocks, total_blocks - first);
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
                                                                   const int* __restrict__ idx,
                                                                   const float* __restrict__ lse,
                                                                   float* __restrict__ ws) {
-  pdl_enter();
+  pdl_launch_dependents();  // coarse rows are staged before waiting (see attn_fwd_bf16_kernel)
   extern __shared__ uint8_t co_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -442,6 +445,7 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
     mbar_fence_init();
   }
   __syncwarp();
+  pdl_wait();  // LSE and Delta (the pairs' inputs) come from the kernels ahead
   float dk[8][4], dv[8][4];
 #pragma unroll
   for (int n = 0; n < 8; ++n)
