@@ -491,7 +491,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
                                                                               const int* __restrict__ row_ptr,
                                                                               const int* __restrict__ col,
                                                                               float* __restrict__ ws) {
-  pdl_enter();
+  pdl_launch_dependents();  // the CSR (joined before this launch) and the selection are read
+  // before waiting; the partials, written by the kernel ahead, after
   __shared__ float2 red_k[kReduceWarps][32], red_v[kReduceWarps][32];
   __shared__ int slot_of[64];
   __shared__ int anc_of[64];
@@ -539,6 +540,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
       anc_of[e] = a;
     }
     __syncthreads();
+    pdl_wait();  // returns at once after the first chunk
     const int pairs = cnt * span;
     // four pairs per iteration: their loads are independent, the sums stay in pair order
     for (int p0 = warp * 4; p0 < pairs; p0 += kReduceWarps * 4) {
