@@ -126,9 +126,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const float* __restrict__ k_pyr, const float* __restrict__ v_pyr, const int* __restrict__ idx,
     const __nv_bfloat16* __restrict__ o, const float* __restrict__ lse, __nv_bfloat16* __restrict__ dq_out,
     float* __restrict__ ws) {
-  pdl_launch_dependents();  // the coarse tiles come from the pyramid and the
-  // coarser selection levels, complete before the kernel ahead of this one started; they are
-  // staged before waiting for it
+  // the coarse tiles come from the pyramid and the coarser selection levels, two or more
+  // kernels back, so they are staged before waiting for the kernel ahead (see pdl_wait)
   extern __shared__ uint8_t dq_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -151,6 +150,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     __syncthreads();
   }
   pdl_wait();
+  pdl_launch_dependents();
   const int first = cta_first + warp * kUnitBlocks;
   if (first >= total_blocks) return;  // warp-uniform; no CTA-wide barrier after this point
   const int nblk = min(kUnitBlocks, total_blocks - first);
@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
                                                                   const int* __restrict__ idx,
                                                                   const float* __restrict__ lse,
                                                                   float* __restrict__ ws) {
-  pdl_launch_dependents();  // coarse rows are staged before waiting (see attn_fwd_bf16_kernel)
+  // coarse rows are staged before waiting (two or more kernels back; see pdl_wait)
   extern __shared__ uint8_t co_smem_raw[];
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -446,6 +446,7 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
   }
   __syncwarp();
   pdl_wait();  // LSE and Delta (the pairs' inputs) come from the kernels ahead
+  pdl_launch_dependents();
   float dk[8][4], dv[8][4];
 #pragma unroll
   for (int n = 0; n < 8; ++n)
@@ -491,8 +492,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
                                                                               const int* __restrict__ row_ptr,
                                                                               const int* __restrict__ col,
                                                                               float* __restrict__ ws) {
-  pdl_launch_dependents();  // the CSR (joined before this launch) and the selection are read
-  // before waiting; the partials, written by the kernel ahead, after
+  // The CSR rows and the selection (two or more kernels back, or joined before this launch) are
+  // read before waiting; the partials, written by the kernel ahead, after (see pdl_wait).
   __shared__ float2 red_k[kReduceWarps][32], red_v[kReduceWarps][32];
   __shared__ int slot_of[64];
   __shared__ int anc_of[64];
@@ -525,6 +526,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
   const long long n2 = g.n[2];
   float2 sk = make_float2(0.f, 0.f), sv = make_float2(0.f, 0.f);
   // CSR rows are processed in chunks of 64 entries: slots first, then the (entry, group) pairs
+  bool waited = false;
   for (int c0 = rs; c0 < re; c0 += 64) {
     const int cnt = min(64, re - c0);
     __syncthreads();
@@ -540,7 +542,11 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
       anc_of[e] = a;
     }
     __syncthreads();
-    pdl_wait();  // returns at once after the first chunk
+    if (!waited) {
+      pdl_wait();
+      pdl_launch_dependents();
+      waited = true;
+    }
     const int pairs = cnt * span;
     // four pairs per iteration: their loads are independent, the sums stay in pair order
     for (int p0 = warp * 4; p0 < pairs; p0 += kReduceWarps * 4) {
@@ -566,6 +572,10 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
         sv.y += y[u].y;
       }
     }
+  }
+  if (!waited) {  // an empty row: nothing was read from the kernel ahead
+    pdl_wait();
+    pdl_launch_dependents();
   }
   red_k[warp][lane] = sk;
   red_v[warp][lane] = sv;

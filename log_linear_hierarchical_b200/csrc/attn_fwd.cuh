@@ -230,9 +230,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
                                                             const float* __restrict__ v_pyr,
                                                             const int* __restrict__ idx, __nv_bfloat16* __restrict__ o,
                                                             float* __restrict__ lse) {
-  pdl_launch_dependents();  // the coarse tiles come from the pyramid and the
-  // coarser selection levels, complete before the kernel ahead of this one started; they are
-  // staged before waiting for it
+  // the coarse tiles come from the pyramid and the coarser selection levels, two or more
+  // kernels back, so they are staged before waiting for the kernel ahead (see pdl_wait)
   extern __shared__ uint8_t fwd_smem_raw[];
   const Geometry& g = P.g;
   const int lane = lane_id();
@@ -254,6 +253,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     __syncthreads();
   }
   pdl_wait();
+  pdl_launch_dependents();
   const int first = cta_first + warp * kUnitBlocks;
   if (first >= total_blocks) return;  // warp-uniform; no CTA-wide barrier after this point
   const int nblk = min(kUnitBlocks, total_blocks - first);

@@ -165,10 +165,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Programmatic dependent launch.  Every kernel is launched with programmatic stream
 // serialization, so it may be scheduled before the kernel ahead of it on the stream has
 // finished.  pdl_wait blocks until that kernel has completed and its writes are visible
-// (it returns at once for a kernel launched without the attribute); no kernel touches
-// global memory before it, unless the kernel documents what it reads early.
+// (it returns at once for a kernel launched without the attribute).
 // pdl_launch_dependents lets the next kernel's CTAs be scheduled once every CTA of this
-// grid has issued it.
+// grid has issued it.  Every kernel issues it only after its own pdl_wait, so when a kernel
+// starts, the kernel two places ahead of it on the stream has completed.  A kernel may
+// therefore read, before its pdl_wait, only data written two or more kernels back or by
+// work joined to its stream with an event; each such early read is documented where it is.
+// (dK/dV, the last kernel of a step, signals before its deferred wait: the step's first
+// kernel reads nothing before its own wait.)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_enter() {
