@@ -149,10 +149,12 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     stage_coarse_rows(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
     __syncthreads();
   }
-  pdl_wait();
-  pdl_launch_dependents();
   const int first = cta_first + warp * kUnitBlocks;
-  if (first >= total_blocks) return;  // warp-uniform; no CTA-wide barrier after this point
+  if (first >= total_blocks) {  // warp-uniform; no CTA-wide barrier after this point
+    pdl_wait();
+    pdl_launch_dependents();
+    return;
+  }
   const int nblk = min(kUnitBlocks, total_blocks - first);
   const uint32_t qd = smem_u32(cs.tiles(base, warp));
   const uint32_t ring = qd + 4 * kTileBytes;
@@ -189,10 +191,13 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     tma_load_2d(dst + kTileBytes, &tm_do, 0, row, bar);
     bulk_load(smem_u32(slse + (i & 1) * kBlock), lse + row, kBlock * 4, bar);
   };
-  if (lane == 0) {
-    issue_qd(0);
+  // the level-1 selection (two kernels back) and K, V are ready: the first K/V tiles are
+  // requested before waiting; Q/dO/LSE and O follow the forward, the kernel ahead
+  if (lane == 0)
     for (int s = 0; s < min(STAGES, total_loads); ++s) issue_kv(s);
-  }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (lane == 0) issue_qd(0);
 
   bool ok = true;
   int next_seq = 0, next_q = 0;

@@ -155,11 +155,25 @@ bool allow_smem(Kern k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
 }
 
+// Set while a public call whose first kernel reads data before its pdl_wait (the forward,
+// and dQ in a build without the order phase) launches that kernel: the launch then goes
+// without the attribute, so it starts only once everything ahead of it on the caller's
+// stream has completed, whatever the caller launched there.  Inside a step the kernels
+// ahead are this library's own and the pdl_wait ordering rule covers the early reads.
+thread_local bool g_serial_next = false;
+
+struct SerialFirstLaunch {
+  SerialFirstLaunch() { g_serial_next = true; }
+  ~SerialFirstLaunch() { g_serial_next = false; }
+};
+
 // Launch with programmatic stream serialization (see pdl_wait): the kernel may be scheduled
 // while the one ahead of it on the stream drains; it waits for it on the device.  A failed
 // launch is reported by cudaGetLastError, as for a triple-chevron launch.
 template <typename... KArgs, typename... Args>
 void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t cs, Args&&... args) {
+  const bool serial = g_serial_next;
+  g_serial_next = false;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -169,7 +183,7 @@ void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cuda
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = serial ? 0 : 1;
   cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -498,6 +512,42 @@ llsa_status validate_step(const llsa_shape* s, const llsa_step_buffers* b) {
 // (forked after the selection, joined before the backward key side), or on `cs` if side
 // is null.  The join is made on every path once the fork was made, so a capture that
 // fails part-way still ends with both streams joined.
+// The forward launch shared by llsa_forward and the step.
+llsa_status forward_impl(const llsa_shape* s, const void* q, const void* k, const void* v, const float* k_pyr,
+                         const float* v_pyr, const int32_t* idx, void* o, float* lse, llsa_stream_t stream) {
+  llsa_status st = validate(s);
+  if (st != LLSA_OK) return st;
+  const void* ptrs[8] = {q, k, v, k_pyr, v_pyr, idx, o, lse};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const float scale = 1.0f / sqrtf((float)kD);
+  const int total_blocks = g.BH * g.n[1];
+  if (s->dtype == LLSA_BF16) {
+    CUtensorMap tq, tk, tv;
+    const long long rows = (long long)g.BH * g.N;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
+      return LLSA_ERR_CUDA;
+    AttnParams P{g, scale * kLog2e, scale};
+    const size_t smem = (size_t)fwd_smem<kFwdStages>(g, kAttnWarps).total();
+    auto kern = attn_fwd_bf16_kernel<kFwdStages>;
+    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+    const int per_cta = kAttnWarps * kUnitBlocks;
+    return launch(kKFwdBf16, cs, [&] {
+      launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, 
+          tq, tk, tv, P, k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse);
+    });
+  }
+  const size_t smem = simt_fwd_smem(g);
+  if (!allow_smem(attn_fwd_f32_kernel, smem)) return LLSA_ERR_CUDA;
+  return launch(kKFwdF32, cs, [&] {
+    launch_pdl(attn_fwd_f32_kernel, dim3(total_blocks), dim3(kSimtThreads), smem, cs, 
+        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
+        v_pyr, idx, static_cast<float*>(o), lse);
+  });
+}
+
 llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStream_t cs, cudaStream_t side) {
   // pooled levels >= 3 are made by the coarsest-selection launch when they are small
   const Geometry g = make_geometry(s);
@@ -522,7 +572,7 @@ llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStrea
                            b->dq, b->dk, b->dv, b->backward_workspace, kOrder, side);
     if (cudaEventRecord(join, side) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
   }
-  if (st == LLSA_OK) st = llsa_forward(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs);
+  if (st == LLSA_OK) st = forward_impl(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs);
   if (st == LLSA_OK)
     st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
                          b->dq, b->dk, b->dv, b->backward_workspace, kQuerySide, cs);
@@ -657,38 +707,10 @@ llsa_status llsa_index_transpose_noalloc(const llsa_shape* s, const int32_t* idx
 
 llsa_status llsa_forward(const llsa_shape* s, const void* q, const void* k, const void* v, const float* k_pyr,
                          const float* v_pyr, const int32_t* idx, void* o, float* lse, llsa_stream_t stream) {
-  llsa_status st = validate(s);
-  if (st != LLSA_OK) return st;
-  const void* ptrs[8] = {q, k, v, k_pyr, v_pyr, idx, o, lse};
-  for (const void* p : ptrs)
-    if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
-  const Geometry g = make_geometry(s);
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const float scale = 1.0f / sqrtf((float)kD);
-  const int total_blocks = g.BH * g.n[1];
-  if (s->dtype == LLSA_BF16) {
-    CUtensorMap tq, tk, tv;
-    const long long rows = (long long)g.BH * g.N;
-    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
-      return LLSA_ERR_CUDA;
-    AttnParams P{g, scale * kLog2e, scale};
-    const size_t smem = (size_t)fwd_smem<kFwdStages>(g, kAttnWarps).total();
-    auto kern = attn_fwd_bf16_kernel<kFwdStages>;
-    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
-    const int per_cta = kAttnWarps * kUnitBlocks;
-    return launch(kKFwdBf16, cs, [&] {
-      launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, 
-          tq, tk, tv, P, k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse);
-    });
-  }
-  const size_t smem = simt_fwd_smem(g);
-  if (!allow_smem(attn_fwd_f32_kernel, smem)) return LLSA_ERR_CUDA;
-  return launch(kKFwdF32, cs, [&] {
-    launch_pdl(attn_fwd_f32_kernel, dim3(total_blocks), dim3(kSimtThreads), smem, cs, 
-        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
-        v_pyr, idx, static_cast<float*>(o), lse);
-  });
+  SerialFirstLaunch serial;
+  return forward_impl(s, q, k, v, k_pyr, v_pyr, idx, o, lse, stream);
 }
+
 
 llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
@@ -700,6 +722,7 @@ llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, con
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
   if (workspace_bytes < (size_t)bwd_workspace_layout(make_geometry(s)).total * sizeof(float)) return LLSA_ERR_WORKSPACE;
+  SerialFirstLaunch serial;
   return backward_phases(s, q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace,
                          kOrder | kQuerySide | kKeySide, reinterpret_cast<cudaStream_t>(stream));
 }
