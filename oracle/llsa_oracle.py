@@ -45,6 +45,10 @@ Readings where the pages are silent (each one is also listed in the design notes
 * Enrichment variant, off by default (``log_bias=True``): a level-l coarse token's
   scaled score gets + ln(16^l), the log of the number of input tokens it averages, so
   that it carries the softmax mass of those tokens when they are all equal.
+* Enrichment variant, off by default (``all_top=True``): for L >= 2 the level-L part of
+  the list is every one of the n_L coarsest tokens, in index order, instead of the K the
+  level-L ancestor selected (levels 2..L-1 are unchanged, and so is the selection).
+  With L = 1 there are no coarse entries and the variant changes nothing.
 * Gradients: the selection and the pooled queries carry no gradient; coarse K/V
   tokens pass their gradient back to the input tokens through the mean-pool
   adjoint (each of the 16^l tokens under a level-l token receives 1/16^l of it).
@@ -175,37 +179,45 @@ def kv_sources(x: np.ndarray, x_pyr: list[np.ndarray]) -> tuple[np.ndarray, list
     return np.concatenate([p.astype(np.float64) for p in parts], axis=2), offsets
 
 
-def kv_index(p: int, bh: tuple[int, int], idx: list[np.ndarray], offsets: list[int]) -> np.ndarray:
+def kv_index(p: int, bh: tuple[int, int], idx: list[np.ndarray], offsets: list[int],
+             all_top: bool = False) -> np.ndarray:
     """Rows (into ``kv_sources``) of query block p's KV list: the 16 tokens of each
     selected level-1 block, then for l = 2..L the K level-l tokens selected by p's
-    level-l ancestor p // 16^(l-1)."""
+    level-l ancestor p // 16^(l-1).  With ``all_top`` the level-L part is instead every
+    level-L token 0..n_L-1."""
     b, h = bh
     L = len(idx)
     rows = [children(idx[0][b, h, p])]
     for lev in range(2, L + 1):
+        if all_top and lev == L:
+            rows.append(offsets[lev] + np.arange(idx[lev - 1].shape[2], dtype=np.int64))
+            continue
         anc = p // BLOCK ** (lev - 1)
         rows.append(offsets[lev] + idx[lev - 1][b, h, anc].astype(np.int64))
     return np.concatenate(rows)
 
 
-def kv_index_table(b: int, h: int, idx: list[np.ndarray], offsets: list[int]) -> np.ndarray:
+def kv_index_table(b: int, h: int, idx: list[np.ndarray], offsets: list[int], all_top: bool = False) -> np.ndarray:
     """[n_1, T] table of ``kv_index`` for every query block of (b, h)."""
     n1 = idx[0].shape[2]
-    return np.stack([kv_index(p, (b, h), idx, offsets) for p in range(n1)])
+    return np.stack([kv_index(p, (b, h), idx, offsets, all_top) for p in range(n1)])
 
 
-def kv_bias(topk: int, levels: int) -> np.ndarray:
+def kv_bias(topk: int, levels: int, n_top: int | None = None) -> np.ndarray:
     """Additive score bias of each KV-list entry under the log-count enrichment variant:
-    0 for the 16K fine tokens, ln(16^l) for each of the K level-l coarse tokens."""
+    0 for the 16K fine tokens, ln(16^l) for each of the K level-l coarse tokens.  With
+    ``n_top`` (the all-coarsest variant) the level-L part has n_top entries."""
     parts = [np.zeros(BLOCK * topk)]
     for lev in range(2, levels + 1):
-        parts.append(np.full(topk, lev * math.log(BLOCK)))
+        count = n_top if (n_top is not None and lev == levels) else topk
+        parts.append(np.full(count, lev * math.log(BLOCK)))
     return np.concatenate(parts)
 
 
 # ----------------------------------------------------------------------------- step 4: attention
 
-def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False):
+def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False,
+            all_top: bool = False):
     """Softmax attention of every query over its block's KV list.
 
     Returns (O [B, H, N, D], LSE [B, H, N]) in fp64.  For query i of block p with
@@ -214,6 +226,7 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias:
     ``kv_bias`` (ln(16^l) for a level-l coarse token).
     ``blocks`` (ascending level-1 block indices) restricts the work to those query
     blocks of every (b, h); the other rows of O and LSE are left as NaN.
+    ``all_top`` takes the all-coarsest KV list of ``kv_index``.
     """
     q = np.asarray(q, dtype=np.float64)
     B, H, N, D = q.shape
@@ -223,11 +236,12 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias:
     o = np.full((B, H, N, D), np.nan)
     lse = np.full((B, H, N), np.nan)
     scale = 1.0 / math.sqrt(D)
-    bias = kv_bias(idx[0].shape[-1], len(idx)) if log_bias else 0.0
+    n_top = idx[-1].shape[2] if all_top else None
+    bias = kv_bias(idx[0].shape[-1], len(idx), n_top) if log_bias else 0.0
     sel_blocks = np.arange(n1) if blocks is None else np.asarray(blocks, dtype=np.int64)
     for b in range(B):
         for h in range(H):
-            table = kv_index_table(b, h, idx, offsets)
+            table = kv_index_table(b, h, idx, offsets, all_top)
             qb = q[b, h].reshape(n1, BLOCK, D)
             for s0 in range(0, len(sel_blocks), chunk):
                 sl = sel_blocks[s0:s0 + chunk]
@@ -242,7 +256,8 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias:
     return o, lse
 
 
-def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False):
+def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False,
+             all_top: bool = False):
     """Exact gradient of the attention above with the selection held fixed.
 
     With P = softmax(z) on each query's list, Delta_i = sum_d dO_id O_id and
@@ -251,7 +266,8 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
     level-l tokens are then spread over their 16^l input tokens with weight 1/16^l
     (the adjoint of the mean pool).  Returns (dQ, dK, dV) [B, H, N, D] in fp64.
     ``blocks`` restricts the sum to those query blocks (dQ rows of the others are NaN).
-    ``log_bias`` as in ``forward`` (a constant bias leaves the gradient formulas as they are).
+    ``log_bias`` as in ``forward`` (a constant bias leaves the gradient formulas as they are);
+    ``all_top`` as in ``forward``.
     """
     q = np.asarray(q, dtype=np.float64)
     do = np.asarray(do, dtype=np.float64)
@@ -263,14 +279,15 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
     vsrc, _ = kv_sources(v, v_pyr)
     n1 = N // BLOCK
     scale = 1.0 / math.sqrt(D)
-    bias = kv_bias(idx[0].shape[-1], L) if log_bias else 0.0
+    n_top = idx[-1].shape[2] if all_top else None
+    bias = kv_bias(idx[0].shape[-1], L, n_top) if log_bias else 0.0
     dq = np.full((B, H, N, D), np.nan)
     dk = np.empty((B, H, N, D))
     dv = np.empty((B, H, N, D))
     sel_blocks = np.arange(n1) if blocks is None else np.asarray(blocks, dtype=np.int64)
     for b in range(B):
         for h in range(H):
-            table = kv_index_table(b, h, idx, offsets)
+            table = kv_index_table(b, h, idx, offsets, all_top)
             qb = q[b, h].reshape(n1, BLOCK, D)
             dob = do[b, h].reshape(n1, BLOCK, D)
             delta = (do[b, h] * o[b, h]).sum(axis=-1).reshape(n1, BLOCK)
@@ -375,17 +392,18 @@ def from_z_order(x: np.ndarray) -> np.ndarray:
 
 # ----------------------------------------------------------------------------- whole path
 
-def llsa_step(q, k, v, do, levels: int, topk: int, log_bias: bool = False):
+def llsa_step(q, k, v, do, levels: int, topk: int, log_bias: bool = False, all_top: bool = False):
     """Pyramid, selection, forward, backward and transposes with the oracle's own
     selection.  Inputs are exact widenings of the device inputs."""
     q_pyr = build_pyramid(q, levels)
     k_pyr = build_pyramid(k, levels)
     v_pyr = build_pyramid(v, levels)
     idx = select(q_pyr, k_pyr, topk)
-    o, lse = forward(q, k, v, k_pyr, v_pyr, idx, log_bias=log_bias)
+    o, lse = forward(q, k, v, k_pyr, v_pyr, idx, log_bias=log_bias, all_top=all_top)
     out = dict(q_pyr=q_pyr, k_pyr=k_pyr, v_pyr=v_pyr, idx=idx, o=o, lse=lse)
     if do is not None:
-        out["dq"], out["dk"], out["dv"] = backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, log_bias=log_bias)
+        out["dq"], out["dk"], out["dv"] = backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, log_bias=log_bias,
+                                                   all_top=all_top)
     out["row_ptr"], out["col"] = index_transpose_all(idx)
     return out
 

@@ -6,6 +6,12 @@ same vector, a level-l pooled token equals each of the 16^l input tokens it aver
 attention over the biased list must equal plain softmax attention (torch, fp64) over the
 explicit multiset in which each coarse token is repeated 16^l times.  Finite differences
 check the backward with the bias on.
+
+The all-coarsest variant (``all_top``) is pinned three ways: with K = n_L the level-L
+selection is already every coarsest token, so the variant must change nothing; with the
+bias and grouped K/V its level-L part stands for every input token, so the result is
+dense attention over the whole sequence plus the finer picks; finite differences and the
+sum invariants (sum dV = sum dO, sum dK = 0) check its backward.
 """
 import math
 
@@ -14,7 +20,8 @@ import pytest
 import torch
 import torch.nn.functional as F
 
-from oracle.llsa_oracle import (BLOCK, backward, build_pyramid, forward, kv_index, kv_sources, select)
+from oracle.llsa_oracle import (BLOCK, backward, build_pyramid, forward, kv_index, kv_sources, llsa_step,
+                                 select)
 
 
 def grouped(rng, B, H, N, D, group):
@@ -82,6 +89,83 @@ def test_log_bias_finite_differences_with_frozen_selection():
     picks = [(0, 0, 7, 1), (0, 0, 2049, 3), (0, 0, 8190, 0), (0, 0, 5000, 2)]
     for name, grad in (("q", dq), ("k", dk), ("v", dv)):
         for pos in picks:
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[name][pos] += eps
+            up = loss(args["q"], args["k"], args["v"])
+            args[name][pos] -= 2 * eps
+            dn = loss(args["q"], args["k"], args["v"])
+            fd = (up - dn) / (2 * eps)
+            assert abs(fd - grad[pos]) < 1e-7 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
+
+
+# ---------------------------------------------------------------- all-coarsest variant
+
+def test_all_top_equals_default_when_every_coarsest_token_is_selected():
+    # K = n_L: the level-L selection is already every coarsest token in index order
+    rng = np.random.default_rng(21)
+    B, H, N, D, L = 1, 2, 4096, 8, 2
+    K = N // BLOCK ** L
+    q, k, v, do = (rng.standard_normal((B, H, N, D)) for _ in range(4))
+    a = llsa_step(q, k, v, do, L, K)
+    b = llsa_step(q, k, v, do, L, K, all_top=True)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert np.array_equal(a[name], b[name]), name
+
+
+@pytest.mark.parametrize("N,L,K", [(4096, 2, 2), (8192, 3, 2)])
+def test_all_top_with_log_bias_is_dense_attention_plus_the_finer_picks(N, L, K):
+    # K and V constant over each coarsest-level group: a level-l token stands for 16^l equal
+    # input tokens, so with the bias the list is the multiset {selected fine tokens} +
+    # {each selected level-l token 16^l times, l < L} + {every input token} (all of level L)
+    rng = np.random.default_rng(22)
+    B, H, D = 1, 1, 8
+    group = BLOCK ** L
+    q = rng.standard_normal((B, H, N, D))
+    k = grouped(rng, B, H, N, D, group)
+    v = grouped(rng, B, H, N, D, group)
+    qp, kp, vp = (build_pyramid(x, L, np.float64) for x in (q, k, v))
+    idx = select(qp, kp, K)
+    o, lse = forward(q, k, v, kp, vp, idx, log_bias=True, all_top=True)
+    ksrc, offsets = kv_sources(k, kp)
+    vsrc, _ = kv_sources(v, vp)
+    for p in range(0, N // BLOCK, max(1, N // BLOCK // 16)):
+        fine = kv_index(p, (0, 0), idx, offsets)[:BLOCK * K]
+        parts_k, parts_v = [ksrc[0, 0][fine], k[0, 0]], [vsrc[0, 0][fine], v[0, 0]]
+        for lev in range(2, L):
+            rows = offsets[lev] + idx[lev - 1][0, 0, p // BLOCK ** (lev - 1)]
+            parts_k.append(np.repeat(ksrc[0, 0][rows], BLOCK ** lev, axis=0))
+            parts_v.append(np.repeat(vsrc[0, 0][rows], BLOCK ** lev, axis=0))
+        km = torch.tensor(np.concatenate(parts_k))[None, None]
+        vm = torch.tensor(np.concatenate(parts_v))[None, None]
+        qb = torch.tensor(q[0, 0, p * BLOCK:(p + 1) * BLOCK])[None, None]
+        ref = F.scaled_dot_product_attention(qb, km, vm)[0, 0].numpy()
+        ref_lse = torch.logsumexp(qb @ km.transpose(-1, -2) / math.sqrt(D), dim=-1)[0, 0].numpy()
+        assert np.abs(o[0, 0, p * BLOCK:(p + 1) * BLOCK] - ref).max() < 1e-12
+        assert np.abs(lse[0, 0, p * BLOCK:(p + 1) * BLOCK] - ref_lse).max() < 1e-11
+
+
+@pytest.mark.parametrize("log_bias", [False, True])
+def test_all_top_finite_differences_and_sums(log_bias):
+    rng = np.random.default_rng(23)
+    B, H, N, D, K, L = 1, 1, 8192, 4, 2, 3
+    q, k, v, do = (rng.standard_normal((B, H, N, D)) for _ in range(4))
+    idx = select(build_pyramid(q, L, np.float64), build_pyramid(k, L, np.float64), K)
+    kw = dict(log_bias=log_bias, all_top=True)
+
+    def loss(q_, k_, v_):
+        kp, vp = build_pyramid(k_, L, np.float64), build_pyramid(v_, L, np.float64)
+        o, _ = forward(q_, k_, v_, kp, vp, idx, **kw)
+        return float((o * do).sum())
+
+    kp, vp = build_pyramid(k, L, np.float64), build_pyramid(v, L, np.float64)
+    o, lse = forward(q, k, v, kp, vp, idx, **kw)
+    dq, dk, dv = backward(q, k, v, o, lse, do, kp, vp, idx, **kw)
+    # rows of P sum to 1 and the pooled adjoint keeps sums: sum dV = sum dO; sum_e dS = 0
+    assert np.abs(dv.sum(axis=2) - do.sum(axis=2)).max() < 1e-9
+    assert np.abs(dk.sum(axis=2)).max() < 1e-9
+    eps = 1e-6
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for pos in [(0, 0, 7, 1), (0, 0, 2049, 3), (0, 0, 8190, 0), (0, 0, 5000, 2)]:
             args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
             args[name][pos] += eps
             up = loss(args["q"], args["k"], args["v"])
