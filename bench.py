@@ -135,7 +135,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- algorithmic counts
 
-def workload_counts(cfg, pairs_l1: int):
+def workload_counts(cfg, pairs_l1: int, all_top: bool = False):
     """Algorithmic bytes and FLOPs per launch of each kernel for one step of ``cfg``.
 
     Per query block the forward gathers the KV list (T tokens x 64 channels x 2 bytes for K
@@ -149,7 +149,8 @@ def workload_counts(cfg, pairs_l1: int):
     bh = cfg.B * cfg.H
     n = cfg.level_sizes()
     n1 = n[1]
-    T = cfg.kv_len
+    coarse = coarse_entries(cfg, all_top)
+    T = 16 * cfg.topk + coarse
     blocks = bh * n1
     tile = 16 * D * e
     row_stream = 16 * 4
@@ -188,7 +189,6 @@ def workload_counts(cfg, pairs_l1: int):
     counts["dkdv_order_count"] = dict(bytes=bh * (n1 + 1) * 4, flops=0)
     counts["dkdv_order_scatter"] = dict(bytes=bh * (n1 + 1) * 4 + bh * n1 * 16, flops=0)
     if L >= 2:
-        coarse = (L - 1) * K
         ctas = bh * n[2] * ((coarse + 15) // 16)
         # per (level-2 group, coarse tile): 16 query blocks' Q, dO, LSE, Delta, the coarse K/V
         # rows (fp32), the fp32 partials written
@@ -200,9 +200,29 @@ def workload_counts(cfg, pairs_l1: int):
     return counts
 
 
+def coarse_entries(cfg, all_top: bool = False) -> int:
+    """Coarse KV entries per query block: (L-1) K, or (L-2) K + n_L for the all-coarsest variant."""
+    L, K = cfg.levels, cfg.topk
+    if L < 2:
+        return 0
+    return (L - 2) * K + cfg.level_sizes()[L] if all_top else (L - 1) * K
+
+
+def enrichment(args) -> dict:
+    """Keyword arguments of the enrichment variants chosen on the command line."""
+    return dict(log_bias=args.log_bias, all_top=args.all_top)
+
+
+def enrichment_text(args) -> str:
+    parts = ["log-count bias ln(16^l) on coarse scores" if args.log_bias else "unit weight"]
+    if args.all_top:
+        parts.append("all n_L coarsest tokens in every list")
+    return "; ".join(parts)
+
+
 # ----------------------------------------------------------------------------- oracle sample
 
-def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool = False):
+def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool = False, all_top: bool = False):
     """Time the CPU oracle on ``heads`` (b=0) heads of the workload: pyramid, selection and
     transpose for each whole head, forward and backward for ``nblocks`` query blocks per
     head (all blocks if None).  Returns (tokens/s extrapolated to the full workload, dict)."""
@@ -226,9 +246,9 @@ def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool =
             idx = orc.select(qp, kp, cfg.topk)
             orc.index_transpose_all(idx)
             t1 = time.perf_counter()
-            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks, log_bias=log_bias)
+            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top)
             if cfg.backward:
-                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks, log_bias=log_bias)
+                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top)
             t2 = time.perf_counter()
             t_fixed += t1 - t0
             t_attn += t2 - t1
@@ -257,7 +277,7 @@ def run_ours(args):
     host = make_config_inputs(cfg, with_do=True)
     pinned = {k: v.pin_memory() for k, v in host.items()}
     dev = {k: v.cuda(non_blocking=True) for k, v in pinned.items()}
-    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, log_bias=args.log_bias)
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, **enrichment(args))
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     stream = torch.cuda.current_stream()
 
@@ -338,7 +358,7 @@ def run_ours(args):
     # algorithmic roofline of the dominant kernel
     rps, _ = buf.csr_levels()
     pairs_l1 = int(rps[0][..., -1].sum().item())
-    counts = workload_counts(cfg, pairs_l1)
+    counts = workload_counts(cfg, pairs_l1, args.all_top)
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
     hbm_peak = peaks["hbm_gbs"] if peaks else 6650.0
@@ -442,7 +462,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, info = oracle_sample(cfg, host, heads=2, nblocks=None, log_bias=args.log_bias)
+        val, info = oracle_sample(cfg, host, heads=2, nblocks=None, **enrichment(args))
         cpu = {"value": round(val, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": (f"numpy fp64 oracle, 1 thread: pyramid, selection, transpose, forward and backward of "
                           f"heads (b=0, h=0..1), {info['seconds']:.1f} s, extrapolated to {cfg.B * cfg.H} heads")}
@@ -462,9 +482,10 @@ def run_ours(args):
         "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
         "data": "synthetic (seeded smooth-field Q/K in Z order, N(0,1) V and dO)",
         "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
-                   "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk, "kv_len": cfg.kv_len,
+                   "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk,
+                   "kv_len": 16 * cfg.topk + coarse_entries(cfg, args.all_top),
                    "step": "pyramid + select + forward + index transpose + backward",
-                   "enrichment": "log-count bias ln(16^l) on coarse scores" if args.log_bias else "unit weight",
+                   "enrichment": enrichment_text(args),
                    "launch": ("K steps as one CUDA graph (llsa_plan_create repeat=K), kernels chained by "
                               "programmatic dependent launch; transpose on a second stream"),
                    "kernel_times_from": ("a second plan of the same K steps with trace events around every "
@@ -531,14 +552,14 @@ def run_reference(args):
     n1 = cfg.N // 16
     # size each step's sample so that warm-up + steps stay near two minutes
     budget = 120.0 / max(1, args.steps + args.warmup)
-    _, probe = oracle_sample(cfg, host, heads=1, nblocks=16, log_bias=args.log_bias)
+    _, probe = oracle_sample(cfg, host, heads=1, nblocks=16, **enrichment(args))
     per_block = max(1e-6, probe["t_attn_per_block"])
     nblocks = int(max(16, min(n1, (budget - probe["t_fixed_per_head"]) / per_block)))
     for _ in range(args.warmup):
-        oracle_sample(cfg, host, heads=1, nblocks=nblocks, log_bias=args.log_bias)
+        oracle_sample(cfg, host, heads=1, nblocks=nblocks, **enrichment(args))
     vals, secs = [], 0.0
     for _ in range(args.steps):
-        v, info = oracle_sample(cfg, host, heads=1, nblocks=nblocks, log_bias=args.log_bias)
+        v, info = oracle_sample(cfg, host, heads=1, nblocks=nblocks, **enrichment(args))
         vals.append(v)
         secs += info["seconds"]
     value = statistics.median(vals)
@@ -570,7 +591,7 @@ def run_profile(args):
     cfg = CONFIGS[args.config]
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     dev = {k: v.cuda() for k, v in make_config_inputs(cfg, with_do=True).items()}
-    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, log_bias=args.log_bias)
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, **enrichment(args))
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     for _ in range(args.warmup + args.steps):
         api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
@@ -592,6 +613,8 @@ def main():
     ap.add_argument("--profile", action="store_true", help="run only the steps (for ncu), print no metric")
     ap.add_argument("--log-bias", action="store_true",
                     help="the log-count enrichment variant (ln 16^l on level-l coarse scores)")
+    ap.add_argument("--all-top", action="store_true",
+                    help="the all-coarsest enrichment variant (every level-L token in every list)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

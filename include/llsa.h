@@ -83,6 +83,15 @@ typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
  * carries their softmax mass when they are all equal.  Default 0: unit-weight entries.
  */
 #define LLSA_FLAG_LOG_BIAS 1
+/*
+ * Enrichment variant: with LLSA_FLAG_ALL_TOP (and levels >= 2) the level-L part of every
+ * query block's KV list is all n_L coarsest tokens, in index order, instead of the K that
+ * the block's level-L ancestor selected; levels 2..L-1 and the selection are unchanged.
+ * The list then has C = (L-2) K + n_L coarse entries; C > 96 -> LLSA_ERR_UNSUPPORTED.  It
+ * combines with LLSA_FLAG_LOG_BIAS.  The level-L rows of the index transpose are still
+ * produced (the backward does not need them).
+ */
+#define LLSA_FLAG_ALL_TOP 2
 
 typedef struct {
   int32_t B, H, N, D;
@@ -90,7 +99,7 @@ typedef struct {
   int32_t topk;    /* K, a power of two */
   int32_t levels;  /* L, number of pooled levels; llsa_l1 <-> 1, llsa_l2 <-> 2 */
   int32_t dtype;   /* llsa_dtype of q, k, v, o, dO, dq, dk, dv */
-  int32_t flags;   /* 0 or LLSA_FLAG_LOG_BIAS; other bits -> LLSA_ERR_INVALID_ARG */
+  int32_t flags;   /* LLSA_FLAG_* bits (0: the default enrichment); others -> INVALID_ARG */
 } llsa_shape;
 
 /* Static text for a status code. */

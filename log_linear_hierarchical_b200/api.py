@@ -28,10 +28,12 @@ class LLSAError(RuntimeError):
 
 
 def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16,
-               log_bias: bool = False) -> LLSAShape:
-    """``log_bias``: the log-count enrichment variant (LLSA_FLAG_LOG_BIAS)."""
+               log_bias: bool = False, all_top: bool = False) -> LLSAShape:
+    """``log_bias``: the log-count enrichment variant (LLSA_FLAG_LOG_BIAS); ``all_top``: the
+    all-coarsest variant (LLSA_FLAG_ALL_TOP).  Both may be set."""
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
-    return LLSAShape(B, H, N, D, block, topk, levels, code, _lib.LLSA_FLAG_LOG_BIAS if log_bias else 0)
+    flags = (_lib.LLSA_FLAG_LOG_BIAS if log_bias else 0) | (_lib.LLSA_FLAG_ALL_TOP if all_top else 0)
+    return LLSAShape(B, H, N, D, block, topk, levels, code, flags)
 
 
 def _check(fn: str, status: int) -> None:

@@ -416,19 +416,15 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
 
   // stage this tile's 16 coarse K and V rows (bf16) like the forward does
   {
-    const int K = g.K;
     for (int t = lane; t < kBlock * 8; t += 32) {
       const int r = t >> 3;
       const int ch = t & 7;
       const int row = tile * kBlock + r;
       uint4 pk = make_uint4(0u, 0u, 0u, 0u), pv = make_uint4(0u, 0u, 0u, 0u);
       if (row < g.coarse) {
-        const int lev = 2 + row / K;
-        const int slot = row - (lev - 2) * K;
-        int span = 1;
-        for (int i = 1; i < lev; ++i) span *= kBlock;
+        int lev;
+        const int j = coarse_token(g, idx, bh, p0, row, lev);
         const int nl = g.n[lev];
-        const int j = checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + p0 / span) * K + slot), nl);
         const long long off = g.pyr_off[lev] + ((long long)bh * nl + j) * kD + ch * 8;
         const float4 a = __ldg(reinterpret_cast<const float4*>(k_pyr + off));
         const float4 b = __ldg(reinterpret_cast<const float4*>(k_pyr + off) + 1);
@@ -488,6 +484,8 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
 
 // Per coarse level-l token j (one CTA of kReduceWarps warps each): the sum of the group
 // partials of every level-l query a in CSR row j, over the 16^(l-2) level-2 groups under a.
+// In the level-L part of the all-coarsest variant every level-L query a lists j (at entry
+// top_first + j), so the row is a = 0..n_L-1 and the CSR is not read.
 // The (a, group) pairs are dealt round-robin to the warps; the warps' sums are added in warp
 // order, so the result does not depend on timing.
 constexpr int kReduceWarps = 8;
@@ -519,10 +517,11 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
   const int j = (int)(cid - (long long)bh * nl);
   int span = 1;  // level-2 groups under one level-l token: 16^(l-2)
   for (int i = 2; i < lev; ++i) span *= kBlock;
+  const bool dense = lev >= g.L && g.top_first < g.coarse;  // all-coarsest level-L part
   const int* rp = row_ptr + g.rp_off[lev] + (long long)bh * (nl + 1);
   const int E = nl * K;
-  int rs = rp[j], re = rp[j + 1];
-  if (rs < 0 || re > E || rs > re) {
+  int rs = dense ? 0 : rp[j], re = dense ? nl : rp[j + 1];
+  if (!dense && (rs < 0 || re > E || rs > re)) {
     if (threadIdx.x == 0) record_error(LLSA_ERR_INTERNAL);
     rs = re = 0;
   }
@@ -536,6 +535,11 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
     const int cnt = min(64, re - c0);
     __syncthreads();
     for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
+      if (dense) {
+        slot_of[e] = g.top_first + j;
+        anc_of[e] = c0 + e;
+        continue;
+      }
       const int a = checked_index(__ldg(cl + c0 + e), nl);
       int lo = 0, hi = K - 1;  // slot of j in the ascending list of a
       while (lo < hi) {

@@ -70,25 +70,20 @@ __device__ __forceinline__ void mma_a_b(float (&acc)[8][4], uint32_t a0, uint32_
   }
 }
 
-// Stage (L-1)K coarse rows of a pyramid (fp32) as bf16 16-row swizzled tiles; padding rows
-// (index >= C) are zero.  Row c is level 2 + c / K, slot c % K of the ancestor's list.
+// Stage the C coarse rows of a pyramid (fp32) as bf16 16-row swizzled tiles; padding rows
+// (index >= C) are zero.  Row c is the pyramid row of coarse entry c (see coarse_token).
 // Threads `tid` = 0..nthreads-1 share the work (a warp or a whole CTA).
 __device__ __forceinline__ void stage_coarse_rows(const Geometry& g, const float* __restrict__ pyr,
                                                   const int* __restrict__ idx, int bh, int p, uint32_t dst, int tid,
                                                   int nthreads) {
-  const int K = g.K;
   for (int t = tid; t < g.coarse_pad * 8; t += nthreads) {
     const int row = t >> 3;
     const int ch = t & 7;
     uint4 packed = make_uint4(0u, 0u, 0u, 0u);
     if (row < g.coarse) {
-      const int lev = 2 + row / K;
-      const int slot = row - (lev - 2) * K;
-      int span = 1;
-      for (int i = 1; i < lev; ++i) span *= kBlock;      // 16^(lev-1)
-      const int anc = p / span;
+      int lev;
+      const int j = coarse_token(g, idx, bh, p, row, lev);
       const int nl = g.n[lev];
-      const int j = checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + anc) * K + slot), nl);
       const float4* src = reinterpret_cast<const float4*>(pyr + g.pyr_off[lev] + ((long long)bh * nl + j) * kD + ch * 8);
       const float4 x = __ldg(src);
       const float4 y = __ldg(src + 1);

@@ -11,7 +11,7 @@ namespace llsa {
 
 constexpr int kSimtThreads = 128;
 
-// Row pointers of block p's KV list: 16K fine tokens then (L-1)K coarse pyramid rows.
+// Row pointers of block p's KV list: 16K fine tokens then the C coarse pyramid rows.
 __device__ __forceinline__ void simt_kv_rows(const Geometry& g, int bh, int p, const float* __restrict__ k,
                                              const float* __restrict__ v, const float* __restrict__ k_pyr,
                                              const float* __restrict__ v_pyr, const int* __restrict__ idx,
@@ -29,14 +29,9 @@ __device__ __forceinline__ void simt_kv_rows(const Geometry& g, int bh, int p, c
       kb = k;
       vb = v;
     } else {
-      const int c = e - kBlock * K;
-      const int lev = 2 + c / K;
-      const int slot = c - (lev - 2) * K;
-      int span = 1;
-      for (int i = 1; i < lev; ++i) span *= kBlock;
-      const int nl = g.n[lev];
-      const int jj = checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + p / span) * K + slot), nl);
-      r = (long long)bh * nl + jj;
+      int lev;
+      const int jj = coarse_token(g, idx, bh, p, e - kBlock * K, lev);
+      r = (long long)bh * g.n[lev] + jj;
       kb = k_pyr + g.pyr_off[lev];
       vb = v_pyr + g.pyr_off[lev];
     }

@@ -39,7 +39,7 @@ llsa_status validate(const llsa_shape* s) {
   if (s->B < 1 || s->H < 1 || s->N < 1 || s->D < 1 || s->block < 1 || s->topk < 1 || s->levels < 1)
     return LLSA_ERR_INVALID_ARG;
   if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
-  if (s->flags & ~LLSA_FLAG_LOG_BIAS) return LLSA_ERR_INVALID_ARG;  // unknown flag bits
+  if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP)) return LLSA_ERR_INVALID_ARG;  // unknown flag bits
   if (!is_pow2(s->N) || !is_pow2(s->topk)) return LLSA_ERR_INVALID_ARG;  // README usage notes
   if (s->block != kBlock) return LLSA_ERR_UNSUPPORTED;
   if (s->D != kD) return LLSA_ERR_UNSUPPORTED;
@@ -51,6 +51,8 @@ llsa_status validate(const llsa_shape* s) {
   if (nL > 16384) return LLSA_ERR_UNSUPPORTED;
   if (s->topk > 64) return LLSA_ERR_UNSUPPORTED;
   if ((long long)(s->levels - 1) * s->topk > 32) return LLSA_ERR_UNSUPPORTED;
+  if ((s->flags & LLSA_FLAG_ALL_TOP) && s->levels >= 2 && (long long)(s->levels - 2) * s->topk + nL > 96)
+    return LLSA_ERR_UNSUPPORTED;  // the coarse entries of the all-coarsest variant
   if ((long long)s->B * s->H * s->N >= (1LL << 31)) return LLSA_ERR_UNSUPPORTED;
   return LLSA_OK;
 }
@@ -76,9 +78,11 @@ Geometry make_geometry(const llsa_shape* s) {
   }
   g.log_k = ilog2(g.K);
   g.log_n1 = ilog2(g.n[1]);
-  g.coarse = (g.L - 1) * g.K;
+  const bool all_top = (s->flags & LLSA_FLAG_ALL_TOP) && g.L >= 2;
+  g.coarse = all_top ? (g.L - 2) * g.K + g.n[g.L] : (g.L - 1) * g.K;
   g.coarse_pad = (g.coarse + kBlock - 1) / kBlock * kBlock;
   g.log_bias = (s->flags & LLSA_FLAG_LOG_BIAS) ? 1 : 0;
+  g.top_first = all_top ? (g.L - 2) * g.K : g.coarse;
   return g;
 }
 

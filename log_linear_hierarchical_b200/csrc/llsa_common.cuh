@@ -55,16 +55,25 @@ struct Geometry {
   long long pyr_off[kMaxLevels + 1];     // element offset of level l (1..L) in a pyramid
   long long idx_off[kMaxLevels + 1];     // element offset of level l in idx / col
   long long rp_off[kMaxLevels + 1];      // element offset of level l in row_ptr
-  int coarse;                            // C = (L-1) K coarse KV entries per query block
+  int coarse;                            // C coarse KV entries per query block: (L-1) K,
+                                         // or (L-2) K + n_L under LLSA_FLAG_ALL_TOP
   int coarse_pad;                        // C rounded up to a multiple of 16
   int log_bias;                          // LLSA_FLAG_LOG_BIAS: coarse scores + ln(16^l)
+  int top_first;                         // LLSA_FLAG_ALL_TOP (L >= 2): (L-2) K, the first
+                                         // entry of the level-L part; C (never reached) otherwise
 };
 
-// Additive score bias of coarse entry c (0 <= c < C, level 2 + c / K) under the log-count
-// enrichment variant, in units of the scaled score: ln(16^l) = l ln 16; 0 when it is off.
+// Level of coarse entry c (0 <= c < C): 2 + c / K, except that under the all-coarsest
+// variant the entries from top_first on are level L.
+__host__ __device__ inline int coarse_level(const Geometry& g, int c) {
+  return c >= g.top_first ? g.L : 2 + (c >> g.log_k);  // K = 2^log_k
+}
+
+// Additive score bias of coarse entry c under the log-count enrichment variant, in units
+// of the scaled score: ln(16^l) = l ln 16 for a level-l entry; 0 when it is off.
 constexpr float kLn16 = 2.7725887222397811f;
 __host__ __device__ inline float coarse_log_bias(const Geometry& g, int c) {
-  return g.log_bias ? (float)(2 + (c >> g.log_k)) * kLn16 : 0.0f;  // K = 2^log_k
+  return g.log_bias ? (float)coarse_level(g, c) * kLn16 : 0.0f;
 }
 
 // ---------------------------------------------------------------------------- status word
@@ -83,6 +92,21 @@ __device__ __forceinline__ int checked_index(int v, int n) {
     return 0;
   }
   return v;
+}
+
+// Token index (in its level) of coarse entry c of level-1 query block p of head bh: slot
+// c % K of the list that p's level-l ancestor selected, or, in the level-L part of the
+// all-coarsest variant, token c - top_first.  The index read from `idx` is range-checked.
+__device__ __forceinline__ int coarse_token(const Geometry& g, const int* __restrict__ idx, int bh, int p, int c,
+                                            int& lev) {
+  if (c >= g.top_first) {
+    lev = g.L;
+    return c - g.top_first;
+  }
+  lev = 2 + (c >> g.log_k);
+  const int nl = g.n[lev];
+  const int anc = p >> (4 * (lev - 1));  // p / 16^(l-1)
+  return checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + anc) * g.K + (c & (g.K - 1))), nl);
 }
 
 // ---------------------------------------------------------------------------- smem / swizzle

@@ -119,12 +119,29 @@ def test_step_and_plan_rejected_before_launch(lib):
 
 def test_flags_validated(lib):
     s = shape()
-    s.flags = 1  # LLSA_FLAG_LOG_BIAS
-    assert lib.llsa_validate_shape(ctypes.byref(s)) == 0
-    for bad in (2, 4, 1 << 30, -1):
+    for good in (1, 2, 3):  # LLSA_FLAG_LOG_BIAS, LLSA_FLAG_ALL_TOP, both
+        s.flags = good
+        assert lib.llsa_validate_shape(ctypes.byref(s)) == 0, good
+    for bad in (4, 8, 1 << 30, -1):
         s.flags = bad
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 1, bad
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True).flags == _lib.LLSA_FLAG_LOG_BIAS
+    assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True, all_top=True).flags == 3
+
+
+def test_all_top_coarse_limit(lib):
+    # C = (L-2) K + n_L coarse entries; more than 96 is unsupported
+    cases = [((262144, 3, 16), 0),    # C = 16 + 64
+             ((16384, 2, 8), 0),      # C = 64
+             ((65536, 2, 8), 2),      # C = 256
+             ((1 << 20, 3, 16), 2),   # C = 16 + 256
+             ((1 << 20, 4, 8), 0),    # C = 16 + 16
+             ((4096, 1, 8), 0)]       # L = 1: no coarse entries
+    for (N, L, K), want in cases:
+        s = api.make_shape(1, 1, N, 64, K, L, 0, all_top=True)
+        assert lib.llsa_validate_shape(ctypes.byref(s)) == want, (N, L, K)
+        s.flags = 0
+        assert lib.llsa_validate_shape(ctypes.byref(s)) == 0, (N, L, K)
 
 
 def test_token_permute_rejected_before_launch(lib):
