@@ -49,6 +49,11 @@ Readings where the pages are silent (each one is also listed in the design notes
   the list is every one of the n_L coarsest tokens, in index order, instead of the K the
   level-L ancestor selected (levels 2..L-1 are unchanged, and so is the selection).
   With L = 1 there are no coarse entries and the variant changes nothing.
+* Enrichment variant, off by default (``level1=True``): the list also holds the level-1
+  pooled token of each of the K selected fine blocks (the block's mean K and V), placed
+  after the fine tokens; with ``log_bias`` those entries get + ln 16.  Their gradient
+  goes back to the block's 16 input tokens through the mean-pool adjoint like any other
+  pooled token's.
 * Gradients: the selection and the pooled queries carry no gradient; coarse K/V
   tokens pass their gradient back to the input tokens through the mean-pool
   adjoint (each of the 16^l tokens under a level-l token receives 1/16^l of it).
@@ -166,13 +171,13 @@ def select(q_pyr: list[np.ndarray], k_pyr: list[np.ndarray], topk: int) -> list[
 
 def kv_sources(x: np.ndarray, x_pyr: list[np.ndarray]) -> tuple[np.ndarray, list[int]]:
     """Stack, per (b, h), the attended token sources: the input tokens (level 0) followed
-    by the pooled levels 2..L.  Returns the stacked [B, H, rows, D] array and the row
-    offset of each level (offset[0] = 0, offset[1] unused, offset[l] for l >= 2)."""
+    by the pooled levels 1..L.  Returns the stacked [B, H, rows, D] array and the row
+    offset of each level (offset[0] = 0, offset[l] for l >= 1)."""
     L = len(x_pyr)
     parts = [np.asarray(x)]
-    offsets = [0, -1]
+    offsets = [0]
     rows = x.shape[2]
-    for lev in range(2, L + 1):
+    for lev in range(1, L + 1):
         offsets.append(rows)
         parts.append(x_pyr[lev - 1])
         rows += x_pyr[lev - 1].shape[2]
@@ -180,14 +185,17 @@ def kv_sources(x: np.ndarray, x_pyr: list[np.ndarray]) -> tuple[np.ndarray, list
 
 
 def kv_index(p: int, bh: tuple[int, int], idx: list[np.ndarray], offsets: list[int],
-             all_top: bool = False) -> np.ndarray:
+             all_top: bool = False, level1: bool = False) -> np.ndarray:
     """Rows (into ``kv_sources``) of query block p's KV list: the 16 tokens of each
     selected level-1 block, then for l = 2..L the K level-l tokens selected by p's
     level-l ancestor p // 16^(l-1).  With ``all_top`` the level-L part is instead every
-    level-L token 0..n_L-1."""
+    level-L token 0..n_L-1; with ``level1`` the level-1 pooled tokens of the K selected
+    blocks follow the fine tokens."""
     b, h = bh
     L = len(idx)
     rows = [children(idx[0][b, h, p])]
+    if level1:
+        rows.append(offsets[1] + idx[0][b, h, p].astype(np.int64))
     for lev in range(2, L + 1):
         if all_top and lev == L:
             rows.append(offsets[lev] + np.arange(idx[lev - 1].shape[2], dtype=np.int64))
@@ -197,17 +205,21 @@ def kv_index(p: int, bh: tuple[int, int], idx: list[np.ndarray], offsets: list[i
     return np.concatenate(rows)
 
 
-def kv_index_table(b: int, h: int, idx: list[np.ndarray], offsets: list[int], all_top: bool = False) -> np.ndarray:
+def kv_index_table(b: int, h: int, idx: list[np.ndarray], offsets: list[int], all_top: bool = False,
+                   level1: bool = False) -> np.ndarray:
     """[n_1, T] table of ``kv_index`` for every query block of (b, h)."""
     n1 = idx[0].shape[2]
-    return np.stack([kv_index(p, (b, h), idx, offsets, all_top) for p in range(n1)])
+    return np.stack([kv_index(p, (b, h), idx, offsets, all_top, level1) for p in range(n1)])
 
 
-def kv_bias(topk: int, levels: int, n_top: int | None = None) -> np.ndarray:
+def kv_bias(topk: int, levels: int, n_top: int | None = None, level1: bool = False) -> np.ndarray:
     """Additive score bias of each KV-list entry under the log-count enrichment variant:
     0 for the 16K fine tokens, ln(16^l) for each of the K level-l coarse tokens.  With
-    ``n_top`` (the all-coarsest variant) the level-L part has n_top entries."""
+    ``n_top`` (the all-coarsest variant) the level-L part has n_top entries; with
+    ``level1`` the K level-1 pooled entries after the fine tokens get ln 16."""
     parts = [np.zeros(BLOCK * topk)]
+    if level1:
+        parts.append(np.full(topk, math.log(BLOCK)))
     for lev in range(2, levels + 1):
         count = n_top if (n_top is not None and lev == levels) else topk
         parts.append(np.full(count, lev * math.log(BLOCK)))
@@ -217,7 +229,7 @@ def kv_bias(topk: int, levels: int, n_top: int | None = None) -> np.ndarray:
 # ----------------------------------------------------------------------------- step 4: attention
 
 def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False,
-            all_top: bool = False):
+            all_top: bool = False, level1: bool = False):
     """Softmax attention of every query over its block's KV list.
 
     Returns (O [B, H, N, D], LSE [B, H, N]) in fp64.  For query i of block p with
@@ -226,7 +238,7 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias:
     ``kv_bias`` (ln(16^l) for a level-l coarse token).
     ``blocks`` (ascending level-1 block indices) restricts the work to those query
     blocks of every (b, h); the other rows of O and LSE are left as NaN.
-    ``all_top`` takes the all-coarsest KV list of ``kv_index``.
+    ``all_top`` and ``level1`` select the enrichment variants of ``kv_index``.
     """
     q = np.asarray(q, dtype=np.float64)
     B, H, N, D = q.shape
@@ -237,11 +249,11 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias:
     lse = np.full((B, H, N), np.nan)
     scale = 1.0 / math.sqrt(D)
     n_top = idx[-1].shape[2] if all_top else None
-    bias = kv_bias(idx[0].shape[-1], len(idx), n_top) if log_bias else 0.0
+    bias = kv_bias(idx[0].shape[-1], len(idx), n_top, level1) if log_bias else 0.0
     sel_blocks = np.arange(n1) if blocks is None else np.asarray(blocks, dtype=np.int64)
     for b in range(B):
         for h in range(H):
-            table = kv_index_table(b, h, idx, offsets, all_top)
+            table = kv_index_table(b, h, idx, offsets, all_top, level1)
             qb = q[b, h].reshape(n1, BLOCK, D)
             for s0 in range(0, len(sel_blocks), chunk):
                 sl = sel_blocks[s0:s0 + chunk]
@@ -257,7 +269,7 @@ def forward(q, k, v, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias:
 
 
 def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=None, log_bias: bool = False,
-             all_top: bool = False):
+             all_top: bool = False, level1: bool = False):
     """Exact gradient of the attention above with the selection held fixed.
 
     With P = softmax(z) on each query's list, Delta_i = sum_d dO_id O_id and
@@ -267,7 +279,7 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
     (the adjoint of the mean pool).  Returns (dQ, dK, dV) [B, H, N, D] in fp64.
     ``blocks`` restricts the sum to those query blocks (dQ rows of the others are NaN).
     ``log_bias`` as in ``forward`` (a constant bias leaves the gradient formulas as they are);
-    ``all_top`` as in ``forward``.
+    ``all_top`` and ``level1`` as in ``forward``.
     """
     q = np.asarray(q, dtype=np.float64)
     do = np.asarray(do, dtype=np.float64)
@@ -280,14 +292,14 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
     n1 = N // BLOCK
     scale = 1.0 / math.sqrt(D)
     n_top = idx[-1].shape[2] if all_top else None
-    bias = kv_bias(idx[0].shape[-1], L, n_top) if log_bias else 0.0
+    bias = kv_bias(idx[0].shape[-1], L, n_top, level1) if log_bias else 0.0
     dq = np.full((B, H, N, D), np.nan)
     dk = np.empty((B, H, N, D))
     dv = np.empty((B, H, N, D))
     sel_blocks = np.arange(n1) if blocks is None else np.asarray(blocks, dtype=np.int64)
     for b in range(B):
         for h in range(H):
-            table = kv_index_table(b, h, idx, offsets, all_top)
+            table = kv_index_table(b, h, idx, offsets, all_top, level1)
             qb = q[b, h].reshape(n1, BLOCK, D)
             dob = do[b, h].reshape(n1, BLOCK, D)
             delta = (do[b, h] * o[b, h]).sum(axis=-1).reshape(n1, BLOCK)
@@ -311,7 +323,7 @@ def backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, chunk: int = 256, blocks=No
                     dvsrc[rows[i]] += dve[i]
             gk = dksrc[:N].copy()
             gv = dvsrc[:N].copy()
-            for lev in range(2, L + 1):
+            for lev in range(1, L + 1):   # level 1 is attended only under ``level1``
                 n_l = N // BLOCK ** lev
                 span = BLOCK ** lev
                 ck = dksrc[offsets[lev]:offsets[lev] + n_l]
@@ -392,18 +404,19 @@ def from_z_order(x: np.ndarray) -> np.ndarray:
 
 # ----------------------------------------------------------------------------- whole path
 
-def llsa_step(q, k, v, do, levels: int, topk: int, log_bias: bool = False, all_top: bool = False):
+def llsa_step(q, k, v, do, levels: int, topk: int, log_bias: bool = False, all_top: bool = False,
+              level1: bool = False):
     """Pyramid, selection, forward, backward and transposes with the oracle's own
     selection.  Inputs are exact widenings of the device inputs."""
     q_pyr = build_pyramid(q, levels)
     k_pyr = build_pyramid(k, levels)
     v_pyr = build_pyramid(v, levels)
     idx = select(q_pyr, k_pyr, topk)
-    o, lse = forward(q, k, v, k_pyr, v_pyr, idx, log_bias=log_bias, all_top=all_top)
+    o, lse = forward(q, k, v, k_pyr, v_pyr, idx, log_bias=log_bias, all_top=all_top, level1=level1)
     out = dict(q_pyr=q_pyr, k_pyr=k_pyr, v_pyr=v_pyr, idx=idx, o=o, lse=lse)
     if do is not None:
         out["dq"], out["dk"], out["dv"] = backward(q, k, v, o, lse, do, k_pyr, v_pyr, idx, log_bias=log_bias,
-                                                   all_top=all_top)
+                                                   all_top=all_top, level1=level1)
     out["row_ptr"], out["col"] = index_transpose_all(idx)
     return out
 

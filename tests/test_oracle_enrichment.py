@@ -12,6 +12,12 @@ selection is already every coarsest token, so the variant must change nothing; w
 bias and grouped K/V its level-L part stands for every input token, so the result is
 dense attention over the whole sequence plus the finer picks; finite differences and the
 sum invariants (sum dV = sum dO, sum dK = 0) check its backward.
+
+The level-1 variant (``level1``: each selected block's pooled token joins the list) is
+pinned by dense attention over the tokens and the block means when every block is
+selected (L = 1, K = n_1), by the multiset in which, with the bias, each selected block
+counts twice, and by finite differences and the sum invariants, alone and with both other
+variants.
 """
 import math
 
@@ -161,6 +167,86 @@ def test_all_top_finite_differences_and_sums(log_bias):
     o, lse = forward(q, k, v, kp, vp, idx, **kw)
     dq, dk, dv = backward(q, k, v, o, lse, do, kp, vp, idx, **kw)
     # rows of P sum to 1 and the pooled adjoint keeps sums: sum dV = sum dO; sum_e dS = 0
+    assert np.abs(dv.sum(axis=2) - do.sum(axis=2)).max() < 1e-9
+    assert np.abs(dk.sum(axis=2)).max() < 1e-9
+    eps = 1e-6
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for pos in [(0, 0, 7, 1), (0, 0, 2049, 3), (0, 0, 16380, 0), (0, 0, 9000, 2)]:
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[name][pos] += eps
+            up = loss(args["q"], args["k"], args["v"])
+            args[name][pos] -= 2 * eps
+            dn = loss(args["q"], args["k"], args["v"])
+            fd = (up - dn) / (2 * eps)
+            assert abs(fd - grad[pos]) < 1e-7 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
+
+
+# ---------------------------------------------------------------- level-1 pooled tokens
+
+def test_level1_with_every_block_selected_is_dense_attention_over_tokens_and_block_means():
+    # L = 1 and K = n_1: every block is selected, so the list is every input token plus
+    # every level-1 pooled token: dense attention over the concatenation [K; K^(1)]
+    rng = np.random.default_rng(41)
+    B, H, N, D = 1, 2, 256, 8
+    K = N // BLOCK
+    q, k, v = (rng.standard_normal((B, H, N, D)) for _ in range(3))
+    out = llsa_step(q, k, v, None, 1, K, level1=True)
+    for h in range(H):
+        kc = torch.tensor(np.concatenate([k[0, h], out["k_pyr"][0][0, h].astype(np.float64)]))[None, None]
+        vc = torch.tensor(np.concatenate([v[0, h], out["v_pyr"][0][0, h].astype(np.float64)]))[None, None]
+        qt = torch.tensor(q[0, h])[None, None]
+        ref = F.scaled_dot_product_attention(qt, kc, vc)[0, 0].numpy()
+        ref_lse = torch.logsumexp(qt @ kc.transpose(-1, -2) / math.sqrt(D), dim=-1)[0, 0].numpy()
+        assert np.abs(out["o"][0, h] - ref).max() < 1e-12
+        assert np.abs(out["lse"][0, h] - ref_lse).max() < 1e-11
+
+
+@pytest.mark.parametrize("N,L,K", [(4096, 2, 2), (16384, 3, 2)])
+def test_level1_with_log_bias_counts_each_selected_block_twice(N, L, K):
+    # K and V constant over each coarsest-level group: a selected block's pooled token equals
+    # each of its 16 tokens, so with + ln 16 it weighs as those 16 tokens once more
+    rng = np.random.default_rng(42)
+    B, H, D = 1, 1, 8
+    q = rng.standard_normal((B, H, N, D))
+    k = grouped(rng, B, H, N, D, BLOCK ** L)
+    v = grouped(rng, B, H, N, D, BLOCK ** L)
+    qp, kp, vp = (build_pyramid(x, L, np.float64) for x in (q, k, v))
+    idx = select(qp, kp, K)
+    o, lse = forward(q, k, v, kp, vp, idx, log_bias=True, level1=True)
+    ksrc, offsets = kv_sources(k, kp)
+    vsrc, _ = kv_sources(v, vp)
+    for p in range(0, N // BLOCK, max(1, N // BLOCK // 16)):
+        rows = kv_index(p, (0, 0), idx, offsets)        # the default list
+        reps = np.ones(len(rows), dtype=np.int64)
+        reps[:BLOCK * K] = 2
+        for lev in range(2, L + 1):
+            start = BLOCK * K + (lev - 2) * K
+            reps[start:start + K] = BLOCK ** lev
+        km = torch.tensor(np.repeat(ksrc[0, 0][rows], reps, axis=0))[None, None]
+        vm = torch.tensor(np.repeat(vsrc[0, 0][rows], reps, axis=0))[None, None]
+        qb = torch.tensor(q[0, 0, p * BLOCK:(p + 1) * BLOCK])[None, None]
+        ref = F.scaled_dot_product_attention(qb, km, vm)[0, 0].numpy()
+        ref_lse = torch.logsumexp(qb @ km.transpose(-1, -2) / math.sqrt(D), dim=-1)[0, 0].numpy()
+        assert np.abs(o[0, 0, p * BLOCK:(p + 1) * BLOCK] - ref).max() < 1e-12
+        assert np.abs(lse[0, 0, p * BLOCK:(p + 1) * BLOCK] - ref_lse).max() < 1e-11
+
+
+@pytest.mark.parametrize("log_bias,all_top", [(False, False), (True, True)])
+def test_level1_finite_differences_and_sums(log_bias, all_top):
+    rng = np.random.default_rng(43)
+    B, H, N, D, K, L = 1, 1, 16384, 4, 2, 3
+    q, k, v, do = (rng.standard_normal((B, H, N, D)) for _ in range(4))
+    idx = select(build_pyramid(q, L, np.float64), build_pyramid(k, L, np.float64), K)
+    kw = dict(log_bias=log_bias, all_top=all_top, level1=True)
+
+    def loss(q_, k_, v_):
+        kp, vp = build_pyramid(k_, L, np.float64), build_pyramid(v_, L, np.float64)
+        o, _ = forward(q_, k_, v_, kp, vp, idx, **kw)
+        return float((o * do).sum())
+
+    kp, vp = build_pyramid(k, L, np.float64), build_pyramid(v, L, np.float64)
+    o, lse = forward(q, k, v, kp, vp, idx, **kw)
+    dq, dk, dv = backward(q, k, v, o, lse, do, kp, vp, idx, **kw)
     assert np.abs(dv.sum(axis=2) - do.sum(axis=2)).max() < 1e-9
     assert np.abs(dk.sum(axis=2)).max() < 1e-9
     eps = 1e-6
