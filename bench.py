@@ -210,19 +210,22 @@ def coarse_entries(cfg, all_top: bool = False) -> int:
 
 def enrichment(args) -> dict:
     """Keyword arguments of the enrichment variants chosen on the command line."""
-    return dict(log_bias=args.log_bias, all_top=args.all_top)
+    return dict(log_bias=args.log_bias, all_top=args.all_top, level1=args.level1)
 
 
 def enrichment_text(args) -> str:
     parts = ["log-count bias ln(16^l) on coarse scores" if args.log_bias else "unit weight"]
     if args.all_top:
         parts.append("all n_L coarsest tokens in every list")
+    if args.level1:
+        parts.append("level-1 pooled token of every selected block (folded into its fine tile)")
     return "; ".join(parts)
 
 
 # ----------------------------------------------------------------------------- oracle sample
 
-def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool = False, all_top: bool = False):
+def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool = False, all_top: bool = False,
+                  level1: bool = False):
     """Time the CPU oracle on ``heads`` (b=0) heads of the workload: pyramid, selection and
     transpose for each whole head, forward and backward for ``nblocks`` query blocks per
     head (all blocks if None).  Returns (tokens/s extrapolated to the full workload, dict)."""
@@ -246,9 +249,11 @@ def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool =
             idx = orc.select(qp, kp, cfg.topk)
             orc.index_transpose_all(idx)
             t1 = time.perf_counter()
-            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top)
+            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top,
+                                 level1=level1)
             if cfg.backward:
-                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top)
+                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top,
+                             level1=level1)
             t2 = time.perf_counter()
             t_fixed += t1 - t0
             t_attn += t2 - t1
@@ -483,7 +488,7 @@ def run_ours(args):
         "data": "synthetic (seeded smooth-field Q/K in Z order, N(0,1) V and dO)",
         "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
                    "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk,
-                   "kv_len": 16 * cfg.topk + coarse_entries(cfg, args.all_top),
+                   "kv_len": 16 * cfg.topk + (cfg.topk if args.level1 else 0) + coarse_entries(cfg, args.all_top),
                    "step": "pyramid + select + forward + index transpose + backward",
                    "enrichment": enrichment_text(args),
                    "launch": ("K steps as one CUDA graph (llsa_plan_create repeat=K), kernels chained by "
@@ -615,6 +620,8 @@ def main():
                     help="the log-count enrichment variant (ln 16^l on level-l coarse scores)")
     ap.add_argument("--all-top", action="store_true",
                     help="the all-coarsest enrichment variant (every level-L token in every list)")
+    ap.add_argument("--level1", action="store_true",
+                    help="the level-1 enrichment variant (each selected block's mean token in the list)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

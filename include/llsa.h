@@ -44,7 +44,7 @@
  *  - Shape rules: B, H >= 1; N a power of two with N >= 16^L (so N / 16^L >= 1);
  *    topk a power of two with 1 <= topk <= n_L; block == 16; 1 <= levels <= 4;
  *    D == 64; N <= 2^20; n_L <= 16384; topk <= 64; (levels - 1) * topk <= 32;
- *    B * H * N < 2^31.
+ *    B * H * N < 2^31; with LLSA_FLAG_ALL_TOP also (levels - 2) * topk + n_L <= 96.
  *  - Device-side checks: every gathered index (idx entries, CSR entries) is range
  *    checked on the device; an out-of-range value is not dereferenced, and the call
  *    records LLSA_ERR_INTERNAL in a device status word that llsa_device_status reads.
@@ -92,6 +92,13 @@ typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
  * produced (the backward does not need them).
  */
 #define LLSA_FLAG_ALL_TOP 2
+/*
+ * Enrichment variant: with LLSA_FLAG_LEVEL1 the list also holds the level-1 pooled token
+ * (the mean K and V of the 16 tokens) of each of the K selected fine blocks, so T grows by
+ * K; with LLSA_FLAG_LOG_BIAS those entries get + ln 16.  Their gradient reaches the block's
+ * 16 tokens through the mean-pool adjoint.  Combines with the other flags, at any levels.
+ */
+#define LLSA_FLAG_LEVEL1 4
 
 typedef struct {
   int32_t B, H, N, D;

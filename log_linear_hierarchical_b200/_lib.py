@@ -41,6 +41,7 @@ class LLSAShape(ctypes.Structure):
 # llsa_shape.flags: log-count score bias on the coarse KV entries (ln 16^l at level l)
 LLSA_FLAG_LOG_BIAS = 1
 LLSA_FLAG_ALL_TOP = 2
+LLSA_FLAG_LEVEL1 = 4
 
 
 _SP = ctypes.POINTER(LLSAShape)

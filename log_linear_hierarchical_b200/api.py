@@ -28,11 +28,13 @@ class LLSAError(RuntimeError):
 
 
 def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16,
-               log_bias: bool = False, all_top: bool = False) -> LLSAShape:
+               log_bias: bool = False, all_top: bool = False, level1: bool = False) -> LLSAShape:
     """``log_bias``: the log-count enrichment variant (LLSA_FLAG_LOG_BIAS); ``all_top``: the
-    all-coarsest variant (LLSA_FLAG_ALL_TOP).  Both may be set."""
+    all-coarsest variant (LLSA_FLAG_ALL_TOP); ``level1``: the selected blocks' level-1 pooled
+    tokens join the list (LLSA_FLAG_LEVEL1).  Any combination may be set."""
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
-    flags = (_lib.LLSA_FLAG_LOG_BIAS if log_bias else 0) | (_lib.LLSA_FLAG_ALL_TOP if all_top else 0)
+    flags = ((_lib.LLSA_FLAG_LOG_BIAS if log_bias else 0) | (_lib.LLSA_FLAG_ALL_TOP if all_top else 0)
+             | (_lib.LLSA_FLAG_LEVEL1 if level1 else 0))
     return LLSAShape(B, H, N, D, block, topk, levels, code, flags)
 
 

@@ -92,16 +92,29 @@ __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
 }
 
 // One 16-token chunk of the query-major backward: dQ += dS K with dS = P (dP - Delta).
-template <bool MASK>
+// POOL (level-1 variant, fine chunks): the block-mean entry has score mean(S) + pool_bias
+// and dP mean(dP); its dS, times the mean K row, is dS / 16 added to each of the 16 dS.
+template <bool MASK, bool POOL = false>
 __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[4][4], const uint32_t (&df)[4][4], uint32_t ktile,
                                          uint32_t vtile, int valid, float scale_log2, const float (&lse2)[2],
                                          const float (&delta)[2], float (&dq)[8][4], const Geometry* bias_g = nullptr,
-                                         int c0 = 0) {
+                                         int c0 = 0, float pool_bias = 0.f) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt(s, qf, ktile);
   mma_a_bt(dp, df, vtile);
+  float pds[2] = {0.f, 0.f};  // pooled entry's dS / 16, rows r0 and r0 + 8
+  if (POOL) {
+    float t[2], u[2];
+    quad_row_sums(s, t[0], t[1]);
+    quad_row_sums(dp, u[0], u[1]);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float pb = ex2(fmaf(fmaf(t[r], 1.0f / kBlock, pool_bias), scale_log2, -lse2[r]));
+      pds[r] = pb * fmaf(u[r], 1.0f / kBlock, -delta[r]) * (1.0f / kBlock);
+    }
+  }
   float ds[2][4];
 #pragma unroll
   for (int n = 0; n < 2; ++n)
@@ -112,14 +125,15 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[4][4], const uint3
       float sb = s[n][e];
       if (MASK && bias_g && bias_g->log_bias && col < valid) sb += coarse_log_bias(*bias_g, c0 + col) * kSqrtD;
       const float p = (!MASK || col < valid) ? ex2(fmaf(sb, scale_log2, -lse2[r])) : 0.0f;
-      ds[n][e] = p * (dp[n][e] - delta[r]);
+      ds[n][e] = POOL ? fmaf(p, dp[n][e] - delta[r], pds[r]) : p * (dp[n][e] - delta[r]);
     }
   mma_a_b(dq, pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]), pack_bf16(ds[1][0], ds[1][1]),
           pack_bf16(ds[1][2], ds[1][3]), ktile);
 }
 
 // Same CTA shape as the forward: 4 warps x 4 query blocks, coarse KV staged once per CTA.
-template <int STAGES>
+// POOL: the level-1 variant (see dq_chunk).
+template <int STAGES, bool POOL>
 __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
@@ -265,7 +279,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
       if (!ok) break;
       next_seq = seq + 1;
       const uint32_t kt = ring + stage * 2 * kTileBytes;
-      dq_chunk<false>(qf, df, kt, kt + kTileBytes, kBlock, P.scale_log2, lse2, delta, dq);
+      dq_chunk<false, POOL>(qf, df, kt, kt + kTileBytes, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
+                            pool_log_bias(g));
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }
@@ -291,10 +306,15 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 //   dS^T = P^T (dP^T - Delta), dV += P^T dO, dK += dS^T Q  (dK unscaled).
 // BIAS: the key rows are coarse tokens under the log-count variant; kb[0], kb[1] are the
 // biases (unscaled-dot units) of this lane's key rows r0 and r0 + 8.
-template <bool BIAS = false>
+// POOL (level-1 variant; the key rows are a fine block): the block-mean entry, with score
+// mean over the 16 keys of S + pool_bias and dP the mean of dP, sends dV_mean = p dO and
+// dK_mean = dS q to the block's 16 rows with weight 1/16 each: p / 16 is added to every
+// P^T entry of its query column and dS / 16 to every dS^T entry.
+template <bool BIAS = false, bool POOL = false>
 __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32_t (&vf)[4][4], uint32_t qt,
                                         uint32_t dt, const float* ls, const float* dl, float scale_log2,
-                                        float (&dk)[8][4], float (&dv)[8][4], const float (&kb)[2] = {0.f, 0.f}) {
+                                        float (&dk)[8][4], float (&dv)[8][4], const float (&kb)[2] = {0.f, 0.f},
+                                        float pool_bias = 0.f) {
   const int c2 = 2 * (lane_id() & 3);
   float st[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dpt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -307,6 +327,35 @@ __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32
   const float2 d1 = *reinterpret_cast<const float2*>(dl + 8 + c2);
   const float lq[2][2] = {{l0.x * kLog2e, l0.y * kLog2e}, {l1.x * kLog2e, l1.y * kLog2e}};
   const float dq[2][2] = {{d0.x, d0.y}, {d1.x, d1.y}};
+  float pa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, da[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // pooled p/16, dS/16
+  if (POOL) {
+    // column sums over the 16 key rows: this lane's rows r0, r0 + 8, then the 8 row groups
+    float ts[2][2], tp[2][2];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        ts[n][c] = st[n][c] + st[n][2 + c];
+        tp[n][c] = dpt[n][c] + dpt[n][2 + c];
+      }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          ts[n][c] += __shfl_xor_sync(0xffffffffu, ts[n][c], off);
+          tp[n][c] += __shfl_xor_sync(0xffffffffu, tp[n][c], off);
+        }
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float pb = ex2(fmaf(fmaf(ts[n][c], 1.0f / kBlock, pool_bias), scale_log2, -lq[n][c]));
+        pa[n][c] = pb * (1.0f / kBlock);
+        da[n][c] = pa[n][c] * fmaf(tp[n][c], 1.0f / kBlock, -dq[n][c]);
+      }
+  }
   float pt[2][4], dst[2][4];
 #pragma unroll
   for (int n = 0; n < 2; ++n)
@@ -314,6 +363,10 @@ __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32
     for (int e = 0; e < 4; ++e) {
       pt[n][e] = ex2(fmaf(BIAS ? st[n][e] + kb[e >> 1] : st[n][e], scale_log2, -lq[n][e & 1]));
       dst[n][e] = pt[n][e] * (dpt[n][e] - dq[n][e & 1]);
+      if (POOL) {
+        pt[n][e] += pa[n][e & 1];
+        dst[n][e] += da[n][e & 1];
+      }
     }
   mma_a_b(dv, pack_bf16(pt[0][0], pt[0][1]), pack_bf16(pt[0][2], pt[0][3]), pack_bf16(pt[1][0], pt[1][1]),
           pack_bf16(pt[1][2], pt[1][3]), dt);
@@ -338,13 +391,13 @@ __host__ __device__ inline CtaSmem kv_smem(int nwarps) {
 // `bar_tile` is non-zero the key tile is still arriving on that mbarrier (phase 0) and is
 // waited for after the first pair loads are issued.  Returns false (after draining the
 // copies in flight) if a wait timed out.
-template <int STAGES, bool BIAS = false, class PairBlock>
+template <int STAGES, bool BIAS = false, bool POOL = false, class PairBlock>
 __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtensorMap* tm_do,
                                           const float* __restrict__ lse, const float* __restrict__ delta,
                                           uint32_t kvtile, uint32_t bar_tile, uint32_t ring, float* sls, float* sdl,
                                           uint32_t bar_ring, int npairs, PairBlock pair_block, float scale_log2,
                                           float (&dk)[8][4], float (&dv)[8][4],
-                                          const float (&kbias)[2] = {0.f, 0.f}) {
+                                          const float (&kbias)[2] = {0.f, 0.f}, float pool_bias = 0.f) {
   const int lane = lane_id();
   // called by the whole warp (pair_block may shuffle); lane 0 issues the copies
   auto issue_pair = [&](int i) {
@@ -376,7 +429,8 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
       return false;
     }
     const uint32_t qt = ring + stage * 2 * kTileBytes;
-    kv_pair<BIAS>(kf, vf, qt, qt + kTileBytes, sls + stage * kBlock, sdl + stage * kBlock, scale_log2, dk, dv, kbias);
+    kv_pair<BIAS, POOL>(kf, vf, qt, qt + kTileBytes, sls + stage * kBlock, sdl + stage * kBlock, scale_log2, dk, dv,
+                        kbias, pool_bias);
     __syncwarp();
     if (i + STAGES < npairs) issue_pair(i + STAGES);
   }
@@ -741,7 +795,7 @@ __global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometr
 // whose output (the coarse-token gradients) only the epilogue reads; everything the main
 // loop reads was complete before that kernel could start, so the wait for it is deferred
 // to the epilogue and the main loop overlaps the reduction.
-template <int STAGES>
+template <int STAGES, bool POOL>
 __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
@@ -860,7 +914,8 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   // the row's query blocks are read 32 at a time by the whole warp and handed to the
   // issuing lane by shuffle, so no load sits on the TMA issue path
   int cached_base = -64, cached = 0;
-  const bool ok = kv_stream<STAGES>(&tm_q, &tm_do, lse, ws + W.delta, kvt, bar_kv, ring, sls, sdl, bar_ring, re - rs,
+  const bool ok = kv_stream<STAGES, false, POOL>(&tm_q, &tm_do, lse, ws + W.delta, kvt, bar_kv, ring, sls, sdl,
+                                                 bar_ring, re - rs,
                                     [&](int i) {
                                       const int base32 = i & ~31;
                                       if (base32 != cached_base) {
@@ -870,7 +925,7 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
                                       }
                                       return bh_block0 + __shfl_sync(0xffffffffu, cached, i & 31);
                                     },
-                                    P.scale_log2, dk, dv);
+                                    P.scale_log2, dk, dv, {0.f, 0.f}, pool_log_bias(g));
   if (!ok) return;
   if (coarse_late) pdl_wait();
   // epilogue: scale dK, add the mean-pool adjoint of the ancestors' coarse gradients

@@ -129,17 +129,41 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[8][4], float 
 
 constexpr float kSqrtD = 8.0f;  // sqrt(kD): score bias in units of the unscaled dot product
 
+// Bias of a level-1 pooled entry (level-1 variant) in unscaled-dot units: ln 16 under the
+// log-count variant, else 0.
+__host__ __device__ inline float pool_log_bias(const Geometry& g) { return g.log_bias ? kLn16 * kSqrtD : 0.0f; }
+
+// Row sums of a 16 x 16 score fragment (C layout): rows r0 and r0 + 8 of this lane's quad.
+__device__ __forceinline__ void quad_row_sums(const float (&s)[2][4], float& t0, float& t1) {
+  t0 = (s[0][0] + s[0][1]) + (s[1][0] + s[1][1]);
+  t1 = (s[0][2] + s[0][3]) + (s[1][2] + s[1][3]);
+  t0 += __shfl_xor_sync(0xffffffffu, t0, 1);
+  t0 += __shfl_xor_sync(0xffffffffu, t0, 2);
+  t1 += __shfl_xor_sync(0xffffffffu, t1, 1);
+  t1 += __shfl_xor_sync(0xffffffffu, t1, 2);
+}
+
 // One 16-token chunk of the online softmax.  With MASK (the coarse chunks), columns >=
 // `valid` (the padding of the last coarse tile) are excluded and, under the log-count
 // variant, column c gets the bias of coarse entry c0 + c.  m holds the running row maxima
 // of the scaled scores (log2 domain), l the per-lane partial row sums.
-template <bool MASK>
+// POOL (the level-1 variant, fine chunks only): the chunk's block mean is one more KV
+// entry.  Its score is the mean of the 16 scores (q . mean k = mean of q . k), plus
+// `pool_bias` (unscaled-dot units), and since its value is the mean of the 16 V rows its
+// weight p folds into the chunk as p / 16 added to each of the 16 probabilities.
+template <bool MASK, bool POOL = false>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t ktile, uint32_t vtile, int valid,
                                           float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[8][4],
-                                          const Geometry* bias_g = nullptr, int c0 = 0) {
+                                          const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt(s, qf, ktile);
+  float sb0 = 0.f, sb1 = 0.f;  // pooled scores of rows r0, r0 + 8
+  if (POOL) {
+    quad_row_sums(s, sb0, sb1);
+    sb0 = fmaf(sb0, 1.0f / kBlock, pool_bias);
+    sb1 = fmaf(sb1, 1.0f / kBlock, pool_bias);
+  }
   if (MASK) {
 #pragma unroll
     for (int n = 0; n < 2; ++n)
@@ -156,6 +180,10 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
   mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
   mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
   mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  if (POOL) {
+    mx0 = fmaxf(mx0, sb0);
+    mx1 = fmaxf(mx1, sb1);
+  }
   // the scale is positive, so the maximum of the scaled scores is the scaled maximum
   const float mn0 = fmaxf(m[0], mx0 * scale_log2);
   const float mn1 = fmaxf(m[1], mx1 * scale_log2);
@@ -166,6 +194,17 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
     p[n][1] = ex2(fmaf(s[n][1], scale_log2, -mn0));
     p[n][2] = ex2(fmaf(s[n][2], scale_log2, -mn1));
     p[n][3] = ex2(fmaf(s[n][3], scale_log2, -mn1));
+  }
+  if (POOL) {
+    const float a0 = ex2(fmaf(sb0, scale_log2, -mn0)) * (1.0f / kBlock);
+    const float a1 = ex2(fmaf(sb1, scale_log2, -mn1)) * (1.0f / kBlock);
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      p[n][0] += a0;
+      p[n][1] += a0;
+      p[n][2] += a1;
+      p[n][3] += a1;
+    }
   }
   // rescale the running sums only when a row maximum moved (decided for the whole warp)
   if (__any_sync(0xffffffffu, mn0 != m[0] || mn1 != m[1])) {
@@ -216,8 +255,9 @@ __host__ __device__ inline CtaSmem fwd_smem(const Geometry& g, int nwarps) {
 
 // One CTA = 4 warps = 16 consecutive query blocks (one level-2 group when L >= 2, so the
 // coarse KV entries are staged once per CTA).  Each warp owns 4 blocks and streams their
-// fine KV tiles through its own ring of STAGES mbarrier-tracked TMA stages.
-template <int STAGES>
+// fine KV tiles through its own ring of STAGES mbarrier-tracked TMA stages.  POOL: the
+// level-1 variant (see fwd_chunk).
+template <int STAGES, bool POOL>
 __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                             const __grid_constant__ CUtensorMap tm_k,
                                                             const __grid_constant__ CUtensorMap tm_v, AttnParams P,
@@ -314,7 +354,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
       if (!ok) break;
       next_seq = seq + 1;
       const uint32_t kt = ring + stage * 2 * kTileBytes;
-      fwd_chunk<false>(qf, kt, kt + kTileBytes, kBlock, P.scale_log2, m, l, acc);
+      fwd_chunk<false, POOL>(qf, kt, kt + kTileBytes, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias(g));
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }

@@ -11,14 +11,29 @@ namespace llsa {
 
 constexpr int kSimtThreads = 128;
 
-// Row pointers of block p's KV list: 16K fine tokens then the C coarse pyramid rows.
+// KV list of a query block in these kernels: 16K fine tokens, then (level-1 variant) the K
+// selected blocks' level-1 pyramid rows, then the C coarse pyramid rows.
+__host__ __device__ inline int simt_coarse_start(const Geometry& g) { return kBlock * g.K + (g.pool1 ? g.K : 0); }
+__host__ __device__ inline int simt_T(const Geometry& g) { return simt_coarse_start(g) + g.coarse; }
+
+// Score bias of list entry e (scaled units): ln 16 for a level-1 pooled entry and the
+// coarse entries' bias, both under the log-count variant only.
+__device__ __forceinline__ float simt_entry_bias(const Geometry& g, int e) {
+  if (e < kBlock * g.K) return 0.0f;
+  const int c0 = simt_coarse_start(g);
+  if (e < c0) return g.log_bias ? kLn16 : 0.0f;
+  return coarse_log_bias(g, e - c0);
+}
+
+// Row pointers of block p's KV list (see simt_coarse_start).
 __device__ __forceinline__ void simt_kv_rows(const Geometry& g, int bh, int p, const float* __restrict__ k,
                                              const float* __restrict__ v, const float* __restrict__ k_pyr,
                                              const float* __restrict__ v_pyr, const int* __restrict__ idx,
                                              const float** krow, const float** vrow) {
   const int K = g.K;
   const int n1 = g.n[1];
-  const int T = kBlock * K + g.coarse;
+  const int T = simt_T(g);
+  const int c0 = simt_coarse_start(g);
   for (int e = threadIdx.x; e < T; e += blockDim.x) {
     long long r;
     const float* kb;
@@ -28,9 +43,14 @@ __device__ __forceinline__ void simt_kv_rows(const Geometry& g, int bh, int p, c
       r = (long long)bh * g.N + (long long)j * kBlock + (e % kBlock);
       kb = k;
       vb = v;
+    } else if (e < c0) {  // level-1 pooled token of selected block e - 16K
+      const int j = checked_index(__ldg(idx + g.idx_off[1] + ((long long)bh * n1 + p) * K + (e - kBlock * K)), n1);
+      r = (long long)bh * n1 + j;
+      kb = k_pyr + g.pyr_off[1];
+      vb = v_pyr + g.pyr_off[1];
     } else {
       int lev;
-      const int jj = coarse_token(g, idx, bh, p, e - kBlock * K, lev);
+      const int jj = coarse_token(g, idx, bh, p, e - c0, lev);
       r = (long long)bh * g.n[lev] + jj;
       kb = k_pyr + g.pyr_off[lev];
       vb = v_pyr + g.pyr_off[lev];
@@ -58,7 +78,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
                                                                     float* __restrict__ lse) {
   pdl_enter();
   extern __shared__ __align__(16) uint8_t simt_smem[];
-  const int T = kBlock * g.K + g.coarse;
+  const int T = simt_T(g);
   const int gb = blockIdx.x;
   const int bh = gb / g.n[1];
   const int p = gb - bh * g.n[1];
@@ -73,7 +93,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
   for (int pr = threadIdx.x; pr < kBlock * T; pr += blockDim.x) {
     const int qi = pr / T;
     const int e = pr - qi * T;
-    S[pr] = dot64(qs + qi * kD, krow[e]) * scale + (e >= kBlock * g.K ? coarse_log_bias(g, e - kBlock * g.K) : 0.0f);
+    S[pr] = dot64(qs + qi * kD, krow[e]) * scale + simt_entry_bias(g, e);
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,7 +127,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
 }
 
 inline size_t simt_fwd_smem(const Geometry& g) {
-  const int T = kBlock * g.K + g.coarse;
+  const int T = simt_T(g);
   return sizeof(float) * kBlock * kD + 2 * sizeof(void*) * T + sizeof(float) * kBlock * T;
 }
 
@@ -122,7 +142,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
   pdl_enter();
   extern __shared__ __align__(16) uint8_t simt_smem[];
   const BwdWorkspace W = bwd_workspace_layout(g);
-  const int T = kBlock * g.K + g.coarse;
+  const int T = simt_T(g);
   const int C = g.coarse;
   const int per_cta = g.L >= 2 ? kBlock : 1;
   float* qs = reinterpret_cast<float*>(simt_smem);
@@ -161,7 +181,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
     for (int pr = threadIdx.x; pr < kBlock * T; pr += blockDim.x) {
       const int qi = pr / T;
       const int e = pr - qi * T;
-      const float bias = e >= kBlock * g.K ? coarse_log_bias(g, e - kBlock * g.K) : 0.0f;
+      const float bias = simt_entry_bias(g, e);
       const float pe = expf(dot64(qs + qi * kD, krow[e]) * scale + bias - lse[rbase + qi]);
       const float dp = dot64(ds_ + qi * kD, vrow[e]);
       Pm[pr] = pe;
@@ -178,7 +198,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
     for (int cd = threadIdx.x; cd < C * kD; cd += blockDim.x) {
       const int c = cd / kD;
       const int d = cd - c * kD;
-      const int e = kBlock * g.K + c;
+      const int e = simt_coarse_start(g) + c;
       float ak = 0.f, av = 0.f;
       for (int qi = 0; qi < kBlock; ++qi) {
         ak = fmaf(dS[qi * T + e], qs[qi * kD + d], ak);
@@ -198,22 +218,26 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
 }
 
 inline size_t simt_dq_smem(const Geometry& g) {
-  const int T = kBlock * g.K + g.coarse;
+  const int T = simt_T(g);
   return sizeof(float) * 2 * kBlock * kD + 2 * sizeof(void*) * T + sizeof(float) * 2 * kBlock * T +
          sizeof(float) * 2 * g.coarse * kD + sizeof(float) * kBlock;
 }
 
 // Key-major fp32 backward: one CTA per fine key block; thread t owns 8 of the 16 x 64 dK and
 // dV outputs.  smem: K_j, V_j, Q_p, dO_p [16][64]; Pt, dSt [16][16]; lse, delta [16].
+// Level-1 variant: the block's level-1 pyramid row (kbar, vbar) is in the list of every query
+// block p of the row; its dK, dV reach the 16 rows with weight 1/16, which adds p / 16 to
+// every Pt entry of query i and dS / 16 to every dSt entry.
 __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
     Geometry g, float scale, const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
-    const float* __restrict__ lse, const float* __restrict__ dO, const int* __restrict__ row_ptr,
-    const int* __restrict__ col, const float* __restrict__ ws, float* __restrict__ dk_out,
-    float* __restrict__ dv_out) {
+    const float* __restrict__ k_pyr, const float* __restrict__ v_pyr, const float* __restrict__ lse,
+    const float* __restrict__ dO, const int* __restrict__ row_ptr, const int* __restrict__ col,
+    const float* __restrict__ ws, float* __restrict__ dk_out, float* __restrict__ dv_out) {
   pdl_enter();
   __shared__ float ks[kBlock * kD], vs[kBlock * kD], qs[kBlock * kD], dos[kBlock * kD];
   __shared__ float Pt[kBlock][kBlock + 1], dSt[kBlock][kBlock + 1];
   __shared__ float ls[kBlock], dl[kBlock];
+  __shared__ float kbar[kD], vbar[kD], pool_p[kBlock], pool_ds[kBlock];
   const BwdWorkspace W = bwd_workspace_layout(g);
   const int n1 = g.n[1];
   const int kb = blockIdx.x;
@@ -224,6 +248,11 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
     ks[i] = k[krow0 * kD + i];
     vs[i] = v[krow0 * kD + i];
   }
+  if (g.pool1)
+    for (int d = threadIdx.x; d < kD; d += blockDim.x) {
+      kbar[d] = k_pyr[g.pyr_off[1] + (long long)kb * kD + d];
+      vbar[d] = v_pyr[g.pyr_off[1] + (long long)kb * kD + d];
+    }
   const int E = n1 * g.K;
   const int* rp = row_ptr + g.rp_off[1] + (long long)bh * (n1 + 1);
   int rs = rp[j], re = rp[j + 1];
@@ -248,13 +277,20 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
       dl[threadIdx.x] = ws[W.delta + qrow0 + threadIdx.x];
     }
     __syncthreads();
+    if (g.pool1 && threadIdx.x < kBlock) {  // the level-1 entry's p / 16 and dS / 16 per query
+      const int qi = threadIdx.x;
+      const float pb = expf(dot64(kbar, qs + qi * kD) * scale + (g.log_bias ? kLn16 : 0.0f) - ls[qi]);
+      pool_p[qi] = pb * (1.0f / kBlock);
+      pool_ds[qi] = pb * (dot64(vbar, dos + qi * kD) - dl[qi]) * (1.0f / kBlock);
+    }
+    if (g.pool1) __syncthreads();
     for (int pr = threadIdx.x; pr < kBlock * kBlock; pr += blockDim.x) {
       const int kk = pr / kBlock;
       const int qi = pr - kk * kBlock;
       const float pe = expf(dot64(ks + kk * kD, qs + qi * kD) * scale - ls[qi]);
       const float dp = dot64(vs + kk * kD, dos + qi * kD);
-      Pt[kk][qi] = pe;
-      dSt[kk][qi] = pe * (dp - dl[qi]);
+      Pt[kk][qi] = g.pool1 ? pe + pool_p[qi] : pe;
+      dSt[kk][qi] = g.pool1 ? fmaf(pe, dp - dl[qi], pool_ds[qi]) : pe * (dp - dl[qi]);
     }
     __syncthreads();
 #pragma unroll

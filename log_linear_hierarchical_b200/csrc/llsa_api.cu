@@ -39,7 +39,8 @@ llsa_status validate(const llsa_shape* s) {
   if (s->B < 1 || s->H < 1 || s->N < 1 || s->D < 1 || s->block < 1 || s->topk < 1 || s->levels < 1)
     return LLSA_ERR_INVALID_ARG;
   if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
-  if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP)) return LLSA_ERR_INVALID_ARG;  // unknown flag bits
+  if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP | LLSA_FLAG_LEVEL1))
+    return LLSA_ERR_INVALID_ARG;  // unknown flag bits
   if (!is_pow2(s->N) || !is_pow2(s->topk)) return LLSA_ERR_INVALID_ARG;  // README usage notes
   if (s->block != kBlock) return LLSA_ERR_UNSUPPORTED;
   if (s->D != kD) return LLSA_ERR_UNSUPPORTED;
@@ -83,6 +84,7 @@ Geometry make_geometry(const llsa_shape* s) {
   g.coarse_pad = (g.coarse + kBlock - 1) / kBlock * kBlock;
   g.log_bias = (s->flags & LLSA_FLAG_LOG_BIAS) ? 1 : 0;
   g.top_first = all_top ? (g.L - 2) * g.K : g.coarse;
+  g.pool1 = (s->flags & LLSA_FLAG_LEVEL1) ? 1 : 0;
   return g;
 }
 
@@ -329,7 +331,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
     const size_t kv_bytes = (size_t)kv_smem<kDkvStages>(1).total();
     if (phases & kQuerySide) {
       const size_t smem = (size_t)dq_smem<kDqStages>(g, kAttnWarps).total();
-      auto kern = attn_bwd_dq_bf16_kernel<kDqStages>;
+      auto kern = g.pool1 ? attn_bwd_dq_bf16_kernel<kDqStages, true> : attn_bwd_dq_bf16_kernel<kDqStages, false>;
       if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
       const int per_cta = kAttnWarps * kUnitBlocks;
       st = launch(kKBwdDqBf16, cs, [&] {
@@ -351,6 +353,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
     if (!(phases & kKeySide)) return LLSA_OK;
     if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
 #if LLSA_KEY_MAJOR_TC
+    if (g.pool1) return LLSA_ERR_UNSUPPORTED;  // the tcgen05 key-major kernel has no level-1 fold
     {
       int dev = 0, sms = 0;
       if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -369,7 +372,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
       });
     }
 #endif
-    auto kern = attn_bwd_dkdv_bf16_kernel<kDkvStages>;
+    auto kern = g.pool1 ? attn_bwd_dkdv_bf16_kernel<kDkvStages, true> : attn_bwd_dkdv_bf16_kernel<kDkvStages, false>;
     if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
     return launch(kKBwdDkdvBf16, cs, [&] {
       launch_pdl(kern, dim3(total_blocks), dim3(32), kv_bytes, cs, tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
@@ -392,8 +395,9 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
   if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
   return launch(kKBwdDkdvF32, cs, [&] {
     launch_pdl(attn_bwd_dkdv_f32_kernel, dim3(total_blocks), dim3(kSimtThreads), 0, cs, 
-        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), lse,
-        static_cast<const float*>(dO), row_ptr, col, ws, static_cast<float*>(dk), static_cast<float*>(dv));
+        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
+        v_pyr, lse, static_cast<const float*>(dO), row_ptr, col, ws, static_cast<float*>(dk),
+        static_cast<float*>(dv));
   });
 }
 
@@ -535,7 +539,7 @@ llsa_status forward_impl(const llsa_shape* s, const void* q, const void* k, cons
       return LLSA_ERR_CUDA;
     AttnParams P{g, scale * kLog2e, scale};
     const size_t smem = (size_t)fwd_smem<kFwdStages>(g, kAttnWarps).total();
-    auto kern = attn_fwd_bf16_kernel<kFwdStages>;
+    auto kern = g.pool1 ? attn_fwd_bf16_kernel<kFwdStages, true> : attn_fwd_bf16_kernel<kFwdStages, false>;
     if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
     const int per_cta = kAttnWarps * kUnitBlocks;
     return launch(kKFwdBf16, cs, [&] {

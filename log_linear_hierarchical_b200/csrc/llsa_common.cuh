@@ -61,6 +61,8 @@ struct Geometry {
   int log_bias;                          // LLSA_FLAG_LOG_BIAS: coarse scores + ln(16^l)
   int top_first;                         // LLSA_FLAG_ALL_TOP (L >= 2): (L-2) K, the first
                                          // entry of the level-L part; C (never reached) otherwise
+  int pool1;                             // LLSA_FLAG_LEVEL1: each selected fine block's
+                                         // level-1 mean is one more KV entry
 };
 
 // Level of coarse entry c (0 <= c < C): 2 + c / K, except that under the all-coarsest

@@ -20,10 +20,12 @@ TOL = {"f32": 1e-4, "bf16": 2e-2}
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 
-def run_gpu(B, H, N, D, topk, levels, dtype, inputs, backward=True, device="cuda", log_bias=False, all_top=False):
+def run_gpu(B, H, N, D, topk, levels, dtype, inputs, backward=True, device="cuda", log_bias=False, all_top=False,
+            level1=False):
     """All five calls on one stream; returns CPU tensors of every output."""
     tdt = TORCH_DTYPE[dtype]
-    shape = api.make_shape(B, H, N, D, topk, levels, tdt, log_bias=log_bias, all_top=all_top)
+    shape = api.make_shape(B, H, N, D, topk, levels, tdt, log_bias=log_bias, all_top=all_top,
+                           level1=level1)
     dev = {k: v.to(device) for k, v in inputs.items()}
     buf = api.LLSABuffers.allocate(shape, device, tdt)
     assert api.llsa_device_status() == 0
@@ -76,7 +78,7 @@ def check_transpose_bitexact(gpu):
         assert np.array_equal(gpu["col"][lev], cl), f"col level {lev + 1}"
 
 
-def replay(inputs, gpu, backward=True, heads=None, log_bias=False, all_top=False):
+def replay(inputs, gpu, backward=True, heads=None, log_bias=False, all_top=False, level1=False):
     """Oracle forward (and backward) on the GPU's indices; ``heads`` = (b, h slice) subset."""
     def sl(x):
         return x if heads is None else x[heads[0]:heads[0] + 1, heads[1]]
@@ -84,12 +86,12 @@ def replay(inputs, gpu, backward=True, heads=None, log_bias=False, all_top=False
     kp = [sl(x) for x in gpu["k_pyr"]]
     vp = [sl(x) for x in gpu["v_pyr"]]
     idx = [sl(x) for x in gpu["idx"]]
-    o, lse = orc.forward(q, k, v, kp, vp, idx, log_bias=log_bias, all_top=all_top)
+    o, lse = orc.forward(q, k, v, kp, vp, idx, log_bias=log_bias, all_top=all_top, level1=level1)
     out = {"o": o, "lse": lse}
     if backward:
         do = sl(to_f64_numpy(inputs["do"]))
         out["dq"], out["dk"], out["dv"] = orc.backward(q, k, v, o, lse, do, kp, vp, idx, log_bias=log_bias,
-                                                           all_top=all_top)
+                                                           all_top=all_top, level1=level1)
     return out
 
 

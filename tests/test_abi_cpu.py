@@ -119,14 +119,15 @@ def test_step_and_plan_rejected_before_launch(lib):
 
 def test_flags_validated(lib):
     s = shape()
-    for good in (1, 2, 3):  # LLSA_FLAG_LOG_BIAS, LLSA_FLAG_ALL_TOP, both
+    for good in range(1, 8):  # any combination of LOG_BIAS (1), ALL_TOP (2), LEVEL1 (4)
         s.flags = good
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 0, good
-    for bad in (4, 8, 1 << 30, -1):
+    for bad in (8, 16, 1 << 30, -1):
         s.flags = bad
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 1, bad
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True).flags == _lib.LLSA_FLAG_LOG_BIAS
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True, all_top=True).flags == 3
+    assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, level1=True).flags == _lib.LLSA_FLAG_LEVEL1 == 4
 
 
 def test_all_top_coarse_limit(lib):
