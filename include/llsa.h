@@ -8,7 +8,8 @@
  * Sparse Attention", Core Technique 1-3).  The LLSA GitHub README's usage section makes
  * it a drop-in for scaled_dot_product_attention(q, k, v, dropout_p=0, is_causal=False)
  * with block_size=16, and states that only non-causal attention is supported and that
- * the token length and topk must be powers of two.
+ * the token length and topk must be powers of two.  This library lifts the second limit:
+ * any topk, and any N that the 16x pyramid divides (a multiple of 16^L).
  *
  * The path is split into five calls, in this order for one training step:
  *   llsa_build_pyramid -> llsa_select -> llsa_forward            (forward)
@@ -41,9 +42,9 @@
  *    nothing and returns LLSA_ERR_INVALID_ARG (bad value, null pointer, misalignment,
  *    shape rules below) or LLSA_ERR_UNSUPPORTED (a legal value this build does not
  *    implement).  A launch failure returns LLSA_ERR_CUDA.  No exception crosses the ABI.
- *  - Shape rules: B, H >= 1; N a power of two with N >= 16^L (so N / 16^L >= 1);
- *    topk a power of two with 1 <= topk <= n_L; block == 16; 1 <= levels <= 4;
- *    D == 64; N <= 2^20; n_L <= 16384; topk <= 64; (levels - 1) * topk <= 32;
+ *  - Shape rules: B, H >= 1; N a multiple of 16^L (so every n_l = N / 16^l is whole
+ *    and n_L >= 1; N need not be a power of two); 1 <= topk <= n_L, any integer;
+ *    block == 16; 1 <= levels <= 4; D == 64; N <= 2^20; n_L <= 16384; topk <= 64; (levels - 1) * topk <= 32;
  *    B * H * N < 2^31; with LLSA_FLAG_ALL_TOP also (levels - 2) * topk + n_L <= 96.
  *  - Device-side checks: every gathered index (idx entries, CSR entries) is range
  *    checked on the device; an out-of-range value is not dereferenced, and the call
@@ -103,7 +104,7 @@ typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
 typedef struct {
   int32_t B, H, N, D;
   int32_t block;   /* must be 16 (README usage section: block_size=16) */
-  int32_t topk;    /* K, a power of two */
+  int32_t topk;    /* K, 1 <= K <= n_L */
   int32_t levels;  /* L, number of pooled levels; llsa_l1 <-> 1, llsa_l2 <-> 2 */
   int32_t dtype;   /* llsa_dtype of q, k, v, o, dO, dq, dk, dv */
   int32_t flags;   /* LLSA_FLAG_* bits (0: the default enrichment); others -> INVALID_ARG */

@@ -187,8 +187,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int gb = first + (seq >> g.log_k);
-    const int row = ((gb >> g.log_n1) << (g.log_n1 + 4)) + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
+    const int gb = first + div_k(g, seq);
+    const int row = div_n1(g, gb) * g.N + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * kTileBytes;
@@ -667,7 +667,8 @@ __device__ __forceinline__ int order_class(int len) {
 // CSR extent [rs, re) of flat level-1 row kb = bh * n_1 + j (empty for kb past the end).
 __device__ __forceinline__ int2 order_row(const Geometry& g, const int* __restrict__ rp1, int kb) {
   if (kb >= g.BH * g.n[1]) return make_int2(0, 0);
-  const int* r = rp1 + (long long)(kb >> g.log_n1) * (g.n[1] + 1) + (kb & (g.n[1] - 1));
+  const int bh = div_n1(g, kb);
+  const int* r = rp1 + (long long)bh * (g.n[1] + 1) + (kb - bh * g.n[1]);
   return make_int2(__ldg(r), __ldg(r + 1));
 }
 

@@ -308,8 +308,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int gb = first + (seq >> g.log_k);
-    const int row = ((gb >> g.log_n1) << (g.log_n1 + 4)) + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
+    const int gb = first + div_k(g, seq);
+    const int row = div_n1(g, gb) * g.N + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * kTileBytes;

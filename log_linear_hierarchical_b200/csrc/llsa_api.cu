@@ -41,11 +41,12 @@ llsa_status validate(const llsa_shape* s) {
   if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
   if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP | LLSA_FLAG_LEVEL1))
     return LLSA_ERR_INVALID_ARG;  // unknown flag bits
-  if (!is_pow2(s->N) || !is_pow2(s->topk)) return LLSA_ERR_INVALID_ARG;  // README usage notes
+  // N: any multiple of 16^L (the pages' implementation wants powers of two for N and topk;
+  // the kernels here take any multiple and any topk)
   if (s->block != kBlock) return LLSA_ERR_UNSUPPORTED;
   if (s->D != kD) return LLSA_ERR_UNSUPPORTED;
   if (s->levels > kMaxLevels) return LLSA_ERR_UNSUPPORTED;
-  if (ilog2(s->N) < 4 * s->levels) return LLSA_ERR_INVALID_ARG;  // need N / 16^L >= 1
+  if (s->N % (1LL << (4 * s->levels)) != 0) return LLSA_ERR_INVALID_ARG;  // n_L = N / 16^L whole
   const long long nL = (long long)s->N >> (4 * s->levels);
   if (s->topk > nL) return LLSA_ERR_INVALID_ARG;  // the coarsest level must hold K keys
   if (s->N > (1 << 20)) return LLSA_ERR_UNSUPPORTED;
@@ -77,8 +78,8 @@ Geometry make_geometry(const llsa_shape* s) {
     io += (long long)g.BH * g.n[l] * g.K;
     ro += (long long)g.BH * (g.n[l] + 1);
   }
-  g.log_k = ilog2(g.K);
-  g.log_n1 = ilog2(g.n[1]);
+  g.log_k = is_pow2(g.K) ? ilog2(g.K) : -1;
+  g.log_n1 = is_pow2(g.n[1]) ? ilog2(g.n[1]) : -1;
   const bool all_top = (s->flags & LLSA_FLAG_ALL_TOP) && g.L >= 2;
   g.coarse = all_top ? (g.L - 2) * g.K + g.n[g.L] : (g.L - 1) * g.K;
   g.coarse_pad = (g.coarse + kBlock - 1) / kBlock * kBlock;
@@ -100,8 +101,10 @@ TransposeGeo make_transpose_geo(const Geometry& g, long long* ent_total, long lo
     L.n = g.n[l];
     L.E = g.n[l] * g.K;
     L.tiles = (L.E + kTrTile - 1) / kTrTile;
-    L.nb = L.n < kTrMaxBuckets ? L.n : kTrMaxBuckets;
-    L.wshift = ilog2(L.n / L.nb);
+    int w = 1;  // keys per bucket: the smallest power of two giving at most kTrMaxBuckets buckets
+    while ((L.n + w - 1) / w > kTrMaxBuckets) w <<= 1;
+    L.nb = (L.n + w - 1) / w;
+    L.wshift = ilog2(w);
     L.cta_tiles = cta_t;
     L.cta_buckets = cta_b;
     L.hist_off = hist;
@@ -353,7 +356,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
     if (!(phases & kKeySide)) return LLSA_OK;
     if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
 #if LLSA_KEY_MAJOR_TC
-    if (g.pool1) return LLSA_ERR_UNSUPPORTED;  // the tcgen05 key-major kernel has no level-1 fold
+    if (g.pool1 || g.log_n1 < 0) return LLSA_ERR_UNSUPPORTED;  // the tcgen05 kernel: no level-1 fold, n_1 = 2^m
     {
       int dev = 0, sms = 0;
       if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -465,7 +468,7 @@ llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* 
       gq = kBlock;
       while (gq > 1 && (gq > n || (long long)gq * n > 16384)) gq >>= 1;
     }
-    if (sparse && g.K >= 2 && g.K <= 16) {
+    if (sparse && (g.K == 2 || g.K == 4 || g.K == 8 || g.K == 16)) {
       // children of the parent's K keys scored in registers (select_children_kernel)
       const size_t smem = select_children_smem_bytes(nc);
       const float* qpl = q_pyr + g.pyr_off[l];
@@ -794,6 +797,7 @@ llsa_status llsa_token_permute(const llsa_shape* s, const void* src, void* dst, 
   llsa_status st = validate(s);
   if (st != LLSA_OK) return st;
   if (!src || !dst || !aligned16(src) || !aligned16(dst) || src == dst) return LLSA_ERR_INVALID_ARG;
+  if (!is_pow2(s->N)) return LLSA_ERR_INVALID_ARG;
   const int lg = ilog2(s->N);
   if (lg & 1) return LLSA_ERR_INVALID_ARG;  // N must be a square grid: side = 2^(lg/2)
   const long long rows = (long long)s->B * s->H * s->N;

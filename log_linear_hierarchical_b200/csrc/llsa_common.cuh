@@ -50,7 +50,7 @@ constexpr int kQmUnroll = LLSA_QM_UNROLL;
 // Per-call geometry: level sizes and the level-major offsets of every packed buffer.
 struct Geometry {
   int B, H, N, D, K, L, BH;
-  int log_k, log_n1;                     // log2 K and log2 n_1 (both powers of two)
+  int log_k, log_n1;                     // log2 K and log2 n_1 where they are powers of two, else -1
   int n[kMaxLevels + 1];                 // n[l] = N / 16^l, l = 0..L
   long long pyr_off[kMaxLevels + 1];     // element offset of level l (1..L) in a pyramid
   long long idx_off[kMaxLevels + 1];     // element offset of level l in idx / col
@@ -65,10 +65,14 @@ struct Geometry {
                                          // level-1 mean is one more KV entry
 };
 
+// x / K and x / n_1, by a shift when the divisor is a power of two.
+__host__ __device__ inline int div_k(const Geometry& g, int x) { return g.log_k >= 0 ? x >> g.log_k : x / g.K; }
+__host__ __device__ inline int div_n1(const Geometry& g, int x) { return g.log_n1 >= 0 ? x >> g.log_n1 : x / g.n[1]; }
+
 // Level of coarse entry c (0 <= c < C): 2 + c / K, except that under the all-coarsest
 // variant the entries from top_first on are level L.
 __host__ __device__ inline int coarse_level(const Geometry& g, int c) {
-  return c >= g.top_first ? g.L : 2 + (c >> g.log_k);  // K = 2^log_k
+  return c >= g.top_first ? g.L : 2 + div_k(g, c);
 }
 
 // Additive score bias of coarse entry c under the log-count enrichment variant, in units
@@ -105,10 +109,11 @@ __device__ __forceinline__ int coarse_token(const Geometry& g, const int* __rest
     lev = g.L;
     return c - g.top_first;
   }
-  lev = 2 + (c >> g.log_k);
+  lev = 2 + div_k(g, c);
   const int nl = g.n[lev];
   const int anc = p >> (4 * (lev - 1));  // p / 16^(l-1)
-  return checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + anc) * g.K + (c & (g.K - 1))), nl);
+  const int slot = c - (lev - 2) * g.K;
+  return checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + anc) * g.K + slot), nl);
 }
 
 // ---------------------------------------------------------------------------- smem / swizzle

@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(kTrThreads) transpose_bucket_kernel(TransposeG
   }
   __syncthreads();
   int* rp = row_ptr + L.rp_off + (long long)bh * (L.n + 1);
-  for (int k = tid; k < W; k += kTrThreads) rp[kbase + k] = start + kpre[k];
+  for (int k = tid; k < W && kbase + k < L.n; k += kTrThreads) rp[kbase + k] = start + kpre[k];  // last bucket may be partial
   if (b == L.nb - 1 && tid == 0) rp[L.n] = start + size;
   // scatter queries to their final CSR slots
   for (int k = tid; k < W; k += kTrThreads) {

@@ -44,8 +44,13 @@ def shape(**kw):
 @pytest.mark.parametrize("kw,status", [
     ({}, 0),
     (dict(levels=1, N=1024, topk=8, dtype=1, H=2), 0),
-    (dict(N=3000), 1),                 # not a power of two
-    (dict(topk=6), 1),                 # not a power of two
+    (dict(N=3000), 1),                 # not a multiple of 16^L
+    (dict(N=3840), 1),                 # 15 * 256: not a multiple of 16^3
+    (dict(N=61440), 0),                # 15 * 4096: n_L = 15
+    (dict(N=12 * 4096), 0),            # a multiple of 16^L that is not a power of two: n_L = 12
+    (dict(levels=1, N=16 * 65, topk=5), 0),   # n_1 = 65, K = 5
+    (dict(topk=6), 0),                 # K need not be a power of two
+    (dict(topk=17), 1),                # topk > n_L = 16
     (dict(topk=32), 1),                # topk > n_L = 16
     (dict(N=2048), 1),                 # N < 16^L
     (dict(B=0), 1),

@@ -24,7 +24,7 @@ def int_vectors(rng, shape, lo=-2, hi=2):
     return rng.integers(lo, hi + 1, size=shape).astype(np.float32)
 
 
-@pytest.mark.parametrize("K", [1, 2, 4])
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 5])   # K need not be a power of two
 def test_single_level_equals_brute_force(K):
     rng = np.random.default_rng(100 + K)
     n, D = 16, 8

@@ -26,7 +26,7 @@ def dense_mask_transpose(idx, n_k):
     return np.array(row_ptr, dtype=np.int32), np.array(col, dtype=np.int32)
 
 
-@pytest.mark.parametrize("n,K", [(16, 1), (16, 4), (64, 8), (256, 16), (64, 64)])
+@pytest.mark.parametrize("n,K", [(16, 1), (16, 4), (64, 8), (256, 16), (64, 64), (48, 3), (80, 6)])
 def test_equals_dense_mask_transpose(n, K):
     rng = np.random.default_rng(n * 100 + K)
     idx = random_lists(rng, n, n, K)
