@@ -173,12 +173,14 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
   const uint32_t qd = smem_u32(cs.tiles(base, warp));
   const uint32_t ring = qd + 4 * kTileBytes;
   float* slse = reinterpret_cast<float*>(cs.tail(base, warp));  // [2][16]
-  int* sidx = reinterpret_cast<int*>(slse + 2 * kBlock);
-  const uint32_t bar_qd = smem_u32(sidx) + ((kUnitBlocks * K * 4 + 15) & ~15);
+  int* srow = reinterpret_cast<int*>(slse + 2 * kBlock);
+  const uint32_t bar_qd = smem_u32(srow) + ((kUnitBlocks * K * 4 + 15) & ~15);
   const uint32_t bar_kv = bar_qd + 16;
 
   for (int i = lane; i < nblk * K; i += 32)
-    sidx[i] = checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1);
+    // the first K/V row of each load: (b*H + h) * N + 16 j, computed here off the issue path
+    srow[i] = div_n1(g, first + div_k(g, i)) * g.N +
+              checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1) * kBlock;
   if (lane == 0) {
     for (int b = 0; b < 2 + STAGES; ++b) mbar_init(bar_qd + 8 * b, 1);
     mbar_fence_init();
@@ -187,8 +189,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int gb = first + div_k(g, seq);
-    const int row = div_n1(g, gb) * g.N + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
+    const int row = srow[seq];
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * kTileBytes;

@@ -294,12 +294,14 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   const int nblk = min(kUnitBlocks, total_blocks - first);
   const uint32_t sq = smem_u32(cs.tiles(base, warp));
   const uint32_t ring = sq + 2 * kTileBytes;
-  int* sidx = reinterpret_cast<int*>(cs.tail(base, warp));
-  const uint32_t bar_q = smem_u32(sidx) + ((kUnitBlocks * K * 4 + 15) & ~15);
+  int* srow = reinterpret_cast<int*>(cs.tail(base, warp));
+  const uint32_t bar_q = smem_u32(srow) + ((kUnitBlocks * K * 4 + 15) & ~15);
   const uint32_t bar_kv = bar_q + 16;
 
   for (int i = lane; i < nblk * K; i += 32)
-    sidx[i] = checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1);
+    // the first K/V row of each load: (b*H + h) * N + 16 j, computed here off the issue path
+    srow[i] = div_n1(g, first + div_k(g, i)) * g.N +
+              checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1) * kBlock;
   if (lane == 0) {
     for (int b = 0; b < 2 + STAGES; ++b) mbar_init(bar_q + 8 * b, 1);
     mbar_fence_init();
@@ -308,8 +310,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int gb = first + div_k(g, seq);
-    const int row = div_n1(g, gb) * g.N + sidx[seq] * kBlock;  // (b*H + h) * N + 16 j
+    const int row = srow[seq];
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * kTileBytes;
