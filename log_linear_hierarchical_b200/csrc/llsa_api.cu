@@ -413,16 +413,20 @@ llsa_status pyramid_launch(const Geometry& g, int dtype, const void* q, const vo
   if (dtype == LLSA_BF16) {
     constexpr int rows = kPyrThreads / (kD / 8);
     dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
+    constexpr int span = pyramid_span_bytes<__nv_bfloat16>();
+    if (!allow_smem(pyramid_l12_kernel<__nv_bfloat16>, span)) return LLSA_ERR_CUDA;
     st = launch(kKPyramidL12, cs, [&] {
-      launch_pdl(pyramid_l12_kernel<__nv_bfloat16>, dim3(grid), dim3(kPyrThreads), 0, cs, g,
+      launch_pdl(pyramid_l12_kernel<__nv_bfloat16>, dim3(grid), dim3(kPyrThreads), span, cs, g,
                  static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                  static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr);
     });
   } else {
     constexpr int rows = kPyrThreads / (kD / 4);
     dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
+    constexpr int span = pyramid_span_bytes<float>();
+    if (!allow_smem(pyramid_l12_kernel<float>, span)) return LLSA_ERR_CUDA;
     st = launch(kKPyramidL12, cs, [&] {
-      launch_pdl(pyramid_l12_kernel<float>, dim3(grid), dim3(kPyrThreads), 0, cs, g, static_cast<const float*>(q),
+      launch_pdl(pyramid_l12_kernel<float>, dim3(grid), dim3(kPyrThreads), span, cs, g, static_cast<const float*>(q),
                  static_cast<const float*>(k), static_cast<const float*>(v), q_pyr, k_pyr, v_pyr);
     });
   }

@@ -10,7 +10,9 @@
 // Bound: HBM streaming.  Reads B*H*N*D input elements of each of q, k, v once and writes
 // B*H*D*sum_l n_l fp32 values per tensor; levels 1 and 2 are produced by one kernel (the
 // 16 level-1 rows that make a level-2 row stay in shared memory), levels >= 3 by a small
-// kernel per level reading the L2-resident level below.
+// kernel per level reading the L2-resident level below.  The level-1/2 kernel brings its
+// input span (ROWS * 16 contiguous token rows, 64 KB) into shared memory with one bulk copy
+// completing on an mbarrier, so a CTA has its whole span in flight at once.
 #pragma once
 
 #include "llsa_common.cuh"
@@ -23,8 +25,8 @@ struct Vec16 {};
 template <>
 struct Vec16<__nv_bfloat16> {
   static constexpr int kElems = 8;
-  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&out)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&out)[8]) {  // shared memory
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -38,8 +40,8 @@ struct Vec16<__nv_bfloat16> {
 template <>
 struct Vec16<float> {
   static constexpr int kElems = 4;
-  __device__ __forceinline__ static void load(const float* p, float (&out)[4]) {
-    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+  __device__ __forceinline__ static void load(const float* p, float (&out)[4]) {  // shared memory
+    const float4 u = *reinterpret_cast<const float4*>(p);
     out[0] = u.x;
     out[1] = u.y;
     out[2] = u.z;
@@ -48,6 +50,12 @@ struct Vec16<float> {
 };
 
 constexpr int kPyrThreads = 256;
+
+// Dynamic shared memory of pyramid_l12_kernel<T>: its span of ROWS * 16 input rows.
+template <typename T>
+constexpr int pyramid_span_bytes() {
+  return (kPyrThreads / (kD / (16 / (int)sizeof(T)))) * kBlock * kD * (int)sizeof(T);
+}
 
 // grid.x = B*H * ceil(n_1 / rows_per_cta), grid.y = 3 (q, k, v).
 // Each thread owns kElems consecutive channels of one level-1 output row.
@@ -61,6 +69,8 @@ __global__ void __launch_bounds__(kPyrThreads) pyramid_l12_kernel(Geometry g, co
   constexpr int TPR = kD / VE;                   // threads per row
   constexpr int ROWS = kPyrThreads / TPR;         // level-1 rows per CTA (32 for bf16, 16 for fp32)
   __shared__ float s1[ROWS][kD];
+  __shared__ __align__(8) uint64_t bar_storage;
+  extern __shared__ __align__(128) uint8_t pyr_span[];  // ROWS * 16 input rows (pyramid_span_bytes)
 
   const T* x = blockIdx.y == 0 ? x0 : (blockIdx.y == 1 ? x1 : x2);
   float* pyr = blockIdx.y == 0 ? p0 : (blockIdx.y == 1 ? p1 : p2);
@@ -74,8 +84,24 @@ __global__ void __launch_bounds__(kPyrThreads) pyramid_l12_kernel(Geometry g, co
   const int c0 = (t % TPR) * VE;
   const int j1 = tile * ROWS + o;
 
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (t == 0) {
+    const uint32_t bytes = (uint32_t)(min(ROWS, n1 - tile * ROWS) * kBlock * kD * (int)sizeof(T));
+    mbar_expect_tx(bar, bytes);
+    bulk_load(smem_u32(pyr_span), x + ((long long)bh * g.N + (long long)tile * ROWS * kBlock) * kD, bytes, bar);
+  }
+  if (!mbar_wait(bar, 0)) {  // recorded as LLSA_ERR_TIMEOUT; give the copy one more bounded wait
+    mbar_wait(bar, 0);
+    return;
+  }
+
   if (j1 < n1) {
-    const T* src = x + ((long long)bh * g.N + (long long)j1 * kBlock) * kD + c0;
+    const T* src = reinterpret_cast<const T*>(pyr_span) + (o * kBlock) * kD + c0;
     float v[kBlock][VE];
 #pragma unroll
     for (int r = 0; r < kBlock; ++r) Vec16<T>::load(src + r * kD, v[r]);
