@@ -135,7 +135,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- algorithmic counts
 
-def workload_counts(cfg, pairs_l1: int, all_top: bool = False):
+def workload_counts(cfg, pairs_l1: int, all_top: bool = False, select_launches: int | None = None):
     """Algorithmic bytes and FLOPs per launch of each kernel for one step of ``cfg``.
 
     Per query block the forward gathers the KV list (T tokens x 64 channels x 2 bytes for K
@@ -178,7 +178,10 @@ def workload_counts(cfg, pairs_l1: int, all_top: bool = False):
         groups = bh * n[lev + 1]
         sel_bytes += groups * (16 * K * D * f4 + 16 * D * f4 + K * 4) + bh * n[lev] * K * 4
         sel_flops += 2 * bh * n[lev] * 16 * K * D
-    counts["select"] = dict(bytes=sel_bytes // L, flops=sel_flops // L)  # per launch (L per step)
+    # per launch: the step's selection work over its selection launches (L, or L - 1 when the
+    # level-2 selection runs inside the level-1 launch)
+    nsel = select_launches or L
+    counts["select"] = dict(bytes=sel_bytes // nsel, flops=sel_flops // nsel)
     # transpose: E entries over all levels; hist reads idx, scatter reads idx and writes the
     # bucketed entries, bucket reads them and writes col and row_ptr
     entries = sum(bh * n[lev] * K for lev in range(1, L + 1))
@@ -363,7 +366,8 @@ def run_ours(args):
     # algorithmic roofline of the dominant kernel
     rps, _ = buf.csr_levels()
     pairs_l1 = int(rps[0][..., -1].sum().item())
-    counts = workload_counts(cfg, pairs_l1, args.all_top)
+    sel_launches = round(kern["select"]["launches"] / args.steps) if "select" in kern else None
+    counts = workload_counts(cfg, pairs_l1, args.all_top, sel_launches)
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
     hbm_peak = peaks["hbm_gbs"] if peaks else 6650.0

@@ -59,3 +59,20 @@ def test_general_shape_step_and_plan_match_separate_calls():
     torch.cuda.synchronize()
     assert np.array_equal(buf.dk.float().cpu().numpy(), ref["dk"])
     plan.close()
+
+
+@pytest.mark.parametrize("topk", [2, 4])
+def test_four_levels_with_register_resident_selection_at_every_sparse_level(topk):
+    # L = 4 with K in {2, 4}: levels 3, 2 and 1 all take the register-resident children
+    # selection.  N(0,1) inputs: with smooth fields at N = 2^20 the most popular key blocks
+    # gather hundreds of query blocks and the bf16 rounding of P and dS before the dK product
+    # puts a few elements just over the bf16 bound
+    B, H, N, L = 1, 1, 1 << 18, 4
+    inputs = inputs_for(B, H, N, 64, "bf16", "normal", 63)
+    gpu = run_gpu(B, H, N, 64, topk, L, "bf16", inputs)
+    assert gpu["status"] == 0
+    check_pyramid_bitexact(inputs, gpu, L)
+    check_selection(gpu, topk)
+    check_transpose_bitexact(gpu)
+    ref = replay(inputs, gpu)
+    compare_outputs(gpu, ref, "bf16", ["o", "lse", "dq", "dk", "dv"])
