@@ -341,10 +341,10 @@ class LLSAPlan:
 
 class _LLSAFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, topk: int, levels: int):
+    def forward(ctx, q, k, v, topk: int, levels: int, flags: dict):
         B, H, N, D = q.shape
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        shape = make_shape(B, H, N, D, topk, levels, q.dtype)
+        shape = make_shape(B, H, N, D, topk, levels, q.dtype, **flags)
         buf = LLSABuffers.allocate(shape, q.device, q.dtype)
         llsa_forward_path(shape, q, k, v, buf)
         ctx.save_for_backward(q, k, v)
@@ -357,24 +357,27 @@ class _LLSAFunction(torch.autograd.Function):
         q, k, v = ctx.saved_tensors
         buf = ctx.buf
         llsa_backward_path(ctx.shape, q, k, v, do.contiguous(), buf)
-        return buf.dq, buf.dk, buf.dv, None, None
+        return buf.dq, buf.dk, buf.dv, None, None, None
 
 
-def llsa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk: int = 8, levels: int = 1) -> torch.Tensor:
+def llsa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk: int = 8, levels: int = 1,
+                   log_bias: bool = False, all_top: bool = False, level1: bool = False) -> torch.Tensor:
     """Drop-in for ``F.scaled_dot_product_attention(q, k, v)`` (non-causal, no dropout) on
-    [B, H, N, 64] CUDA tensors, bf16 or fp32, with LLSA's hierarchical block-sparse KV lists."""
-    return _LLSAFunction.apply(q, k, v, topk, levels)
+    [B, H, N, 64] CUDA tensors, bf16 or fp32, with LLSA's hierarchical block-sparse KV lists.
+    ``log_bias``, ``all_top`` and ``level1`` select the enrichment variants (see make_shape)."""
+    flags = dict(log_bias=log_bias, all_top=all_top, level1=level1)
+    return _LLSAFunction.apply(q, k, v, topk, levels, flags)
 
 
-def llsa_l1(q, k, v, block_size: int = 16, topk: int = 8):
+def llsa_l1(q, k, v, block_size: int = 16, topk: int = 8, **variants):
     """One pooled level (the README recommends it for sequences shorter than 16384 tokens)."""
     if block_size != 16:
         raise ValueError("block_size must be 16")
-    return llsa_attention(q, k, v, topk=topk, levels=1)
+    return llsa_attention(q, k, v, topk=topk, levels=1, **variants)
 
 
-def llsa_l2(q, k, v, block_size: int = 16, topk: int = 8):
+def llsa_l2(q, k, v, block_size: int = 16, topk: int = 8, **variants):
     """Two pooled levels (the README recommends it from 16384 tokens on)."""
     if block_size != 16:
         raise ValueError("block_size must be 16")
-    return llsa_attention(q, k, v, topk=topk, levels=2)
+    return llsa_attention(q, k, v, topk=topk, levels=2, **variants)

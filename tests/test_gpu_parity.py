@@ -141,16 +141,17 @@ def test_out_of_range_index_is_recorded_not_dereferenced():
     assert api.llsa_device_status() == 0   # cleared by the read
 
 
-def test_autograd_op_matches_buffers_path():
+@pytest.mark.parametrize("variants", [{}, dict(log_bias=True, all_top=True, level1=True)])
+def test_autograd_op_matches_buffers_path(variants):
     from log_linear_hierarchical_b200 import llsa_attention
     inputs = inputs_for(1, 2, 4096, 64, "bf16", "smooth", 9)
     q, k, v, do = (inputs[n].cuda() for n in ("q", "k", "v", "do"))
     q.requires_grad_(True)
     k.requires_grad_(True)
     v.requires_grad_(True)
-    o = llsa_attention(q, k, v, topk=4, levels=2)
+    o = llsa_attention(q, k, v, topk=4, levels=2, **variants)
     o.backward(do)
-    gpu = run_gpu(1, 2, 4096, 64, 4, 2, "bf16", inputs)
+    gpu = run_gpu(1, 2, 4096, 64, 4, 2, "bf16", inputs, **variants)
     assert np.array_equal(o.detach().float().cpu().numpy(), gpu["o"])
     assert np.array_equal(q.grad.float().cpu().numpy(), gpu["dq"])
     assert np.array_equal(k.grad.float().cpu().numpy(), gpu["dk"])
