@@ -5,7 +5,7 @@ One step = the whole hot path on one batch of device-resident synthetic input:
 pyramid -> hierarchical selection -> attention forward -> index transpose -> attention
 backward (five C-ABI calls, 12 kernel launches at the default workload).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 4]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload headline-65536]
 
 Multi-GPU runs (torchrun, one process per GPU) are weak-scaled independent replicas: every
 rank runs the whole workload on its own GPU, with no data-path collective; the step time is
@@ -275,12 +275,12 @@ def run_ours(args):
     import torch.nn.functional as F
 
     from log_linear_hierarchical_b200 import api
-    from synthetic import CONFIGS, make_config_inputs
+    from synthetic import WORKLOADS, make_config_inputs
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dist_init(world, local)
-    cfg = CONFIGS[args.config]
+    cfg = WORKLOADS[args.workload]
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     host = make_config_inputs(cfg, with_do=True)
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -585,9 +585,9 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    from synthetic import CONFIGS, make_config_inputs
+    from synthetic import WORKLOADS, make_config_inputs
 
-    cfg = CONFIGS[args.config]
+    cfg = WORKLOADS[args.workload]
     host = make_config_inputs(cfg, with_do=True)
     n1 = cfg.N // 16
     # size each step's sample so that warm-up + steps stay near two minutes
@@ -626,9 +626,9 @@ def run_profile(args):
     import torch
 
     from log_linear_hierarchical_b200 import api
-    from synthetic import CONFIGS, make_config_inputs
+    from synthetic import WORKLOADS, make_config_inputs
 
-    cfg = CONFIGS[args.config]
+    cfg = WORKLOADS[args.workload]
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     dev = {k: v.cuda() for k, v in make_config_inputs(cfg, with_do=True).items()}
     shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, **enrichment(args))
@@ -642,13 +642,19 @@ def run_profile(args):
         sys.exit(1)
 
 
+def _workload_names():
+    from synthetic import WORKLOADS
+    return WORKLOADS.keys()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=4, help="workload number (4 = the headline N=65536 step)")
+    ap.add_argument("--workload", default="headline-65536", choices=list(_workload_names()),
+                    help="synthetic workload (default: the headline N=65536 step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--profile", action="store_true", help="run only the steps (for ncu), print no metric")
     ap.add_argument("--log-bias", action="store_true",

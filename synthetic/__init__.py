@@ -4,7 +4,7 @@ This package holds only random-number recipes and token placement. It holds none
 of the attention method's arithmetic, so both the CUDA path's tests and the CPU
 oracle can draw identical inputs from it without sharing any method code.
 """
-from .configs import CONFIGS, WorkloadConfig, get_config  # noqa: F401
+from .configs import WORKLOADS, WorkloadConfig, workload  # noqa: F401
 from .generate import (  # noqa: F401
     make_config_inputs,
     make_inputs,

@@ -11,7 +11,7 @@ from dataclasses import dataclass
 
 @dataclass(frozen=True)
 class WorkloadConfig:
-    cfg_id: int
+    seed_base: int      # inputs are drawn with seed 1000 * seed_base + tensor slot
     name: str
     B: int
     H: int
@@ -44,19 +44,21 @@ class WorkloadConfig:
                 f"block={self.block} L={self.levels} topk={self.topk} {self.dtype} q/k={self.qk_kind}")
 
 
-CONFIGS = {
-    1: WorkloadConfig(1, "tiny-f32", B=1, H=2, N=1024, D=64, levels=1, topk=8, dtype="f32",
-                      qk_kind="normal", backward=True),
-    2: WorkloadConfig(2, "dit-s-4096", B=4, H=6, N=4096, D=64, levels=1, topk=16, dtype="bf16",
-                      qk_kind="smooth", backward=True),
-    3: WorkloadConfig(3, "two-level-16384", B=2, H=6, N=16384, D=64, levels=2, topk=8, dtype="bf16",
-                      qk_kind="smooth", backward=True),
-    4: WorkloadConfig(4, "headline-65536", B=1, H=6, N=65536, D=64, levels=3, topk=8, dtype="bf16",
-                      qk_kind="smooth", backward=True),
-    5: WorkloadConfig(5, "scaleout-262144", B=1, H=6, N=262144, D=64, levels=3, topk=16, dtype="bf16",
-                      qk_kind="smooth", backward=False),
-}
+WORKLOADS = {w.name: w for w in (
+    WorkloadConfig(1, "tiny-f32", B=1, H=2, N=1024, D=64, levels=1, topk=8, dtype="f32",
+                   qk_kind="normal", backward=True),
+    WorkloadConfig(2, "dit-s-4096", B=4, H=6, N=4096, D=64, levels=1, topk=16, dtype="bf16",
+                   qk_kind="smooth", backward=True),
+    WorkloadConfig(3, "two-level-16384", B=2, H=6, N=16384, D=64, levels=2, topk=8, dtype="bf16",
+                   qk_kind="smooth", backward=True),
+    WorkloadConfig(4, "headline-65536", B=1, H=6, N=65536, D=64, levels=3, topk=8, dtype="bf16",
+                   qk_kind="smooth", backward=True),
+    WorkloadConfig(5, "scaleout-262144", B=1, H=6, N=262144, D=64, levels=3, topk=16, dtype="bf16",
+                   qk_kind="smooth", backward=False),
+)}
 
 
-def get_config(cfg_id: int) -> WorkloadConfig:
-    return CONFIGS[cfg_id]
+def workload(name: str) -> WorkloadConfig:
+    """The workload of that name (tiny-f32, dit-s-4096, two-level-16384, headline-65536,
+    scaleout-262144)."""
+    return WORKLOADS[name]

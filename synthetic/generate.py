@@ -124,7 +124,7 @@ def make_config_inputs(cfg, with_do: bool | None = None) -> dict:
     """Inputs of one of the named workloads (seed base = its number)."""
     if with_do is None:
         with_do = cfg.backward
-    return make_inputs(cfg.B, cfg.H, cfg.N, cfg.D, cfg.dtype, cfg.qk_kind, cfg.cfg_id, with_do)
+    return make_inputs(cfg.B, cfg.H, cfg.N, cfg.D, cfg.dtype, cfg.qk_kind, cfg.seed_base, with_do)
 
 
 def to_f64_numpy(t: torch.Tensor) -> np.ndarray:

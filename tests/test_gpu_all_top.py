@@ -9,7 +9,7 @@ import torch
 from log_linear_hierarchical_b200 import api
 from llsa_testlib import (TORCH_DTYPE, check_pyramid_bitexact, check_selection, check_transpose_bitexact,
                           compare_outputs, inputs_for, replay, run_gpu)
-from synthetic import CONFIGS, make_config_inputs
+from synthetic import WORKLOADS, make_config_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -71,7 +71,7 @@ def test_all_top_changes_nothing_at_one_level_and_something_above():
 
 
 def test_all_top_step_and_plan_match_separate_calls():
-    cfg = CONFIGS[4]
+    cfg = WORKLOADS["headline-65536"]
     inputs = make_config_inputs(cfg)
     ref = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs, all_top=True)
     tdt = TORCH_DTYPE[cfg.dtype]

@@ -8,7 +8,7 @@ import torch
 from log_linear_hierarchical_b200 import api
 from llsa_testlib import (TORCH_DTYPE, check_pyramid_bitexact, check_selection, check_transpose_bitexact,
                           compare_outputs, inputs_for, replay, run_gpu)
-from synthetic import CONFIGS, make_config_inputs
+from synthetic import WORKLOADS, make_config_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -50,7 +50,7 @@ def test_log_bias_changes_the_result_when_there_are_coarse_tokens():
 
 
 def test_log_bias_step_and_plan_match_separate_calls():
-    cfg = CONFIGS[4]
+    cfg = WORKLOADS["headline-65536"]
     inputs = make_config_inputs(cfg)
     ref = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs, log_bias=True)
     tdt = TORCH_DTYPE[cfg.dtype]

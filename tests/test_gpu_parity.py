@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-from synthetic import CONFIGS, make_config_inputs
+from synthetic import WORKLOADS, make_config_inputs
 
 from llsa_testlib import (check_pyramid_bitexact, check_selection, check_transpose_bitexact, compare_outputs,
                           inputs_for, replay, run_gpu)
@@ -65,14 +65,14 @@ def test_degenerate_shapes(B, H, N, topk, levels, dtype):
 
 
 def test_tiny_workload_f32():
-    cfg = CONFIGS[1]
-    sel, rep = full_check(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, cfg.qk_kind, seed=cfg.cfg_id)
+    cfg = WORKLOADS["tiny-f32"]
+    sel, rep = full_check(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, cfg.qk_kind, seed=cfg.seed_base)
     assert sel["exact"] == sel["rows"]
 
 
-@pytest.mark.parametrize("cfg_id", [2, 3])
-def test_mid_workloads(cfg_id):
-    cfg = CONFIGS[cfg_id]
+@pytest.mark.parametrize("name", ["dit-s-4096", "two-level-16384"])
+def test_mid_workloads(name):
+    cfg = WORKLOADS[name]
     inputs = make_config_inputs(cfg)
     gpu = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs)
     assert gpu["status"] == 0
@@ -85,7 +85,7 @@ def test_mid_workloads(cfg_id):
 
 def test_headline_workload_full_size():
     """B=1 H=6 N=65536 L=3 K=8 bf16, the benchmarked step: every stage, every head."""
-    cfg = CONFIGS[4]
+    cfg = WORKLOADS["headline-65536"]
     inputs = make_config_inputs(cfg)
     gpu = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs)
     assert gpu["status"] == 0
@@ -101,7 +101,7 @@ def test_headline_workload_full_size():
 def test_scaleout_workload_forward_sampled():
     """B=1 H=6 N=262144 L=3 K=16 bf16, forward + transpose: pyramid, selection and CSR on
     every head, outputs on one head."""
-    cfg = CONFIGS[5]
+    cfg = WORKLOADS["scaleout-262144"]
     inputs = make_config_inputs(cfg, with_do=False)
     gpu = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs, backward=False)
     assert gpu["status"] == 0
@@ -113,7 +113,7 @@ def test_scaleout_workload_forward_sampled():
 
 
 def test_repeat_calls_are_deterministic():
-    cfg = CONFIGS[3]
+    cfg = WORKLOADS["two-level-16384"]
     inputs = make_config_inputs(cfg)
     a = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs)
     b = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs)

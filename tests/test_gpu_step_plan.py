@@ -6,7 +6,7 @@ import torch
 
 from log_linear_hierarchical_b200 import api
 from llsa_testlib import TORCH_DTYPE, run_gpu
-from synthetic import CONFIGS, make_config_inputs, make_inputs
+from synthetic import WORKLOADS, make_config_inputs, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -51,9 +51,9 @@ def flat(out):
     return {k: (v.ravel() if k in ("idx", "row_ptr", "col") else v) for k, v in out.items()}
 
 
-@pytest.mark.parametrize("cfg_id", [1, 3])
-def test_train_step_matches_separate_calls(cfg_id):
-    cfg = CONFIGS[cfg_id]
+@pytest.mark.parametrize("name", ["tiny-f32", "two-level-16384"])
+def test_train_step_matches_separate_calls(name):
+    cfg = WORKLOADS[name]
     inputs = make_config_inputs(cfg)
     ref = separate_calls(cfg, inputs)
     shape, dev, buf = setup(cfg, inputs)
@@ -64,7 +64,7 @@ def test_train_step_matches_separate_calls(cfg_id):
 
 
 def test_train_step_without_side_stream():
-    cfg = CONFIGS[3]
+    cfg = WORKLOADS["two-level-16384"]
     inputs = make_config_inputs(cfg)
     ref = separate_calls(cfg, inputs)
     shape, dev, buf = setup(cfg, inputs)
@@ -75,7 +75,7 @@ def test_train_step_without_side_stream():
 
 
 def test_plan_replays_match_separate_calls():
-    cfg = CONFIGS[3]
+    cfg = WORKLOADS["two-level-16384"]
     inputs = make_config_inputs(cfg)
     ref = separate_calls(cfg, inputs)
     shape, dev, buf = setup(cfg, inputs)
@@ -88,7 +88,7 @@ def test_plan_replays_match_separate_calls():
         assert api.llsa_device_status() == 0
         assert_same(flat(outputs(buf)), ref)
     # the plan reads its inputs at launch time: new inputs in the same buffers, new results
-    other = make_inputs(cfg.B, cfg.H, cfg.N, cfg.D, cfg.dtype, cfg.qk_kind, cfg.cfg_id + 100)
+    other = make_inputs(cfg.B, cfg.H, cfg.N, cfg.D, cfg.dtype, cfg.qk_kind, cfg.seed_base + 100)
     ref2 = separate_calls(cfg, other)
     for k in ("q", "k", "v", "do"):
         dev[k].copy_(other[k].cuda())
@@ -99,7 +99,7 @@ def test_plan_replays_match_separate_calls():
 
 
 def test_plan_is_traced_at_every_launch():
-    cfg = CONFIGS[3]
+    cfg = WORKLOADS["two-level-16384"]
     inputs = make_config_inputs(cfg)
     shape, dev, buf = setup(cfg, inputs)
     with api.LaunchTrace(64) as eager:
@@ -121,7 +121,7 @@ def test_plan_headline_matches_serialized_calls():
     """Full headline size: the plan (kernels chained by programmatic dependent launch, dK/dV
     overlapping the coarse reduction) against the five calls run with trace events between
     every kernel, which serialises them; bit for bit over three replays."""
-    cfg = CONFIGS[4]
+    cfg = WORKLOADS["headline-65536"]
     inputs = make_config_inputs(cfg)
     shape, dev, buf = setup(cfg, inputs)
     with api.LaunchTrace(64):

@@ -2,7 +2,7 @@
 import numpy as np
 import torch
 
-from synthetic import CONFIGS, make_inputs, morton_order, quadtree_order_recursive
+from synthetic import WORKLOADS, make_inputs, morton_order, quadtree_order_recursive
 
 
 def test_morton_matches_recursive_quadrants():
@@ -61,6 +61,6 @@ def test_smooth_fields_are_spatially_smooth():
 
 
 def test_config_table():
-    assert [CONFIGS[i].N for i in range(1, 6)] == [1024, 4096, 16384, 65536, 262144]
-    assert CONFIGS[4].level_sizes() == [65536, 4096, 256, 16]
-    assert CONFIGS[4].kv_len == 144 and CONFIGS[5].kv_len == 288
+    assert [w.N for w in WORKLOADS.values()] == [1024, 4096, 16384, 65536, 262144]
+    assert WORKLOADS["headline-65536"].level_sizes() == [65536, 4096, 256, 16]
+    assert WORKLOADS["headline-65536"].kv_len == 144 and WORKLOADS["scaleout-262144"].kv_len == 288

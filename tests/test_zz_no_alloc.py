@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from log_linear_hierarchical_b200 import _lib, api
-from synthetic import CONFIGS, make_config_inputs
+from synthetic import WORKLOADS, make_config_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -35,7 +35,7 @@ def _selection(cfg):
 def test_noalloc_transpose_equals_workspace_transpose_on_consecutive_calls():
     # two calls in a row on different workloads: the second reuses the scratch array that
     # the first left behind
-    for cfg in (CONFIGS[4], CONFIGS[3]):
+    for cfg in (WORKLOADS["headline-65536"], WORKLOADS["two-level-16384"]):
         shape, buf = _selection(cfg)
         assert api.llsa_transpose_workspace_bytes(shape) <= _lib.NOALLOC_SCRATCH_BYTES
         api.llsa_index_transpose(shape, buf.idx, buf.row_ptr, buf.col, buf.ws_transpose)
