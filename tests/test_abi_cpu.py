@@ -66,6 +66,19 @@ def test_validation(lib, kw, status):
     assert api.llsa_validate_shape(shape(**kw)) == status
 
 
+@pytest.mark.parametrize("B,H,N,K,L", [(2, 3, 12288, 6, 2), (1, 2, 1040, 5, 1), (1, 1, 61440, 12, 3)])
+def test_sizes_match_layout_at_general_shapes(lib, B, H, N, K, L):
+    # n_l = N / 16^l need not be powers of two, nor K
+    s = api.make_shape(B, H, N, 64, K, L, 0)
+    assert api.llsa_validate_shape(s) == 0
+    n = [N // 16 ** l for l in range(1, L + 1)]
+    assert api.llsa_pyramid_elems(s) == B * H * 64 * sum(n)
+    assert api.llsa_index_elems(s) == B * H * K * sum(n)
+    assert api.llsa_row_ptr_elems(s) == B * H * sum(x + 1 for x in n)
+    assert api.llsa_transpose_workspace_bytes(s) >= 4 * B * H * K * sum(n)
+    assert api.llsa_backward_workspace_bytes(s) >= 4 * B * H * N
+
+
 def test_sizes_match_layout(lib):
     s = shape()
     n = [4096, 256, 16]
