@@ -1,6 +1,8 @@
 """Pins for the oracle's quadtree (Z) token order, on CPU: a recursive quadrant
 construction written independently of the oracle's bit interleave, bijection, and the
 round trip."""
+import os
+
 import numpy as np
 import pytest
 
@@ -52,3 +54,28 @@ def test_round_trip_and_neighbourhoods():
     assert np.all(r.max(1) - r.min(1) == 3) and np.all(c.max(1) - c.min(1) == 3)
     with pytest.raises(ValueError):
         to_z_order(np.zeros((1, 1, 8, 2)))
+
+
+def _golden_zorder():
+    """Sections of tests/golden/zorder_grid_4x4.txt (values from the README's token
+    reordering example; see the file's header)."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "zorder_grid_4x4.txt")
+    sections, name = {}, None
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line[0].isalpha():
+            name = line
+            sections[name] = []
+        else:
+            sections[name].append([int(t) for t in line.split()])
+    return {k: np.array(v) for k, v in sections.items()}
+
+
+def test_zorder_matches_the_readme_example():
+    g = _golden_zorder()
+    assert np.array_equal(zorder_index(2).reshape(2, 2), g["grid2"])
+    assert np.array_equal(zorder_index(4).reshape(4, 4), g["grid4"])
+    tokens = np.arange(16, dtype=np.float64).reshape(1, 1, 16, 1)
+    assert np.array_equal(to_z_order(tokens)[0, 0, :, 0].astype(int), g["order4"][0])
