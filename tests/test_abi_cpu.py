@@ -170,3 +170,22 @@ def test_token_permute_rejected_before_launch(lib):
     assert lib.llsa_token_permute(ctypes.byref(s), 256, 256, 1, None) == 1   # in place
     assert lib.llsa_token_permute(ctypes.byref(s), None, 256, 0, None) == 1
     assert lib.llsa_token_permute(ctypes.byref(s), 264, 512, 0, None) == 1   # misaligned
+
+
+def test_variant_flags_change_only_the_backward_workspace(lib):
+    base = api.make_shape(1, 6, 65536, 64, 8, 3, 0)
+    for kw in (dict(log_bias=True), dict(level1=True), dict(all_top=True), dict(all_top=True, level1=True)):
+        s = api.make_shape(1, 6, 65536, 64, 8, 3, 0, **kw)
+        for fn in (api.llsa_pyramid_elems, api.llsa_index_elems, api.llsa_row_ptr_elems,
+                   api.llsa_transpose_workspace_bytes):
+            assert fn(s) == fn(base), (kw, fn.__name__)
+        ws, ws0 = api.llsa_backward_workspace_bytes(s), api.llsa_backward_workspace_bytes(base)
+        if kw.get("all_top"):
+            # coarse partials [B*H*n_2][C][64] for dK and dV: C goes from (L-1) K = 16 to
+            # (L-2) K + n_L = 24
+            assert ws - ws0 >= 2 * 4 * 6 * 256 * (24 - 16) * 64
+        else:
+            assert ws == ws0
+    one = api.make_shape(1, 2, 4096, 64, 8, 1, 0)
+    assert api.llsa_backward_workspace_bytes(api.make_shape(1, 2, 4096, 64, 8, 1, 0, all_top=True)) == \
+        api.llsa_backward_workspace_bytes(one)   # L = 1: no coarse entries either way
