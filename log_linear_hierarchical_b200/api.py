@@ -43,12 +43,49 @@ def _check(fn: str, status: int) -> None:
         raise LLSAError(fn, status)
 
 
-def _p(t: torch.Tensor | None) -> int | None:
+def _p(t: torch.Tensor | None, name: str = "buffer") -> int | None:
+    """Device address of a contiguous CUDA tensor on the current device.  The library reads
+    and writes these addresses from its kernels, so a host tensor or one on another device
+    is refused here rather than faulting there."""
     if t is None:
         return None
     if not t.is_contiguous():
-        raise ValueError("LLSA buffers must be contiguous")
+        raise ValueError(f"{name}: LLSA buffers must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: LLSA buffers must be CUDA tensors (the kernels read device memory)")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name}: on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
     return t.data_ptr()
+
+
+_ACT_DTYPE = {0: torch.bfloat16, 1: torch.float32}  # LLSA_BF16, LLSA_F32
+
+
+def _act(shape: LLSAShape, t: torch.Tensor, name: str) -> tuple:
+    """An activation (q, k, v, o, dO, dq, dk, dv, a permute's src or dst): the shape's dtype
+    and exactly B*H*N*D elements.  Returns (t, name) for _ptrs."""
+    want = _ACT_DTYPE.get(shape.dtype)
+    if t.dtype != want:
+        raise ValueError(f"{name}: dtype {t.dtype}, but the shape is {want}")
+    n = shape.B * shape.H * shape.N * shape.D
+    if t.numel() != n:
+        raise ValueError(f"{name}: {t.numel()} elements, but the shape needs B*H*N*D = {n}")
+    return t, name
+
+
+def _buf(t: torch.Tensor, dtype: torch.dtype, need: int, name: str) -> tuple:
+    """An internal buffer (pyramid, indices, CSR, LSE): its dtype and at least ``need`` elements."""
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.numel() < need:
+        raise ValueError(f"{name}: {t.numel()} elements, the shape needs {need}")
+    return t, name
+
+
+def _ptrs(*checked) -> list:
+    """Device addresses of (tensor, name) pairs whose dtype and size were checked: every
+    argument's shape is checked before any one's residency."""
+    return [_p(t, name) for t, name in checked]
 
 
 def _stream(stream) -> int | None:
@@ -91,46 +128,70 @@ def llsa_backward_workspace_bytes(shape: LLSAShape) -> int:
 
 # ----------------------------------------------------------------------------- the five calls
 
+def _pyr(shape, t, name):
+    return _buf(t, torch.float32, llsa_pyramid_elems(shape), name)
+
+
+def _idx(shape, t, name):
+    return _buf(t, torch.int32, llsa_index_elems(shape), name)
+
+
+def _rp(shape, t, name):
+    return _buf(t, torch.int32, llsa_row_ptr_elems(shape), name)
+
+
+def _lse(shape, t, name="lse"):
+    return _buf(t, torch.float32, shape.B * shape.H * shape.N, name)
+
+
 def llsa_build_pyramid(shape, q, k, v, q_pyr, k_pyr, v_pyr, stream=None) -> None:
-    _check("llsa_build_pyramid", _lib.load().llsa_build_pyramid(
-        _ref(shape), _p(q), _p(k), _p(v), _p(q_pyr), _p(k_pyr), _p(v_pyr), _stream(stream)))
+    args = _ptrs(_act(shape, q, "q"), _act(shape, k, "k"), _act(shape, v, "v"), _pyr(shape, q_pyr, "q_pyr"),
+            _pyr(shape, k_pyr, "k_pyr"), _pyr(shape, v_pyr, "v_pyr"))
+    _check("llsa_build_pyramid", _lib.load().llsa_build_pyramid(_ref(shape), *args, _stream(stream)))
 
 
 def llsa_select(shape, q_pyr, k_pyr, idx, stream=None) -> None:
-    _check("llsa_select", _lib.load().llsa_select(_ref(shape), _p(q_pyr), _p(k_pyr), _p(idx), _stream(stream)))
+    args = _ptrs(_pyr(shape, q_pyr, "q_pyr"), _pyr(shape, k_pyr, "k_pyr"), _idx(shape, idx, "idx"))
+    _check("llsa_select", _lib.load().llsa_select(_ref(shape), *args, _stream(stream)))
 
 
 def llsa_index_transpose(shape, idx, row_ptr, col, workspace, stream=None) -> None:
     nbytes = workspace.numel() * workspace.element_size()
-    _check("llsa_index_transpose", _lib.load().llsa_index_transpose(
-        _ref(shape), _p(idx), _p(row_ptr), _p(col), _p(workspace), nbytes, _stream(stream)))
+    args = _ptrs(_idx(shape, idx, "idx"), _rp(shape, row_ptr, "row_ptr"), _idx(shape, col, "col"),
+            (workspace, "workspace"))
+    _check("llsa_index_transpose", _lib.load().llsa_index_transpose(_ref(shape), *args, nbytes, _stream(stream)))
 
 
 def llsa_index_transpose_noalloc(shape, idx, row_ptr, col, stream=None) -> None:
     """llsa_index_transpose without a workspace, for callers that cannot allocate device
     memory: the library's own fixed 8 MiB scratch array is used (calls on overlapping
     streams race on it; the first call on a device must precede any stream capture)."""
-    _check("llsa_index_transpose_noalloc", _lib.load().llsa_index_transpose_noalloc(
-        _ref(shape), _p(idx), _p(row_ptr), _p(col), _stream(stream)))
+    args = _ptrs(_idx(shape, idx, "idx"), _rp(shape, row_ptr, "row_ptr"), _idx(shape, col, "col"))
+    _check("llsa_index_transpose_noalloc", _lib.load().llsa_index_transpose_noalloc(_ref(shape), *args,
+                                                                                  _stream(stream)))
 
 
 def llsa_forward(shape, q, k, v, k_pyr, v_pyr, idx, o, lse, stream=None) -> None:
-    _check("llsa_forward", _lib.load().llsa_forward(
-        _ref(shape), _p(q), _p(k), _p(v), _p(k_pyr), _p(v_pyr), _p(idx), _p(o), _p(lse), _stream(stream)))
+    args = _ptrs(_act(shape, q, "q"), _act(shape, k, "k"), _act(shape, v, "v"), _pyr(shape, k_pyr, "k_pyr"),
+            _pyr(shape, v_pyr, "v_pyr"), _idx(shape, idx, "idx"), _act(shape, o, "o"), _lse(shape, lse))
+    _check("llsa_forward", _lib.load().llsa_forward(_ref(shape), *args, _stream(stream)))
 
 
 def llsa_backward(shape, q, k, v, o, lse, do, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace,
                   stream=None) -> None:
     nbytes = workspace.numel() * workspace.element_size()
-    _check("llsa_backward", _lib.load().llsa_backward(
-        _ref(shape), _p(q), _p(k), _p(v), _p(o), _p(lse), _p(do), _p(k_pyr), _p(v_pyr), _p(idx), _p(row_ptr),
-        _p(col), _p(dq), _p(dk), _p(dv), _p(workspace), nbytes, _stream(stream)))
+    args = _ptrs(_act(shape, q, "q"), _act(shape, k, "k"), _act(shape, v, "v"), _act(shape, o, "o"), _lse(shape, lse),
+            _act(shape, do, "do"), _pyr(shape, k_pyr, "k_pyr"), _pyr(shape, v_pyr, "v_pyr"), _idx(shape, idx, "idx"),
+            _rp(shape, row_ptr, "row_ptr"), _idx(shape, col, "col"), _act(shape, dq, "dq"), _act(shape, dk, "dk"),
+            _act(shape, dv, "dv"), (workspace, "workspace"))
+    _check("llsa_backward", _lib.load().llsa_backward(_ref(shape), *args, nbytes, _stream(stream)))
 
 
 def llsa_token_permute(shape, src, dst, to_z_order: bool = True, stream=None) -> None:
     """Quadtree (Z) token order of a square token grid: row-major -> Z (``to_z_order``) or
     back; src and dst are distinct [B, H, N, D] tensors."""
-    _check("llsa_token_permute", _lib.load().llsa_token_permute(_ref(shape), _p(src), _p(dst), int(bool(to_z_order)),
+    args = _ptrs(_act(shape, src, "src"), _act(shape, dst, "dst"))
+    _check("llsa_token_permute", _lib.load().llsa_token_permute(_ref(shape), *args, int(bool(to_z_order)),
                                                                 _stream(stream)))
 
 
@@ -275,13 +336,13 @@ def llsa_backward_path(shape, q, k, v, do, buf: LLSABuffers, stream=None) -> Non
 
 def step_buffers(shape, q, k, v, do, buf: LLSABuffers) -> _lib.LLSAStepBuffers:
     """The ``llsa_step_buffers`` of one step over ``buf`` (raw device addresses)."""
-    for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
-        if not t.is_contiguous():
-            raise ValueError(f"{name} must be contiguous")
-    return _lib.LLSAStepBuffers(
-        _p(q), _p(k), _p(v), _p(do), _p(buf.q_pyr), _p(buf.k_pyr), _p(buf.v_pyr), _p(buf.idx), _p(buf.row_ptr),
-        _p(buf.col), _p(buf.o), _p(buf.lse), _p(buf.dq), _p(buf.dk), _p(buf.dv),
-        _p(buf.ws_transpose), buf.ws_transpose.numel() * 4, _p(buf.ws_backward), buf.ws_backward.numel() * 4)
+    p = _ptrs(
+        _act(shape, q, "q"), _act(shape, k, "k"), _act(shape, v, "v"), _act(shape, do, "do"),
+        _pyr(shape, buf.q_pyr, "q_pyr"), _pyr(shape, buf.k_pyr, "k_pyr"), _pyr(shape, buf.v_pyr, "v_pyr"),
+        _idx(shape, buf.idx, "idx"), _rp(shape, buf.row_ptr, "row_ptr"), _idx(shape, buf.col, "col"),
+        _act(shape, buf.o, "o"), _lse(shape, buf.lse), _act(shape, buf.dq, "dq"), _act(shape, buf.dk, "dk"),
+        _act(shape, buf.dv, "dv"), (buf.ws_transpose, "ws_transpose"), (buf.ws_backward, "ws_backward"))
+    return _lib.LLSAStepBuffers(*p[:16], buf.ws_transpose.numel() * 4, p[16], buf.ws_backward.numel() * 4)
 
 
 _side_streams: dict[int, torch.cuda.Stream] = {}

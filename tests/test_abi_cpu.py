@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from log_linear_hierarchical_b200 import _lib
 from log_linear_hierarchical_b200 import api
@@ -189,3 +190,28 @@ def test_variant_flags_change_only_the_backward_workspace(lib):
     one = api.make_shape(1, 2, 4096, 64, 8, 1, 0)
     assert api.llsa_backward_workspace_bytes(api.make_shape(1, 2, 4096, 64, 8, 1, 0, all_top=True)) == \
         api.llsa_backward_workspace_bytes(one)   # L = 1: no coarse entries either way
+
+
+def test_binding_refuses_tensors_the_kernels_would_misread():
+    # wrong dtype, wrong size or host memory is refused before anything is launched
+    B, H, N, K, L = 1, 2, 4096, 4, 2
+    shape = api.make_shape(B, H, N, 64, K, L, torch.bfloat16)
+    act = lambda dt=torch.bfloat16, n=B * H * N * 64: torch.zeros(n, dtype=dt)  # noqa: E731
+    pyr = torch.zeros(api.llsa_pyramid_elems(shape), dtype=torch.float32)
+    idx = torch.zeros(api.llsa_index_elems(shape), dtype=torch.int32)
+    lse = torch.zeros(B * H * N, dtype=torch.float32)
+    cases = [
+        (dict(q=act(torch.float32)), "q: dtype"),            # fp32 under a bf16 shape
+        (dict(k=act(n=B * H * N * 64 - 64)), "k: "),          # one token short
+        (dict(idx=idx.float()), "idx: dtype"),
+        (dict(k_pyr=pyr[:-1]), "k_pyr: "),                    # pyramid too small
+        (dict(lse=lse[: B * H * N // 2]), "lse: "),
+        ({}, "CUDA"),                                         # everything right but on the host
+    ]
+    for override, msg in cases:
+        args = dict(q=act(), k=act(), v=act(), k_pyr=pyr, v_pyr=pyr, idx=idx, o=act(), lse=lse)
+        args.update(override)
+        with pytest.raises(ValueError, match=msg):
+            api.llsa_forward(shape, **args)
+    with pytest.raises(ValueError, match="dst: dtype"):
+        api.llsa_token_permute(shape, act(), act(torch.float32))
