@@ -26,10 +26,10 @@ def full_idx(B, H, n_q, n_k):
     return np.broadcast_to(np.arange(n_k, dtype=np.int32), (B, H, n_q, n_k)).copy()
 
 
-@pytest.mark.parametrize("N", [256, 768])   # 768: n_1 = 48, not a power of two
-def test_single_level_all_blocks_is_dense_attention(N):
+@pytest.mark.parametrize("N,D", [(256, 16), (768, 16), (256, 128)])   # 768: n_1 = 48; D = 128 for wider heads
+def test_single_level_all_blocks_is_dense_attention(N, D):
     rng = np.random.default_rng(0)
-    B, H, D = 1, 2, 16
+    B, H = 1, 2
     q, k, v, do = (rand(rng, B, H, N, D) for _ in range(4))
     kp, vp = build_pyramid(k, 1, np.float64), build_pyramid(v, 1, np.float64)
     idx = [full_idx(B, H, N // 16, N // 16)]
