@@ -614,7 +614,9 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the CUDA arm)",
         "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
-                   "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk},
+                   "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk,
+                   "kv_len": 16 * cfg.topk + (cfg.topk if args.level1 else 0) + coarse_entries(cfg, args.all_top),
+                   "enrichment": enrichment_text(args)},
         "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
