@@ -424,13 +424,37 @@ def llsa_step(q, k, v, do, levels: int, topk: int, log_bias: bool = False, all_t
 # ----------------------------------------------------------------------------- selection check
 
 def dot_error_floor(q_rows: np.ndarray, k_rows: np.ndarray) -> np.ndarray:
-    """Forward error bound of an fp32 length-D dot product, gamma_D * sum_d |q_d k_d| / sqrt(D)
-    with gamma_D = D u / (1 - D u), u = 2^-24 (Higham, Accuracy and Stability of
-    Numerical Algorithms, section 3.1).  Used only as the absolute floor of the tie window."""
+    """Forward error bound of one fp32 length-D dot product, in the units of the scaled
+    score: gamma_D * sum_d |q_d k_d| / sqrt(D) with gamma_D = D u / (1 - D u) and
+    u = 2^-24 (Higham, Accuracy and Stability of Numerical Algorithms, 2nd ed., section 3.1,
+    bound (3.5)).  It holds for any summation order, with or without fused multiply-adds.
+    Returns one bound per (query row, key row) pair: [Rq, Rk]."""
     D = q_rows.shape[-1]
     u = 2.0 ** -24
     gamma = D * u / (1.0 - D * u)
     return gamma * (np.abs(q_rows.astype(np.float64)) @ np.abs(k_rows.astype(np.float64)).T) / math.sqrt(D)
+
+
+def _row_verdict(s: np.ndarray, fl: np.ndarray, cand: np.ndarray, selm: np.ndarray, rel_tol: float) -> str:
+    """Classify one row whose selected set ``selm`` differs from the oracle's Top-K.
+
+    Every (selected x, rejected y) pair that the oracle orders the other way (s_y > s_x,
+    or equal scores with y the lower index) must be a near tie: s_y - s_x below
+    rel_tol * max(|s_x|, |s_y|) (the stated window), or else below the sum of the two
+    scores' fp32 error bounds fl_x + fl_y (a selection computed in fp32 can only invert
+    such a pair).  Returns "tie_window", "floor" (some pair needed the fp32 bound) or "bad".
+    """
+    sx, sy = s[selm][:, None], s[~selm][None, :]
+    ix, iy = cand[selm][:, None], cand[~selm][None, :]
+    gap = sy - sx
+    inverted = (gap > 0) | ((gap == 0) & (iy < ix))
+    if not inverted.any():          # cannot happen for a row that differs from the Top-K
+        return "tie_window"
+    rel = rel_tol * np.maximum(np.abs(sx), np.abs(sy))
+    pair_floor = fl[selm][:, None] + fl[~selm][None, :]
+    if np.any(inverted & (gap > np.maximum(rel, pair_floor))):
+        return "bad"
+    return "floor" if np.any(inverted & (gap > rel)) else "tie_window"
 
 
 def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5) -> dict:
@@ -438,11 +462,12 @@ def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5) ->
 
     At level l the candidates of query a are taken from ``idx_test`` at level l+1 (so a
     near-tie swap above does not cascade into failures below).  A row passes if it is
-    the oracle's Top-K exactly, or if it is a valid Top-K under the tie window: the
-    lowest selected score is at least the highest rejected score minus
-    max(rel_tol * max(|s_sel|, |s_rej|), fp32 dot-product error floor).
-    Returns counts: exact rows, tie-window rows, rows that used the absolute floor,
-    bad rows, and the first few bad rows for diagnosis.
+    the oracle's Top-K exactly, or if every pair it orders differently from the oracle is
+    a near tie (``_row_verdict``): within rel_tol relative, or within the fp32 error bounds
+    of the pair's two scores.
+    Returns counts: exact rows, rows accepted by the relative window alone
+    (``tie_window``), rows that needed the fp32 bound of some pair (``floor_used``, also
+    counted in ``tie_window``), bad rows, and the first few bad rows for diagnosis.
     """
     L = len(q_pyr)
     res = {"rows": 0, "exact": 0, "tie_window": 0, "floor_used": 0, "bad": 0, "bad_examples": []}
@@ -472,20 +497,14 @@ def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5) ->
                         pos = np.searchsorted(cand, got)
                         valid = (np.all(np.diff(got) > 0) and np.all(pos < cand.size)
                                  and np.array_equal(cand[np.minimum(pos, cand.size - 1)], got))
-                        ok = False
-                        used_floor = False
+                        verdict = "bad"
                         if valid:
                             selm = np.zeros(cand.size, dtype=bool)
                             selm[pos] = True
-                            lo = s[r, selm].min()
-                            hi = s[r, ~selm].max() if (~selm).any() else -np.inf
-                            rel = rel_tol * max(abs(lo), abs(hi))
-                            fl = max(floor[r, selm].max(), floor[r, ~selm].max() if (~selm).any() else 0.0)
-                            ok = lo >= hi - max(rel, fl)
-                            used_floor = ok and not (lo >= hi - rel)
-                        if ok:
+                            verdict = _row_verdict(s[r], floor[r], cand, selm, rel_tol)
+                        if verdict != "bad":
                             res["tie_window"] += 1
-                            res["floor_used"] += int(used_floor)
+                            res["floor_used"] += int(verdict == "floor")
                         else:
                             res["bad"] += 1
                             if len(res["bad_examples"]) < 5:

@@ -65,9 +65,19 @@ def check_pyramid_bitexact(inputs, gpu, levels):
                 raise AssertionError(f"{name} pyramid level {lev + 1} differs at {bad.tolist()}")
 
 
+# Rows whose selection needed the fp32 error bound of a pair (beyond the stated 1e-5
+# relative window) may be at most this fraction of all rows, plus FLOOR_ROWS_SLACK.
+FLOOR_ROWS_FRACTION = 1e-3
+FLOOR_ROWS_SLACK = 2
+
+
 def check_selection(gpu, topk):
+    """Selection parity: no bad row, and few rows that lean on the fp32 bound."""
     res = orc.check_selection(gpu["q_pyr"], gpu["k_pyr"], gpu["idx"], topk)
     assert res["bad"] == 0, res
+    assert res["floor_used"] <= FLOOR_ROWS_FRACTION * res["rows"] + FLOOR_ROWS_SLACK, res
+    print("selection rows", res["rows"], "exact", res["exact"], "tie window", res["tie_window"],
+          "fp32 bound", res["floor_used"])
     return res
 
 
@@ -100,30 +110,47 @@ def max_err(a, b):
 
 
 def bf16_half_ulp(x):
-    """Half a unit in the last place of bf16 (8 significant bits) at |x|: the error of
-    storing an exact value in the output format alone, bounded by |x| * 2^-8."""
-    return np.abs(np.asarray(x, np.float64)) * 2.0 ** -8
+    """Half a unit in the last place of bf16 (8 significant bits) at |x|: the most that
+    storing an exact value in the output format changes it, 2^(floor(log2 |x|) - 8)."""
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.where(a > 0, 2.0 ** (e - 8), 0.0)
+
+
+# From |ref| = 8 on, the bf16 output store alone can change a value by 2^-5 > 2e-2.
+BF16_STORE_FROM = 8.0
+
+
+def output_limit(ref, dtype, name):
+    """Per-element bound of |gpu - ref|.  fp32 outputs: 1e-4.  bf16 outputs: 2e-2, plus the
+    bf16 store's half-ulp where |ref| >= 8 (there the rounding of the stored result alone
+    exceeds 2e-2).  LSE is fp32 in both dtypes: 1e-4, or 1e-2 on the bf16 path (coarse K/V
+    rows are rounded to bf16 before the score products)."""
+    r = np.asarray(ref, np.float64)
+    if name == "lse":
+        return np.full_like(r, 1e-4 if dtype == "f32" else 1e-2)
+    if dtype == "bf16":
+        return TOL["bf16"] + np.where(np.abs(r) >= BF16_STORE_FROM, bf16_half_ulp(r), 0.0)
+    return np.full_like(r, TOL[dtype])
 
 
 def compare_outputs(gpu, ref, dtype, names, heads=None):
-    """Element-wise check: |gpu - ref| <= tol (+ the bf16 output half-ulp of ref for bf16
-    outputs, since a bf16 store alone errs by up to |ref| * 2^-8, more than 2e-2 once
-    |ref| > 5).  LSE is fp32 in both dtypes."""
-    tol = TOL[dtype]
+    """Element-wise check |gpu - ref| <= output_limit.  The report records, per output, the
+    largest error, the largest |ref|, the worst excess over the bound, and how many elements
+    exceed the plain stated tolerance (2e-2 bf16, 1e-4 fp32) -- only elements with
+    |ref| >= 8 can do so and still pass."""
     report = {}
     for n in names:
         g = np.asarray(gpu[n] if heads is None else gpu[n][heads[0]:heads[0] + 1, heads[1]], np.float64)
         r = np.asarray(ref[n], np.float64)
         err = np.abs(g - r)
-        if n == "lse":
-            lim = np.full_like(r, 1e-4 if dtype == "f32" else 1e-2)
-        elif dtype == "bf16":
-            lim = tol + bf16_half_ulp(r)
-        else:
-            lim = np.full_like(r, tol)
+        lim = output_limit(r, dtype, n)
+        plain = 1e-2 if (n == "lse" and dtype == "bf16") else (1e-4 if n == "lse" else TOL[dtype])
         worst = np.unravel_index(np.argmax(err - lim), err.shape)
         report[n] = dict(max_abs=float(err.max()), max_ref=float(np.abs(r).max()),
-                         worst_excess=float((err - lim)[worst]), ok=bool(np.all(err <= lim)))
+                         worst_excess=float((err - lim)[worst]), over_plain=int(np.count_nonzero(err > plain)),
+                         ok=bool(np.all(err <= lim)))
+    print("outputs", {n: (round(v["max_abs"], 6), round(v["max_ref"], 3), v["over_plain"]) for n, v in report.items()})
     for n, rep in report.items():
         assert rep["ok"], f"{n}: error exceeds tolerance by {rep['worst_excess']:.3g}; all: {report}"
     return report

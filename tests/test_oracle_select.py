@@ -133,3 +133,113 @@ def test_rejects_topk_above_coarsest_level_size():
     q = np.zeros((1, 1, 1, 4), dtype=np.float32)
     with pytest.raises(ValueError):
         select([q], [q], 2)
+
+
+# ----------------------------------------------------------------------------- fp32 error floor
+# The selection kernels rank fp32 dot products of the fp32 pyramid rows, so two keys whose
+# fp64 scores differ by less than the rounding error of those dot products may come out in
+# either order.  The checker therefore accepts an inverted pair when its fp64 gap is below
+# the sum of the two scores' fp32 error bounds.  These pins tie that bound to real fp32
+# arithmetic (it must cover what an fp32 summation actually does) and keep it from being
+# loose (a swap well beyond it must fail), with each pair judged on its own bound.
+
+D64 = 64
+BIG = np.float32(2.0 ** 24)
+
+
+def _cancelling_key(small):
+    """[2^24, small x 62, -2^24]: the fp64 dot with a ones query is 62 * small, while an fp32
+    running sum starting at 2^24 rounds every small term (below one ulp) away."""
+    k = np.full(D64, np.float32(small), dtype=np.float32)
+    k[0], k[-1] = BIG, -BIG
+    return k
+
+
+def _fp32_sequential_dot(q, k):
+    acc = np.float32(0.0)
+    for a, b in zip(q.astype(np.float32), k.astype(np.float32)):
+        acc = np.float32(acc + np.float32(a * b))
+    return float(acc)
+
+
+def _rows(keys):
+    k = np.stack(keys).astype(np.float32)[None, None]          # [1, 1, n, D]
+    q = np.ones_like(k)                                          # every query row is all ones
+    return q, k
+
+
+def test_floor_accepts_an_inversion_that_fp32_summation_makes():
+    x = _cancelling_key(1.0)                  # fp64 score 62/8 = 7.75; fp32 running sum 0
+    y = np.zeros(D64, np.float32)
+    y[0] = 0.5                                # score 0.0625 in both precisions
+    bad1 = np.full(D64, -1.0, np.float32)
+    bad2 = np.full(D64, -2.0, np.float32)
+    q, k = _rows([x, y, bad1, bad2])
+    fp32 = [_fp32_sequential_dot(q[0, 0, 0], k[0, 0, j]) for j in range(4)]
+    assert fp32[0] == 0.0 and fp32[1] == 0.5          # fp32 ranks y above x
+    gpu_like = np.full((1, 1, 4, 1), int(np.argmax(fp32)), dtype=np.int32)
+    assert gpu_like[0, 0, 0, 0] == 1
+    (want,) = select([q], [k], 1)
+    assert want[0, 0, 0, 0] == 0                       # fp64 ranks x first
+    res = check_selection([q], [k], [gpu_like], 1)
+    # the gap (61.5 / 8) is far outside 1e-5 relative, inside the fp32 bound of x (about 16)
+    assert res["bad"] == 0 and res["floor_used"] == 4, res
+
+
+def test_floor_rejects_a_swap_beyond_the_pair_bound():
+    w = _cancelling_key(3.0)                  # fp64 score 186 / 8 = 23.25, bound about 16.0
+    y = np.zeros(D64, np.float32)
+    y[0] = 0.5
+    q, k = _rows([w, y, np.full(D64, -1.0, np.float32), np.full(D64, -2.0, np.float32)])
+    planted = np.full((1, 1, 4, 1), 1, dtype=np.int32)   # y kept, w rejected: gap 23.19
+    assert check_selection([q], [k], [planted], 1)["bad"] == 4
+
+
+def test_floor_is_judged_per_pair_not_per_row():
+    # Key z has a huge sum |q_d k_d| (so a huge fp32 bound) and the lowest score; the planted
+    # swap is between a and b, whose own bounds are tiny.  A row-wide bound would hide it.
+    a = np.zeros(D64, np.float32)
+    a[0] = 1.0
+    b = np.zeros(D64, np.float32)
+    b[0] = 0.999
+    z = np.zeros(D64, np.float32)
+    z[0], z[1], z[2] = 2.0 ** 30, -(2.0 ** 30), -1.0
+    q, k = _rows([a, b, z, np.full(D64, -3.0, np.float32)])
+    planted = np.full((1, 1, 4, 1), 1, dtype=np.int32)   # b instead of a: gap 1.25e-4
+    assert check_selection([q], [k], [planted], 1)["bad"] == 4
+    honest = np.full((1, 1, 4, 1), 0, dtype=np.int32)
+    assert check_selection([q], [k], [honest], 1)["exact"] == 4
+
+
+def test_floor_covers_fp32_summation_orders_and_is_not_loose():
+    # Cancellation-heavy rows: the realised fp32 error of several summation orders (running
+    # sum, reversed, pairwise tree, fused multiply-add chain emulated exactly) never exceeds
+    # the bound, and the worst case is not far below it (a bound 8x too large, as with a
+    # dropped 1/sqrt(D), would put every ratio under 0.015).
+    from oracle.llsa_oracle import dot_error_floor
+    rng = np.random.default_rng(2024)
+    worst = 0.0
+    for trial in range(300):
+        big = np.float32(2.0 ** rng.integers(8, 30))
+        k = (rng.standard_normal(D64) * rng.choice([1e-3, 1.0, 50.0])).astype(np.float32)
+        k[rng.integers(0, D64)] += big
+        k[rng.integers(0, D64)] -= big
+        q = rng.choice([1.0, -1.0], D64).astype(np.float32) * np.float32(rng.uniform(0.5, 2.0))
+        exact = float(q.astype(np.float64) @ k.astype(np.float64)) / 8.0
+        bound = float(dot_error_floor(q[None], k[None])[0, 0])
+        prods = (q * k).astype(np.float32)                      # each product rounded once
+        orders = [prods, prods[::-1]]
+        sums = [float(np.float32(np.cumsum(o, dtype=np.float32)[-1])) for o in orders]
+        tree = prods.copy()
+        while tree.size > 1:
+            tree = (tree[0::2] + tree[1::2]).astype(np.float32)
+        sums.append(float(tree[0]))
+        acc = np.float64(0.0)                                   # fma: product exact, one rounding
+        for a, b in zip(q.astype(np.float64), k.astype(np.float64)):
+            acc = np.float64(np.float32(acc + a * b))
+        sums.append(float(acc))
+        for s in sums:
+            err = abs(s / 8.0 - exact)
+            assert err <= bound, (trial, err, bound)
+            worst = max(worst, err / bound)
+    assert worst > 0.05, worst
