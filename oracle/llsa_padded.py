@@ -11,11 +11,13 @@ result.  This module fixes what that means (parity unpinned against the pages, w
 nothing about it; pinned below by closed forms):
 
 * Pooling: level-l token j averages only the real tokens of its span; its count c_{l,j} is
-  the number of them, and a token with c = 0 is empty.  Sums are carried in fp32: level 1
-  adds the c real tokens in index order, level l >= 2 adds its 16 children's sums in index
-  order, and the mean is sum / c.  For a sequence without padding every count is 16^l and
-  the result is bit-identical to ``llsa_oracle.build_pyramid`` (scaling by a power of two
-  commutes with rounding).
+  the number of them, and a token with c = 0 is empty (its value is 0).  Each level is made
+  from the stored level below, in fp32: level 1 adds the c real tokens in index order and
+  divides by c; level l >= 2 adds, in index order, each child's count times its stored mean
+  (c_{l-1} * mean, rounded), then divides by c_{l,j}.  So a level is always a function of the
+  level below, as in the unpadded pyramid.  For a full token the products are exact (powers
+  of two), and a sequence without padding gives results bit-identical to
+  ``llsa_oracle.build_pyramid`` (scaling by a power of two commutes with rounding).
 * Selection: empty tokens are never candidates.  The real tokens of every level form a
   prefix [0, m_l) with m_l = ceil(n_valid / 16^l); K <= m_L keeps every list full (each
   picked parent has a real child).  Queries of empty tokens select from their zero mean.
@@ -52,16 +54,20 @@ def build_pyramid_padded(x: np.ndarray, levels: int, n_valid: int) -> list[np.nd
     real = np.asarray(x, dtype=np.float32).copy()
     real[:, :, n_valid:] = 0.0  # padding contributes nothing to the sums
     out = []
-    prev_sum = real
+    prev = real                                          # level 0: the tokens, count 1 or 0
+    prev_count = np.ones(N, dtype=np.float32)
     for lev in range(levels):
-        groups = prev_sum.reshape(B, H, -1, BLOCK, D)
+        groups = prev.reshape(B, H, -1, BLOCK, D)
+        cnt = prev_count.reshape(-1, BLOCK)
         s = np.zeros(groups.shape[:3] + (D,), dtype=np.float32)
         for r in range(BLOCK):
-            s = s + groups[:, :, :, r, :]
+            term = groups[:, :, :, r, :] if lev == 0 else (cnt[None, None, :, r, None] * groups[:, :, :, r, :])
+            s = s + term.astype(np.float32)
         c = counts[lev].astype(np.float32)[None, None, :, None]
         mean = np.where(c > 0, s / np.where(c > 0, c, np.float32(1.0)), np.float32(0.0)).astype(np.float32)
         out.append(mean)
-        prev_sum = s
+        prev = mean
+        prev_count = counts[lev].astype(np.float32)
     return out
 
 
