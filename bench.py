@@ -3,7 +3,8 @@
 
 One step = the whole hot path on one batch of device-resident synthetic input:
 pyramid -> hierarchical selection -> attention forward -> index transpose -> attention
-backward (five C-ABI calls, 12 kernel launches at the default workload).
+backward (the five C-ABI calls as one llsa_train_step; 15 kernel launches at the default
+workload, counted live in `gpu_launches`).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload headline-65536]
 
@@ -182,6 +183,8 @@ def workload_counts(cfg, pairs_l1: int, all_top: bool = False, select_launches: 
     # level-2 selection runs inside the level-1 launch)
     nsel = select_launches or L
     counts["select"] = dict(bytes=sel_bytes // nsel, flops=sel_flops // nsel)
+    # the pyramid and every selection level in one launch (bf16, small coarsest level)
+    counts["pyramid_select"] = dict(bytes=counts["pyramid_l12"]["bytes"] + sel_bytes, flops=sel_flops)
     # transpose: E entries over all levels; hist reads idx, scatter reads idx and writes the
     # bucketed entries, bucket reads them and writes col and row_ptr
     entries = sum(bh * n[lev] * K for lev in range(1, L + 1))
@@ -189,6 +192,13 @@ def workload_counts(cfg, pairs_l1: int, all_top: bool = False, select_launches: 
     counts["transpose_hist"] = dict(bytes=entries * 4, flops=0)
     counts["transpose_scatter"] = dict(bytes=2 * entries * 4, flops=0)
     counts["transpose_bucket"] = dict(bytes=2 * entries * 4 + rows * 4, flops=0)
+    hist = 0   # the scan reads and rewrites every (bucket, tile) count of every problem
+    for lev in range(1, L + 1):
+        width = 1
+        while -(-n[lev] // width) > 64:
+            width *= 2
+        hist += bh * (-(-n[lev] // width) * -(-(n[lev] * K) // 4096) + 1)
+    counts["transpose_scan"] = dict(bytes=2 * hist * 4, flops=0)
     counts["dkdv_order_count"] = dict(bytes=bh * (n1 + 1) * 4, flops=0)
     counts["dkdv_order_scatter"] = dict(bytes=bh * (n1 + 1) * 4 + bh * n1 * 16, flops=0)
     if L >= 2:
@@ -211,6 +221,47 @@ def coarse_entries(cfg, all_top: bool = False) -> int:
     return (L - 2) * K + cfg.level_sizes()[L] if all_top else (L - 1) * K
 
 
+def compulsory_bytes(cfg, elem: int) -> int:
+    """DRAM bytes no implementation of the step can avoid: q, k, v, dO read once; o, dq, dk,
+    dv and LSE written once; the pyramids, the selection and its CSR written once."""
+    bh = cfg.B * cfg.H
+    n = cfg.level_sizes()
+    L, K, D = cfg.levels, cfg.topk, cfg.D
+    act = 8 * bh * cfg.N * D * elem
+    lse = bh * cfg.N * 4
+    pyr = 3 * sum(bh * n[lev] * D * 4 for lev in range(1, L + 1))
+    sel = 2 * sum(bh * n[lev] * K * 4 for lev in range(1, L + 1)) + sum(bh * (n[lev] + 1) * 4 for lev in range(1, L + 1))
+    return act + lse + pyr + sel
+
+
+def measure_gather_peak(api, torch, stream, sms: int) -> dict:
+    """L2 -> SM gather ceiling: llsa_gather_probe (the attention kernels' 16 x 64 bf16 TMA tile
+    gather and nothing else) over random tiles of a 32 MiB buffer that stays in L2; the best
+    bytes per second over ring depths and CTAs per SM."""
+    rows = 1 << 18
+    gen = torch.Generator().manual_seed(11)
+    src = torch.randn(rows, 64, generator=gen).to(torch.bfloat16).cuda()
+    ntiles = 1 << 19
+    tile_rows = (torch.randint(0, rows // 16, (ntiles,), generator=gen) * 16).to(torch.int32).cuda()
+    best = {"gbs": 0.0}
+    for stages in (2, 4, 8):
+        for per_sm in (2, 4, 8):
+            ctas = sms * per_sm
+            api.llsa_gather_probe(src, tile_rows, stages, ctas, stream)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 3
+            e0.record(stream)
+            for _ in range(reps):
+                api.llsa_gather_probe(src, tile_rows, stages, ctas, stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            gbs = reps * ntiles * 2048 / (e0.elapsed_time(e1) * 1e-3) / 1e9
+            if gbs > best["gbs"]:
+                best = {"gbs": round(gbs, 1), "stages": stages, "ctas": ctas}
+    best.update(buffer_mib=rows * 128 >> 20, tile_bytes=2048, tiles_per_launch=ntiles)
+    return best
+
+
 def enrichment(args) -> dict:
     """Keyword arguments of the enrichment variants chosen on the command line."""
     return dict(log_bias=args.log_bias, all_top=args.all_top, level1=args.level1)
@@ -225,47 +276,131 @@ def enrichment_text(args) -> str:
     return "; ".join(parts)
 
 
-# ----------------------------------------------------------------------------- oracle sample
+# ----------------------------------------------------------------------------- oracle on host cores
+# The CPU baseline and the reference arm run the oracle, as it stands, on every host core: a
+# pool of worker processes (spawn start method) over (head, query-block chunk).  Inputs live
+# in shared memory (fp32, the exact values of the device inputs); each task writes its query
+# blocks' O, LSE and dQ rows in place and adds its dK/dV contribution to its head's shared
+# fp64 accumulator under that head's lock.  A step is: per head, pyramid + selection + index
+# transpose; then per (head, chunk), forward + backward of the chunk's query blocks.
 
-def oracle_sample(cfg, inputs, heads: int, nblocks: int | None, log_bias: bool = False, all_top: bool = False,
-                  level1: bool = False):
-    """Time the CPU oracle on ``heads`` (b=0) heads of the workload: pyramid, selection and
-    transpose for each whole head, forward and backward for ``nblocks`` query blocks per
-    head (all blocks if None).  Returns (tokens/s extrapolated to the full workload, dict)."""
+_ORC = {}
+
+
+def _orc_attach(names, shape, flags, levels, topk, locks):
+    """Worker initializer: map the shared inputs and outputs, one BLAS thread per process."""
     import numpy as np
+    from multiprocessing import shared_memory
     from threadpoolctl import threadpool_limits
 
-    from oracle import llsa_oracle as orc
-    from synthetic import to_f32_numpy, to_f64_numpy
+    threadpool_limits(1)
+    _ORC["shm"] = {k: shared_memory.SharedMemory(name=v) for k, v in names.items()}
+    B, H, N, D = shape
+    for k, m in _ORC["shm"].items():
+        if k in ("q", "k", "v", "do"):
+            _ORC[k] = np.ndarray((B, H, N, D), dtype=np.float32, buffer=m.buf)
+        elif k == "lse":
+            _ORC[k] = np.ndarray((B, H, N), dtype=np.float64, buffer=m.buf)
+        else:
+            _ORC[k] = np.ndarray((B, H, N, D), dtype=np.float64, buffer=m.buf)
+    _ORC.update(flags=flags, levels=levels, topk=topk, locks=locks)
 
-    n1 = cfg.N // 16
-    blocks = None if nblocks is None or nblocks >= n1 else np.linspace(0, n1 - 1, nblocks).astype(np.int64)
-    nb = n1 if blocks is None else len(blocks)
-    t_fixed = t_attn = 0.0
-    with threadpool_limits(1):
-        for h in range(heads):
-            sl = (slice(0, 1), slice(h, h + 1))
-            q32, k32, v32 = (to_f32_numpy(inputs[x][sl]) for x in ("q", "k", "v"))
-            q, k, v, do = (to_f64_numpy(inputs[x][sl]) for x in ("q", "k", "v", "do"))
-            t0 = time.perf_counter()
-            qp, kp, vp = (orc.build_pyramid(a, cfg.levels) for a in (q32, k32, v32))
-            idx = orc.select(qp, kp, cfg.topk)
-            orc.index_transpose_all(idx)
-            t1 = time.perf_counter()
-            o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top,
-                                 level1=level1)
-            if cfg.backward:
-                orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks, log_bias=log_bias, all_top=all_top,
-                             level1=level1)
-            t2 = time.perf_counter()
-            t_fixed += t1 - t0
-            t_attn += t2 - t1
-    # per head: fixed part + attention scaled from nb sampled blocks to all n1 blocks
-    per_head = (t_fixed + t_attn * (n1 / nb)) / heads
-    full_step = per_head * cfg.B * cfg.H
-    info = {"heads": heads, "blocks_per_head": nb, "seconds": t_fixed + t_attn, "t_full_step_est_s": full_step,
-            "t_fixed_per_head": t_fixed / heads, "t_attn_per_block": t_attn / (heads * nb)}
-    return cfg.B * cfg.N / full_step, info
+
+def _orc_head(bh):
+    """Pyramid, selection and index transpose of one head; returns what the chunks need."""
+    from oracle import llsa_oracle as orc
+    b, h = bh
+    sl = (slice(b, b + 1), slice(h, h + 1))
+    qp, kp, vp = (orc.build_pyramid(_ORC[x][sl], _ORC["levels"]) for x in ("q", "k", "v"))
+    idx = orc.select(qp, kp, _ORC["topk"])
+    orc.index_transpose_all(idx)
+    return kp, vp, idx
+
+
+def _orc_chunk(task):
+    """Forward and backward of one chunk of query blocks of one head."""
+    import numpy as np
+    from oracle import llsa_oracle as orc
+    (b, h), blocks, kp, vp, idx, head_no, backward = task
+    sl = (slice(b, b + 1), slice(h, h + 1))
+    q, k, v = (_ORC[x][sl].astype(np.float64) for x in ("q", "k", "v"))
+    o, lse = orc.forward(q, k, v, kp, vp, idx, blocks=blocks, **_ORC["flags"])
+    rows = (blocks[:, None] * 16 + np.arange(16)).ravel()
+    _ORC["o"][b, h, rows] = o[0, 0, rows]
+    _ORC["lse"][b, h, rows] = lse[0, 0, rows]
+    if backward:
+        do = _ORC["do"][sl].astype(np.float64)
+        dq, dk, dv = orc.backward(q, k, v, o, lse, do, kp, vp, idx, blocks=blocks, **_ORC["flags"])
+        _ORC["dq"][b, h, rows] = dq[0, 0, rows]
+        with _ORC["locks"][head_no]:
+            _ORC["dk"][b, h] += dk[0, 0]
+            _ORC["dv"][b, h] += dv[0, 0]
+    return len(blocks)
+
+
+def host_cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class OraclePool:
+    """The oracle on ``cores`` worker processes over one workload's seeded inputs."""
+
+    def __init__(self, cfg, host_inputs, flags: dict, cores: int | None = None):
+        import multiprocessing as mp
+        import numpy as np
+        from multiprocessing import shared_memory
+
+        self.cfg = cfg
+        self.cores = cores or len(os.sched_getaffinity(0))
+        B, H, N, D = cfg.B, cfg.H, cfg.N, cfg.D
+        sizes = {"q": 4, "k": 4, "v": 4, "do": 4, "o": 8, "dq": 8, "dk": 8, "dv": 8}
+        self.shm = {k: shared_memory.SharedMemory(create=True, size=B * H * N * D * w) for k, w in sizes.items()}
+        self.shm["lse"] = shared_memory.SharedMemory(create=True, size=B * H * N * 8)
+        for k in ("q", "k", "v", "do"):
+            np.ndarray((B, H, N, D), dtype=np.float32, buffer=self.shm[k].buf)[...] = \
+                host_inputs[k].float().numpy()
+        self.dk = np.ndarray((B, H, N, D), dtype=np.float64, buffer=self.shm["dk"].buf)
+        self.dv = np.ndarray((B, H, N, D), dtype=np.float64, buffer=self.shm["dv"].buf)
+        ctx = mp.get_context("spawn")
+        locks = [ctx.Lock() for _ in range(B * H)]
+        self.pool = ctx.Pool(self.cores, initializer=_orc_attach,
+                             initargs=({k: m.name for k, m in self.shm.items()}, (B, H, N, D), flags, cfg.levels,
+                                       cfg.topk, locks))
+
+    def step(self, heads=None, backward=None) -> float:
+        """One oracle step over ``heads`` ((b, h) pairs; all by default); returns seconds."""
+        import numpy as np
+        cfg = self.cfg
+        heads = heads or [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
+        backward = cfg.backward if backward is None else backward
+        n1 = cfg.N // 16
+        chunks = max(1, min(n1, (2 * self.cores + len(heads) - 1) // len(heads)))
+        t0 = time.perf_counter()
+        for b, h in heads:
+            self.dk[b, h] = 0.0
+            self.dv[b, h] = 0.0
+        per_head = self.pool.map(_orc_head, heads)
+        tasks = []
+        for no, (bh, (kp, vp, idx)) in enumerate(zip(heads, per_head)):
+            for blocks in np.array_split(np.arange(n1), chunks):
+                if blocks.size:
+                    tasks.append((bh, blocks, kp, vp, idx, bh[0] * cfg.H + bh[1], backward))
+        done = sum(self.pool.map(_orc_chunk, tasks, chunksize=1))
+        assert done == n1 * len(heads)
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+        for m in self.shm.values():
+            m.close()
+            m.unlink()
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -385,6 +520,7 @@ def run_ours(args):
                     "algorithmic_bytes_per_launch": c["bytes"],
                     "tensor_achieved_tflops": round(c["flops"] / sec / 1e12, 2),
                     "tensor_frac_of_sustained_bf16": round(c["flops"] / sec / 1e12 / tensor_peak, 4)}
+    step_compulsory = compulsory_bytes(cfg, 2 if cfg.dtype == "bf16" else 4)
     kernels_roof = {}
     for k, c in counts.items():
         if k in kern:
@@ -395,7 +531,7 @@ def run_ours(args):
     # whole-step roofline as the workload defines it: the slower of the selected attention's
     # FLOPs at the bf16 tensor peak and its modelled bytes (gathers and pyramid) at the HBM
     # peak; the other kernels have their own fractions in `kernels`
-    step_kernels = ("attn_fwd_bf16", "attn_bwd_dq_bf16", "attn_bwd_dkdv_bf16", "pyramid_l12")
+    step_kernels = ("attn_fwd_bf16", "attn_bwd_dq_bf16", "attn_bwd_dkdv_bf16", "pyramid_l12", "pyramid_select")
     step_bytes = sum(c["bytes"] for k, c in counts.items() if k in kern and k in step_kernels)
     step_flops = sum(c["flops"] for k, c in counts.items() if k in kern and k in step_kernels)
     step_roof_ms = 1000 * max(step_bytes / (hbm_peak * 1e9), step_flops / (tensor_peak * 1e12))
@@ -421,6 +557,7 @@ def run_ours(args):
         computed[si].record(stream)
         drained[si].record(stream)
     in_bytes = sum(t.numel() * t.element_size() for t in pinned.values())
+    in_mb = in_bytes / 1e6
     out_bytes = sum(t.numel() * t.element_size() for t in host_out[0].values())
     dist_barrier(world)
     torch.cuda.synchronize()
@@ -476,6 +613,47 @@ def run_ours(args):
                  "gbs": round(zbytes / (zus * 1e-6) / 1e9, 1), "hbm_frac": round(zbytes / (zus * 1e-6) / 1e9 / hbm_peak, 4)}
         del zdst
 
+    # forward only (pyramid, selection, forward: the inference path) and the standalone index
+    # transpose, each timed eagerly on the launching stream after warm-up
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b2.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b2) / reps
+
+    fwd_ms = timed(lambda: api.llsa_forward_path(shape, dev["q"], dev["k"], dev["v"], buf), 20)
+    forward_only = {"ms_per_step": round(fwd_ms, 4), "tokens_per_s": round(tokens_per_step / (fwd_ms / 1000.0), 1),
+                    "calls": "llsa_build_pyramid + llsa_select + llsa_forward, eager on one stream"}
+    tr_ms = timed(lambda: api.llsa_index_transpose(shape, buf.idx, buf.row_ptr, buf.col, buf.ws_transpose), 50)
+    entries = sum(cfg.B * cfg.H * n * cfg.topk for n in cfg.level_sizes()[1:])
+    tr_bytes = counts["transpose_hist"]["bytes"] + counts["transpose_scatter"]["bytes"] + \
+        counts["transpose_bucket"]["bytes"] + counts.get("transpose_scan", {"bytes": 0})["bytes"]
+    transpose = {"avg_us": round(1000 * tr_ms, 2), "entries": entries,
+                 "entries_per_s": round(entries / (tr_ms / 1000.0), 1),
+                 "gbs": round(tr_bytes / (tr_ms / 1000.0) / 1e9, 1),
+                 "calls": "llsa_index_transpose (all levels, 4 launches), eager"}
+    gather = measure_gather_peak(api, torch, stream, props.multi_processor_count)
+    if roofline:
+        c = counts[dominant]
+        sec = kern[dominant]["avg_us"] * 1e-6
+        roofline["l2_gather_peak_gbs"] = gather["gbs"]
+        roofline["l2_frac"] = round(c["bytes"] / sec / 1e9 / gather["gbs"], 4)
+        roofline["compulsory_frac"] = round(step_compulsory / (hbm_peak * 1e9) / (ms_per_step * 1e-3), 4)
+        roofline["note"] = ("frac charges every gathered tile at HBM speed, but L2 serves most gathers, so "
+                            "frac > 1 means the model overstates the HBM bytes; l2_frac is the same bytes "
+                            "against the measured L2 -> SM tile-gather ceiling; compulsory_frac is the whole "
+                            "step's unavoidable DRAM bytes at the HBM peak over the measured step time")
+    for k, v in kernels_roof.items():
+        if k.startswith("attn_"):
+            c = counts[k]
+            v["l2_frac"] = round(c["bytes"] / (kern[k]["avg_us"] * 1e-6) / 1e9 / gather["gbs"], 4)
+
     # dense attention at the same shape (torch SDPA, flash backend), forward + backward
     dense = None
     if world == 1:
@@ -500,10 +678,17 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, info = oracle_sample(cfg, host, heads=2, nblocks=None, **enrichment(args))
-        cpu = {"value": round(val, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": (f"numpy fp64 oracle, 1 thread: pyramid, selection, transpose, forward and backward of "
-                          f"heads (b=0, h=0..1), {info['seconds']:.1f} s, extrapolated to {cfg.B * cfg.H} heads")}
+        pool = OraclePool(cfg, host, enrichment(args))
+        try:
+            pool.step(heads=[(0, 0)])          # workers import the oracle and page in
+            secs = pool.step(backward=True)    # the whole step the CUDA arm times
+        finally:
+            pool.close()
+        cpu = {"value": round(tokens_per_step / secs, 2), "unit": UNIT, "cores": pool.cores, "kind": "oracle",
+               "cpu_model": host_cpu_model(), "seconds": round(secs, 3),
+               "sample": (f"the whole step of the workload (all {cfg.B * cfg.H} heads: pyramid, selection, "
+                          f"index transpose, forward and backward), numpy fp64 oracle on {pool.cores} worker "
+                          "processes (one thread each) over (head, query-block chunk)")}
 
     clocks = sampler.summary() if sampler else None
     result = {
@@ -529,10 +714,19 @@ def run_ours(args):
                    "kernel_times_from": ("a second plan of the same K steps with trace events around every "
                                          f"kernel, launched after the timed one: {traced_ms_per_step:.4f} ms per step"),
                    "parallelism": f"dp{world}: independent replicas, no collective",
-                   "l2": "inputs larger than L2: q, k, v, dO are 201 MB per replica vs 126 MB L2; no flush"},
+                   "l2": (f"inputs larger than L2: q, k, v, dO are {in_mb:.0f} MB per replica vs 126 MB L2; "
+                          "no flush")},
         "roofline": roofline,
         "step_roofline": {"modelled_bytes": step_bytes, "flops": step_flops, "roofline_ms": round(step_roof_ms, 4),
                           "frac": round(step_roof_ms / ms_per_step, 4)},
+        "compulsory": {"bytes": step_compulsory,
+                       "floor_ms": round(1000 * step_compulsory / (hbm_peak * 1e9), 4),
+                       "frac": round(1000 * step_compulsory / (hbm_peak * 1e9) / ms_per_step, 4),
+                       "what": ("q, k, v, dO read once; o, dq, dk, dv, LSE, pyramids, selection and CSR "
+                                "written once, at the measured HBM peak")},
+        "l2_gather_peak": gather,
+        "forward_only": forward_only,
+        "index_transpose": transpose,
         "kernels": kernels_roof,
         "kernel_times": {k: {"launches": v["launches"], "avg_us": round(v["avg_us"], 2), "share": round(v["share"], 4)}
                          for k, v in sorted(kern.items(), key=lambda kv: -kv[1]["total_ms"])},
@@ -581,7 +775,10 @@ def source_hash() -> str:
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
-    """The CPU oracle as the reference arm: rank 0 only, each step a bounded sample."""
+    """The CPU oracle as the reference arm, on every host core: rank 0 only.  Each step is the
+    oracle's whole step over a sample of the workload's heads (all of them when that fits in
+    about two and a half minutes for warm-up plus steps); the value is the sample's tokens
+    (its share of B*N) per second of the sample's measured time, with nothing extrapolated."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
@@ -589,25 +786,28 @@ def run_reference(args):
 
     cfg = WORKLOADS[args.workload]
     host = make_config_inputs(cfg, with_do=True)
-    n1 = cfg.N // 16
-    # size each step's sample so that warm-up + steps stay near two minutes
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    _, probe = oracle_sample(cfg, host, heads=1, nblocks=16, **enrichment(args))
-    per_block = max(1e-6, probe["t_attn_per_block"])
-    nblocks = int(max(16, min(n1, (budget - probe["t_fixed_per_head"]) / per_block)))
-    for _ in range(args.warmup):
-        oracle_sample(cfg, host, heads=1, nblocks=nblocks, **enrichment(args))
-    vals, secs = [], 0.0
-    for _ in range(args.steps):
-        v, info = oracle_sample(cfg, host, heads=1, nblocks=nblocks, **enrichment(args))
-        vals.append(v)
-        secs += info["seconds"]
-    value = statistics.median(vals)
-    tokens_per_step = cfg.B * cfg.N
-    ms_per_step = 1000.0 * tokens_per_step / value
-    sample = (f"numpy fp64 oracle, 1 thread, per step: pyramid, selection and transpose of head (b=0, h=0) and "
-              f"forward+backward of {nblocks} of its {n1} query blocks, extrapolated to all blocks and "
-              f"{cfg.B * cfg.H} heads; median over {args.steps} steps")
+    pool = OraclePool(cfg, host, enrichment(args))
+    heads_all = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
+    try:
+        t_head = pool.step(heads=heads_all[:1], backward=True)
+        per_step = len(heads_all)
+        while per_step > 1 and (args.steps + args.warmup) * t_head * per_step > 150.0:
+            per_step -= 1
+        secs = []
+        for i in range(args.warmup + args.steps):
+            heads = [heads_all[(i * per_step + j) % len(heads_all)] for j in range(per_step)]
+            t = pool.step(heads=heads, backward=True)
+            if i >= args.warmup:
+                secs.append(t)
+    finally:
+        pool.close()
+    total_s = sum(secs)
+    tokens_per_step = cfg.B * cfg.N * per_step / len(heads_all)
+    value = tokens_per_step * args.steps / total_s
+    ms_per_step = 1000.0 * total_s / args.steps
+    sample = (f"numpy fp64 oracle on {pool.cores} worker processes ({host_cpu_model()}), per step the whole "
+              f"step (pyramid, selection, index transpose, forward, backward) of {per_step} of the "
+              f"{len(heads_all)} heads; value = those heads' share of the step's tokens per measured second")
     result = {
         "impl": "reference",
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -616,8 +816,10 @@ def run_reference(args):
         "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
                    "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk,
                    "kv_len": 16 * cfg.topk + (cfg.topk if args.level1 else 0) + coarse_entries(cfg, args.all_top),
-                   "enrichment": enrichment_text(args)},
-        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+                   "enrichment": enrichment_text(args), "heads_per_step": per_step,
+                   "tokens_per_step": tokens_per_step},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": pool.cores, "kind": "oracle",
+                         "cpu_model": host_cpu_model(), "sample": sample},
         "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(result), flush=True)

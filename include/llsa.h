@@ -43,8 +43,9 @@
  *    shape rules below) or LLSA_ERR_UNSUPPORTED (a legal value this build does not
  *    implement).  A launch failure returns LLSA_ERR_CUDA.  No exception crosses the ABI.
  *  - Shape rules: B, H >= 1; N a multiple of 16^L (so every n_l = N / 16^l is whole
- *    and n_L >= 1; N need not be a power of two); 1 <= topk <= n_L, any integer;
- *    block == 16; 1 <= levels <= 4; D == 64; N <= 2^20; n_L <= 16384; topk <= 64; (levels - 1) * topk <= 32;
+ *    and n_L >= 1; N need not be a power of two; a shorter sequence is padded up to such an N
+ *    and n_valid says where its padding starts); 1 <= topk <= n_L, any integer;
+ *    block == 16; 1 <= levels <= 4; D == 64 or 128; N <= 2^20; n_L <= 16384; topk <= 64; (levels - 1) * topk <= 32;
  *    B * H * N < 2^31; with LLSA_FLAG_ALL_TOP also (levels - 2) * topk + n_L <= 96.
  *  - Device-side checks: every gathered index (idx entries, CSR entries) is range
  *    checked on the device; an out-of-range value is not dereferenced, and the call
@@ -108,7 +109,26 @@ typedef struct {
   int32_t levels;  /* L, number of pooled levels; llsa_l1 <-> 1, llsa_l2 <-> 2 */
   int32_t dtype;   /* llsa_dtype of q, k, v, o, dO, dq, dk, dv */
   int32_t flags;   /* LLSA_FLAG_* bits (0: the default enrichment); others -> INVALID_ARG */
+  int32_t n_valid; /* real tokens per sequence: 0 (or N) = no padding; see "Padded sequences" */
 } llsa_shape;
+
+/*
+ * Padded sequences (no counterpart on the pages, whose kernels need the token length to be a
+ * power of two; the README's usage section says a later update will lift that).  With
+ * 0 < n_valid < N, positions n_valid..N-1 of every (b, h) sequence are padding and take no
+ * part in the result, whatever they hold:
+ *  - a pooled token averages only the real tokens of its span (c of them, 0 <= c <= 16^l):
+ *    level 1 adds its real tokens in index order and divides by c; level l >= 2 adds each
+ *    child's count times its stored mean in index order and divides by c; a token with c = 0
+ *    is 0.  Full tokens come out exactly as without padding;
+ *  - empty tokens are never selected: the candidates of level l are the real tokens
+ *    [0, ceil(n_valid / 16^l)); topk must not exceed ceil(n_valid / 16^L);
+ *  - padding keys are masked out of every softmax; padding queries get O = 0, LSE = 0 and
+ *    dQ = 0 and send no gradient; padding positions get dK = dV = 0;
+ *  - a pooled token's gradient reaches each of its c real tokens with weight 1 / c.
+ * Selection rows of padding query tokens are still written (scores of a zero mean).
+ * Padding combines with no enrichment flag (flags != 0 -> LLSA_ERR_UNSUPPORTED).
+ */
 
 /* Static text for a status code. */
 const char* llsa_status_string(llsa_status status);
@@ -151,7 +171,7 @@ llsa_status llsa_select(const llsa_shape* shape, const float* q_pyr, const float
  * works on the sparse indices and builds no dense mask).  For every level, batch and head
  * it turns the query -> key lists `idx` into key -> query CSR lists (row_ptr, col),
  * queries ascending within each row.  It is a stable counting sort by key bucket then by
- * key (histogram + scan + scatter), with no atomics, so the output is deterministic.
+ * key (histogram, scan, scatter), with no atomics, so the output is deterministic.
  * workspace: device scratch of at least llsa_transpose_workspace_bytes(shape) bytes,
  * 256-byte aligned; its contents are not read before being written.
  */
@@ -259,6 +279,36 @@ llsa_status llsa_token_permute(const llsa_shape* shape, const void* src, void* d
  * call.  Returns LLSA_ERR_CUDA if the device cannot be queried.
  */
 llsa_status llsa_device_status(int32_t* code_out, llsa_stream_t stream);
+
+/*
+ * Check of the bounded-wait failure path (no counterpart on the pages: a failure-detection
+ * aid of this library).  Every wait of the kernels on an asynchronous copy gives up after a
+ * cycle limit (about two seconds at the maximum SM clock), records LLSA_ERR_TIMEOUT in the
+ * device status word and lets the kernel return, so a copy that never lands cannot hang the
+ * GPU.  This call runs that same wait in a one-thread kernel on an mbarrier armed for 16
+ * bytes that no copy will ever deliver (none is issued, so nothing is left in flight), with
+ * a limit of `limit_cycles` SM cycles: the wait gives up, and the next llsa_device_status
+ * returns LLSA_ERR_TIMEOUT.  limit_cycles outside [1, 4e9] -> LLSA_ERR_INVALID_ARG.
+ * While the recorded timeout has not been read and cleared, the waits of other kernels give
+ * up at their next check, so call it only when no other work of the library is in flight.
+ */
+llsa_status llsa_check_bounded_wait(int64_t limit_cycles, llsa_stream_t stream);
+
+/*
+ * L2 -> SM gather probe (a measurement aid; no counterpart on the pages).  The attention
+ * kernels gather 16-row x 64-channel bf16 tiles by index with 2-D TMA copies (128-byte
+ * swizzle); when the gathered K, V, Q and dO fit in L2 those copies are served from L2 and
+ * HBM bandwidth does not bound them.  This call runs only that gather: `ctas` CTAs of 4 warps,
+ * every warp streaming its share of the tiles through a ring of `stages` mbarrier stages and
+ * doing nothing else with them.  Timing it on a buffer kept resident in L2 gives the gather
+ * ceiling the attention kernels are compared with.
+ * src: [rows, 64] bf16, rows a multiple of 16 and < 2^31, 16-byte aligned; tile_rows:
+ * int32 [ntiles] first rows of the tiles (device-checked against rows; out-of-range values
+ * read row 0 and record LLSA_ERR_INTERNAL); stages in {2, 4, 8}; 1 <= ctas <= 65535.
+ * Writes nothing in global memory.
+ */
+llsa_status llsa_gather_probe(const void* src, int64_t rows, const int32_t* tile_rows, int32_t ntiles,
+                              int32_t stages, int32_t ctas, llsa_stream_t stream);
 
 /*
  * Index transpose for callers that cannot hand the library any device memory

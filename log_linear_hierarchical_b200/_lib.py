@@ -35,7 +35,7 @@ class LLSAShape(ctypes.Structure):
 
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("block", ctypes.c_int32), ("topk", ctypes.c_int32), ("levels", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32), ("n_valid", ctypes.c_int32)]
 
 
 # llsa_shape.flags: log-count score bias on the coarse KV entries (ln 16^l at level l)
@@ -78,6 +78,8 @@ SIGNATURES = {
     "llsa_plan_destroy": (None, [_P]),
     "llsa_token_permute": (_I, [_SP, _P, _P, ctypes.c_int32, _P]),
     "llsa_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _P]),
+    "llsa_check_bounded_wait": (_I, [ctypes.c_int64, _P]),
+    "llsa_gather_probe": (_I, [_P, ctypes.c_int64, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P]),
     "llsa_trace_begin": (_I, [ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]),
     "llsa_trace_end": (_I, [ctypes.POINTER(ctypes.c_int32)]),
     "llsa_kernel_name": (ctypes.c_char_p, [ctypes.c_int32]),

@@ -28,14 +28,15 @@ class LLSAError(RuntimeError):
 
 
 def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16,
-               log_bias: bool = False, all_top: bool = False, level1: bool = False) -> LLSAShape:
+               log_bias: bool = False, all_top: bool = False, level1: bool = False, n_valid: int = 0) -> LLSAShape:
     """``log_bias``: the log-count enrichment variant (LLSA_FLAG_LOG_BIAS); ``all_top``: the
     all-coarsest variant (LLSA_FLAG_ALL_TOP); ``level1``: the selected blocks' level-1 pooled
-    tokens join the list (LLSA_FLAG_LEVEL1).  Any combination may be set."""
+    tokens join the list (LLSA_FLAG_LEVEL1).  Any combination may be set.  ``n_valid``: the
+    real tokens of a padded sequence (positions from n_valid on are padding; 0 = none)."""
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     flags = ((_lib.LLSA_FLAG_LOG_BIAS if log_bias else 0) | (_lib.LLSA_FLAG_ALL_TOP if all_top else 0)
              | (_lib.LLSA_FLAG_LEVEL1 if level1 else 0))
-    return LLSAShape(B, H, N, D, block, topk, levels, code, flags)
+    return LLSAShape(B, H, N, D, block, topk, levels, code, flags, n_valid)
 
 
 def _check(fn: str, status: int) -> None:
@@ -201,6 +202,24 @@ def llsa_device_status(stream=None) -> int:
     return int(code.value)
 
 
+def llsa_check_bounded_wait(limit_cycles: int, stream=None) -> None:
+    """Runs the kernels' bounded wait on an mbarrier that nothing will complete, with a limit
+    of ``limit_cycles``; the wait gives up and the device status becomes LLSA_ERR_TIMEOUT."""
+    _check("llsa_check_bounded_wait", _lib.load().llsa_check_bounded_wait(int(limit_cycles), _stream(stream)))
+
+
+def llsa_gather_probe(src: torch.Tensor, tile_rows: torch.Tensor, stages: int = 4, ctas: int = 148 * 4,
+                      stream=None) -> None:
+    """Only the attention kernels' tile gather: 2-D TMA copies of the 16 x 64 bf16 tiles of
+    ``src`` ([rows, 64] bf16) whose first rows are ``tile_rows`` (int32)."""
+    if src.dtype != torch.bfloat16 or src.dim() != 2 or src.shape[1] != 64:
+        raise ValueError("src must be a [rows, 64] bf16 tensor")
+    if tile_rows.dtype != torch.int32:
+        raise ValueError("tile_rows must be int32")
+    _check("llsa_gather_probe", _lib.load().llsa_gather_probe(_p(src, "src"), src.shape[0], _p(tile_rows, "tile_rows"),
+                                                              tile_rows.numel(), stages, ctas, _stream(stream)))
+
+
 def llsa_kernel_name(kernel_id: int) -> str:
     return _lib.load().llsa_kernel_name(kernel_id).decode()
 
@@ -248,16 +267,18 @@ class LLSABuffers:
     idx: torch.Tensor
     row_ptr: torch.Tensor
     col: torch.Tensor
-    o: torch.Tensor
+    o: torch.Tensor | None
     lse: torch.Tensor
-    dq: torch.Tensor
-    dk: torch.Tensor
-    dv: torch.Tensor
+    dq: torch.Tensor | None
+    dk: torch.Tensor | None
+    dv: torch.Tensor | None
     ws_transpose: torch.Tensor
     ws_backward: torch.Tensor
 
     @staticmethod
-    def allocate(shape: LLSAShape, device, dtype: torch.dtype) -> "LLSABuffers":
+    def allocate(shape: LLSAShape, device, dtype: torch.dtype, with_grads: bool = True) -> "LLSABuffers":
+        """Every buffer of one step; ``with_grads=False`` leaves dq, dk, dv as None (the
+        autograd op allocates them when its backward runs)."""
         st = llsa_validate_shape(shape)
         if st != 0:
             raise LLSAError("llsa_validate_shape", st)
@@ -277,9 +298,9 @@ class LLSABuffers:
             col=torch.empty(llsa_index_elems(shape), **i32),
             o=torch.empty(B, H, N, D, device=device, dtype=dtype),
             lse=torch.empty(B, H, N, **f32),
-            dq=torch.empty(B, H, N, D, device=device, dtype=dtype),
-            dk=torch.empty(B, H, N, D, device=device, dtype=dtype),
-            dv=torch.empty(B, H, N, D, device=device, dtype=dtype),
+            dq=torch.empty(B, H, N, D, device=device, dtype=dtype) if with_grads else None,
+            dk=torch.empty(B, H, N, D, device=device, dtype=dtype) if with_grads else None,
+            dv=torch.empty(B, H, N, D, device=device, dtype=dtype) if with_grads else None,
             ws_transpose=bytes_buf(llsa_transpose_workspace_bytes(shape)),
             ws_backward=bytes_buf(llsa_backward_workspace_bytes(shape)),
         )
@@ -401,30 +422,43 @@ class LLSAPlan:
 # ----------------------------------------------------------------------------- autograd op
 
 class _LLSAFunction(torch.autograd.Function):
+    """The op's output O is handed to autograd through ``save_for_backward`` and is not kept
+    in the buffers held on ``ctx`` (a tensor returned by forward and also stored as a ctx
+    attribute would close a reference cycle output -> grad_fn -> ctx -> output, which keeps
+    every buffer of the call alive until the cycle collector runs).  The gradient buffers are
+    allocated only when backward runs, and the ctx buffers are dropped after it."""
+
     @staticmethod
     def forward(ctx, q, k, v, topk: int, levels: int, flags: dict):
         B, H, N, D = q.shape
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         shape = make_shape(B, H, N, D, topk, levels, q.dtype, **flags)
-        buf = LLSABuffers.allocate(shape, q.device, q.dtype)
+        buf = LLSABuffers.allocate(shape, q.device, q.dtype, with_grads=False)
         llsa_forward_path(shape, q, k, v, buf)
-        ctx.save_for_backward(q, k, v)
+        o = buf.o
+        buf.o = None
+        ctx.save_for_backward(q, k, v, o)
         ctx.buf = buf
         ctx.shape = shape
-        return buf.o
+        return o
 
     @staticmethod
     def backward(ctx, do):
-        q, k, v = ctx.saved_tensors
-        buf = ctx.buf
-        llsa_backward_path(ctx.shape, q, k, v, do.contiguous(), buf)
-        return buf.dq, buf.dk, buf.dv, None, None, None
+        q, k, v, o = ctx.saved_tensors
+        buf, shape = ctx.buf, ctx.shape
+        ctx.buf = None
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        do = do.contiguous()
+        llsa_index_transpose(shape, buf.idx, buf.row_ptr, buf.col, buf.ws_transpose)
+        llsa_backward(shape, q, k, v, o, buf.lse, do, buf.k_pyr, buf.v_pyr, buf.idx, buf.row_ptr, buf.col,
+                      dq, dk, dv, buf.ws_backward)
+        return dq, dk, dv, None, None, None
 
 
 def llsa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk: int = 8, levels: int = 1,
                    log_bias: bool = False, all_top: bool = False, level1: bool = False) -> torch.Tensor:
     """Drop-in for ``F.scaled_dot_product_attention(q, k, v)`` (non-causal, no dropout) on
-    [B, H, N, 64] CUDA tensors, bf16 or fp32, with LLSA's hierarchical block-sparse KV lists.
+    [B, H, N, D] CUDA tensors (D = 64 or 128), bf16 or fp32, with LLSA's hierarchical block-sparse KV lists.
     ``log_bias``, ``all_top`` and ``level1`` select the enrichment variants (see make_shape)."""
     flags = dict(log_bias=log_bias, all_top=all_top, level1=level1)
     return _LLSAFunction.apply(q, k, v, topk, levels, flags)

@@ -2,8 +2,7 @@
 
 Usage: python -m log_linear_hierarchical_b200.build [--verbose-ptxas] [--define NAME=VALUE ...]
 
---define passes a compile-time switch to nvcc, e.g. LLSA_KEY_MAJOR_TC=1 selects the tcgen05
-key-major dK/dV kernel instead of the mma.sync one.
+--define passes a compile-time switch to nvcc, e.g. LLSA_KV_STAGES=3 for a deeper dK/dV ring.
 """
 from __future__ import annotations
 

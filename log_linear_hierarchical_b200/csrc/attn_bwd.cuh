@@ -34,6 +34,7 @@ struct BwdWorkspace {
   long long order;          // int4 [B*H*n_1] {key block, CSR row start, row end, 0}, longest row first
   long long order_counts;   // int32 [kOrdClasses][order tiles]
   long long order_nonempty; // int32: rows with at least one query block (they come first)
+  long long barrier;        // uint32[16]: the grid-barrier counter of the fused pyramid + selection
   long long total;
 };
 
@@ -54,7 +55,7 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   long long off = 0;
   w.delta = off;
   off = up(off + (long long)g.BH * g.N);
-  const long long parts = g.L >= 2 ? (long long)g.BH * g.n[2] * g.coarse * kD : 0;
+  const long long parts = g.L >= 2 ? (long long)g.BH * g.n[2] * g.coarse * g.D : 0;
   w.part_k = off;
   off = up(off + parts);
   w.part_v = off;
@@ -63,7 +64,7 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   for (int l = 0; l <= kMaxLevels; ++l) w.cg_off[l] = 0;
   for (int l = 2; l <= g.L; ++l) {
     w.cg_off[l] = cg;
-    cg += (long long)g.BH * g.n[l] * kD;
+    cg += (long long)g.BH * g.n[l] * g.D;
   }
   w.cg_k = off;
   off = up(off + cg);
@@ -75,17 +76,19 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   off = up(off + (long long)kOrdClasses * order_tiles(g));
   w.order_nonempty = off;
   off = up(off + 1);
+  w.barrier = off;
+  off = up(off + 16);
   w.total = off;
   return w;
 }
 
 // ---------------------------------------------------------------------------- query-major dQ
 
-template <int STAGES>
+template <int D, int STAGES>
 __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
   CtaSmem c;
-  c.coarse_bytes = 2 * g.coarse_pad * 128;
-  c.warp_tiles = 4 * kTileBytes + STAGES * 2 * kTileBytes;      // [2][Q, dO] + ring of [K, V]
+  c.coarse_bytes = 2 * g.coarse_pad * D * 2;
+  c.warp_tiles = 4 * tile_bytes<D>() + STAGES * 2 * tile_bytes<D>();  // [2][Q, dO] + ring of [K, V]
   c.warp_tail = 2 * kBlock * 4 + ((kUnitBlocks * g.K * 4 + 15) & ~15) + ((8 * (2 + STAGES) + 15) & ~15);
   c.nwarps = nwarps;
   return c;
@@ -94,16 +97,16 @@ __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
 // One 16-token chunk of the query-major backward: dQ += dS K with dS = P (dP - Delta).
 // POOL (level-1 variant, fine chunks): the block-mean entry has score mean(S) + pool_bias
 // and dP mean(dP); its dS, times the mean K row, is dS / 16 added to each of the 16 dS.
-template <bool MASK, bool POOL = false>
-__device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[4][4], const uint32_t (&df)[4][4], uint32_t ktile,
-                                         uint32_t vtile, int valid, float scale_log2, const float (&lse2)[2],
-                                         const float (&delta)[2], float (&dq)[8][4], const Geometry* bias_g = nullptr,
-                                         int c0 = 0, float pool_bias = 0.f) {
+template <int D, bool MASK, bool POOL = false>
+__device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const uint32_t (&df)[D / 16][4],
+                                         uint32_t ktile, uint32_t vtile, int valid, float scale_log2,
+                                         const float (&lse2)[2], const float (&delta)[2], float (&dq)[D / 8][4],
+                                         const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  mma_a_bt(s, qf, ktile);
-  mma_a_bt(dp, df, vtile);
+  mma_a_bt<D>(s, qf, ktile);
+  mma_a_bt<D>(dp, df, vtile);
   float pds[2] = {0.f, 0.f};  // pooled entry's dS / 16, rows r0 and r0 + 8
   if (POOL) {
     float t[2], u[2];
@@ -123,17 +126,19 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[4][4], const uint3
       const int col = n * 8 + 2 * (lane & 3) + (e & 1);
       const int r = e >> 1;
       float sb = s[n][e];
-      if (MASK && bias_g && bias_g->log_bias && col < valid) sb += coarse_log_bias(*bias_g, c0 + col) * kSqrtD;
+      if (MASK && bias_g && bias_g->log_bias && col < valid) sb += coarse_log_bias(*bias_g, c0 + col) * sqrt_d<D>();
       const float p = (!MASK || col < valid) ? ex2(fmaf(sb, scale_log2, -lse2[r])) : 0.0f;
       ds[n][e] = POOL ? fmaf(p, dp[n][e] - delta[r], pds[r]) : p * (dp[n][e] - delta[r]);
     }
-  mma_a_b(dq, pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]), pack_bf16(ds[1][0], ds[1][1]),
-          pack_bf16(ds[1][2], ds[1][3]), ktile);
+  mma_a_b<D>(dq, pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]), pack_bf16(ds[1][0], ds[1][1]),
+             pack_bf16(ds[1][2], ds[1][3]), ktile);
 }
 
 // Same CTA shape as the forward: 4 warps x 4 query blocks, coarse KV staged once per CTA.
-// POOL: the level-1 variant (see dq_chunk).
-template <int STAGES, bool POOL>
+// POOL: the level-1 variant (see dq_chunk).  PAD: a padded sequence -- the fine tile that
+// holds the last real token masks its padding keys; padding queries (zero Q and dO rows,
+// O = 0, LSE = 0) get dS = 0 and so dQ = 0 and Delta = 0 without a mask.
+template <int D, int STAGES, bool POOL, bool PAD>
 __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
@@ -151,16 +156,17 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
   const int n1 = g.n[1];
   const int K = g.K;
   const int total_blocks = g.BH * n1;
-  const CtaSmem cs = dq_smem<STAGES>(g, nwarps);
+  const CtaSmem cs = dq_smem<D, STAGES>(g, nwarps);
+  constexpr int TB = tile_bytes<D>();
   uint8_t* base = align1024(dq_smem_raw);
   const uint32_t ck = smem_u32(base);
-  const uint32_t cv = ck + g.coarse_pad * 128;
+  const uint32_t cv = ck + g.coarse_pad * D * 2;
   const int cta_first = blockIdx.x * nwarps * kUnitBlocks;
   if (g.L >= 2) {
     const int bh0 = cta_first / n1;
     const int p0 = cta_first - bh0 * n1;
-    stage_coarse_rows(g, k_pyr, idx, bh0, p0, ck, threadIdx.x, blockDim.x);
-    stage_coarse_rows(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
+    stage_coarse_rows<D>(g, k_pyr, idx, bh0, p0, ck, threadIdx.x, blockDim.x);
+    stage_coarse_rows<D>(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
     __syncthreads();
   }
   const int first = cta_first + warp * kUnitBlocks;
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
   }
   const int nblk = min(kUnitBlocks, total_blocks - first);
   const uint32_t qd = smem_u32(cs.tiles(base, warp));
-  const uint32_t ring = qd + 4 * kTileBytes;
+  const uint32_t ring = qd + 4 * TB;
   float* slse = reinterpret_cast<float*>(cs.tail(base, warp));  // [2][16]
   int* srow = reinterpret_cast<int*>(slse + 2 * kBlock);
   const uint32_t bar_qd = smem_u32(srow) + ((kUnitBlocks * K * 4 + 15) & ~15);
@@ -192,18 +198,18 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const int row = srow[seq];
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
-    const uint32_t dst = ring + stage * 2 * kTileBytes;
-    mbar_expect_tx(bar, 2 * kTileBytes);
-    tma_load_2d(dst, &tm_k, 0, row, bar);
-    tma_load_2d(dst + kTileBytes, &tm_v, 0, row, bar);
+    const uint32_t dst = ring + stage * 2 * TB;
+    mbar_expect_tx(bar, 2 * TB);
+    tma_load_tile<D>(dst, &tm_k, g, row, bar);
+    tma_load_tile<D>(dst + TB, &tm_v, g, row, bar);
   };
   auto issue_qd = [&](int i) {
     const uint32_t bar = bar_qd + 8 * (i & 1);
     const int row = (first + i) * kBlock;
-    const uint32_t dst = qd + (i & 1) * 2 * kTileBytes;
-    mbar_expect_tx(bar, 2 * kTileBytes + kBlock * 4);
-    tma_load_2d(dst, &tm_q, 0, row, bar);
-    tma_load_2d(dst + kTileBytes, &tm_do, 0, row, bar);
+    const uint32_t dst = qd + (i & 1) * 2 * TB;
+    mbar_expect_tx(bar, 2 * TB + kBlock * 4);
+    tma_load_tile<D>(dst, &tm_q, g, row, bar);
+    tma_load_tile<D>(dst + TB, &tm_do, g, row, bar);
     bulk_load(smem_u32(slse + (i & 1) * kBlock), lse + row, kBlock * 4, bar);
   };
   // the level-1 selection (two kernels back) and K, V are ready: the first K/V tiles are
@@ -216,44 +222,51 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 
   bool ok = true;
   int next_seq = 0, next_q = 0;
-  // O rows of the block being started, loaded one block ahead (lane: row lane/2, half lane%2)
-  auto load_o = [&](int i, uint4 (&dst)[4]) {
+  // O rows of a block (lane: row lane/2, channels (lane%2) * D/2 onwards).  At D = 64 they
+  // are loaded one block ahead; at D = 128 (twice the registers) when the block starts.
+  constexpr int OC = D / 16;  // 16-byte chunks per lane
+  constexpr bool kPrefetchO = D == 64;
+  auto load_o = [&](int i, uint4 (&dst)[OC]) {
     const uint4* orow =
-        reinterpret_cast<const uint4*>(o + ((long long)(first + i) * kBlock + (lane >> 1)) * kD + (lane & 1) * 32);
+        reinterpret_cast<const uint4*>(o + ((long long)(first + i) * kBlock + (lane >> 1)) * D + (lane & 1) * (D / 2));
 #pragma unroll
-    for (int c = 0; c < 4; ++c) dst[c] = __ldg(orow + c);
+    for (int c = 0; c < OC; ++c) dst[c] = __ldg(orow + c);
   };
-  uint4 onext[4];
-  load_o(0, onext);
+  uint4 onext[OC];
+  if constexpr (kPrefetchO) load_o(0, onext);
   for (int i = 0; i < nblk && ok; ++i) {
     const int gb = first + i;
-    uint4 ocur[4];
+    uint4 ocur[OC];
+    if constexpr (kPrefetchO) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) ocur[c] = onext[c];
-    if (i + 1 < nblk) load_o(i + 1, onext);
+      for (int c = 0; c < OC; ++c) ocur[c] = onext[c];
+      if (i + 1 < nblk) load_o(i + 1, onext);
+    } else {
+      load_o(i, ocur);
+    }
     ok = __all_sync(0xffffffffu, mbar_wait(bar_qd + 8 * (i & 1), (i >> 1) & 1));
     if (!ok) break;
     next_q = i + 1;
     // the other buffer was released at the end of block i-1
     if (lane == 0 && i + 1 < nblk) issue_qd(i + 1);
-    const uint32_t qt = qd + (i & 1) * 2 * kTileBytes;
-    const uint32_t dt = qt + kTileBytes;
-    uint32_t qf[4][4], df[4][4];
-    load_a_frags(qt, qf);
-    load_a_frags(dt, df);
-    // Delta_r = sum_d dO[r][d] * O[r][d] (O loaded a block ahead, dO from the staged tile)
+    const uint32_t qt = qd + (i & 1) * 2 * TB;
+    const uint32_t dt = qt + TB;
+    uint32_t qf[D / 16][4], df[D / 16][4];
+    load_a_frags<D>(qt, qf);
+    load_a_frags<D>(dt, df);
+    // Delta_r = sum_d dO[r][d] * O[r][d] (O from registers, dO from the staged tile)
     float dlt;
     {
       const int r = lane >> 1;
       const int h = lane & 1;
       float acc = 0.0f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < OC; ++c) {
         const uint4 ov = ocur[c];
         uint4 dv;
         asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                      : "=r"(dv.x), "=r"(dv.y), "=r"(dv.z), "=r"(dv.w)
-                     : "r"(dt + swz(r, h * 4 + c)));
+                     : "r"(dt + tswz(r, h * OC + c)));
         const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
         const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
@@ -269,9 +282,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const float delta[2] = {__shfl_sync(0xffffffffu, dlt, 2 * r0), __shfl_sync(0xffffffffu, dlt, 2 * r0 + 16)};
     const float lse2[2] = {slse[(i & 1) * kBlock + r0] * kLog2e, slse[(i & 1) * kBlock + r0 + 8] * kLog2e};
 
-    float dq[8][4];
+    float dq[D / 8][4];
 #pragma unroll
-    for (int n = 0; n < 8; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
+    for (int n = 0; n < D / 8; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
 #pragma unroll kQmUnroll
     for (int s = 0; s < K; ++s) {
       const int seq = i * K + s;
@@ -279,18 +292,22 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
       ok = __all_sync(0xffffffffu, mbar_wait(bar_kv + 8 * stage, (seq / STAGES) & 1));
       if (!ok) break;
       next_seq = seq + 1;
-      const uint32_t kt = ring + stage * 2 * kTileBytes;
-      dq_chunk<false, POOL>(qf, df, kt, kt + kTileBytes, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
-                            pool_log_bias(g));
+      const uint32_t kt = ring + stage * 2 * TB;
+      if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
+        dq_chunk<D, true>(qf, df, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - div_n1(g, gb) * g.N)),
+                          P.scale_log2, lse2, delta, dq);
+      else
+        dq_chunk<D, false, POOL>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
+                                 pool_log_bias<D>(g));
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
-      dq_chunk<true>(qf, df, ck + cc * kTileBytes, cv + cc * kTileBytes, min(kBlock, g.coarse - cc * kBlock),
+      dq_chunk<D, true>(qf, df, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock),
                      P.scale_log2, lse2, delta, dq, &g, cc * kBlock);
     __syncwarp();
-    store_tile_bf16(dq, P.scale, P.scale, qt, dq_out + (long long)gb * kBlock * kD);
+    store_tile_bf16<D>(dq, P.scale, P.scale, qt, dq_out + (long long)gb * kBlock * D);
   }
   if (!ok) {
     for (int seq = next_seq; seq < min(total_loads, next_seq + STAGES); ++seq)
@@ -304,23 +321,39 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 // One (key tile, query block) pair: with the key tile's K and V as A fragments (rows = keys),
 // and the query block's Q and dO tiles, LSE and Delta staged:
 //   S^T = K Q^T, P^T = exp2(S^T*scale*log2e - LSE*log2e), dP^T = V dO^T,
-//   dS^T = P^T (dP^T - Delta), dV += P^T dO, dK += dS^T Q  (dK unscaled).
+//   dS^T = P^T (dP^T - Delta), dV += P^T dO, dK += dS^T Q  (dK unscaled; P^T and dS^T as
+//   bf16 hi + lo pairs).
+// It runs as two phases: kv_scores (S^T, dP^T and the elementwise step) and kv_accumulate
+// (the dV, dK products).  At D = 64 the key tile's K and V fragments stay in registers; at
+// D = 128 (twice the accumulators) they are read from the staged tile at each k-step.
 // BIAS: the key rows are coarse tokens under the log-count variant; kb[0], kb[1] are the
 // biases (unscaled-dot units) of this lane's key rows r0 and r0 + 8.
 // POOL (level-1 variant; the key rows are a fine block): the block-mean entry, with score
 // mean over the 16 keys of S + pool_bias and dP the mean of dP, sends dV_mean = p dO and
 // dK_mean = dS q to the block's 16 rows with weight 1/16 each: p / 16 is added to every
 // P^T entry of its query column and dS / 16 to every dS^T entry.
-template <bool BIAS = false, bool POOL = false>
-__device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32_t (&vf)[4][4], uint32_t qt,
-                                        uint32_t dt, const float* ls, const float* dl, float scale_log2,
-                                        float (&dk)[8][4], float (&dv)[8][4], const float (&kb)[2] = {0.f, 0.f},
-                                        float pool_bias = 0.f) {
+template <int D>
+__host__ __device__ constexpr bool kv_frags_in_regs() {
+  return D == 64;
+}
+
+// kvalid < 16: the key tile holds the last real token of a padded sequence, and its rows
+// from kvalid on are padding (zero rows) whose P^T and dS^T are masked to 0.
+template <int D, bool BIAS = false, bool POOL = false>
+__device__ __forceinline__ void kv_scores(const uint32_t (&kf)[D / 16][4], const uint32_t (&vf)[D / 16][4],
+                                          uint32_t kvtile, uint32_t qt, uint32_t dt, const float* ls,
+                                          const float* dl, float scale_log2, float (&pt)[2][4], float (&dst)[2][4],
+                                          const float (&kb)[2], float pool_bias, int kvalid) {
   const int c2 = 2 * (lane_id() & 3);
   float st[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dpt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  mma_a_bt(st, kf, qt);   // S^T: rows = keys, cols = queries
-  mma_a_bt(dpt, vf, dt);  // dP^T
+  if constexpr (kv_frags_in_regs<D>()) {
+    mma_a_bt<D>(st, kf, qt);   // S^T: rows = keys, cols = queries
+    mma_a_bt<D>(dpt, vf, dt);  // dP^T
+  } else {
+    mma_at_bt<D>(st, kvtile, qt);
+    mma_at_bt<D>(dpt, kvtile + tile_bytes<D>(), dt);
+  }
   // this lane's four query columns: c2, c2 + 1 (n = 0) and c2 + 8, c2 + 9 (n = 1)
   const float2 l0 = *reinterpret_cast<const float2*>(ls + c2);
   const float2 l1 = *reinterpret_cast<const float2*>(ls + 8 + c2);
@@ -357,7 +390,6 @@ __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32
         da[n][c] = pa[n][c] * fmaf(tp[n][c], 1.0f / kBlock, -dq[n][c]);
       }
   }
-  float pt[2][4], dst[2][4];
 #pragma unroll
   for (int n = 0; n < 2; ++n)
 #pragma unroll
@@ -369,19 +401,46 @@ __device__ __forceinline__ void kv_pair(const uint32_t (&kf)[4][4], const uint32
         dst[n][e] += da[n][e & 1];
       }
     }
-  mma_a_b(dv, pack_bf16(pt[0][0], pt[0][1]), pack_bf16(pt[0][2], pt[0][3]), pack_bf16(pt[1][0], pt[1][1]),
-          pack_bf16(pt[1][2], pt[1][3]), dt);
-  mma_a_b(dk, pack_bf16(dst[0][0], dst[0][1]), pack_bf16(dst[0][2], dst[0][3]), pack_bf16(dst[1][0], dst[1][1]),
-          pack_bf16(dst[1][2], dst[1][3]), qt);
+  if (kvalid < kBlock) {
+    const int r0 = lane_id() >> 2;
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (r0 + 8 * (e >> 1) >= kvalid) pt[n][e] = dst[n][e] = 0.0f;
+  }
+}
+
+// dV += P^T dO and dK += dS^T Q for one pair.  P^T and dS^T enter the products as two bf16
+// terms each (value and rounding remainder).  A key's dV and dK sum P dO and dS q over every
+// query that selected it; with P and dS rounded once to bf16 (relative error 2^-9 per term)
+// the error of a key picked by hundreds of query blocks grew past the output tolerance (for
+// dK the terms also cancel: the dS of a query sum to zero, so |dK| stays moderate while its
+// error grows).
+template <int D>
+__device__ __forceinline__ void kv_accumulate(const float (&pt)[2][4], const float (&dst)[2][4], uint32_t qt,
+                                              uint32_t dt, float (&dk)[D / 8][4], float (&dv)[D / 8][4]) {
+  uint32_t phi[4], plo[4];
+  split_bf16(pt[0][0], pt[0][1], phi[0], plo[0]);
+  split_bf16(pt[0][2], pt[0][3], phi[1], plo[1]);
+  split_bf16(pt[1][0], pt[1][1], phi[2], plo[2]);
+  split_bf16(pt[1][2], pt[1][3], phi[3], plo[3]);
+  mma_a2_b<D>(dv, phi, plo, dt);
+  uint32_t dhi[4], dlo[4];
+  split_bf16(dst[0][0], dst[0][1], dhi[0], dlo[0]);
+  split_bf16(dst[0][2], dst[0][3], dhi[1], dlo[1]);
+  split_bf16(dst[1][0], dst[1][1], dhi[2], dlo[2]);
+  split_bf16(dst[1][2], dst[1][3], dhi[3], dlo[3]);
+  mma_a2_b<D>(dk, dhi, dlo, qt);
 }
 
 // Per-warp shared memory of the key-major kernels: the key tile's K and V, then a ring of
 // STAGES (Q tile, dO tile) stages; the tail holds LSE/Delta of each stage and the mbarriers.
-template <int STAGES>
+template <int D, int STAGES>
 __host__ __device__ inline CtaSmem kv_smem(int nwarps) {
   CtaSmem c;
   c.coarse_bytes = 0;
-  c.warp_tiles = 2 * kTileBytes + STAGES * 2 * kTileBytes;
+  c.warp_tiles = 2 * tile_bytes<D>() + STAGES * 2 * tile_bytes<D>();
   c.warp_tail = 2 * STAGES * kBlock * 4 + ((8 * (1 + STAGES) + 15) & ~15);
   c.nwarps = nwarps;
   return c;
@@ -392,13 +451,15 @@ __host__ __device__ inline CtaSmem kv_smem(int nwarps) {
 // `bar_tile` is non-zero the key tile is still arriving on that mbarrier (phase 0) and is
 // waited for after the first pair loads are issued.  Returns false (after draining the
 // copies in flight) if a wait timed out.
-template <int STAGES, bool BIAS = false, bool POOL = false, class PairBlock>
-__device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtensorMap* tm_do,
+template <int D, int STAGES, bool BIAS = false, bool POOL = false, class PairBlock>
+__device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* tm_q, const CUtensorMap* tm_do,
                                           const float* __restrict__ lse, const float* __restrict__ delta,
                                           uint32_t kvtile, uint32_t bar_tile, uint32_t ring, float* sls, float* sdl,
                                           uint32_t bar_ring, int npairs, PairBlock pair_block, float scale_log2,
-                                          float (&dk)[8][4], float (&dv)[8][4],
-                                          const float (&kbias)[2] = {0.f, 0.f}, float pool_bias = 0.f) {
+                                          float (&dk)[D / 8][4], float (&dv)[D / 8][4],
+                                          const float (&kbias)[2] = {0.f, 0.f}, float pool_bias = 0.f,
+                                          int kvalid = kBlock) {
+  constexpr int TB = tile_bytes<D>();
   const int lane = lane_id();
   // called by the whole warp (pair_block may shuffle); lane 0 issues the copies
   auto issue_pair = [&](int i) {
@@ -406,10 +467,10 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
     if (lane == 0) {
       const int stage = i % STAGES;
       const uint32_t bar = bar_ring + 8 * stage;
-      const uint32_t dst = ring + stage * 2 * kTileBytes;
-      mbar_expect_tx(bar, 2 * kTileBytes + 2 * kBlock * 4);
-      tma_load_2d(dst, tm_q, 0, row, bar);
-      tma_load_2d(dst + kTileBytes, tm_do, 0, row, bar);
+      const uint32_t dst = ring + stage * 2 * TB;
+      mbar_expect_tx(bar, 2 * TB + 2 * kBlock * 4);
+      tma_load_tile<D>(dst, tm_q, g, row, bar);
+      tma_load_tile<D>(dst + TB, tm_do, g, row, bar);
       bulk_load(smem_u32(sls + stage * kBlock), lse + row, kBlock * 4, bar);
       bulk_load(smem_u32(sdl + stage * kBlock), delta + row, kBlock * 4, bar);
     }
@@ -419,9 +480,11 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
     for (int j = 0; j < min(npairs, STAGES); ++j) mbar_wait(bar_ring + 8 * (j % STAGES), (j / STAGES) & 1);
     return false;
   }
-  uint32_t kf[4][4], vf[4][4];
-  load_a_frags(kvtile, kf);
-  load_a_frags(kvtile + kTileBytes, vf);
+  uint32_t kf[D / 16][4], vf[D / 16][4];
+  if constexpr (kv_frags_in_regs<D>()) {
+    load_a_frags<D>(kvtile, kf);
+    load_a_frags<D>(kvtile + TB, vf);
+  }
 #pragma unroll kKvUnroll
   for (int i = 0; i < npairs; ++i) {
     const int stage = i % STAGES;
@@ -429,9 +492,11 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
       for (int j = i; j < min(npairs, i + STAGES); ++j) mbar_wait(bar_ring + 8 * (j % STAGES), (j / STAGES) & 1);
       return false;
     }
-    const uint32_t qt = ring + stage * 2 * kTileBytes;
-    kv_pair<BIAS, POOL>(kf, vf, qt, qt + kTileBytes, sls + stage * kBlock, sdl + stage * kBlock, scale_log2, dk, dv,
-                        kbias, pool_bias);
+    const uint32_t qt = ring + stage * 2 * TB;
+    float pt[2][4], dst[2][4];
+    kv_scores<D, BIAS, POOL>(kf, vf, kvtile, qt, qt + TB, sls + stage * kBlock, sdl + stage * kBlock, scale_log2,
+                             pt, dst, kbias, pool_bias, kvalid);
+    kv_accumulate<D>(pt, dst, qt, qt + TB, dk, dv);
     __syncwarp();
     if (i + STAGES < npairs) issue_pair(i + STAGES);
   }
@@ -440,8 +505,8 @@ __device__ __forceinline__ bool kv_stream(const CUtensorMap* tm_q, const CUtenso
 
 // Coarse-token partial gradients.  One warp per (level-2 group, 16-token coarse tile): the
 // pairs are the group's 16 query blocks.  Rows >= C of the last tile are padding and are not
-// written.  Output: part_k / part_v [group][C][64] fp32 (dK unscaled).
-template <int STAGES>
+// written.  Output: part_k / part_v [group][C][D] fp32 (dK unscaled).
+template <int D, int STAGES>
 __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                   const __grid_constant__ CUtensorMap tm_do,
                                                                   AttnParams P, const float* __restrict__ k_pyr,
@@ -461,26 +526,28 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
   const int first_block = group * kBlock;  // flat index of the group's first query block
   const int bh = first_block / n1;
   const int p0 = first_block - bh * n1;
-  const CtaSmem cs = kv_smem<STAGES>(1);
+  const CtaSmem cs = kv_smem<D, STAGES>(1);
+  constexpr int TB = tile_bytes<D>();
   uint8_t* base = align1024(co_smem_raw);
   const uint32_t kvt = smem_u32(cs.tiles(base, 0));
-  const uint32_t ring = kvt + 2 * kTileBytes;
+  const uint32_t ring = kvt + 2 * TB;
   float* sls = reinterpret_cast<float*>(cs.tail(base, 0));
   float* sdl = sls + STAGES * kBlock;
   const uint32_t bar_ring = smem_u32(sdl + STAGES * kBlock);
 
   // stage this tile's 16 coarse K and V rows (bf16) like the forward does
   {
-    for (int t = lane; t < kBlock * 8; t += 32) {
-      const int r = t >> 3;
-      const int ch = t & 7;
+    constexpr int CH = D / 8;
+    for (int t = lane; t < kBlock * CH; t += 32) {
+      const int r = t / CH;
+      const int ch = t - r * CH;
       const int row = tile * kBlock + r;
       uint4 pk = make_uint4(0u, 0u, 0u, 0u), pv = make_uint4(0u, 0u, 0u, 0u);
       if (row < g.coarse) {
         int lev;
         const int j = coarse_token(g, idx, bh, p0, row, lev);
         const int nl = g.n[lev];
-        const long long off = g.pyr_off[lev] + ((long long)bh * nl + j) * kD + ch * 8;
+        const long long off = g.pyr_off[lev] + ((long long)bh * nl + j) * D + ch * 8;
         const float4 a = __ldg(reinterpret_cast<const float4*>(k_pyr + off));
         const float4 b = __ldg(reinterpret_cast<const float4*>(k_pyr + off) + 1);
         const float4 c = __ldg(reinterpret_cast<const float4*>(v_pyr + off));
@@ -488,10 +555,10 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
         pk = make_uint4(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
         pv = make_uint4(pack_bf16(c.x, c.y), pack_bf16(c.z, c.w), pack_bf16(d.x, d.y), pack_bf16(d.z, d.w));
       }
-      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kvt + swz(r, ch)), "r"(pk.x), "r"(pk.y),
+      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kvt + tswz(r, ch)), "r"(pk.x), "r"(pk.y),
                    "r"(pk.z), "r"(pk.w)
                    : "memory");
-      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kvt + kTileBytes + swz(r, ch)), "r"(pv.x),
+      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kvt + TB + tswz(r, ch)), "r"(pv.x),
                    "r"(pv.y), "r"(pv.z), "r"(pv.w)
                    : "memory");
     }
@@ -503,35 +570,35 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
   __syncwarp();
   pdl_wait();  // LSE and Delta (the pairs' inputs) come from the kernels ahead
   pdl_launch_dependents();
-  float dk[8][4], dv[8][4];
+  float dk[D / 8][4], dv[D / 8][4];
 #pragma unroll
-  for (int n = 0; n < 8; ++n)
+  for (int n = 0; n < D / 8; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
   bool ok;
   if (g.log_bias) {  // this lane's key rows are coarse entries tile * 16 + r0 and + 8
     const int r0 = tile * kBlock + (lane >> 2);
-    const float kb[2] = {r0 < g.coarse ? coarse_log_bias(g, r0) * kSqrtD : 0.f,
-                         r0 + 8 < g.coarse ? coarse_log_bias(g, r0 + 8) * kSqrtD : 0.f};
-    ok = kv_stream<STAGES, true>(&tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
+    const float kb[2] = {r0 < g.coarse ? coarse_log_bias(g, r0) * sqrt_d<D>() : 0.f,
+                         r0 + 8 < g.coarse ? coarse_log_bias(g, r0 + 8) * sqrt_d<D>() : 0.f};
+    ok = kv_stream<D, STAGES, true>(g, &tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
                                  [&](int i) { return first_block + i; }, P.scale_log2, dk, dv, kb);
   } else {
-    ok = kv_stream<STAGES>(&tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
+    ok = kv_stream<D, STAGES>(g, &tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
                            [&](int i) { return first_block + i; }, P.scale_log2, dk, dv);
   }
   if (!ok) return;
   const int r0 = lane >> 2;
   const int c2 = 2 * (lane & 3);
-  float* pk = ws + W.part_k + (long long)group * g.coarse * kD;
-  float* pv = ws + W.part_v + (long long)group * g.coarse * kD;
+  float* pk = ws + W.part_k + (long long)group * g.coarse * D;
+  float* pv = ws + W.part_v + (long long)group * g.coarse * D;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int row = tile * kBlock + r0 + 8 * h;
     if (row < g.coarse) {
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        *reinterpret_cast<float2*>(pk + row * kD + n * 8 + c2) = make_float2(dk[n][2 * h], dk[n][2 * h + 1]);
-        *reinterpret_cast<float2*>(pv + row * kD + n * 8 + c2) = make_float2(dv[n][2 * h], dv[n][2 * h + 1]);
+      for (int n = 0; n < D / 8; ++n) {
+        *reinterpret_cast<float2*>(pk + row * D + n * 8 + c2) = make_float2(dk[n][2 * h], dk[n][2 * h + 1]);
+        *reinterpret_cast<float2*>(pv + row * D + n * 8 + c2) = make_float2(dv[n][2 * h], dv[n][2 * h + 1]);
       }
     }
   }
@@ -545,6 +612,37 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
 // order, so the result does not depend on timing.
 constexpr int kReduceWarps = 8;
 
+// D/32 consecutive fp32 channels of one lane (a float2 at D = 64, a float4 at D = 128).
+template <int D>
+struct LaneVec {
+  float v[D / 32];
+};
+template <int D>
+__device__ __forceinline__ LaneVec<D> lane_load(const float* p) {
+  LaneVec<D> r;
+  if constexpr (D == 64) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    r.v[0] = x.x;
+    r.v[1] = x.y;
+  } else {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    r.v[0] = x.x;
+    r.v[1] = x.y;
+    r.v[2] = x.z;
+    r.v[3] = x.w;
+  }
+  return r;
+}
+template <int D>
+__device__ __forceinline__ void lane_store(float* p, const LaneVec<D>& r, float scale) {
+  if constexpr (D == 64) {
+    *reinterpret_cast<float2*>(p) = make_float2(r.v[0] * scale, r.v[1] * scale);
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(r.v[0] * scale, r.v[1] * scale, r.v[2] * scale, r.v[3] * scale);
+  }
+}
+
+template <int D>
 __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(Geometry g, float scale,
                                                                               const int* __restrict__ idx,
                                                                               const int* __restrict__ row_ptr,
@@ -552,7 +650,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
                                                                               float* __restrict__ ws) {
   // The CSR rows and the selection (two or more kernels back, or joined before this launch) are
   // read before waiting; the partials, written by the kernel ahead, after (see pdl_wait).
-  __shared__ float2 red_k[kReduceWarps][32], red_v[kReduceWarps][32];
+  constexpr int V = D / 32;  // channels per lane: V * lane .. V * lane + V - 1
+  __shared__ LaneVec<D> red_k[kReduceWarps][32], red_v[kReduceWarps][32];
   __shared__ int slot_of[64];
   __shared__ int anc_of[64];
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -583,7 +682,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
   const int* cl = col + g.idx_off[lev] + (long long)bh * E;
   const int* il = idx + g.idx_off[lev] + (long long)bh * E;
   const long long n2 = g.n[2];
-  float2 sk = make_float2(0.f, 0.f), sv = make_float2(0.f, 0.f);
+  LaneVec<D> sk, sv;
+#pragma unroll
+  for (int c = 0; c < V; ++c) sk.v[c] = sv.v[c] = 0.f;
   // CSR rows are processed in chunks of 64 entries: slots first, then the (entry, group) pairs
   bool waited = false;
   for (int c0 = rs; c0 < re; c0 += 64) {
@@ -614,27 +715,28 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
     const int pairs = cnt * span;
     // four pairs per iteration: their loads are independent, the sums stay in pair order
     for (int p0 = warp * 4; p0 < pairs; p0 += kReduceWarps * 4) {
-      float2 x[4], y[4];
+      LaneVec<D> x[4], y[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int pi = p0 + u;
-        x[u] = y[u] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < V; ++c) x[u].v[c] = y[u].v[c] = 0.f;
         if (pi < pairs) {
           const int e = pi / span;
           const int gi = pi - e * span;
           const long long grp = (long long)bh * n2 + (long long)anc_of[e] * span + gi;
-          const long long off = (grp * g.coarse + slot_of[e]) * kD + 2 * lane;
-          x[u] = *reinterpret_cast<const float2*>(ws + W.part_k + off);
-          y[u] = *reinterpret_cast<const float2*>(ws + W.part_v + off);
+          const long long off = (grp * g.coarse + slot_of[e]) * D + V * lane;
+          x[u] = lane_load<D>(ws + W.part_k + off);
+          y[u] = lane_load<D>(ws + W.part_v + off);
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        sk.x += x[u].x;
-        sk.y += x[u].y;
-        sv.x += y[u].x;
-        sv.y += y[u].y;
-      }
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int c = 0; c < V; ++c) {
+          sk.v[c] += x[u].v[c];
+          sv.v[c] += y[u].v[c];
+        }
     }
   }
   if (!waited) {  // an empty row: nothing was read from the kernel ahead
@@ -645,17 +747,19 @@ __global__ void __launch_bounds__(kReduceWarps * 32) coarse_grad_reduce_kernel(G
   red_v[warp][lane] = sv;
   __syncthreads();
   if (warp == 0) {
-    float2 tk = make_float2(0.f, 0.f), tv = make_float2(0.f, 0.f);
+    LaneVec<D> tk, tv;
 #pragma unroll
-    for (int w = 0; w < kReduceWarps; ++w) {
-      tk.x += red_k[w][lane].x;
-      tk.y += red_k[w][lane].y;
-      tv.x += red_v[w][lane].x;
-      tv.y += red_v[w][lane].y;
-    }
-    const long long out = W.cg_off[lev] + ((long long)bh * nl + j) * kD + 2 * lane;
-    *reinterpret_cast<float2*>(ws + W.cg_k + out) = make_float2(tk.x * scale, tk.y * scale);
-    *reinterpret_cast<float2*>(ws + W.cg_v + out) = tv;
+    for (int c = 0; c < V; ++c) tk.v[c] = tv.v[c] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w)
+#pragma unroll
+      for (int c = 0; c < V; ++c) {
+        tk.v[c] += red_k[w][lane].v[c];
+        tv.v[c] += red_v[w][lane].v[c];
+      }
+    const long long out = W.cg_off[lev] + ((long long)bh * nl + j) * D + V * lane;
+    lane_store<D>(ws + W.cg_k + out, tk, scale);
+    lane_store<D>(ws + W.cg_v + out, tv, 1.0f);
   }
 }
 
@@ -797,7 +901,7 @@ __global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometr
 // whose output (the coarse-token gradients) only the epilogue reads; everything the main
 // loop reads was complete before that kernel could start, so the wait for it is deferred
 // to the epilogue and the main loop overlaps the reduction.
-template <int STAGES, bool POOL>
+template <int D, int STAGES, bool POOL>
 __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
@@ -825,8 +929,9 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
       const int cnt = min(kBlock, g.BH * n1 - e0);
       const int my_kb = lane < cnt ? checked_index(__ldg(&order[e0 + lane].x), g.BH * n1) : 0;
       // four rows at a time: all their coarse-gradient loads are issued before any sum
+      constexpr int V = D / 32;  // channels per lane
       for (int r0 = 0; r0 < cnt; r0 += 4) {
-        float2 xk[4][kMaxLevels], xv[4][kMaxLevels];
+        LaneVec<D> xk[4][kMaxLevels], xv[4][kMaxLevels];
         int kbs[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -836,14 +941,15 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
           long long cg_level = 0;
 #pragma unroll
           for (int lev = 2; lev <= kMaxLevels; ++lev) {
-            xk[u][lev - 1] = xv[u][lev - 1] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < V; ++c) xk[u][lev - 1].v[c] = xv[u][lev - 1].v[c] = 0.f;
             if (lev <= g.L) {
               span *= kBlock;
               nl /= kBlock;
-              const long long off = cg_level + ((long long)bh * nl + j / span) * kD + 2 * lane;
-              xk[u][lev - 1] = *reinterpret_cast<const float2*>(ws + W.cg_k + off);
-              xv[u][lev - 1] = *reinterpret_cast<const float2*>(ws + W.cg_v + off);
-              cg_level += (long long)g.BH * nl * kD;
+              const long long off = cg_level + ((long long)bh * nl + j / span) * D + V * lane;
+              xk[u][lev - 1] = lane_load<D>(ws + W.cg_k + off);
+              xv[u][lev - 1] = lane_load<D>(ws + W.cg_v + off);
+              cg_level += (long long)g.BH * nl * D;
             }
           }
         }
@@ -851,23 +957,43 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
         for (int u = 0; u < 4; ++u) {
           if (r0 + u >= cnt) break;
           const int bh = kbs[u] / n1, j = kbs[u] - bh * n1;
-          float2 ak = make_float2(0.f, 0.f), av = make_float2(0.f, 0.f);  // channels 2 lane, 2 lane + 1
-          float wgt = 1.0f / kBlock;
+          float ak[V], av[V];  // channels V lane .. V lane + V - 1
+#pragma unroll
+          for (int c = 0; c < V; ++c) ak[c] = av[c] = 0.f;
+          int span = 1;
 #pragma unroll
           for (int lev = 2; lev <= kMaxLevels; ++lev) {
             if (lev > g.L) break;
-            wgt *= 1.0f / kBlock;
-            ak.x += wgt * xk[u][lev - 1].x;
-            ak.y += wgt * xk[u][lev - 1].y;
-            av.x += wgt * xv[u][lev - 1].x;
-            av.y += wgt * xv[u][lev - 1].y;
+            span *= kBlock;
+            // 1 / 16^l, or 1 / (real tokens) of an ancestor a padded sequence cuts
+            const int c = pool_count(g, lev, j / span);
+            const float wgt = c > 0 ? 1.0f / (float)c : 0.0f;
+#pragma unroll
+            for (int c = 0; c < V; ++c) {
+              ak[c] += wgt * xk[u][lev - 1].v[c];
+              av[c] += wgt * xv[u][lev - 1].v[c];
+            }
           }
-          const uint32_t pk = pack_bf16(ak.x, ak.y), pv = pack_bf16(av.x, av.y);
+          uint32_t pk[V / 2], pv[V / 2];
+#pragma unroll
+          for (int c = 0; c < V / 2; ++c) {
+            pk[c] = pack_bf16(ak[2 * c], ak[2 * c + 1]);
+            pv[c] = pack_bf16(av[2 * c], av[2 * c + 1]);
+          }
           const long long row0 = (long long)bh * g.N + (long long)j * kBlock;
+          const int kvalid = g.nv - j * kBlock;  // padding positions get 0
 #pragma unroll
           for (int t = 0; t < kBlock; ++t) {
-            reinterpret_cast<uint32_t*>(dk_out + (row0 + t) * kD)[lane] = pk;
-            reinterpret_cast<uint32_t*>(dv_out + (row0 + t) * kD)[lane] = pv;
+            const bool real = t < kvalid;
+            if constexpr (V == 2) {
+              reinterpret_cast<uint32_t*>(dk_out + (row0 + t) * D)[lane] = real ? pk[0] : 0u;
+              reinterpret_cast<uint32_t*>(dv_out + (row0 + t) * D)[lane] = real ? pv[0] : 0u;
+            } else {
+              reinterpret_cast<uint2*>(dk_out + (row0 + t) * D)[lane] =
+                  real ? make_uint2(pk[0], pk[1]) : make_uint2(0u, 0u);
+              reinterpret_cast<uint2*>(dv_out + (row0 + t) * D)[lane] =
+                  real ? make_uint2(pv[0], pv[1]) : make_uint2(0u, 0u);
+            }
           }
         }
       }
@@ -880,10 +1006,11 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   const int kb = checked_index(ent.x, g.BH * n1);
   const int bh = kb / n1;
   const int j = kb - bh * n1;
-  const CtaSmem cs = kv_smem<STAGES>(1);
+  const CtaSmem cs = kv_smem<D, STAGES>(1);
+  constexpr int TB = tile_bytes<D>();
   uint8_t* base = align1024(dkv_smem_raw);
   const uint32_t kvt = smem_u32(cs.tiles(base, 0));
-  const uint32_t ring = kvt + 2 * kTileBytes;
+  const uint32_t ring = kvt + 2 * TB;
   float* sls = reinterpret_cast<float*>(cs.tail(base, 0));
   float* sdl = sls + STAGES * kBlock;
   const uint32_t bar_kv = smem_u32(sdl + STAGES * kBlock);
@@ -903,53 +1030,53 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   }
   __syncwarp();
   if (lane == 0) {
-    mbar_expect_tx(bar_kv, 2 * kTileBytes);
-    tma_load_2d(kvt, &tm_k, 0, bh * g.N + j * kBlock, bar_kv);
-    tma_load_2d(kvt + kTileBytes, &tm_v, 0, bh * g.N + j * kBlock, bar_kv);
+    mbar_expect_tx(bar_kv, 2 * TB);
+    tma_load_tile<D>(kvt, &tm_k, g, bh * g.N + j * kBlock, bar_kv);
+    tma_load_tile<D>(kvt + TB, &tm_v, g, bh * g.N + j * kBlock, bar_kv);
   }
-  float dk[8][4], dv[8][4];
+  float dk[D / 8][4], dv[D / 8][4];
 #pragma unroll
-  for (int n = 0; n < 8; ++n)
+  for (int n = 0; n < D / 8; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
   const int bh_block0 = bh * n1;
   // the row's query blocks are read 32 at a time by the whole warp and handed to the
   // issuing lane by shuffle, so no load sits on the TMA issue path
   int cached_base = -64, cached = 0;
-  const bool ok = kv_stream<STAGES, false, POOL>(&tm_q, &tm_do, lse, ws + W.delta, kvt, bar_kv, ring, sls, sdl,
-                                                 bar_ring, re - rs,
-                                    [&](int i) {
-                                      const int base32 = i & ~31;
-                                      if (base32 != cached_base) {
-                                        cached_base = base32;
-                                        const int e = base32 + lane;
-                                        cached = e < re - rs ? checked_index(__ldg(cl + e), n1) : 0;
-                                      }
-                                      return bh_block0 + __shfl_sync(0xffffffffu, cached, i & 31);
-                                    },
-                                    P.scale_log2, dk, dv, {0.f, 0.f}, pool_log_bias(g));
+  auto pair_block = [&](int i) {
+    const int base32 = i & ~31;
+    if (base32 != cached_base) {
+      cached_base = base32;
+      const int e = base32 + lane;
+      cached = e < re - rs ? checked_index(__ldg(cl + e), n1) : 0;
+    }
+    return bh_block0 + __shfl_sync(0xffffffffu, cached, i & 31);
+  };
+  const int kvalid = min(kBlock, g.nv - j * kBlock);  // real keys of this block (16 unless padded)
+  const bool ok = kv_stream<D, STAGES, false, POOL>(g, &tm_q, &tm_do, lse, ws + W.delta, kvt, bar_kv, ring, sls, sdl,
+                                                    bar_ring, re - rs, pair_block, P.scale_log2, dk, dv, {0.f, 0.f},
+                                                    pool_log_bias<D>(g), kvalid);
   if (!ok) return;
   if (coarse_late) pdl_wait();
   // epilogue: scale dK, add the mean-pool adjoint of the ancestors' coarse gradients
   const int c2 = 2 * (lane & 3);
 #pragma unroll
-  for (int n = 0; n < 8; ++n)
+  for (int n = 0; n < D / 8; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] *= P.scale;
   int span = 1;  // 16^(l-1): level-1 blocks under one level-l token
-  float wgt = 1.0f / kBlock;
   long long cg_level = 0;  // offset of level l in the coarse-gradient arrays
   int nl = n1;
   for (int lev = 2; lev <= g.L; ++lev) {
     span *= kBlock;
-    wgt *= 1.0f / kBlock;  // 1 / 16^l
     nl /= kBlock;          // n_l
     const int a = j / span;
-    const float* ck = ws + W.cg_k + cg_level + ((long long)bh * nl + a) * kD;
-    const float* cv = ws + W.cg_v + cg_level + ((long long)bh * nl + a) * kD;
-    cg_level += (long long)g.BH * nl * kD;
+    const float wgt = 1.0f / (float)pool_count(g, lev, a);  // 1 / 16^l unless a padded sequence cuts a
+    const float* ck = ws + W.cg_k + cg_level + ((long long)bh * nl + a) * D;
+    const float* cv = ws + W.cg_v + cg_level + ((long long)bh * nl + a) * D;
+    cg_level += (long long)g.BH * nl * D;
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
+    for (int n = 0; n < D / 8; ++n) {
       const float2 xk = *reinterpret_cast<const float2*>(ck + n * 8 + c2);
       const float2 xv = *reinterpret_cast<const float2*>(cv + n * 8 + c2);
       dk[n][0] += wgt * xk.x;
@@ -963,8 +1090,10 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
     }
   }
   const long long row0 = (long long)bh * g.N + (long long)j * kBlock;
-  store_tile_bf16(dk, 1.0f, 1.0f, kvt, dk_out + row0 * kD);
-  store_tile_bf16(dv, 1.0f, 1.0f, kvt + kTileBytes, dv_out + row0 * kD);
+  const int r0 = lane >> 2;  // padding positions of a padded sequence get dK = dV = 0
+  const float s0 = r0 < kvalid ? 1.0f : 0.0f, s1 = r0 + 8 < kvalid ? 1.0f : 0.0f;
+  store_tile_bf16<D>(dk, s0, s1, kvt, dk_out + row0 * D);
+  store_tile_bf16<D>(dv, s0, s1, kvt + TB, dv_out + row0 * D);
 }
 
 }  // namespace llsa

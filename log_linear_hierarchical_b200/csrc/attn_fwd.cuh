@@ -12,9 +12,13 @@
 //   O = O*exp2(m_old - m) + P V.
 // Coarse rows are fp32 in the pyramid; they are rounded to bf16 as they are staged.
 //
-// Bound: the gathered K/V bytes (T * 64 * 2 * 2 per query block; one head's K and V are
-// 16.8 MB at N = 65536, so most re-gathers hit L2) against HBM bandwidth, and the
-// 4 * 16 * T * 64 tensor FLOPs per block.
+// Head width D is 64 or 128 (a template parameter of every kernel).  A 16-token tile of D
+// bf16 channels is D/64 sub-tiles of 16 rows x 128 bytes, each one 2-D TMA box with
+// 128-byte swizzle (x = 0 and x = 64), stored one after the other.
+//
+// Bound: the gathered K/V bytes (T * D * 2 * 2 per query block; one head's K and V are
+// 16.8 MB at N = 65536, D = 64, so most re-gathers hit L2) against HBM bandwidth, and the
+// 4 * 16 * T * D tensor FLOPs per block.
 #pragma once
 
 #include "llsa_common.cuh"
@@ -35,103 +39,190 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// A-operand fragments of a 16 x 64 bf16 tile (rows = M, channels = K) for the 4 k-steps.
-__device__ __forceinline__ void load_a_frags(uint32_t tile, uint32_t (&f)[4][4]) {
-  const int lane = lane_id();
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk)
-    ldsm_x4(tile + swz(lane & 15, 2 * kk + (lane >> 4)), f[kk][0], f[kk][1], f[kk][2], f[kk][3]);
+// Bytes of one 16-token tile of D bf16 channels, and the byte offset of 16-byte chunk `ch`
+// (0 <= ch < D/8) of row `row` in it: sub-tile ch / 8, swizzled chunk ch % 8.
+template <int D>
+__host__ __device__ constexpr int tile_bytes() {
+  return kBlock * D * 2;
+}
+__device__ __forceinline__ uint32_t tswz(int row, int ch) {
+  return static_cast<uint32_t>((ch >> 3) * kSubTileBytes) + swz(row, ch & 7);
 }
 
-// acc[2][4] (16 x 16) += A (16 x 64, fragments) * B^T where B is a 16-row x 64 tile (rows = N).
-__device__ __forceinline__ void mma_a_bt(float (&acc)[2][4], const uint32_t (&a)[4][4], uint32_t btile) {
+// A-operand fragments of a 16 x D bf16 tile (rows = M, channels = K) for the D/16 k-steps.
+template <int D>
+__device__ __forceinline__ void load_a_frags(uint32_t tile, uint32_t (&f)[D / 16][4]) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    ldsm_x4(tile + tswz(lane & 15, 2 * kk + (lane >> 4)), f[kk][0], f[kk][1], f[kk][2], f[kk][3]);
+}
+
+// acc[2][4] (16 x 16) += A (16 x D, fragments) * B^T where B is a 16-row x D tile (rows = N).
+template <int D>
+__device__ __forceinline__ void mma_a_bt(float (&acc)[2][4], const uint32_t (&a)[D / 16][4], uint32_t btile) {
   const int lane = lane_id();
   const int row = (lane & 7) + ((lane >> 4) << 3);
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
+  for (int kk = 0; kk < D / 16; ++kk) {
     uint32_t b0, b1, b2, b3;
-    ldsm_x4(btile + swz(row, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
+    ldsm_x4(btile + tswz(row, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
     mma_bf16(acc[0], a[kk][0], a[kk][1], a[kk][2], a[kk][3], b0, b1);
     mma_bf16(acc[1], a[kk][0], a[kk][1], a[kk][2], a[kk][3], b2, b3);
   }
 }
 
-// acc[8][4] (16 x 64) += A (16 x 16: a0..a3) * B where B is a 16-row x 64 tile (rows = K).
-__device__ __forceinline__ void mma_a_b(float (&acc)[8][4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+// The same with A read from its shared-memory tile one k-step at a time (no A fragments
+// held in registers).
+template <int D>
+__device__ __forceinline__ void mma_at_bt(float (&acc)[2][4], uint32_t atile, uint32_t btile) {
+  const int lane = lane_id();
+  const int row = (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+    ldsm_x4(atile + tswz(lane & 15, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
+    ldsm_x4(btile + tswz(row, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
+    mma_bf16(acc[0], a0, a1, a2, a3, b0, b1);
+    mma_bf16(acc[1], a0, a1, a2, a3, b2, b3);
+  }
+}
+
+// acc[D/8][4] (16 x D) += A (16 x 16: a0..a3) * B where B is a 16-row x D tile (rows = K).
+template <int D>
+__device__ __forceinline__ void mma_a_b(float (&acc)[D / 8][4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t btile) {
   const int lane = lane_id();
   const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
-  for (int dc = 0; dc < 4; ++dc) {
+  for (int dc = 0; dc < D / 16; ++dc) {
     uint32_t b0, b1, b2, b3;
-    ldsm_x4_t(btile + swz(row, 2 * dc + (lane >> 4)), b0, b1, b2, b3);
+    ldsm_x4_t(btile + tswz(row, 2 * dc + (lane >> 4)), b0, b1, b2, b3);
     mma_bf16(acc[2 * dc], a0, a1, a2, a3, b0, b1);
     mma_bf16(acc[2 * dc + 1], a0, a1, a2, a3, b2, b3);
   }
 }
 
+// acc[D/8][4] (16 x D) += (A_hi + A_lo) (16 x 16) * B, B a 16-row x D tile (rows = K): one
+// set of B fragments serves both halves of a two-term bf16 operand; the products of the
+// high half are issued before those of the low half (no accumulator waits on its own
+// previous product), 64 channels at a time.
+template <int D>
+__device__ __forceinline__ void mma_a2_b(float (&acc)[D / 8][4], const uint32_t (&hi)[4], const uint32_t (&lo)[4],
+                                         uint32_t btile) {
+  const int lane = lane_id();
+  const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    uint32_t b[4][4];
+#pragma unroll
+    for (int dc = 0; dc < 4; ++dc)
+      ldsm_x4_t(btile + tswz(row, 8 * h + 2 * dc + (lane >> 4)), b[dc][0], b[dc][1], b[dc][2], b[dc][3]);
+#pragma unroll
+    for (int dc = 0; dc < 4; ++dc) {
+      mma_bf16(acc[8 * h + 2 * dc], hi[0], hi[1], hi[2], hi[3], b[dc][0], b[dc][1]);
+      mma_bf16(acc[8 * h + 2 * dc + 1], hi[0], hi[1], hi[2], hi[3], b[dc][2], b[dc][3]);
+    }
+#pragma unroll
+    for (int dc = 0; dc < 4; ++dc) {
+      mma_bf16(acc[8 * h + 2 * dc], lo[0], lo[1], lo[2], lo[3], b[dc][0], b[dc][1]);
+      mma_bf16(acc[8 * h + 2 * dc + 1], lo[0], lo[1], lo[2], lo[3], b[dc][2], b[dc][3]);
+    }
+  }
+}
+
+// Two fp32 values as a bf16 pair hi (round to nearest) and the pair of their bf16-rounded
+// remainders lo, so that hi + lo carries about 16 significant bits of each value.
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(a, b);
+  lo = pack_bf16(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
+
 // Stage the C coarse rows of a pyramid (fp32) as bf16 16-row swizzled tiles; padding rows
 // (index >= C) are zero.  Row c is the pyramid row of coarse entry c (see coarse_token).
 // Threads `tid` = 0..nthreads-1 share the work (a warp or a whole CTA).
+template <int D>
 __device__ __forceinline__ void stage_coarse_rows(const Geometry& g, const float* __restrict__ pyr,
                                                   const int* __restrict__ idx, int bh, int p, uint32_t dst, int tid,
                                                   int nthreads) {
-  for (int t = tid; t < g.coarse_pad * 8; t += nthreads) {
-    const int row = t >> 3;
-    const int ch = t & 7;
+  constexpr int CH = D / 8;  // 16-byte bf16 chunks per row
+  for (int t = tid; t < g.coarse_pad * CH; t += nthreads) {
+    const int row = t / CH;
+    const int ch = t - row * CH;
     uint4 packed = make_uint4(0u, 0u, 0u, 0u);
     if (row < g.coarse) {
       int lev;
       const int j = coarse_token(g, idx, bh, p, row, lev);
       const int nl = g.n[lev];
-      const float4* src = reinterpret_cast<const float4*>(pyr + g.pyr_off[lev] + ((long long)bh * nl + j) * kD + ch * 8);
+      const float4* src = reinterpret_cast<const float4*>(pyr + g.pyr_off[lev] + ((long long)bh * nl + j) * D + ch * 8);
       const float4 x = __ldg(src);
       const float4 y = __ldg(src + 1);
       packed = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
     }
-    const uint32_t addr = dst + (row >> 4) * kTileBytes + swz(row & 15, ch);
+    const uint32_t addr = dst + (row >> 4) * tile_bytes<D>() + tswz(row & 15, ch);
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(packed.x), "r"(packed.y), "r"(packed.z),
                  "r"(packed.w)
                  : "memory");
   }
 }
 
-// Write a 16 x 64 fp32 accumulator (fragment layout, already scaled) as bf16 rows
-// [row0, row0 + 16) of a [rows, 64] global array, through a swizzled shared staging tile.
-__device__ __forceinline__ void store_tile_bf16(const float (&acc)[8][4], float s0, float s1, uint32_t stage,
+// Write a 16 x D fp32 accumulator (fragment layout, already scaled) as bf16 rows
+// [row0, row0 + 16) of a [rows, D] global array, through a swizzled shared staging tile.
+template <int D>
+__device__ __forceinline__ void store_tile_bf16(const float (&acc)[D / 8][4], float s0, float s1, uint32_t stage,
                                                 __nv_bfloat16* __restrict__ dst_rows) {
   const int lane = lane_id();
   const int r0 = lane >> 2;
   const uint32_t cb = (lane & 3) * 4;
 #pragma unroll
-  for (int n = 0; n < 8; ++n) {
+  for (int n = 0; n < D / 8; ++n) {
     const uint32_t v0 = pack_bf16(acc[n][0] * s0, acc[n][1] * s0);
     const uint32_t v1 = pack_bf16(acc[n][2] * s1, acc[n][3] * s1);
-    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(stage + swz(r0, n) + cb), "r"(v0) : "memory");
-    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(stage + swz(r0 + 8, n) + cb), "r"(v1) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(stage + tswz(r0, n) + cb), "r"(v0) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(stage + tswz(r0 + 8, n) + cb), "r"(v1) : "memory");
   }
   __syncwarp();
+  constexpr int CH = D / 8;
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
+  for (int it = 0; it < D / 16; ++it) {
     const int ci = lane + 32 * it;
-    const int row = ci >> 3;
-    const int c = ci & 7;
+    const int row = ci / CH;
+    const int c = ci - row * CH;
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(stage + swz(row, c)));
-    *reinterpret_cast<uint4*>(dst_rows + row * kD + c * 8) = v;
+                 : "r"(stage + tswz(row, c)));
+    *reinterpret_cast<uint4*>(dst_rows + row * D + c * 8) = v;
   }
   // the staging tile is refilled by TMA later: order these generic accesses before it
   fence_proxy_async();
   __syncwarp();
 }
 
-constexpr float kSqrtD = 8.0f;  // sqrt(kD): score bias in units of the unscaled dot product
+// Loads of the 16-token x D tile that starts at flat token row `row` (= (b*H + h) * N + t):
+// D/64 boxes of the [B*H][n_valid][D] tensor map, at x = 0, 64.  Rows at or past n_valid
+// (the padding of a padded sequence) arrive as zeros.
+template <int D>
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, const Geometry& g, int row,
+                                              uint32_t bar) {
+  const int bh = div_n(g, row);
+  const int t = row - bh * g.N;
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * kSubTileBytes, map, 64 * h, t, bh, bar);
+}
+
+// sqrt(D): a score bias in units of the unscaled dot product is the scaled bias times this.
+template <int D>
+__host__ __device__ constexpr float sqrt_d() {
+  return D == 64 ? 8.0f : 11.313708498984761f;
+}
 
 // Bias of a level-1 pooled entry (level-1 variant) in unscaled-dot units: ln 16 under the
 // log-count variant, else 0.
-__host__ __device__ inline float pool_log_bias(const Geometry& g) { return g.log_bias ? kLn16 * kSqrtD : 0.0f; }
+template <int D>
+__host__ __device__ inline float pool_log_bias(const Geometry& g) {
+  return g.log_bias ? kLn16 * sqrt_d<D>() : 0.0f;
+}
 
 // Row sums of a 16 x 16 score fragment (C layout): rows r0 and r0 + 8 of this lane's quad.
 __device__ __forceinline__ void quad_row_sums(const float (&s)[2][4], float& t0, float& t1) {
@@ -151,13 +242,13 @@ __device__ __forceinline__ void quad_row_sums(const float (&s)[2][4], float& t0,
 // entry.  Its score is the mean of the 16 scores (q . mean k = mean of q . k), plus
 // `pool_bias` (unscaled-dot units), and since its value is the mean of the 16 V rows its
 // weight p folds into the chunk as p / 16 added to each of the 16 probabilities.
-template <bool MASK, bool POOL = false>
-__device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t ktile, uint32_t vtile, int valid,
-                                          float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[8][4],
+template <int D, bool MASK, bool POOL = false>
+__device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint32_t ktile, uint32_t vtile, int valid,
+                                          float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[D / 8][4],
                                           const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  mma_a_bt(s, qf, ktile);
+  mma_a_bt<D>(s, qf, ktile);
   float sb0 = 0.f, sb1 = 0.f;  // pooled scores of rows r0, r0 + 8
   if (POOL) {
     quad_row_sums(s, sb0, sb1);
@@ -171,7 +262,7 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
       for (int e = 0; e < 4; ++e) {
         const int col = n * 8 + 2 * (lane & 3) + (e & 1);
         if (col >= valid) s[n][e] = -INFINITY;
-        else if (bias_g && bias_g->log_bias) s[n][e] += coarse_log_bias(*bias_g, c0 + col) * kSqrtD;
+        else if (bias_g && bias_g->log_bias) s[n][e] += coarse_log_bias(*bias_g, c0 + col) * sqrt_d<D>();
       }
   }
   float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
@@ -213,7 +304,7 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
     l[0] *= c0;
     l[1] *= c1;
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
+    for (int n = 0; n < D / 8; ++n) {
       acc[n][0] *= c0;
       acc[n][1] *= c0;
       acc[n][2] *= c1;
@@ -224,15 +315,15 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[4][4], uint32_t k
   }
   l[0] += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
   l[1] += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
-  mma_a_b(acc, pack_bf16(p[0][0], p[0][1]), pack_bf16(p[0][2], p[0][3]), pack_bf16(p[1][0], p[1][1]),
-          pack_bf16(p[1][2], p[1][3]), vtile);
+  mma_a_b<D>(acc, pack_bf16(p[0][0], p[0][1]), pack_bf16(p[0][2], p[0][3]), pack_bf16(p[1][0], p[1][1]),
+             pack_bf16(p[1][2], p[1][3]), vtile);
 }
 
 // Shared memory of the attention kernels: a CTA region (the group's coarse K and V tiles),
 // then per warp a block of 1024-aligned tiles, then per warp a small tail (indices,
 // mbarriers).  Offsets are in bytes from the 1024-aligned base.
 struct CtaSmem {
-  int coarse_bytes;  // 2 * coarse_pad * 128
+  int coarse_bytes;  // 2 * coarse_pad * D * 2
   int warp_tiles;    // bytes of tiles per warp (multiple of 1024)
   int warp_tail;     // bytes of tail per warp (multiple of 16)
   int nwarps;
@@ -243,11 +334,11 @@ struct CtaSmem {
   }
 };
 
-template <int STAGES>
+template <int D, int STAGES>
 __host__ __device__ inline CtaSmem fwd_smem(const Geometry& g, int nwarps) {
   CtaSmem c;
-  c.coarse_bytes = 2 * g.coarse_pad * 128;
-  c.warp_tiles = 2 * kTileBytes + STAGES * 2 * kTileBytes;
+  c.coarse_bytes = 2 * g.coarse_pad * D * 2;
+  c.warp_tiles = 2 * tile_bytes<D>() + STAGES * 2 * tile_bytes<D>();
   c.warp_tail = ((kUnitBlocks * g.K * 4 + 15) & ~15) + ((8 * (2 + STAGES) + 15) & ~15);
   c.nwarps = nwarps;
   return c;
@@ -256,8 +347,10 @@ __host__ __device__ inline CtaSmem fwd_smem(const Geometry& g, int nwarps) {
 // One CTA = 4 warps = 16 consecutive query blocks (one level-2 group when L >= 2, so the
 // coarse KV entries are staged once per CTA).  Each warp owns 4 blocks and streams their
 // fine KV tiles through its own ring of STAGES mbarrier-tracked TMA stages.  POOL: the
-// level-1 variant (see fwd_chunk).
-template <int STAGES, bool POOL>
+// level-1 variant (see fwd_chunk).  PAD: a padded sequence -- the fine tile that holds the
+// last real token masks its padding keys (which arrive as zero rows), and padding queries
+// write O = 0 and LSE = 0.
+template <int D, int STAGES, bool POOL, bool PAD>
 __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                             const __grid_constant__ CUtensorMap tm_k,
                                                             const __grid_constant__ CUtensorMap tm_v, AttnParams P,
@@ -275,16 +368,16 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   const int n1 = g.n[1];
   const int K = g.K;
   const int total_blocks = g.BH * n1;
-  const CtaSmem cs = fwd_smem<STAGES>(g, nwarps);
+  const CtaSmem cs = fwd_smem<D, STAGES>(g, nwarps);
   uint8_t* base = align1024(fwd_smem_raw);
   const uint32_t ck = smem_u32(base);
-  const uint32_t cv = ck + g.coarse_pad * 128;
+  const uint32_t cv = ck + g.coarse_pad * D * 2;
   const int cta_first = blockIdx.x * nwarps * kUnitBlocks;
   if (g.L >= 2) {  // the CTA's 16 blocks share one ancestor per level (n_1 % 16 == 0 here)
     const int bh0 = cta_first / n1;
     const int p0 = cta_first - bh0 * n1;
-    stage_coarse_rows(g, k_pyr, idx, bh0, p0, ck, threadIdx.x, blockDim.x);
-    stage_coarse_rows(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
+    stage_coarse_rows<D>(g, k_pyr, idx, bh0, p0, ck, threadIdx.x, blockDim.x);
+    stage_coarse_rows<D>(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
     __syncthreads();
   }
   pdl_wait();
@@ -293,7 +386,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   if (first >= total_blocks) return;  // warp-uniform; no CTA-wide barrier after this point
   const int nblk = min(kUnitBlocks, total_blocks - first);
   const uint32_t sq = smem_u32(cs.tiles(base, warp));
-  const uint32_t ring = sq + 2 * kTileBytes;
+  constexpr int TB = tile_bytes<D>();
+  const uint32_t ring = sq + 2 * TB;
   int* srow = reinterpret_cast<int*>(cs.tail(base, warp));
   const uint32_t bar_q = smem_u32(srow) + ((kUnitBlocks * K * 4 + 15) & ~15);
   const uint32_t bar_kv = bar_q + 16;
@@ -313,15 +407,15 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     const int row = srow[seq];
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
-    const uint32_t dst = ring + stage * 2 * kTileBytes;
-    mbar_expect_tx(bar, 2 * kTileBytes);
-    tma_load_2d(dst, &tm_k, 0, row, bar);
-    tma_load_2d(dst + kTileBytes, &tm_v, 0, row, bar);
+    const uint32_t dst = ring + stage * 2 * TB;
+    mbar_expect_tx(bar, 2 * TB);
+    tma_load_tile<D>(dst, &tm_k, g, row, bar);
+    tma_load_tile<D>(dst + TB, &tm_v, g, row, bar);
   };
   auto issue_q = [&](int i) {
     const uint32_t bar = bar_q + 8 * (i & 1);
-    mbar_expect_tx(bar, kTileBytes);
-    tma_load_2d(sq + (i & 1) * kTileBytes, &tm_q, 0, (first + i) * kBlock, bar);
+    mbar_expect_tx(bar, TB);
+    tma_load_tile<D>(sq + (i & 1) * TB, &tm_q, g, (first + i) * kBlock, bar);
   };
   if (lane == 0) {
     issue_q(0);
@@ -333,19 +427,22 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   int next_q = 0;    // first Q load not yet consumed
   for (int i = 0; i < nblk && ok; ++i) {
     const int gb = first + i;
+    const int bh_i = div_n1(g, gb);
+    // real queries of this block (16 unless the sequence is padded)
+    const int qvalid = PAD ? g.nv - (gb - bh_i * n1) * kBlock : kBlock;
     ok = __all_sync(0xffffffffu, mbar_wait(bar_q + 8 * (i & 1), (i >> 1) & 1));
     if (!ok) break;
     next_q = i + 1;
-    uint32_t qf[4][4];
-    load_a_frags(sq + (i & 1) * kTileBytes, qf);
+    uint32_t qf[D / 16][4];
+    load_a_frags<D>(sq + (i & 1) * TB, qf);
     __syncwarp();
     if (lane == 0 && i + 1 < nblk) issue_q(i + 1);
 
     float m[2] = {-INFINITY, -INFINITY};
     float l[2] = {0.f, 0.f};
-    float acc[8][4];
+    float acc[D / 8][4];
 #pragma unroll
-    for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 
 #pragma unroll kQmUnroll
     for (int s = 0; s < K; ++s) {
@@ -354,25 +451,30 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
       ok = __all_sync(0xffffffffu, mbar_wait(bar_kv + 8 * stage, (seq / STAGES) & 1));
       if (!ok) break;
       next_seq = seq + 1;
-      const uint32_t kt = ring + stage * 2 * kTileBytes;
-      fwd_chunk<false, POOL>(qf, kt, kt + kTileBytes, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias(g));
+      const uint32_t kt = ring + stage * 2 * TB;
+      if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
+        fwd_chunk<D, true>(qf, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - bh_i * g.N)), P.scale_log2, m, l, acc);
+      else
+        fwd_chunk<D, false, POOL>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias<D>(g));
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
-      fwd_chunk<true>(qf, ck + cc * kTileBytes, cv + cc * kTileBytes, min(kBlock, g.coarse - cc * kBlock),
+      fwd_chunk<D, true>(qf, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock),
                       P.scale_log2, m, l, acc, &g, cc * kBlock);
 
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 1);
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 2);
     l[1] += __shfl_xor_sync(0xffffffffu, l[1], 1);
     l[1] += __shfl_xor_sync(0xffffffffu, l[1], 2);
-    store_tile_bf16(acc, 1.0f / l[0], 1.0f / l[1], sq + (i & 1) * kTileBytes, o + (long long)gb * kBlock * kD);
+    const int r0 = lane >> 2;
+    const bool real0 = !PAD || r0 < qvalid, real1 = !PAD || r0 + 8 < qvalid;
+    store_tile_bf16<D>(acc, real0 ? 1.0f / l[0] : 0.0f, real1 ? 1.0f / l[1] : 0.0f, sq + (i & 1) * TB,
+                       o + (long long)gb * kBlock * D);
     if ((lane & 3) == 0) {
-      const int r0 = lane >> 2;
-      lse[(long long)gb * kBlock + r0] = (m[0] + log2f(l[0])) * kLn2;
-      lse[(long long)gb * kBlock + r0 + 8] = (m[1] + log2f(l[1])) * kLn2;
+      lse[(long long)gb * kBlock + r0] = real0 ? (m[0] + log2f(l[0])) * kLn2 : 0.0f;
+      lse[(long long)gb * kBlock + r0 + 8] = real1 ? (m[1] + log2f(l[1])) * kLn2 : 0.0f;
     }
   }
   if (!ok) {

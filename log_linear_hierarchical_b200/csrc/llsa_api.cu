@@ -7,10 +7,9 @@
 #include <new>
 
 #include "attn_simt.cuh"
-#if LLSA_KEY_MAJOR_TC
-#include "attn_bwd_tc.cuh"
-#endif
+#include "probe.cuh"
 #include "pyramid.cuh"
+#include "pyramid_select.cuh"
 #include "select.cuh"
 #include "transpose.cuh"
 #include "zorder.cuh"
@@ -41,10 +40,11 @@ llsa_status validate(const llsa_shape* s) {
   if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
   if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP | LLSA_FLAG_LEVEL1))
     return LLSA_ERR_INVALID_ARG;  // unknown flag bits
+  if (s->n_valid < 0 || s->n_valid > s->N) return LLSA_ERR_INVALID_ARG;
   // N: any multiple of 16^L (the pages' implementation wants powers of two for N and topk;
   // the kernels here take any multiple and any topk)
   if (s->block != kBlock) return LLSA_ERR_UNSUPPORTED;
-  if (s->D != kD) return LLSA_ERR_UNSUPPORTED;
+  if (s->D != 64 && s->D != 128) return LLSA_ERR_UNSUPPORTED;
   if (s->levels > kMaxLevels) return LLSA_ERR_UNSUPPORTED;
   if (s->N % (1LL << (4 * s->levels)) != 0) return LLSA_ERR_INVALID_ARG;  // n_L = N / 16^L whole
   const long long nL = (long long)s->N >> (4 * s->levels);
@@ -56,6 +56,11 @@ llsa_status validate(const llsa_shape* s) {
   if ((s->flags & LLSA_FLAG_ALL_TOP) && s->levels >= 2 && (long long)(s->levels - 2) * s->topk + nL > 96)
     return LLSA_ERR_UNSUPPORTED;  // the coarse entries of the all-coarsest variant
   if ((long long)s->B * s->H * s->N >= (1LL << 31)) return LLSA_ERR_UNSUPPORTED;
+  if (s->n_valid != 0 && s->n_valid < s->N) {  // a padded sequence
+    const long long span = 1LL << (4 * s->levels);
+    if (s->topk > (s->n_valid + span - 1) / span) return LLSA_ERR_INVALID_ARG;  // K real coarsest tokens
+    if (s->flags != 0) return LLSA_ERR_UNSUPPORTED;  // padding takes the default enrichment only
+  }
   return LLSA_OK;
 }
 
@@ -74,18 +79,21 @@ Geometry make_geometry(const llsa_shape* s) {
     g.pyr_off[l] = po;
     g.idx_off[l] = io;
     g.rp_off[l] = ro;
-    po += (long long)g.BH * g.n[l] * kD;
+    po += (long long)g.BH * g.n[l] * s->D;
     io += (long long)g.BH * g.n[l] * g.K;
     ro += (long long)g.BH * (g.n[l] + 1);
   }
   g.log_k = is_pow2(g.K) ? ilog2(g.K) : -1;
   g.log_n1 = is_pow2(g.n[1]) ? ilog2(g.n[1]) : -1;
+  g.log_n = is_pow2(g.N) ? ilog2(g.N) : -1;
   const bool all_top = (s->flags & LLSA_FLAG_ALL_TOP) && g.L >= 2;
   g.coarse = all_top ? (g.L - 2) * g.K + g.n[g.L] : (g.L - 1) * g.K;
   g.coarse_pad = (g.coarse + kBlock - 1) / kBlock * kBlock;
   g.log_bias = (s->flags & LLSA_FLAG_LOG_BIAS) ? 1 : 0;
   g.top_first = all_top ? (g.L - 2) * g.K : g.coarse;
   g.pool1 = (s->flags & LLSA_FLAG_LEVEL1) ? 1 : 0;
+  g.nv = (s->n_valid > 0 && s->n_valid < s->N) ? s->n_valid : s->N;
+  for (int l = 0; l <= kMaxLevels; ++l) g.m[l] = l <= g.L ? (int)((g.nv + (1LL << (4 * l)) - 1) >> (4 * l)) : 0;
   return g;
 }
 
@@ -107,12 +115,13 @@ TransposeGeo make_transpose_geo(const Geometry& g, long long* ent_total, long lo
     L.wshift = ilog2(w);
     L.cta_tiles = cta_t;
     L.cta_buckets = cta_b;
+    L.hstride = L.nb * L.tiles + 1;
     L.hist_off = hist;
     L.ent_off = g.idx_off[l];
     L.rp_off = g.rp_off[l];
     cta_t += g.BH * L.tiles;
     cta_b += g.BH * L.nb;
-    hist += (long long)g.BH * L.nb * L.tiles;
+    hist += (long long)g.BH * L.hstride;
   }
   *ent_total = (long long)g.BH * g.K * [&] {
     long long s = 0;
@@ -143,13 +152,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows, 64] bf16 row-major viewed as 2-D; box = 16 rows x 64 channels, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* m, const void* base, long long rows) {
+// q, k, v, dO as [B*H][n_valid][D] bf16 (row stride D, head stride N * D); box = 64
+// channels (128 bytes, the swizzle span) x 16 rows x 1 head, so a 16-token tile is D / 64
+// boxes at x = 0, 64.  Rows at or past n_valid (padding) are read as zeros.
+bool make_tile_map(CUtensorMap* m, const void* base, const Geometry& g) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)kBlock};
+  cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.nv, (cuuint64_t)g.BH};
+  cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.N * g.D * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)kBlock, 1u};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, 64] bf16 viewed as 2-D, box 64 x 16 with 128-byte swizzle (the gather probe).
+bool make_probe_map(CUtensorMap* m, const void* base, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {64u, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128u};
+  cuuint32_t box[2] = {64u, (cuuint32_t)kBlock};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -212,19 +236,23 @@ enum KernelId {
   kKBwdDqF32,
   kKBwdDkdvF32,
   kKBwdCoarseBf16,
-  kKBwdDkdvTc,
-  kKBwdDkdvEmpty,
   kKDkdvOrderCount,
   kKDkdvOrderScatter,
   kKZOrder,
+  kKTransposeScan,
+  kKWaitCheck,
+  kKGatherProbe,
+  kKPyramidSelect,
   kKNumKernels
 };
 
 const char* const kKernelNames[kKNumKernels] = {
-    "unknown",          "pyramid_l12",          "pyramid_up",   "select",           "transpose_hist",
-    "transpose_scatter", "transpose_bucket",    "attn_fwd_bf16", "attn_bwd_dq_bf16", "coarse_grad_reduce",
-    "attn_bwd_dkdv_bf16", "attn_fwd_f32",      "attn_bwd_dq_f32", "attn_bwd_dkdv_f32", "attn_bwd_coarse_bf16", "attn_bwd_dkdv_tc", "dkdv_empty_rows",
-    "dkdv_order_count", "dkdv_order_scatter", "zorder_permute"};
+    "unknown",           "pyramid_l12",        "pyramid_up",       "select",
+    "transpose_hist",    "transpose_scatter",  "transpose_bucket", "attn_fwd_bf16",
+    "attn_bwd_dq_bf16",  "coarse_grad_reduce", "attn_bwd_dkdv_bf16", "attn_fwd_f32",
+    "attn_bwd_dq_f32",   "attn_bwd_dkdv_f32",  "attn_bwd_coarse_bf16", "dkdv_order_count",
+    "dkdv_order_scatter", "zorder_permute",    "transpose_scan",   "bounded_wait_check",
+    "gather_probe",      "pyramid_select"};
 
 struct TraceState {
   cudaEvent_t* ev = nullptr;
@@ -264,13 +292,14 @@ constexpr int kDqStages = LLSA_DQ_STAGES;
 constexpr int kDkvStages = LLSA_KV_STAGES;
 constexpr int kAttnWarps = 4;
 
+template <int D>
 llsa_status launch_coarse_reduce(const Geometry& g, float scale, const int32_t* idx, const int32_t* row_ptr,
                                  const int32_t* col, float* ws, cudaStream_t cs) {
   if (g.L < 2) return LLSA_OK;
   long long tokens = 0;
   for (int l = 2; l <= g.L; ++l) tokens += (long long)g.BH * g.n[l];
   return launch(kKBwdCoarseReduce, cs, [&] {
-    launch_pdl(coarse_grad_reduce_kernel, dim3((unsigned)tokens), dim3(kReduceWarps * 32), 0, cs, g, scale, idx, row_ptr, col, ws);
+    launch_pdl(coarse_grad_reduce_kernel<D>, dim3((unsigned)tokens), dim3(kReduceWarps * 32), 0, cs, g, scale, idx, row_ptr, col, ws);
   });
 }
 
@@ -306,16 +335,17 @@ namespace {
 // level-1 CSR and can run beside the query side too.
 constexpr unsigned kQuerySide = 1, kKeySide = 2, kOrder = 4;
 
-llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
-                            const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
-                            const int32_t* idx, const int32_t* row_ptr, const int32_t* col, void* dq, void* dk,
-                            void* dv, void* workspace, unsigned phases, cudaStream_t cs) {
+template <int D>
+llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
+                              const int32_t* idx, const int32_t* row_ptr, const int32_t* col, void* dq, void* dk,
+                              void* dv, void* workspace, unsigned phases, cudaStream_t cs) {
   llsa_status st = LLSA_OK;
   const Geometry g = make_geometry(s);
   float* ws = static_cast<float*>(workspace);
-  const float scale = 1.0f / sqrtf((float)kD);
+  const float scale = 1.0f / sqrtf((float)D);
   const int total_blocks = g.BH * g.n[1];
-  if ((phases & kOrder) && s->dtype == LLSA_BF16 && !LLSA_KEY_MAJOR_TC) {
+  if ((phases & kOrder) && s->dtype == LLSA_BF16) {
     const int tiles = order_tiles(g);
     st = launch(kKDkdvOrderCount, cs,
                 [&] { launch_pdl(dkdv_order_count_kernel, dim3(tiles), dim3(kOrdThreads), 0, cs, g, row_ptr, ws); });
@@ -326,15 +356,16 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
   }
   if (s->dtype == LLSA_BF16) {
     CUtensorMap tq, tk, tv, tdo;
-    const long long rows = (long long)g.BH * g.N;
-    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
-        !make_tile_map(&tdo, dO, rows))
+    if (!make_tile_map(&tq, q, g) || !make_tile_map(&tk, k, g) || !make_tile_map(&tv, v, g) ||
+        !make_tile_map(&tdo, dO, g))
       return LLSA_ERR_CUDA;
     AttnParams P{g, scale * kLog2e, scale};
-    const size_t kv_bytes = (size_t)kv_smem<kDkvStages>(1).total();
+    const size_t kv_bytes = (size_t)kv_smem<D, kDkvStages>(1).total();
     if (phases & kQuerySide) {
-      const size_t smem = (size_t)dq_smem<kDqStages>(g, kAttnWarps).total();
-      auto kern = g.pool1 ? attn_bwd_dq_bf16_kernel<kDqStages, true> : attn_bwd_dq_bf16_kernel<kDqStages, false>;
+      const size_t smem = (size_t)dq_smem<D, kDqStages>(g, kAttnWarps).total();
+      auto kern = g.nv < g.N ? attn_bwd_dq_bf16_kernel<D, kDqStages, false, true>
+                  : g.pool1  ? attn_bwd_dq_bf16_kernel<D, kDqStages, true, false>
+                             : attn_bwd_dq_bf16_kernel<D, kDqStages, false, false>;
       if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
       const int per_cta = kAttnWarps * kUnitBlocks;
       st = launch(kKBwdDqBf16, cs, [&] {
@@ -344,7 +375,7 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
       });
       if (st != LLSA_OK) return st;
       if (g.L >= 2) {
-        auto ckern = attn_bwd_coarse_bf16_kernel<kDkvStages>;
+        auto ckern = attn_bwd_coarse_bf16_kernel<D, kDkvStages>;
         if (!allow_smem(ckern, kv_bytes)) return LLSA_ERR_CUDA;
         const int ctas = g.BH * g.n[2] * (g.coarse_pad / kBlock);
         st = launch(kKBwdCoarseBf16, cs, [&] {
@@ -354,28 +385,8 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
       }
     }
     if (!(phases & kKeySide)) return LLSA_OK;
-    if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
-#if LLSA_KEY_MAJOR_TC
-    if (g.pool1 || g.log_n1 < 0) return LLSA_ERR_UNSUPPORTED;  // the tcgen05 kernel: no level-1 fold, n_1 = 2^m
-    {
-      int dev = 0, sms = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return LLSA_ERR_CUDA;
-      if (!allow_smem(attn_bwd_dkdv_tc_kernel, kTcSmemBytes)) return LLSA_ERR_CUDA;
-      const int grid = total_blocks < 2 * sms ? total_blocks : 2 * sms;
-      st = launch(kKBwdDkdvEmpty, cs, [&] {
-        launch_pdl(dkdv_empty_rows_kernel, dim3((total_blocks + 3) / 4), dim3(128), 0, cs, P, row_ptr, ws, static_cast<__nv_bfloat16*>(dk),
-                                                                      static_cast<__nv_bfloat16*>(dv));
-      });
-      if (st != LLSA_OK) return st;
-      return launch(kKBwdDkdvTc, cs, [&] {
-        launch_pdl(attn_bwd_dkdv_tc_kernel, dim3(grid), dim3(kTcThreads), kTcSmemBytes, cs, 
-            tq, tk, tv, tdo, P, lse, row_ptr, col, ws, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
-      });
-    }
-#endif
-    auto kern = g.pool1 ? attn_bwd_dkdv_bf16_kernel<kDkvStages, true> : attn_bwd_dkdv_bf16_kernel<kDkvStages, false>;
+    if ((st = launch_coarse_reduce<D>(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
+    auto kern = g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, kDkvStages, true> : attn_bwd_dkdv_bf16_kernel<D, kDkvStages, false>;
     if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
     return launch(kKBwdDkdvBf16, cs, [&] {
       launch_pdl(kern, dim3(total_blocks), dim3(32), kv_bytes, cs, tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
@@ -383,11 +394,11 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
     });
   }
   if (phases & kQuerySide) {
-    const size_t smem = simt_dq_smem(g);
-    if (!allow_smem(attn_bwd_dq_f32_kernel, smem)) return LLSA_ERR_CUDA;
+    const size_t smem = simt_dq_smem<D>(g);
+    if (!allow_smem(attn_bwd_dq_f32_kernel<D>, smem)) return LLSA_ERR_CUDA;
     const int per_cta = g.L >= 2 ? kBlock : 1;
     st = launch(kKBwdDqF32, cs, [&] {
-      launch_pdl(attn_bwd_dq_f32_kernel, dim3(total_blocks / per_cta), dim3(kSimtThreads), smem, cs, 
+      launch_pdl(attn_bwd_dq_f32_kernel<D>, dim3(total_blocks / per_cta), dim3(kSimtThreads), smem, cs, 
           g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
           static_cast<const float*>(o), lse, static_cast<const float*>(dO), k_pyr, v_pyr, idx,
           static_cast<float*>(dq), ws);
@@ -395,50 +406,57 @@ llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, c
     if (st != LLSA_OK) return st;
   }
   if (!(phases & kKeySide)) return LLSA_OK;
-  if ((st = launch_coarse_reduce(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
+  if ((st = launch_coarse_reduce<D>(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
   return launch(kKBwdDkdvF32, cs, [&] {
-    launch_pdl(attn_bwd_dkdv_f32_kernel, dim3(total_blocks), dim3(kSimtThreads), 0, cs, 
+    launch_pdl(attn_bwd_dkdv_f32_kernel<D>, dim3(total_blocks), dim3(kSimtThreads), 0, cs, 
         g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
         v_pyr, lse, static_cast<const float*>(dO), row_ptr, col, ws, static_cast<float*>(dk),
         static_cast<float*>(dv));
   });
 }
 
+llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
+                            const int32_t* idx, const int32_t* row_ptr, const int32_t* col, void* dq, void* dk,
+                            void* dv, void* workspace, unsigned phases, cudaStream_t cs) {
+  auto f = s->D == 128 ? backward_phases_d<128> : backward_phases_d<64>;
+  return f(s, q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace, phases, cs);
+}
 
 // ---------------------------------------------------------------------------- pyramid, select
 // Levels 1-2 of the pyramid, and levels 3..L too when `upper`.
-llsa_status pyramid_launch(const Geometry& g, int dtype, const void* q, const void* k, const void* v, float* q_pyr,
-                           float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs) {
-  llsa_status st;
-  if (dtype == LLSA_BF16) {
-    constexpr int rows = kPyrThreads / (kD / 8);
-    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
-    constexpr int span = pyramid_span_bytes<__nv_bfloat16>();
-    if (!allow_smem(pyramid_l12_kernel<__nv_bfloat16>, span)) return LLSA_ERR_CUDA;
-    st = launch(kKPyramidL12, cs, [&] {
-      launch_pdl(pyramid_l12_kernel<__nv_bfloat16>, dim3(grid), dim3(kPyrThreads), span, cs, g,
-                 static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                 static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr);
-    });
-  } else {
-    constexpr int rows = kPyrThreads / (kD / 4);
-    dim3 grid(g.BH * ((g.n[1] + rows - 1) / rows), 3);
-    constexpr int span = pyramid_span_bytes<float>();
-    if (!allow_smem(pyramid_l12_kernel<float>, span)) return LLSA_ERR_CUDA;
-    st = launch(kKPyramidL12, cs, [&] {
-      launch_pdl(pyramid_l12_kernel<float>, dim3(grid), dim3(kPyrThreads), span, cs, g, static_cast<const float*>(q),
-                 static_cast<const float*>(k), static_cast<const float*>(v), q_pyr, k_pyr, v_pyr);
-    });
-  }
+template <typename T, int D>
+llsa_status pyramid_l12_launch(const Geometry& g, const void* q, const void* k, const void* v, float* q_pyr,
+                               float* k_pyr, float* v_pyr, cudaStream_t cs) {
+  using C = PyrCfg<T, D>;
+  dim3 grid(g.BH * ((g.n[1] + C::ROWS - 1) / C::ROWS), 3);
+  if (!allow_smem(pyramid_l12_kernel<T, D>, C::SPAN)) return LLSA_ERR_CUDA;
+  return launch(kKPyramidL12, cs, [&] {
+    launch_pdl(pyramid_l12_kernel<T, D>, dim3(grid), dim3(C::THREADS), C::SPAN, cs, g, static_cast<const T*>(q),
+               static_cast<const T*>(k), static_cast<const T*>(v), q_pyr, k_pyr, v_pyr);
+  });
+}
+
+template <int D>
+llsa_status pyramid_launch_d(const Geometry& g, int dtype, const void* q, const void* k, const void* v, float* q_pyr,
+                             float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs) {
+  llsa_status st = dtype == LLSA_BF16 ? pyramid_l12_launch<__nv_bfloat16, D>(g, q, k, v, q_pyr, k_pyr, v_pyr, cs)
+                                      : pyramid_l12_launch<float, D>(g, q, k, v, q_pyr, k_pyr, v_pyr, cs);
   if (st != LLSA_OK || !upper) return st;
   for (int l = 3; l <= g.L; ++l) {
-    const long long total = (long long)g.BH * g.n[l] * kD;
+    const long long total = (long long)g.BH * g.n[l] * D;
     dim3 grid((unsigned)((total + kPyrThreads - 1) / kPyrThreads), 3);
     st = launch(kKPyramidUp, cs,
-                [&] { launch_pdl(pyramid_up_kernel, dim3(grid), dim3(kPyrThreads), 0, cs, g, l, q_pyr, k_pyr, v_pyr); });
+                [&] { launch_pdl(pyramid_up_kernel<D>, dim3(grid), dim3(kPyrThreads), 0, cs, g, l, q_pyr, k_pyr, v_pyr); });
     if (st != LLSA_OK) return st;
   }
   return LLSA_OK;
+}
+
+llsa_status pyramid_launch(const Geometry& g, int dtype, const void* q, const void* k, const void* v, float* q_pyr,
+                           float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs) {
+  auto f = g.D == 128 ? pyramid_launch_d<128> : pyramid_launch_d<64>;
+  return f(g, dtype, q, k, v, q_pyr, k_pyr, v_pyr, upper, cs);
 }
 
 // The pooled levels 3..L and the coarsest selection fit one small kernel per (b, h).
@@ -447,18 +465,19 @@ bool small_top(const Geometry& g) { return g.n[g.L] <= kTopMaxN && g.K <= 32 && 
 // Selection of every level, coarsest first.  With `pool_top` (only when small_top), the
 // coarsest launch also pools levels 3..L (pyramid_launch was made with upper = false);
 // v_pyr is needed only then.
-llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* v_pyr, int32_t* idx, bool pool_top,
-                          cudaStream_t cs) {
+template <int D>
+llsa_status select_launch_d(const Geometry& g, float* q_pyr, float* k_pyr, float* v_pyr, int32_t* idx, bool pool_top,
+                            cudaStream_t cs) {
   llsa_status st;
   for (int l = g.L; l >= 1; --l) {
     const bool sparse = l < g.L;
     const int n = g.n[l];
     if (!sparse && small_top(g)) {
+      auto kern = pool_top ? coarsest_small_kernel<D, true> : coarsest_small_kernel<D, false>;
+      constexpr int smem = coarsest_small_smem<D>();
+      if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
       st = launch(kKSelect, cs, [&] {
-        if (pool_top)
-          launch_pdl(coarsest_small_kernel<true>, dim3(g.BH), dim3(kTopThreads), 0, cs, g, q_pyr, k_pyr, v_pyr, idx);
-        else
-          launch_pdl(coarsest_small_kernel<false>, dim3(g.BH), dim3(kTopThreads), 0, cs, g, q_pyr, k_pyr, v_pyr, idx);
+        launch_pdl(kern, dim3(g.BH), dim3(kTopThreads), smem, cs, g, q_pyr, k_pyr, v_pyr, idx);
       });
       if (st != LLSA_OK) return st;
       continue;
@@ -474,7 +493,7 @@ llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* 
     }
     if (sparse && (g.K == 2 || g.K == 4 || g.K == 8 || g.K == 16)) {
       // children of the parent's K keys scored in registers (select_children_kernel)
-      const size_t smem = select_children_smem_bytes(nc);
+      const size_t smem = select_children_smem_bytes<D>(nc);
       const float* qpl = q_pyr + g.pyr_off[l];
       const float* kpl = k_pyr + g.pyr_off[l];
       const int* par = idx + g.idx_off[l + 1];
@@ -485,24 +504,79 @@ llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* 
         return launch(kKSelect, cs, [&] { launch_pdl(kern, dim3(grid), dim3(kSelThreads), smem, cs, g, l, qpl, kpl, par, out); });
       };
       switch (g.K) {
-        case 2: st = run(select_children_kernel<1>); break;
-        case 4: st = run(select_children_kernel<2>); break;
-        case 8: st = run(select_children_kernel<4>); break;
-        default: st = run(select_children_kernel<8>); break;
+        case 2: st = run(select_children_kernel<D, 1>); break;
+        case 4: st = run(select_children_kernel<D, 2>); break;
+        case 8: st = run(select_children_kernel<D, 4>); break;
+        default: st = run(select_children_kernel<D, 8>); break;
       }
       if (st != LLSA_OK) return st;
       continue;
     }
-    const size_t smem = select_smem_bytes(gq, nc, g.K, sparse);
-    if (!allow_smem(select_kernel, smem)) return LLSA_ERR_CUDA;
+    const size_t smem = select_smem_bytes<D>(gq, nc, g.K, sparse);
+    if (!allow_smem(select_kernel<D>, smem)) return LLSA_ERR_CUDA;
     const int groups = (n + gq - 1) / gq;
     st = launch(kKSelect, cs, [&] {
-      launch_pdl(select_kernel, dim3(g.BH * groups), dim3(kSelThreads), smem, cs, g, l, gq, q_pyr + g.pyr_off[l],
+      launch_pdl(select_kernel<D>, dim3(g.BH * groups), dim3(kSelThreads), smem, cs, g, l, gq, q_pyr + g.pyr_off[l],
                  k_pyr + g.pyr_off[l], sparse ? idx + g.idx_off[l + 1] : nullptr, idx + g.idx_off[l]);
     });
     if (st != LLSA_OK) return st;
   }
   return LLSA_OK;
+}
+
+llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* v_pyr, int32_t* idx, bool pool_top,
+                          cudaStream_t cs) {
+  auto f = g.D == 128 ? select_launch_d<128> : select_launch_d<64>;
+  return f(g, q_pyr, k_pyr, v_pyr, idx, pool_top, cs);
+}
+
+// The pyramid and every selection level in one cooperative launch (pyramid_select_kernel):
+// bf16, L >= 2, a small coarsest level and K in {2, 4, 8, 16} (the register-resident
+// children selection).
+bool fused_pyramid_select(const Geometry& g, int dtype) {
+  return dtype == LLSA_BF16 && g.L >= 2 && small_top(g) && (g.K == 2 || g.K == 4 || g.K == 8 || g.K == 16);
+}
+
+template <int D, int CPT>
+llsa_status pyramid_select_launch_k(const Geometry& g, const void* q, const void* k, const void* v, float* q_pyr,
+                                    float* k_pyr, float* v_pyr, int32_t* idx, unsigned* barrier, cudaStream_t cs) {
+  auto kern = pyramid_select_kernel<D, CPT>;
+  constexpr int smem = pyramid_select_smem<D, CPT>();
+  if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSelThreads, smem) != cudaSuccess || per_sm < 1)
+    return LLSA_ERR_CUDA;
+  // no more CTAs than the largest phase has units
+  long long units = 3LL * g.BH * ((g.n[1] + PyrCfg<__nv_bfloat16, D>::ROWS - 1) / PyrCfg<__nv_bfloat16, D>::ROWS);
+  for (int l = 1; l < g.L; ++l) units = units > (long long)g.BH * (g.n[l] / kBlock) ? units : (long long)g.BH * (g.n[l] / kBlock);
+  const int grid = (int)((long long)sms * per_sm < units ? (long long)sms * per_sm : units);
+  if (cudaMemsetAsync(barrier, 0, 16 * sizeof(unsigned), cs) != cudaSuccess) return LLSA_ERR_CUDA;
+  return launch(kKPyramidSelect, cs, [&] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barriers complete
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                       static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr, idx, barrier);
+  });
+}
+
+template <int D>
+llsa_status pyramid_select_launch_d(const Geometry& g, const void* q, const void* k, const void* v, float* q_pyr,
+                                    float* k_pyr, float* v_pyr, int32_t* idx, unsigned* barrier, cudaStream_t cs) {
+  switch (g.K) {
+    case 2: return pyramid_select_launch_k<D, 1>(g, q, k, v, q_pyr, k_pyr, v_pyr, idx, barrier, cs);
+    case 4: return pyramid_select_launch_k<D, 2>(g, q, k, v, q_pyr, k_pyr, v_pyr, idx, barrier, cs);
+    case 8: return pyramid_select_launch_k<D, 4>(g, q, k, v, q_pyr, k_pyr, v_pyr, idx, barrier, cs);
+    default: return pyramid_select_launch_k<D, 8>(g, q, k, v, q_pyr, k_pyr, v_pyr, idx, barrier, cs);
+  }
 }
 
 // ---------------------------------------------------------------------------- one step
@@ -527,6 +601,36 @@ llsa_status validate_step(const llsa_shape* s, const llsa_step_buffers* b) {
 // (forked after the selection, joined before the backward key side), or on `cs` if side
 // is null.  The join is made on every path once the fork was made, so a capture that
 // fails part-way still ends with both streams joined.
+template <int D>
+llsa_status forward_launch(const Geometry& g, int dtype, const void* q, const void* k, const void* v,
+                           const float* k_pyr, const float* v_pyr, const int32_t* idx, void* o, float* lse,
+                           cudaStream_t cs) {
+  const float scale = 1.0f / sqrtf((float)D);
+  const int total_blocks = g.BH * g.n[1];
+  if (dtype == LLSA_BF16) {
+    CUtensorMap tq, tk, tv;
+    if (!make_tile_map(&tq, q, g) || !make_tile_map(&tk, k, g) || !make_tile_map(&tv, v, g)) return LLSA_ERR_CUDA;
+    AttnParams P{g, scale * kLog2e, scale};
+    const size_t smem = (size_t)fwd_smem<D, kFwdStages>(g, kAttnWarps).total();
+    auto kern = g.nv < g.N ? attn_fwd_bf16_kernel<D, kFwdStages, false, true>
+                : g.pool1  ? attn_fwd_bf16_kernel<D, kFwdStages, true, false>
+                           : attn_fwd_bf16_kernel<D, kFwdStages, false, false>;
+    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+    const int per_cta = kAttnWarps * kUnitBlocks;
+    return launch(kKFwdBf16, cs, [&] {
+      launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, tq, tk, tv, P,
+                 k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse);
+    });
+  }
+  const size_t smem = simt_fwd_smem<D>(g);
+  if (!allow_smem(attn_fwd_f32_kernel<D>, smem)) return LLSA_ERR_CUDA;
+  return launch(kKFwdF32, cs, [&] {
+    launch_pdl(attn_fwd_f32_kernel<D>, dim3(total_blocks), dim3(kSimtThreads), smem, cs, g, scale,
+               static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
+               v_pyr, idx, static_cast<float*>(o), lse);
+  });
+}
+
 // The forward launch shared by llsa_forward and the step.
 llsa_status forward_impl(const llsa_shape* s, const void* q, const void* k, const void* v, const float* k_pyr,
                          const float* v_pyr, const int32_t* idx, void* o, float* lse, llsa_stream_t stream) {
@@ -537,38 +641,25 @@ llsa_status forward_impl(const llsa_shape* s, const void* q, const void* k, cons
     if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
   const Geometry g = make_geometry(s);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const float scale = 1.0f / sqrtf((float)kD);
-  const int total_blocks = g.BH * g.n[1];
-  if (s->dtype == LLSA_BF16) {
-    CUtensorMap tq, tk, tv;
-    const long long rows = (long long)g.BH * g.N;
-    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
-      return LLSA_ERR_CUDA;
-    AttnParams P{g, scale * kLog2e, scale};
-    const size_t smem = (size_t)fwd_smem<kFwdStages>(g, kAttnWarps).total();
-    auto kern = g.pool1 ? attn_fwd_bf16_kernel<kFwdStages, true> : attn_fwd_bf16_kernel<kFwdStages, false>;
-    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
-    const int per_cta = kAttnWarps * kUnitBlocks;
-    return launch(kKFwdBf16, cs, [&] {
-      launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, 
-          tq, tk, tv, P, k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse);
-    });
-  }
-  const size_t smem = simt_fwd_smem(g);
-  if (!allow_smem(attn_fwd_f32_kernel, smem)) return LLSA_ERR_CUDA;
-  return launch(kKFwdF32, cs, [&] {
-    launch_pdl(attn_fwd_f32_kernel, dim3(total_blocks), dim3(kSimtThreads), smem, cs, 
-        g, scale, static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), k_pyr,
-        v_pyr, idx, static_cast<float*>(o), lse);
-  });
+  auto f = g.D == 128 ? forward_launch<128> : forward_launch<64>;
+  return f(g, s->dtype, q, k, v, k_pyr, v_pyr, idx, o, lse, cs);
 }
 
 llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStream_t cs, cudaStream_t side) {
-  // pooled levels >= 3 are made by the coarsest-selection launch when they are small
   const Geometry g = make_geometry(s);
-  const bool fuse_top = g.L >= 3 && small_top(g);
-  llsa_status st = pyramid_launch(g, s->dtype, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, !fuse_top, cs);
-  if (st == LLSA_OK) st = select_launch(g, b->q_pyr, b->k_pyr, b->v_pyr, b->idx, fuse_top, cs);
+  llsa_status st;
+  const bool fused = fused_pyramid_select(g, s->dtype);
+  if (fused) {  // pyramid and selection in one cooperative launch
+    unsigned* barrier =
+        reinterpret_cast<unsigned*>(static_cast<float*>(b->backward_workspace) + bwd_workspace_layout(g).barrier);
+    auto f = g.D == 128 ? pyramid_select_launch_d<128> : pyramid_select_launch_d<64>;
+    st = f(g, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, b->idx, barrier, cs);
+  } else {
+    // pooled levels >= 3 are made by the coarsest-selection launch when they are small
+    const bool fuse_top = g.L >= 3 && small_top(g);
+    st = pyramid_launch(g, s->dtype, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, !fuse_top, cs);
+    if (st == LLSA_OK) st = select_launch(g, b->q_pyr, b->k_pyr, b->v_pyr, b->idx, fuse_top, cs);
+  }
   if (st != LLSA_OK) return st;
   cudaEvent_t fork = nullptr, join = nullptr;
   if (side) {
@@ -587,7 +678,12 @@ llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStrea
                            b->dq, b->dk, b->dv, b->backward_workspace, kOrder, side);
     if (cudaEventRecord(join, side) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
   }
-  if (st == LLSA_OK) st = forward_impl(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs);
+  if (st == LLSA_OK) {
+    // after the fused launch the forward's early reads (coarse rows and selections) would
+    // be of the kernel right ahead of it, so it starts only once that kernel is complete
+    if (fused) g_serial_next = true;
+    st = forward_impl(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs);
+  }
   if (st == LLSA_OK)
     st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
                          b->dq, b->dk, b->dv, b->backward_workspace, kQuerySide, cs);
@@ -634,7 +730,7 @@ llsa_status llsa_validate_shape(const llsa_shape* shape) { return validate(shape
 size_t llsa_pyramid_elems(const llsa_shape* s) {
   if (validate(s) != LLSA_OK) return 0;
   const Geometry g = make_geometry(s);
-  return (size_t)(g.pyr_off[g.L] + (long long)g.BH * g.n[g.L] * kD);
+  return (size_t)(g.pyr_off[g.L] + (long long)g.BH * g.n[g.L] * g.D);
 }
 
 size_t llsa_index_elems(const llsa_shape* s) {
@@ -700,11 +796,21 @@ llsa_status llsa_index_transpose(const llsa_shape* s, const int32_t* idx, int32_
   st = launch(kKTransposeHist, cs,
               [&] { launch_pdl(transpose_hist_kernel, dim3(tile_ctas), dim3(kTrThreads), 0, cs, tg, idx, ws_hist); });
   if (st != LLSA_OK) return st;
+  int max_tiles = 0;
+  for (int l = 0; l < g.L; ++l) max_tiles = tg.lv[l].tiles > max_tiles ? tg.lv[l].tiles : max_tiles;
+  const bool scanned = max_tiles > kTrScanTiles;
+  if (scanned) {
+    st = launch(kKTransposeScan, cs,
+                [&] { launch_pdl(transpose_scan_kernel, dim3(g.L * g.BH), dim3(kTrThreads), 0, cs, tg, ws_hist); });
+    if (st != LLSA_OK) return st;
+  }
+  auto scatter = scanned ? transpose_scatter_kernel<true> : transpose_scatter_kernel<false>;
+  auto bucket = scanned ? transpose_bucket_kernel<true> : transpose_bucket_kernel<false>;
   st = launch(kKTransposeScatter, cs,
-              [&] { launch_pdl(transpose_scatter_kernel, dim3(tile_ctas), dim3(kTrThreads), 0, cs, tg, idx, ws_hist, ws_ent); });
+              [&] { launch_pdl(scatter, dim3(tile_ctas), dim3(kTrThreads), 0, cs, tg, idx, ws_hist, ws_ent); });
   if (st != LLSA_OK) return st;
   return launch(kKTransposeBucket, cs, [&] {
-    launch_pdl(transpose_bucket_kernel, dim3(bucket_ctas), dim3(kTrThreads), 0, cs, tg, ws_ent, ws_hist, row_ptr, col);
+    launch_pdl(bucket, dim3(bucket_ctas), dim3(kTrThreads), 0, cs, tg, ws_ent, ws_hist, row_ptr, col);
   });
 }
 
@@ -805,7 +911,7 @@ llsa_status llsa_token_permute(const llsa_shape* s, const void* src, void* dst, 
   const int lg = ilog2(s->N);
   if (lg & 1) return LLSA_ERR_INVALID_ARG;  // N must be a square grid: side = 2^(lg/2)
   const long long rows = (long long)s->B * s->H * s->N;
-  const int row_bytes = kD * (s->dtype == LLSA_BF16 ? 2 : 4);
+  const int row_bytes = s->D * (s->dtype == LLSA_BF16 ? 2 : 4);
   const int pieces = row_bytes / 16;
   const long long threads = rows * pieces;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -826,6 +932,32 @@ llsa_status llsa_device_status(int32_t* code_out, llsa_stream_t stream) {
   if (cudaMemcpyToSymbol(g_llsa_status, &zero, sizeof(int)) != cudaSuccess) return LLSA_ERR_CUDA;
   *code_out = v;
   return LLSA_OK;
+}
+
+llsa_status llsa_check_bounded_wait(int64_t limit_cycles, llsa_stream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > kWaitLimitCycles) return LLSA_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  return launch(kKWaitCheck, cs, [&] { bounded_wait_check_kernel<<<1, 32, 0, cs>>>((long long)limit_cycles); });
+}
+
+llsa_status llsa_gather_probe(const void* src, int64_t rows, const int32_t* tile_rows, int32_t ntiles,
+                              int32_t stages, int32_t ctas, llsa_stream_t stream) {
+  if (!src || !tile_rows || !aligned16(src) || !aligned16(tile_rows)) return LLSA_ERR_INVALID_ARG;
+  if (rows < kBlock || rows % kBlock != 0 || rows >= (1LL << 31) || ntiles < 1 || ctas < 1 || ctas > 65535)
+    return LLSA_ERR_INVALID_ARG;
+  if (stages != 2 && stages != 4 && stages != 8) return LLSA_ERR_INVALID_ARG;
+  CUtensorMap tm;
+  if (!make_probe_map(&tm, src, rows)) return LLSA_ERR_CUDA;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  auto run = [&](auto kern, int smem) -> llsa_status {
+    if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
+    return launch(kKGatherProbe, cs, [&] {
+      kern<<<ctas, kProbeWarps * 32, smem, cs>>>(tm, tile_rows, ntiles, (int)rows);
+    });
+  };
+  if (stages == 2) return run(gather_probe_kernel<2>, gather_probe_smem<2>());
+  if (stages == 4) return run(gather_probe_kernel<4>, gather_probe_smem<4>());
+  return run(gather_probe_kernel<8>, gather_probe_smem<8>());
 }
 
 llsa_status llsa_trace_begin(void** events, int32_t* kernel_ids, int32_t capacity) {

@@ -11,9 +11,9 @@
 namespace llsa {
 
 constexpr int kBlock = 16;      // tokens per block (README usage section: block_size=16)
-constexpr int kD = 64;          // channels per head handled by this build
+constexpr int kMaxD = 128;      // head widths D = 64 and 128 are built (every kernel is templated on D)
 constexpr int kMaxLevels = 4;
-constexpr int kTileBytes = 2048;  // one 16-token x 64-channel bf16 tile
+constexpr int kSubTileBytes = 2048;  // 16 rows x 128 bytes: 64 bf16 channels of a 16-token tile
 
 // TMA ring depths of the attention kernels (forward, query-major dQ, key-major dK/dV).  A
 // sweep on B200 at the headline workload preferred 2 stages everywhere: deeper rings cost
@@ -38,19 +38,11 @@ constexpr int kTileBytes = 2048;  // one 16-token x 64-channel bf16 tile
 #endif
 constexpr int kKvUnroll = LLSA_KV_UNROLL;
 constexpr int kQmUnroll = LLSA_QM_UNROLL;
-// Key-major dK/dV on tcgen05 (1) or on mma.sync warps (0, the default).  At 16-key blocks
-// the tcgen05 kernel is the slower one on B200 (301 us against 195 us at B1 H6 N65536 L3
-// K8): every MMA reads its 4 KB query-side operand from shared memory, Q and dO are read
-// twice per batch, and 4 batches in flight per SM do not cover the ~2 us latency of the
-// gathered tiles; the mma.sync warps keep K/V fragments and accumulators in registers.
-#ifndef LLSA_KEY_MAJOR_TC
-#define LLSA_KEY_MAJOR_TC 0
-#endif
 
 // Per-call geometry: level sizes and the level-major offsets of every packed buffer.
 struct Geometry {
   int B, H, N, D, K, L, BH;
-  int log_k, log_n1;                     // log2 K and log2 n_1 where they are powers of two, else -1
+  int log_k, log_n1, log_n;              // log2 K, log2 n_1, log2 N where they are powers of two, else -1
   int n[kMaxLevels + 1];                 // n[l] = N / 16^l, l = 0..L
   long long pyr_off[kMaxLevels + 1];     // element offset of level l (1..L) in a pyramid
   long long idx_off[kMaxLevels + 1];     // element offset of level l in idx / col
@@ -63,11 +55,22 @@ struct Geometry {
                                          // entry of the level-L part; C (never reached) otherwise
   int pool1;                             // LLSA_FLAG_LEVEL1: each selected fine block's
                                          // level-1 mean is one more KV entry
+  int nv;                                // real tokens per sequence (N when not padded)
+  int m[kMaxLevels + 1];                 // real tokens of level l: ceil(nv / 16^l)
 };
 
-// x / K and x / n_1, by a shift when the divisor is a power of two.
+// Real tokens under level-l token j of a sequence with nv real tokens: clamp(nv - j 16^l,
+// 0, 16^l) (16^l for every token when the sequence is not padded).
+__host__ __device__ inline int pool_count(const Geometry& g, int l, int j) {
+  const long long span = 1LL << (4 * l);
+  const long long c = (long long)g.nv - (long long)j * span;
+  return c <= 0 ? 0 : (c >= span ? (int)span : (int)c);
+}
+
+// x / K, x / n_1 and x / N, by a shift when the divisor is a power of two.
 __host__ __device__ inline int div_k(const Geometry& g, int x) { return g.log_k >= 0 ? x >> g.log_k : x / g.K; }
 __host__ __device__ inline int div_n1(const Geometry& g, int x) { return g.log_n1 >= 0 ? x >> g.log_n1 : x / g.n[1]; }
+__host__ __device__ inline int div_n(const Geometry& g, int x) { return g.log_n >= 0 ? x >> g.log_n : x / g.N; }
 
 // Level of coarse entry c (0 <= c < C): 2 + c / K, except that under the all-coarsest
 // variant the entries from top_first on are level L.
@@ -140,10 +143,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
-// D = A (16x16 bf16, row) * B (16x8 bf16, col) + D, fp32 accumulate.
+// D = A (16x16 bf16, row) * B (16x8 bf16, col) + D, fp32 accumulate.  Registers in and out
+// only (no side effects), so the compiler may schedule it like arithmetic.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -223,18 +227,21 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after about two seconds at the maximum SM clock, records
-// LLSA_ERR_TIMEOUT and returns false, so a copy that never lands cannot hang the GPU.
-// Once any wait has timed out (the status word holds LLSA_ERR_TIMEOUT) the others give up
-// at their next check instead of spending their own two seconds.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Limit of a bounded wait: about two seconds at the maximum SM clock.
+constexpr long long kWaitLimitCycles = 4000000000LL;
+
+// Bounded wait: gives up after `limit` SM cycles, records LLSA_ERR_TIMEOUT and returns
+// false, so a copy that never lands cannot hang the GPU.  Once any wait has timed out (the
+// status word holds LLSA_ERR_TIMEOUT) the others give up at their next check instead of
+// spending their own limit.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (unsigned it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*reinterpret_cast<volatile int*>(&g_llsa_status) == LLSA_ERR_TIMEOUT) return false;
-      if (clock64() - t0 > 4000000000LL) {
+      if (clock64() - t0 > limit) {
         record_error(LLSA_ERR_TIMEOUT);
         return false;
       }
@@ -242,8 +249,31 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Check of the timeout path of mbar_wait, the wait every kernel uses: one thread arms an
+// mbarrier for 16 bytes of a transfer that is never issued (so no copy is ever in flight),
+// waits on it with a limit of `limit` cycles, and the wait gives up and records
+// LLSA_ERR_TIMEOUT.  Nothing else is touched.
+__global__ void __launch_bounds__(32) bounded_wait_check_kernel(long long limit) {
+  __shared__ __align__(8) unsigned long long bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+  mbar_init(b, 1);
+  mbar_fence_init();
+  mbar_expect_tx(b, 16);
+  mbar_wait(b, 0, limit);
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// 3-D tiled TMA load (no multicast) of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
 }
 
 // 2-D tiled TMA load (no multicast) of one box into shared memory, completing on `bar`.

@@ -6,6 +6,9 @@
 // 16j..16j+15, each addition rounded to fp32 in that order (__fadd_rn keeps the compiler
 // from re-associating or contracting), so results are bit-identical to any other
 // implementation of the same order.
+// A padded sequence (nv < N real tokens) changes only the tokens whose span reaches past nv
+// (pooled_mean below): they average their c real tokens, level 1 as (sum of the real tokens
+// in order) / c, level l >= 2 as (sum in order of c_child * child) / c, and empty ones are 0.
 //
 // Bound: HBM streaming.  Reads B*H*N*D input elements of each of q, k, v once and writes
 // B*H*D*sum_l n_l fp32 values per tensor; levels 1 and 2 are produced by one kernel (the
@@ -51,71 +54,87 @@ struct Vec16<float> {
 
 constexpr int kPyrThreads = 256;
 
-// Dynamic shared memory of pyramid_l12_kernel<T>: its span of ROWS * 16 input rows.
-template <typename T>
-constexpr int pyramid_span_bytes() {
-  return (kPyrThreads / (kD / (16 / (int)sizeof(T)))) * kBlock * kD * (int)sizeof(T);
+// Mean of a token from its in-order fp32 sum and its count of real tokens: the exact
+// power-of-two scaling for a full token (the unpadded pyramid), 0 for an empty one, a
+// correctly rounded division otherwise.
+__device__ __forceinline__ float pooled_mean(float sum, int count, int full) {
+  if (count == full) return __fmul_rn(sum, 1.0f / (float)full);
+  return count == 0 ? 0.0f : __fdiv_rn(sum, (float)count);
 }
 
-// grid.x = B*H * ceil(n_1 / rows_per_cta), grid.y = 3 (q, k, v).
-// Each thread owns kElems consecutive channels of one level-1 output row.
-template <typename T>
-__global__ void __launch_bounds__(kPyrThreads) pyramid_l12_kernel(Geometry g, const T* __restrict__ x0,
-                                                                  const T* __restrict__ x1,
-                                                                  const T* __restrict__ x2, float* __restrict__ p0,
-                                                                  float* __restrict__ p1, float* __restrict__ p2) {
-  pdl_enter();
-  constexpr int VE = Vec16<T>::kElems;
-  constexpr int TPR = kD / VE;                   // threads per row
-  constexpr int ROWS = kPyrThreads / TPR;         // level-1 rows per CTA (32 for bf16, 16 for fp32)
-  __shared__ float s1[ROWS][kD];
-  __shared__ __align__(8) uint64_t bar_storage;
-  extern __shared__ __align__(128) uint8_t pyr_span[];  // ROWS * 16 input rows (pyramid_span_bytes)
+// Level-l token j (l >= 2) of level-(l-1) rows src[r * stride], r < 16: (sum of the 16
+// rows) / 16 for a full token; the count-weighted form for a token a padded sequence cuts.
+__device__ __forceinline__ float pool_up(const Geometry& g, int l, int j, const float (&x)[kBlock]) {
+  const int c = pool_count(g, l, j);
+  const int full = 1 << (4 * l);
+  float acc = 0.0f;
+  if (c == full) {
+#pragma unroll
+    for (int r = 0; r < kBlock; ++r) acc = __fadd_rn(acc, x[r]);
+    return __fmul_rn(acc, 0.0625f);
+  }
+#pragma unroll
+  for (int r = 0; r < kBlock; ++r) acc = __fadd_rn(acc, __fmul_rn((float)pool_count(g, l - 1, j * kBlock + r), x[r]));
+  return c == 0 ? 0.0f : __fdiv_rn(acc, (float)c);
+}
 
-  const T* x = blockIdx.y == 0 ? x0 : (blockIdx.y == 1 ? x1 : x2);
-  float* pyr = blockIdx.y == 0 ? p0 : (blockIdx.y == 1 ? p1 : p2);
+// Launch shape of pyramid_l12_kernel<T, D>: each thread owns VE consecutive channels of one
+// level-1 output row; a CTA makes ROWS level-1 rows (at least 16, so whole level-2 rows)
+// from its span of ROWS * 16 input rows.
+template <typename T, int D>
+struct PyrCfg {
+  static constexpr int VE = Vec16<T>::kElems;
+  static constexpr int TPR = D / VE;                                          // threads per row
+  static constexpr int ROWS = kPyrThreads / TPR > kBlock ? kPyrThreads / TPR : kBlock;
+  static constexpr int THREADS = ROWS * TPR;
+  static constexpr int SPAN = ROWS * kBlock * D * (int)sizeof(T);             // dynamic smem bytes
+};
 
+// One unit of levels 1-2: ROWS level-1 rows (tile `tile` of head bh) of one tensor x, and
+// the level-2 rows they make.  The CTA's input span (ROWS * 16 token rows) arrives by one
+// bulk copy completing on `bar` with phase parity `parity`; `span` and `s1` are the CTA's
+// shared buffers.  Every thread of the CTA calls it; returns false (for the whole CTA) if
+// the copy did not land within the bounded wait.
+template <typename T, int D>
+__device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __restrict__ x,
+                                                 float* __restrict__ pyr, int bh, int tile, uint8_t* span,
+                                                 float (*s1)[D], uint32_t bar, uint32_t parity) {
+  using C = PyrCfg<T, D>;
+  constexpr int VE = C::VE;
+  constexpr int TPR = C::TPR;
+  constexpr int ROWS = C::ROWS;
   const int n1 = g.n[1];
-  const int tiles = (n1 + ROWS - 1) / ROWS;
-  const int bh = blockIdx.x / tiles;
-  const int tile = blockIdx.x - bh * tiles;
   const int t = threadIdx.x;
   const int o = t / TPR;
   const int c0 = (t % TPR) * VE;
   const int j1 = tile * ROWS + o;
-
-  const uint32_t bar = smem_u32(&bar_storage);
+  __syncthreads();  // the span and s1 of the previous unit are no longer read
   if (t == 0) {
-    mbar_init(bar, 1);
-    mbar_fence_init();
-  }
-  __syncthreads();
-  if (t == 0) {
-    const uint32_t bytes = (uint32_t)(min(ROWS, n1 - tile * ROWS) * kBlock * kD * (int)sizeof(T));
+    const uint32_t bytes = (uint32_t)(min(ROWS, n1 - tile * ROWS) * kBlock * D * (int)sizeof(T));
     mbar_expect_tx(bar, bytes);
-    bulk_load(smem_u32(pyr_span), x + ((long long)bh * g.N + (long long)tile * ROWS * kBlock) * kD, bytes, bar);
+    bulk_load(smem_u32(span), x + ((long long)bh * g.N + (long long)tile * ROWS * kBlock) * D, bytes, bar);
   }
-  if (!mbar_wait(bar, 0)) {  // recorded as LLSA_ERR_TIMEOUT; give the copy one more bounded wait
-    mbar_wait(bar, 0);
-    return;
+  if (!__syncthreads_and(mbar_wait(bar, parity))) {
+    mbar_wait(bar, parity);  // recorded as LLSA_ERR_TIMEOUT; one more bounded wait for the copy
+    return false;
   }
-
   if (j1 < n1) {
-    const T* src = reinterpret_cast<const T*>(pyr_span) + (o * kBlock) * kD + c0;
+    const T* src = reinterpret_cast<const T*>(span) + (o * kBlock) * D + c0;
     float v[kBlock][VE];
 #pragma unroll
-    for (int r = 0; r < kBlock; ++r) Vec16<T>::load(src + r * kD, v[r]);
+    for (int r = 0; r < kBlock; ++r) Vec16<T>::load(src + r * D, v[r]);
     float acc[VE];
 #pragma unroll
     for (int e = 0; e < VE; ++e) acc[e] = 0.0f;
+    const int c1 = pool_count(g, 1, j1);  // 16 unless the sequence is padded
 #pragma unroll
     for (int r = 0; r < kBlock; ++r)
 #pragma unroll
-      for (int e = 0; e < VE; ++e) acc[e] = __fadd_rn(acc[e], v[r][e]);
-    float* dst = pyr + g.pyr_off[1] + ((long long)bh * n1 + j1) * kD + c0;
+      for (int e = 0; e < VE; ++e) acc[e] = __fadd_rn(acc[e], r < c1 ? v[r][e] : 0.0f);
+    float* dst = pyr + g.pyr_off[1] + ((long long)bh * n1 + j1) * D + c0;
 #pragma unroll
     for (int e = 0; e < VE; ++e) {
-      acc[e] = __fmul_rn(acc[e], 0.0625f);
+      acc[e] = pooled_mean(acc[e], c1, kBlock);
       s1[o][c0 + e] = acc[e];
     }
     if constexpr (VE == 8) {
@@ -125,40 +144,67 @@ __global__ void __launch_bounds__(kPyrThreads) pyramid_l12_kernel(Geometry g, co
       reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
   }
-  if (g.L < 2) return;
+  if (g.L < 2) return true;
   __syncthreads();
-  constexpr int OUT2 = ROWS / kBlock;  // level-2 rows per CTA
-  if (t < OUT2 * kD) {
-    const int o2 = t / kD;
-    const int d = t % kD;
+  constexpr int OUT2 = ROWS / kBlock;  // level-2 rows per unit
+  for (int i = t; i < OUT2 * D; i += blockDim.x) {
+    const int o2 = i / D;
+    const int d = i % D;
     const int j2 = tile * OUT2 + o2;
     if (j2 < g.n[2] && (j2 + 1) * kBlock <= n1) {
-      float acc = 0.0f;
+      float xr[kBlock];
 #pragma unroll
-      for (int r = 0; r < kBlock; ++r) acc = __fadd_rn(acc, s1[o2 * kBlock + r][d]);
-      pyr[g.pyr_off[2] + ((long long)bh * g.n[2] + j2) * kD + d] = __fmul_rn(acc, 0.0625f);
+      for (int r = 0; r < kBlock; ++r) xr[r] = s1[o2 * kBlock + r][d];
+      pyr[g.pyr_off[2] + ((long long)bh * g.n[2] + j2) * D + d] = pool_up(g, 2, j2, xr);
     }
   }
+  return true;
+}
+
+// grid.x = B*H * ceil(n_1 / ROWS), grid.y = 3 (q, k, v).
+template <typename T, int D>
+__global__ void __launch_bounds__(PyrCfg<T, D>::THREADS) pyramid_l12_kernel(Geometry g, const T* __restrict__ x0,
+                                                                            const T* __restrict__ x1,
+                                                                            const T* __restrict__ x2,
+                                                                            float* __restrict__ p0,
+                                                                            float* __restrict__ p1,
+                                                                            float* __restrict__ p2) {
+  pdl_enter();
+  using C = PyrCfg<T, D>;
+  __shared__ float s1[C::ROWS][D];
+  __shared__ __align__(8) uint64_t bar_storage;
+  extern __shared__ __align__(128) uint8_t pyr_span[];  // ROWS * 16 input rows (C::SPAN bytes)
+  const int tiles = (g.n[1] + C::ROWS - 1) / C::ROWS;
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  const T* x = blockIdx.y == 0 ? x0 : (blockIdx.y == 1 ? x1 : x2);
+  float* pyr = blockIdx.y == 0 ? p0 : (blockIdx.y == 1 ? p1 : p2);
+  const int bh = blockIdx.x / tiles;
+  pyramid_l12_unit<T, D>(g, x, pyr, bh, blockIdx.x - bh * tiles, pyr_span, s1, bar, 0);
 }
 
 // Level l >= 3 from level l-1 (fp32).  One thread per output value; grid.y = tensor.
+template <int D>
 __global__ void __launch_bounds__(kPyrThreads) pyramid_up_kernel(Geometry g, int level, float* __restrict__ p0,
                                                                  float* __restrict__ p1, float* __restrict__ p2) {
   pdl_enter();
   float* pyr = blockIdx.y == 0 ? p0 : (blockIdx.y == 1 ? p1 : p2);
-  const long long total = (long long)g.BH * g.n[level] * kD;
+  const long long total = (long long)g.BH * g.n[level] * D;
   const long long i = (long long)blockIdx.x * kPyrThreads + threadIdx.x;
   if (i >= total) return;
-  const int d = (int)(i % kD);
-  const long long row = i / kD;  // bh * n_l + j
+  const int d = (int)(i % D);
+  const long long row = i / D;  // bh * n_l + j
   const int nl = g.n[level];
   const long long bh = row / nl;
   const int j = (int)(row - bh * nl);
-  const float* src = pyr + g.pyr_off[level - 1] + (bh * g.n[level - 1] + (long long)j * kBlock) * kD + d;
-  float acc = 0.0f;
+  const float* src = pyr + g.pyr_off[level - 1] + (bh * g.n[level - 1] + (long long)j * kBlock) * D + d;
+  float x[kBlock];
 #pragma unroll
-  for (int r = 0; r < kBlock; ++r) acc = __fadd_rn(acc, src[r * kD]);
-  pyr[g.pyr_off[level] + row * kD + d] = __fmul_rn(acc, 0.0625f);
+  for (int r = 0; r < kBlock; ++r) x[r] = src[r * D];
+  pyr[g.pyr_off[level] + row * D + d] = pool_up(g, level, j, x);
 }
 
 }  // namespace llsa

@@ -15,7 +15,7 @@
 // reused by its 16 queries); the arithmetic is 16 * 16K * 64 FMA per group.
 #pragma once
 
-#include "llsa_common.cuh"
+#include "pyramid.cuh"
 
 namespace llsa {
 
@@ -29,12 +29,18 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Candidate rows are staged in shared memory with a padded stride (68 floats: a quarter
+// Candidate rows are staged in shared memory with a padded stride (D + 4 floats: a quarter
 // warp's 16-byte reads of 8 consecutive rows hit 8 distinct bank groups).
-constexpr int kSelRowStride = kD + 4;
-// Candidates scored per pass; larger candidate sets (coarsest level with n_L > 256) are
-// scored in passes of this many rows.
-constexpr int kSelChunk = 256;
+template <int D>
+__host__ __device__ constexpr int sel_row_stride() {
+  return D + 4;
+}
+// Candidates scored per pass (256 rows at D = 64, 128 at D = 128: about 68 KB of staged
+// rows); larger candidate sets (the coarsest level) are scored in passes of this many rows.
+template <int D>
+__host__ __device__ constexpr int sel_chunk() {
+  return D == 64 ? 256 : 128;
+}
 
 // Top-K of one query's score keys krow[0..nc) by one warp: each lane keeps the best of its
 // candidates c = lane + 32 i; redux.sync finds the largest key, then the lowest candidate
@@ -72,6 +78,7 @@ __device__ __forceinline__ void warp_topk(uint32_t* krow, int nc, int K, int* wr
 
 // grid.x = B*H * groups; dynamic smem: see select_smem_bytes.
 // parent_idx == nullptr selects the coarsest-level mode.
+template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int level, int gq,
                                                              const float* __restrict__ qp,
                                                              const float* __restrict__ kp,
@@ -88,17 +95,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
   const int grp = blockIdx.x - bh * groups;
   const int a0 = grp * gq;
   const int rows = min(gq, n - a0);
-  const int chunk = min(nc, kSelChunk);
+  const int chunk = min(nc, sel_chunk<D>());
 
-  float* qs = sel_smem;                                             // [gq][64]
-  float* ks = qs + gq * kD;                                         // [chunk][68]
-  int* cand = reinterpret_cast<int*>(ks + chunk * kSelRowStride);   // [nc] (sparse only)
+  constexpr int RS = sel_row_stride<D>();
+  float* qs = sel_smem;                                             // [gq][D]
+  float* ks = qs + gq * D;                                          // [chunk][D + 4]
+  int* cand = reinterpret_cast<int*>(ks + chunk * RS);              // [nc] (sparse only)
   uint32_t* sk = reinterpret_cast<uint32_t*>(cand + (sparse ? nc : 0));  // [gq][nc] score keys
   int* win = reinterpret_cast<int*>(sk + gq * nc);                  // [gq][K]
 
   const int tid = threadIdx.x;
-  const float* qbase = qp + ((long long)bh * n + a0) * kD;
-  for (int i = tid; i < gq * kD; i += kSelThreads) qs[i] = (i < rows * kD) ? qbase[i] : 0.0f;
+  const float* qbase = qp + ((long long)bh * n + a0) * D;
+  for (int i = tid; i < gq * D; i += kSelThreads) qs[i] = (i < rows * D) ? qbase[i] : 0.0f;
   if (sparse) {
     const int np = g.n[level + 1];
     const int* prow = parent_idx + ((long long)bh * np + a0 / kBlock) * K;
@@ -119,12 +127,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
   for (int c0 = 0; c0 < nc; c0 += chunk) {
     const int cn = min(chunk, nc - c0);
     // stage rows c0 .. c0+cn-1 (coalesced: 16 threads copy one 256-byte row)
-    for (int i = tid; i < cn * (kD / 4); i += kSelThreads) {
-      const int r = i / (kD / 4);
-      const int piece = i - r * (kD / 4);
+    for (int i = tid; i < cn * (D / 4); i += kSelThreads) {
+      const int r = i / (D / 4);
+      const int piece = i - r * (D / 4);
       const int key = sparse ? cand[c0 + r] : c0 + r;
-      const float4 v = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + key) * kD) + piece);
-      *reinterpret_cast<float4*>(ks + r * kSelRowStride + piece * 4) = v;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + key) * D) + piece);
+      *reinterpret_cast<float4*>(ks + r * RS + piece * 4) = v;
     }
     __syncthreads();
     for (int c = ct0; c < cn; c += 4 * tpq) {
@@ -135,12 +143,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
         for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
       const float4* kr[4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) kr[v] = reinterpret_cast<const float4*>(ks + min(c + v * tpq, cn - 1) * kSelRowStride);
+      for (int v = 0; v < 4; ++v) kr[v] = reinterpret_cast<const float4*>(ks + min(c + v * tpq, cn - 1) * RS);
       const float4* qr[2];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) qr[u] = reinterpret_cast<const float4*>(qs + min(2 * qg + u, gq - 1) * kD);
+      for (int u = 0; u < 2; ++u) qr[u] = reinterpret_cast<const float4*>(qs + min(2 * qg + u, gq - 1) * D);
 #pragma unroll 4
-      for (int i = 0; i < kD / 4; ++i) {
+      for (int i = 0; i < D / 4; ++i) {
         float4 kv[4], qv[2];
 #pragma unroll
         for (int v = 0; v < 4; ++v) kv[v] = kr[v][i];
@@ -162,7 +170,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int cc = c + v * tpq;
-          if (qi < gq && cc < cn) sk[qi * nc + c0 + cc] = score_key(acc[u][v]);
+          if (qi < gq && cc < cn) {
+            // empty tokens of a padded sequence (index >= the level's real count) are never
+            // candidates: key 0 marks a removed candidate
+            const int key = sparse ? cand[c0 + cc] : c0 + cc;
+            sk[qi * nc + c0 + cc] = key < g.m[level] ? score_key(acc[u][v]) : 0u;
+          }
         }
       }
     }
@@ -187,10 +200,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
   }
 }
 
+template <int D>
 inline size_t select_smem_bytes(int gq, int nc, int K, bool sparse) {
-  const int chunk = nc < kSelChunk ? nc : kSelChunk;
-  return sizeof(float) * ((size_t)gq * kD + (size_t)chunk * kSelRowStride + (sparse ? nc : 0) + (size_t)gq * nc +
-                          (size_t)gq * K);
+  const int chunk = nc < sel_chunk<D>() ? nc : sel_chunk<D>();
+  return sizeof(float) * ((size_t)gq * D + (size_t)chunk * sel_row_stride<D>() + (sparse ? nc : 0) +
+                          (size_t)gq * nc + (size_t)gq * K);
 }
 
 // Finer levels with 16K = 32 * CPT candidates (K = 2, 4, 8, 16): the 16 sibling queries of
@@ -200,37 +214,52 @@ inline size_t select_smem_bytes(int gq, int nc, int K, bool sparse) {
 // (score desc, position asc); then K rounds of redux.sync max (score key) then min
 // (candidate position) over the lanes' heads, the two queries' rounds interleaved.  The dot products
 // accumulate channels 0..63 in order, as in select_kernel, so both give the same scores.
-template <int CPT>
-__global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g, int level,
-                                                                      const float* __restrict__ qp,
-                                                                      const float* __restrict__ kp,
-                                                                      const int* __restrict__ parent_idx,
-                                                                      int* __restrict__ out_idx) {
-  pdl_enter();
+// A load of data that the same launch may have written (RO = false: the coherent path) or
+// of data read-only for the whole launch (RO = true: the read-only data cache).
+template <bool RO, typename T>
+__device__ __forceinline__ T ld_in(const T* p) {
+  if constexpr (RO) return __ldg(p);
+  else return *p;
+}
+
+// One sibling group (unit = (b*H + h) * (n_l / 16) + group) of select_children_kernel;
+// `sel_smem` is the CTA's shared buffer (select_children_smem_bytes).  kSelThreads threads.
+// RO: the pyramid and the parent selection were written by earlier launches (read through
+// the read-only cache); false inside the fused launch that writes them.
+template <int D, int CPT, bool RO = true>
+__device__ __forceinline__ void select_children_unit(const Geometry& g, int level, const float* __restrict__ qp,
+                                                     const float* __restrict__ kp, const int* __restrict__ parent_idx,
+                                                     int* __restrict__ out_idx, int unit, float* sel_smem) {
   constexpr int NC = 32 * CPT;
   constexpr int K = 2 * CPT;  // NC = 16 K
-  extern __shared__ __align__(16) float sel_smem[];
   const int n = g.n[level];
   const int groups = n / kBlock;
-  const int bh = blockIdx.x / groups;
-  const int grp = blockIdx.x - bh * groups;
+  const int bh = unit / groups;
+  const int grp = unit - bh * groups;
   const int a0 = grp * kBlock;
 
-  float* qs = sel_smem;                                          // [16][64]
-  float* ks = qs + kBlock * kD;                                  // [NC][68]
-  int* cand = reinterpret_cast<int*>(ks + NC * kSelRowStride);   // [NC]
+  constexpr int RS = sel_row_stride<D>();
+  constexpr int PR = D / 4;                                      // float4 pieces per row
+  float* qs = sel_smem;                                          // [16][D]
+  float* ks = qs + kBlock * D;                                   // [NC][D + 4]
+  int* cand = reinterpret_cast<int*>(ks + NC * RS);              // [NC]
 
   const int tid = threadIdx.x;
-  const float4* qbase = reinterpret_cast<const float4*>(qp + ((long long)bh * n + a0) * kD);
-  const float4 qv = __ldg(qbase + tid);  // 16 rows x 16 pieces = one per thread
+  const float4* qbase = reinterpret_cast<const float4*>(qp + ((long long)bh * n + a0) * D);
+  constexpr int QP = kBlock * PR / kSelThreads;  // query pieces per thread (16 rows x D/4)
+  float4 qv[QP];
+#pragma unroll
+  for (int u = 0; u < QP; ++u) qv[u] = ld_in<RO>(qbase + tid + u * kSelThreads);
   const int np = g.n[level + 1];
   const int* prow = parent_idx + ((long long)bh * np + a0 / kBlock) * K;
-  for (int i = tid; i < NC; i += kSelThreads) cand[i] = checked_index(__ldg(prow + i / kBlock), np) * kBlock + (i % kBlock);
-  reinterpret_cast<float4*>(qs)[tid] = qv;
+  __syncthreads();  // the previous unit's shared rows are no longer read
+  for (int i = tid; i < NC; i += kSelThreads) cand[i] = checked_index(ld_in<RO>(prow + i / kBlock), np) * kBlock + (i % kBlock);
+#pragma unroll
+  for (int u = 0; u < QP; ++u) reinterpret_cast<float4*>(qs)[tid + u * kSelThreads] = qv[u];
   __syncthreads();
   // candidate rows: 16 threads copy one 256-byte row; each thread issues all its loads
   // (up to 8 at a time) before storing any, so they share one memory latency
-  constexpr int kPer = NC * (kD / 4) / kSelThreads;  // float4 pieces per thread
+  constexpr int kPer = NC * PR / kSelThreads;  // float4 pieces per thread
   constexpr int kBatch = kPer < 8 ? kPer : 8;
 #pragma unroll
   for (int b0 = 0; b0 < kPer; b0 += kBatch) {
@@ -238,28 +267,28 @@ __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = tid + (b0 + u) * kSelThreads;
-      v[u] = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + cand[i >> 4]) * kD) + (i & 15));
+      v[u] = ld_in<RO>(reinterpret_cast<const float4*>(kp + ((long long)bh * n + cand[i / PR]) * D) + (i % PR));
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = tid + (b0 + u) * kSelThreads;
-      *reinterpret_cast<float4*>(ks + (i >> 4) * kSelRowStride + (i & 15) * 4) = v[u];
+      *reinterpret_cast<float4*>(ks + (i / PR) * RS + (i % PR) * 4) = v[u];
     }
   }
   __syncthreads();
 
   const int warp = tid >> 5, lane = tid & 31;
-  const float4* q0 = reinterpret_cast<const float4*>(qs + (2 * warp) * kD);
-  const float4* q1 = reinterpret_cast<const float4*>(qs + (2 * warp + 1) * kD);
+  const float4* q0 = reinterpret_cast<const float4*>(qs + (2 * warp) * D);
+  const float4* q1 = reinterpret_cast<const float4*>(qs + (2 * warp + 1) * D);
   float acc[2][CPT];
 #pragma unroll
   for (int j = 0; j < CPT; ++j) acc[0][j] = acc[1][j] = 0.f;
 #pragma unroll 4
-  for (int i = 0; i < kD / 4; ++i) {
+  for (int i = 0; i < D / 4; ++i) {
     const float4 a = q0[i], b = q1[i];
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-      const float4 kv = reinterpret_cast<const float4*>(ks + (lane + 32 * j) * kSelRowStride)[i];
+      const float4 kv = reinterpret_cast<const float4*>(ks + (lane + 32 * j) * RS)[i];
       acc[0][j] = fmaf(a.x, kv.x, acc[0][j]);
       acc[0][j] = fmaf(a.y, kv.y, acc[0][j]);
       acc[0][j] = fmaf(a.z, kv.z, acc[0][j]);
@@ -276,11 +305,12 @@ __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g
   // each lane orders its CPT candidates once (score desc, index asc); a winner's owner then
   // only shifts its list
   int ci[2][CPT];
+  const int mreal = g.m[level];  // real tokens of the level (all n of them unless padded)
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-      key[u][j] = score_key(acc[u][j]);
+      key[u][j] = cand[lane + 32 * j] < mreal ? score_key(acc[u][j]) : 0u;
       ci[u][j] = lane + 32 * j;
     }
 #pragma unroll
@@ -336,8 +366,20 @@ __global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g
   }
 }
 
+template <int D, int CPT>
+__global__ void __launch_bounds__(kSelThreads) select_children_kernel(Geometry g, int level,
+                                                                      const float* __restrict__ qp,
+                                                                      const float* __restrict__ kp,
+                                                                      const int* __restrict__ parent_idx,
+                                                                      int* __restrict__ out_idx) {
+  pdl_enter();
+  extern __shared__ __align__(16) float sel_smem[];
+  select_children_unit<D, CPT>(g, level, qp, kp, parent_idx, out_idx, blockIdx.x, sel_smem);
+}
+
+template <int D>
 inline size_t select_children_smem_bytes(int nc) {
-  return sizeof(float) * ((size_t)kBlock * kD + (size_t)nc * kSelRowStride + (size_t)nc);
+  return sizeof(float) * ((size_t)kBlock * D + (size_t)nc * sel_row_stride<D>() + (size_t)nc);
 }
 
 // Coarsest level with few tokens (n_L <= 64), one CTA per (b, h): optionally first the
@@ -350,69 +392,77 @@ constexpr int kTopMaxN = 64;
 
 constexpr int kTopThreads = 512;
 
-template <bool POOL>
-__global__ void __launch_bounds__(kTopThreads) coarsest_small_kernel(Geometry g, float* __restrict__ q_pyr,
-                                                                     float* __restrict__ k_pyr,
-                                                                     float* __restrict__ v_pyr,
-                                                                     int* __restrict__ idx) {
-  pdl_enter();
-  __shared__ __align__(16) float qs[kTopMaxN * kSelRowStride];
-  __shared__ __align__(16) float ks[kTopMaxN * kSelRowStride];
-  const int bh = blockIdx.x;
+// Dynamic shared memory: the n_L query and key rows at stride D + 4.
+template <int D>
+__host__ __device__ constexpr int coarsest_small_smem() {
+  return 2 * kTopMaxN * sel_row_stride<D>() * (int)sizeof(float);
+}
+
+// One (b, h) of coarsest_small_kernel, by any number of whole warps; `top_smem` is the
+// CTA's shared buffer (coarsest_small_smem).
+template <int D, bool POOL>
+__device__ __forceinline__ void coarsest_small_unit(const Geometry& g, float* __restrict__ q_pyr,
+                                                    float* __restrict__ k_pyr, float* __restrict__ v_pyr,
+                                                    int* __restrict__ idx, int bh, float* top_smem) {
+  constexpr int RS = sel_row_stride<D>();
+  constexpr int PR = D / 4;
+  float* qs = top_smem;                    // [n_L][D + 4]
+  float* ks = top_smem + kTopMaxN * RS;    // [n_L][D + 4]
+  const int nth = blockDim.x;
   const int L = g.L, K = g.K, n = g.n[L];
   if (POOL) {
     for (int l = 3; l <= L; ++l) {
       const int nl = g.n[l], np = g.n[l - 1];
-      const int items = 3 * nl * kD;
+      const int items = 3 * nl * D;
       // two values per pass: their 32 loads are issued before the in-order sums
-      for (int i0 = threadIdx.x; i0 < items; i0 += 2 * kTopThreads) {
+      for (int i0 = threadIdx.x; i0 < items; i0 += 2 * nth) {
         float x[2][kBlock];
         float* dst[2] = {nullptr, nullptr};
+        int jj[2] = {0, 0};
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int i = i0 + u * kTopThreads;
+          const int i = i0 + u * nth;
           if (i < items) {
-            const int t = i / (nl * kD);
-            const int rem = i - t * nl * kD;
-            const int j = rem >> 6, d = rem & (kD - 1);
+            const int t = i / (nl * D);
+            const int rem = i - t * nl * D;
+            const int j = rem / D, d = rem - j * D;
+            jj[u] = j;
             float* pyr = t == 0 ? q_pyr : (t == 1 ? k_pyr : v_pyr);
-            const float* src = pyr + g.pyr_off[l - 1] + ((long long)bh * np + (long long)j * kBlock) * kD + d;
+            const float* src = pyr + g.pyr_off[l - 1] + ((long long)bh * np + (long long)j * kBlock) * D + d;
 #pragma unroll
-            for (int r = 0; r < kBlock; ++r) x[u][r] = src[r * kD];
-            dst[u] = pyr + g.pyr_off[l] + ((long long)bh * nl + j) * kD + d;
+            for (int r = 0; r < kBlock; ++r) x[u][r] = src[r * D];
+            dst[u] = pyr + g.pyr_off[l] + ((long long)bh * nl + j) * D + d;
           }
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           if (!dst[u]) continue;
-          float acc = 0.0f;
-#pragma unroll
-          for (int r = 0; r < kBlock; ++r) acc = __fadd_rn(acc, x[u][r]);
-          *dst[u] = __fmul_rn(acc, 0.0625f);
+          *dst[u] = pool_up(g, l, jj[u], x[u]);
         }
       }
       __syncthreads();  // level l is read back by this CTA
     }
   }
-  const float* qrow = q_pyr + g.pyr_off[L] + (long long)bh * n * kD;
-  const float* krow = k_pyr + g.pyr_off[L] + (long long)bh * n * kD;
-  for (int i = threadIdx.x; i < n * (kD / 4); i += blockDim.x) {
-    const int r = i >> 4, piece = i & 15;
-    *reinterpret_cast<float4*>(qs + r * kSelRowStride + piece * 4) = reinterpret_cast<const float4*>(qrow + r * kD)[piece];
-    *reinterpret_cast<float4*>(ks + r * kSelRowStride + piece * 4) = reinterpret_cast<const float4*>(krow + r * kD)[piece];
+  __syncthreads();  // the previous unit's shared rows are no longer read
+  const float* qrow = q_pyr + g.pyr_off[L] + (long long)bh * n * D;
+  const float* krow = k_pyr + g.pyr_off[L] + (long long)bh * n * D;
+  for (int i = threadIdx.x; i < n * PR; i += blockDim.x) {
+    const int r = i / PR, piece = i - r * PR;
+    *reinterpret_cast<float4*>(qs + r * RS + piece * 4) = reinterpret_cast<const float4*>(qrow + r * D)[piece];
+    *reinterpret_cast<float4*>(ks + r * RS + piece * 4) = reinterpret_cast<const float4*>(krow + r * D)[piece];
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int a = warp; a < n; a += blockDim.x >> 5) {
-    const float4* qa = reinterpret_cast<const float4*>(qs + a * kSelRowStride);
+    const float4* qa = reinterpret_cast<const float4*>(qs + a * RS);
     float acc[2] = {0.f, 0.f};
 #pragma unroll 4
-    for (int i = 0; i < kD / 4; ++i) {
+    for (int i = 0; i < D / 4; ++i) {
       const float4 qv = qa[i];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int c = min(lane + 32 * j, n - 1);
-        const float4 kv = reinterpret_cast<const float4*>(ks + c * kSelRowStride)[i];
+        const float4 kv = reinterpret_cast<const float4*>(ks + c * RS)[i];
         acc[j] = fmaf(qv.x, kv.x, acc[j]);
         acc[j] = fmaf(qv.y, kv.y, acc[j]);
         acc[j] = fmaf(qv.z, kv.z, acc[j]);
@@ -424,7 +474,7 @@ __global__ void __launch_bounds__(kTopThreads) coarsest_small_kernel(Geometry g,
     int bc = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      key[j] = lane + 32 * j < n ? score_key(acc[j]) : 0u;
+      key[j] = lane + 32 * j < g.m[L] ? score_key(acc[j]) : 0u;  // real tokens only
       if (key[j] > bk) {
         bk = key[j];
         bc = lane + 32 * j;
@@ -452,6 +502,16 @@ __global__ void __launch_bounds__(kTopThreads) coarsest_small_kernel(Geometry g,
     for (int r2 = 0; r2 < K; ++r2) rank += __shfl_sync(0xffffffffu, win, r2) < win;
     if (lane < K) idx[g.idx_off[L] + ((long long)bh * n + a) * K + rank] = min(max(win, 0), n - 1);
   }
+}
+
+template <int D, bool POOL>
+__global__ void __launch_bounds__(kTopThreads) coarsest_small_kernel(Geometry g, float* __restrict__ q_pyr,
+                                                                     float* __restrict__ k_pyr,
+                                                                     float* __restrict__ v_pyr,
+                                                                     int* __restrict__ idx) {
+  pdl_enter();
+  extern __shared__ __align__(16) float top_smem[];
+  coarsest_small_unit<D, POOL>(g, q_pyr, k_pyr, v_pyr, idx, blockIdx.x, top_smem);
 }
 
 }  // namespace llsa

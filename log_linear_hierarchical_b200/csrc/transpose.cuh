@@ -9,9 +9,14 @@
 //   1. transpose_hist_kernel    one CTA per 4096-entry tile: per-warp bucket counts
 //                               (bucket = key / W, at most 64 buckets) via __match_any_sync,
 //                               summed into hist[bucket][tile].
-//   2. transpose_scatter_kernel one CTA per tile: bucket offsets from a scan of hist, then a
-//                               stable scatter of (key, query) pairs into bucket order.
-//   3. transpose_bucket_kernel  one CTA per bucket: per-key counts (warp-private, again via
+//   2. transpose_scan_kernel    one CTA per problem: an exclusive scan of hist in (bucket,
+//                               tile) order, in place, so hist[bucket][tile] becomes the
+//                               first output slot of that tile's entries of that bucket.
+//                               Only for problems of more than kTrScanTiles tiles; below
+//                               that, kernels 3 and 4 sum the few counts they need.
+//   3. transpose_scatter_kernel one CTA per tile: a stable scatter of (key, query) pairs into
+//                               bucket order from those offsets.
+//   4. transpose_bucket_kernel  one CTA per bucket: per-key counts (warp-private, again via
 //                               __match_any_sync), a scan that writes row_ptr, and a stable
 //                               scatter of the queries into col.
 //
@@ -39,8 +44,9 @@ struct TransposeLevel {
   int tiles;        // ceil(E / kTrTile)
   int nb;           // buckets per problem
   int wshift;       // log2(keys per bucket)
-  int cta_tiles;    // first tile-CTA of this level in kernels 1-2
-  int cta_buckets;  // first bucket-CTA of this level in kernel 3
+  int cta_tiles;    // first tile-CTA of this level in the hist and scatter kernels
+  int cta_buckets;  // first bucket-CTA of this level in the bucket kernel
+  int hstride;      // ints of hist per problem: nb * tiles counts, then their total
   long long hist_off;  // int offset of this level's hist in the workspace
   long long ent_off;   // entry offset of this level (same as idx/col level offset)
   long long rp_off;    // row_ptr offset of this level
@@ -105,17 +111,17 @@ __global__ void __launch_bounds__(kTrThreads) transpose_hist_kernel(TransposeGeo
     int s = 0;
 #pragma unroll
     for (int ww = 0; ww < kTrWarps; ++ww) s += cnt[ww][b];
-    ws_hist[L.hist_off + ((long long)bh * L.nb + b) * L.tiles + t] = s;
+    ws_hist[L.hist_off + (long long)bh * L.hstride + b * L.tiles + t] = s;
   }
 }
 
-// Exclusive scan of up to 64 values held in smem, by warp 0; also returns the total.
-__device__ __forceinline__ void tr_scan64(int* vals, int count, int* total_out) {
+// Exclusive scan of up to 64 values held in smem, by warp 0.
+__device__ __forceinline__ void tr_scan64(int* vals, int count) {
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    int a = (2 * lane < count) ? vals[2 * lane] : 0;
-    int b = (2 * lane + 1 < count) ? vals[2 * lane + 1] : 0;
-    int s = a + b;
+    const int a = (2 * lane < count) ? vals[2 * lane] : 0;
+    const int b = (2 * lane + 1 < count) ? vals[2 * lane + 1] : 0;
+    const int s = a + b;
     int incl = s;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -125,37 +131,103 @@ __device__ __forceinline__ void tr_scan64(int* vals, int count, int* total_out) 
     const int excl = incl - s;
     if (2 * lane < count) vals[2 * lane] = excl;
     if (2 * lane + 1 < count) vals[2 * lane + 1] = excl + a;
-    if (lane == 31 && total_out) *total_out = incl;
   }
 }
 
+// Problems with at most this many tiles per level skip the scan launch: each scatter and
+// bucket CTA then sums the few hist entries it needs itself (O(nb * tiles) per CTA, which
+// is less than a launch costs at that size).  Larger problems scan hist once.
+constexpr int kTrScanTiles = 16;
+
+// Exclusive scan, in place, of the nb * tiles counts of one problem (level, b, h), laid out
+// bucket-major: afterwards hist[b][t] is the slot of the first entry of bucket b that tile
+// t holds, i.e. (entries of buckets < b) + (entries of bucket b in tiles < t).  Each thread
+// scans a contiguous run; the runs' totals are scanned by warp 0.  The total (every entry
+// with an in-range key) goes to hist[nb * tiles].  O(nb * tiles) per problem.
+__global__ void __launch_bounds__(kTrThreads) transpose_scan_kernel(TransposeGeo tg, int* __restrict__ ws_hist) {
+  pdl_enter();
+  __shared__ int part[kTrThreads];
+  const int l = blockIdx.x / tg.BH;
+  const int bh = blockIdx.x - l * tg.BH;
+  const TransposeLevel& L = tg.lv[l];
+  const int count = L.nb * L.tiles;
+  int* hist = ws_hist + L.hist_off + (long long)bh * L.hstride;
+  const int tid = threadIdx.x;
+  const int per = (count + kTrThreads - 1) / kTrThreads;
+  const int i0 = min(count, tid * per);
+  const int i1 = min(count, i0 + per);
+  int sum = 0;
+  for (int i = i0; i < i1; ++i) sum += hist[i];
+  part[tid] = sum;
+  __syncthreads();
+  if (tid < 32) {
+    constexpr int kPer = kTrThreads / 32;
+    int acc = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) acc += part[tid * kPer + k];
+    int incl = acc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (tid >= off) incl += o;
+    }
+    int run = incl - acc;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int v = part[tid * kPer + k];
+      part[tid * kPer + k] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  int run = part[tid];
+  for (int i = i0; i < i1; ++i) {
+    const int v = hist[i];
+    hist[i] = run;
+    run += v;
+  }
+  if (tid == kTrThreads - 1) hist[count] = run;  // entries with an in-range key
+}
+
+// SCANNED: hist was scanned by transpose_scan_kernel; otherwise each CTA sums the raw
+// counts it needs (only for problems of at most kTrScanTiles tiles).
+template <bool SCANNED>
 __global__ void __launch_bounds__(kTrThreads) transpose_scatter_kernel(TransposeGeo tg, const int* __restrict__ idx,
                                                                        const int* __restrict__ ws_hist,
                                                                        uint32_t* __restrict__ ws_ent) {
   pdl_enter();
   __shared__ int cnt[kTrWarps][kTrMaxBuckets];
-  __shared__ int tot[kTrMaxBuckets];
-  __shared__ int pre[kTrMaxBuckets];
+  __shared__ int start[kTrMaxBuckets];
+  __shared__ int lower[kTrMaxBuckets];
   const int l = tr_level_of(tg, blockIdx.x, false);
   const TransposeLevel& L = tg.lv[l];
   const int local = blockIdx.x - L.cta_tiles;
   const int bh = local / L.tiles;
   const int t = local - bh * L.tiles;
-  const int* hist = ws_hist + L.hist_off + (long long)bh * L.nb * L.tiles;
+  const int* hist = ws_hist + L.hist_off + (long long)bh * L.hstride;
 
   for (int i = threadIdx.x; i < kTrWarps * kTrMaxBuckets; i += kTrThreads) (&cnt[0][0])[i] = 0;
-  for (int b = threadIdx.x; b < L.nb; b += kTrThreads) {
-    int s = 0, p = 0;
-    for (int tt = 0; tt < L.tiles; ++tt) {
-      const int h = hist[b * L.tiles + tt];
-      s += h;
-      if (tt < t) p += h;
+  if (SCANNED) {
+    for (int b = threadIdx.x; b < L.nb; b += kTrThreads) start[b] = hist[b * L.tiles + t];
+  } else {
+    // start of bucket b in this tile: entries of lower buckets (a scan of the bucket
+    // totals) plus entries of bucket b in earlier tiles
+    for (int b = threadIdx.x; b < L.nb; b += kTrThreads) {
+      int tot = 0, pre = 0;
+      for (int tt = 0; tt < L.tiles; ++tt) {
+        const int h = hist[b * L.tiles + tt];
+        tot += h;
+        if (tt < t) pre += h;
+      }
+      start[b] = tot;
+      lower[b] = pre;
     }
-    tot[b] = s;
-    pre[b] = p;
+    __syncthreads();
+    tr_scan64(start, L.nb);
+    __syncthreads();
+    for (int b = threadIdx.x; b < L.nb; b += kTrThreads) start[b] += lower[b];
   }
   __syncthreads();
-  tr_scan64(tot, L.nb, nullptr);  // tot[b] <- start of bucket b
   const int w = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int seg_begin = t * kTrTile + w * kTrWarpSeg;
@@ -163,9 +235,9 @@ __global__ void __launch_bounds__(kTrThreads) transpose_scatter_kernel(Transpose
   const int* keys = idx + L.ent_off + (long long)bh * L.E;
   tr_warp_bucket_counts(keys, L.E, L.n, L.wshift, seg_begin, seg_end, cnt[w]);
   __syncthreads();
-  // per-warp write cursors: bucket start + earlier tiles + earlier warps of this tile
+  // per-warp write cursors: this tile's first slot of the bucket + earlier warps of this tile
   for (int b = threadIdx.x; b < L.nb; b += kTrThreads) {
-    int run = tot[b] + pre[b];
+    int run = start[b];
 #pragma unroll
     for (int ww = 0; ww < kTrWarps; ++ww) {
       const int c = cnt[ww][b];
@@ -193,6 +265,7 @@ __global__ void __launch_bounds__(kTrThreads) transpose_scatter_kernel(Transpose
   }
 }
 
+template <bool SCANNED>
 __global__ void __launch_bounds__(kTrThreads) transpose_bucket_kernel(TransposeGeo tg, const uint32_t* __restrict__ ws_ent,
                                                                       const int* __restrict__ ws_hist,
                                                                       int* __restrict__ row_ptr, int* __restrict__ col) {
@@ -211,30 +284,39 @@ __global__ void __launch_bounds__(kTrThreads) transpose_bucket_kernel(TransposeG
   const int w = tid >> 5;
   const int lane = tid & 31;
 
-  // bucket start (all entries of lower buckets) and size, from hist
-  const int* hist = ws_hist + L.hist_off + (long long)bh * L.nb * L.tiles;
-  int s_before = 0, s_mine = 0;
-  for (int i = tid; i < (b + 1) * L.tiles; i += kTrThreads) {
-    const int h = hist[i];
-    if (i < b * L.tiles) s_before += h; else s_mine += h;
-  }
+  // bucket start and size: from the scanned hist, its first tile's slot and the next
+  // bucket's (the total for the last bucket); from the raw hist, the sums of the counts of
+  // the lower buckets and of its own
+  const int* hist = ws_hist + L.hist_off + (long long)bh * L.hstride;
+  int start, size;
+  if (SCANNED) {
+    start = hist[b * L.tiles];
+    size = hist[(b + 1) * L.tiles] - start;
+  } else {
+    int s_before = 0, s_mine = 0;
+    for (int i = tid; i < (b + 1) * L.tiles; i += kTrThreads) {
+      const int h = hist[i];
+      if (i < b * L.tiles) s_before += h; else s_mine += h;
+    }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    s_before += __shfl_xor_sync(0xffffffffu, s_before, off);
-    s_mine += __shfl_xor_sync(0xffffffffu, s_mine, off);
-  }
-  if (lane == 0) {
-    red[w][0] = s_before;
-    red[w][1] = s_mine;
+    for (int off = 16; off > 0; off >>= 1) {
+      s_before += __shfl_xor_sync(0xffffffffu, s_before, off);
+      s_mine += __shfl_xor_sync(0xffffffffu, s_mine, off);
+    }
+    if (lane == 0) {
+      red[w][0] = s_before;
+      red[w][1] = s_mine;
+    }
+    __syncthreads();
+    start = size = 0;
+#pragma unroll
+    for (int ww = 0; ww < kTrWarps; ++ww) {
+      start += red[ww][0];
+      size += red[ww][1];
+    }
   }
   for (int i = tid; i < kTrWarps * W; i += kTrThreads) kc[i / W][i % W] = 0;
   __syncthreads();
-  int start = 0, size = 0;
-#pragma unroll
-  for (int ww = 0; ww < kTrWarps; ++ww) {
-    start += red[ww][0];
-    size += red[ww][1];
-  }
 
   // per-key counts, warp-private, each warp on a contiguous segment of the bucket
   const uint32_t* ent = ws_ent + L.ent_off + (long long)bh * L.E + start;

@@ -457,7 +457,7 @@ def _row_verdict(s: np.ndarray, fl: np.ndarray, cand: np.ndarray, selm: np.ndarr
     return "floor" if np.any(inverted & (gap > rel)) else "tie_window"
 
 
-def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5) -> dict:
+def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5, n_valid: int | None = None) -> dict:
     """Check a selection produced elsewhere, level by level from the coarsest down.
 
     At level l the candidates of query a are taken from ``idx_test`` at level l+1 (so a
@@ -468,6 +468,8 @@ def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5) ->
     Returns counts: exact rows, rows accepted by the relative window alone
     (``tie_window``), rows that needed the fp32 bound of some pair (``floor_used``, also
     counted in ``tie_window``), bad rows, and the first few bad rows for diagnosis.
+    ``n_valid`` (a padded sequence): only the real tokens of each level, index < ceil(n_valid
+    / 16^l), are candidates (the padded-sequence reading in ``llsa_padded``).
     """
     L = len(q_pyr)
     res = {"rows": 0, "exact": 0, "tie_window": 0, "floor_used": 0, "bad": 0, "bad_examples": []}
@@ -484,6 +486,9 @@ def check_selection(q_pyr, k_pyr, idx_test, topk: int, rel_tol: float = 1e-5) ->
                 else:
                     groups = [(np.arange(BLOCK * g, BLOCK * (g + 1)), children(idx_test[lev][b, h, g]))
                               for g in range(n // BLOCK)]
+                if n_valid is not None:
+                    real = -(-n_valid // BLOCK ** lev)
+                    groups = [(qrows, cand[cand < real]) for qrows, cand in groups]
                 for qrows, cand in groups:
                     s = selection_scores(qs[qrows], ks[cand])
                     floor = dot_error_floor(qs[qrows], ks[cand])

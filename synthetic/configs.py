@@ -1,4 +1,4 @@
-"""The five synthetic LLSA workloads, by shape.
+"""The synthetic LLSA workloads, by shape.
 
 Each workload is a non-causal multi-head attention problem over a square pixel
 grid whose tokens are laid out in quadtree (Z) order, as the LLSA README's token
@@ -55,10 +55,13 @@ WORKLOADS = {w.name: w for w in (
                    qk_kind="smooth", backward=True),
     WorkloadConfig(5, "scaleout-262144", B=1, H=6, N=262144, D=64, levels=3, topk=16, dtype="bf16",
                    qk_kind="smooth", backward=False),
+    # the headline geometry with 128-channel heads (DiT-B/L/XL-class head width)
+    WorkloadConfig(6, "headline-65536-d128", B=1, H=6, N=65536, D=128, levels=3, topk=8, dtype="bf16",
+                   qk_kind="smooth", backward=True),
 )}
 
 
 def workload(name: str) -> WorkloadConfig:
     """The workload of that name (tiny-f32, dit-s-4096, two-level-16384, headline-65536,
-    scaleout-262144)."""
+    scaleout-262144, headline-65536-d128)."""
     return WORKLOADS[name]

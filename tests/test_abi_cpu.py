@@ -56,7 +56,8 @@ def shape(**kw):
     (dict(N=2048), 1),                 # N < 16^L
     (dict(B=0), 1),
     (dict(dtype=7), 1),
-    (dict(D=128), 2),                  # legal, not built
+    (dict(D=128), 0),                  # D = 128 is built
+    (dict(D=96), 2),                   # other head widths: legal, not built
     (dict(block=32), 2),
     (dict(levels=5, N=1 << 20, topk=1), 2),
     (dict(N=1 << 21), 2),
@@ -215,3 +216,18 @@ def test_binding_refuses_tensors_the_kernels_would_misread():
             api.llsa_forward(shape, **args)
     with pytest.raises(ValueError, match="dst: dtype"):
         api.llsa_token_permute(shape, act(), act(torch.float32))
+
+
+@pytest.mark.parametrize("limit", [0, -5, 4_000_000_001])
+def test_bounded_wait_check_rejects_limits_outside_range(lib, limit):
+    assert lib.llsa_check_bounded_wait(limit, None) == 1   # LLSA_ERR_INVALID_ARG, nothing launched
+
+
+def test_buffer_sizes_scale_with_head_width(lib):
+    s64 = api.make_shape(1, 6, 65536, 64, 8, 3, 0)
+    s128 = api.make_shape(1, 6, 65536, 128, 8, 3, 0)
+    assert api.llsa_pyramid_elems(s128) == 2 * api.llsa_pyramid_elems(s64) == 2 * 6 * (4096 + 256 + 16) * 64
+    assert api.llsa_index_elems(s128) == api.llsa_index_elems(s64)
+    assert api.llsa_transpose_workspace_bytes(s128) == api.llsa_transpose_workspace_bytes(s64)
+    # Delta and the dK/dV order do not grow with D; the coarse partials and gradients double
+    assert api.llsa_backward_workspace_bytes(s128) > api.llsa_backward_workspace_bytes(s64)

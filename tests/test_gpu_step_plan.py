@@ -139,3 +139,31 @@ def test_plan_headline_matches_serialized_calls():
         assert api.llsa_device_status() == 0
         assert_same(outputs(buf), ref)
     plan.close()
+
+
+@pytest.mark.parametrize("B,H,N,K,L,D", [
+    (1, 2, 65536, 8, 3, 64),     # the headline geometry: levels 3 pooled with the coarsest Top-K
+    (1, 1, 65536, 4, 4, 64),     # four levels, n_4 = 1
+    (2, 1, 16384, 16, 2, 128),   # two levels, D = 128, K = 16
+    (1, 2, 4096, 2, 2, 64),      # n_2 = 16
+])
+def test_fused_pyramid_and_selection_equal_the_separate_launches(B, H, N, K, L, D):
+    """In a step the pyramid and every selection level run as one cooperative launch
+    (pyramid_select); its pyramid, selection and all results are bit-identical to the
+    separate pyramid and selection kernels of the five calls."""
+    inputs = make_inputs(B, H, N, D, "bf16", "smooth", 150 + L)
+    ref = run_gpu(B, H, N, D, K, L, "bf16", inputs)
+    shape = api.make_shape(B, H, N, D, K, L, torch.bfloat16)
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    buf = api.LLSABuffers.allocate(shape, "cuda", torch.bfloat16)
+    with api.LaunchTrace(64) as tr:
+        api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+    names = [n for n, _ in tr.launches()]
+    assert api.llsa_device_status() == 0
+    assert names[0] == "pyramid_select" and "select" not in names and "pyramid_l12" not in names, names
+    for name, got in (("q_pyr", buf.q_pyr), ("k_pyr", buf.k_pyr), ("v_pyr", buf.v_pyr)):
+        want = np.concatenate([x.ravel() for x in ref[name]])
+        assert np.array_equal(got.cpu().numpy().view(np.uint32), want.view(np.uint32)), name
+    assert np.array_equal(buf.idx.cpu().numpy(), np.concatenate([x.ravel() for x in ref["idx"]]))
+    for k in KEYS:
+        assert np.array_equal(getattr(buf, k).float().cpu().numpy(), ref[k]), k

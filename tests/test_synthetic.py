@@ -61,6 +61,7 @@ def test_smooth_fields_are_spatially_smooth():
 
 
 def test_config_table():
-    assert [w.N for w in WORKLOADS.values()] == [1024, 4096, 16384, 65536, 262144]
+    assert [w.N for w in WORKLOADS.values()] == [1024, 4096, 16384, 65536, 262144, 65536]
+    assert [w.D for w in WORKLOADS.values()] == [64, 64, 64, 64, 64, 128]
     assert WORKLOADS["headline-65536"].level_sizes() == [65536, 4096, 256, 16]
     assert WORKLOADS["headline-65536"].kv_len == 144 and WORKLOADS["scaleout-262144"].kv_len == 288
