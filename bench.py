@@ -267,6 +267,15 @@ def enrichment(args) -> dict:
     return dict(log_bias=args.log_bias, all_top=args.all_top, level1=args.level1)
 
 
+def to_grid_order(host: dict, cfg) -> dict:
+    """The synthetic tokens (generated in quadtree order) moved to the row-major order of the
+    square grid: what a caller that passes LLSA_FLAG_GRID_ORDER hands the library."""
+    import torch
+    from synthetic import morton_order
+    perm = torch.from_numpy(morton_order(cfg.grid))   # raster position of each Z position
+    return {k: torch.empty_like(v).index_copy_(2, perm, v) for k, v in host.items()}
+
+
 def enrichment_text(args) -> str:
     parts = ["log-count bias ln(16^l) on coarse scores" if args.log_bias else "unit weight"]
     if args.all_top:
@@ -418,9 +427,12 @@ def run_ours(args):
     cfg = WORKLOADS[args.workload]
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     host = make_config_inputs(cfg, with_do=True)
+    if args.grid_order:
+        host = to_grid_order(host, cfg)
     pinned = {k: v.pin_memory() for k, v in host.items()}
     dev = {k: v.cuda(non_blocking=True) for k, v in pinned.items()}
-    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, **enrichment(args))
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, grid_order=args.grid_order,
+                           one_launch_select=args.one_launch_select, **enrichment(args))
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     stream = torch.cuda.current_stream()
 
@@ -709,8 +721,12 @@ def run_ours(args):
                    "kv_len": 16 * cfg.topk + (cfg.topk if args.level1 else 0) + coarse_entries(cfg, args.all_top),
                    "step": "pyramid + select + forward + index transpose + backward",
                    "enrichment": enrichment_text(args),
+                   "token_order": ("row-major grid, read and written through the quadtree order in the kernels "
+                                   "(LLSA_FLAG_GRID_ORDER)" if args.grid_order else "quadtree (Z) order"),
                    "launch": ("K steps as one CUDA graph (llsa_plan_create repeat=K), kernels chained by "
-                              "programmatic dependent launch; transpose on a second stream"),
+                              "programmatic dependent launch; transpose on a second stream"
+                              + ("; pyramid and selection as one cooperative launch (LLSA_FLAG_ONE_LAUNCH_SELECT)"
+                                 if args.one_launch_select else "")),
                    "kernel_times_from": ("a second plan of the same K steps with trace events around every "
                                          f"kernel, launched after the timed one: {traced_ms_per_step:.4f} ms per step"),
                    "parallelism": f"dp{world}: independent replicas, no collective",
@@ -835,7 +851,8 @@ def run_profile(args):
     cfg = WORKLOADS[args.workload]
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     dev = {k: v.cuda() for k, v in make_config_inputs(cfg, with_do=True).items()}
-    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, **enrichment(args))
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype,
+                           one_launch_select=args.one_launch_select, **enrichment(args))
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     for _ in range(args.warmup + args.steps):
         api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
@@ -867,6 +884,10 @@ def main():
                     help="the all-coarsest enrichment variant (every level-L token in every list)")
     ap.add_argument("--level1", action="store_true",
                     help="the level-1 enrichment variant (each selected block's mean token in the list)")
+    ap.add_argument("--grid-order", action="store_true",
+                    help="inputs and outputs in row-major grid order (LLSA_FLAG_GRID_ORDER)")
+    ap.add_argument("--one-launch-select", action="store_true",
+                    help="pyramid and selection as one cooperative launch (LLSA_FLAG_ONE_LAUNCH_SELECT)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

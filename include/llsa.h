@@ -101,6 +101,28 @@ typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
  * 16 tokens through the mean-pool adjoint.  Combines with the other flags, at any levels.
  */
 #define LLSA_FLAG_LEVEL1 4
+/*
+ * Token order (LLSA GitHub README, token reordering example: image tokens should be in the
+ * quadtree order, so that every 16-token block is a 4 x 4 patch and every level-l pooled
+ * token a 4^l x 4^l patch).  With LLSA_FLAG_GRID_ORDER, q, k, v, dO, o, dq, dk, dv and lse
+ * are in the row-major order of a square G x G token grid (N = G * G, G a power of two,
+ * N >= 256); the kernels read and write them in place through that order, so no separate
+ * permutation pass is needed.  The pyramid, idx and the CSR refer to quadtree positions:
+ * the results equal those of the same call on inputs permuted by llsa_token_permute, with
+ * its outputs permuted back.  Not combined with padding (n_valid).
+ */
+#define LLSA_FLAG_GRID_ORDER 8
+/*
+ * Launch shape only; results are bit-identical with and without it.  With
+ * LLSA_FLAG_ONE_LAUNCH_SELECT, llsa_train_step and plans run the pyramid and every selection
+ * level as one cooperative persistent kernel whose phases are separated by grid-wide barriers,
+ * instead of one launch per stage chained by programmatic dependent launch.  It applies to
+ * bf16 inputs with levels >= 2, n_L <= 64 and topk in {2, 4, 8, 16}; elsewhere, and in the
+ * separate calls, the flag changes nothing.  Off by default: on one B200 the chained launches
+ * are faster (the forward can start its set-up while they drain, but not while a cooperative
+ * kernel does).
+ */
+#define LLSA_FLAG_ONE_LAUNCH_SELECT 16
 
 typedef struct {
   int32_t B, H, N, D;

@@ -42,6 +42,8 @@ class LLSAShape(ctypes.Structure):
 LLSA_FLAG_LOG_BIAS = 1
 LLSA_FLAG_ALL_TOP = 2
 LLSA_FLAG_LEVEL1 = 4
+LLSA_FLAG_GRID_ORDER = 8
+LLSA_FLAG_ONE_LAUNCH_SELECT = 16
 
 
 _SP = ctypes.POINTER(LLSAShape)

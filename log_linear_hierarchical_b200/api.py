@@ -28,14 +28,20 @@ class LLSAError(RuntimeError):
 
 
 def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16,
-               log_bias: bool = False, all_top: bool = False, level1: bool = False, n_valid: int = 0) -> LLSAShape:
+               log_bias: bool = False, all_top: bool = False, level1: bool = False, n_valid: int = 0,
+               grid_order: bool = False, one_launch_select: bool = False) -> LLSAShape:
     """``log_bias``: the log-count enrichment variant (LLSA_FLAG_LOG_BIAS); ``all_top``: the
     all-coarsest variant (LLSA_FLAG_ALL_TOP); ``level1``: the selected blocks' level-1 pooled
     tokens join the list (LLSA_FLAG_LEVEL1).  Any combination may be set.  ``n_valid``: the
-    real tokens of a padded sequence (positions from n_valid on are padding; 0 = none)."""
+    real tokens of a padded sequence (positions from n_valid on are padding; 0 = none).
+    ``grid_order``: token rows are in the row-major order of a square grid
+    (LLSA_FLAG_GRID_ORDER); the path reads and writes them through its quadtree order.
+    ``one_launch_select``: a step runs the pyramid and selection as one cooperative launch
+    (LLSA_FLAG_ONE_LAUNCH_SELECT; same results)."""
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     flags = ((_lib.LLSA_FLAG_LOG_BIAS if log_bias else 0) | (_lib.LLSA_FLAG_ALL_TOP if all_top else 0)
-             | (_lib.LLSA_FLAG_LEVEL1 if level1 else 0))
+             | (_lib.LLSA_FLAG_LEVEL1 if level1 else 0) | (_lib.LLSA_FLAG_GRID_ORDER if grid_order else 0)
+             | (_lib.LLSA_FLAG_ONE_LAUNCH_SELECT if one_launch_select else 0))
     return LLSAShape(B, H, N, D, block, topk, levels, code, flags, n_valid)
 
 

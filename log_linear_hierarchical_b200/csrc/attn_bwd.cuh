@@ -27,7 +27,10 @@ namespace llsa {
 
 // Backward workspace layout (fp32, offsets in floats, each 64-float aligned).
 struct BwdWorkspace {
-  long long delta;          // [B*H*N]
+  // bf16 path: per query block [B*H*n_1][32] = its 16 LSE * log2(e) then its 16 Delta, in
+  // the block's shared-memory tile-row order (written by dQ; one 128-byte copy per pair in
+  // the key-major kernels).  fp32 path: Delta [B*H*N] in the first half.
+  long long lsd;
   long long part_k, part_v; // [B*H*n_2][C][64]
   long long cg_k, cg_v;     // coarse gradients, level-major [l=2..L][B*H*n_l][64]
   long long cg_off[kMaxLevels + 1];
@@ -53,8 +56,8 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   auto up = [](long long x) { return (x + 63) & ~63LL; };
   BwdWorkspace w{};
   long long off = 0;
-  w.delta = off;
-  off = up(off + (long long)g.BH * g.N);
+  w.lsd = off;
+  off = up(off + 2LL * g.BH * g.N);
   const long long parts = g.L >= 2 ? (long long)g.BH * g.n[2] * g.coarse * g.D : 0;
   w.part_k = off;
   off = up(off + parts);
@@ -101,12 +104,13 @@ template <int D, bool MASK, bool POOL = false>
 __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const uint32_t (&df)[D / 16][4],
                                          uint32_t ktile, uint32_t vtile, int valid, float scale_log2,
                                          const float (&lse2)[2], const float (&delta)[2], float (&dq)[D / 8][4],
-                                         const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f) {
+                                         const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
+                                         int perm = 0) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  mma_a_bt<D>(s, qf, ktile);
-  mma_a_bt<D>(dp, df, vtile);
+  mma_a_bt<D>(s, qf, ktile, perm);
+  mma_a_bt<D>(dp, df, vtile, perm);
   float pds[2] = {0.f, 0.f};  // pooled entry's dS / 16, rows r0 and r0 + 8
   if (POOL) {
     float t[2], u[2];
@@ -131,14 +135,14 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const 
       ds[n][e] = POOL ? fmaf(p, dp[n][e] - delta[r], pds[r]) : p * (dp[n][e] - delta[r]);
     }
   mma_a_b<D>(dq, pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]), pack_bf16(ds[1][0], ds[1][1]),
-             pack_bf16(ds[1][2], ds[1][3]), ktile);
+             pack_bf16(ds[1][2], ds[1][3]), ktile, perm);
 }
 
 // Same CTA shape as the forward: 4 warps x 4 query blocks, coarse KV staged once per CTA.
-// POOL: the level-1 variant (see dq_chunk).  PAD: a padded sequence -- the fine tile that
-// holds the last real token masks its padding keys; padding queries (zero Q and dO rows,
-// O = 0, LSE = 0) get dS = 0 and so dQ = 0 and Delta = 0 without a mask.
-template <int D, int STAGES, bool POOL, bool PAD>
+// POOL: the level-1 variant (see dq_chunk).  LAYOUT (see Layout): under kPadded the fine
+// tile that holds the last real token masks its padding keys; padding queries (zero Q and
+// dO rows, O = 0, LSE = 0) get dS = 0 and so dQ = 0 and Delta = 0 without a mask.
+template <int D, int STAGES, bool POOL, int LAYOUT>
 __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
@@ -148,6 +152,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
   // the coarse tiles come from the pyramid and the coarser selection levels, two or more
   // kernels back, so they are staged before waiting for the kernel ahead (see pdl_wait)
   extern __shared__ uint8_t dq_smem_raw[];
+  constexpr bool PAD = LAYOUT == kPadded;
+  constexpr int PERM = LAYOUT == kGrid ? 1 : 0;
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
   const int lane = lane_id();
@@ -200,17 +206,17 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * TB;
     mbar_expect_tx(bar, 2 * TB);
-    tma_load_tile<D>(dst, &tm_k, g, row, bar);
-    tma_load_tile<D>(dst + TB, &tm_v, g, row, bar);
+    tma_load_tile<D, LAYOUT>(dst, &tm_k, g, row, bar);
+    tma_load_tile<D, LAYOUT>(dst + TB, &tm_v, g, row, bar);
   };
   auto issue_qd = [&](int i) {
     const uint32_t bar = bar_qd + 8 * (i & 1);
     const int row = (first + i) * kBlock;
     const uint32_t dst = qd + (i & 1) * 2 * TB;
     mbar_expect_tx(bar, 2 * TB + kBlock * 4);
-    tma_load_tile<D>(dst, &tm_q, g, row, bar);
-    tma_load_tile<D>(dst + TB, &tm_do, g, row, bar);
-    bulk_load(smem_u32(slse + (i & 1) * kBlock), lse + row, kBlock * 4, bar);
+    tma_load_tile<D, LAYOUT>(dst, &tm_q, g, row, bar);
+    tma_load_tile<D, LAYOUT>(dst + TB, &tm_do, g, row, bar);
+    bulk_load_block_rows<LAYOUT>(smem_u32(slse + (i & 1) * kBlock), lse, g, row, bar);
   };
   // the level-1 selection (two kernels back) and K, V are ready: the first K/V tiles are
   // requested before waiting; Q/dO/LSE and O follow the forward, the kernel ahead
@@ -222,13 +228,15 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 
   bool ok = true;
   int next_seq = 0, next_q = 0;
-  // O rows of a block (lane: row lane/2, channels (lane%2) * D/2 onwards).  At D = 64 they
-  // are loaded one block ahead; at D = 128 (twice the registers) when the block starts.
+  // O rows of a block (lane: shared-memory tile row lane/2, channels (lane%2) * D/2 onwards;
+  // the row's token is tile_row of it).  At D = 64 they are loaded one block ahead; at
+  // D = 128 (twice the registers) when the block starts.
   constexpr int OC = D / 16;  // 16-byte chunks per lane
   constexpr bool kPrefetchO = D == 64;
   auto load_o = [&](int i, uint4 (&dst)[OC]) {
-    const uint4* orow =
-        reinterpret_cast<const uint4*>(o + ((long long)(first + i) * kBlock + (lane >> 1)) * D + (lane & 1) * (D / 2));
+    const int bhi = div_n1(g, first + i);
+    const long long orow_i = token_row<LAYOUT>(g, bhi, (first + i - bhi * n1) * kBlock + tile_row(lane >> 1, PERM));
+    const uint4* orow = reinterpret_cast<const uint4*>(o + orow_i * D + (lane & 1) * (D / 2));
 #pragma unroll
     for (int c = 0; c < OC; ++c) dst[c] = __ldg(orow + c);
   };
@@ -252,8 +260,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     const uint32_t qt = qd + (i & 1) * 2 * TB;
     const uint32_t dt = qt + TB;
     uint32_t qf[D / 16][4], df[D / 16][4];
-    load_a_frags<D>(qt, qf);
-    load_a_frags<D>(dt, df);
+    load_a_frags<D>(qt, qf, PERM);
+    load_a_frags<D>(dt, df, PERM);
     // Delta_r = sum_d dO[r][d] * O[r][d] (O from registers, dO from the staged tile)
     float dlt;
     {
@@ -276,11 +284,15 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
         }
       }
       dlt = acc + __shfl_xor_sync(0xffffffffu, acc, 1);
-      if (h == 0) ws[W.delta + (long long)gb * kBlock + r] = dlt;
+      // the block's record for the key-major kernels: lanes 0-15 LSE * log2(e), 16-31 Delta
+      const float drow = __shfl_sync(0xffffffffu, dlt, 2 * (lane & 15));
+      ws[W.lsd + (long long)gb * 2 * kBlock + lane] = lane < kBlock ? slse[(i & 1) * kBlock + lane] * kLog2e : drow;
     }
+    // Delta and LSE are in shared-memory tile-row order: row r0 of the fragments is tile row p0
     const int r0 = lane >> 2;
-    const float delta[2] = {__shfl_sync(0xffffffffu, dlt, 2 * r0), __shfl_sync(0xffffffffu, dlt, 2 * r0 + 16)};
-    const float lse2[2] = {slse[(i & 1) * kBlock + r0] * kLog2e, slse[(i & 1) * kBlock + r0 + 8] * kLog2e};
+    const int p0 = tile_row(r0, PERM);
+    const float delta[2] = {__shfl_sync(0xffffffffu, dlt, 2 * p0), __shfl_sync(0xffffffffu, dlt, 2 * p0 + 16)};
+    const float lse2[2] = {slse[(i & 1) * kBlock + p0] * kLog2e, slse[(i & 1) * kBlock + p0 + 8] * kLog2e};
 
     float dq[D / 8][4];
 #pragma unroll
@@ -298,7 +310,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
                           P.scale_log2, lse2, delta, dq);
       else
         dq_chunk<D, false, POOL>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
-                                 pool_log_bias<D>(g));
+                                 pool_log_bias<D>(g), PERM);
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }
@@ -307,7 +319,10 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
       dq_chunk<D, true>(qf, df, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock),
                      P.scale_log2, lse2, delta, dq, &g, cc * kBlock);
     __syncwarp();
-    store_tile_bf16<D>(dq, P.scale, P.scale, qt, dq_out + (long long)gb * kBlock * D);
+    {
+      const int bhi = div_n1(g, gb);
+      store_tile_bf16<D, LAYOUT>(dq, P.scale, P.scale, qt, dq_out, g, bhi, (gb - bhi * n1) * kBlock);
+    }
   }
   if (!ok) {
     for (int seq = next_seq; seq < min(total_loads, next_seq + STAGES); ++seq)
@@ -339,27 +354,33 @@ __host__ __device__ constexpr bool kv_frags_in_regs() {
 
 // kvalid < 16: the key tile holds the last real token of a padded sequence, and its rows
 // from kvalid on are padding (zero rows) whose P^T and dS^T are masked to 0.
+// kvperm, qperm: the tile_row permutations of the key tile and of the query block's tiles.
+// lsd: the query block's record (16 LSE * log2(e), then 16 Delta, in the shared-memory row
+// order of its tiles).
 template <int D, bool BIAS = false, bool POOL = false>
 __device__ __forceinline__ void kv_scores(const uint32_t (&kf)[D / 16][4], const uint32_t (&vf)[D / 16][4],
-                                          uint32_t kvtile, uint32_t qt, uint32_t dt, const float* ls,
-                                          const float* dl, float scale_log2, float (&pt)[2][4], float (&dst)[2][4],
-                                          const float (&kb)[2], float pool_bias, int kvalid) {
+                                          uint32_t kvtile, uint32_t qt, uint32_t dt, const float* lsd,
+                                          float scale_log2, float (&pt)[2][4], float (&dst)[2][4],
+                                          const float (&kb)[2], float pool_bias, int kvalid, int kvperm,
+                                          int qperm) {
   const int c2 = 2 * (lane_id() & 3);
   float st[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dpt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   if constexpr (kv_frags_in_regs<D>()) {
-    mma_a_bt<D>(st, kf, qt);   // S^T: rows = keys, cols = queries
-    mma_a_bt<D>(dpt, vf, dt);  // dP^T
+    mma_a_bt<D>(st, kf, qt, qperm);   // S^T: rows = keys, cols = queries
+    mma_a_bt<D>(dpt, vf, dt, qperm);  // dP^T
   } else {
-    mma_at_bt<D>(st, kvtile, qt);
-    mma_at_bt<D>(dpt, kvtile + tile_bytes<D>(), dt);
+    mma_at_bt<D>(st, kvtile, qt, kvperm, qperm);
+    mma_at_bt<D>(dpt, kvtile + tile_bytes<D>(), dt, kvperm, qperm);
   }
-  // this lane's four query columns: c2, c2 + 1 (n = 0) and c2 + 8, c2 + 9 (n = 1)
-  const float2 l0 = *reinterpret_cast<const float2*>(ls + c2);
-  const float2 l1 = *reinterpret_cast<const float2*>(ls + 8 + c2);
-  const float2 d0 = *reinterpret_cast<const float2*>(dl + c2);
-  const float2 d1 = *reinterpret_cast<const float2*>(dl + 8 + c2);
-  const float lq[2][2] = {{l0.x * kLog2e, l0.y * kLog2e}, {l1.x * kLog2e, l1.y * kLog2e}};
+  // this lane's four query columns: c2, c2 + 1 (n = 0) and c2 + 8, c2 + 9 (n = 1); the tile
+  // row permutation keeps bit 0, so each pair stays adjacent
+  const int pc = tile_row(c2, qperm);
+  const float2 l0 = *reinterpret_cast<const float2*>(lsd + pc);
+  const float2 l1 = *reinterpret_cast<const float2*>(lsd + 8 + pc);
+  const float2 d0 = *reinterpret_cast<const float2*>(lsd + kBlock + pc);
+  const float2 d1 = *reinterpret_cast<const float2*>(lsd + kBlock + 8 + pc);
+  const float lq[2][2] = {{l0.x, l0.y}, {l1.x, l1.y}};
   const float dq[2][2] = {{d0.x, d0.y}, {d1.x, d1.y}};
   float pa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, da[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // pooled p/16, dS/16
   if (POOL) {
@@ -419,19 +440,19 @@ __device__ __forceinline__ void kv_scores(const uint32_t (&kf)[D / 16][4], const
 // error grows).
 template <int D>
 __device__ __forceinline__ void kv_accumulate(const float (&pt)[2][4], const float (&dst)[2][4], uint32_t qt,
-                                              uint32_t dt, float (&dk)[D / 8][4], float (&dv)[D / 8][4]) {
+                                              uint32_t dt, float (&dk)[D / 8][4], float (&dv)[D / 8][4], int qperm) {
   uint32_t phi[4], plo[4];
   split_bf16(pt[0][0], pt[0][1], phi[0], plo[0]);
   split_bf16(pt[0][2], pt[0][3], phi[1], plo[1]);
   split_bf16(pt[1][0], pt[1][1], phi[2], plo[2]);
   split_bf16(pt[1][2], pt[1][3], phi[3], plo[3]);
-  mma_a2_b<D>(dv, phi, plo, dt);
+  mma_a2_b<D>(dv, phi, plo, dt, qperm);
   uint32_t dhi[4], dlo[4];
   split_bf16(dst[0][0], dst[0][1], dhi[0], dlo[0]);
   split_bf16(dst[0][2], dst[0][3], dhi[1], dlo[1]);
   split_bf16(dst[1][0], dst[1][1], dhi[2], dlo[2]);
   split_bf16(dst[1][2], dst[1][3], dhi[3], dlo[3]);
-  mma_a2_b<D>(dk, dhi, dlo, qt);
+  mma_a2_b<D>(dk, dhi, dlo, qt, qperm);
 }
 
 // Per-warp shared memory of the key-major kernels: the key tile's K and V, then a ring of
@@ -451,15 +472,16 @@ __host__ __device__ inline CtaSmem kv_smem(int nwarps) {
 // `bar_tile` is non-zero the key tile is still arriving on that mbarrier (phase 0) and is
 // waited for after the first pair loads are issued.  Returns false (after draining the
 // copies in flight) if a wait timed out.
-template <int D, int STAGES, bool BIAS = false, bool POOL = false, class PairBlock>
+template <int D, int STAGES, int LAYOUT, bool BIAS = false, bool POOL = false, class PairBlock>
 __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* tm_q, const CUtensorMap* tm_do,
-                                          const float* __restrict__ lse, const float* __restrict__ delta,
-                                          uint32_t kvtile, uint32_t bar_tile, uint32_t ring, float* sls, float* sdl,
+                                          const float* __restrict__ lsd, uint32_t kvtile, uint32_t bar_tile,
+                                          uint32_t ring, float* slsd,
                                           uint32_t bar_ring, int npairs, PairBlock pair_block, float scale_log2,
                                           float (&dk)[D / 8][4], float (&dv)[D / 8][4],
                                           const float (&kbias)[2] = {0.f, 0.f}, float pool_bias = 0.f,
-                                          int kvalid = kBlock) {
+                                          int kvalid = kBlock, int kvperm = 0) {
   constexpr int TB = tile_bytes<D>();
+  constexpr int qperm = LAYOUT == kGrid ? 1 : 0;
   const int lane = lane_id();
   // called by the whole warp (pair_block may shuffle); lane 0 issues the copies
   auto issue_pair = [&](int i) {
@@ -469,10 +491,9 @@ __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* 
       const uint32_t bar = bar_ring + 8 * stage;
       const uint32_t dst = ring + stage * 2 * TB;
       mbar_expect_tx(bar, 2 * TB + 2 * kBlock * 4);
-      tma_load_tile<D>(dst, tm_q, g, row, bar);
-      tma_load_tile<D>(dst + TB, tm_do, g, row, bar);
-      bulk_load(smem_u32(sls + stage * kBlock), lse + row, kBlock * 4, bar);
-      bulk_load(smem_u32(sdl + stage * kBlock), delta + row, kBlock * 4, bar);
+      tma_load_tile<D, LAYOUT>(dst, tm_q, g, row, bar);
+      tma_load_tile<D, LAYOUT>(dst + TB, tm_do, g, row, bar);
+      bulk_load(smem_u32(slsd + stage * 2 * kBlock), lsd + 2LL * row, 2 * kBlock * 4, bar);
     }
   };
   for (int i = 0; i < min(STAGES, npairs); ++i) issue_pair(i);
@@ -482,8 +503,8 @@ __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* 
   }
   uint32_t kf[D / 16][4], vf[D / 16][4];
   if constexpr (kv_frags_in_regs<D>()) {
-    load_a_frags<D>(kvtile, kf);
-    load_a_frags<D>(kvtile + TB, vf);
+    load_a_frags<D>(kvtile, kf, kvperm);
+    load_a_frags<D>(kvtile + TB, vf, kvperm);
   }
 #pragma unroll kKvUnroll
   for (int i = 0; i < npairs; ++i) {
@@ -494,9 +515,9 @@ __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* 
     }
     const uint32_t qt = ring + stage * 2 * TB;
     float pt[2][4], dst[2][4];
-    kv_scores<D, BIAS, POOL>(kf, vf, kvtile, qt, qt + TB, sls + stage * kBlock, sdl + stage * kBlock, scale_log2,
-                             pt, dst, kbias, pool_bias, kvalid);
-    kv_accumulate<D>(pt, dst, qt, qt + TB, dk, dv);
+    kv_scores<D, BIAS, POOL>(kf, vf, kvtile, qt, qt + TB, slsd + stage * 2 * kBlock, scale_log2, pt, dst, kbias,
+                             pool_bias, kvalid, kvperm, qperm);
+    kv_accumulate<D>(pt, dst, qt, qt + TB, dk, dv, qperm);
     __syncwarp();
     if (i + STAGES < npairs) issue_pair(i + STAGES);
   }
@@ -505,14 +526,13 @@ __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* 
 
 // Coarse-token partial gradients.  One warp per (level-2 group, 16-token coarse tile): the
 // pairs are the group's 16 query blocks.  Rows >= C of the last tile are padding and are not
-// written.  Output: part_k / part_v [group][C][D] fp32 (dK unscaled).
-template <int D, int STAGES>
+// written.  Output: part_k / part_v [group][C][D] fp32 (dK unscaled).  LAYOUT: see Layout.
+template <int D, int STAGES, int LAYOUT>
 __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                   const __grid_constant__ CUtensorMap tm_do,
                                                                   AttnParams P, const float* __restrict__ k_pyr,
                                                                   const float* __restrict__ v_pyr,
                                                                   const int* __restrict__ idx,
-                                                                  const float* __restrict__ lse,
                                                                   float* __restrict__ ws) {
   // coarse rows are staged before waiting (two or more kernels back; see pdl_wait)
   extern __shared__ uint8_t co_smem_raw[];
@@ -531,9 +551,8 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
   uint8_t* base = align1024(co_smem_raw);
   const uint32_t kvt = smem_u32(cs.tiles(base, 0));
   const uint32_t ring = kvt + 2 * TB;
-  float* sls = reinterpret_cast<float*>(cs.tail(base, 0));
-  float* sdl = sls + STAGES * kBlock;
-  const uint32_t bar_ring = smem_u32(sdl + STAGES * kBlock);
+  float* slsd = reinterpret_cast<float*>(cs.tail(base, 0));  // [STAGES][32] LSE + Delta records
+  const uint32_t bar_ring = smem_u32(slsd + STAGES * 2 * kBlock);
 
   // stage this tile's 16 coarse K and V rows (bf16) like the forward does
   {
@@ -580,11 +599,11 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
     const int r0 = tile * kBlock + (lane >> 2);
     const float kb[2] = {r0 < g.coarse ? coarse_log_bias(g, r0) * sqrt_d<D>() : 0.f,
                          r0 + 8 < g.coarse ? coarse_log_bias(g, r0 + 8) * sqrt_d<D>() : 0.f};
-    ok = kv_stream<D, STAGES, true>(g, &tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
-                                 [&](int i) { return first_block + i; }, P.scale_log2, dk, dv, kb);
+    ok = kv_stream<D, STAGES, LAYOUT, true>(g, &tm_q, &tm_do, ws + W.lsd, kvt, 0u, ring, slsd, bar_ring, kBlock,
+                                            [&](int i) { return first_block + i; }, P.scale_log2, dk, dv, kb);
   } else {
-    ok = kv_stream<D, STAGES>(g, &tm_q, &tm_do, lse, ws + W.delta, kvt, 0u, ring, sls, sdl, bar_ring, kBlock,
-                           [&](int i) { return first_block + i; }, P.scale_log2, dk, dv);
+    ok = kv_stream<D, STAGES, LAYOUT>(g, &tm_q, &tm_do, ws + W.lsd, kvt, 0u, ring, slsd, bar_ring, kBlock,
+                                      [&](int i) { return first_block + i; }, P.scale_log2, dk, dv);
   }
   if (!ok) return;
   const int r0 = lane >> 2;
@@ -901,13 +920,12 @@ __global__ void __launch_bounds__(kOrdThreads) dkdv_order_scatter_kernel(Geometr
 // whose output (the coarse-token gradients) only the epilogue reads; everything the main
 // loop reads was complete before that kernel could start, so the wait for it is deferred
 // to the epilogue and the main loop overlaps the reduction.
-template <int D, int STAGES, bool POOL>
+template <int D, int STAGES, bool POOL, int LAYOUT>
 __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, AttnParams P,
-    const float* __restrict__ lse, const int* __restrict__ row_ptr, const int* __restrict__ col,
-    const float* __restrict__ ws, __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out,
-    int coarse_late) {
+    const int* __restrict__ row_ptr, const int* __restrict__ col, const float* __restrict__ ws,
+    __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out, int coarse_late) {
   if (!coarse_late) pdl_wait();
   pdl_launch_dependents();
   extern __shared__ uint8_t dkv_smem_raw[];
@@ -980,19 +998,17 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
             pk[c] = pack_bf16(ak[2 * c], ak[2 * c + 1]);
             pv[c] = pack_bf16(av[2 * c], av[2 * c + 1]);
           }
-          const long long row0 = (long long)bh * g.N + (long long)j * kBlock;
-          const int kvalid = g.nv - j * kBlock;  // padding positions get 0
+          const int kvalid = LAYOUT == kPadded ? g.nv - j * kBlock : kBlock;  // padding positions get 0
 #pragma unroll
           for (int t = 0; t < kBlock; ++t) {
             const bool real = t < kvalid;
+            const long long row = token_row<LAYOUT>(g, bh, j * kBlock + t);
             if constexpr (V == 2) {
-              reinterpret_cast<uint32_t*>(dk_out + (row0 + t) * D)[lane] = real ? pk[0] : 0u;
-              reinterpret_cast<uint32_t*>(dv_out + (row0 + t) * D)[lane] = real ? pv[0] : 0u;
+              reinterpret_cast<uint32_t*>(dk_out + row * D)[lane] = real ? pk[0] : 0u;
+              reinterpret_cast<uint32_t*>(dv_out + row * D)[lane] = real ? pv[0] : 0u;
             } else {
-              reinterpret_cast<uint2*>(dk_out + (row0 + t) * D)[lane] =
-                  real ? make_uint2(pk[0], pk[1]) : make_uint2(0u, 0u);
-              reinterpret_cast<uint2*>(dv_out + (row0 + t) * D)[lane] =
-                  real ? make_uint2(pv[0], pv[1]) : make_uint2(0u, 0u);
+              reinterpret_cast<uint2*>(dk_out + row * D)[lane] = real ? make_uint2(pk[0], pk[1]) : make_uint2(0u, 0u);
+              reinterpret_cast<uint2*>(dv_out + row * D)[lane] = real ? make_uint2(pv[0], pv[1]) : make_uint2(0u, 0u);
             }
           }
         }
@@ -1011,9 +1027,8 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   uint8_t* base = align1024(dkv_smem_raw);
   const uint32_t kvt = smem_u32(cs.tiles(base, 0));
   const uint32_t ring = kvt + 2 * TB;
-  float* sls = reinterpret_cast<float*>(cs.tail(base, 0));
-  float* sdl = sls + STAGES * kBlock;
-  const uint32_t bar_kv = smem_u32(sdl + STAGES * kBlock);
+  float* slsd = reinterpret_cast<float*>(cs.tail(base, 0));  // [STAGES][32] LSE + Delta records
+  const uint32_t bar_kv = smem_u32(slsd + STAGES * 2 * kBlock);
   const uint32_t bar_ring = bar_kv + 8;
 
   const int E = n1 * K;
@@ -1031,8 +1046,8 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   __syncwarp();
   if (lane == 0) {
     mbar_expect_tx(bar_kv, 2 * TB);
-    tma_load_tile<D>(kvt, &tm_k, g, bh * g.N + j * kBlock, bar_kv);
-    tma_load_tile<D>(kvt + TB, &tm_v, g, bh * g.N + j * kBlock, bar_kv);
+    tma_load_tile<D, LAYOUT>(kvt, &tm_k, g, bh * g.N + j * kBlock, bar_kv);
+    tma_load_tile<D, LAYOUT>(kvt + TB, &tm_v, g, bh * g.N + j * kBlock, bar_kv);
   }
   float dk[D / 8][4], dv[D / 8][4];
 #pragma unroll
@@ -1052,10 +1067,12 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
     }
     return bh_block0 + __shfl_sync(0xffffffffu, cached, i & 31);
   };
-  const int kvalid = min(kBlock, g.nv - j * kBlock);  // real keys of this block (16 unless padded)
-  const bool ok = kv_stream<D, STAGES, false, POOL>(g, &tm_q, &tm_do, lse, ws + W.delta, kvt, bar_kv, ring, sls, sdl,
-                                                    bar_ring, re - rs, pair_block, P.scale_log2, dk, dv, {0.f, 0.f},
-                                                    pool_log_bias<D>(g), kvalid);
+  // real keys of this block (16 unless padded)
+  const int kvalid = LAYOUT == kPadded ? min(kBlock, g.nv - j * kBlock) : kBlock;
+  const bool ok = kv_stream<D, STAGES, LAYOUT, false, POOL>(g, &tm_q, &tm_do, ws + W.lsd, kvt, bar_kv, ring, slsd,
+                                                            bar_ring, re - rs, pair_block, P.scale_log2, dk, dv,
+                                                            {0.f, 0.f}, pool_log_bias<D>(g), kvalid,
+                                                            LAYOUT == kGrid ? 1 : 0);
   if (!ok) return;
   if (coarse_late) pdl_wait();
   // epilogue: scale dK, add the mean-pool adjoint of the ancestors' coarse gradients
@@ -1089,11 +1106,10 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
       dv[n][3] += wgt * xv.y;
     }
   }
-  const long long row0 = (long long)bh * g.N + (long long)j * kBlock;
   const int r0 = lane >> 2;  // padding positions of a padded sequence get dK = dV = 0
   const float s0 = r0 < kvalid ? 1.0f : 0.0f, s1 = r0 + 8 < kvalid ? 1.0f : 0.0f;
-  store_tile_bf16<D>(dk, s0, s1, kvt, dk_out + row0 * D);
-  store_tile_bf16<D>(dv, s0, s1, kvt + TB, dv_out + row0 * D);
+  store_tile_bf16<D, LAYOUT>(dk, s0, s1, kvt, dk_out, g, bh, j * kBlock);
+  store_tile_bf16<D, LAYOUT>(dv, s0, s1, kvt + TB, dv_out, g, bh, j * kBlock);
 }
 
 }  // namespace llsa

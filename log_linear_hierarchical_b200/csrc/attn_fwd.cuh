@@ -49,20 +49,26 @@ __device__ __forceinline__ uint32_t tswz(int row, int ch) {
   return static_cast<uint32_t>((ch >> 3) * kSubTileBytes) + swz(row, ch & 7);
 }
 
+// Every fragment load below takes `perm` (0 or 1): 1 for a tile that a grid-order TMA box
+// brought in (its shared-memory rows are pixel rows, tile_row maps the block's quadtree row to
+// them), 0 for a tile whose rows are already in order.
+
 // A-operand fragments of a 16 x D bf16 tile (rows = M, channels = K) for the D/16 k-steps.
 template <int D>
-__device__ __forceinline__ void load_a_frags(uint32_t tile, uint32_t (&f)[D / 16][4]) {
+__device__ __forceinline__ void load_a_frags(uint32_t tile, uint32_t (&f)[D / 16][4], int perm = 0) {
   const int lane = lane_id();
+  const int row = tile_row(lane & 15, perm);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk)
-    ldsm_x4(tile + tswz(lane & 15, 2 * kk + (lane >> 4)), f[kk][0], f[kk][1], f[kk][2], f[kk][3]);
+    ldsm_x4(tile + tswz(row, 2 * kk + (lane >> 4)), f[kk][0], f[kk][1], f[kk][2], f[kk][3]);
 }
 
 // acc[2][4] (16 x 16) += A (16 x D, fragments) * B^T where B is a 16-row x D tile (rows = N).
 template <int D>
-__device__ __forceinline__ void mma_a_bt(float (&acc)[2][4], const uint32_t (&a)[D / 16][4], uint32_t btile) {
+__device__ __forceinline__ void mma_a_bt(float (&acc)[2][4], const uint32_t (&a)[D / 16][4], uint32_t btile,
+                                         int perm = 0) {
   const int lane = lane_id();
-  const int row = (lane & 7) + ((lane >> 4) << 3);
+  const int row = tile_row((lane & 7) + ((lane >> 4) << 3), perm);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     uint32_t b0, b1, b2, b3;
@@ -75,13 +81,15 @@ __device__ __forceinline__ void mma_a_bt(float (&acc)[2][4], const uint32_t (&a)
 // The same with A read from its shared-memory tile one k-step at a time (no A fragments
 // held in registers).
 template <int D>
-__device__ __forceinline__ void mma_at_bt(float (&acc)[2][4], uint32_t atile, uint32_t btile) {
+__device__ __forceinline__ void mma_at_bt(float (&acc)[2][4], uint32_t atile, uint32_t btile, int aperm = 0,
+                                          int bperm = 0) {
   const int lane = lane_id();
-  const int row = (lane & 7) + ((lane >> 4) << 3);
+  const int row = tile_row((lane & 7) + ((lane >> 4) << 3), bperm);
+  const int arow = tile_row(lane & 15, aperm);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-    ldsm_x4(atile + tswz(lane & 15, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
+    ldsm_x4(atile + tswz(arow, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
     ldsm_x4(btile + tswz(row, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
     mma_bf16(acc[0], a0, a1, a2, a3, b0, b1);
     mma_bf16(acc[1], a0, a1, a2, a3, b2, b3);
@@ -91,9 +99,9 @@ __device__ __forceinline__ void mma_at_bt(float (&acc)[2][4], uint32_t atile, ui
 // acc[D/8][4] (16 x D) += A (16 x 16: a0..a3) * B where B is a 16-row x D tile (rows = K).
 template <int D>
 __device__ __forceinline__ void mma_a_b(float (&acc)[D / 8][4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                        uint32_t btile) {
+                                        uint32_t btile, int perm = 0) {
   const int lane = lane_id();
-  const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+  const int row = tile_row((lane & 7) + (((lane >> 3) & 1) << 3), perm);
 #pragma unroll
   for (int dc = 0; dc < D / 16; ++dc) {
     uint32_t b0, b1, b2, b3;
@@ -109,9 +117,9 @@ __device__ __forceinline__ void mma_a_b(float (&acc)[D / 8][4], uint32_t a0, uin
 // previous product), 64 channels at a time.
 template <int D>
 __device__ __forceinline__ void mma_a2_b(float (&acc)[D / 8][4], const uint32_t (&hi)[4], const uint32_t (&lo)[4],
-                                         uint32_t btile) {
+                                         uint32_t btile, int perm = 0) {
   const int lane = lane_id();
-  const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+  const int row = tile_row((lane & 7) + (((lane >> 3) & 1) << 3), perm);
 #pragma unroll
   for (int h = 0; h < D / 64; ++h) {
     uint32_t b[4][4];
@@ -166,11 +174,12 @@ __device__ __forceinline__ void stage_coarse_rows(const Geometry& g, const float
   }
 }
 
-// Write a 16 x D fp32 accumulator (fragment layout, already scaled) as bf16 rows
-// [row0, row0 + 16) of a [rows, D] global array, through a swizzled shared staging tile.
-template <int D>
+// Write a 16 x D fp32 accumulator (fragment layout, already scaled) as the bf16 rows of the
+// 16 tokens t0 .. t0 + 15 of head bh of a [B*H*N, D] global array (token_row: in grid order
+// each row goes to its pixel), through a swizzled shared staging tile.
+template <int D, int LAYOUT>
 __device__ __forceinline__ void store_tile_bf16(const float (&acc)[D / 8][4], float s0, float s1, uint32_t stage,
-                                                __nv_bfloat16* __restrict__ dst_rows) {
+                                                __nv_bfloat16* __restrict__ out, const Geometry& g, int bh, int t0) {
   const int lane = lane_id();
   const int r0 = lane >> 2;
   const uint32_t cb = (lane & 3) * 4;
@@ -192,7 +201,7 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[D / 8][4], fl
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(stage + tswz(row, c)));
-    *reinterpret_cast<uint4*>(dst_rows + row * D + c * 8) = v;
+    *reinterpret_cast<uint4*>(out + token_row<LAYOUT>(g, bh, t0 + row) * D + c * 8) = v;
   }
   // the staging tile is refilled by TMA later: order these generic accesses before it
   fence_proxy_async();
@@ -200,15 +209,48 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[D / 8][4], fl
 }
 
 // Loads of the 16-token x D tile that starts at flat token row `row` (= (b*H + h) * N + t):
-// D/64 boxes of the [B*H][n_valid][D] tensor map, at x = 0, 64.  Rows at or past n_valid
-// (the padding of a padded sequence) arrive as zeros.
-template <int D>
+// D/64 boxes at x = 0, 64 of the flat [B*H*N][D] tensor map, or of the [B*H][n_valid][D]
+// one for a padded sequence, whose rows at or past n_valid arrive as zeros.
+// Under LLSA_FLAG_GRID_ORDER the map is [B*H*G][G][D] (pixel rows) and the box a 4 x 4 patch: the
+// block at quadtree position t / 16 is the patch at block-grid row and column R, C, whose 16
+// pixel rows arrive in row-major order (see tile_row).
+template <int D, int LAYOUT>
 __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, const Geometry& g, int row,
                                               uint32_t bar) {
+  if constexpr (LAYOUT == kFlat) {
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) tma_load_2d(dst + h * kSubTileBytes, map, 64 * h, row, bar);
+    return;
+  }
+  const int bh = div_n(g, row);
+  const int t = row - bh * g.N;
+  if constexpr (LAYOUT == kGrid) {
+    const int p = z_to_rowmajor(t >> 4, g.log_g - 2);  // R * (G / 4) + C
+    const int R = p >> (g.log_g - 2), C = p & ((1 << (g.log_g - 2)) - 1);
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h)
+      tma_load_3d(dst + h * kSubTileBytes, map, 64 * h, 4 * C, (bh << g.log_g) + 4 * R, bar);
+    return;
+  }
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * kSubTileBytes, map, 64 * h, t, bh, bar);
+}
+
+// The 16 LSE values of the query block whose first token row is `row` (flat), into `dst`
+// in the tile's shared-memory row order: one 64-byte bulk copy, or under grid order four
+// 16-byte copies of the patch's pixel rows.
+template <int LAYOUT>
+__device__ __forceinline__ void bulk_load_block_rows(uint32_t dst, const float* src, const Geometry& g, int row,
+                                                     uint32_t bar) {
+  if constexpr (LAYOUT != kGrid) {
+    bulk_load(dst, src + row, kBlock * 4, bar);
+    return;
+  }
   const int bh = div_n(g, row);
   const int t = row - bh * g.N;
 #pragma unroll
-  for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * kSubTileBytes, map, 64 * h, t, bh, bar);
+  for (int r = 0; r < 4; ++r)
+    bulk_load(dst + 16 * r, src + token_row<kGrid>(g, bh, t + 2 * (r & 1) + 8 * (r >> 1)), 16, bar);
 }
 
 // sqrt(D): a score bias in units of the unscaled dot product is the scaled bias times this.
@@ -245,10 +287,11 @@ __device__ __forceinline__ void quad_row_sums(const float (&s)[2][4], float& t0,
 template <int D, bool MASK, bool POOL = false>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint32_t ktile, uint32_t vtile, int valid,
                                           float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[D / 8][4],
-                                          const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f) {
+                                          const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
+                                          int perm = 0) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  mma_a_bt<D>(s, qf, ktile);
+  mma_a_bt<D>(s, qf, ktile, perm);
   float sb0 = 0.f, sb1 = 0.f;  // pooled scores of rows r0, r0 + 8
   if (POOL) {
     quad_row_sums(s, sb0, sb1);
@@ -316,7 +359,7 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint3
   l[0] += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
   l[1] += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
   mma_a_b<D>(acc, pack_bf16(p[0][0], p[0][1]), pack_bf16(p[0][2], p[0][3]), pack_bf16(p[1][0], p[1][1]),
-             pack_bf16(p[1][2], p[1][3]), vtile);
+             pack_bf16(p[1][2], p[1][3]), vtile, perm);
 }
 
 // Shared memory of the attention kernels: a CTA region (the group's coarse K and V tiles),
@@ -347,10 +390,10 @@ __host__ __device__ inline CtaSmem fwd_smem(const Geometry& g, int nwarps) {
 // One CTA = 4 warps = 16 consecutive query blocks (one level-2 group when L >= 2, so the
 // coarse KV entries are staged once per CTA).  Each warp owns 4 blocks and streams their
 // fine KV tiles through its own ring of STAGES mbarrier-tracked TMA stages.  POOL: the
-// level-1 variant (see fwd_chunk).  PAD: a padded sequence -- the fine tile that holds the
-// last real token masks its padding keys (which arrive as zero rows), and padding queries
-// write O = 0 and LSE = 0.
-template <int D, int STAGES, bool POOL, bool PAD>
+// level-1 variant (see fwd_chunk).  LAYOUT (see Layout): under kPadded the fine tile that
+// holds the last real token masks its padding keys (which arrive as zero rows), and padding
+// queries write O = 0 and LSE = 0.
+template <int D, int STAGES, bool POOL, int LAYOUT>
 __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                             const __grid_constant__ CUtensorMap tm_k,
                                                             const __grid_constant__ CUtensorMap tm_v, AttnParams P,
@@ -361,6 +404,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   // the coarse tiles come from the pyramid and the coarser selection levels, two or more
   // kernels back, so they are staged before waiting for the kernel ahead (see pdl_wait)
   extern __shared__ uint8_t fwd_smem_raw[];
+  constexpr bool PAD = LAYOUT == kPadded;
+  constexpr int PERM = LAYOUT == kGrid ? 1 : 0;
   const Geometry& g = P.g;
   const int lane = lane_id();
   const int warp = threadIdx.x >> 5;
@@ -409,13 +454,13 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * TB;
     mbar_expect_tx(bar, 2 * TB);
-    tma_load_tile<D>(dst, &tm_k, g, row, bar);
-    tma_load_tile<D>(dst + TB, &tm_v, g, row, bar);
+    tma_load_tile<D, LAYOUT>(dst, &tm_k, g, row, bar);
+    tma_load_tile<D, LAYOUT>(dst + TB, &tm_v, g, row, bar);
   };
   auto issue_q = [&](int i) {
     const uint32_t bar = bar_q + 8 * (i & 1);
     mbar_expect_tx(bar, TB);
-    tma_load_tile<D>(sq + (i & 1) * TB, &tm_q, g, (first + i) * kBlock, bar);
+    tma_load_tile<D, LAYOUT>(sq + (i & 1) * TB, &tm_q, g, (first + i) * kBlock, bar);
   };
   if (lane == 0) {
     issue_q(0);
@@ -434,7 +479,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     if (!ok) break;
     next_q = i + 1;
     uint32_t qf[D / 16][4];
-    load_a_frags<D>(sq + (i & 1) * TB, qf);
+    load_a_frags<D>(sq + (i & 1) * TB, qf, PERM);
     __syncwarp();
     if (lane == 0 && i + 1 < nblk) issue_q(i + 1);
 
@@ -455,7 +500,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
       if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
         fwd_chunk<D, true>(qf, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - bh_i * g.N)), P.scale_log2, m, l, acc);
       else
-        fwd_chunk<D, false, POOL>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias<D>(g));
+        fwd_chunk<D, false, POOL>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias<D>(g),
+                                  PERM);
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }
@@ -470,11 +516,12 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     l[1] += __shfl_xor_sync(0xffffffffu, l[1], 2);
     const int r0 = lane >> 2;
     const bool real0 = !PAD || r0 < qvalid, real1 = !PAD || r0 + 8 < qvalid;
-    store_tile_bf16<D>(acc, real0 ? 1.0f / l[0] : 0.0f, real1 ? 1.0f / l[1] : 0.0f, sq + (i & 1) * TB,
-                       o + (long long)gb * kBlock * D);
+    const int t0 = (gb - bh_i * n1) * kBlock;  // the block's first token in its head
+    store_tile_bf16<D, LAYOUT>(acc, real0 ? 1.0f / l[0] : 0.0f, real1 ? 1.0f / l[1] : 0.0f, sq + (i & 1) * TB, o, g,
+                               bh_i, t0);
     if ((lane & 3) == 0) {
-      lse[(long long)gb * kBlock + r0] = real0 ? (m[0] + log2f(l[0])) * kLn2 : 0.0f;
-      lse[(long long)gb * kBlock + r0 + 8] = real1 ? (m[1] + log2f(l[1])) * kLn2 : 0.0f;
+      lse[token_row<LAYOUT>(g, bh_i, t0 + r0)] = real0 ? (m[0] + log2f(l[0])) * kLn2 : 0.0f;
+      lse[token_row<LAYOUT>(g, bh_i, t0 + r0 + 8)] = real1 ? (m[1] + log2f(l[1])) * kLn2 : 0.0f;
     }
   }
   if (!ok) {

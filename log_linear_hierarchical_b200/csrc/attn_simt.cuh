@@ -45,7 +45,7 @@ __device__ __forceinline__ void simt_kv_rows(const Geometry& g, int bh, int p, c
     if (e < kBlock * K) {
       const int j = checked_index(__ldg(idx + g.idx_off[1] + ((long long)bh * n1 + p) * K + e / kBlock), n1);
       const int t = j * kBlock + (e % kBlock);
-      r = (long long)bh * g.N + t;
+      r = token_row(g, bh, t);
       is_real = t < g.nv;
       kb = k;
       vb = v;
@@ -98,8 +98,8 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
   float* S = reinterpret_cast<float*>(vrow + T);
   int* real = reinterpret_cast<int*>(S + kBlock * T);
   const int qvalid = g.nv - p * kBlock;  // real queries of the block (>= 16 unless padded)
-  const float* qb = q + (long long)gb * kBlock * D;
-  for (int i = threadIdx.x; i < kBlock * D; i += blockDim.x) qs[i] = i / D < qvalid ? qb[i] : 0.0f;
+  for (int i = threadIdx.x; i < kBlock * D; i += blockDim.x)
+    qs[i] = i / D < qvalid ? q[token_row(g, bh, p * kBlock + i / D) * D + i % D] : 0.0f;
   simt_kv_rows<D>(g, bh, p, k, v, k_pyr, v_pyr, idx, krow, vrow, real);
   __syncthreads();
   for (int pr = threadIdx.x; pr < kBlock * T; pr += blockDim.x) {
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
     for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
     const float inv = 1.0f / l;
     for (int e = lane; e < T; e += 32) row[e] *= inv;
-    if (lane == 0) lse[(long long)gb * kBlock + qi] = qi < qvalid ? m + logf(l) : 0.0f;
+    if (lane == 0) lse[token_row(g, bh, p * kBlock + qi)] = qi < qvalid ? m + logf(l) : 0.0f;
   }
   __syncthreads();
   for (int od = threadIdx.x; od < kBlock * D; od += blockDim.x) {
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_fwd_f32_kernel(Geometry g, 
     float acc = 0.f;
     for (int e = 0; e < T; ++e)
       if (real[e]) acc = fmaf(prow[e], vrow[e][d], acc);
-    o[(long long)gb * kBlock * D + od] = qi < qvalid ? acc : 0.0f;
+    o[token_row(g, bh, p * kBlock + qi) * D + d] = qi < qvalid ? acc : 0.0f;
   }
 }
 
@@ -183,20 +183,22 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
     __syncthreads();
     for (int i = threadIdx.x; i < kBlock * D; i += blockDim.x) {
       const bool rq = i / D < qvalid;
-      qs[i] = rq ? q[rbase * D + i] : 0.0f;
-      ds_[i] = rq ? dO[rbase * D + i] : 0.0f;
+      const long long src = token_row(g, bh, p * kBlock + i / D) * D + i % D;
+      qs[i] = rq ? q[src] : 0.0f;
+      ds_[i] = rq ? dO[src] : 0.0f;
     }
     simt_kv_rows<D>(g, bh, p, k, v, k_pyr, v_pyr, idx, krow, vrow, real);
     __syncthreads();
     for (int qi = warp; qi < kBlock; qi += blockDim.x >> 5) {
       float s = 0.f;
       if (qi < qvalid)
-        for (int d = lane; d < D; d += 32) s = fmaf(ds_[qi * D + d], o[(rbase + qi) * D + d], s);
+        for (int d = lane; d < D; d += 32)
+          s = fmaf(ds_[qi * D + d], o[token_row(g, bh, p * kBlock + qi) * D + d], s);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
       if (lane == 0) {
         delta[qi] = s;
-        ws[W.delta + rbase + qi] = s;
+        ws[W.lsd + rbase + qi] = s;
       }
     }
     __syncthreads();
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
         continue;
       }
       const float bias = simt_entry_bias(g, e);
-      const float pe = expf(dotD<D>(qs + qi * D, krow[e]) * scale + bias - lse[rbase + qi]);
+      const float pe = expf(dotD<D>(qs + qi * D, krow[e]) * scale + bias - lse[token_row(g, bh, p * kBlock + qi)]);
       const float dp = dotD<D>(ds_ + qi * D, vrow[e]);
       Pm[pr] = pe;
       dS[pr] = pe * (dp - delta[qi]);
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dq_f32_kernel(
       float acc = 0.f;
       for (int e = 0; e < T; ++e)
         if (real[e]) acc = fmaf(dS[qi * T + e], krow[e][d], acc);
-      dq_out[rbase * D + od] = acc * scale;
+      dq_out[token_row(g, bh, p * kBlock + qi) * D + d] = acc * scale;
     }
     for (int cd = threadIdx.x; cd < C * D; cd += blockDim.x) {
       const int c = cd / D;
@@ -273,12 +275,12 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
   const int kb = blockIdx.x;
   const int bh = kb / n1;
   const int j = kb - bh * n1;
-  const long long krow0 = (long long)bh * g.N + (long long)j * kBlock;
   const int kvalid = g.nv - j * kBlock;  // real keys of the block (>= 16 unless padded)
   for (int i = threadIdx.x; i < kBlock * D; i += blockDim.x) {
     const bool rk = i / D < kvalid;
-    ks[i] = rk ? k[krow0 * D + i] : 0.0f;
-    vs[i] = rk ? v[krow0 * D + i] : 0.0f;
+    const long long src = token_row(g, bh, j * kBlock + i / D) * D + i % D;
+    ks[i] = rk ? k[src] : 0.0f;
+    vs[i] = rk ? v[src] : 0.0f;
   }
   if (g.pool1)
     for (int d = threadIdx.x; d < D; d += blockDim.x) {
@@ -304,12 +306,13 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
     __syncthreads();
     for (int i = threadIdx.x; i < kBlock * D; i += blockDim.x) {
       const bool rq = i / D < qvalid;
-      qs[i] = rq ? q[qrow0 * D + i] : 0.0f;
-      dos[i] = rq ? dO[qrow0 * D + i] : 0.0f;
+      const long long src = token_row(g, bh, p * kBlock + i / D) * D + i % D;
+      qs[i] = rq ? q[src] : 0.0f;
+      dos[i] = rq ? dO[src] : 0.0f;
     }
     if (threadIdx.x < kBlock) {
-      ls[threadIdx.x] = lse[qrow0 + threadIdx.x];
-      dl[threadIdx.x] = ws[W.delta + qrow0 + threadIdx.x];
+      ls[threadIdx.x] = lse[token_row(g, bh, p * kBlock + threadIdx.x)];
+      dl[threadIdx.x] = ws[W.lsd + qrow0 + threadIdx.x];
     }
     __syncthreads();
     if (g.pool1 && threadIdx.x < kBlock) {  // the level-1 entry's p / 16 and dS / 16 per query
@@ -360,8 +363,9 @@ __global__ void __launch_bounds__(kSimtThreads) attn_bwd_dkdv_f32_kernel(
       rk += wgt * ws[W.cg_k + crow];
       rv += wgt * ws[W.cg_v + crow];
     }
-    dk_out[(krow0 + kk) * D + d] = kk < kvalid ? rk : 0.0f;
-    dv_out[(krow0 + kk) * D + d] = kk < kvalid ? rv : 0.0f;
+    const long long dst = token_row(g, bh, j * kBlock + kk) * D + d;
+    dk_out[dst] = kk < kvalid ? rk : 0.0f;
+    dv_out[dst] = kk < kvalid ? rv : 0.0f;
   }
 }
 

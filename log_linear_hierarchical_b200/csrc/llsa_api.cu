@@ -38,7 +38,8 @@ llsa_status validate(const llsa_shape* s) {
   if (s->B < 1 || s->H < 1 || s->N < 1 || s->D < 1 || s->block < 1 || s->topk < 1 || s->levels < 1)
     return LLSA_ERR_INVALID_ARG;
   if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
-  if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP | LLSA_FLAG_LEVEL1))
+  if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP | LLSA_FLAG_LEVEL1 | LLSA_FLAG_GRID_ORDER |
+                   LLSA_FLAG_ONE_LAUNCH_SELECT))
     return LLSA_ERR_INVALID_ARG;  // unknown flag bits
   if (s->n_valid < 0 || s->n_valid > s->N) return LLSA_ERR_INVALID_ARG;
   // N: any multiple of 16^L (the pages' implementation wants powers of two for N and topk;
@@ -59,7 +60,11 @@ llsa_status validate(const llsa_shape* s) {
   if (s->n_valid != 0 && s->n_valid < s->N) {  // a padded sequence
     const long long span = 1LL << (4 * s->levels);
     if (s->topk > (s->n_valid + span - 1) / span) return LLSA_ERR_INVALID_ARG;  // K real coarsest tokens
-    if (s->flags != 0) return LLSA_ERR_UNSUPPORTED;  // padding takes the default enrichment only
+    if (s->flags & ~LLSA_FLAG_ONE_LAUNCH_SELECT) return LLSA_ERR_UNSUPPORTED;  // default enrichment only
+  }
+  if (s->flags & LLSA_FLAG_GRID_ORDER) {  // a square grid of side 2^(log2 N / 2), 16 x 16 at least
+    if (!is_pow2(s->N) || (ilog2(s->N) & 1)) return LLSA_ERR_INVALID_ARG;
+    if (s->N < 256) return LLSA_ERR_UNSUPPORTED;
   }
   return LLSA_OK;
 }
@@ -93,6 +98,8 @@ Geometry make_geometry(const llsa_shape* s) {
   g.top_first = all_top ? (g.L - 2) * g.K : g.coarse;
   g.pool1 = (s->flags & LLSA_FLAG_LEVEL1) ? 1 : 0;
   g.nv = (s->n_valid > 0 && s->n_valid < s->N) ? s->n_valid : s->N;
+  g.grid = (s->flags & LLSA_FLAG_GRID_ORDER) ? 1 : 0;
+  g.log_g = g.grid ? ilog2(s->N) / 2 : 0;
   for (int l = 0; l <= kMaxLevels; ++l) g.m[l] = l <= g.L ? (int)((g.nv + (1LL << (4 * l)) - 1) >> (4 * l)) : 0;
   return g;
 }
@@ -154,10 +161,32 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // q, k, v, dO as [B*H][n_valid][D] bf16 (row stride D, head stride N * D); box = 64
 // channels (128 bytes, the swizzle span) x 16 rows x 1 head, so a 16-token tile is D / 64
-// boxes at x = 0, 64.  Rows at or past n_valid (padding) are read as zeros.
+// boxes at x = 0, 64.  Rows at or past n_valid (padding) are read as zeros.  Without
+// padding the view is the flat [B*H*N][D] (box 64 x 16, row coordinate = flat token row).
+// Under LLSA_FLAG_GRID_ORDER: [B*H*G][G][D] (pixel rows of every head's grid) with a
+// 64-channel x 4 x 4 pixel box (one 16-token block of the quadtree order).
 bool make_tile_map(CUtensorMap* m, const void* base, const Geometry& g) {
   auto fn = encode_fn();
   if (!fn) return false;
+  if (g.grid) {  // the heads' grids stacked: pixel rows of all heads, G pixels each
+    const cuuint64_t G = 1ULL << g.log_g;
+    cuuint64_t dims[3] = {(cuuint64_t)g.D, G, (cuuint64_t)g.BH * G};
+    cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, G * g.D * 2};
+    cuuint32_t box[3] = {64u, 4u, 4u};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  if (g.nv == g.N) {  // no padding: one flat [B*H*N][D] view (cheaper per copy than 3-D)
+    cuuint64_t dims[2] = {(cuuint64_t)g.D, (cuuint64_t)g.BH * g.N};
+    cuuint64_t strides[1] = {(cuuint64_t)g.D * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)kBlock};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.nv, (cuuint64_t)g.BH};
   cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.N * g.D * 2};
   cuuint32_t box[3] = {64u, (cuuint32_t)kBlock, 1u};
@@ -165,6 +194,25 @@ bool make_tile_map(CUtensorMap* m, const void* base, const Geometry& g) {
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The pyramid's view of a grid-order input: [B*H][G][G][D] (bf16 or fp32), box = one 16 x 16
+// pixel patch of all D channels (a level-2 token), no swizzle.  A zeroed map when the input
+// is in quadtree order (the pyramid then reads contiguous spans by bulk copy).
+bool make_patch_map(CUtensorMap* m, const void* base, const Geometry& g, int dtype) {
+  *m = CUtensorMap{};
+  if (!g.grid) return true;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t G = 1ULL << g.log_g;
+  const cuuint64_t e = dtype == LLSA_BF16 ? 2 : 4;
+  cuuint64_t dims[4] = {(cuuint64_t)g.D, G, G, (cuuint64_t)g.BH};
+  cuuint64_t strides[3] = {(cuuint64_t)g.D * e, G * g.D * e, (cuuint64_t)g.N * g.D * e};
+  cuuint32_t box[4] = {(cuuint32_t)g.D, 16u, 16u, 1u};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, dtype == LLSA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // [rows, 64] bf16 viewed as 2-D, box 64 x 16 with 128-byte swizzle (the gather probe).
@@ -335,6 +383,45 @@ namespace {
 // level-1 CSR and can run beside the query side too.
 constexpr unsigned kQuerySide = 1, kKeySide = 2, kOrder = 4;
 
+// The bf16 attention kernels' addressing (Layout) for this geometry.
+int layout_of(const Geometry& g) { return g.grid ? kGrid : (g.nv < g.N ? kPadded : kFlat); }
+
+// The instantiation of each bf16 attention kernel for a geometry: its Layout, and the
+// level-1 variant (POOL), which padding does not combine with.
+template <int D>
+auto pick_fwd(const Geometry& g) {
+  constexpr int S = kFwdStages;
+  const int lay = layout_of(g);
+  if (lay == kPadded) return attn_fwd_bf16_kernel<D, S, false, kPadded>;
+  if (lay == kGrid) return g.pool1 ? attn_fwd_bf16_kernel<D, S, true, kGrid> : attn_fwd_bf16_kernel<D, S, false, kGrid>;
+  return g.pool1 ? attn_fwd_bf16_kernel<D, S, true, kFlat> : attn_fwd_bf16_kernel<D, S, false, kFlat>;
+}
+template <int D>
+auto pick_dq(const Geometry& g) {
+  constexpr int S = kDqStages;
+  const int lay = layout_of(g);
+  if (lay == kPadded) return attn_bwd_dq_bf16_kernel<D, S, false, kPadded>;
+  if (lay == kGrid)
+    return g.pool1 ? attn_bwd_dq_bf16_kernel<D, S, true, kGrid> : attn_bwd_dq_bf16_kernel<D, S, false, kGrid>;
+  return g.pool1 ? attn_bwd_dq_bf16_kernel<D, S, true, kFlat> : attn_bwd_dq_bf16_kernel<D, S, false, kFlat>;
+}
+template <int D>
+auto pick_dkdv(const Geometry& g) {
+  constexpr int S = kDkvStages;
+  const int lay = layout_of(g);
+  if (lay == kPadded) return attn_bwd_dkdv_bf16_kernel<D, S, false, kPadded>;
+  if (lay == kGrid)
+    return g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, S, true, kGrid> : attn_bwd_dkdv_bf16_kernel<D, S, false, kGrid>;
+  return g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, S, true, kFlat> : attn_bwd_dkdv_bf16_kernel<D, S, false, kFlat>;
+}
+template <int D>
+auto pick_coarse(const Geometry& g) {
+  const int lay = layout_of(g);
+  if (lay == kPadded) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kPadded>;
+  if (lay == kGrid) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kGrid>;
+  return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kFlat>;
+}
+
 template <int D>
 llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
                               const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
@@ -363,9 +450,7 @@ llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k,
     const size_t kv_bytes = (size_t)kv_smem<D, kDkvStages>(1).total();
     if (phases & kQuerySide) {
       const size_t smem = (size_t)dq_smem<D, kDqStages>(g, kAttnWarps).total();
-      auto kern = g.nv < g.N ? attn_bwd_dq_bf16_kernel<D, kDqStages, false, true>
-                  : g.pool1  ? attn_bwd_dq_bf16_kernel<D, kDqStages, true, false>
-                             : attn_bwd_dq_bf16_kernel<D, kDqStages, false, false>;
+      auto kern = pick_dq<D>(g);
       if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
       const int per_cta = kAttnWarps * kUnitBlocks;
       st = launch(kKBwdDqBf16, cs, [&] {
@@ -375,21 +460,21 @@ llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k,
       });
       if (st != LLSA_OK) return st;
       if (g.L >= 2) {
-        auto ckern = attn_bwd_coarse_bf16_kernel<D, kDkvStages>;
+        auto ckern = pick_coarse<D>(g);
         if (!allow_smem(ckern, kv_bytes)) return LLSA_ERR_CUDA;
         const int ctas = g.BH * g.n[2] * (g.coarse_pad / kBlock);
         st = launch(kKBwdCoarseBf16, cs, [&] {
-          launch_pdl(ckern, dim3(ctas), dim3(32), kv_bytes, cs, tq, tdo, P, k_pyr, v_pyr, idx, lse, ws);
+          launch_pdl(ckern, dim3(ctas), dim3(32), kv_bytes, cs, tq, tdo, P, k_pyr, v_pyr, idx, ws);
         });
         if (st != LLSA_OK) return st;
       }
     }
     if (!(phases & kKeySide)) return LLSA_OK;
     if ((st = launch_coarse_reduce<D>(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
-    auto kern = g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, kDkvStages, true> : attn_bwd_dkdv_bf16_kernel<D, kDkvStages, false>;
+    auto kern = pick_dkdv<D>(g);
     if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
     return launch(kKBwdDkdvBf16, cs, [&] {
-      launch_pdl(kern, dim3(total_blocks), dim3(32), kv_bytes, cs, tq, tk, tv, tdo, P, lse, row_ptr, col, ws,
+      launch_pdl(kern, dim3(total_blocks), dim3(32), kv_bytes, cs, tq, tk, tv, tdo, P, row_ptr, col, ws,
                  static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), g.L >= 2 ? 1 : 0);
     });
   }
@@ -431,9 +516,13 @@ llsa_status pyramid_l12_launch(const Geometry& g, const void* q, const void* k, 
   using C = PyrCfg<T, D>;
   dim3 grid(g.BH * ((g.n[1] + C::ROWS - 1) / C::ROWS), 3);
   if (!allow_smem(pyramid_l12_kernel<T, D>, C::SPAN)) return LLSA_ERR_CUDA;
+  const int dtype = sizeof(T) == 2 ? LLSA_BF16 : LLSA_F32;
+  CUtensorMap pq, pk, pv;
+  if (!make_patch_map(&pq, q, g, dtype) || !make_patch_map(&pk, k, g, dtype) || !make_patch_map(&pv, v, g, dtype))
+    return LLSA_ERR_CUDA;
   return launch(kKPyramidL12, cs, [&] {
     launch_pdl(pyramid_l12_kernel<T, D>, dim3(grid), dim3(C::THREADS), C::SPAN, cs, g, static_cast<const T*>(q),
-               static_cast<const T*>(k), static_cast<const T*>(v), q_pyr, k_pyr, v_pyr);
+               static_cast<const T*>(k), static_cast<const T*>(v), q_pyr, k_pyr, v_pyr, pq, pk, pv);
   });
 }
 
@@ -533,8 +622,10 @@ llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* 
 // The pyramid and every selection level in one cooperative launch (pyramid_select_kernel):
 // bf16, L >= 2, a small coarsest level and K in {2, 4, 8, 16} (the register-resident
 // children selection).
-bool fused_pyramid_select(const Geometry& g, int dtype) {
-  return dtype == LLSA_BF16 && g.L >= 2 && small_top(g) && (g.K == 2 || g.K == 4 || g.K == 8 || g.K == 16);
+// Requested by LLSA_FLAG_ONE_LAUNCH_SELECT.
+bool fused_pyramid_select(const Geometry& g, const llsa_shape* s) {
+  return (s->flags & LLSA_FLAG_ONE_LAUNCH_SELECT) && s->dtype == LLSA_BF16 && g.L >= 2 && small_top(g) &&
+         (g.K == 2 || g.K == 4 || g.K == 8 || g.K == 16);
 }
 
 template <int D, int CPT>
@@ -551,6 +642,10 @@ llsa_status pyramid_select_launch_k(const Geometry& g, const void* q, const void
   long long units = 3LL * g.BH * ((g.n[1] + PyrCfg<__nv_bfloat16, D>::ROWS - 1) / PyrCfg<__nv_bfloat16, D>::ROWS);
   for (int l = 1; l < g.L; ++l) units = units > (long long)g.BH * (g.n[l] / kBlock) ? units : (long long)g.BH * (g.n[l] / kBlock);
   const int grid = (int)((long long)sms * per_sm < units ? (long long)sms * per_sm : units);
+  CUtensorMap pq, pk, pv;
+  if (!make_patch_map(&pq, q, g, LLSA_BF16) || !make_patch_map(&pk, k, g, LLSA_BF16) ||
+      !make_patch_map(&pv, v, g, LLSA_BF16))
+    return LLSA_ERR_CUDA;
   if (cudaMemsetAsync(barrier, 0, 16 * sizeof(unsigned), cs) != cudaSuccess) return LLSA_ERR_CUDA;
   return launch(kKPyramidSelect, cs, [&] {
     cudaLaunchConfig_t cfg = {};
@@ -564,7 +659,7 @@ llsa_status pyramid_select_launch_k(const Geometry& g, const void* q, const void
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaLaunchKernelEx(&cfg, kern, g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                       static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr, idx, barrier);
+                       static_cast<const __nv_bfloat16*>(v), q_pyr, k_pyr, v_pyr, idx, barrier, pq, pk, pv);
   });
 }
 
@@ -612,9 +707,7 @@ llsa_status forward_launch(const Geometry& g, int dtype, const void* q, const vo
     if (!make_tile_map(&tq, q, g) || !make_tile_map(&tk, k, g) || !make_tile_map(&tv, v, g)) return LLSA_ERR_CUDA;
     AttnParams P{g, scale * kLog2e, scale};
     const size_t smem = (size_t)fwd_smem<D, kFwdStages>(g, kAttnWarps).total();
-    auto kern = g.nv < g.N ? attn_fwd_bf16_kernel<D, kFwdStages, false, true>
-                : g.pool1  ? attn_fwd_bf16_kernel<D, kFwdStages, true, false>
-                           : attn_fwd_bf16_kernel<D, kFwdStages, false, false>;
+    auto kern = pick_fwd<D>(g);
     if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
     const int per_cta = kAttnWarps * kUnitBlocks;
     return launch(kKFwdBf16, cs, [&] {
@@ -648,7 +741,7 @@ llsa_status forward_impl(const llsa_shape* s, const void* q, const void* k, cons
 llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStream_t cs, cudaStream_t side) {
   const Geometry g = make_geometry(s);
   llsa_status st;
-  const bool fused = fused_pyramid_select(g, s->dtype);
+  const bool fused = fused_pyramid_select(g, s);
   if (fused) {  // pyramid and selection in one cooperative launch
     unsigned* barrier =
         reinterpret_cast<unsigned*>(static_cast<float*>(b->backward_workspace) + bwd_workspace_layout(g).barrier);

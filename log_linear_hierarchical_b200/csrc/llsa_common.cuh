@@ -57,7 +57,55 @@ struct Geometry {
                                          // level-1 mean is one more KV entry
   int nv;                                // real tokens per sequence (N when not padded)
   int m[kMaxLevels + 1];                 // real tokens of level l: ceil(nv / 16^l)
+  int grid;                              // LLSA_FLAG_GRID_ORDER: token rows in memory are in the
+                                         // row-major order of a G x G grid (G = 2^log_g); the
+                                         // path works in its quadtree (Z) order
+  int log_g;
 };
+
+// Even bits of x, packed: bit 2i of x becomes bit i.
+__host__ __device__ inline int compact_even_bits(int x) {
+  x &= 0x55555555;
+  x = (x | (x >> 1)) & 0x33333333;
+  x = (x | (x >> 2)) & 0x0f0f0f0f;
+  x = (x | (x >> 4)) & 0x00ff00ff;
+  x = (x | (x >> 8)) & 0x0000ffff;
+  return x;
+}
+
+// Row-major position r * side + c (side = 2^log_side) of quadtree index z, where c takes the
+// even bits of z and r the odd ones (z = sum_b (2 r_b + c_b) 4^b: top-left, top-right,
+// bottom-left, bottom-right at every scale).
+__host__ __device__ inline int z_to_rowmajor(int z, int log_side) {
+  return (compact_even_bits(z >> 1) << log_side) | compact_even_bits(z);
+}
+
+// Memory row of token t (in the path's Z order) of head bh: (b*H + h) * N + t, or the
+// row-major grid position of t under LLSA_FLAG_GRID_ORDER.
+__host__ __device__ inline long long token_row(const Geometry& g, int bh, int t) {
+  return (long long)bh * g.N + (g.grid ? z_to_rowmajor(t, g.log_g) : t);
+}
+
+// How the bf16 attention kernels address q, k, v, dO and their outputs.  A template
+// parameter, so the default instantiation carries no per-access test:
+//   kFlat:   [B*H*N][D] rows in quadtree order (flat 2-D tensor maps);
+//   kPadded: the same with rows at or past n_valid as padding (3-D maps read them as zeros);
+//   kGrid:   row-major G x G grids (LLSA_FLAG_GRID_ORDER: 4-D patch maps, the tile_row map).
+enum Layout : int { kFlat = 0, kPadded = 1, kGrid = 2 };
+
+template <int LAYOUT>
+__device__ __forceinline__ long long token_row(const Geometry& g, int bh, int t) {
+  return (long long)bh * g.N + (LAYOUT == kGrid ? z_to_rowmajor(t, g.log_g) : t);
+}
+
+// Under LLSA_FLAG_GRID_ORDER a 16-token block is a 4 x 4 pixel patch that a TMA box brings
+// in row by row (shared-memory row 4 r + c for pixel (r, c)), while the block's token order
+// is the quadtree order (z = 8 r1 + 4 c1 + 2 r0 + c0): row z of the block is shared-memory
+// row tile_row(z) (bits 1 and 2 swapped when `perm`, the identity otherwise).
+__host__ __device__ inline int tile_row(int z, int perm) {
+  const int x = ((z >> 1) ^ (z >> 2)) & perm;
+  return z ^ (x * 6);
+}
 
 // Real tokens under level-l token j of a sequence with nv real tokens: clamp(nv - j 16^l,
 // 0, 16^l) (16^l for every token when the sequence is not padded).
@@ -265,6 +313,16 @@ __global__ void __launch_bounds__(32) bounded_wait_check_kernel(long long limit)
 
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// 4-D tiled TMA load (no multicast) of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
 }
 
 // 3-D tiled TMA load (no multicast) of one box into shared memory, completing on `bar`.

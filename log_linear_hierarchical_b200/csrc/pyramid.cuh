@@ -92,13 +92,15 @@ struct PyrCfg {
 
 // One unit of levels 1-2: ROWS level-1 rows (tile `tile` of head bh) of one tensor x, and
 // the level-2 rows they make.  The CTA's input span (ROWS * 16 token rows) arrives by one
-// bulk copy completing on `bar` with phase parity `parity`; `span` and `s1` are the CTA's
-// shared buffers.  Every thread of the CTA calls it; returns false (for the whole CTA) if
-// the copy did not land within the bounded wait.
+// bulk copy completing on `bar` with phase parity `parity`, or, under grid order, as ROWS/16
+// 16 x 16 pixel patches (one level-2 token each) by TMA boxes of `pmap`; `span` and `s1` are
+// the CTA's shared buffers.  Every thread of the CTA calls it; returns false (for the whole
+// CTA) if the copy did not land within the bounded wait.
 template <typename T, int D>
 __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __restrict__ x,
                                                  float* __restrict__ pyr, int bh, int tile, uint8_t* span,
-                                                 float (*s1)[D], uint32_t bar, uint32_t parity) {
+                                                 float (*s1)[D], uint32_t bar, uint32_t parity,
+                                                 const CUtensorMap* pmap) {
   using C = PyrCfg<T, D>;
   constexpr int VE = C::VE;
   constexpr int TPR = C::TPR;
@@ -109,20 +111,43 @@ __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __r
   const int c0 = (t % TPR) * VE;
   const int j1 = tile * ROWS + o;
   __syncthreads();  // the span and s1 of the previous unit are no longer read
+  constexpr int OUT2 = ROWS / kBlock;  // level-2 rows per unit
+  constexpr int PATCH = kBlock * kBlock * D * (int)sizeof(T);
   if (t == 0) {
     const uint32_t bytes = (uint32_t)(min(ROWS, n1 - tile * ROWS) * kBlock * D * (int)sizeof(T));
     mbar_expect_tx(bar, bytes);
-    bulk_load(smem_u32(span), x + ((long long)bh * g.N + (long long)tile * ROWS * kBlock) * D, bytes, bar);
+    if (g.grid) {
+      const int lg2 = g.log_g - 4;  // level-2 tokens per grid row: G / 16
+      for (int o2 = 0; o2 < OUT2 && (tile * OUT2 + o2) * kBlock < n1; ++o2) {
+        const int p = z_to_rowmajor(tile * OUT2 + o2, lg2);
+        tma_load_4d(smem_u32(span) + o2 * PATCH, pmap, 0, 16 * (p & ((1 << lg2) - 1)), 16 * (p >> lg2), bh, bar);
+      }
+    } else {
+      bulk_load(smem_u32(span), x + ((long long)bh * g.N + (long long)tile * ROWS * kBlock) * D, bytes, bar);
+    }
   }
   if (!__syncthreads_and(mbar_wait(bar, parity))) {
     mbar_wait(bar, parity);  // recorded as LLSA_ERR_TIMEOUT; one more bounded wait for the copy
     return false;
   }
   if (j1 < n1) {
-    const T* src = reinterpret_cast<const T*>(span) + (o * kBlock) * D + c0;
     float v[kBlock][VE];
+    if (g.grid) {
+      // level-1 token o is block o % 16 (quadtree order) of patch o / 16; its token r is
+      // pixel (4 br + tr, 4 bc + tc) of the patch, rows of 16 pixels
+      const T* patch = reinterpret_cast<const T*>(span + (o >> 4) * PATCH) + c0;
+      const int b = o & 15;
+      const int br = compact_even_bits(b >> 1), bc = compact_even_bits(b);
 #pragma unroll
-    for (int r = 0; r < kBlock; ++r) Vec16<T>::load(src + r * D, v[r]);
+      for (int r = 0; r < kBlock; ++r) {
+        const int tr = compact_even_bits(r >> 1), tc = compact_even_bits(r);
+        Vec16<T>::load(patch + ((4 * br + tr) * kBlock + 4 * bc + tc) * D, v[r]);
+      }
+    } else {
+      const T* src = reinterpret_cast<const T*>(span) + (o * kBlock) * D + c0;
+#pragma unroll
+      for (int r = 0; r < kBlock; ++r) Vec16<T>::load(src + r * D, v[r]);
+    }
     float acc[VE];
 #pragma unroll
     for (int e = 0; e < VE; ++e) acc[e] = 0.0f;
@@ -146,7 +171,6 @@ __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __r
   }
   if (g.L < 2) return true;
   __syncthreads();
-  constexpr int OUT2 = ROWS / kBlock;  // level-2 rows per unit
   for (int i = t; i < OUT2 * D; i += blockDim.x) {
     const int o2 = i / D;
     const int d = i % D;
@@ -162,13 +186,17 @@ __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __r
 }
 
 // grid.x = B*H * ceil(n_1 / ROWS), grid.y = 3 (q, k, v).
+// pm0..pm2: the grid-order patch maps of q, k, v (unused in quadtree order).
 template <typename T, int D>
 __global__ void __launch_bounds__(PyrCfg<T, D>::THREADS) pyramid_l12_kernel(Geometry g, const T* __restrict__ x0,
                                                                             const T* __restrict__ x1,
                                                                             const T* __restrict__ x2,
                                                                             float* __restrict__ p0,
                                                                             float* __restrict__ p1,
-                                                                            float* __restrict__ p2) {
+                                                                            float* __restrict__ p2,
+                                                                            const __grid_constant__ CUtensorMap pm0,
+                                                                            const __grid_constant__ CUtensorMap pm1,
+                                                                            const __grid_constant__ CUtensorMap pm2) {
   pdl_enter();
   using C = PyrCfg<T, D>;
   __shared__ float s1[C::ROWS][D];
@@ -182,8 +210,9 @@ __global__ void __launch_bounds__(PyrCfg<T, D>::THREADS) pyramid_l12_kernel(Geom
   }
   const T* x = blockIdx.y == 0 ? x0 : (blockIdx.y == 1 ? x1 : x2);
   float* pyr = blockIdx.y == 0 ? p0 : (blockIdx.y == 1 ? p1 : p2);
+  const CUtensorMap* pm = blockIdx.y == 0 ? &pm0 : (blockIdx.y == 1 ? &pm1 : &pm2);
   const int bh = blockIdx.x / tiles;
-  pyramid_l12_unit<T, D>(g, x, pyr, bh, blockIdx.x - bh * tiles, pyr_span, s1, bar, 0);
+  pyramid_l12_unit<T, D>(g, x, pyr, bh, blockIdx.x - bh * tiles, pyr_span, s1, bar, 0, pm);
 }
 
 // Level l >= 3 from level l-1 (fp32).  One thread per output value; grid.y = tensor.

@@ -75,7 +75,10 @@ __global__ void __launch_bounds__(kSelThreads) pyramid_select_kernel(Geometry g,
                                                                      float* __restrict__ q_pyr,
                                                                      float* __restrict__ k_pyr,
                                                                      float* __restrict__ v_pyr, int* __restrict__ idx,
-                                                                     unsigned* __restrict__ barrier) {
+                                                                     unsigned* __restrict__ barrier,
+                                                                     const __grid_constant__ CUtensorMap pm0,
+                                                                     const __grid_constant__ CUtensorMap pm1,
+                                                                     const __grid_constant__ CUtensorMap pm2) {
   using C = PyrCfg<__nv_bfloat16, D>;
   static_assert(C::THREADS == kSelThreads, "one block shape for every phase");
   extern __shared__ __align__(128) uint8_t ps_smem[];
@@ -99,7 +102,8 @@ __global__ void __launch_bounds__(kSelThreads) pyramid_select_kernel(Geometry g,
       const int bh = rem / tiles;
       const __nv_bfloat16* x = t == 0 ? q : (t == 1 ? k : v);
       float* pyr = t == 0 ? q_pyr : (t == 1 ? k_pyr : v_pyr);
-      ok = pyramid_l12_unit<__nv_bfloat16, D>(g, x, pyr, bh, rem - bh * tiles, ps_smem, s1, bar, parity);
+      const CUtensorMap* pm = t == 0 ? &pm0 : (t == 1 ? &pm1 : &pm2);
+      ok = pyramid_l12_unit<__nv_bfloat16, D>(g, x, pyr, bh, rem - bh * tiles, ps_smem, s1, bar, parity, pm);
       parity ^= 1u;
     }
   }

@@ -139,10 +139,11 @@ def test_step_and_plan_rejected_before_launch(lib):
 
 def test_flags_validated(lib):
     s = shape()
-    for good in range(1, 8):  # any combination of LOG_BIAS (1), ALL_TOP (2), LEVEL1 (4)
+    # any combination of LOG_BIAS (1), ALL_TOP (2), LEVEL1 (4), GRID_ORDER (8), ONE_LAUNCH_SELECT (16)
+    for good in range(1, 32):
         s.flags = good
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 0, good
-    for bad in (8, 16, 1 << 30, -1):
+    for bad in (32, 64, 1 << 30, -1):
         s.flags = bad
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 1, bad
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True).flags == _lib.LLSA_FLAG_LOG_BIAS
@@ -231,3 +232,22 @@ def test_buffer_sizes_scale_with_head_width(lib):
     assert api.llsa_transpose_workspace_bytes(s128) == api.llsa_transpose_workspace_bytes(s64)
     # Delta and the dK/dV order do not grow with D; the coarse partials and gradients double
     assert api.llsa_backward_workspace_bytes(s128) > api.llsa_backward_workspace_bytes(s64)
+
+
+def test_grid_order_and_padding_rules(lib):
+    grid = _lib.LLSA_FLAG_GRID_ORDER
+    ok = api.make_shape(1, 2, 4096, 64, 4, 2, 0, grid_order=True)
+    assert lib.llsa_validate_shape(ctypes.byref(ok)) == 0
+    assert lib.llsa_validate_shape(ctypes.byref(api.make_shape(1, 2, 12288, 64, 4, 2, 0, grid_order=True))) == 1
+    assert lib.llsa_validate_shape(ctypes.byref(api.make_shape(1, 2, 8192, 64, 4, 2, 0, grid_order=True))) == 1
+    assert lib.llsa_validate_shape(ctypes.byref(api.make_shape(1, 2, 64, 64, 2, 1, 0, grid_order=True))) == 2
+    padded = api.make_shape(1, 2, 4096, 64, 4, 2, 0, n_valid=3000)
+    assert lib.llsa_validate_shape(ctypes.byref(padded)) == 0
+    padded.flags = grid
+    assert lib.llsa_validate_shape(ctypes.byref(padded)) == 2        # padding takes no variant flag
+    padded.flags = _lib.LLSA_FLAG_ONE_LAUNCH_SELECT                  # only the launch-shape one
+    assert lib.llsa_validate_shape(ctypes.byref(padded)) == 0
+    assert api.make_shape(1, 2, 4096, 64, 4, 2, 0, one_launch_select=True).flags == 16
+    assert lib.llsa_validate_shape(ctypes.byref(api.make_shape(1, 2, 4096, 64, 13, 2, 0, n_valid=2900))) == 1
+    assert lib.llsa_validate_shape(ctypes.byref(api.make_shape(1, 2, 4096, 64, 4, 2, 0, n_valid=5000))) == 1
+    assert lib.llsa_validate_shape(ctypes.byref(api.make_shape(1, 2, 4096, 64, 4, 2, 0, n_valid=-1))) == 1

@@ -99,12 +99,13 @@ def test_unpadded_n_valid_is_the_plain_path():
         assert np.array_equal(a[name], b[name]), name
 
 
-def test_padded_step_and_plan_match_separate_calls():
+@pytest.mark.parametrize("one_launch", [False, True])
+def test_padded_step_and_plan_match_separate_calls(one_launch):
     B, H, N, K, L, nv = 1, 2, 16384, 8, 2, 15000
     inputs = inputs_for(B, H, N, 64, "bf16", "smooth", 144)
     ref = run_gpu(B, H, N, 64, K, L, "bf16", inputs, n_valid=nv)
     tdt = TORCH_DTYPE["bf16"]
-    shape = api.make_shape(B, H, N, 64, K, L, tdt, n_valid=nv)
+    shape = api.make_shape(B, H, N, 64, K, L, tdt, n_valid=nv, one_launch_select=one_launch)
     dev = {k: v.cuda() for k, v in inputs.items()}
     buf = api.LLSABuffers.allocate(shape, "cuda", tdt)
     api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)

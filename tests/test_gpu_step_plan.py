@@ -143,17 +143,17 @@ def test_plan_headline_matches_serialized_calls():
 
 @pytest.mark.parametrize("B,H,N,K,L,D", [
     (1, 2, 65536, 8, 3, 64),     # the headline geometry: levels 3 pooled with the coarsest Top-K
-    (1, 1, 65536, 4, 4, 64),     # four levels, n_4 = 1
+    (1, 1, 1 << 18, 2, 4, 64),   # four levels, n_4 = 4
     (2, 1, 16384, 16, 2, 128),   # two levels, D = 128, K = 16
     (1, 2, 4096, 2, 2, 64),      # n_2 = 16
 ])
 def test_fused_pyramid_and_selection_equal_the_separate_launches(B, H, N, K, L, D):
-    """In a step the pyramid and every selection level run as one cooperative launch
-    (pyramid_select); its pyramid, selection and all results are bit-identical to the
-    separate pyramid and selection kernels of the five calls."""
+    """With LLSA_FLAG_ONE_LAUNCH_SELECT a step runs the pyramid and every selection level as
+    one cooperative launch (pyramid_select); its pyramid, selection and all results are
+    bit-identical to the separate pyramid and selection kernels of the five calls."""
     inputs = make_inputs(B, H, N, D, "bf16", "smooth", 150 + L)
     ref = run_gpu(B, H, N, D, K, L, "bf16", inputs)
-    shape = api.make_shape(B, H, N, D, K, L, torch.bfloat16)
+    shape = api.make_shape(B, H, N, D, K, L, torch.bfloat16, one_launch_select=True)
     dev = {k: v.cuda() for k, v in inputs.items()}
     buf = api.LLSABuffers.allocate(shape, "cuda", torch.bfloat16)
     with api.LaunchTrace(64) as tr:
@@ -167,3 +167,18 @@ def test_fused_pyramid_and_selection_equal_the_separate_launches(B, H, N, K, L, 
     assert np.array_equal(buf.idx.cpu().numpy(), np.concatenate([x.ravel() for x in ref["idx"]]))
     for k in KEYS:
         assert np.array_equal(getattr(buf, k).float().cpu().numpy(), ref[k]), k
+    plan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=2)
+    for k in KEYS:
+        getattr(buf, k).zero_()
+    plan.launch()
+    torch.cuda.synchronize()
+    assert api.llsa_device_status() == 0
+    for k in KEYS:
+        assert np.array_equal(getattr(buf, k).float().cpu().numpy(), ref[k]), k
+    plan.close()
+    # without the flag the same step takes the separate launches
+    plain = api.make_shape(B, H, N, D, K, L, torch.bfloat16)
+    with api.LaunchTrace(64) as tr:
+        api.llsa_train_step(plain, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+    names = [n for n, _ in tr.launches()]
+    assert names[0] == "pyramid_l12" and "pyramid_select" not in names, names
