@@ -432,7 +432,7 @@ def run_ours(args):
     pinned = {k: v.pin_memory() for k, v in host.items()}
     dev = {k: v.cuda(non_blocking=True) for k, v in pinned.items()}
     shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, grid_order=args.grid_order,
-                           one_launch_select=args.one_launch_select, **enrichment(args))
+                           one_launch_select=args.one_launch_select, causal=args.causal, **enrichment(args))
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     stream = torch.cuda.current_stream()
 
@@ -721,6 +721,7 @@ def run_ours(args):
                    "kv_len": 16 * cfg.topk + (cfg.topk if args.level1 else 0) + coarse_entries(cfg, args.all_top),
                    "step": "pyramid + select + forward + index transpose + backward",
                    "enrichment": enrichment_text(args),
+                   "mask": "causal (LLSA_FLAG_CAUSAL)" if args.causal else "none (non-causal)",
                    "token_order": ("row-major grid, read and written through the quadtree order in the kernels "
                                    "(LLSA_FLAG_GRID_ORDER)" if args.grid_order else "quadtree (Z) order"),
                    "launch": ("K steps as one CUDA graph (llsa_plan_create repeat=K), kernels chained by "
@@ -798,6 +799,9 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
+    if args.causal:
+        print(json.dumps({"impl": "reference", "unavailable": "the timed oracle arm covers the non-causal step only"}))
+        return
     from synthetic import WORKLOADS, make_config_inputs
 
     cfg = WORKLOADS[args.workload]
@@ -832,7 +836,8 @@ def run_reference(args):
         "config": {"workload": f"{cfg.name}: {cfg.describe()}", "B": cfg.B, "H": cfg.H, "N": cfg.N, "D": cfg.D,
                    "block": cfg.block, "levels": cfg.levels, "topk": cfg.topk,
                    "kv_len": 16 * cfg.topk + (cfg.topk if args.level1 else 0) + coarse_entries(cfg, args.all_top),
-                   "enrichment": enrichment_text(args), "heads_per_step": per_step,
+                   "enrichment": enrichment_text(args),
+                   "mask": "causal (LLSA_FLAG_CAUSAL)" if args.causal else "none (non-causal)", "heads_per_step": per_step,
                    "tokens_per_step": tokens_per_step},
         "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": pool.cores, "kind": "oracle",
                          "cpu_model": host_cpu_model(), "sample": sample},
@@ -852,7 +857,7 @@ def run_profile(args):
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     dev = {k: v.cuda() for k, v in make_config_inputs(cfg, with_do=True).items()}
     shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype,
-                           one_launch_select=args.one_launch_select, **enrichment(args))
+                           one_launch_select=args.one_launch_select, causal=args.causal, **enrichment(args))
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     for _ in range(args.warmup + args.steps):
         api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
@@ -886,6 +891,8 @@ def main():
                     help="the level-1 enrichment variant (each selected block's mean token in the list)")
     ap.add_argument("--grid-order", action="store_true",
                     help="inputs and outputs in row-major grid order (LLSA_FLAG_GRID_ORDER)")
+    ap.add_argument("--causal", action="store_true",
+                    help="causal attention (LLSA_FLAG_CAUSAL; bf16, default enrichment)")
     ap.add_argument("--one-launch-select", action="store_true",
                     help="pyramid and selection as one cooperative launch (LLSA_FLAG_ONE_LAUNCH_SELECT)")
     args = ap.parse_args()

@@ -123,6 +123,24 @@ typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
  * kernel does).
  */
 #define LLSA_FLAG_ONE_LAUNCH_SELECT 16
+/*
+ * Causal attention (LLSA GitHub README, usage section: the released kernels are non-causal
+ * only, to be addressed later; the pages define no causal variant, so this is a reading
+ * that keeps SDPA's is_causal=True meaning -- query position i sees key positions t <= i --
+ * and changes as little else as possible):
+ *  - selection: a level-l query token a picks only among key tokens j <= a (the non-causal
+ *    candidates with index <= a); a list with fewer than K such candidates ends in
+ *    LLSA_NO_PICK entries (lists stay ascending).  Scores and pooled queries are the
+ *    non-causal ones, so the choice of keys may depend on later queries of a coarse span;
+ *  - attention: a picked block j < p is seen whole by query block p, the block's own block
+ *    (j = p) with key t visible to query i only when t <= i, and a coarse level-l token j
+ *    only when j is below p's level-l ancestor (the token lies wholly before the block);
+ *  - index transpose: LLSA_NO_PICK entries are dropped (row_ptr[n_l] = number of picks).
+ * bf16 only (fp32 -> LLSA_ERR_UNSUPPORTED); combines with no other flag except
+ * LLSA_FLAG_ONE_LAUNCH_SELECT (ignored) and with no padding.
+ */
+#define LLSA_FLAG_CAUSAL 32
+#define LLSA_NO_PICK 0x7fffffff
 
 typedef struct {
   int32_t B, H, N, D;

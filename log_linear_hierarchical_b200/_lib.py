@@ -44,6 +44,8 @@ LLSA_FLAG_ALL_TOP = 2
 LLSA_FLAG_LEVEL1 = 4
 LLSA_FLAG_GRID_ORDER = 8
 LLSA_FLAG_ONE_LAUNCH_SELECT = 16
+LLSA_FLAG_CAUSAL = 32
+LLSA_NO_PICK = 0x7FFFFFFF
 
 
 _SP = ctypes.POINTER(LLSAShape)

@@ -29,7 +29,7 @@ class LLSAError(RuntimeError):
 
 def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, block: int = 16,
                log_bias: bool = False, all_top: bool = False, level1: bool = False, n_valid: int = 0,
-               grid_order: bool = False, one_launch_select: bool = False) -> LLSAShape:
+               grid_order: bool = False, one_launch_select: bool = False, causal: bool = False) -> LLSAShape:
     """``log_bias``: the log-count enrichment variant (LLSA_FLAG_LOG_BIAS); ``all_top``: the
     all-coarsest variant (LLSA_FLAG_ALL_TOP); ``level1``: the selected blocks' level-1 pooled
     tokens join the list (LLSA_FLAG_LEVEL1).  Any combination may be set.  ``n_valid``: the
@@ -37,11 +37,13 @@ def make_shape(B: int, H: int, N: int, D: int, topk: int, levels: int, dtype, bl
     ``grid_order``: token rows are in the row-major order of a square grid
     (LLSA_FLAG_GRID_ORDER); the path reads and writes them through its quadtree order.
     ``one_launch_select``: a step runs the pyramid and selection as one cooperative launch
-    (LLSA_FLAG_ONE_LAUNCH_SELECT; same results)."""
+    (LLSA_FLAG_ONE_LAUNCH_SELECT; same results).  ``causal``: keys at or before the query
+    only (LLSA_FLAG_CAUSAL; see include/llsa.h for the reading)."""
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     flags = ((_lib.LLSA_FLAG_LOG_BIAS if log_bias else 0) | (_lib.LLSA_FLAG_ALL_TOP if all_top else 0)
              | (_lib.LLSA_FLAG_LEVEL1 if level1 else 0) | (_lib.LLSA_FLAG_GRID_ORDER if grid_order else 0)
-             | (_lib.LLSA_FLAG_ONE_LAUNCH_SELECT if one_launch_select else 0))
+             | (_lib.LLSA_FLAG_ONE_LAUNCH_SELECT if one_launch_select else 0)
+             | (_lib.LLSA_FLAG_CAUSAL if causal else 0))
     return LLSAShape(B, H, N, D, block, topk, levels, code, flags, n_valid)
 
 
@@ -462,11 +464,13 @@ class _LLSAFunction(torch.autograd.Function):
 
 
 def llsa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk: int = 8, levels: int = 1,
-                   log_bias: bool = False, all_top: bool = False, level1: bool = False) -> torch.Tensor:
-    """Drop-in for ``F.scaled_dot_product_attention(q, k, v)`` (non-causal, no dropout) on
+                   log_bias: bool = False, all_top: bool = False, level1: bool = False,
+                   is_causal: bool = False) -> torch.Tensor:
+    """Drop-in for ``F.scaled_dot_product_attention(q, k, v, is_causal=...)`` (no dropout) on
     [B, H, N, D] CUDA tensors (D = 64 or 128), bf16 or fp32, with LLSA's hierarchical block-sparse KV lists.
-    ``log_bias``, ``all_top`` and ``level1`` select the enrichment variants (see make_shape)."""
-    flags = dict(log_bias=log_bias, all_top=all_top, level1=level1)
+    ``log_bias``, ``all_top`` and ``level1`` select the enrichment variants (see make_shape);
+    ``is_causal`` the causal reading (bf16, default enrichment)."""
+    flags = dict(log_bias=log_bias, all_top=all_top, level1=level1, causal=is_causal)
     return _LLSAFunction.apply(q, k, v, topk, levels, flags)
 
 

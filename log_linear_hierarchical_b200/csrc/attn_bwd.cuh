@@ -100,12 +100,13 @@ __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
 // One 16-token chunk of the query-major backward: dQ += dS K with dS = P (dP - Delta).
 // POOL (level-1 variant, fine chunks): the block-mean entry has score mean(S) + pool_bias
 // and dP mean(dP); its dS, times the mean K row, is dS / 16 added to each of the 16 dS.
-template <int D, bool MASK, bool POOL = false>
+// MASK, cmask and DIAG as in fwd_chunk (masked entries get P = 0, hence dS = 0).
+template <int D, bool MASK, bool POOL = false, bool DIAG = false>
 __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const uint32_t (&df)[D / 16][4],
                                          uint32_t ktile, uint32_t vtile, int valid, float scale_log2,
                                          const float (&lse2)[2], const float (&delta)[2], float (&dq)[D / 8][4],
                                          const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
-                                         int perm = 0) {
+                                         int perm = 0, uint32_t cmask = 0xffffffffu) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -131,7 +132,8 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const 
       const int r = e >> 1;
       float sb = s[n][e];
       if (MASK && bias_g && bias_g->log_bias && col < valid) sb += coarse_log_bias(*bias_g, c0 + col) * sqrt_d<D>();
-      const float p = (!MASK || col < valid) ? ex2(fmaf(sb, scale_log2, -lse2[r])) : 0.0f;
+      const bool vis = (!MASK || (col < valid && ((cmask >> col) & 1u))) && (!DIAG || col <= (lane >> 2) + 8 * r);
+      const float p = vis ? ex2(fmaf(sb, scale_log2, -lse2[r])) : 0.0f;
       ds[n][e] = POOL ? fmaf(p, dp[n][e] - delta[r], pds[r]) : p * (dp[n][e] - delta[r]);
     }
   mma_a_b<D>(dq, pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]), pack_bf16(ds[1][0], ds[1][1]),
@@ -153,6 +155,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
   // kernels back, so they are staged before waiting for the kernel ahead (see pdl_wait)
   extern __shared__ uint8_t dq_smem_raw[];
   constexpr bool PAD = LAYOUT == kPadded;
+  constexpr bool CAUSAL = LAYOUT == kCausal;
   constexpr int PERM = LAYOUT == kGrid ? 1 : 0;
   const Geometry& g = P.g;
   const BwdWorkspace W = bwd_workspace_layout(g);
@@ -175,6 +178,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     stage_coarse_rows<D>(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
     __syncthreads();
   }
+  const uint32_t cmask =
+      (CAUSAL && g.L >= 2) ? coarse_visible_mask(g, idx, cta_first / n1, cta_first % n1) : 0xffffffffu;
   const int first = cta_first + warp * kUnitBlocks;
   if (first >= total_blocks) {  // warp-uniform; no CTA-wide barrier after this point
     pdl_wait();
@@ -189,10 +194,16 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
   const uint32_t bar_qd = smem_u32(srow) + ((kUnitBlocks * K * 4 + 15) & ~15);
   const uint32_t bar_kv = bar_qd + 16;
 
-  for (int i = lane; i < nblk * K; i += 32)
+  for (int i = lane; i < nblk * K; i += 32) {
     // the first K/V row of each load: (b*H + h) * N + 16 j, computed here off the issue path
-    srow[i] = div_n1(g, first + div_k(g, i)) * g.N +
-              checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1) * kBlock;
+    // (a causal kNoPick entry: the complement of the block's own first row, as in the forward)
+    const int pick = __ldg(idx + g.idx_off[1] + (long long)first * K + i);
+    const int qb = first + div_k(g, i);
+    if (CAUSAL && pick == kNoPick)
+      srow[i] = ~(qb * kBlock);
+    else
+      srow[i] = div_n1(g, qb) * g.N + checked_index(pick, n1) * kBlock;
+  }
   if (lane == 0) {
     for (int b = 0; b < 2 + STAGES; ++b) mbar_init(bar_qd + 8 * b, 1);
     mbar_fence_init();
@@ -201,7 +212,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int row = srow[seq];
+    const int row = CAUSAL ? max(srow[seq], ~srow[seq]) : srow[seq];
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * TB;
@@ -308,7 +319,12 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
       if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
         dq_chunk<D, true>(qf, df, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - div_n1(g, gb) * g.N)),
                           P.scale_log2, lse2, delta, dq);
-      else
+      else if (CAUSAL) {
+        if (srow[seq] == gb * kBlock)
+          dq_chunk<D, false, false, true>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq);
+        else if (srow[seq] >= 0)
+          dq_chunk<D, false>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq);
+      } else
         dq_chunk<D, false, POOL>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
                                  pool_log_bias<D>(g), PERM);
       __syncwarp();
@@ -316,8 +332,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_bf16_kernel(
     }
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
-      dq_chunk<D, true>(qf, df, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock),
-                     P.scale_log2, lse2, delta, dq, &g, cc * kBlock);
+      dq_chunk<D, true>(qf, df, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock), P.scale_log2, lse2,
+                        delta, dq, &g, cc * kBlock, 0.f, 0, cmask >> (cc * kBlock));
     __syncwarp();
     {
       const int bhi = div_n1(g, gb);
@@ -355,6 +371,8 @@ __host__ __device__ constexpr bool kv_frags_in_regs() {
 // kvalid < 16: the key tile holds the last real token of a padded sequence, and its rows
 // from kvalid on are padding (zero rows) whose P^T and dS^T are masked to 0.
 // kvperm, qperm: the tile_row permutations of the key tile and of the query block's tiles.
+// kmask: key rows whose bit is clear are not attended (causal coarse entries); diag: the
+// causal diagonal pair (key row r is visible to query column c only when r <= c).
 // lsd: the query block's record (16 LSE * log2(e), then 16 Delta, in the shared-memory row
 // order of its tiles).
 template <int D, bool BIAS = false, bool POOL = false>
@@ -362,7 +380,7 @@ __device__ __forceinline__ void kv_scores(const uint32_t (&kf)[D / 16][4], const
                                           uint32_t kvtile, uint32_t qt, uint32_t dt, const float* lsd,
                                           float scale_log2, float (&pt)[2][4], float (&dst)[2][4],
                                           const float (&kb)[2], float pool_bias, int kvalid, int kvperm,
-                                          int qperm) {
+                                          int qperm, uint32_t kmask = 0xffffu, bool diag = false) {
   const int c2 = 2 * (lane_id() & 3);
   float st[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dpt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -422,13 +440,16 @@ __device__ __forceinline__ void kv_scores(const uint32_t (&kf)[D / 16][4], const
         dst[n][e] += da[n][e & 1];
       }
     }
-  if (kvalid < kBlock) {
+  if (kvalid < kBlock || kmask != 0xffffu || diag) {
     const int r0 = lane_id() >> 2;
 #pragma unroll
     for (int n = 0; n < 2; ++n)
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (r0 + 8 * (e >> 1) >= kvalid) pt[n][e] = dst[n][e] = 0.0f;
+      for (int e = 0; e < 4; ++e) {
+        const int kr = r0 + 8 * (e >> 1);  // key row; the query column is n * 8 + c2 + (e & 1)
+        if (kr >= kvalid || !((kmask >> kr) & 1u) || (diag && kr > n * 8 + c2 + (e & 1)))
+          pt[n][e] = dst[n][e] = 0.0f;
+      }
   }
 }
 
@@ -471,7 +492,9 @@ __host__ __device__ inline CtaSmem kv_smem(int nwarps) {
 // accumulates dK, dV.  `pair_block(i)` gives the flat query-block index of pair i.  If
 // `bar_tile` is non-zero the key tile is still arriving on that mbarrier (phase 0) and is
 // waited for after the first pair loads are issued.  Returns false (after draining the
-// copies in flight) if a wait timed out.
+// copies in flight) if a wait timed out.  kmask: see kv_scores.  diag_first (kCausal): pair
+// 0 is the key block's own query block (a causal CSR row lists only query blocks at or after
+// its key block, ascending, so the diagonal pair can only come first).
 template <int D, int STAGES, int LAYOUT, bool BIAS = false, bool POOL = false, class PairBlock>
 __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* tm_q, const CUtensorMap* tm_do,
                                           const float* __restrict__ lsd, uint32_t kvtile, uint32_t bar_tile,
@@ -479,7 +502,8 @@ __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* 
                                           uint32_t bar_ring, int npairs, PairBlock pair_block, float scale_log2,
                                           float (&dk)[D / 8][4], float (&dv)[D / 8][4],
                                           const float (&kbias)[2] = {0.f, 0.f}, float pool_bias = 0.f,
-                                          int kvalid = kBlock, int kvperm = 0) {
+                                          int kvalid = kBlock, int kvperm = 0, uint32_t kmask = 0xffffu,
+                                          bool diag_first = false) {
   constexpr int TB = tile_bytes<D>();
   constexpr int qperm = LAYOUT == kGrid ? 1 : 0;
   const int lane = lane_id();
@@ -516,7 +540,8 @@ __device__ __forceinline__ bool kv_stream(const Geometry& g, const CUtensorMap* 
     const uint32_t qt = ring + stage * 2 * TB;
     float pt[2][4], dst[2][4];
     kv_scores<D, BIAS, POOL>(kf, vf, kvtile, qt, qt + TB, slsd + stage * 2 * kBlock, scale_log2, pt, dst, kbias,
-                             pool_bias, kvalid, kvperm, qperm);
+                             pool_bias, kvalid, kvperm, qperm, kmask,
+                             LAYOUT == kCausal && i == 0 && diag_first);
     kv_accumulate<D>(pt, dst, qt, qt + TB, dk, dv, qperm);
     __syncwarp();
     if (i + STAGES < npairs) issue_pair(i + STAGES);
@@ -562,9 +587,9 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
       const int ch = t - r * CH;
       const int row = tile * kBlock + r;
       uint4 pk = make_uint4(0u, 0u, 0u, 0u), pv = make_uint4(0u, 0u, 0u, 0u);
-      if (row < g.coarse) {
-        int lev;
-        const int j = coarse_token(g, idx, bh, p0, row, lev);
+      int lev;
+      const int j = row < g.coarse ? coarse_token(g, idx, bh, p0, row, lev) : -1;
+      if (j >= 0) {  // entries past C and causal entries that are not attended stay zero
         const int nl = g.n[lev];
         const long long off = g.pyr_off[lev] + ((long long)bh * nl + j) * D + ch * 8;
         const float4 a = __ldg(reinterpret_cast<const float4*>(k_pyr + off));
@@ -582,6 +607,7 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
                    : "memory");
     }
   }
+  const uint32_t cmask = LAYOUT == kCausal ? coarse_visible_mask(g, idx, bh, p0) : 0xffffffffu;
   if (lane == 0) {
     for (int b = 0; b < STAGES; ++b) mbar_init(bar_ring + 8 * b, 1);
     mbar_fence_init();
@@ -602,8 +628,11 @@ __global__ void __launch_bounds__(32) attn_bwd_coarse_bf16_kernel(const __grid_c
     ok = kv_stream<D, STAGES, LAYOUT, true>(g, &tm_q, &tm_do, ws + W.lsd, kvt, 0u, ring, slsd, bar_ring, kBlock,
                                             [&](int i) { return first_block + i; }, P.scale_log2, dk, dv, kb);
   } else {
+    // causal: the tile's entries that the group's blocks attend (the same for all 16)
+    const uint32_t kmask = LAYOUT == kCausal ? (cmask >> (tile * kBlock)) & 0xffffu : 0xffffu;
     ok = kv_stream<D, STAGES, LAYOUT>(g, &tm_q, &tm_do, ws + W.lsd, kvt, 0u, ring, slsd, bar_ring, kBlock,
-                                      [&](int i) { return first_block + i; }, P.scale_log2, dk, dv);
+                                      [&](int i) { return first_block + i; }, P.scale_log2, dk, dv, {0.f, 0.f}, 0.f,
+                                      kBlock, 0, kmask);
   }
   if (!ok) return;
   const int r0 = lane >> 2;
@@ -1069,10 +1098,12 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
   };
   // real keys of this block (16 unless padded)
   const int kvalid = LAYOUT == kPadded ? min(kBlock, g.nv - j * kBlock) : kBlock;
+  // causal: whether the row's first query block is the key block itself
+  const bool diag_first = LAYOUT == kCausal && re > rs && __ldg(cl) == j;
   const bool ok = kv_stream<D, STAGES, LAYOUT, false, POOL>(g, &tm_q, &tm_do, ws + W.lsd, kvt, bar_kv, ring, slsd,
                                                             bar_ring, re - rs, pair_block, P.scale_log2, dk, dv,
                                                             {0.f, 0.f}, pool_log_bias<D>(g), kvalid,
-                                                            LAYOUT == kGrid ? 1 : 0);
+                                                            LAYOUT == kGrid ? 1 : 0, 0xffffu, diag_first);
   if (!ok) return;
   if (coarse_late) pdl_wait();
   // epilogue: scale dK, add the mean-pool adjoint of the ancestors' coarse gradients

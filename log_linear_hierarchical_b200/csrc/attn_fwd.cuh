@@ -147,7 +147,8 @@ __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint3
 }
 
 // Stage the C coarse rows of a pyramid (fp32) as bf16 16-row swizzled tiles; padding rows
-// (index >= C) are zero.  Row c is the pyramid row of coarse entry c (see coarse_token).
+// (index >= C) and causal entries that are not attended are zero.  Row c is the pyramid row
+// of coarse entry c (see coarse_token).
 // Threads `tid` = 0..nthreads-1 share the work (a warp or a whole CTA).
 template <int D>
 __device__ __forceinline__ void stage_coarse_rows(const Geometry& g, const float* __restrict__ pyr,
@@ -161,11 +162,14 @@ __device__ __forceinline__ void stage_coarse_rows(const Geometry& g, const float
     if (row < g.coarse) {
       int lev;
       const int j = coarse_token(g, idx, bh, p, row, lev);
-      const int nl = g.n[lev];
-      const float4* src = reinterpret_cast<const float4*>(pyr + g.pyr_off[lev] + ((long long)bh * nl + j) * D + ch * 8);
-      const float4 x = __ldg(src);
-      const float4 y = __ldg(src + 1);
-      packed = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+      if (j >= 0) {
+        const int nl = g.n[lev];
+        const float4* src =
+            reinterpret_cast<const float4*>(pyr + g.pyr_off[lev] + ((long long)bh * nl + j) * D + ch * 8);
+        const float4 x = __ldg(src);
+        const float4 y = __ldg(src + 1);
+        packed = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+      }
     }
     const uint32_t addr = dst + (row >> 4) * tile_bytes<D>() + tswz(row & 15, ch);
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(packed.x), "r"(packed.y), "r"(packed.z),
@@ -217,7 +221,7 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[D / 8][4], fl
 template <int D, int LAYOUT>
 __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, const Geometry& g, int row,
                                               uint32_t bar) {
-  if constexpr (LAYOUT == kFlat) {
+  if constexpr (flat_tile_map(LAYOUT)) {  // the 2-D map (make_tile_map makes the same choice)
 #pragma unroll
     for (int h = 0; h < D / 64; ++h) tma_load_2d(dst + h * kSubTileBytes, map, 64 * h, row, bar);
     return;
@@ -277,18 +281,20 @@ __device__ __forceinline__ void quad_row_sums(const float (&s)[2][4], float& t0,
 }
 
 // One 16-token chunk of the online softmax.  With MASK (the coarse chunks), columns >=
-// `valid` (the padding of the last coarse tile) are excluded and, under the log-count
-// variant, column c gets the bias of coarse entry c0 + c.  m holds the running row maxima
+// `valid` (the padding of the last coarse tile) and columns whose bit of `cmask` is clear
+// (causal entries that are not attended) are excluded and, under the log-count variant,
+// column c gets the bias of coarse entry c0 + c.  DIAG (causal, the query block's own key
+// block): key column c is visible to query row r only when c <= r.  m holds the running row maxima
 // of the scaled scores (log2 domain), l the per-lane partial row sums.
 // POOL (the level-1 variant, fine chunks only): the chunk's block mean is one more KV
 // entry.  Its score is the mean of the 16 scores (q . mean k = mean of q . k), plus
 // `pool_bias` (unscaled-dot units), and since its value is the mean of the 16 V rows its
 // weight p folds into the chunk as p / 16 added to each of the 16 probabilities.
-template <int D, bool MASK, bool POOL = false>
+template <int D, bool MASK, bool POOL = false, bool DIAG = false>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint32_t ktile, uint32_t vtile, int valid,
                                           float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[D / 8][4],
                                           const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
-                                          int perm = 0) {
+                                          int perm = 0, uint32_t cmask = 0xffffffffu) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt<D>(s, qf, ktile, perm);
@@ -304,9 +310,16 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint3
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = n * 8 + 2 * (lane & 3) + (e & 1);
-        if (col >= valid) s[n][e] = -INFINITY;
+        if (col >= valid || !((cmask >> col) & 1u)) s[n][e] = -INFINITY;
         else if (bias_g && bias_g->log_bias) s[n][e] += coarse_log_bias(*bias_g, c0 + col) * sqrt_d<D>();
       }
+  }
+  if (DIAG) {
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (n * 8 + 2 * (lane & 3) + (e & 1) > (lane >> 2) + 8 * (e >> 1)) s[n][e] = -INFINITY;
   }
   float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
   float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
@@ -405,6 +418,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   // kernels back, so they are staged before waiting for the kernel ahead (see pdl_wait)
   extern __shared__ uint8_t fwd_smem_raw[];
   constexpr bool PAD = LAYOUT == kPadded;
+  constexpr bool CAUSAL = LAYOUT == kCausal;
   constexpr int PERM = LAYOUT == kGrid ? 1 : 0;
   const Geometry& g = P.g;
   const int lane = lane_id();
@@ -425,6 +439,9 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     stage_coarse_rows<D>(g, v_pyr, idx, bh0, p0, cv, threadIdx.x, blockDim.x);
     __syncthreads();
   }
+  // causal: the coarse entries the CTA's blocks attend (the same ancestors for all 16)
+  const uint32_t cmask =
+      (CAUSAL && g.L >= 2) ? coarse_visible_mask(g, idx, cta_first / n1, cta_first % n1) : 0xffffffffu;
   pdl_wait();
   pdl_launch_dependents();
   const int first = cta_first + warp * kUnitBlocks;
@@ -437,10 +454,17 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
   const uint32_t bar_q = smem_u32(srow) + ((kUnitBlocks * K * 4 + 15) & ~15);
   const uint32_t bar_kv = bar_q + 16;
 
-  for (int i = lane; i < nblk * K; i += 32)
-    // the first K/V row of each load: (b*H + h) * N + 16 j, computed here off the issue path
-    srow[i] = div_n1(g, first + div_k(g, i)) * g.N +
-              checked_index(__ldg(idx + g.idx_off[1] + (long long)first * K + i), n1) * kBlock;
+  for (int i = lane; i < nblk * K; i += 32) {
+    // the first K/V row of each load: (b*H + h) * N + 16 j, computed here off the issue path;
+    // a causal list's kNoPick entry loads the block's own rows and is stored as their
+    // complement (negative), so that nothing is computed for it
+    const int pick = __ldg(idx + g.idx_off[1] + (long long)first * K + i);
+    const int qb = first + div_k(g, i);
+    if (CAUSAL && pick == kNoPick)
+      srow[i] = ~(qb * kBlock);
+    else
+      srow[i] = div_n1(g, qb) * g.N + checked_index(pick, n1) * kBlock;
+  }
   if (lane == 0) {
     for (int b = 0; b < 2 + STAGES; ++b) mbar_init(bar_q + 8 * b, 1);
     mbar_fence_init();
@@ -449,7 +473,7 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
 
   const int total_loads = nblk * K;
   auto issue_kv = [&](int seq) {
-    const int row = srow[seq];
+    const int row = CAUSAL ? max(srow[seq], ~srow[seq]) : srow[seq];
     const int stage = seq % STAGES;
     const uint32_t bar = bar_kv + 8 * stage;
     const uint32_t dst = ring + stage * 2 * TB;
@@ -499,7 +523,12 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
       const uint32_t kt = ring + stage * 2 * TB;
       if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
         fwd_chunk<D, true>(qf, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - bh_i * g.N)), P.scale_log2, m, l, acc);
-      else
+      else if (CAUSAL) {  // kNoPick: nothing; the block's own keys: the causal diagonal
+        if (srow[seq] == gb * kBlock)
+          fwd_chunk<D, false, false, true>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc);
+        else if (srow[seq] >= 0)
+          fwd_chunk<D, false>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc);
+      } else
         fwd_chunk<D, false, POOL>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias<D>(g),
                                   PERM);
       __syncwarp();
@@ -507,8 +536,8 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
     }
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
-      fwd_chunk<D, true>(qf, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock),
-                      P.scale_log2, m, l, acc, &g, cc * kBlock);
+      fwd_chunk<D, true>(qf, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock), P.scale_log2, m, l,
+                         acc, &g, cc * kBlock, 0.f, 0, cmask >> (cc * kBlock));
 
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 1);
     l[0] += __shfl_xor_sync(0xffffffffu, l[0], 2);

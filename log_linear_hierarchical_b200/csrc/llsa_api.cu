@@ -39,7 +39,7 @@ llsa_status validate(const llsa_shape* s) {
     return LLSA_ERR_INVALID_ARG;
   if (s->dtype != LLSA_BF16 && s->dtype != LLSA_F32) return LLSA_ERR_INVALID_ARG;
   if (s->flags & ~(LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP | LLSA_FLAG_LEVEL1 | LLSA_FLAG_GRID_ORDER |
-                   LLSA_FLAG_ONE_LAUNCH_SELECT))
+                   LLSA_FLAG_ONE_LAUNCH_SELECT | LLSA_FLAG_CAUSAL))
     return LLSA_ERR_INVALID_ARG;  // unknown flag bits
   if (s->n_valid < 0 || s->n_valid > s->N) return LLSA_ERR_INVALID_ARG;
   // N: any multiple of 16^L (the pages' implementation wants powers of two for N and topk;
@@ -61,6 +61,12 @@ llsa_status validate(const llsa_shape* s) {
     const long long span = 1LL << (4 * s->levels);
     if (s->topk > (s->n_valid + span - 1) / span) return LLSA_ERR_INVALID_ARG;  // K real coarsest tokens
     if (s->flags & ~LLSA_FLAG_ONE_LAUNCH_SELECT) return LLSA_ERR_UNSUPPORTED;  // default enrichment only
+  }
+  if (s->flags & LLSA_FLAG_CAUSAL) {  // bf16, the default enrichment, no padding, no grid order
+    if (s->dtype != LLSA_BF16) return LLSA_ERR_UNSUPPORTED;
+    if (s->flags & (LLSA_FLAG_LOG_BIAS | LLSA_FLAG_ALL_TOP | LLSA_FLAG_LEVEL1 | LLSA_FLAG_GRID_ORDER))
+      return LLSA_ERR_UNSUPPORTED;
+    if (s->n_valid != 0 && s->n_valid < s->N) return LLSA_ERR_UNSUPPORTED;
   }
   if (s->flags & LLSA_FLAG_GRID_ORDER) {  // a square grid of side 2^(log2 N / 2), 16 x 16 at least
     if (!is_pow2(s->N) || (ilog2(s->N) & 1)) return LLSA_ERR_INVALID_ARG;
@@ -100,6 +106,7 @@ Geometry make_geometry(const llsa_shape* s) {
   g.nv = (s->n_valid > 0 && s->n_valid < s->N) ? s->n_valid : s->N;
   g.grid = (s->flags & LLSA_FLAG_GRID_ORDER) ? 1 : 0;
   g.log_g = g.grid ? ilog2(s->N) / 2 : 0;
+  g.causal = (s->flags & LLSA_FLAG_CAUSAL) ? 1 : 0;
   for (int l = 0; l <= kMaxLevels; ++l) g.m[l] = l <= g.L ? (int)((g.nv + (1LL << (4 * l)) - 1) >> (4 * l)) : 0;
   return g;
 }
@@ -168,7 +175,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool make_tile_map(CUtensorMap* m, const void* base, const Geometry& g) {
   auto fn = encode_fn();
   if (!fn) return false;
-  if (g.grid) {  // the heads' grids stacked: pixel rows of all heads, G pixels each
+  const int lay = layout_of(g);  // the rank here must match the kernels' tma_load_tile<D, lay>
+  if (lay == kGrid) {  // the heads' grids stacked: pixel rows of all heads, G pixels each
     const cuuint64_t G = 1ULL << g.log_g;
     cuuint64_t dims[3] = {(cuuint64_t)g.D, G, (cuuint64_t)g.BH * G};
     cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, G * g.D * 2};
@@ -178,7 +186,7 @@ bool make_tile_map(CUtensorMap* m, const void* base, const Geometry& g) {
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   }
-  if (g.nv == g.N) {  // no padding: one flat [B*H*N][D] view (cheaper per copy than 3-D)
+  if (flat_tile_map(lay)) {  // no padding: one flat [B*H*N][D] view (cheaper per copy than 3-D)
     cuuint64_t dims[2] = {(cuuint64_t)g.D, (cuuint64_t)g.BH * g.N};
     cuuint64_t strides[1] = {(cuuint64_t)g.D * 2};
     cuuint32_t box[2] = {64u, (cuuint32_t)kBlock};
@@ -383,9 +391,6 @@ namespace {
 // level-1 CSR and can run beside the query side too.
 constexpr unsigned kQuerySide = 1, kKeySide = 2, kOrder = 4;
 
-// The bf16 attention kernels' addressing (Layout) for this geometry.
-int layout_of(const Geometry& g) { return g.grid ? kGrid : (g.nv < g.N ? kPadded : kFlat); }
-
 // The instantiation of each bf16 attention kernel for a geometry: its Layout, and the
 // level-1 variant (POOL), which padding does not combine with.
 template <int D>
@@ -393,6 +398,7 @@ auto pick_fwd(const Geometry& g) {
   constexpr int S = kFwdStages;
   const int lay = layout_of(g);
   if (lay == kPadded) return attn_fwd_bf16_kernel<D, S, false, kPadded>;
+  if (lay == kCausal) return attn_fwd_bf16_kernel<D, S, false, kCausal>;
   if (lay == kGrid) return g.pool1 ? attn_fwd_bf16_kernel<D, S, true, kGrid> : attn_fwd_bf16_kernel<D, S, false, kGrid>;
   return g.pool1 ? attn_fwd_bf16_kernel<D, S, true, kFlat> : attn_fwd_bf16_kernel<D, S, false, kFlat>;
 }
@@ -401,6 +407,7 @@ auto pick_dq(const Geometry& g) {
   constexpr int S = kDqStages;
   const int lay = layout_of(g);
   if (lay == kPadded) return attn_bwd_dq_bf16_kernel<D, S, false, kPadded>;
+  if (lay == kCausal) return attn_bwd_dq_bf16_kernel<D, S, false, kCausal>;
   if (lay == kGrid)
     return g.pool1 ? attn_bwd_dq_bf16_kernel<D, S, true, kGrid> : attn_bwd_dq_bf16_kernel<D, S, false, kGrid>;
   return g.pool1 ? attn_bwd_dq_bf16_kernel<D, S, true, kFlat> : attn_bwd_dq_bf16_kernel<D, S, false, kFlat>;
@@ -410,6 +417,7 @@ auto pick_dkdv(const Geometry& g) {
   constexpr int S = kDkvStages;
   const int lay = layout_of(g);
   if (lay == kPadded) return attn_bwd_dkdv_bf16_kernel<D, S, false, kPadded>;
+  if (lay == kCausal) return attn_bwd_dkdv_bf16_kernel<D, S, false, kCausal>;
   if (lay == kGrid)
     return g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, S, true, kGrid> : attn_bwd_dkdv_bf16_kernel<D, S, false, kGrid>;
   return g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, S, true, kFlat> : attn_bwd_dkdv_bf16_kernel<D, S, false, kFlat>;
@@ -419,6 +427,7 @@ auto pick_coarse(const Geometry& g) {
   const int lay = layout_of(g);
   if (lay == kPadded) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kPadded>;
   if (lay == kGrid) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kGrid>;
+  if (lay == kCausal) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kCausal>;
   return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kFlat>;
 }
 
@@ -624,7 +633,7 @@ llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* 
 // children selection).
 // Requested by LLSA_FLAG_ONE_LAUNCH_SELECT.
 bool fused_pyramid_select(const Geometry& g, const llsa_shape* s) {
-  return (s->flags & LLSA_FLAG_ONE_LAUNCH_SELECT) && s->dtype == LLSA_BF16 && g.L >= 2 && small_top(g) &&
+  return (s->flags & LLSA_FLAG_ONE_LAUNCH_SELECT) && !g.causal && s->dtype == LLSA_BF16 && g.L >= 2 && small_top(g) &&
          (g.K == 2 || g.K == 4 || g.K == 8 || g.K == 16);
 }
 

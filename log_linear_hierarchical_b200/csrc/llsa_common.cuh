@@ -61,7 +61,12 @@ struct Geometry {
                                          // row-major order of a G x G grid (G = 2^log_g); the
                                          // path works in its quadtree (Z) order
   int log_g;
+  int causal;                            // LLSA_FLAG_CAUSAL: keys at or before the query only
 };
+
+// The entry of a causal selection list that holds no pick (a query token with fewer than K
+// candidates at or before it); as the largest int it keeps every list ascending.
+constexpr int kNoPick = 0x7fffffff;
 
 // Even bits of x, packed: bit 2i of x becomes bit i.
 __host__ __device__ inline int compact_even_bits(int x) {
@@ -90,8 +95,16 @@ __host__ __device__ inline long long token_row(const Geometry& g, int bh, int t)
 // parameter, so the default instantiation carries no per-access test:
 //   kFlat:   [B*H*N][D] rows in quadtree order (flat 2-D tensor maps);
 //   kPadded: the same with rows at or past n_valid as padding (3-D maps read them as zeros);
-//   kGrid:   row-major G x G grids (LLSA_FLAG_GRID_ORDER: 4-D patch maps, the tile_row map).
-enum Layout : int { kFlat = 0, kPadded = 1, kGrid = 2 };
+//   kGrid:   row-major G x G grids (LLSA_FLAG_GRID_ORDER: 3-D patch maps, the tile_row map);
+//   kCausal: flat rows under LLSA_FLAG_CAUSAL (diagonal blocks masked element-wise, lists
+//            that may end in kNoPick, coarse entries attended only before the block).
+enum Layout : int { kFlat = 0, kPadded = 1, kGrid = 2, kCausal = 3 };
+
+// The layout of a geometry, and whether its tile tensor map is the flat 2-D [B*H*N][D] view
+// (kFlat, kCausal) rather than a 3-D one: the host's tensor map and the kernels' copy
+// instruction must agree on the rank.
+inline int layout_of(const Geometry& g) { return g.causal ? kCausal : g.grid ? kGrid : (g.nv < g.N ? kPadded : kFlat); }
+__host__ __device__ constexpr bool flat_tile_map(int layout) { return layout == kFlat || layout == kCausal; }
 
 template <int LAYOUT>
 __device__ __forceinline__ long long token_row(const Geometry& g, int bh, int t) {
@@ -154,6 +167,8 @@ __device__ __forceinline__ int checked_index(int v, int n) {
 // Token index (in its level) of coarse entry c of level-1 query block p of head bh: slot
 // c % K of the list that p's level-l ancestor selected, or, in the level-L part of the
 // all-coarsest variant, token c - top_first.  The index read from `idx` is range-checked.
+// Under LLSA_FLAG_CAUSAL an entry is attended only if its token lies wholly before the block,
+// i.e. its index is below the ancestor's (kNoPick and the ancestor itself are not); -1 then.
 __device__ __forceinline__ int coarse_token(const Geometry& g, const int* __restrict__ idx, int bh, int p, int c,
                                             int& lev) {
   if (c >= g.top_first) {
@@ -164,7 +179,23 @@ __device__ __forceinline__ int coarse_token(const Geometry& g, const int* __rest
   const int nl = g.n[lev];
   const int anc = p >> (4 * (lev - 1));  // p / 16^(l-1)
   const int slot = c - (lev - 2) * g.K;
-  return checked_index(__ldg(idx + g.idx_off[lev] + ((long long)bh * nl + anc) * g.K + slot), nl);
+  const int j = __ldg(idx + g.idx_off[lev] + ((long long)bh * nl + anc) * g.K + slot);
+  if (g.causal && j >= anc) return -1;
+  return checked_index(j, nl);
+}
+
+// Bit c set: coarse entry c of query block p is attended (every entry unless causal).
+// Called by a whole warp; C <= 32.
+__device__ __forceinline__ uint32_t coarse_visible_mask(const Geometry& g, const int* __restrict__ idx, int bh,
+                                                        int p) {
+  if (!g.causal) return 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  bool vis = false;
+  if (lane < g.coarse) {
+    int lev;
+    vis = coarse_token(g, idx, bh, p, lane, lev) >= 0;
+  }
+  return __ballot_sync(0xffffffffu, vis);
 }
 
 // ---------------------------------------------------------------------------- smem / swizzle

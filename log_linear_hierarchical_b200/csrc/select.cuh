@@ -59,8 +59,8 @@ __device__ __forceinline__ void warp_topk(uint32_t* krow, int nc, int K, int* wr
   for (int r = 0; r < K; ++r) {
     const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
     const uint32_t w = __reduce_min_sync(0xffffffffu, bk == m ? (uint32_t)bc : 0x7fffffffu);
-    if (lane == 0) wrow[r] = (int)w;
-    if (bc == (int)w && bk == m) {  // the owner drops its winner and finds its next best
+    if (lane == 0) wrow[r] = (int)w;  // 0x7fffffff: no candidate left (a short causal list)
+    if (m != 0u && bc == (int)w && bk == m) {  // the owner drops its winner and finds its next best
       krow[w] = 0u;
       bk = 0u;
       bc = 0x7fffffff;
@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
     const int np = g.n[level + 1];
     const int* prow = parent_idx + ((long long)bh * np + a0 / kBlock) * K;
     for (int i = tid; i < nc; i += kSelThreads) {
-      const int c = checked_index(__ldg(prow + i / kBlock), np);
-      cand[i] = c * kBlock + (i % kBlock);
+      const int raw = __ldg(prow + i / kBlock);  // a causal parent list may end in kNoPick: no children
+      cand[i] = (g.causal && raw == kNoPick) ? -1 : checked_index(raw, np) * kBlock + (i % kBlock);
     }
   }
   __syncthreads();
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
     for (int i = tid; i < cn * (D / 4); i += kSelThreads) {
       const int r = i / (D / 4);
       const int piece = i - r * (D / 4);
-      const int key = sparse ? cand[c0 + r] : c0 + r;
+      const int key = max(sparse ? cand[c0 + r] : c0 + r, 0);
       const float4 v = __ldg(reinterpret_cast<const float4*>(kp + ((long long)bh * n + key) * D) + piece);
       *reinterpret_cast<float4*>(ks + r * RS + piece * 4) = v;
     }
@@ -171,10 +171,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
         for (int v = 0; v < 4; ++v) {
           const int cc = c + v * tpq;
           if (qi < gq && cc < cn) {
-            // empty tokens of a padded sequence (index >= the level's real count) are never
+            // empty tokens of a padded sequence (index >= the level's real count), missing
+            // children and, under the causal rule, keys after the query token are never
             // candidates: key 0 marks a removed candidate
             const int key = sparse ? cand[c0 + cc] : c0 + cc;
-            sk[qi * nc + c0 + cc] = key < g.m[level] ? score_key(acc[u][v]) : 0u;
+            const bool ok = key >= 0 && key < g.m[level] && (!g.causal || key <= a0 + qi);
+            sk[qi * nc + c0 + cc] = ok ? score_key(acc[u][v]) : 0u;
           }
         }
       }
@@ -192,9 +194,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geometry g, int lev
     int* orow = out_idx + ((long long)bh * n + a0 + qi) * K;
     for (int r = lane; r < K; r += 32) {
       const int mine = min(max(wrow[r], 0), nc - 1);
-      int rank = 0;
-      for (int r2 = 0; r2 < K; ++r2) rank += wrow[r2] < wrow[r];
-      orow[rank] = sparse ? cand[mine] : mine;
+      int rank = 0;  // rounds without a winner (0x7fffffff) rank last, in round order
+      for (int r2 = 0; r2 < K; ++r2) rank += wrow[r2] < wrow[r] || (wrow[r2] == wrow[r] && r2 < r);
+      orow[rank] = wrow[r] == 0x7fffffff ? kNoPick : (sparse ? cand[mine] : mine);
     }
     __syncwarp();
   }
@@ -253,7 +255,10 @@ __device__ __forceinline__ void select_children_unit(const Geometry& g, int leve
   const int np = g.n[level + 1];
   const int* prow = parent_idx + ((long long)bh * np + a0 / kBlock) * K;
   __syncthreads();  // the previous unit's shared rows are no longer read
-  for (int i = tid; i < NC; i += kSelThreads) cand[i] = checked_index(ld_in<RO>(prow + i / kBlock), np) * kBlock + (i % kBlock);
+  for (int i = tid; i < NC; i += kSelThreads) {
+    const int raw = ld_in<RO>(prow + i / kBlock);  // a causal parent list may end in kNoPick
+    cand[i] = (g.causal && raw == kNoPick) ? -1 : checked_index(raw, np) * kBlock + (i % kBlock);
+  }
 #pragma unroll
   for (int u = 0; u < QP; ++u) reinterpret_cast<float4*>(qs)[tid + u * kSelThreads] = qv[u];
   __syncthreads();
@@ -267,7 +272,7 @@ __device__ __forceinline__ void select_children_unit(const Geometry& g, int leve
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = tid + (b0 + u) * kSelThreads;
-      v[u] = ld_in<RO>(reinterpret_cast<const float4*>(kp + ((long long)bh * n + cand[i / PR]) * D) + (i % PR));
+      v[u] = ld_in<RO>(reinterpret_cast<const float4*>(kp + ((long long)bh * n + max(cand[i / PR], 0)) * D) + (i % PR));
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -310,7 +315,8 @@ __device__ __forceinline__ void select_children_unit(const Geometry& g, int leve
   for (int u = 0; u < 2; ++u) {
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-      key[u][j] = cand[lane + 32 * j] < mreal ? score_key(acc[u][j]) : 0u;
+      const int c = cand[lane + 32 * j];  // missing children and (causal) keys after the query: none
+      key[u][j] = (c >= 0 && c < mreal && (!g.causal || c <= a0 + 2 * warp + u)) ? score_key(acc[u][j]) : 0u;
       ci[u][j] = lane + 32 * j;
     }
 #pragma unroll
@@ -326,7 +332,7 @@ __device__ __forceinline__ void select_children_unit(const Geometry& g, int leve
           ci[u][j + 1] = tc;
         }
     bk[u] = key[u][0];
-    bc[u] = ci[u][0];
+    bc[u] = key[u][0] ? ci[u][0] : 0x7fffffff;
   }
   int win[2] = {0, 0};
 #pragma unroll 1
@@ -356,12 +362,15 @@ __device__ __forceinline__ void select_children_unit(const Geometry& g, int leve
   // ascending order: each winner's rank is the number of smaller winners
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
-    int rank = 0;
+    int rank = 0;  // rounds without a winner (0x7fffffff) rank last, in round order
 #pragma unroll
-    for (int r2 = 0; r2 < K; ++r2) rank += __shfl_sync(0xffffffffu, win[u], r2) < win[u];
+    for (int r2 = 0; r2 < K; ++r2) {
+      const int w2 = __shfl_sync(0xffffffffu, win[u], r2);
+      rank += w2 < win[u] || (w2 == win[u] && r2 < lane);
+    }
     if (lane < K) {
       int* orow = out_idx + ((long long)bh * n + a0 + 2 * warp + u) * K;
-      orow[rank] = cand[min(max(win[u], 0), NC - 1)];
+      orow[rank] = win[u] == 0x7fffffff ? kNoPick : cand[min(max(win[u], 0), NC - 1)];
     }
   }
 }
@@ -474,7 +483,8 @@ __device__ __forceinline__ void coarsest_small_unit(const Geometry& g, float* __
     int bc = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      key[j] = lane + 32 * j < g.m[L] ? score_key(acc[j]) : 0u;  // real tokens only
+      const int c = lane + 32 * j;  // real tokens only; under the causal rule none after a
+      key[j] = (c < g.m[L] && (!g.causal || c <= a)) ? score_key(acc[j]) : 0u;
       if (key[j] > bk) {
         bk = key[j];
         bc = lane + 32 * j;
@@ -498,9 +508,12 @@ __device__ __forceinline__ void coarsest_small_unit(const Geometry& g, float* __
         }
       }
     }
-    int rank = 0;
-    for (int r2 = 0; r2 < K; ++r2) rank += __shfl_sync(0xffffffffu, win, r2) < win;
-    if (lane < K) idx[g.idx_off[L] + ((long long)bh * n + a) * K + rank] = min(max(win, 0), n - 1);
+    int rank = 0;  // rounds without a winner (0x7fffffff) rank last, in round order
+    for (int r2 = 0; r2 < K; ++r2) {
+      const int w2 = __shfl_sync(0xffffffffu, win, r2);
+      rank += w2 < win || (w2 == win && r2 < lane);
+    }
+    if (lane < K) idx[g.idx_off[L] + ((long long)bh * n + a) * K + rank] = win == 0x7fffffff ? kNoPick : min(max(win, 0), n - 1);
   }
 }
 

@@ -3,8 +3,9 @@
 // it, and building a dense query x key mask for that would cost O(n^2)).
 //
 // For each problem (level l, batch b, head h) the n_l x K list idx becomes a CSR matrix
-// (row_ptr, col) of the inverse relation with queries ascending in every row.  It is a
-// two-digit stable counting sort of the E = n_l * K entries, with no atomics anywhere:
+// (row_ptr, col) of the inverse relation with queries ascending in every row; kNoPick
+// entries (the empty slots of causal lists) are dropped, so row_ptr[n_l] counts the picks.
+// It is a two-digit stable counting sort of the E = n_l * K entries, with no atomics:
 //
 //   1. transpose_hist_kernel    one CTA per 4096-entry tile: per-warp bucket counts
 //                               (bucket = key / W, at most 64 buckets) via __match_any_sync,
@@ -79,6 +80,7 @@ __device__ __forceinline__ void tr_warp_bucket_counts(const int* __restrict__ ke
     const int e = base + lane;
     bool valid = e < seg_end;
     int key = valid ? __ldg(keys + e) : 0;
+    if (valid && key == kNoPick) valid = false;  // a short causal list's empty slot: no entry
     if (valid && (unsigned)key >= (unsigned)n) {
       record_error(LLSA_ERR_INTERNAL);
       valid = false;

@@ -21,11 +21,11 @@ TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 
 def run_gpu(B, H, N, D, topk, levels, dtype, inputs, backward=True, device="cuda", log_bias=False, all_top=False,
-            level1=False, n_valid=0, grid_order=False):
+            level1=False, n_valid=0, grid_order=False, causal=False):
     """All five calls on one stream; returns CPU tensors of every output."""
     tdt = TORCH_DTYPE[dtype]
     shape = api.make_shape(B, H, N, D, topk, levels, tdt, log_bias=log_bias, all_top=all_top,
-                           level1=level1, n_valid=n_valid, grid_order=grid_order)
+                           level1=level1, n_valid=n_valid, grid_order=grid_order, causal=causal)
     dev = {k: v.to(device) for k, v in inputs.items()}
     buf = api.LLSABuffers.allocate(shape, device, tdt)
     assert api.llsa_device_status() == 0

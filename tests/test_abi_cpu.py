@@ -139,13 +139,32 @@ def test_step_and_plan_rejected_before_launch(lib):
 
 def test_flags_validated(lib):
     s = shape()
-    # any combination of LOG_BIAS (1), ALL_TOP (2), LEVEL1 (4), GRID_ORDER (8), ONE_LAUNCH_SELECT (16)
+    # any combination of LOG_BIAS (1), ALL_TOP (2), LEVEL1 (4), GRID_ORDER (8), ONE_LAUNCH_SELECT (16);
+    # CAUSAL (32) has its own rules below
     for good in range(1, 32):
         s.flags = good
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 0, good
-    for bad in (32, 64, 1 << 30, -1):
+    for bad in (64, 128, 1 << 30, -1):
         s.flags = bad
         assert lib.llsa_validate_shape(ctypes.byref(s)) == 1, bad
+
+
+def test_causal_rules(lib):
+    causal = _lib.LLSA_FLAG_CAUSAL
+    s = shape()
+    for ok in (causal, causal | _lib.LLSA_FLAG_ONE_LAUNCH_SELECT):
+        s.flags = ok
+        assert lib.llsa_validate_shape(ctypes.byref(s)) == 0, ok
+    for other in (_lib.LLSA_FLAG_LOG_BIAS, _lib.LLSA_FLAG_ALL_TOP, _lib.LLSA_FLAG_LEVEL1, _lib.LLSA_FLAG_GRID_ORDER):
+        s.flags = causal | other
+        assert lib.llsa_validate_shape(ctypes.byref(s)) == 2, other     # UNSUPPORTED
+    f32 = shape(dtype=1)
+    f32.flags = causal
+    assert lib.llsa_validate_shape(ctypes.byref(f32)) == 2
+    padded = api.make_shape(1, 2, 4096, 64, 4, 2, 0, n_valid=3000, causal=True)
+    assert lib.llsa_validate_shape(ctypes.byref(padded)) == 2
+    assert api.make_shape(1, 2, 4096, 64, 4, 2, 0, causal=True).flags == causal == 32
+    assert _lib.LLSA_NO_PICK == 2 ** 31 - 1
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True).flags == _lib.LLSA_FLAG_LOG_BIAS
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, log_bias=True, all_top=True).flags == 3
     assert api.make_shape(1, 6, 65536, 64, 8, 3, 0, level1=True).flags == _lib.LLSA_FLAG_LEVEL1 == 4

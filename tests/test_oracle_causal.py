@@ -108,9 +108,11 @@ def test_two_level_selection_is_brute_force_under_the_hierarchical_rule():
         parents = [c for c in idx[1][0, 0, a // 16] if c != NP]
         cand = np.array(sorted(16 * c + r for c in parents for r in range(16) if 16 * c + r <= a))
         assert idx[0][0, 0, a].tolist() == brute_force_topk(s1[a, cand], cand, K), a
-    # NO_PICK only where fewer than K candidates exist, and lists stay ascending
+    # real picks strictly ascending, then only NO_PICK
     for lv in idx:
-        assert np.all(np.diff(lv.astype(np.int64), axis=-1) > 0)
+        real = lv != NP
+        assert np.all(real[..., :-1] >= real[..., 1:])
+        assert np.all((np.diff(lv.astype(np.int64), axis=-1) > 0) | ~real[..., 1:])
 
 
 def dense_causal_mask(N, idx):
