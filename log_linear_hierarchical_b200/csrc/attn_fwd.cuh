@@ -283,18 +283,18 @@ __device__ __forceinline__ void quad_row_sums(const float (&s)[2][4], float& t0,
 // One 16-token chunk of the online softmax.  With MASK (the coarse chunks), columns >=
 // `valid` (the padding of the last coarse tile) and columns whose bit of `cmask` is clear
 // (causal entries that are not attended) are excluded and, under the log-count variant,
-// column c gets the bias of coarse entry c0 + c.  DIAG (causal, the query block's own key
-// block): key column c is visible to query row r only when c <= r.  m holds the running row maxima
+// column c gets the bias of coarse entry c0 + c.  CAUSAL with `diag` (the query block's own
+// key block): key column c is visible to query row r only when c <= r.  m holds the running row maxima
 // of the scaled scores (log2 domain), l the per-lane partial row sums.
 // POOL (the level-1 variant, fine chunks only): the chunk's block mean is one more KV
 // entry.  Its score is the mean of the 16 scores (q . mean k = mean of q . k), plus
 // `pool_bias` (unscaled-dot units), and since its value is the mean of the 16 V rows its
 // weight p folds into the chunk as p / 16 added to each of the 16 probabilities.
-template <int D, bool MASK, bool POOL = false, bool DIAG = false>
+template <int D, bool MASK, bool POOL = false, bool CAUSAL = false>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint32_t ktile, uint32_t vtile, int valid,
                                           float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[D / 8][4],
                                           const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
-                                          int perm = 0, uint32_t cmask = 0xffffffffu) {
+                                          int perm = 0, uint32_t cmask = 0xffffffffu, bool diag = false) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt<D>(s, qf, ktile, perm);
@@ -314,7 +314,7 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint3
         else if (bias_g && bias_g->log_bias) s[n][e] += coarse_log_bias(*bias_g, c0 + col) * sqrt_d<D>();
       }
   }
-  if (DIAG) {
+  if (CAUSAL && diag) {
 #pragma unroll
     for (int n = 0; n < 2; ++n)
 #pragma unroll
@@ -407,7 +407,7 @@ __host__ __device__ inline CtaSmem fwd_smem(const Geometry& g, int nwarps) {
 // holds the last real token masks its padding keys (which arrive as zero rows), and padding
 // queries write O = 0 and LSE = 0.
 template <int D, int STAGES, bool POOL, int LAYOUT>
-__global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                             const __grid_constant__ CUtensorMap tm_k,
                                                             const __grid_constant__ CUtensorMap tm_v, AttnParams P,
                                                             const float* __restrict__ k_pyr,
@@ -524,10 +524,10 @@ __global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(const __grid_constan
       if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
         fwd_chunk<D, true>(qf, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - bh_i * g.N)), P.scale_log2, m, l, acc);
       else if (CAUSAL) {  // kNoPick: nothing; the block's own keys: the causal diagonal
-        if (srow[seq] == gb * kBlock)
-          fwd_chunk<D, false, false, true>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc);
-        else if (srow[seq] >= 0)
-          fwd_chunk<D, false>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc);
+        const int r = srow[seq];
+        if (r >= 0)
+          fwd_chunk<D, false, false, true>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, 0.f, 0,
+                                           0xffffffffu, r == gb * kBlock);
       } else
         fwd_chunk<D, false, POOL>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias<D>(g),
                                   PERM);
