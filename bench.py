@@ -262,6 +262,16 @@ def measure_gather_peak(api, torch, stream, sms: int) -> dict:
     return best
 
 
+def run_probe(args):
+    """Only the L2 gather ceiling (llsa_gather_probe sweep), one JSON line: for profilers."""
+    import torch
+
+    from log_linear_hierarchical_b200 import api
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    best = measure_gather_peak(api, torch, torch.cuda.current_stream(), sms)
+    print(json.dumps({"gather_probe": best}))
+
+
 def enrichment(args) -> dict:
     """Keyword arguments of the enrichment variants chosen on the command line."""
     return dict(log_bias=args.log_bias, all_top=args.all_top, level1=args.level1)
@@ -883,6 +893,7 @@ def main():
                     help="synthetic workload (default: the headline N=65536 step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--profile", action="store_true", help="run only the steps (for ncu), print no metric")
+    ap.add_argument("--probe", action="store_true", help="run only the L2 gather-ceiling sweep (for ncu)")
     ap.add_argument("--log-bias", action="store_true",
                     help="the log-count enrichment variant (ln 16^l on level-l coarse scores)")
     ap.add_argument("--all-top", action="store_true",
@@ -898,7 +909,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.profile:
+    if args.probe:
+        run_probe(args)
+    elif args.profile:
         run_profile(args)
     elif args.impl == "reference":
         run_reference(args)
