@@ -100,13 +100,13 @@ __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
 // One 16-token chunk of the query-major backward: dQ += dS K with dS = P (dP - Delta).
 // POOL (level-1 variant, fine chunks): the block-mean entry has score mean(S) + pool_bias
 // and dP mean(dP); its dS, times the mean K row, is dS / 16 added to each of the 16 dS.
-// MASK, cmask, CAUSAL and diag as in fwd_chunk (masked entries get P = 0, hence dS = 0).
+// MASK, cmask, CAUSAL and shift as in fwd_chunk (masked entries get P = 0, hence dS = 0).
 template <int D, bool MASK, bool POOL = false, bool CAUSAL = false>
 __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const uint32_t (&df)[D / 16][4],
                                          uint32_t ktile, uint32_t vtile, int valid, float scale_log2,
                                          const float (&lse2)[2], const float (&delta)[2], float (&dq)[D / 8][4],
                                          const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
-                                         int perm = 0, uint32_t cmask = 0xffffffffu, bool diag = false) {
+                                         int perm = 0, uint32_t cmask = 0xffffffffu, int shift = 15) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -133,7 +133,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const 
       float sb = s[n][e];
       if (MASK && bias_g && bias_g->log_bias && col < valid) sb += coarse_log_bias(*bias_g, c0 + col) * sqrt_d<D>();
       const bool vis =
-          (!MASK || (col < valid && ((cmask >> col) & 1u))) && (!(CAUSAL && diag) || col <= (lane >> 2) + 8 * r);
+          (!MASK || (col < valid && ((cmask >> col) & 1u))) && (!CAUSAL || col <= (lane >> 2) + 8 * r + shift);
       const float p = vis ? ex2(fmaf(sb, scale_log2, -lse2[r])) : 0.0f;
       ds[n][e] = POOL ? fmaf(p, dp[n][e] - delta[r], pds[r]) : p * (dp[n][e] - delta[r]);
     }
@@ -320,11 +320,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 3 : 2) attn_bwd_dq_bf16_kernel(
       if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
         dq_chunk<D, true>(qf, df, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - div_n1(g, gb) * g.N)),
                           P.scale_log2, lse2, delta, dq);
-      else if (CAUSAL) {  // kNoPick: nothing; the block's own keys: the causal diagonal
+      else if (CAUSAL) {  // kNoPick: every key masked; the block's own keys: the causal diagonal
         const int r = srow[seq];
-        if (r >= 0)
-          dq_chunk<D, false, false, true>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
-                                          0.f, 0, 0xffffffffu, r == gb * kBlock);
+        dq_chunk<D, false, false, true>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0, 0.f,
+                                        0, 0xffffffffu, r < 0 ? -kBlock : (r == gb * kBlock ? 0 : kBlock - 1));
       } else
         dq_chunk<D, false, POOL>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
                                  pool_log_bias<D>(g), PERM);

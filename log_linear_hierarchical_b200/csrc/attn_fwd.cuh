@@ -283,8 +283,9 @@ __device__ __forceinline__ void quad_row_sums(const float (&s)[2][4], float& t0,
 // One 16-token chunk of the online softmax.  With MASK (the coarse chunks), columns >=
 // `valid` (the padding of the last coarse tile) and columns whose bit of `cmask` is clear
 // (causal entries that are not attended) are excluded and, under the log-count variant,
-// column c gets the bias of coarse entry c0 + c.  CAUSAL with `diag` (the query block's own
-// key block): key column c is visible to query row r only when c <= r.  m holds the running row maxima
+// column c gets the bias of coarse entry c0 + c.  CAUSAL: key column c is visible to query
+// row r only when c <= r + `shift` (15: a whole block before the query block, 0: the query
+// block's own block, -16: no block, a list's kNoPick slot), one branch-free test per score.  m holds the running row maxima
 // of the scaled scores (log2 domain), l the per-lane partial row sums.
 // POOL (the level-1 variant, fine chunks only): the chunk's block mean is one more KV
 // entry.  Its score is the mean of the 16 scores (q . mean k = mean of q . k), plus
@@ -294,7 +295,7 @@ template <int D, bool MASK, bool POOL = false, bool CAUSAL = false>
 __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint32_t ktile, uint32_t vtile, int valid,
                                           float scale_log2, float (&m)[2], float (&l)[2], float (&acc)[D / 8][4],
                                           const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
-                                          int perm = 0, uint32_t cmask = 0xffffffffu, bool diag = false) {
+                                          int perm = 0, uint32_t cmask = 0xffffffffu, int shift = 15) {
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   mma_a_bt<D>(s, qf, ktile, perm);
@@ -314,12 +315,12 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t (&qf)[D / 16][4], uint3
         else if (bias_g && bias_g->log_bias) s[n][e] += coarse_log_bias(*bias_g, c0 + col) * sqrt_d<D>();
       }
   }
-  if (CAUSAL && diag) {
+  if (CAUSAL) {
 #pragma unroll
     for (int n = 0; n < 2; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (n * 8 + 2 * (lane & 3) + (e & 1) > (lane >> 2) + 8 * (e >> 1)) s[n][e] = -INFINITY;
+        if (n * 8 + 2 * (lane & 3) + (e & 1) > (lane >> 2) + 8 * (e >> 1) + shift) s[n][e] = -INFINITY;
   }
   float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
   float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
@@ -523,11 +524,10 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attn_fwd_bf16_kernel(con
       const uint32_t kt = ring + stage * 2 * TB;
       if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
         fwd_chunk<D, true>(qf, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - bh_i * g.N)), P.scale_log2, m, l, acc);
-      else if (CAUSAL) {  // kNoPick: nothing; the block's own keys: the causal diagonal
+      else if (CAUSAL) {  // kNoPick: every key masked; the block's own keys: the causal diagonal
         const int r = srow[seq];
-        if (r >= 0)
-          fwd_chunk<D, false, false, true>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, 0.f, 0,
-                                           0xffffffffu, r == gb * kBlock);
+        fwd_chunk<D, false, false, true>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, 0.f, 0,
+                                         0xffffffffu, r < 0 ? -kBlock : (r == gb * kBlock ? 0 : kBlock - 1));
       } else
         fwd_chunk<D, false, POOL>(qf, kt, kt + TB, kBlock, P.scale_log2, m, l, acc, nullptr, 0, pool_log_bias<D>(g),
                                   PERM);
