@@ -865,8 +865,11 @@ def run_profile(args):
 
     cfg = WORKLOADS[args.workload]
     dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
-    dev = {k: v.cuda() for k, v in make_config_inputs(cfg, with_do=True).items()}
-    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype,
+    host = make_config_inputs(cfg, with_do=True)
+    if args.grid_order:
+        host = to_grid_order(host, cfg)
+    dev = {k: v.cuda() for k, v in host.items()}
+    shape = api.make_shape(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, dtype, grid_order=args.grid_order,
                            one_launch_select=args.one_launch_select, causal=args.causal, **enrichment(args))
     buf = api.LLSABuffers.allocate(shape, "cuda", dtype)
     for _ in range(args.warmup + args.steps):

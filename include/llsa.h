@@ -117,8 +117,8 @@ typedef enum { LLSA_BF16 = 0, LLSA_F32 = 1 } llsa_dtype;
  * LLSA_FLAG_ONE_LAUNCH_SELECT, llsa_train_step and plans run the pyramid and every selection
  * level as one cooperative persistent kernel whose phases are separated by grid-wide barriers,
  * instead of one launch per stage chained by programmatic dependent launch.  It applies to
- * bf16 inputs with levels >= 2, n_L <= 64 and topk in {2, 4, 8, 16}; elsewhere, and in the
- * separate calls, the flag changes nothing.  Off by default: on one B200 the chained launches
+ * bf16 inputs with levels >= 2, n_L <= 64 and topk in {2, 4, 8, 16}, without grid order or
+ * the causal mask; elsewhere, and in the separate calls, the flag changes nothing.  Off by default: on one B200 the chained launches
  * are faster (the forward can start its set-up while they drain, but not while a cooperative
  * kernel does).
  */
@@ -181,7 +181,14 @@ size_t llsa_pyramid_elems(const llsa_shape* shape);   /* fp32 elements per pyram
 size_t llsa_index_elems(const llsa_shape* shape);     /* int32 elements of idx and of col */
 size_t llsa_row_ptr_elems(const llsa_shape* shape);   /* int32 elements of row_ptr */
 
-/* Scratch bytes llsa_index_transpose / llsa_backward need in `workspace`. */
+/*
+ * Scratch bytes llsa_index_transpose / llsa_backward need in `workspace`.  For bf16 under
+ * LLSA_FLAG_GRID_ORDER the backward workspace also has room for the quadtree-ordered copies
+ * of q, k, v, dO (4 * B*H*N*D * 2 bytes) and of LSE (B*H*N * 4 bytes) that llsa_train_step
+ * and plans make in it: there the pyramid launch writes those copies while it pools, and the
+ * attention kernels gather whole 2 KB tiles from them instead of 4 x 4-pixel boxes from the
+ * grid (the separate calls still read the grid tensors directly).
+ */
 size_t llsa_transpose_workspace_bytes(const llsa_shape* shape);
 size_t llsa_backward_workspace_bytes(const llsa_shape* shape);
 

@@ -85,6 +85,17 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(const Geometry& g) 
   return w;
 }
 
+// bf16 under LLSA_FLAG_GRID_ORDER (g.zcopy) the host places after that layout the one-call
+// step's quadtree-ordered copies of q, k, v, dO ([B*H*N][D] bf16 each) and of LSE ([B*H*N]
+// fp32).  The kernels get their addresses as arguments, so the layout they compute (every
+// thread, at start) stays as small as it was.
+inline long long bwd_workspace_floats(const Geometry& g) {
+  const long long base = bwd_workspace_layout(g).total;
+  if (!g.zcopy) return base;
+  const long long zt = (long long)g.BH * g.N * g.D / 2;  // one bf16 tensor, in floats (D is even)
+  return base + ((4 * zt + (long long)g.BH * g.N + 63) & ~63LL);
+}
+
 // ---------------------------------------------------------------------------- query-major dQ
 
 template <int D, int STAGES>
@@ -1028,10 +1039,11 @@ __global__ void __launch_bounds__(32) attn_bwd_dkdv_bf16_kernel(
             pv[c] = pack_bf16(av[2 * c], av[2 * c + 1]);
           }
           const int kvalid = LAYOUT == kPadded ? g.nv - j * kBlock : kBlock;  // padding positions get 0
+          const long long row0 = token_row<LAYOUT>(g, bh, j * kBlock);
 #pragma unroll
           for (int t = 0; t < kBlock; ++t) {
             const bool real = t < kvalid;
-            const long long row = token_row<LAYOUT>(g, bh, j * kBlock + t);
+            const long long row = row0 + block_row_offset<LAYOUT>(g, t);
             if constexpr (V == 2) {
               reinterpret_cast<uint32_t*>(dk_out + row * D)[lane] = real ? pk[0] : 0u;
               reinterpret_cast<uint32_t*>(dv_out + row * D)[lane] = real ? pv[0] : 0u;

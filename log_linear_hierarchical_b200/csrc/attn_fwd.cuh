@@ -196,6 +196,7 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[D / 8][4], fl
   }
   __syncwarp();
   constexpr int CH = D / 8;
+  __nv_bfloat16* const base = out + token_row<LAYOUT>(g, bh, t0) * D;
 #pragma unroll
   for (int it = 0; it < D / 16; ++it) {
     const int ci = lane + 32 * it;
@@ -205,7 +206,7 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[D / 8][4], fl
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(stage + tswz(row, c)));
-    *reinterpret_cast<uint4*>(out + token_row<LAYOUT>(g, bh, t0 + row) * D + c * 8) = v;
+    *reinterpret_cast<uint4*>(base + block_row_offset<LAYOUT>(g, row) * D + c * 8) = v;
   }
   // the staging tile is refilled by TMA later: order these generic accesses before it
   fence_proxy_async();
@@ -414,7 +415,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attn_fwd_bf16_kernel(con
                                                             const float* __restrict__ k_pyr,
                                                             const float* __restrict__ v_pyr,
                                                             const int* __restrict__ idx, __nv_bfloat16* __restrict__ o,
-                                                            float* __restrict__ lse) {
+                                                            float* __restrict__ lse, float* __restrict__ lse_z) {
   // the coarse tiles come from the pyramid and the coarser selection levels, two or more
   // kernels back, so they are staged before waiting for the kernel ahead (see pdl_wait)
   extern __shared__ uint8_t fwd_smem_raw[];
@@ -549,8 +550,15 @@ __global__ void __launch_bounds__(128, D == 64 ? 4 : 2) attn_fwd_bf16_kernel(con
     store_tile_bf16<D, LAYOUT>(acc, real0 ? 1.0f / l[0] : 0.0f, real1 ? 1.0f / l[1] : 0.0f, sq + (i & 1) * TB, o, g,
                                bh_i, t0);
     if ((lane & 3) == 0) {
-      lse[token_row<LAYOUT>(g, bh_i, t0 + r0)] = real0 ? (m[0] + log2f(l[0])) * kLn2 : 0.0f;
-      lse[token_row<LAYOUT>(g, bh_i, t0 + r0 + 8)] = real1 ? (m[1] + log2f(l[1])) * kLn2 : 0.0f;
+      const float lse0 = real0 ? (m[0] + log2f(l[0])) * kLn2 : 0.0f;
+      const float lse1 = real1 ? (m[1] + log2f(l[1])) * kLn2 : 0.0f;
+      const long long lrow = token_row<LAYOUT>(g, bh_i, t0);
+      lse[lrow + block_row_offset<LAYOUT>(g, r0)] = lse0;
+      lse[lrow + block_row_offset<LAYOUT>(g, r0 + 8)] = lse1;
+      if (LAYOUT == kZStore) {  // the quadtree-ordered copy that dQ reads
+        lse_z[(long long)gb * kBlock + r0] = lse0;
+        lse_z[(long long)gb * kBlock + r0 + 8] = lse1;
+      }
     }
   }
   if (!ok) {

@@ -107,6 +107,7 @@ Geometry make_geometry(const llsa_shape* s) {
   g.grid = (s->flags & LLSA_FLAG_GRID_ORDER) ? 1 : 0;
   g.log_g = g.grid ? ilog2(s->N) / 2 : 0;
   g.causal = (s->flags & LLSA_FLAG_CAUSAL) ? 1 : 0;
+  g.zcopy = (g.grid && s->dtype == LLSA_BF16) ? 1 : 0;
   for (int l = 0; l <= kMaxLevels; ++l) g.m[l] = l <= g.L ? (int)((g.nv + (1LL << (4 * l)) - 1) >> (4 * l)) : 0;
   return g;
 }
@@ -172,10 +173,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // padding the view is the flat [B*H*N][D] (box 64 x 16, row coordinate = flat token row).
 // Under LLSA_FLAG_GRID_ORDER: [B*H*G][G][D] (pixel rows of every head's grid) with a
 // 64-channel x 4 x 4 pixel box (one 16-token block of the quadtree order).
-bool make_tile_map(CUtensorMap* m, const void* base, const Geometry& g) {
+bool make_tile_map(CUtensorMap* m, const void* base, const Geometry& g, int lay) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const int lay = layout_of(g);  // the rank here must match the kernels' tma_load_tile<D, lay>
+  // lay: the layout of the kernels that use the map; the rank here must match their
+  // tma_load_tile<D, lay>
   if (lay == kGrid) {  // the heads' grids stacked: pixel rows of all heads, G pixels each
     const cuuint64_t G = 1ULL << g.log_g;
     cuuint64_t dims[3] = {(cuuint64_t)g.D, G, (cuuint64_t)g.BH * G};
@@ -391,21 +393,42 @@ namespace {
 // level-1 CSR and can run beside the query side too.
 constexpr unsigned kQuerySide = 1, kKeySide = 2, kOrder = 4;
 
-// The instantiation of each bf16 attention kernel for a geometry: its Layout, and the
-// level-1 variant (POOL), which padding does not combine with.
+// The one-call step's quadtree-ordered copies of q, k, v, dO and LSE under grid order (in
+// its backward workspace, made by the pyramid launch and the forward); the attention kernels
+// then load only from these (layout kZStore).  Null: the separate calls, which read the
+// row-major grid tensors themselves (layout kGrid).
+struct ZCopies {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dO;
+  float* lse;
+};
+
+ZCopies step_zcopies(const Geometry& g, void* workspace) {
+  float* z = static_cast<float*>(workspace) + bwd_workspace_layout(g).total;  // see bwd_workspace_floats
+  const long long zt = (long long)g.BH * g.N * g.D / 2;
+  return ZCopies{z, z + zt, z + 2 * zt, z + 3 * zt, z + 4 * zt};
+}
+
+// The instantiation of each bf16 attention kernel for a geometry and layout (layout_of(g),
+// or kZStore for the step under grid order), and the level-1 variant (POOL), which padding
+// does not combine with.
 template <int D>
-auto pick_fwd(const Geometry& g) {
+auto pick_fwd(const Geometry& g, int lay) {
   constexpr int S = kFwdStages;
-  const int lay = layout_of(g);
+  if (lay == kZStore)
+    return g.pool1 ? attn_fwd_bf16_kernel<D, S, true, kZStore> : attn_fwd_bf16_kernel<D, S, false, kZStore>;
   if (lay == kPadded) return attn_fwd_bf16_kernel<D, S, false, kPadded>;
   if (lay == kCausal) return attn_fwd_bf16_kernel<D, S, false, kCausal>;
   if (lay == kGrid) return g.pool1 ? attn_fwd_bf16_kernel<D, S, true, kGrid> : attn_fwd_bf16_kernel<D, S, false, kGrid>;
   return g.pool1 ? attn_fwd_bf16_kernel<D, S, true, kFlat> : attn_fwd_bf16_kernel<D, S, false, kFlat>;
 }
 template <int D>
-auto pick_dq(const Geometry& g) {
+auto pick_dq(const Geometry& g, int lay) {
   constexpr int S = kDqStages;
-  const int lay = layout_of(g);
+  if (lay == kZStore)
+    return g.pool1 ? attn_bwd_dq_bf16_kernel<D, S, true, kZStore> : attn_bwd_dq_bf16_kernel<D, S, false, kZStore>;
   if (lay == kPadded) return attn_bwd_dq_bf16_kernel<D, S, false, kPadded>;
   if (lay == kCausal) return attn_bwd_dq_bf16_kernel<D, S, false, kCausal>;
   if (lay == kGrid)
@@ -413,9 +436,10 @@ auto pick_dq(const Geometry& g) {
   return g.pool1 ? attn_bwd_dq_bf16_kernel<D, S, true, kFlat> : attn_bwd_dq_bf16_kernel<D, S, false, kFlat>;
 }
 template <int D>
-auto pick_dkdv(const Geometry& g) {
+auto pick_dkdv(const Geometry& g, int lay) {
   constexpr int S = kDkvStages;
-  const int lay = layout_of(g);
+  if (lay == kZStore)
+    return g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, S, true, kZStore> : attn_bwd_dkdv_bf16_kernel<D, S, false, kZStore>;
   if (lay == kPadded) return attn_bwd_dkdv_bf16_kernel<D, S, false, kPadded>;
   if (lay == kCausal) return attn_bwd_dkdv_bf16_kernel<D, S, false, kCausal>;
   if (lay == kGrid)
@@ -423,8 +447,8 @@ auto pick_dkdv(const Geometry& g) {
   return g.pool1 ? attn_bwd_dkdv_bf16_kernel<D, S, true, kFlat> : attn_bwd_dkdv_bf16_kernel<D, S, false, kFlat>;
 }
 template <int D>
-auto pick_coarse(const Geometry& g) {
-  const int lay = layout_of(g);
+auto pick_coarse(const Geometry& g, int lay) {
+  if (lay == kZStore) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kZStore>;
   if (lay == kPadded) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kPadded>;
   if (lay == kGrid) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kGrid>;
   if (lay == kCausal) return attn_bwd_coarse_bf16_kernel<D, kDkvStages, kCausal>;
@@ -435,7 +459,8 @@ template <int D>
 llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
                               const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
                               const int32_t* idx, const int32_t* row_ptr, const int32_t* col, void* dq, void* dk,
-                              void* dv, void* workspace, unsigned phases, cudaStream_t cs) {
+                              void* dv, void* workspace, unsigned phases, cudaStream_t cs,
+                              const ZCopies* z) {
   llsa_status st = LLSA_OK;
   const Geometry g = make_geometry(s);
   float* ws = static_cast<float*>(workspace);
@@ -451,25 +476,27 @@ llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k,
     if (st != LLSA_OK) return st;
   }
   if (s->dtype == LLSA_BF16) {
+    const int lay = z ? kZStore : layout_of(g);
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tile_map(&tq, q, g) || !make_tile_map(&tk, k, g) || !make_tile_map(&tv, v, g) ||
-        !make_tile_map(&tdo, dO, g))
+    if (!make_tile_map(&tq, z ? z->q : q, g, lay) || !make_tile_map(&tk, z ? z->k : k, g, lay) ||
+        !make_tile_map(&tv, z ? z->v : v, g, lay) || !make_tile_map(&tdo, z ? z->dO : dO, g, lay))
       return LLSA_ERR_CUDA;
+    const float* lse_in = z ? z->lse : lse;  // dQ's LSE tiles: the quadtree-ordered copy in the step
     AttnParams P{g, scale * kLog2e, scale};
     const size_t kv_bytes = (size_t)kv_smem<D, kDkvStages>(1).total();
     if (phases & kQuerySide) {
       const size_t smem = (size_t)dq_smem<D, kDqStages>(g, kAttnWarps).total();
-      auto kern = pick_dq<D>(g);
+      auto kern = pick_dq<D>(g, lay);
       if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
       const int per_cta = kAttnWarps * kUnitBlocks;
       st = launch(kKBwdDqBf16, cs, [&] {
         launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, 
-            tq, tk, tv, tdo, P, k_pyr, v_pyr, idx, static_cast<const __nv_bfloat16*>(o), lse,
+            tq, tk, tv, tdo, P, k_pyr, v_pyr, idx, static_cast<const __nv_bfloat16*>(o), lse_in,
             static_cast<__nv_bfloat16*>(dq), ws);
       });
       if (st != LLSA_OK) return st;
       if (g.L >= 2) {
-        auto ckern = pick_coarse<D>(g);
+        auto ckern = pick_coarse<D>(g, lay);
         if (!allow_smem(ckern, kv_bytes)) return LLSA_ERR_CUDA;
         const int ctas = g.BH * g.n[2] * (g.coarse_pad / kBlock);
         st = launch(kKBwdCoarseBf16, cs, [&] {
@@ -480,7 +507,7 @@ llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k,
     }
     if (!(phases & kKeySide)) return LLSA_OK;
     if ((st = launch_coarse_reduce<D>(g, scale, idx, row_ptr, col, ws, cs)) != LLSA_OK) return st;
-    auto kern = pick_dkdv<D>(g);
+    auto kern = pick_dkdv<D>(g, lay);
     if (!allow_smem(kern, kv_bytes)) return LLSA_ERR_CUDA;
     return launch(kKBwdDkdvBf16, cs, [&] {
       launch_pdl(kern, dim3(total_blocks), dim3(32), kv_bytes, cs, tq, tk, tv, tdo, P, row_ptr, col, ws,
@@ -512,34 +539,45 @@ llsa_status backward_phases_d(const llsa_shape* s, const void* q, const void* k,
 llsa_status backward_phases(const llsa_shape* s, const void* q, const void* k, const void* v, const void* o,
                             const float* lse, const void* dO, const float* k_pyr, const float* v_pyr,
                             const int32_t* idx, const int32_t* row_ptr, const int32_t* col, void* dq, void* dk,
-                            void* dv, void* workspace, unsigned phases, cudaStream_t cs) {
+                            void* dv, void* workspace, unsigned phases, cudaStream_t cs,
+                            const ZCopies* z = nullptr) {
   auto f = s->D == 128 ? backward_phases_d<128> : backward_phases_d<64>;
-  return f(s, q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace, phases, cs);
+  return f(s, q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace, phases, cs, z);
 }
 
 // ---------------------------------------------------------------------------- pyramid, select
 // Levels 1-2 of the pyramid, and levels 3..L too when `upper`.
+// With `z` (the step under grid order) the launch also writes the quadtree-ordered copies of
+// q, k, v and, in a fourth slice of CTAs, of dO.
 template <typename T, int D>
 llsa_status pyramid_l12_launch(const Geometry& g, const void* q, const void* k, const void* v, float* q_pyr,
-                               float* k_pyr, float* v_pyr, cudaStream_t cs) {
+                               float* k_pyr, float* v_pyr, cudaStream_t cs, const ZCopies* z, const void* dO) {
   using C = PyrCfg<T, D>;
-  dim3 grid(g.BH * ((g.n[1] + C::ROWS - 1) / C::ROWS), 3);
+  dim3 grid(g.BH * ((g.n[1] + C::ROWS - 1) / C::ROWS), z ? 4 : 3);
   if (!allow_smem(pyramid_l12_kernel<T, D>, C::SPAN)) return LLSA_ERR_CUDA;
   const int dtype = sizeof(T) == 2 ? LLSA_BF16 : LLSA_F32;
-  CUtensorMap pq, pk, pv;
-  if (!make_patch_map(&pq, q, g, dtype) || !make_patch_map(&pk, k, g, dtype) || !make_patch_map(&pv, v, g, dtype))
+  CUtensorMap pq, pk, pv, pd;
+  if (!make_patch_map(&pq, q, g, dtype) || !make_patch_map(&pk, k, g, dtype) || !make_patch_map(&pv, v, g, dtype) ||
+      !make_patch_map(&pd, z ? dO : q, g, dtype))
     return LLSA_ERR_CUDA;
+  ZOut<T> zo{{nullptr, nullptr, nullptr, nullptr}, nullptr};
+  if (z) {
+    auto w = [](const void* p) { return static_cast<T*>(const_cast<void*>(p)); };
+    zo = ZOut<T>{{w(z->q), w(z->k), w(z->v), w(z->dO)}, static_cast<const T*>(dO)};
+  }
   return launch(kKPyramidL12, cs, [&] {
     launch_pdl(pyramid_l12_kernel<T, D>, dim3(grid), dim3(C::THREADS), C::SPAN, cs, g, static_cast<const T*>(q),
-               static_cast<const T*>(k), static_cast<const T*>(v), q_pyr, k_pyr, v_pyr, pq, pk, pv);
+               static_cast<const T*>(k), static_cast<const T*>(v), q_pyr, k_pyr, v_pyr, pq, pk, pv, pd, zo);
   });
 }
 
 template <int D>
 llsa_status pyramid_launch_d(const Geometry& g, int dtype, const void* q, const void* k, const void* v, float* q_pyr,
-                             float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs) {
-  llsa_status st = dtype == LLSA_BF16 ? pyramid_l12_launch<__nv_bfloat16, D>(g, q, k, v, q_pyr, k_pyr, v_pyr, cs)
-                                      : pyramid_l12_launch<float, D>(g, q, k, v, q_pyr, k_pyr, v_pyr, cs);
+                             float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs, const ZCopies* z,
+                             const void* dO) {
+  llsa_status st = dtype == LLSA_BF16
+                       ? pyramid_l12_launch<__nv_bfloat16, D>(g, q, k, v, q_pyr, k_pyr, v_pyr, cs, z, dO)
+                       : pyramid_l12_launch<float, D>(g, q, k, v, q_pyr, k_pyr, v_pyr, cs, nullptr, nullptr);
   if (st != LLSA_OK || !upper) return st;
   for (int l = 3; l <= g.L; ++l) {
     const long long total = (long long)g.BH * g.n[l] * D;
@@ -552,9 +590,10 @@ llsa_status pyramid_launch_d(const Geometry& g, int dtype, const void* q, const 
 }
 
 llsa_status pyramid_launch(const Geometry& g, int dtype, const void* q, const void* k, const void* v, float* q_pyr,
-                           float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs) {
+                           float* k_pyr, float* v_pyr, bool upper, cudaStream_t cs, const ZCopies* z = nullptr,
+                           const void* dO = nullptr) {
   auto f = g.D == 128 ? pyramid_launch_d<128> : pyramid_launch_d<64>;
-  return f(g, dtype, q, k, v, q_pyr, k_pyr, v_pyr, upper, cs);
+  return f(g, dtype, q, k, v, q_pyr, k_pyr, v_pyr, upper, cs, z, dO);
 }
 
 // The pooled levels 3..L and the coarsest selection fit one small kernel per (b, h).
@@ -633,7 +672,8 @@ llsa_status select_launch(const Geometry& g, float* q_pyr, float* k_pyr, float* 
 // children selection).
 // Requested by LLSA_FLAG_ONE_LAUNCH_SELECT.
 bool fused_pyramid_select(const Geometry& g, const llsa_shape* s) {
-  return (s->flags & LLSA_FLAG_ONE_LAUNCH_SELECT) && !g.causal && s->dtype == LLSA_BF16 && g.L >= 2 && small_top(g) &&
+  return (s->flags & LLSA_FLAG_ONE_LAUNCH_SELECT) && !g.causal && !g.grid && s->dtype == LLSA_BF16 && g.L >= 2 &&
+         small_top(g) &&
          (g.K == 2 || g.K == 4 || g.K == 8 || g.K == 16);
 }
 
@@ -697,7 +737,7 @@ llsa_status validate_step(const llsa_shape* s, const llsa_step_buffers* b) {
     if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
   const Geometry g = make_geometry(s);
   if (b->transpose_workspace_bytes < transpose_ws_bytes(g)) return LLSA_ERR_WORKSPACE;
-  if (b->backward_workspace_bytes < (size_t)bwd_workspace_layout(g).total * sizeof(float)) return LLSA_ERR_WORKSPACE;
+  if (b->backward_workspace_bytes < (size_t)bwd_workspace_floats(g) * sizeof(float)) return LLSA_ERR_WORKSPACE;
   return LLSA_OK;
 }
 
@@ -708,20 +748,23 @@ llsa_status validate_step(const llsa_shape* s, const llsa_step_buffers* b) {
 template <int D>
 llsa_status forward_launch(const Geometry& g, int dtype, const void* q, const void* k, const void* v,
                            const float* k_pyr, const float* v_pyr, const int32_t* idx, void* o, float* lse,
-                           cudaStream_t cs) {
+                           cudaStream_t cs, const ZCopies* z) {
   const float scale = 1.0f / sqrtf((float)D);
   const int total_blocks = g.BH * g.n[1];
   if (dtype == LLSA_BF16) {
+    const int lay = z ? kZStore : layout_of(g);
     CUtensorMap tq, tk, tv;
-    if (!make_tile_map(&tq, q, g) || !make_tile_map(&tk, k, g) || !make_tile_map(&tv, v, g)) return LLSA_ERR_CUDA;
+    if (!make_tile_map(&tq, z ? z->q : q, g, lay) || !make_tile_map(&tk, z ? z->k : k, g, lay) ||
+        !make_tile_map(&tv, z ? z->v : v, g, lay))
+      return LLSA_ERR_CUDA;
     AttnParams P{g, scale * kLog2e, scale};
     const size_t smem = (size_t)fwd_smem<D, kFwdStages>(g, kAttnWarps).total();
-    auto kern = pick_fwd<D>(g);
+    auto kern = pick_fwd<D>(g, lay);
     if (!allow_smem(kern, smem)) return LLSA_ERR_CUDA;
     const int per_cta = kAttnWarps * kUnitBlocks;
     return launch(kKFwdBf16, cs, [&] {
       launch_pdl(kern, dim3((total_blocks + per_cta - 1) / per_cta), dim3(32 * kAttnWarps), smem, cs, tq, tk, tv, P,
-                 k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse);
+                 k_pyr, v_pyr, idx, static_cast<__nv_bfloat16*>(o), lse, z ? z->lse : nullptr);
     });
   }
   const size_t smem = simt_fwd_smem<D>(g);
@@ -735,7 +778,8 @@ llsa_status forward_launch(const Geometry& g, int dtype, const void* q, const vo
 
 // The forward launch shared by llsa_forward and the step.
 llsa_status forward_impl(const llsa_shape* s, const void* q, const void* k, const void* v, const float* k_pyr,
-                         const float* v_pyr, const int32_t* idx, void* o, float* lse, llsa_stream_t stream) {
+                         const float* v_pyr, const int32_t* idx, void* o, float* lse, llsa_stream_t stream,
+                         const ZCopies* z = nullptr) {
   llsa_status st = validate(s);
   if (st != LLSA_OK) return st;
   const void* ptrs[8] = {q, k, v, k_pyr, v_pyr, idx, o, lse};
@@ -744,12 +788,16 @@ llsa_status forward_impl(const llsa_shape* s, const void* q, const void* k, cons
   const Geometry g = make_geometry(s);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   auto f = g.D == 128 ? forward_launch<128> : forward_launch<64>;
-  return f(g, s->dtype, q, k, v, k_pyr, v_pyr, idx, o, lse, cs);
+  return f(g, s->dtype, q, k, v, k_pyr, v_pyr, idx, o, lse, cs, z);
 }
 
 llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStream_t cs, cudaStream_t side) {
   const Geometry g = make_geometry(s);
   llsa_status st;
+  // under grid order (bf16) the pyramid launch also writes quadtree-ordered copies of q, k,
+  // v, dO into the workspace, and every attention kernel reads those instead of the grid
+  const ZCopies zc = g.zcopy ? step_zcopies(g, b->backward_workspace) : ZCopies{};
+  const ZCopies* z = g.zcopy ? &zc : nullptr;
   const bool fused = fused_pyramid_select(g, s);
   if (fused) {  // pyramid and selection in one cooperative launch
     unsigned* barrier =
@@ -759,7 +807,7 @@ llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStrea
   } else {
     // pooled levels >= 3 are made by the coarsest-selection launch when they are small
     const bool fuse_top = g.L >= 3 && small_top(g);
-    st = pyramid_launch(g, s->dtype, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, !fuse_top, cs);
+    st = pyramid_launch(g, s->dtype, b->q, b->k, b->v, b->q_pyr, b->k_pyr, b->v_pyr, !fuse_top, cs, z, b->dO);
     if (st == LLSA_OK) st = select_launch(g, b->q_pyr, b->k_pyr, b->v_pyr, b->idx, fuse_top, cs);
   }
   if (st != LLSA_OK) return st;
@@ -777,18 +825,18 @@ llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStrea
                                 side);
     if (st == LLSA_OK)
       st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
-                           b->dq, b->dk, b->dv, b->backward_workspace, kOrder, side);
+                           b->dq, b->dk, b->dv, b->backward_workspace, kOrder, side, z);
     if (cudaEventRecord(join, side) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
   }
   if (st == LLSA_OK) {
     // after the fused launch the forward's early reads (coarse rows and selections) would
     // be of the kernel right ahead of it, so it starts only once that kernel is complete
     if (fused) g_serial_next = true;
-    st = forward_impl(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs);
+    st = forward_impl(s, b->q, b->k, b->v, b->k_pyr, b->v_pyr, b->idx, b->o, b->lse, cs, z);
   }
   if (st == LLSA_OK)
     st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
-                         b->dq, b->dk, b->dv, b->backward_workspace, kQuerySide, cs);
+                         b->dq, b->dk, b->dv, b->backward_workspace, kQuerySide, cs, z);
   if (side) {
     if (cudaStreamWaitEvent(cs, join, 0) != cudaSuccess && st == LLSA_OK) st = LLSA_ERR_CUDA;
     cudaEventDestroy(fork);
@@ -797,11 +845,11 @@ llsa_status step_impl(const llsa_shape* s, const llsa_step_buffers* b, cudaStrea
     st = llsa_index_transpose(s, b->idx, b->row_ptr, b->col, b->transpose_workspace, b->transpose_workspace_bytes, cs);
     if (st == LLSA_OK)
       st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
-                           b->dq, b->dk, b->dv, b->backward_workspace, kOrder, cs);
+                           b->dq, b->dk, b->dv, b->backward_workspace, kOrder, cs, z);
   }
   if (st == LLSA_OK)
     st = backward_phases(s, b->q, b->k, b->v, b->o, b->lse, b->dO, b->k_pyr, b->v_pyr, b->idx, b->row_ptr, b->col,
-                         b->dq, b->dk, b->dv, b->backward_workspace, kKeySide, cs);
+                         b->dq, b->dk, b->dv, b->backward_workspace, kKeySide, cs, z);
   return st;
 }
 
@@ -854,7 +902,7 @@ size_t llsa_transpose_workspace_bytes(const llsa_shape* s) {
 
 size_t llsa_backward_workspace_bytes(const llsa_shape* s) {
   if (validate(s) != LLSA_OK) return 0;
-  return (size_t)bwd_workspace_layout(make_geometry(s)).total * sizeof(float);
+  return (size_t)bwd_workspace_floats(make_geometry(s)) * sizeof(float);
 }
 
 llsa_status llsa_build_pyramid(const llsa_shape* s, const void* q, const void* k, const void* v, float* q_pyr,
@@ -944,7 +992,7 @@ llsa_status llsa_backward(const llsa_shape* s, const void* q, const void* k, con
   const void* ptrs[16] = {q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LLSA_ERR_INVALID_ARG;
-  if (workspace_bytes < (size_t)bwd_workspace_layout(make_geometry(s)).total * sizeof(float)) return LLSA_ERR_WORKSPACE;
+  if (workspace_bytes < (size_t)bwd_workspace_floats(make_geometry(s)) * sizeof(float)) return LLSA_ERR_WORKSPACE;
   SerialFirstLaunch serial;
   return backward_phases(s, q, k, v, o, lse, dO, k_pyr, v_pyr, idx, row_ptr, col, dq, dk, dv, workspace,
                          kOrder | kQuerySide | kKeySide, reinterpret_cast<cudaStream_t>(stream));

@@ -62,6 +62,8 @@ struct Geometry {
                                          // path works in its quadtree (Z) order
   int log_g;
   int causal;                            // LLSA_FLAG_CAUSAL: keys at or before the query only
+  int zcopy;                             // bf16 under LLSA_FLAG_GRID_ORDER: the step keeps
+                                         // quadtree-ordered copies of q, k, v, dO and LSE
 };
 
 // The entry of a causal selection list that holds no pick (a query token with fewer than K
@@ -97,18 +99,34 @@ __host__ __device__ inline long long token_row(const Geometry& g, int bh, int t)
 //   kPadded: the same with rows at or past n_valid as padding (3-D maps read them as zeros);
 //   kGrid:   row-major G x G grids (LLSA_FLAG_GRID_ORDER: 3-D patch maps, the tile_row map);
 //   kCausal: flat rows under LLSA_FLAG_CAUSAL (diagonal blocks masked element-wise, lists
-//            that may end in kNoPick, coarse entries attended only before the block).
-enum Layout : int { kFlat = 0, kPadded = 1, kGrid = 2, kCausal = 3 };
+//            that may end in kNoPick, coarse entries attended only before the block);
+//   kZStore: the one-call step under LLSA_FLAG_GRID_ORDER: q, k, v, dO and LSE are read
+//            from quadtree-ordered copies (flat 2-D maps) and every output row is written
+//            to its row-major grid position.
+enum Layout : int { kFlat = 0, kPadded = 1, kGrid = 2, kCausal = 3, kZStore = 4 };
 
 // The layout of a geometry, and whether its tile tensor map is the flat 2-D [B*H*N][D] view
 // (kFlat, kCausal) rather than a 3-D one: the host's tensor map and the kernels' copy
 // instruction must agree on the rank.
 inline int layout_of(const Geometry& g) { return g.causal ? kCausal : g.grid ? kGrid : (g.nv < g.N ? kPadded : kFlat); }
-__host__ __device__ constexpr bool flat_tile_map(int layout) { return layout == kFlat || layout == kCausal; }
+__host__ __device__ constexpr bool flat_tile_map(int layout) {
+  return layout == kFlat || layout == kCausal || layout == kZStore;
+}
 
 template <int LAYOUT>
 __device__ __forceinline__ long long token_row(const Geometry& g, int bh, int t) {
-  return (long long)bh * g.N + (LAYOUT == kGrid ? z_to_rowmajor(t, g.log_g) : t);
+  return (long long)bh * g.N + ((LAYOUT == kGrid || LAYOUT == kZStore) ? z_to_rowmajor(t, g.log_g) : t);
+}
+
+// Memory-row offset of row r (0..15) of a 16-token block from the row of its first token:
+// r itself, or under grid order the pixel offset r_y G + r_x of quadtree position
+// r = 8 y1 + 4 x1 + 2 y0 + x0 (r_y = 2 y1 + y0, r_x = 2 x1 + x0) -- the same as
+// token_row(t0 + r) - token_row(t0) for a block-aligned t0, with a few bit operations.
+template <int LAYOUT>
+__device__ __forceinline__ long long block_row_offset(const Geometry& g, int r) {
+  if constexpr (LAYOUT == kGrid || LAYOUT == kZStore)
+    return ((long long)(((r >> 1) & 1) | ((r >> 2) & 2)) << g.log_g) + ((r & 1) | ((r >> 1) & 2));
+  return r;
 }
 
 // Under LLSA_FLAG_GRID_ORDER a 16-token block is a 4 x 4 pixel patch that a TMA box brings

@@ -94,13 +94,15 @@ struct PyrCfg {
 // the level-2 rows they make.  The CTA's input span (ROWS * 16 token rows) arrives by one
 // bulk copy completing on `bar` with phase parity `parity`, or, under grid order, as ROWS/16
 // 16 x 16 pixel patches (one level-2 token each) by TMA boxes of `pmap`; `span` and `s1` are
-// the CTA's shared buffers.  Every thread of the CTA calls it; returns false (for the whole
+// the CTA's shared buffers.  Under grid order `zout` (if not null) also receives the span's
+// tokens in quadtree order (the step's copies of q, k, v and dO), and `pyr` may be null for a
+// tensor that is only copied.  Every thread of the CTA calls it; returns false (for the whole
 // CTA) if the copy did not land within the bounded wait.
 template <typename T, int D>
 __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __restrict__ x,
                                                  float* __restrict__ pyr, int bh, int tile, uint8_t* span,
                                                  float (*s1)[D], uint32_t bar, uint32_t parity,
-                                                 const CUtensorMap* pmap) {
+                                                 const CUtensorMap* pmap, T* __restrict__ zout = nullptr) {
   using C = PyrCfg<T, D>;
   constexpr int VE = C::VE;
   constexpr int TPR = C::TPR;
@@ -138,6 +140,16 @@ __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __r
       const T* patch = reinterpret_cast<const T*>(span + (o >> 4) * PATCH) + c0;
       const int b = o & 15;
       const int br = compact_even_bits(b >> 1), bc = compact_even_bits(b);
+      if (zout) {  // the block's 16 tokens, in quadtree order, to the copy (16 bytes a thread)
+        T* zrow = zout + ((long long)bh * g.N + (long long)j1 * kBlock) * D + c0;
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) {
+          const int tr = compact_even_bits(r >> 1), tc = compact_even_bits(r);
+          *reinterpret_cast<uint4*>(zrow + r * D) =
+              *reinterpret_cast<const uint4*>(patch + ((4 * br + tr) * kBlock + 4 * bc + tc) * D);
+        }
+      }
+      if (!pyr) return true;  // a tensor that is only copied (every thread of the CTA returns)
 #pragma unroll
       for (int r = 0; r < kBlock; ++r) {
         const int tr = compact_even_bits(r >> 1), tc = compact_even_bits(r);
@@ -169,7 +181,7 @@ __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __r
       reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
   }
-  if (g.L < 2) return true;
+  if (!pyr || g.L < 2) return true;
   __syncthreads();
   for (int i = t; i < OUT2 * D; i += blockDim.x) {
     const int o2 = i / D;
@@ -185,8 +197,16 @@ __device__ __forceinline__ bool pyramid_l12_unit(const Geometry& g, const T* __r
   return true;
 }
 
-// grid.x = B*H * ceil(n_1 / ROWS), grid.y = 3 (q, k, v).
-// pm0..pm2: the grid-order patch maps of q, k, v (unused in quadtree order).
+// Quadtree-ordered copies made by pyramid_l12_kernel under grid order (the step's q, k, v,
+// dO copies; null pointers: none).  Slice 3 (dO) is copied, not pooled.
+template <typename T>
+struct ZOut {
+  T* z[4];
+  const T* x3;
+};
+
+// grid.x = B*H * ceil(n_1 / ROWS), grid.y = 3 (q, k, v), or 4 with dO copied under grid order.
+// pm0..pm3: the grid-order patch maps of q, k, v, dO (unused in quadtree order).
 template <typename T, int D>
 __global__ void __launch_bounds__(PyrCfg<T, D>::THREADS) pyramid_l12_kernel(Geometry g, const T* __restrict__ x0,
                                                                             const T* __restrict__ x1,
@@ -196,7 +216,9 @@ __global__ void __launch_bounds__(PyrCfg<T, D>::THREADS) pyramid_l12_kernel(Geom
                                                                             float* __restrict__ p2,
                                                                             const __grid_constant__ CUtensorMap pm0,
                                                                             const __grid_constant__ CUtensorMap pm1,
-                                                                            const __grid_constant__ CUtensorMap pm2) {
+                                                                            const __grid_constant__ CUtensorMap pm2,
+                                                                            const __grid_constant__ CUtensorMap pm3,
+                                                                            ZOut<T> zo) {
   pdl_enter();
   using C = PyrCfg<T, D>;
   __shared__ float s1[C::ROWS][D];
@@ -208,11 +230,12 @@ __global__ void __launch_bounds__(PyrCfg<T, D>::THREADS) pyramid_l12_kernel(Geom
     mbar_init(bar, 1);
     mbar_fence_init();
   }
-  const T* x = blockIdx.y == 0 ? x0 : (blockIdx.y == 1 ? x1 : x2);
-  float* pyr = blockIdx.y == 0 ? p0 : (blockIdx.y == 1 ? p1 : p2);
-  const CUtensorMap* pm = blockIdx.y == 0 ? &pm0 : (blockIdx.y == 1 ? &pm1 : &pm2);
+  const int y = blockIdx.y;
+  const T* x = y == 0 ? x0 : (y == 1 ? x1 : (y == 2 ? x2 : zo.x3));
+  float* pyr = y == 0 ? p0 : (y == 1 ? p1 : (y == 2 ? p2 : nullptr));
+  const CUtensorMap* pm = y == 0 ? &pm0 : (y == 1 ? &pm1 : (y == 2 ? &pm2 : &pm3));
   const int bh = blockIdx.x / tiles;
-  pyramid_l12_unit<T, D>(g, x, pyr, bh, blockIdx.x - bh * tiles, pyr_span, s1, bar, 0, pm);
+  pyramid_l12_unit<T, D>(g, x, pyr, bh, blockIdx.x - bh * tiles, pyr_span, s1, bar, 0, pm, zo.z[y]);
 }
 
 // Level l >= 3 from level l-1 (fp32).  One thread per output value; grid.y = tensor.

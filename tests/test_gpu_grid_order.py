@@ -74,21 +74,28 @@ def test_grid_order_against_the_oracle():
     compare_outputs(back, ref, "bf16", ["o", "lse", "dq", "dk", "dv"])
 
 
-@pytest.mark.parametrize("one_launch", [False, True])
-def test_grid_order_step_and_plan_match_separate_calls(one_launch):
-    """The one-call step and a plan, with the pyramid and selection as separate launches or
-    as one cooperative launch (whose pyramid phase reads the grid through patch maps)."""
+@pytest.mark.parametrize("one_launch,D,variants", [
+    (False, 64, {}),
+    (True, 64, {}),                                    # the flag changes nothing under grid order
+    (False, 128, {}),
+    (False, 64, dict(log_bias=True, level1=True)),
+])
+def test_grid_order_step_and_plan_match_separate_calls(one_launch, D, variants):
+    """The one-call step and a plan read quadtree-ordered copies of q, k, v, dO (made by the
+    pyramid launch) and write every output to its grid row; the separate calls read the grid
+    through patch maps.  Both must give the same bits."""
     B, H, N, K, L = 1, 2, 16384, 8, 2
-    ginputs = {k: to_grid(v) for k, v in inputs_for(B, H, N, 64, "bf16", "smooth", 163).items()}
-    ref = run_gpu(B, H, N, 64, K, L, "bf16", ginputs, grid_order=True)
+    ginputs = {k: to_grid(v) for k, v in inputs_for(B, H, N, D, "bf16", "smooth", 163).items()}
+    ref = run_gpu(B, H, N, D, K, L, "bf16", ginputs, grid_order=True, **variants)
     tdt = TORCH_DTYPE["bf16"]
-    shape = api.make_shape(B, H, N, 64, K, L, tdt, grid_order=True, one_launch_select=one_launch)
+    shape = api.make_shape(B, H, N, D, K, L, tdt, grid_order=True, one_launch_select=one_launch, **variants)
     dev = {k: v.cuda() for k, v in ginputs.items()}
     buf = api.LLSABuffers.allocate(shape, "cuda", tdt)
     api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
     torch.cuda.synchronize()
     for n in ("o", "dq", "dk", "dv"):
         assert np.array_equal(getattr(buf, n).float().cpu().numpy(), ref[n]), n
+    assert np.array_equal(buf.lse.cpu().numpy(), ref["lse"])
     plan = api.LLSAPlan(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf, repeat=2)
     buf.dk.zero_()
     plan.launch()
