@@ -253,6 +253,17 @@ def test_buffer_sizes_scale_with_head_width(lib):
     assert api.llsa_backward_workspace_bytes(s128) > api.llsa_backward_workspace_bytes(s64)
 
 
+def test_grid_order_workspace_holds_the_step_copies(lib):
+    # bf16 under grid order: room for quadtree-ordered q, k, v, dO (bf16) and LSE (fp32)
+    B, H, N, D = 1, 6, 65536, 64
+    plain = api.llsa_backward_workspace_bytes(api.make_shape(B, H, N, D, 8, 3, 0))
+    grid = api.llsa_backward_workspace_bytes(api.make_shape(B, H, N, D, 8, 3, 0, grid_order=True))
+    copies = 4 * B * H * N * D * 2 + B * H * N * 4
+    assert copies <= grid - plain < copies + 256
+    f32 = api.llsa_backward_workspace_bytes(api.make_shape(B, H, N, D, 8, 3, 1, grid_order=True))
+    assert f32 == api.llsa_backward_workspace_bytes(api.make_shape(B, H, N, D, 8, 3, 1))
+
+
 def test_grid_order_and_padding_rules(lib):
     grid = _lib.LLSA_FLAG_GRID_ORDER
     ok = api.make_shape(1, 2, 4096, 64, 4, 2, 0, grid_order=True)
