@@ -473,18 +473,21 @@ __device__ __forceinline__ void kv_scores(const uint32_t (&kf)[D / 16][4], const
 template <int D>
 __device__ __forceinline__ void kv_accumulate(const float (&pt)[2][4], const float (&dst)[2][4], uint32_t qt,
                                               uint32_t dt, float (&dk)[D / 8][4], float (&dv)[D / 8][4], int qperm) {
-  uint32_t phi[4], plo[4];
+  uint32_t phi[4], plo[4], dhi[4], dlo[4];
   split_bf16(pt[0][0], pt[0][1], phi[0], plo[0]);
   split_bf16(pt[0][2], pt[0][3], phi[1], plo[1]);
   split_bf16(pt[1][0], pt[1][1], phi[2], plo[2]);
   split_bf16(pt[1][2], pt[1][3], phi[3], plo[3]);
-  mma_a2_b<D>(dv, phi, plo, dt, qperm);
-  uint32_t dhi[4], dlo[4];
   split_bf16(dst[0][0], dst[0][1], dhi[0], dlo[0]);
   split_bf16(dst[0][2], dst[0][3], dhi[1], dlo[1]);
   split_bf16(dst[1][0], dst[1][1], dhi[2], dlo[2]);
   split_bf16(dst[1][2], dst[1][3], dhi[3], dlo[3]);
-  mma_a2_b<D>(dk, dhi, dlo, qt, qperm);
+  // both high halves first, then both low halves: an accumulator's second product is issued
+  // 16 MMAs after its first rather than 8 (same order per accumulator, so the same sums)
+  mma_a_b<D>(dv, phi[0], phi[1], phi[2], phi[3], dt, qperm);
+  mma_a_b<D>(dk, dhi[0], dhi[1], dhi[2], dhi[3], qt, qperm);
+  mma_a_b<D>(dv, plo[0], plo[1], plo[2], plo[3], dt, qperm);
+  mma_a_b<D>(dk, dlo[0], dlo[1], dlo[2], dlo[3], qt, qperm);
 }
 
 // Per-warp shared memory of the key-major kernels: the key tile's K and V, then a ring of
