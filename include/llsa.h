@@ -40,7 +40,7 @@
  *    synchronises the host, except llsa_device_status.
  *  - Arguments are checked on the host before any launch.  A rejected call launches
  *    nothing and returns LLSA_ERR_INVALID_ARG (bad value, null pointer, misalignment,
- *    shape rules below) or LLSA_ERR_UNSUPPORTED (a legal value this build does not
+ *    shape rules below) or LLSA_ERR_UNSUPPORTED (a legal value this library does not
  *    implement).  A launch failure returns LLSA_ERR_CUDA.  No exception crosses the ABI.
  *  - Shape rules: B, H >= 1; N a multiple of 16^L (so every n_l = N / 16^l is whole
  *    and n_L >= 1; N need not be a power of two; a shorter sequence is padded up to such an N
