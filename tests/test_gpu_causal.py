@@ -123,3 +123,22 @@ def test_autograd_is_causal_matches_the_calls():
     assert np.array_equal(o.detach().float().cpu().numpy(), ref["o"])
     for name, t in (("dq", q), ("dk", k), ("dv", v)):
         assert np.array_equal(t.grad.float().cpu().numpy(), ref[name]), name
+
+
+def test_causal_headline_workload_all_heads():
+    """The benchmarked geometry (B=1 H=6 N=65536 L=3 K=8) under the causal mask: every stage
+    of every head against the causal oracle."""
+    from synthetic import WORKLOADS, make_config_inputs
+    cfg = WORKLOADS["headline-65536"]
+    inputs = make_config_inputs(cfg, with_do=True)
+    gpu = run_gpu(cfg.B, cfg.H, cfg.N, cfg.D, cfg.topk, cfg.levels, cfg.dtype, inputs, causal=True)
+    assert gpu["status"] == 0
+    check_pyramid_bitexact(inputs, gpu, cfg.levels)
+    res = oc.check_selection_causal(gpu["q_pyr"], gpu["k_pyr"], gpu["idx"], cfg.topk)
+    assert res["bad"] == 0 and res["floor_used"] <= 1e-3 * res["rows"] + 2, res
+    for h in range(cfg.H):
+        one = {k: v[:, h:h + 1] for k, v in inputs.items()}
+        sub = {n: [x[:, h:h + 1] for x in gpu[n]] for n in ("k_pyr", "v_pyr", "idx")}
+        ref = replay_causal(one, sub)
+        got = {n: gpu[n][:, h:h + 1] for n in ("o", "lse", "dq", "dk", "dv")}
+        compare_outputs(got, ref, "bf16", ["o", "lse", "dq", "dk", "dv"])

@@ -102,3 +102,20 @@ def test_grid_order_step_and_plan_match_separate_calls(one_launch, D, variants):
     torch.cuda.synchronize()
     assert np.array_equal(buf.dk.float().cpu().numpy(), ref["dk"])
     plan.close()
+
+
+def test_grid_order_headline_step_matches_separate_calls():
+    """The benchmarked geometry with row-major grid tensors: the step (quadtree-ordered copies,
+    outputs to grid rows) against the separate calls (4 x 4-pixel boxes), bit for bit."""
+    B, H, N, K, L = 1, 6, 65536, 8, 3
+    ginputs = {k: to_grid(v) for k, v in inputs_for(B, H, N, 64, "bf16", "smooth", 164).items()}
+    ref = run_gpu(B, H, N, 64, K, L, "bf16", ginputs, grid_order=True)
+    tdt = TORCH_DTYPE["bf16"]
+    shape = api.make_shape(B, H, N, 64, K, L, tdt, grid_order=True)
+    dev = {k: v.cuda() for k, v in ginputs.items()}
+    buf = api.LLSABuffers.allocate(shape, "cuda", tdt)
+    api.llsa_train_step(shape, dev["q"], dev["k"], dev["v"], dev["do"], buf)
+    torch.cuda.synchronize()
+    for n in ("o", "dq", "dk", "dv"):
+        assert np.array_equal(getattr(buf, n).float().cpu().numpy(), ref[n]), n
+    assert np.array_equal(buf.lse.cpu().numpy(), ref["lse"])
