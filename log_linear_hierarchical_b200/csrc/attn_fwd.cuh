@@ -111,34 +111,6 @@ __device__ __forceinline__ void mma_a_b(float (&acc)[D / 8][4], uint32_t a0, uin
   }
 }
 
-// acc[D/8][4] (16 x D) += (A_hi + A_lo) (16 x 16) * B, B a 16-row x D tile (rows = K): one
-// set of B fragments serves both halves of a two-term bf16 operand; the products of the
-// high half are issued before those of the low half (no accumulator waits on its own
-// previous product), 64 channels at a time.
-template <int D>
-__device__ __forceinline__ void mma_a2_b(float (&acc)[D / 8][4], const uint32_t (&hi)[4], const uint32_t (&lo)[4],
-                                         uint32_t btile, int perm = 0) {
-  const int lane = lane_id();
-  const int row = tile_row((lane & 7) + (((lane >> 3) & 1) << 3), perm);
-#pragma unroll
-  for (int h = 0; h < D / 64; ++h) {
-    uint32_t b[4][4];
-#pragma unroll
-    for (int dc = 0; dc < 4; ++dc)
-      ldsm_x4_t(btile + tswz(row, 8 * h + 2 * dc + (lane >> 4)), b[dc][0], b[dc][1], b[dc][2], b[dc][3]);
-#pragma unroll
-    for (int dc = 0; dc < 4; ++dc) {
-      mma_bf16(acc[8 * h + 2 * dc], hi[0], hi[1], hi[2], hi[3], b[dc][0], b[dc][1]);
-      mma_bf16(acc[8 * h + 2 * dc + 1], hi[0], hi[1], hi[2], hi[3], b[dc][2], b[dc][3]);
-    }
-#pragma unroll
-    for (int dc = 0; dc < 4; ++dc) {
-      mma_bf16(acc[8 * h + 2 * dc], lo[0], lo[1], lo[2], lo[3], b[dc][0], b[dc][1]);
-      mma_bf16(acc[8 * h + 2 * dc + 1], lo[0], lo[1], lo[2], lo[3], b[dc][2], b[dc][3]);
-    }
-  }
-}
-
 // Two fp32 values as a bf16 pair hi (round to nearest) and the pair of their bf16-rounded
 // remainders lo, so that hi + lo carries about 16 significant bits of each value.
 __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
