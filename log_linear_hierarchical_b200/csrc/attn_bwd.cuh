@@ -98,11 +98,55 @@ inline long long bwd_workspace_floats(const Geometry& g) {
 
 // ---------------------------------------------------------------------------- query-major dQ
 
+// At D = 128 dQ keeps one [Q, dO] tile pair per warp and reads the Q and dO operands from it
+// at each k-step ("lean"): the pair of buffers took 136 KB of shared memory per CTA (one CTA,
+// 4 warps per SM) and the fragments 64 registers; lean, 2 CTAs fit (dQ 331 -> 255 us at the
+// 6-head 65536-token shape).  At D = 64 the double buffer and register fragments are faster
+// (the lean form measured 126 against 115 us there, even at 16 warps per SM).
+template <int D>
+__host__ __device__ constexpr bool dq_lean() {
+  return D == 128;
+}
+
+// The Q and dO operands of dQ's score products: fragments in registers, or (LEAN) the two
+// shared-memory tiles, read at each k-step.
+template <int D, bool LEAN>
+struct QdOps;
+template <int D>
+struct QdOps<D, false> {
+  uint32_t qf[D / 16][4], df[D / 16][4];
+  __device__ __forceinline__ void load(uint32_t qt, uint32_t dt, int perm) {
+    load_a_frags<D>(qt, qf, perm);
+    load_a_frags<D>(dt, df, perm);
+  }
+  __device__ __forceinline__ void scores(float (&s)[2][4], float (&dp)[2][4], uint32_t ktile, uint32_t vtile,
+                                         int bperm) const {
+    mma_a_bt<D>(s, qf, ktile, bperm);
+    mma_a_bt<D>(dp, df, vtile, bperm);
+  }
+};
+template <int D>
+struct QdOps<D, true> {
+  uint32_t qt, dt;
+  int aperm;
+  __device__ __forceinline__ void load(uint32_t q, uint32_t d, int perm) {
+    qt = q;
+    dt = d;
+    aperm = perm;
+  }
+  __device__ __forceinline__ void scores(float (&s)[2][4], float (&dp)[2][4], uint32_t ktile, uint32_t vtile,
+                                         int bperm) const {
+    mma_at_bt<D>(s, qt, ktile, aperm, bperm);
+    mma_at_bt<D>(dp, dt, vtile, aperm, bperm);
+  }
+};
+
 template <int D, int STAGES>
 __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
   CtaSmem c;
   c.coarse_bytes = 2 * g.coarse_pad * D * 2;
-  c.warp_tiles = 4 * tile_bytes<D>() + STAGES * 2 * tile_bytes<D>();  // [2][Q, dO] + ring of [K, V]
+  // [2][Q, dO] (one [Q, dO] pair at D = 128, see dq_lean) + ring of [K, V]
+  c.warp_tiles = (dq_lean<D>() ? 2 : 4) * tile_bytes<D>() + STAGES * 2 * tile_bytes<D>();
   c.warp_tail = 2 * kBlock * 4 + ((kUnitBlocks * g.K * 4 + 15) & ~15) + ((8 * (2 + STAGES) + 15) & ~15);
   c.nwarps = nwarps;
   return c;
@@ -112,8 +156,9 @@ __host__ __device__ inline CtaSmem dq_smem(const Geometry& g, int nwarps) {
 // POOL (level-1 variant, fine chunks): the block-mean entry has score mean(S) + pool_bias
 // and dP mean(dP); its dS, times the mean K row, is dS / 16 added to each of the 16 dS.
 // MASK, cmask, CAUSAL and shift as in fwd_chunk (masked entries get P = 0, hence dS = 0).
-template <int D, bool MASK, bool POOL = false, bool CAUSAL = false>
-__device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const uint32_t (&df)[D / 16][4],
+// ops: the block's Q and dO operands (QdOps).
+template <int D, bool MASK, bool POOL = false, bool CAUSAL = false, class Ops>
+__device__ __forceinline__ void dq_chunk(const Ops& ops,
                                          uint32_t ktile, uint32_t vtile, int valid, float scale_log2,
                                          const float (&lse2)[2], const float (&delta)[2], float (&dq)[D / 8][4],
                                          const Geometry* bias_g = nullptr, int c0 = 0, float pool_bias = 0.f,
@@ -121,8 +166,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&qf)[D / 16][4], const 
   const int lane = lane_id();
   float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float dp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  mma_a_bt<D>(s, qf, ktile, perm);
-  mma_a_bt<D>(dp, df, vtile, perm);
+  ops.scores(s, dp, ktile, vtile, perm);
   float pds[2] = {0.f, 0.f};  // pooled entry's dS / 16, rows r0 and r0 + 8
   if (POOL) {
     float t[2], u[2];
@@ -199,8 +243,9 @@ __global__ void __launch_bounds__(128, D == 64 ? 3 : 2) attn_bwd_dq_bf16_kernel(
     return;
   }
   const int nblk = min(kUnitBlocks, total_blocks - first);
+  constexpr bool LEAN = dq_lean<D>();
   const uint32_t qd = smem_u32(cs.tiles(base, warp));
-  const uint32_t ring = qd + 4 * TB;
+  const uint32_t ring = qd + (LEAN ? 2 : 4) * TB;  // after the [Q, dO] pair(s) (dq_smem)
   float* slse = reinterpret_cast<float*>(cs.tail(base, warp));  // [2][16]
   int* srow = reinterpret_cast<int*>(slse + 2 * kBlock);
   const uint32_t bar_qd = smem_u32(srow) + ((kUnitBlocks * K * 4 + 15) & ~15);
@@ -232,10 +277,13 @@ __global__ void __launch_bounds__(128, D == 64 ? 3 : 2) attn_bwd_dq_bf16_kernel(
     tma_load_tile<D, LAYOUT>(dst, &tm_k, g, row, bar);
     tma_load_tile<D, LAYOUT>(dst + TB, &tm_v, g, row, bar);
   };
+  // block i's Q/dO tiles: buffer i % 2, or (LEAN) the one buffer, which block i+1's tiles
+  // enter once block i has finished with it; the two mbarriers and LSE slots alternate
+  auto qd_tiles = [&](int i) { return LEAN ? qd : qd + (i & 1) * 2 * TB; };
   auto issue_qd = [&](int i) {
     const uint32_t bar = bar_qd + 8 * (i & 1);
     const int row = (first + i) * kBlock;
-    const uint32_t dst = qd + (i & 1) * 2 * TB;
+    const uint32_t dst = qd_tiles(i);
     mbar_expect_tx(bar, 2 * TB + kBlock * 4);
     tma_load_tile<D, LAYOUT>(dst, &tm_q, g, row, bar);
     tma_load_tile<D, LAYOUT>(dst + TB, &tm_do, g, row, bar);
@@ -250,7 +298,7 @@ __global__ void __launch_bounds__(128, D == 64 ? 3 : 2) attn_bwd_dq_bf16_kernel(
   if (lane == 0) issue_qd(0);
 
   bool ok = true;
-  int next_seq = 0, next_q = 0;
+  int next_seq = 0, next_q = 0, q_issued = 1;
   // O rows of a block (lane: shared-memory tile row lane/2, channels (lane%2) * D/2 onwards;
   // the row's token is tile_row of it).  At D = 64 they are loaded one block ahead; at
   // D = 128 (twice the registers) when the block starts.
@@ -278,13 +326,15 @@ __global__ void __launch_bounds__(128, D == 64 ? 3 : 2) attn_bwd_dq_bf16_kernel(
     ok = __all_sync(0xffffffffu, mbar_wait(bar_qd + 8 * (i & 1), (i >> 1) & 1));
     if (!ok) break;
     next_q = i + 1;
-    // the other buffer was released at the end of block i-1
-    if (lane == 0 && i + 1 < nblk) issue_qd(i + 1);
-    const uint32_t qt = qd + (i & 1) * 2 * TB;
+    // with two buffers the other one was released at the end of block i-1
+    if (!LEAN && i + 1 < nblk) {
+      if (lane == 0) issue_qd(i + 1);
+      q_issued = i + 2;
+    }
+    const uint32_t qt = qd_tiles(i);
     const uint32_t dt = qt + TB;
-    uint32_t qf[D / 16][4], df[D / 16][4];
-    load_a_frags<D>(qt, qf, PERM);
-    load_a_frags<D>(dt, df, PERM);
+    QdOps<D, LEAN> ops;
+    ops.load(qt, dt, PERM);
     // Delta_r = sum_d dO[r][d] * O[r][d] (O from registers, dO from the staged tile)
     float dlt;
     {
@@ -329,32 +379,38 @@ __global__ void __launch_bounds__(128, D == 64 ? 3 : 2) attn_bwd_dq_bf16_kernel(
       next_seq = seq + 1;
       const uint32_t kt = ring + stage * 2 * TB;
       if (PAD)  // real keys of this tile: 16 except in the one that holds the last real token
-        dq_chunk<D, true>(qf, df, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - div_n1(g, gb) * g.N)),
-                          P.scale_log2, lse2, delta, dq);
+        dq_chunk<D, true>(ops, kt, kt + TB, min(kBlock, g.nv - (srow[seq] - div_n1(g, gb) * g.N)), P.scale_log2,
+                          lse2, delta, dq);
       else if (CAUSAL) {  // kNoPick: every key masked; the block's own keys: the causal diagonal
         const int r = srow[seq];
-        dq_chunk<D, false, false, true>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0, 0.f,
-                                        0, 0xffffffffu, r < 0 ? -kBlock : (r == gb * kBlock ? 0 : kBlock - 1));
+        dq_chunk<D, false, false, true>(ops, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0, 0.f, 0,
+                                        0xffffffffu, r < 0 ? -kBlock : (r == gb * kBlock ? 0 : kBlock - 1));
       } else
-        dq_chunk<D, false, POOL>(qf, df, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
+        dq_chunk<D, false, POOL>(ops, kt, kt + TB, kBlock, P.scale_log2, lse2, delta, dq, nullptr, 0,
                                  pool_log_bias<D>(g), PERM);
       __syncwarp();
       if (lane == 0 && seq + STAGES < total_loads) issue_kv(seq + STAGES);
     }
     if (!ok) break;
     for (int cc = 0; cc < g.coarse_pad / kBlock; ++cc)
-      dq_chunk<D, true>(qf, df, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock), P.scale_log2, lse2,
+      dq_chunk<D, true>(ops, ck + cc * TB, cv + cc * TB, min(kBlock, g.coarse - cc * kBlock), P.scale_log2, lse2,
                         delta, dq, &g, cc * kBlock, 0.f, 0, cmask >> (cc * kBlock));
     __syncwarp();
     {
       const int bhi = div_n1(g, gb);
       store_tile_bf16<D, LAYOUT>(dq, P.scale, P.scale, qt, dq_out, g, bhi, (gb - bhi * n1) * kBlock);
     }
+    // LEAN: the one Q/dO buffer (and the staging use above) is done with: request the next
+    // block's tiles (store_tile_bf16 ordered its generic accesses before this async copy)
+    if (LEAN && i + 1 < nblk) {
+      if (lane == 0) issue_qd(i + 1);
+      q_issued = i + 2;
+    }
   }
   if (!ok) {
     for (int seq = next_seq; seq < min(total_loads, next_seq + STAGES); ++seq)
       mbar_wait(bar_kv + 8 * (seq % STAGES), (seq / STAGES) & 1);
-    for (int i = next_q; i < min(nblk, next_q + 2); ++i) mbar_wait(bar_qd + 8 * (i & 1), (i >> 1) & 1);
+    for (int i = next_q; i < q_issued; ++i) mbar_wait(bar_qd + 8 * (i & 1), (i >> 1) & 1);
   }
 }
 
