@@ -814,9 +814,10 @@ def run_reference(args):
         return
     from synthetic import WORKLOADS, make_config_inputs
 
+    wall0 = time.perf_counter()
     cfg = WORKLOADS[args.workload]
     host = make_config_inputs(cfg, with_do=True)
-    pool = OraclePool(cfg, host, enrichment(args))
+    pool = OraclePool(cfg, host, enrichment(args), cores=args.ref_cores)
     heads_all = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
     try:
         t_head = pool.step(heads=heads_all[:1], backward=True)
@@ -853,6 +854,12 @@ def run_reference(args):
                          "cpu_model": host_cpu_model(), "sample": sample},
         "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+    # the timed steps are whole oracle steps that ran inside this process: steps x ms_per_step is
+    # measured time, not an extrapolation, and fits in the run's own wall clock
+    wall = time.perf_counter() - wall0
+    timed = args.steps * ms_per_step / 1000.0
+    result["consistency"] = {"timed_seconds": round(timed, 3), "wall_seconds": round(wall, 3), "extrapolated": False,
+                             "fits_in_driver_run": timed <= wall}
     print(json.dumps(result), flush=True)
 
 
@@ -909,6 +916,8 @@ def main():
                     help="causal attention (LLSA_FLAG_CAUSAL; bf16, default enrichment)")
     ap.add_argument("--one-launch-select", action="store_true",
                     help="pyramid and selection as one cooperative launch (LLSA_FLAG_ONE_LAUNCH_SELECT)")
+    ap.add_argument("--ref-cores", type=int, default=None,
+                    help="worker processes of the reference arm's oracle (default: every host core)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
